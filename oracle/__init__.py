@@ -1,0 +1,221 @@
+"""Plain CPU oracle for the Sparse-BitNet BitLinear hot path.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product library never links, loads or calls it, and it shares no
+code with the CUDA path: the arithmetic lives in ``bitnet_oracle.c`` (plain C,
+written from the definitions) and this module only marshals NumPy arrays.
+
+Definitions followed (page title and section):
+  * "BitNet b1.58: Ternary Weights for 1.58-bit LLMs", "The mechanism":
+    absmean scale over the whole matrix, divide, round, clip to {-1, 0, 1};
+    per-token symmetric 8-bit activations; ternary product as signed sums.
+  * "Sparse-BitNet" (gist.science technical summary), section 2
+    "Kerncomponenten": N:M mask from the master magnitudes, quantise then
+    mask; "Training Strategie": dynamic mask, straight-through gradients.
+
+Every function here is pinned by a test in ``tests/test_oracle_pins.py`` to
+something other than itself (math.fsum, brute force, closed forms, hand-worked
+fixtures in ``tests/golden/``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bitnet_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle with gcc (no FMA contraction, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        cmd = ["gcc", "-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math",
+               "-fopenmp", "-shared", "-fPIC", _SRC, "-o", _LIB, "-lm"]
+        subprocess.check_call(cmd)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    build()
+    lib = ctypes.CDLL(_LIB)
+    P = ctypes.c_void_p
+    I64 = ctypes.c_int64
+    F = ctypes.c_float
+    lib.oracle_abs_sum.restype = ctypes.c_double
+    lib.oracle_abs_sum.argtypes = [P, I64]
+    lib.oracle_gamma.restype = F
+    lib.oracle_gamma.argtypes = [P, I64, F]
+    lib.oracle_mask_nm.restype = None
+    lib.oracle_mask_nm.argtypes = [P, I64, I64, ctypes.c_int, ctypes.c_int, P]
+    lib.oracle_ternary.restype = None
+    lib.oracle_ternary.argtypes = [P, I64, F, P]
+    lib.oracle_apply_mask.restype = None
+    lib.oracle_apply_mask.argtypes = [P, P, I64, P]
+    lib.oracle_pack_24.restype = ctypes.c_int
+    lib.oracle_pack_24.argtypes = [P, P, I64, I64, P]
+    lib.oracle_quant_act.restype = None
+    lib.oracle_quant_act.argtypes = [P, I64, I64, F, P, P]
+    lib.oracle_gemm_i32.restype = ctypes.c_int
+    lib.oracle_gemm_i32.argtypes = [P, P, I64, I64, I64, P]
+    lib.oracle_dequant.restype = None
+    lib.oracle_dequant.argtypes = [P, P, F, I64, I64, P]
+    lib.oracle_dequant_f64.restype = None
+    lib.oracle_dequant_f64.argtypes = [P, P, F, I64, I64, P]
+    lib.oracle_dgrad.restype = None
+    lib.oracle_dgrad.argtypes = [P, P, F, I64, I64, I64, P, P]
+    lib.oracle_set_threads.restype = None
+    lib.oracle_set_threads.argtypes = [ctypes.c_int]
+    lib.oracle_max_threads.restype = ctypes.c_int
+    lib.oracle_max_threads.argtypes = []
+    _lib = lib
+    return lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def set_threads(n: int) -> int:
+    lib = _load()
+    lib.oracle_set_threads(int(n))
+    return lib.oracle_max_threads()
+
+
+def max_threads() -> int:
+    return _load().oracle_max_threads()
+
+
+def bf16_to_f32(u16: np.ndarray) -> np.ndarray:
+    """Widen raw bf16 bit patterns (uint16) to fp32 exactly."""
+    return (u16.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def abs_sum(W: np.ndarray) -> float:
+    """fp64 nearest to the exact sum of |W| (whole matrix)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    return float(_load().oracle_abs_sum(_p(W), W.size))
+
+
+def gamma(W: np.ndarray, eps: float = 1e-5) -> np.float32:
+    """Absmean scale: fp32(sum|W| / n) + eps (eps added in fp32)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    return np.float32(_load().oracle_gamma(_p(W), W.size, np.float32(eps)))
+
+
+def mask_nm(W: np.ndarray, n: int = 2, m: int = 4) -> np.ndarray:
+    """uint8 keep-mask, top-n |W| of each m consecutive weights per row."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    rows, k = W.shape
+    assert k % m == 0
+    keep = np.empty((rows, k), np.uint8)
+    _load().oracle_mask_nm(_p(W), rows, k, n, m, _p(keep))
+    return keep
+
+
+def ternary(W: np.ndarray, g: float) -> np.ndarray:
+    """clip(rint(W / g), -1, 1) for every weight (int8)."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    q = np.empty(W.shape, np.int8)
+    _load().oracle_ternary(_p(W), W.size, np.float32(g), _p(q))
+    return q
+
+
+def apply_mask(wt: np.ndarray, keep: np.ndarray) -> np.ndarray:
+    wt = np.ascontiguousarray(wt, dtype=np.int8)
+    keep = np.ascontiguousarray(keep, dtype=np.uint8)
+    out = np.empty_like(wt)
+    _load().oracle_apply_mask(_p(wt), _p(keep), wt.size, _p(out))
+    return out
+
+
+def pack_24(wq: np.ndarray, keep: np.ndarray) -> np.ndarray:
+    """Canonical 2:4 group bytes [rows, k/4]."""
+    wq = np.ascontiguousarray(wq, dtype=np.int8)
+    keep = np.ascontiguousarray(keep, dtype=np.uint8)
+    rows, k = wq.shape
+    gb = np.empty((rows, k // 4), np.uint8)
+    rc = _load().oracle_pack_24(_p(wq), _p(keep), rows, k, _p(gb))
+    if rc != 0:
+        raise ValueError("mask is not 2:4")
+    return gb
+
+
+def quant_act(X: np.ndarray, eps: float = 1e-5):
+    """Per-token absmax int8: returns (Xq int8 [T,K], a fp32 [T] = max(absmax, eps))."""
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    T, K = X.shape
+    Xq = np.empty((T, K), np.int8)
+    a = np.empty((T,), np.float32)
+    _load().oracle_quant_act(_p(X), T, K, np.float32(eps), _p(Xq), _p(a))
+    return Xq, a
+
+
+def gemm_i32(Xq: np.ndarray, Wq: np.ndarray) -> np.ndarray:
+    """acc[t, n] = sum_k Xq[t, k] * Wq[n, k] (exact, int32)."""
+    Xq = np.ascontiguousarray(Xq, dtype=np.int8)
+    Wq = np.ascontiguousarray(Wq, dtype=np.int8)
+    T, K = Xq.shape
+    N = Wq.shape[0]
+    acc = np.empty((T, N), np.int32)
+    if _load().oracle_gemm_i32(_p(Xq), _p(Wq), T, N, K, _p(acc)) != 0:
+        raise OverflowError("int32 accumulator overflow")
+    return acc
+
+
+def dequant(acc: np.ndarray, a: np.ndarray, g: float) -> np.ndarray:
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    T, N = acc.shape
+    Y = np.empty((T, N), np.float32)
+    _load().oracle_dequant(_p(acc), _p(a), np.float32(g), T, N, _p(Y))
+    return Y
+
+
+def dequant_f64(acc: np.ndarray, a: np.ndarray, g: float) -> np.ndarray:
+    acc = np.ascontiguousarray(acc, dtype=np.int32)
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    T, N = acc.shape
+    Y = np.empty((T, N), np.float64)
+    _load().oracle_dequant_f64(_p(acc), _p(a), np.float32(g), T, N, _p(Y))
+    return Y
+
+
+def dgrad(dY: np.ndarray, Wq: np.ndarray, g: float):
+    """dX = g * dY @ Wq in fp64; also returns g * |dY| @ |Wq| (error-bound scale)."""
+    dY = np.ascontiguousarray(dY, dtype=np.float32)
+    Wq = np.ascontiguousarray(Wq, dtype=np.int8)
+    T, N = dY.shape
+    K = Wq.shape[1]
+    dX = np.empty((T, K), np.float64)
+    absdX = np.empty((T, K), np.float64)
+    _load().oracle_dgrad(_p(dY), _p(Wq), np.float32(g), T, N, K, _p(dX), _p(absdX))
+    return dX, absdX
+
+
+def pack_weights(W: np.ndarray, eps: float = 1e-5):
+    """Whole weight side: (gamma, keep, Wq masked ternary, canonical group bytes)."""
+    g = gamma(W, eps)
+    keep = mask_nm(W, 2, 4)
+    wt = ternary(W, g)
+    wq = apply_mask(wt, keep)
+    gb = pack_24(wq, keep)
+    return g, keep, wq, gb
+
+
+def forward(W: np.ndarray, X: np.ndarray, eps_w: float = 1e-5, eps_a: float = 1e-5):
+    """One Sparse-BitLinear forward; returns a dict of every intermediate."""
+    g, keep, wq, gb = pack_weights(W, eps_w)
+    Xq, a = quant_act(X, eps_a)
+    acc = gemm_i32(Xq, wq)
+    Y = dequant(acc, a, g)
+    return dict(gamma=g, keep=keep, wq=wq, gb=gb, xq=Xq, a=a, acc=acc, y=Y)

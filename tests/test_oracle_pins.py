@@ -1,0 +1,289 @@
+"""Pins of the CPU oracle to things other than itself (CPU only).
+
+Each function of ``oracle/`` is checked against an independent route to the
+same defined value: math.fsum for the exact absolute sum, brute-force sorting
+for the top-N mask, hand-worked fixtures in tests/golden/, NumPy integer and
+fp64 matrix products, closed forms for Gaussian weights, and invariants the
+pages state (codes in {-1,0,1}, at most N non-zeros per group of M, symmetric
+activation codes with no zero-point).
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from sparse_linear_layers_bitnet_b200 import synth
+from tests.conftest import ROOT, load_golden
+import os
+
+
+# ---------------------------------------------------------------- abs sum / gamma
+
+def _fsum_abs(W):
+    return math.fsum(abs(float(v)) for v in np.asarray(W, np.float32).ravel())
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_abs_sum_matches_fsum_gaussian(seed):
+    W = synth.master_weights(64, 96, 0.02, seed)
+    assert oracle.abs_sum(W) == _fsum_abs(W)
+
+
+def test_abs_sum_matches_fsum_wide_exponents():
+    r = np.random.default_rng(5)
+    parts = [
+        r.normal(0, 1, 500) * np.float32(1e30),
+        r.normal(0, 1, 500) * np.float32(1e-30),
+        r.normal(0, 1, 500) * np.float32(1e-3),
+        np.array([0.0, -0.0, 1e-45, -1e-45, 1.17549435e-38, 3.4e38, -3.4e38, 2.0 ** -149]),
+        r.normal(0, 1, 500) * np.float32(1e-40),     # subnormal fp32
+    ]
+    W = np.concatenate([np.asarray(p, np.float32) for p in parts]).astype(np.float32)
+    r.shuffle(W)
+    assert oracle.abs_sum(W) == _fsum_abs(W)
+
+
+def test_abs_sum_rounding_tie_cases():
+    # 2^53 + 1 (in units) is a tie between 2^53 and 2^53 + 2; exact-then-round
+    # must give the even neighbour; fsum agrees.
+    W = np.array([2.0 ** 52, 2.0 ** 52, 1.0], np.float32)
+    assert oracle.abs_sum(W) == _fsum_abs(W) == 2.0 ** 53
+    W = np.array([2.0 ** 52, 2.0 ** 52, 1.0, 1.0, 1.0], np.float32)
+    assert oracle.abs_sum(W) == _fsum_abs(W) == 2.0 ** 53 + 4
+    W = np.array([2.0 ** 60] + [1.0] * 300, np.float32)
+    assert oracle.abs_sum(W) == _fsum_abs(W)
+
+
+@pytest.mark.parametrize("eps", [0.0, 1e-5])
+def test_gamma_from_fsum(eps):
+    W = synth.master_weights(32, 64, 0.02, 7)
+    expect = np.float32(np.float32(_fsum_abs(W) / W.size) + np.float32(eps))
+    assert oracle.gamma(W, eps) == expect
+
+
+def test_gamma_is_order_independent():
+    W = synth.master_weights(16, 256, 0.02, 3)
+    perm = np.random.default_rng(0).permutation(W.size)
+    assert oracle.gamma(W) == oracle.gamma(W.ravel()[perm].reshape(W.shape))
+
+
+# ---------------------------------------------------------------- mask
+
+def _brute_mask(W, n, m):
+    keep = np.zeros(W.shape, np.uint8)
+    for r in range(W.shape[0]):
+        for g in range(W.shape[1] // m):
+            vals = [abs(float(W[r, g * m + p])) for p in range(m)]
+            order = sorted(range(m), key=lambda p: (-vals[p], p))
+            for p in order[:n]:
+                keep[r, g * m + p] = 1
+    return keep
+
+
+@pytest.mark.parametrize("n,m", [(2, 4), (1, 4), (3, 4), (6, 8), (4, 8)])
+def test_mask_matches_sorting_brute_force(n, m):
+    W = synth.master_weights(24, 64, 0.02, 11)
+    # plant exact ties and signed zeros
+    W[0, :m] = 0.25
+    W[1, :m] = 0.0
+    W[1, 1] = -0.0
+    W[2, :4] = [-0.5, 0.5, 0.25, -0.25]
+    assert np.array_equal(oracle.mask_nm(W, n, m), _brute_mask(W, n, m))
+
+
+def test_mask_all_permutations_of_distinct_magnitudes():
+    mags = [0.1, 0.2, 0.3, 0.4]
+    rows = []
+    for perm in itertools.permutations(range(4)):
+        rows.append([mags[p] * (1 if i % 2 else -1) for i, p in enumerate(perm)])
+    W = np.array(rows, np.float32)
+    keep = oracle.mask_nm(W, 2, 4)
+    for i, perm in enumerate(itertools.permutations(range(4))):
+        # kept positions hold the two largest magnitudes (0.3 and 0.4)
+        kept = {p for p in range(4) if keep[i, p]}
+        assert kept == {j for j in range(4) if perm[j] >= 2}
+
+
+def test_mask_ties_lower_index():
+    W = np.array([[0.25, 0.25, 0.25, 0.25],
+                  [0.0, -0.0, 0.0, -0.0],
+                  [0.1, 0.3, 0.3, 0.3],
+                  [0.3, 0.1, 0.1, 0.3]], np.float32)
+    keep = oracle.mask_nm(W, 2, 4)
+    assert keep.tolist() == [[1, 1, 0, 0], [1, 1, 0, 0], [0, 1, 1, 0], [1, 0, 0, 1]]
+
+
+# ---------------------------------------------------------------- ternary
+
+def _hexf(s):
+    return np.float32(float.fromhex(s))
+
+
+def test_ternary_boundaries_golden():
+    rows = []
+    with open(os.path.join(ROOT, "tests", "golden", "ternary_boundaries.txt")) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if line:
+                g, w, c = line.split()
+                rows.append((_hexf(g), _hexf(w), int(c)))
+    for g, w, c in rows:
+        assert oracle.ternary(np.array([w], np.float32), g)[0] == c, (g, w, c)
+
+
+def test_ternary_matches_numpy_rint_clip():
+    W = synth.master_weights(64, 64, 0.02, 4)
+    g = oracle.gamma(W)
+    ref = np.clip(np.rint(W / np.float32(g)), -1, 1).astype(np.int8)   # numpy float32 IEEE ops
+    assert np.array_equal(oracle.ternary(W, g), ref)
+
+
+def test_gaussian_zero_fraction_closed_form():
+    # W ~ N(0, s): gamma -> s*sqrt(2/pi) (+eps); a weight is coded 0 when
+    # |W| <= gamma/2, so P(zero) = 2*Phi(c) - 1 with c = gamma / (2 s).
+    # Among the 2 kept of 4 (top-2 by |W|), the zero fraction is
+    # [P(X(3) <= c) + P(X(4) <= c)] / 2 = 2 F^3 (1 - F) + F^4, F = P(zero).
+    s, eps = 0.02, 1e-5
+    W = synth.master_weights(1024, 1024, s, 21)
+    g = float(oracle.gamma(W, eps))
+    c = (s * math.sqrt(2 / math.pi) + eps) / (2 * s)
+    F = math.erf(c / math.sqrt(2))
+    wt = oracle.ternary(W, g)
+    n = W.size
+    dense_zero = float(np.mean(wt == 0))
+    assert abs(dense_zero - F) < 5 * math.sqrt(F * (1 - F) / n)
+    assert abs(F - 0.3101) < 1e-3
+    keep = oracle.mask_nm(W, 2, 4)
+    kept_zero = float(np.mean(wt[keep == 1] == 0))
+    Fk = 2 * F ** 3 * (1 - F) + F ** 4
+    assert abs(kept_zero - Fk) < 6 * math.sqrt(Fk * (1 - Fk) / (n / 2))
+
+
+# ---------------------------------------------------------------- pack
+
+def _decode_group_bytes(gb, k):
+    rows = gb.shape[0]
+    wq = np.zeros((rows, k), np.int8)
+    keep = np.zeros((rows, k), np.uint8)
+    val = {0: 0, 1: 1, 3: -1}
+    for r in range(rows):
+        for g in range(k // 4):
+            b = int(gb[r, g])
+            i0, i1, c0, c1 = b & 3, (b >> 2) & 3, (b >> 4) & 3, (b >> 6) & 3
+            assert i0 < i1 and c0 != 2 and c1 != 2
+            keep[r, 4 * g + i0] = keep[r, 4 * g + i1] = 1
+            wq[r, 4 * g + i0] = val[c0]
+            wq[r, 4 * g + i1] = val[c1]
+    return wq, keep
+
+
+def test_pack_round_trip_and_invariants():
+    W = synth.master_weights(40, 128, 0.02, 9)
+    g, keep, wq, gb = oracle.pack_weights(W)
+    assert set(np.unique(wq)).issubset({-1, 0, 1})
+    assert np.all(keep.reshape(40, -1, 4).sum(-1) == 2)
+    assert np.all((wq != 0).reshape(40, -1, 4).sum(-1) <= 2)
+    dwq, dkeep = _decode_group_bytes(gb, 128)
+    assert np.array_equal(dwq, wq) and np.array_equal(dkeep, keep)
+
+
+# ---------------------------------------------------------------- golden forward
+
+def test_worked_example():
+    G = load_golden("worked_2x8.txt")
+    f = lambda k: np.array([float(v) for v in G[k]], np.float32)
+    i = lambda k: np.array([int(v) for v in G[k]])
+    W = f("W").reshape(2, 8)
+    X = f("X").reshape(2, 8)
+    eps_w, eps_a = float(G["eps_w"][0]), float(G["eps_a"][0])
+    out = oracle.forward(W, X, eps_w, eps_a)
+    assert out["gamma"] == np.float32(float(G["gamma"][0]))
+    assert out["keep"].ravel().tolist() == i("keep").tolist()
+    assert out["wq"].ravel().tolist() == i("wq").tolist()
+    assert out["gb"].ravel().tolist() == i("group_bytes").tolist()
+    assert out["xq"].ravel().tolist() == i("xq").tolist()
+    assert np.array_equal(out["a"], f("a"))
+    assert out["acc"].ravel().tolist() == i("acc").tolist()
+    y_exact = np.array([float(v) for v in G["y_num"]]) / float(G["y_den"][0])
+    assert np.allclose(out["y"].ravel(), y_exact, rtol=1e-6, atol=0)
+    dY = f("dY").reshape(1, 2)
+    dX, _ = oracle.dgrad(dY, out["wq"], out["gamma"])
+    assert np.array_equal(dX.ravel(), np.array([float(v) for v in G["dX"]]))
+
+
+# ---------------------------------------------------------------- activations
+
+def test_quant_act_invariants():
+    X = synth.activations(33, 200, 3, outlier_p=0.01)
+    Xq, a = oracle.quant_act(X)
+    assert Xq.dtype == np.int8 and np.all(np.abs(Xq.astype(int)) <= 127)
+    assert np.all(np.abs(Xq.astype(int)).max(1) == 127)       # the absmax element maps to 127
+    assert np.array_equal(a, np.maximum(np.abs(X).max(1), np.float32(1e-5)))
+    Xn, an = oracle.quant_act(-X)
+    assert np.array_equal(Xn, -Xq) and np.array_equal(an, a)   # symmetric, no zero-point
+    # codes are monotone in x within a token
+    for t in range(4):
+        o = np.argsort(X[t], kind="stable")
+        assert np.all(np.diff(Xq[t][o].astype(int)) >= 0)
+
+
+def test_quant_act_zero_row_uses_eps():
+    X = np.zeros((2, 16), np.float32)
+    X[1, 3] = 1e-7
+    Xq, a = oracle.quant_act(X, 1e-5)
+    assert np.all(Xq[0] == 0) and a[0] == np.float32(1e-5)
+    assert a[1] == np.float32(1e-5) and Xq[1, 3] == round(1e-7 * 127 / 1e-5)
+
+
+# ---------------------------------------------------------------- products
+
+def test_gemm_i32_matches_numpy_int64():
+    r = np.random.default_rng(2)
+    Xq = r.integers(-127, 128, size=(17, 96)).astype(np.int8)
+    Wq = r.integers(-1, 2, size=(40, 96)).astype(np.int8)
+    ref = Xq.astype(np.int64) @ Wq.astype(np.int64).T
+    assert np.array_equal(oracle.gemm_i32(Xq, Wq), ref)
+
+
+def test_gemm_i32_extreme_accumulator():
+    K = 4096
+    Xq = np.full((2, K), 127, np.int8)
+    Xq[1] = -127
+    Wq = np.zeros((1, K), np.int8)
+    Wq[0, ::2] = 1        # 2:4-feasible: half the weights non-zero
+    assert oracle.gemm_i32(Xq, Wq).ravel().tolist() == [127 * K // 2, -127 * K // 2]
+
+
+def test_forward_matches_dense_masked_brute_force():
+    W = synth.master_weights(48, 64, 0.02, 13)
+    X = synth.activations(5, 64, 14)
+    out = oracle.forward(W, X)
+    # brute force: dense fp64 product of dequantised operands
+    yb = (out["xq"].astype(np.float64) * out["a"][:, None] / 127.0) @ \
+         (out["wq"].astype(np.float64) * float(out["gamma"])).T
+    assert np.allclose(out["y"], yb, rtol=2e-6, atol=1e-7)
+    # and the method approximates the full-precision product of the masked weights
+    yfp = X.astype(np.float64) @ (out["wq"] * float(out["gamma"])).T
+    bound = (np.abs(out["wq"]).astype(np.float64) * float(out["gamma"])).sum(1)[None, :] \
+        * (out["a"][:, None] / 127.0) * 0.5 + 1e-6
+    assert np.all(np.abs(out["y"] - yfp) <= bound)
+
+
+def test_dgrad_matches_numpy_fp64():
+    r = np.random.default_rng(8)
+    dY = r.normal(size=(6, 40)).astype(np.float32)
+    Wq = r.integers(-1, 2, size=(40, 24)).astype(np.int8)
+    dX, absdX = oracle.dgrad(dY, Wq, np.float32(0.0173))
+    ref = (dY.astype(np.float64) @ Wq.astype(np.float64)) * float(np.float32(0.0173))
+    assert np.allclose(dX, ref, rtol=1e-12, atol=1e-12)
+    assert np.all(absdX >= np.abs(dX) - 1e-12)
+
+
+def test_quant_act_ties_golden():
+    G = load_golden("quant_ties.txt")
+    X = np.array([float(v) for v in G["X"]], np.float32).reshape(2, 8)
+    Xq, a = oracle.quant_act(X)
+    assert Xq.ravel().tolist() == [int(v) for v in G["xq"]]
+    assert a.tolist() == [float(v) for v in G["a"]]
