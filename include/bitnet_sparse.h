@@ -1,0 +1,200 @@
+/*
+ * bitnet_sparse.h - C ABI of the sparse ternary BitLinear hot path (sm_100a).
+ *
+ * The library implements the forward of one Sparse-BitLinear layer and its
+ * straight-through input gradient:
+ *   pack   : W (fp32 masters) -> 2:4 mask, absmean ternary codes, packed layouts
+ *   quant  : X -> per-token int8 codes and absmax scales
+ *   linear : Y = dequant(Xq . Wq^T)   (int8 x ternary, int32 accumulation)
+ *   dgrad  : dX = gamma * dY . Wq     (straight-through estimator)
+ *
+ * Conventions shared by every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     allocates no memory, never frees, and never synchronises a stream unless
+ *     the entry point says so (bitnet_read_device_status).
+ *   - Every call is asynchronous on `stream` and returns after enqueueing.
+ *   - Arguments are validated on the host before any launch; a failed check
+ *     returns an error status and enqueues nothing.
+ *   - Matrices are row-major with the last index contiguous.
+ *   - No C++ exception crosses this boundary.
+ *   - A call with T == 0 (empty batch) validates its sizes, launches nothing,
+ *     and accepts NULL activation / output buffers.
+ *   - bitnet_last_error() returns a human-readable detail of the last failure
+ *     on the calling thread.
+ */
+#ifndef BITNET_SPARSE_H
+#define BITNET_SPARSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st *bitnet_stream_t;
+
+typedef enum {
+    BITNET_OK = 0,
+    BITNET_ERR_INVALID_ARG = 1,   /* null pointer, bad size, bad alignment */
+    BITNET_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. N:M other than 2:4 for packing) */
+    BITNET_ERR_WORKSPACE = 3,     /* workspace missing or smaller than *_workspace_size() */
+    BITNET_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    BITNET_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (see bitnet_read_device_status) */
+} bitnet_status;
+
+typedef enum { BITNET_F32 = 0, BITNET_BF16 = 1 } bitnet_dtype;
+
+/*
+ * Packed weights of one layer, W in R^{n_out x k}.  Filled by bitnet_pack_nm and
+ * read by bitnet_sparse_linear / bitnet_dgrad.  Every pointer is a device
+ * buffer of the size given below, allocated by the caller; a NULL layout
+ * pointer means "not produced / not available".
+ *
+ *   n, m         N:M pattern; the packed layouts exist for n = 2, m = 4.
+ *   gamma        1 float: the absmean scale (required).
+ *   group_bytes  [n_out, k/4] bytes, canonical 2:4 group byte per 4 weights:
+ *                bits 0-1 idx0, bits 2-3 idx1 (idx0 < idx1: the two kept
+ *                positions), bits 4-5 code(idx0), bits 6-7 code(idx1); code
+ *                00 = 0, 01 = +1, 11 = -1.  Needs k % 4 == 0.
+ *   mma_vals     [n_out, k/2] int8: the two kept codes of every group, in k
+ *                order (the compressed sparse operand of the tensor-core GEMM).
+ *   mma_meta     bitnet_mma_meta_bytes(n_out, k) bytes: the 2:4 metadata in
+ *                blocks of 128 rows x 128 k (16 bytes per row, one 4-bit
+ *                nibble idx0 | idx1 << 2 per group, low nibble first), block
+ *                (kb, rb) at byte offset (kb * ceil(n_out/128) + rb) * 2048.
+ *                Rows >= n_out and k >= k of the padded blocks hold idx (0,1).
+ *   dec_codes    bitnet_dec_bytes(n_out, k) bytes: decode (GEMV) layout.  For
+ *                every 16-row x 64-k tile, 32 lanes x 8 bytes: a 32-bit word
+ *                of 16 two-bit codes and a 32-bit word of 8 metadata nibbles,
+ *                in the register order of the warp-level sparse MMA.  Needs
+ *                n_out % 16 == 0 and k % 64 == 0.
+ */
+typedef struct {
+    int64_t n_out;
+    int64_t k;
+    int32_t n;
+    int32_t m;
+    float *gamma;
+    uint8_t *group_bytes;
+    int8_t *mma_vals;
+    uint8_t *mma_meta;
+    uint8_t *dec_codes;
+} bitnet_packed_w;
+
+/* Buffer sizes of the layouts above (bytes). */
+size_t bitnet_mma_meta_bytes(int64_t n_out, int64_t k);
+size_t bitnet_dec_bytes(int64_t n_out, int64_t k);
+
+/* ------------------------------------------------------------------------
+ * bitnet_pack_nm - per-step mask + ternarise + pack.
+ *
+ * Follows "Sparse-BitNet" (gist.science technical summary), section 2
+ * "Kerncomponenten": the N:M mask is chosen from the magnitudes of the master
+ * weights (top-N of every M consecutive weights along k, ties to the lower
+ * position); the forward quantises to ternary and then applies the mask;
+ * "Training Strategie": the mask is recomputed every step.  The quantiser is
+ * the absmean one of "BitNet b1.58: Ternary Weights for 1.58-bit LLMs",
+ * section "The mechanism":
+ *   gamma = fp32(fp64_rn(exact sum |W|) / (n_out*k)) + eps   (fp32 add)
+ *   code  = clip(rint_half_even(fp32(W / gamma)), -1, 1) for kept weights, 0 else.
+ * gamma is bit-exact and independent of summation order.
+ *
+ *   W         [n_out, k] fp32, 16-byte aligned, k % m == 0.
+ *   out       layouts to fill: out->gamma required; each of group_bytes,
+ *             mma_vals + mma_meta (together), dec_codes is written when
+ *             non-NULL (these need n == 2, m == 4).
+ *   eps       added to the mean (>= 0).
+ *   mask_bits [n_out, k/8] bytes or NULL: bit (c % 8) of byte (r*k + c)/8 is 1
+ *             when weight (r, c) is kept.  Supports any 1 <= n < m, m in {4, 8}.
+ *   ws        device workspace of >= bitnet_pack_workspace_size() bytes,
+ *             16-byte aligned; contents on entry are ignored.
+ * Errors: INVALID_ARG (null W / gamma / ws, bad sizes or alignment),
+ *         UNSUPPORTED (packed layouts requested with n:m != 2:4),
+ *         WORKSPACE (ws_bytes too small), CUDA (launch failure).
+ * ------------------------------------------------------------------------ */
+size_t bitnet_pack_workspace_size(int64_t n_out, int64_t k);
+bitnet_status bitnet_pack_nm(const float *W, bitnet_packed_w *out, float eps,
+                             uint8_t *mask_bits, void *ws, size_t ws_bytes,
+                             bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_quant_act - per-token absmax int8 activation quantisation.
+ *
+ * "BitNet b1.58: Ternary Weights for 1.58-bit LLMs", section "The mechanism"
+ * (Activations): each token is scaled to [-Q_b, Q_b], symmetric, with no
+ * zero-point; Q_b = 127:
+ *   a[t] = max(max_k |X[t,k]|, eps);  s = 127 / a[t] (fp32);
+ *   Xq[t,k] = clamp(rint_half_even(fp32(X[t,k] * s)), -127, 127).
+ *
+ *   X       [T, K] fp32 or bf16 (x_dtype), 16-byte aligned, K % 8 == 0.
+ *   Xq      [T, K] int8 out, 16-byte aligned.   absmax  [T] fp32 out (= a[t]).
+ * Errors: INVALID_ARG, CUDA.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, int64_t K,
+                               float eps, int8_t *Xq, float *absmax, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_sparse_linear - Y = dequant(Xq . Wq^T).
+ *
+ * "BitNet b1.58 ...", section "The mechanism": with ternary weights each
+ * output is a signed sum of activations; "Sparse-BitNet" section 2: the masked
+ * ternary weights are used in the forward pass.
+ *   acc[t,n] = sum_k Xq[t,k] * Wq[n,k]      (int32, exact)
+ *   Y[t,n]   = fp32(acc) * ((gamma * absmax[t]) / 127)   -> fp32 or bf16
+ *
+ *   Xq      [T, K] int8 (from bitnet_quant_act), 16-byte aligned.
+ *   absmax  [T] fp32.
+ *   W       packed weights with K == W->k.  T <= 8 runs the decode GEMV and
+ *           needs W->dec_codes (or W->group_bytes); T > 8 runs the tensor-core
+ *           GEMM and needs W->mma_vals + W->mma_meta, with k % 32 == 0.
+ *   Y       [T, n_out] of y_dtype.
+ *   acc_out [T, n_out] int32 or NULL: raw accumulators (for checking).
+ *   ws      >= bitnet_linear_workspace_size() bytes of device memory, holding
+ *           the device status word of the bounded waits.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+size_t bitnet_linear_workspace_size(void);
+bitnet_status bitnet_sparse_linear(const int8_t *Xq, const float *absmax,
+                                   const bitnet_packed_w *W, int64_t T,
+                                   void *Y, bitnet_dtype y_dtype, int32_t *acc_out,
+                                   void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_dgrad - straight-through input gradient dX = gamma * dY . Wq.
+ *
+ * "Sparse-BitNet" (gist.science technical summary), section 2 "Training
+ * Strategie": both the quantiser and the top-N selection pass the gradient
+ * straight through (dual STE), so the input gradient flows through the
+ * masked ternary weights.  Dense in the contraction over n_out (the 2:4
+ * structure lies along k), bf16 operands, fp32 accumulation.
+ *
+ *   dY      [T, n_out] bf16 (dy_dtype must be BITNET_BF16), 16-byte aligned,
+ *           n_out % 8 == 0.
+ *   W       packed weights with group_bytes.
+ *   dX      [T, k] fp32 or bf16 (dx_dtype).
+ *   ws      >= bitnet_dgrad_workspace_size(W) bytes (holds the expanded bf16
+ *           transpose of gamma-free Wq and the status word).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+size_t bitnet_dgrad_workspace_size(int64_t n_out, int64_t k);
+bitnet_status bitnet_dgrad(const void *dY, bitnet_dtype dy_dtype, const bitnet_packed_w *W,
+                           int64_t T, void *dX, bitnet_dtype dx_dtype,
+                           void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Status helpers.
+ * bitnet_read_device_status synchronises `stream`, reads the status word that
+ * the kernels of the last call on `ws` left (BITNET_OK or BITNET_ERR_TIMEOUT
+ * when a bounded wait gave up) and clears it.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_read_device_status(void *ws, bitnet_stream_t stream);
+const char *bitnet_status_string(bitnet_status s);
+const char *bitnet_last_error(void);
+int bitnet_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BITNET_SPARSE_H */

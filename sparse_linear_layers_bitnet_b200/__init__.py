@@ -1,0 +1,16 @@
+"""Sparse ternary BitLinear (Sparse-BitNet hot path) for NVIDIA B200 (sm_100a).
+
+The compute lives in libbitnet_sparse.so (CUDA kernels behind a C ABI, see
+include/bitnet_sparse.h); this package is its thin Python binding plus the
+seeded synthetic input generators.
+"""
+from ._abi import (  # noqa: F401
+    BITNET_BF16, BITNET_F32, BitnetError, BitnetPackedW, PackedWeights, Workspace,
+    bitnet_dgrad, bitnet_pack_nm, bitnet_quant_act, bitnet_read_device_status, bitnet_sparse_linear, load,
+)
+
+__all__ = [
+    "PackedWeights", "Workspace", "BitnetError", "BitnetPackedW", "load",
+    "bitnet_pack_nm", "bitnet_quant_act", "bitnet_sparse_linear", "bitnet_dgrad", "bitnet_read_device_status",
+    "BITNET_F32", "BITNET_BF16",
+]

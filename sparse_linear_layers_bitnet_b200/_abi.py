@@ -1,0 +1,226 @@
+"""ctypes binding of libbitnet_sparse.so (the C ABI in include/bitnet_sparse.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels.  PyTorch supplies device memory and the current stream.  If the
+library is missing the import fails loudly; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libbitnet_sparse.so")
+
+BITNET_OK = 0
+BITNET_ERR_INVALID_ARG = 1
+BITNET_ERR_UNSUPPORTED = 2
+BITNET_ERR_WORKSPACE = 3
+BITNET_ERR_CUDA = 4
+BITNET_ERR_TIMEOUT = 5
+
+BITNET_F32 = 0
+BITNET_BF16 = 1
+
+# Every symbol include/bitnet_sparse.h declares.
+EXPORTED = [
+    "bitnet_mma_meta_bytes", "bitnet_dec_bytes",
+    "bitnet_pack_workspace_size", "bitnet_pack_nm",
+    "bitnet_quant_act",
+    "bitnet_linear_workspace_size", "bitnet_sparse_linear",
+    "bitnet_dgrad_workspace_size", "bitnet_dgrad",
+    "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
+]
+
+
+class BitnetPackedW(ctypes.Structure):
+    _fields_ = [
+        ("n_out", ctypes.c_int64),
+        ("k", ctypes.c_int64),
+        ("n", ctypes.c_int32),
+        ("m", ctypes.c_int32),
+        ("gamma", ctypes.c_void_p),
+        ("group_bytes", ctypes.c_void_p),
+        ("mma_vals", ctypes.c_void_p),
+        ("mma_meta", ctypes.c_void_p),
+        ("dec_codes", ctypes.c_void_p),
+    ]
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: status {status} ({detail})")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with "
+                          "`python -m sparse_linear_layers_bitnet_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    P, I64, SZ, F, I32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float, ctypes.c_int
+    sig = {
+        "bitnet_mma_meta_bytes": (SZ, [I64, I64]),
+        "bitnet_dec_bytes": (SZ, [I64, I64]),
+        "bitnet_pack_workspace_size": (SZ, [I64, I64]),
+        "bitnet_pack_nm": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P, SZ, P]),
+        "bitnet_quant_act": (I32, [P, I32, I64, I64, F, P, P, P]),
+        "bitnet_linear_workspace_size": (SZ, []),
+        "bitnet_sparse_linear": (I32, [P, P, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, SZ, P]),
+        "bitnet_dgrad_workspace_size": (SZ, [I64, I64]),
+        "bitnet_dgrad": (I32, [P, I32, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, SZ, P]),
+        "bitnet_read_device_status": (I32, [P, P]),
+        "bitnet_status_string": (ctypes.c_char_p, [I32]),
+        "bitnet_last_error": (ctypes.c_char_p, []),
+        "bitnet_abi_version": (I32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def check(status: int, where: str) -> None:
+    if status != BITNET_OK:
+        lib = load()
+        raise BitnetError(status, where, lib.bitnet_last_error().decode(errors="replace"))
+
+
+# ------------------------------------------------------------------ torch helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(dt) -> int:
+    torch = _torch()
+    if dt == torch.float32:
+        return BITNET_F32
+    if dt == torch.bfloat16:
+        return BITNET_BF16
+    raise ValueError(f"unsupported dtype {dt}")
+
+
+class PackedWeights:
+    """Device buffers of one packed layer (see bitnet_packed_w in the header)."""
+
+    def __init__(self, n_out: int, k: int, device="cuda", group_bytes=True, mma=True, dec=True,
+                 n: int = 2, m: int = 4):
+        torch = _torch()
+        lib = load()
+        self.n_out, self.k, self.n, self.m = int(n_out), int(k), int(n), int(m)
+        self.gamma = torch.zeros(1, dtype=torch.float32, device=device)
+        self.group_bytes = torch.empty((n_out, k // 4), dtype=torch.uint8, device=device) if group_bytes else None
+        self.mma_vals = torch.empty((n_out, k // 2), dtype=torch.int8, device=device) if mma else None
+        self.mma_meta = (torch.empty(lib.bitnet_mma_meta_bytes(n_out, k), dtype=torch.uint8, device=device)
+                         if mma else None)
+        nd = lib.bitnet_dec_bytes(n_out, k)
+        self.dec_codes = torch.empty(nd, dtype=torch.uint8, device=device) if (dec and nd > 0) else None
+        self._struct = None
+
+    def struct(self) -> BitnetPackedW:
+        s = BitnetPackedW()
+        s.n_out, s.k, s.n, s.m = self.n_out, self.k, self.n, self.m
+        s.gamma = self.gamma.data_ptr()
+        s.group_bytes = self.group_bytes.data_ptr() if self.group_bytes is not None else None
+        s.mma_vals = self.mma_vals.data_ptr() if self.mma_vals is not None else None
+        s.mma_meta = self.mma_meta.data_ptr() if self.mma_meta is not None else None
+        s.dec_codes = self.dec_codes.data_ptr() if self.dec_codes is not None else None
+        self._struct = s
+        return s
+
+
+class Workspace:
+    """A device byte buffer for the ws argument of the entry points."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        torch = _torch()
+        self.nbytes = int(max(nbytes, 256))
+        self.buf = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.buf.data_ptr())
+
+
+def bitnet_pack_nm(W, out: PackedWeights, eps: float = 1e-5, mask_bits=None, ws: Workspace | None = None,
+                   stream=None):
+    lib = load()
+    assert W.dtype == _torch().float32 and W.is_contiguous()
+    if ws is None:
+        ws = Workspace(lib.bitnet_pack_workspace_size(out.n_out, out.k), W.device)
+    st = out.struct()
+    check(lib.bitnet_pack_nm(_ptr(W), ctypes.byref(st), ctypes.c_float(eps), _ptr(mask_bits), ws.ptr,
+                             ws.nbytes, _stream(stream)), "bitnet_pack_nm")
+    return out
+
+
+def bitnet_quant_act(X, eps: float = 1e-5, Xq=None, absmax=None, stream=None):
+    torch = _torch()
+    lib = load()
+    assert X.is_contiguous() and X.dim() == 2
+    T, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((T, K), dtype=torch.int8, device=X.device)
+    if absmax is None:
+        absmax = torch.empty((T,), dtype=torch.float32, device=X.device)
+    check(lib.bitnet_quant_act(_ptr(X), _dtype_code(X.dtype), T, K, ctypes.c_float(eps), _ptr(Xq), _ptr(absmax),
+                               _stream(stream)), "bitnet_quant_act")
+    return Xq, absmax
+
+
+def bitnet_sparse_linear(Xq, absmax, W: PackedWeights, Y=None, y_dtype=None, acc_out=None,
+                         ws: Workspace | None = None, stream=None):
+    torch = _torch()
+    lib = load()
+    T = Xq.shape[0]
+    if y_dtype is None:
+        y_dtype = torch.bfloat16
+    if Y is None:
+        Y = torch.empty((T, W.n_out), dtype=y_dtype, device=Xq.device)
+    if ws is None:
+        ws = Workspace(lib.bitnet_linear_workspace_size(), Xq.device)
+    st = W.struct()
+    check(lib.bitnet_sparse_linear(_ptr(Xq), _ptr(absmax), ctypes.byref(st), T, _ptr(Y), _dtype_code(Y.dtype),
+                                   _ptr(acc_out), ws.ptr, ws.nbytes, _stream(stream)), "bitnet_sparse_linear")
+    return Y
+
+
+def bitnet_dgrad(dY, W: PackedWeights, dX=None, dx_dtype=None, ws: Workspace | None = None, stream=None):
+    torch = _torch()
+    lib = load()
+    T = dY.shape[0]
+    if dx_dtype is None:
+        dx_dtype = torch.float32
+    if dX is None:
+        dX = torch.empty((T, W.k), dtype=dx_dtype, device=dY.device)
+    if ws is None:
+        ws = Workspace(lib.bitnet_dgrad_workspace_size(W.n_out, W.k), dY.device)
+    st = W.struct()
+    check(lib.bitnet_dgrad(_ptr(dY), _dtype_code(dY.dtype), ctypes.byref(st), T, _ptr(dX), _dtype_code(dX.dtype),
+                           ws.ptr, ws.nbytes, _stream(stream)), "bitnet_dgrad")
+    return dX
+
+
+def bitnet_read_device_status(ws: Workspace, stream=None) -> int:
+    return load().bitnet_read_device_status(ws.ptr, _stream(stream))

@@ -1,0 +1,188 @@
+// C ABI of the sparse ternary BitLinear library: host-side argument checks,
+// shape dispatch and launches.  Declarations and semantics: bitnet_sparse.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/bitnet_sparse.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+bitnet_status fail(bitnet_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof g_err, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+bitnet_status cuda_status(cudaError_t e, const char *what) {
+    if (e == cudaSuccess) return BITNET_OK;
+    return fail(BITNET_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+extern "C" {
+
+int bitnet_abi_version(void) { return 1; }
+
+const char *bitnet_last_error(void) { return g_err; }
+
+const char *bitnet_status_string(bitnet_status s) {
+    switch (s) {
+        case BITNET_OK: return "ok";
+        case BITNET_ERR_INVALID_ARG: return "invalid argument";
+        case BITNET_ERR_UNSUPPORTED: return "unsupported configuration";
+        case BITNET_ERR_WORKSPACE: return "workspace missing or too small";
+        case BITNET_ERR_CUDA: return "CUDA error";
+        case BITNET_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+size_t bitnet_mma_meta_bytes(int64_t n_out, int64_t k) {
+    if (n_out <= 0 || k <= 0) return 0;
+    return static_cast<size_t>(ceil_div(k, 128) * ceil_div(n_out, 128) * 2048);
+}
+
+size_t bitnet_dec_bytes(int64_t n_out, int64_t k) {
+    if (n_out <= 0 || k <= 0 || n_out % 16 || k % 64) return 0;
+    return static_cast<size_t>(n_out / 16) * static_cast<size_t>(k / 64) * 256;
+}
+
+size_t bitnet_pack_workspace_size(int64_t, int64_t) { return bitnet::kPackWsBytes; }
+size_t bitnet_linear_workspace_size(void) { return bitnet::kLinearWsBytes; }
+size_t bitnet_dgrad_workspace_size(int64_t n_out, int64_t k) {
+    if (n_out <= 0 || k <= 0) return bitnet::kDgradWsHeader;
+    return bitnet::kDgradWsHeader + static_cast<size_t>(n_out) * static_cast<size_t>(k) * 2;
+}
+
+bitnet_status bitnet_pack_nm(const float *W, bitnet_packed_w *out, float eps, uint8_t *mask_bits, void *ws,
+                             size_t ws_bytes, bitnet_stream_t stream) {
+    if (!W || !out || !out->gamma) return fail(BITNET_ERR_INVALID_ARG, "pack: W, out and out->gamma are required");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "pack: workspace is required");
+    if (ws_bytes < bitnet::kPackWsBytes) return fail(BITNET_ERR_WORKSPACE, "pack: workspace needs %zu bytes", bitnet::kPackWsBytes);
+    const int64_t n_out = out->n_out, k = out->k;
+    const int n = out->n, m = out->m;
+    if (n_out <= 0 || k <= 0) return fail(BITNET_ERR_INVALID_ARG, "pack: n_out and k must be positive");
+    if (!(m == 4 || m == 8) || n < 1 || n >= m) return fail(BITNET_ERR_UNSUPPORTED, "pack: N:M must have m in {4,8}, 1 <= n < m");
+    if (k % 8 != 0) return fail(BITNET_ERR_INVALID_ARG, "pack: k must be a multiple of 8");
+    if (!(eps >= 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "pack: eps must be >= 0");
+    if (!aligned(W, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "pack: W and ws must be 16-byte aligned");
+    const bool packed = out->group_bytes || out->mma_vals || out->mma_meta || out->dec_codes;
+    if (packed && !(n == 2 && m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "pack: packed layouts exist for 2:4 only");
+    if ((out->mma_vals == nullptr) != (out->mma_meta == nullptr))
+        return fail(BITNET_ERR_INVALID_ARG, "pack: mma_vals and mma_meta go together");
+    if (out->mma_vals && (!aligned(out->mma_vals, 16) || !aligned(out->mma_meta, 16)))
+        return fail(BITNET_ERR_INVALID_ARG, "pack: mma layouts must be 16-byte aligned");
+    if (out->dec_codes) {
+        if (!out->group_bytes) return fail(BITNET_ERR_INVALID_ARG, "pack: dec_codes are derived from group_bytes");
+        if (n_out % 16 || k % 64) return fail(BITNET_ERR_UNSUPPORTED, "pack: dec_codes need n_out %% 16 == 0, k %% 64 == 0");
+        if (!aligned(out->dec_codes, 16)) return fail(BITNET_ERR_INVALID_ARG, "pack: dec_codes must be 16-byte aligned");
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return cuda_status(bitnet::launch_pack(W, n_out, k, n, m, eps, out->gamma, out->group_bytes, out->mma_vals,
+                                           out->mma_meta, out->dec_codes, mask_bits, ws, s),
+                       "pack");
+}
+
+bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, int64_t K, float eps, int8_t *Xq,
+                               float *absmax, bitnet_stream_t stream) {
+    if (T < 0 || K <= 0 || K % 8) return fail(BITNET_ERR_INVALID_ARG, "quant_act: need T >= 0, K > 0, K %% 8 == 0");
+    if (T == 0) return BITNET_OK;   // an empty batch needs no buffers
+    if (!X || !Xq || !absmax) return fail(BITNET_ERR_INVALID_ARG, "quant_act: null pointer");
+    if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return fail(BITNET_ERR_INVALID_ARG, "quant_act: bad dtype");
+    if (!aligned(X, 16) || !aligned(Xq, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_act: X and Xq must be 16-byte aligned");
+    if (!(eps > 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "quant_act: eps must be > 0");
+    if (T > 2147483647LL) return fail(BITNET_ERR_UNSUPPORTED, "quant_act: T too large");
+    return cuda_status(bitnet::launch_quant_act(X, x_dtype == BITNET_BF16, T, K, eps, Xq, absmax,
+                                                reinterpret_cast<cudaStream_t>(stream)),
+                       "quant_act");
+}
+
+bitnet_status bitnet_sparse_linear(const int8_t *Xq, const float *absmax, const bitnet_packed_w *W, int64_t T,
+                                   void *Y, bitnet_dtype y_dtype, int32_t *acc_out, void *ws, size_t ws_bytes,
+                                   bitnet_stream_t stream) {
+    if (!W || !W->gamma) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: null W or gamma");
+    if (T != 0 && (!Xq || !absmax || !Y)) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: null pointer");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "sparse_linear: workspace is required");
+    if (ws_bytes < bitnet::kLinearWsBytes) return fail(BITNET_ERR_WORKSPACE, "sparse_linear: workspace needs %zu bytes", bitnet::kLinearWsBytes);
+    if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: bad dtype");
+    const int64_t n_out = W->n_out, k = W->k;
+    if (T < 0 || n_out <= 0 || k <= 0 || k % 8) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: bad sizes");
+    if (!(W->n == 2 && W->m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "sparse_linear: 2:4 only");
+    if (T == 0) return BITNET_OK;   // an empty batch needs no buffers
+    if (!aligned(Xq, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: Xq and ws must be 16-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool bf16 = y_dtype == BITNET_BF16;
+    if (T <= 8) {
+        if (W->dec_codes && n_out % 16 == 0 && k % 64 == 0) {
+            if (!aligned(W->dec_codes, 16)) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: dec_codes alignment");
+            return cuda_status(bitnet::launch_gemv_dec(Xq, absmax, W->gamma, W->dec_codes, T, n_out, k, Y, bf16,
+                                                       acc_out, s),
+                               "sparse_linear (decode GEMV)");
+        }
+        if (W->group_bytes)
+            return cuda_status(bitnet::launch_gemv_gb(Xq, absmax, W->gamma, W->group_bytes, T, n_out, k, Y, bf16,
+                                                      acc_out, s),
+                               "sparse_linear (group-byte GEMV)");
+        if (!W->mma_vals) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: no packed layout for T <= 8");
+    }
+    if (!W->mma_vals || !W->mma_meta) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: T > 8 needs mma_vals and mma_meta");
+    if (k % 32) return fail(BITNET_ERR_UNSUPPORTED, "sparse_linear: the tensor-core path needs k %% 32 == 0");
+    if (!aligned(W->mma_vals, 16) || !aligned(W->mma_meta, 16)) return fail(BITNET_ERR_INVALID_ARG, "sparse_linear: mma layouts must be 16-byte aligned");
+    if (n_out > 2147483647LL / 2 || T > 65535LL * 256) return fail(BITNET_ERR_UNSUPPORTED, "sparse_linear: sizes too large");
+    uint32_t *status = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + bitnet::kStatusOffset);
+    return cuda_status(bitnet::launch_gemm_sp(Xq, absmax, W->gamma, W->mma_vals, W->mma_meta, T, n_out, k, Y, bf16,
+                                              acc_out, status, s),
+                       "sparse_linear (tensor-core GEMM)");
+}
+
+bitnet_status bitnet_dgrad(const void *dY, bitnet_dtype dy_dtype, const bitnet_packed_w *W, int64_t T, void *dX,
+                           bitnet_dtype dx_dtype, void *ws, size_t ws_bytes, bitnet_stream_t stream) {
+    if (!W || !W->gamma) return fail(BITNET_ERR_INVALID_ARG, "dgrad: null W or gamma");
+    if (T != 0 && (!dY || !dX)) return fail(BITNET_ERR_INVALID_ARG, "dgrad: null pointer");
+    if (!W->group_bytes) return fail(BITNET_ERR_INVALID_ARG, "dgrad: needs W->group_bytes");
+    if (dy_dtype != BITNET_BF16) return fail(BITNET_ERR_UNSUPPORTED, "dgrad: dY must be bf16");
+    if (dx_dtype != BITNET_F32 && dx_dtype != BITNET_BF16) return fail(BITNET_ERR_INVALID_ARG, "dgrad: bad dX dtype");
+    const int64_t n_out = W->n_out, k = W->k;
+    if (T < 0 || n_out <= 0 || k <= 0 || k % 8 || n_out % 8) return fail(BITNET_ERR_INVALID_ARG, "dgrad: bad sizes (k, n_out multiples of 8)");
+    if (!(W->n == 2 && W->m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "dgrad: 2:4 only");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "dgrad: workspace is required");
+    if (ws_bytes < bitnet_dgrad_workspace_size(n_out, k)) return fail(BITNET_ERR_WORKSPACE, "dgrad: workspace needs %zu bytes", bitnet_dgrad_workspace_size(n_out, k));
+    if (T == 0) return BITNET_OK;   // an empty batch needs no buffers
+    if (!aligned(dY, 16) || !aligned(dX, 16) || !aligned(ws, 128)) return fail(BITNET_ERR_INVALID_ARG, "dgrad: dY, dX 16-byte and ws 128-byte alignment");
+    if (T > 65535LL * 128) return fail(BITNET_ERR_UNSUPPORTED, "dgrad: T too large");
+    return cuda_status(bitnet::launch_dgrad(dY, W->gamma, W->group_bytes, T, n_out, k, dX,
+                                            dx_dtype == BITNET_BF16, ws, reinterpret_cast<cudaStream_t>(stream)),
+                       "dgrad");
+}
+
+bitnet_status bitnet_read_device_status(void *ws, bitnet_stream_t stream) {
+    if (!ws) return fail(BITNET_ERR_INVALID_ARG, "read_device_status: null workspace");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, static_cast<uint8_t *>(ws) + bitnet::kStatusOffset, sizeof word,
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_status(e, "read_device_status");
+    if (word) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyAsync(static_cast<uint8_t *>(ws) + bitnet::kStatusOffset, &zero, sizeof zero,
+                            cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return cuda_status(e, "read_device_status");
+        return fail(BITNET_ERR_TIMEOUT, "a device-side bounded wait gave up (status word 0x%x)", word);
+    }
+    return BITNET_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,47 @@
+// Host-side launchers of the kernels behind the C ABI (internal header).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bitnet {
+
+// Workspace layout shared by the entry points: the device status word is
+// always the first 4 bytes.
+constexpr size_t kStatusOffset = 0;
+// pack: threshold bits, 128-bit window sum, 256 exponent bins
+constexpr size_t kPackWsThrOffset = 8;
+constexpr size_t kPackWsWinOffset = 16;
+constexpr size_t kPackWsBinsOffset = 256;
+constexpr size_t kPackWsBytes = 256 + 256 * 8;
+// linear: status word only
+constexpr size_t kLinearWsBytes = 256;
+// dgrad: status word, then the bf16 [k, n_out] expansion of Wq^T
+constexpr size_t kDgradWsHeader = 256;
+
+int num_sms();
+
+cudaError_t launch_pack(const float *W, int64_t n_out, int64_t k, int n, int m, float eps, float *gamma,
+                        uint8_t *gb, int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws,
+                        cudaStream_t s);
+
+cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xq, float *amax,
+                             cudaStream_t s);
+
+cudaError_t launch_gemv_dec(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *dec,
+                            int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
+                            cudaStream_t s);
+
+cudaError_t launch_gemv_gb(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *gb,
+                           int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
+                           cudaStream_t s);
+
+cudaError_t launch_gemm_sp(const int8_t *Xq, const float *amax, const float *gamma, const int8_t *vals,
+                           const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16,
+                           int32_t *acc, uint32_t *status, cudaStream_t s);
+
+cudaError_t launch_dgrad(const void *dY, const float *gamma, const uint8_t *gb, int64_t T, int64_t n_out,
+                         int64_t k, void *dX, bool dx_bf16, void *ws, cudaStream_t s);
+
+}  // namespace bitnet

@@ -1,0 +1,132 @@
+// Per-token absmax int8 activation quantisation (sm_100a).
+//
+// "BitNet b1.58: Ternary Weights for 1.58-bit LLMs", section "The mechanism"
+// (Activations): every token is scaled to the symmetric range [-Q_b, Q_b]
+// with no zero-point; Q_b = 127.
+//   a = max(max_k |x_k|, eps),  s = 127 / a,  q_k = clamp(rint(x_k * s), -127, 127)
+// Division, product and rounding are single IEEE operations (round to
+// nearest even), so the codes are bit-exact.
+//
+// One CTA per token.  The row is read once with 16-byte loads into registers,
+// reduced to its absmax, then quantised from registers and written with
+// vector stores: 2 bytes read + 1 byte written per bf16 element.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bitnet {
+
+constexpr int kQuantThreads = 256;
+constexpr int kQuantMaxChunks = 8;   // 16-byte chunks kept in registers per thread
+
+template <bool BF16>
+struct Chunk {
+    static constexpr int kElems = BF16 ? 8 : 4;
+    uint4 raw;
+    __device__ __forceinline__ float get(int j) const {
+        const uint32_t w = (&raw.x)[BF16 ? (j >> 1) : j];
+        if (BF16) return __uint_as_float((j & 1) ? (w & 0xffff0000u) : (w << 16));
+        return __uint_as_float(w);
+    }
+};
+
+__device__ __forceinline__ float block_max(float v, float *s_red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) s_red[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+        v = (lane < (int)(blockDim.x >> 5)) ? s_red[lane] : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+        if (lane == 0) s_red[0] = v;
+    }
+    __syncthreads();
+    return s_red[0];
+}
+
+__device__ __forceinline__ int8_t quant_one(float x, float s) {
+    const float p = __fmul_rn(x, s);
+    int q = __float2int_rn(p);
+    q = q > 127 ? 127 : (q < -127 ? -127 : q);
+    return static_cast<int8_t>(q);
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(kQuantThreads) k_quant_act(const uint4 *__restrict__ X, int64_t K, float eps,
+                                                             int8_t *__restrict__ Xq, float *__restrict__ amax) {
+    using C = Chunk<BF16>;
+    __shared__ float s_red[32];
+    const int64_t t = blockIdx.x;
+    const int64_t nchunk = K / C::kElems;
+    const uint4 *row = X + t * nchunk;
+    C reg[kQuantMaxChunks];
+    float m = 0.0f;
+    const bool fits = nchunk <= static_cast<int64_t>(kQuantMaxChunks) * kQuantThreads;
+#pragma unroll
+    for (int u = 0; u < kQuantMaxChunks; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        if (c < nchunk) {
+            reg[u].raw = __ldg(row + c);
+#pragma unroll
+            for (int j = 0; j < C::kElems; ++j) m = fmaxf(m, fabsf(reg[u].get(j)));
+        }
+    }
+    if (!fits) {   // rows longer than the register cache: a second read later
+        for (int64_t c = threadIdx.x + static_cast<int64_t>(kQuantMaxChunks) * kQuantThreads; c < nchunk;
+             c += kQuantThreads) {
+            C ch;
+            ch.raw = __ldg(row + c);
+#pragma unroll
+            for (int j = 0; j < C::kElems; ++j) m = fmaxf(m, fabsf(ch.get(j)));
+        }
+    }
+    m = block_max(m, s_red);
+    const float a = m > eps ? m : eps;
+    const float s = __fdiv_rn(127.0f, a);
+    if (threadIdx.x == 0) amax[t] = a;
+    int8_t *out = Xq + t * K;
+#pragma unroll
+    for (int u = 0; u < kQuantMaxChunks; ++u) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        if (c < nchunk) {
+            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < C::kElems; ++j)
+                w[j >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(quant_one(reg[u].get(j), s))) << (8 * (j & 3));
+            if (BF16)
+                *reinterpret_cast<uint2 *>(out + c * 8) = make_uint2(w[0], w[1]);
+            else
+                *reinterpret_cast<uint32_t *>(out + c * 4) = w[0];
+        }
+    }
+    if (!fits) {
+        for (int64_t c = threadIdx.x + static_cast<int64_t>(kQuantMaxChunks) * kQuantThreads; c < nchunk;
+             c += kQuantThreads) {
+            C ch;
+            ch.raw = __ldg(row + c);
+            uint32_t w[2] = {0u, 0u};
+#pragma unroll
+            for (int j = 0; j < C::kElems; ++j)
+                w[j >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(quant_one(ch.get(j), s))) << (8 * (j & 3));
+            if (BF16)
+                *reinterpret_cast<uint2 *>(out + c * 8) = make_uint2(w[0], w[1]);
+            else
+                *reinterpret_cast<uint32_t *>(out + c * 4) = w[0];
+        }
+    }
+}
+
+cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xq, float *amax,
+                             cudaStream_t s) {
+    if (T <= 0) return cudaSuccess;
+    if (bf16)
+        k_quant_act<true><<<static_cast<unsigned>(T), kQuantThreads, 0, s>>>(static_cast<const uint4 *>(X), K, eps,
+                                                                            Xq, amax);
+    else
+        k_quant_act<false><<<static_cast<unsigned>(T), kQuantThreads, 0, s>>>(static_cast<const uint4 *>(X), K,
+                                                                             eps, Xq, amax);
+    return cudaGetLastError();
+}
+
+}  // namespace bitnet

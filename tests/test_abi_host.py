@@ -1,0 +1,142 @@
+"""Host-side checks of the C-ABI library (no GPU needed, no compute calls).
+
+The library must load on a machine without a GPU, export every symbol that
+include/bitnet_sparse.h declares, report its buffer sizes, and reject bad
+arguments on the host before any launch.  Every call below fails validation,
+so none reaches a CUDA call.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from sparse_linear_layers_bitnet_b200 import _abi
+from sparse_linear_layers_bitnet_b200 import build as nvbuild
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "bitnet_sparse.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nvbuild.build()
+    return _abi.load()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = set(re.findall(r"\b(bitnet_[a-z_0-9]+)\s*\(", src))
+    return sorted(names)
+
+
+def test_header_and_binding_agree():
+    assert sorted(_abi.EXPORTED) == declared_functions()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (bitnet_\w+)", out))
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(lib, name)
+
+
+def test_library_links_no_torch_and_no_oracle():
+    out = subprocess.run(["ldd", _abi.LIB_PATH], capture_output=True, text=True).stdout
+    assert "torch" not in out and "oracle" not in out and "libcudart" not in out
+
+
+def test_sizes(lib):
+    assert lib.bitnet_abi_version() == 1
+    # metadata: ceil(k/128) * ceil(n_out/128) blocks of 128 rows x 16 bytes
+    assert lib.bitnet_mma_meta_bytes(256, 256) == 2 * 2 * 2048
+    assert lib.bitnet_mma_meta_bytes(200, 352) == 3 * 2 * 2048
+    assert lib.bitnet_mma_meta_bytes(8640, 3200) == 25 * 68 * 2048
+    # decode layout: 0.25 byte per weight, tiles of 16 x 64
+    assert lib.bitnet_dec_bytes(2560, 6912) == 2560 * 6912 // 4
+    assert lib.bitnet_dec_bytes(200, 256) == 0
+    assert lib.bitnet_pack_workspace_size(3200, 3200) >= 256 + 2048
+    assert lib.bitnet_linear_workspace_size() >= 4
+    assert lib.bitnet_dgrad_workspace_size(3200, 8640) >= 3200 * 8640 * 2
+
+
+def _fake(addr=4096):
+    return ctypes.c_void_p(addr)   # never dereferenced: every call below fails validation
+
+
+def _pw(n_out=256, k=256, n=2, m=4, gamma=True, gb=True, mma=False, dec=False):
+    s = _abi.BitnetPackedW()
+    s.n_out, s.k, s.n, s.m = n_out, k, n, m
+    s.gamma = 4096 if gamma else None
+    s.group_bytes = 8192 if gb else None
+    s.mma_vals = 16384 if mma else None
+    s.mma_meta = 32768 if mma else None
+    s.dec_codes = 65536 if dec else None
+    return s
+
+
+def test_pack_rejects_bad_arguments(lib):
+    st = _pw()
+    ws_n = lib.bitnet_pack_workspace_size(256, 256)
+    assert lib.bitnet_pack_nm(None, ctypes.byref(st), 1e-5, None, _fake(), ws_n, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_pack_nm(_fake(), ctypes.byref(st), 1e-5, None, None, ws_n, None) == _abi.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_pack_nm(_fake(), ctypes.byref(st), 1e-5, None, _fake(), 16, None) == _abi.BITNET_ERR_WORKSPACE
+    bad = _pw(n=6, m=8)
+    assert lib.bitnet_pack_nm(_fake(), ctypes.byref(bad), 1e-5, None, _fake(), ws_n, None) == _abi.BITNET_ERR_UNSUPPORTED
+    bad = _pw(n=3, m=5, gb=False)
+    assert lib.bitnet_pack_nm(_fake(), ctypes.byref(bad), 1e-5, None, _fake(), ws_n, None) == _abi.BITNET_ERR_UNSUPPORTED
+    bad = _pw(k=250)
+    assert lib.bitnet_pack_nm(_fake(), ctypes.byref(bad), 1e-5, None, _fake(), ws_n, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_pack_nm(_fake(4100), ctypes.byref(_pw()), 1e-5, None, _fake(), ws_n, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_pack_nm(_fake(), ctypes.byref(_pw()), -1.0, None, _fake(), ws_n, None) == _abi.BITNET_ERR_INVALID_ARG
+    bad = _pw(gamma=False)
+    assert lib.bitnet_pack_nm(_fake(), ctypes.byref(bad), 1e-5, None, _fake(), ws_n, None) == _abi.BITNET_ERR_INVALID_ARG
+    bad = _pw(gb=False, dec=True)
+    assert lib.bitnet_pack_nm(_fake(), ctypes.byref(bad), 1e-5, None, _fake(), ws_n, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert b"required" in lib.bitnet_last_error() or b"derived" in lib.bitnet_last_error()
+
+
+def test_quant_rejects_bad_arguments(lib):
+    f = lib.bitnet_quant_act
+    assert f(None, 0, 4, 256, 1e-5, _fake(), _fake(), None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(_fake(), 0, 4, 250, 1e-5, _fake(), _fake(), None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(_fake(), 7, 4, 256, 1e-5, _fake(), _fake(), None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(_fake(), 0, 4, 256, 0.0, _fake(), _fake(), None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(_fake(4104), 0, 4, 256, 1e-5, _fake(), _fake(), None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(_fake(), 0, -1, 256, 1e-5, _fake(), _fake(), None) == _abi.BITNET_ERR_INVALID_ARG
+
+
+def test_linear_rejects_bad_arguments(lib):
+    f = lib.bitnet_sparse_linear
+    ws = lib.bitnet_linear_workspace_size()
+    st = _pw(gb=False, mma=False)
+    # T > 8 needs the tensor-core layouts
+    assert f(_fake(), _fake(), ctypes.byref(st), 64, _fake(), 0, None, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    st = _pw(k=272, mma=True)   # k % 32 != 0 on the tensor-core path
+    assert f(_fake(), _fake(), ctypes.byref(st), 64, _fake(), 0, None, _fake(), ws, None) == _abi.BITNET_ERR_UNSUPPORTED
+    st = _pw(mma=True)
+    assert f(_fake(), _fake(), ctypes.byref(st), 64, _fake(), 0, None, None, ws, None) == _abi.BITNET_ERR_WORKSPACE
+    assert f(_fake(), _fake(), ctypes.byref(st), 64, _fake(), 0, None, _fake(), 0, None) == _abi.BITNET_ERR_WORKSPACE
+    assert f(_fake(), _fake(), ctypes.byref(st), 64, _fake(), 9, None, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    st = _pw(n=1, m=4, mma=True)
+    assert f(_fake(), _fake(), ctypes.byref(st), 64, _fake(), 0, None, _fake(), ws, None) == _abi.BITNET_ERR_UNSUPPORTED
+    assert f(None, _fake(), ctypes.byref(_pw()), 4, _fake(), 0, None, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+
+
+def test_dgrad_rejects_bad_arguments(lib):
+    f = lib.bitnet_dgrad
+    ws = lib.bitnet_dgrad_workspace_size(256, 256)
+    st = _pw()
+    assert f(_fake(), _abi.BITNET_F32, ctypes.byref(st), 64, _fake(), 0, _fake(), ws, None) == _abi.BITNET_ERR_UNSUPPORTED
+    assert f(_fake(), _abi.BITNET_BF16, ctypes.byref(st), 64, _fake(), 0, _fake(), 100, None) == _abi.BITNET_ERR_WORKSPACE
+    assert f(_fake(), _abi.BITNET_BF16, ctypes.byref(_pw(gb=False)), 64, _fake(), 0, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(_fake(), _abi.BITNET_BF16, ctypes.byref(_pw(n_out=250)), 64, _fake(), 0, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert lib.bitnet_status_string(s)
+    assert lib.bitnet_read_device_status(None, None) == _abi.BITNET_ERR_INVALID_ARG
