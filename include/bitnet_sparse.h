@@ -162,6 +162,32 @@ bitnet_status bitnet_sparse_linear(const int8_t *Xq, const float *absmax,
                                    void *ws, size_t ws_bytes, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_quant_linear - per-token quantisation fused with the sparse linear.
+ *
+ * Same result as bitnet_quant_act followed by bitnet_sparse_linear (bit for
+ * bit): "BitNet b1.58 ...", section "The mechanism" (per-token symmetric
+ * 8-bit activations; ternary product as signed sums).  For T <= 8 with the
+ * decode layout it is ONE kernel: each CTA starts streaming its packed weights
+ * before waiting on the previous kernel of the stream (programmatic dependent
+ * launch), then forms the token scales from X and quantises in registers.
+ * Otherwise it runs the quantisation into the workspace and the GEMM.
+ *
+ *   X        [T, K] fp32 or bf16 (x_dtype), 16-byte aligned, K == W->k.
+ *   eps      activation eps (> 0).
+ *   W        packed weights (dec_codes for T <= 8; mma layouts for T > 8).
+ *   Y        [T, n_out] of y_dtype.   acc_out  [T, n_out] int32 or NULL.
+ *   xq_out   [T, K] int8 or NULL; absmax_out [T] fp32 or NULL: copies of the
+ *            activation codes and scales (for checking).
+ *   ws       >= bitnet_quant_linear_workspace_size(T, K) bytes.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+size_t bitnet_quant_linear_workspace_size(int64_t T, int64_t K);
+bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps,
+                                  const bitnet_packed_w *W, int64_t T, void *Y, bitnet_dtype y_dtype,
+                                  int32_t *acc_out, int8_t *xq_out, float *absmax_out,
+                                  void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * bitnet_dgrad - straight-through input gradient dX = gamma * dY . Wq.
  *
  * "Sparse-BitNet" (gist.science technical summary), section 2 "Training

@@ -28,6 +28,7 @@ EXPORTED = [
     "bitnet_pack_workspace_size", "bitnet_pack_nm",
     "bitnet_quant_act",
     "bitnet_linear_workspace_size", "bitnet_sparse_linear",
+    "bitnet_quant_linear_workspace_size", "bitnet_quant_linear",
     "bitnet_dgrad_workspace_size", "bitnet_dgrad",
     "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
 ]
@@ -74,6 +75,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_quant_act": (I32, [P, I32, I64, I64, F, P, P, P]),
         "bitnet_linear_workspace_size": (SZ, []),
         "bitnet_sparse_linear": (I32, [P, P, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, SZ, P]),
+        "bitnet_quant_linear_workspace_size": (SZ, [I64, I64]),
+        "bitnet_quant_linear": (I32, [P, I32, F, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, P, P, SZ, P]),
         "bitnet_dgrad_workspace_size": (SZ, [I64, I64]),
         "bitnet_dgrad": (I32, [P, I32, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, SZ, P]),
         "bitnet_read_device_status": (I32, [P, P]),
@@ -203,6 +206,25 @@ def bitnet_sparse_linear(Xq, absmax, W: PackedWeights, Y=None, y_dtype=None, acc
     st = W.struct()
     check(lib.bitnet_sparse_linear(_ptr(Xq), _ptr(absmax), ctypes.byref(st), T, _ptr(Y), _dtype_code(Y.dtype),
                                    _ptr(acc_out), ws.ptr, ws.nbytes, _stream(stream)), "bitnet_sparse_linear")
+    return Y
+
+
+def bitnet_quant_linear(X, W: PackedWeights, eps: float = 1e-5, Y=None, y_dtype=None, acc_out=None, xq_out=None,
+                        absmax_out=None, ws: Workspace | None = None, stream=None):
+    """Fused per-token quantisation + sparse linear (one kernel for decode batches)."""
+    torch = _torch()
+    lib = load()
+    T = X.shape[0]
+    if y_dtype is None:
+        y_dtype = torch.bfloat16
+    if Y is None:
+        Y = torch.empty((T, W.n_out), dtype=y_dtype, device=X.device)
+    if ws is None:
+        ws = Workspace(lib.bitnet_quant_linear_workspace_size(T, W.k), X.device)
+    st = W.struct()
+    check(lib.bitnet_quant_linear(_ptr(X), _dtype_code(X.dtype), ctypes.c_float(eps), ctypes.byref(st), T, _ptr(Y),
+                                  _dtype_code(Y.dtype), _ptr(acc_out), _ptr(xq_out), _ptr(absmax_out), ws.ptr,
+                                  ws.nbytes, _stream(stream)), "bitnet_quant_linear")
     return Y
 
 

@@ -146,6 +146,57 @@ bitnet_status bitnet_sparse_linear(const int8_t *Xq, const float *absmax, const 
                        "sparse_linear (tensor-core GEMM)");
 }
 
+static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+size_t bitnet_quant_linear_workspace_size(int64_t T, int64_t K) {
+    if (T <= 0 || K <= 0) return bitnet::kLinearWsBytes;
+    return bitnet::kLinearWsBytes + align256(static_cast<size_t>(T) * static_cast<size_t>(K)) +
+           align256(static_cast<size_t>(T) * 4);
+}
+
+bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps, const bitnet_packed_w *W,
+                                  int64_t T, void *Y, bitnet_dtype y_dtype, int32_t *acc_out, int8_t *xq_out,
+                                  float *absmax_out, void *ws, size_t ws_bytes, bitnet_stream_t stream) {
+    if (!W || !W->gamma) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: null W or gamma");
+    if (T < 0) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: T < 0");
+    if (T != 0 && (!X || !Y)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: null pointer");
+    if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: bad x dtype");
+    if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: bad y dtype");
+    if (!(eps > 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: eps must be > 0");
+    const int64_t n_out = W->n_out, k = W->k;
+    if (n_out <= 0 || k <= 0 || k % 8) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: bad sizes");
+    if (!(W->n == 2 && W->m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "quant_linear: 2:4 only");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "quant_linear: workspace is required");
+    if (ws_bytes < bitnet_quant_linear_workspace_size(T, k))
+        return fail(BITNET_ERR_WORKSPACE, "quant_linear: workspace needs %zu bytes", bitnet_quant_linear_workspace_size(T, k));
+    if (T == 0) return BITNET_OK;   // an empty batch needs no buffers
+    if (!aligned(X, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: X and ws must be 16-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool xb = x_dtype == BITNET_BF16, yb = y_dtype == BITNET_BF16;
+    if (T <= 8 && W->dec_codes && n_out % 16 == 0 && k % 64 == 0) {
+        if (!aligned(W->dec_codes, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: dec_codes alignment");
+        return cuda_status(bitnet::launch_gemv_fused(X, xb, eps, W->gamma, W->dec_codes, T, n_out, k, Y, yb, acc_out,
+                                                     xq_out, absmax_out, s),
+                           "quant_linear (fused decode GEMV)");
+    }
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    int8_t *xq = reinterpret_cast<int8_t *>(w8 + bitnet::kLinearWsBytes);
+    float *am = reinterpret_cast<float *>(w8 + bitnet::kLinearWsBytes + align256(static_cast<size_t>(T) * k));
+    bitnet_status st = bitnet_quant_act(X, x_dtype, T, k, eps, xq, am, stream);
+    if (st != BITNET_OK) return st;
+    st = bitnet_sparse_linear(xq, am, W, T, Y, y_dtype, acc_out, ws, ws_bytes, stream);
+    if (st != BITNET_OK) return st;
+    if (xq_out) {
+        cudaError_t e = cudaMemcpyAsync(xq_out, xq, static_cast<size_t>(T) * k, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_status(e, "quant_linear copy");
+    }
+    if (absmax_out) {
+        cudaError_t e = cudaMemcpyAsync(absmax_out, am, static_cast<size_t>(T) * 4, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_status(e, "quant_linear copy");
+    }
+    return BITNET_OK;
+}
+
 bitnet_status bitnet_dgrad(const void *dY, bitnet_dtype dy_dtype, const bitnet_packed_w *W, int64_t T, void *dX,
                            bitnet_dtype dx_dtype, void *ws, size_t ws_bytes, bitnet_stream_t stream) {
     if (!W || !W->gamma) return fail(BITNET_ERR_INVALID_ARG, "dgrad: null W or gamma");

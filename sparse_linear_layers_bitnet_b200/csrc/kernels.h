@@ -33,6 +33,10 @@ cudaError_t launch_gemv_dec(const int8_t *Xq, const float *amax, const float *ga
                             int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                             cudaStream_t s);
 
+cudaError_t launch_gemv_fused(const void *X, bool x_bf16, float eps, const float *gamma, const uint8_t *dec,
+                              int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
+                              int8_t *xq_out, float *amax_out, cudaStream_t s);
+
 cudaError_t launch_gemv_gb(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *gb,
                            int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                            cudaStream_t s);

@@ -314,3 +314,75 @@ def test_device_status_clear_after_runs(bn):
     ws = bn.Workspace(256)
     ref, acc, Y = _linear_case(bn, 256, 256, 64, seed=5)
     assert bn.bitnet_read_device_status(ws) == 0
+
+
+# ------------------------------------------------------------------ fused quantisation + linear
+
+@pytest.mark.parametrize("T,x_dtype", [(1, "bf16"), (3, "bf16"), (8, "bf16"), (2, "f32"), (8, "f32")])
+@pytest.mark.parametrize("n_out,k", [(3840, 2560), (2560, 6912), (208, 320)])
+def test_quant_linear_fused_decode(bn, T, x_dtype, n_out, k):
+    W = synth.master_weights(n_out, k, 0.02, seed=400 + T)
+    X = synth.activations(T, k, seed=401 + T, outlier_p=0.01)
+    if x_dtype == "bf16":
+        Xd, X32 = bf16_dev(X)
+    else:
+        Xd, X32 = dev_f32(X), X
+    ref = oracle.forward(W, X32, 1e-5, 1e-5)
+    pw = bn.PackedWeights(n_out, k, mma=False)
+    bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5)
+    acc = torch.full((T, n_out), -7, dtype=torch.int32, device="cuda")
+    xq = torch.zeros((T, k), dtype=torch.int8, device="cuda")
+    am = torch.zeros((T,), dtype=torch.float32, device="cuda")
+    Y = bn.bitnet_quant_linear(Xd, pw, 1e-5, y_dtype=torch.float32, acc_out=acc, xq_out=xq, absmax_out=am)
+    torch.cuda.synchronize()
+    assert np.array_equal(xq.cpu().numpy(), ref["xq"])
+    assert np.array_equal(am.cpu().numpy(), ref["a"])
+    _check_outputs(ref, acc.cpu().numpy(), Y)
+
+
+@pytest.mark.parametrize("T", [16, 100])
+def test_quant_linear_unfused_path(bn, T):
+    n_out, k = 384, 1024
+    W = synth.master_weights(n_out, k, 0.02, seed=500 + T)
+    Xd, X32 = bf16_dev(synth.activations(T, k, seed=501 + T))
+    ref = oracle.forward(W, X32, 1e-5, 1e-5)
+    pw = bn.PackedWeights(n_out, k)
+    bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5)
+    acc = torch.empty((T, n_out), dtype=torch.int32, device="cuda")
+    Y = bn.bitnet_quant_linear(Xd, pw, 1e-5, y_dtype=torch.bfloat16, acc_out=acc)
+    torch.cuda.synchronize()
+    _check_outputs(ref, acc.cpu().numpy(), Y)
+
+
+def test_quant_linear_chain_in_graph(bn):
+    """Consecutive fused kernels (programmatic dependent launch) inside a CUDA
+    graph: each layer consumes the previous layer's output."""
+    T, h = 2, 512
+    layers = 6
+    Ws = [synth.master_weights(h, h, 0.02, seed=600 + l) for l in range(layers)]
+    pws = []
+    for W in Ws:
+        pw = bn.PackedWeights(h, h, mma=False)
+        bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5)
+        pws.append(pw)
+    x0 = synth.activations(T, h, seed=700)
+    xs = [dev_f32(x0)] + [torch.empty((T, h), dtype=torch.float32, device="cuda") for _ in range(layers)]
+    ws = bn.Workspace(bn.load().bitnet_quant_linear_workspace_size(T, h))
+
+    def run():
+        for l in range(layers):
+            bn.bitnet_quant_linear(xs[l], pws[l], 1e-5, Y=xs[l + 1], ws=ws)
+
+    run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    for x in xs[1:]:
+        x.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    x = x0
+    for l in range(layers):
+        x = oracle.forward(Ws[l], x, 1e-5, 1e-5)["y"]
+        assert np.array_equal(xs[l + 1].cpu().numpy(), x), l
