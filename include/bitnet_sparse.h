@@ -210,6 +210,33 @@ bitnet_status bitnet_dgrad(const void *dY, bitnet_dtype dy_dtype, const bitnet_p
                            void *ws, size_t ws_bytes, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_pack_nm_noalloc - bitnet_pack_nm for callers that cannot allocate.
+ *
+ * No counterpart in the paper: this is a library convenience.  Some callers
+ * cannot allocate device memory where they pack (an optimizer step inside a
+ * fixed memory pool, an embedded runtime whose allocator the call site cannot
+ * reach, a latency-critical path that must not call cudaMalloc).  This entry
+ * point needs no workspace: the pack's scratch lives in a fixed device array of
+ * bitnet_pack_workspace_size() bytes (2304) inside the library, present on every
+ * GPU that loads the library until the process exits.  Everything else is as
+ * in bitnet_pack_nm, with bit-identical results.
+ *
+ *   Limit: n_out * k <= 2^40 weights (the exactness bound of the fixed
+ *          scratch's 64-bit exponent bins); larger matrices are rejected with
+ *          BITNET_ERR_UNSUPPORTED.
+ *   First call on a device looks up the array's device address with
+ *          cudaGetSymbolAddress (once per device, with that device current);
+ *          make that first call before any stream capture.
+ *   Sharing: every call reuses the same array and clears it first; calls whose
+ *          kernels overlap on the GPU (other streams, other host threads on the
+ *          same device) race on it - serialise them on one stream.
+ *   Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * Errors: as bitnet_pack_nm (no WORKSPACE error), plus UNSUPPORTED above the limit.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_pack_nm_noalloc(const float *W, bitnet_packed_w *out, float eps,
+                                     uint8_t *mask_bits, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Status helpers.
  * bitnet_read_device_status synchronises `stream`, reads the status word that
  * the kernels of the last call on `ws` left (BITNET_OK or BITNET_ERR_TIMEOUT

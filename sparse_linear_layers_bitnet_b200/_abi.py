@@ -25,7 +25,7 @@ BITNET_BF16 = 1
 # Every symbol include/bitnet_sparse.h declares.
 EXPORTED = [
     "bitnet_mma_meta_bytes", "bitnet_dec_bytes",
-    "bitnet_pack_workspace_size", "bitnet_pack_nm",
+    "bitnet_pack_workspace_size", "bitnet_pack_nm", "bitnet_pack_nm_noalloc",
     "bitnet_quant_act",
     "bitnet_linear_workspace_size", "bitnet_sparse_linear",
     "bitnet_quant_linear_workspace_size", "bitnet_quant_linear",
@@ -72,6 +72,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_dec_bytes": (SZ, [I64, I64]),
         "bitnet_pack_workspace_size": (SZ, [I64, I64]),
         "bitnet_pack_nm": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P, SZ, P]),
+        "bitnet_pack_nm_noalloc": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P]),
         "bitnet_quant_act": (I32, [P, I32, I64, I64, F, P, P, P]),
         "bitnet_linear_workspace_size": (SZ, []),
         "bitnet_sparse_linear": (I32, [P, P, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, SZ, P]),

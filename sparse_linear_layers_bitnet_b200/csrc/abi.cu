@@ -30,6 +30,10 @@ int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 }  // namespace
 
+namespace bitnet {
+void set_last_error(const char *msg) { snprintf(g_err, sizeof g_err, "%s", msg); }
+}  // namespace bitnet
+
 extern "C" {
 
 int bitnet_abi_version(void) { return 1; }

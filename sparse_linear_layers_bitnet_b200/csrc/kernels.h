@@ -22,6 +22,9 @@ constexpr size_t kDgradWsHeader = 256;
 
 int num_sms();
 
+// Sets the message bitnet_last_error() returns on this thread.
+void set_last_error(const char *msg);
+
 cudaError_t launch_pack(const float *W, int64_t n_out, int64_t k, int n, int m, float eps, float *gamma,
                         uint8_t *gb, int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws,
                         cudaStream_t s);
