@@ -57,6 +57,10 @@ def parse_args():
     ap.add_argument("--layers", type=int, default=30)
     ap.add_argument("--no-rows", action="store_true", help="skip the sub-measurements of the other rows")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
+    ap.add_argument("--pack-layers", type=int, default=None, help="layers of the pack workload (default: all 26)")
+    ap.add_argument("--flip-steps", type=int, default=100, help="random-walk steps of the mask flip-rate study")
+    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks"], default=None,
+                    help="run one sub-measurement alone and print it (for profiling)")
     return ap.parse_args()
 
 
@@ -194,9 +198,15 @@ def decode_bytes(T, K, N):
     return quant, gemv
 
 
+def decode_bytes_fused(T, K, N):
+    """Algorithmic bytes of one fused projection: bf16 activations in, packed
+    weights (0.25 B each), gamma, bf16 outputs."""
+    return 2 * T * K + N * K // 4 + 4 + 2 * T * N
+
+
 class Decode:
-    def __init__(self, torch, bn, synth, T, layers, seed_base=0):
-        self.torch, self.bn, self.T, self.L = torch, bn, T, layers
+    def __init__(self, torch, bn, synth, T, layers, seed_base=0, fused=True):
+        self.torch, self.bn, self.T, self.L, self.fused = torch, bn, T, layers, fused
         dev = torch.device("cuda", torch.cuda.current_device())
         self.mats = decode_shapes()
         self.packed = []
@@ -231,24 +241,31 @@ class Decode:
             self.y_views.append(ry)
         self.xq = [torch.empty((T, K), dtype=torch.int8, device=dev) for _, K, _ in self.mats]
         self.amax = [torch.empty((T,), dtype=torch.float32, device=dev) for _ in self.mats]
-        self.ws = bn.Workspace(bn.load().bitnet_linear_workspace_size(), dev)
+        self.ws = bn.Workspace(max(bn.load().bitnet_linear_workspace_size(),
+                                   max(bn.load().bitnet_quant_linear_workspace_size(T, K) for _, K, _ in self.mats)),
+                               dev)
         q, g = 0, 0
         for _, K, N in self.mats:
             a, b = decode_bytes(T, K, N)
             q += a
             g += b
         self.quant_bytes_per_layer, self.gemv_bytes_per_layer = q, g
-        self.step_bytes = (q + g) * layers
+        self.fused_bytes_per_layer = sum(decode_bytes_fused(T, K, N) for _, K, N in self.mats)
+        self.step_bytes = (self.fused_bytes_per_layer if fused else q + g) * layers
         self.weight_bytes = sum(N * K // 4 for _, K, N in self.mats) * layers
-        self.launches_per_step = 2 * len(self.mats) * layers
+        self.launches_per_step = (1 if fused else 2) * len(self.mats) * layers
 
     def step(self):
         bn = self.bn
         for l in range(self.L):
             for j in range(len(self.mats)):
-                bn.bitnet_quant_act(self.x_views[l][j], 1e-5, Xq=self.xq[j], absmax=self.amax[j])
-                bn.bitnet_sparse_linear(self.xq[j], self.amax[j], self.packed[l][j], Y=self.y_views[l][j],
-                                        ws=self.ws)
+                if self.fused:
+                    bn.bitnet_quant_linear(self.x_views[l][j], self.packed[l][j], 1e-5, Y=self.y_views[l][j],
+                                           ws=self.ws)
+                else:
+                    bn.bitnet_quant_act(self.x_views[l][j], 1e-5, Xq=self.xq[j], absmax=self.amax[j])
+                    bn.bitnet_sparse_linear(self.xq[j], self.amax[j], self.packed[l][j], Y=self.y_views[l][j],
+                                            ws=self.ws)
 
     def gemv_only(self):
         bn = self.bn
@@ -318,22 +335,55 @@ def measure_prefill(torch, bn, synth, peaks, reps=10):
     return out
 
 
+def measure_library_peaks(torch, n=8192, reps=10):
+    """Dense int8 (cuBLASLt via torch._int_mm) and bf16 (cuBLAS) GEMM throughput
+    on this GPU, run only: the measured denominators for the tensor-core rows
+    (MEASURED_PEAKS.json carries no int8 figure)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    out = {}
+    a8 = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+    b8 = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev).t()   # column-major operand
+    for _ in range(3):
+        torch._int_mm(a8, b8)
+    ts = []
+    for _ in range(reps):
+        with Timer(torch) as t:
+            torch._int_mm(a8, b8)
+        ts.append(t.ms())
+    out["int8_dense_tops"] = round(2.0 * n ** 3 / min(ts) / 1e9, 1)
+    del a8, b8
+    a = torch.randn((n, n), dtype=torch.bfloat16, device=dev)
+    b = torch.randn((n, n), dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        a @ b
+    ts = []
+    for _ in range(reps):
+        with Timer(torch) as t:
+            a @ b
+        ts.append(t.ms())
+    out["bf16_dense_tflops"] = round(2.0 * n ** 3 / min(ts) / 1e9, 1)
+    out["how"] = f"{n}^3, best of {reps}, CUDA events; int8: torch._int_mm (cuBLASLt), bf16: torch.matmul"
+    del a, b
+    torch.cuda.empty_cache()
+    return out
+
+
 def popcount_u8(torch, x):
     lut = torch.tensor([bin(i).count("1") for i in range(256)], dtype=torch.int64, device=x.device)
     return lut[x.long()].sum().item()
 
 
-def measure_pack(torch, bn, synth, peaks, steps=3, flip_steps=100):
+def measure_pack(torch, bn, synth, peaks, steps=3, flip_steps=100, layers=None):
     """Per-step pack over every linear weight of a 3B LLaMA-alike (26 layers)."""
     dev = torch.device("cuda", torch.cuda.current_device())
-    layers = synth.LLAMA_3B["layers"]
+    layers = layers or synth.LLAMA_3B["layers"]
     mats = synth.LAYER_3B_MATRICES
     Ws, pws = [], []
     for l in range(layers):
         for j, (name, N, K) in enumerate(mats):
             Ws.append(synth.torch_master_weights(N, K, 0.02, seed=50000 + 10 * l + j, device=dev))
             pws.append(bn.PackedWeights(N, K, dev, group_bytes=True, mma=True, dec=False))
-    ws = bn.Workspace(bn.load().bitnet_pack_workspace_size(1, 1), dev)
+    ws = bn.Workspace(max(bn.load().bitnet_pack_update_workspace_size(N, K) for _, N, K in mats), dev)
     n_w = sum(N * K for _, N, K in mats) * layers
     alg_bytes = n_w * (4 + 0.25 + 0.5 + 0.125)   # read fp32, write group bytes, int8 values, metadata
     for W, pw in zip(Ws, pws):
@@ -345,13 +395,18 @@ def measure_pack(torch, bn, synth, peaks, steps=3, flip_steps=100):
             synth.torch_random_walk_(W, 1e-4, seed=s * 1000 + i)
         with Timer(torch) as t:
             for W, pw in zip(Ws, pws):
-                bn.bitnet_pack_nm(W, pw, 1e-5, ws=ws)
+                bn.bitnet_pack_nm_update(W, pw, 1e-5, ws=ws)
         ms.append(t.ms())
     step_ms = statistics.mean(ms)
     gbs = alg_bytes / step_ms / 1e6
     out = {"weights": n_w, "step_ms": round(step_ms, 3), "gbs": round(gbs, 1),
            "frac_of_hbm": round(gbs / peaks["hbm"], 4),
-           "alg_bytes_per_weight": 4.875, "launches_per_matrix": 4}
+           "alg_bytes_per_weight": 4.875, "launches_per_matrix": 3,
+           "entry": "bitnet_pack_nm_update (previous step's gamma as hint; bit-identical to bitnet_pack_nm)"}
+    if flip_steps <= 0:
+        del Ws, pws
+        torch.cuda.empty_cache()
+        return out
     # mask flip rate over 100 random-walk steps of one layer
     del Ws[len(mats):]
     del pws
@@ -482,12 +537,28 @@ def run_reference(args):
 
 # ------------------------------------------------------------------ main arm
 
+def run_only(args):
+    import torch
+
+    import sparse_linear_layers_bitnet_b200 as bn
+    from sparse_linear_layers_bitnet_b200 import synth
+    bn.load()
+    peaks = load_peaks()
+    fn = {"prefill": measure_prefill, "pack": measure_pack, "dgrad": measure_dgrad,
+          "peaks": lambda torch, bn, synth, peaks: measure_library_peaks(torch)}[args.only]
+    kw = {"steps": args.steps, "flip_steps": args.flip_steps, "layers": args.pack_layers} if args.only == "pack" else {}
+    print(json.dumps({args.only: fn(torch, bn, synth, peaks, **kw)}), flush=True)
+    return 0
+
+
 def run_ours(args):
     import torch
 
     import sparse_linear_layers_bitnet_b200 as bn
     from sparse_linear_layers_bitnet_b200 import dist, synth
 
+    if args.only:
+        return run_only(args)
     info = dist.init()
     torch.cuda.set_device(info.local_rank)
     bn.load()
@@ -496,9 +567,8 @@ def run_ours(args):
     assert 1 <= T <= 8, "decode batch must be 1..8"
     dev_index = torch.cuda.current_device()
 
-    dec = Decode(torch, bn, synth, T, args.layers, seed_base=info.rank * 7919)
+    dec = Decode(torch, bn, synth, T, args.layers, seed_base=info.rank * 7919, fused=False)
     g_step = dec.capture(dec.step)
-    g_gemv = dec.capture(dec.gemv_only)
 
     clocks = ClockSampler(dev_index).start()
     # pre-roll so that clocks settle (untimed, counted as warm-up)
@@ -520,17 +590,20 @@ def run_ours(args):
     ms_total = dist.max_over_ranks(ms_total, device=torch.device("cuda", dev_index))
     value = dec.step_bytes * args.steps * info.world / (ms_total / 1e3) / 1e9
 
-    # dominant kernel: the GEMV alone, same stream, same graph mechanism
+    # dominant kernel: the GEMV alone, replayed from a graph of the same 120
+    # launches on the same stream
+    g_gemv = dec.capture(dec.gemv_only)
     for _ in range(3):
         g_gemv.replay()
+    reps = max(args.steps, 10)
     with Timer(torch) as tk:
-        reps = max(args.steps, 10)
         for _ in range(reps):
             g_gemv.replay()
     gemv_ms_per_launch = tk.ms() / reps / (len(dec.mats) * dec.L)
     gemv_bytes_per_launch = dec.gemv_bytes_per_layer / len(dec.mats)
     achieved = gemv_bytes_per_launch / (gemv_ms_per_launch / 1e3) / 1e9
     traffic = ncu_traffic("k_gemv_dec", ["gemv.cu"])
+    del g_gemv
 
     # end to end: activations from pinned host memory, outputs back to host
     x_host = torch.empty(dec.x_flat.shape, dtype=dec.x_flat.dtype, pin_memory=True)
@@ -553,24 +626,29 @@ def run_ours(args):
 
     rows = {}
     if not args.no_rows and info.world == 1:
-        rows["decode_gemv_batches"] = {}
-        for t2 in (4, 8):
-            d2 = Decode(torch, bn, synth, t2, args.layers, seed_base=31)
-            g2 = d2.capture(d2.gemv_only)
+        rows["decode_batches"] = {}
+        for t2, fused in ((1, True), (4, False), (4, True), (8, False), (8, True)):
+            d2 = Decode(torch, bn, synth, t2, args.layers, seed_base=31, fused=fused)
+            g2 = d2.capture(d2.step)
             for _ in range(3):
                 g2.replay()
             with Timer(torch) as t:
                 for _ in range(10):
                     g2.replay()
             per = t.ms() / 10
-            rows["decode_gemv_batches"][f"T{t2}"] = {
-                "gemv_gbs": round(d2.gemv_bytes_per_layer * d2.L / (per / 1e3) / 1e9, 1),
-                "ms_per_pass": round(per, 4)}
+            rows["decode_batches"][f"T{t2}_{'fused' if fused else 'quant+gemv'}"] = {
+                "gbs": round(d2.step_bytes / (per / 1e3) / 1e9, 1), "ms_per_step": round(per, 4),
+                "launches_per_step": d2.launches_per_step}
             del g2, d2
             torch.cuda.empty_cache()
+        rows["library_peaks"] = measure_library_peaks(torch)
         rows["prefill_gemm"] = measure_prefill(torch, bn, synth, peaks)
+        lp = rows["library_peaks"]["int8_dense_tops"]
+        pc = rows["prefill_gemm"]["combined"]
+        pc["frac_of_2x_measured_int8_dense"] = round(pc["tops"] / (2 * lp), 4)
+        pc["frac_of_measured_int8_dense"] = round(pc["tops"] / lp, 4)
         rows["dgrad"] = measure_dgrad(torch, bn, synth, peaks)
-        rows["pack"] = measure_pack(torch, bn, synth, peaks)
+        rows["pack"] = measure_pack(torch, bn, synth, peaks, flip_steps=args.flip_steps)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": info.world, "steps": args.steps,
@@ -579,7 +657,8 @@ def run_ours(args):
         "config": {"workload": f"decode GEMV, 2B LLaMA-alike (hidden 2560, FFN 6912), {args.layers} layers, batch {T}",
                    "tokens": T, "layers": args.layers,
                    "projections": [f"{n} {K}->{N}" for n, K, N in dec.mats],
-                   "step": "per layer and projection: int8 act quant + sparse ternary GEMV (CUDA graph)",
+                   "step": "per layer and projection: int8 act quant (bitnet_quant_act) + sparse ternary GEMV "
+                           "(bitnet_sparse_linear), programmatic dependent launch, CUDA graph",
                    "l2": f"inputs larger than L2: {dec.weight_bytes / 1e6:.0f} MB of packed weights per step",
                    "parallelism": f"replicas x{info.world} (independent layers, no collective)"},
         "roofline": {"bound": "hbm", "kernel": "k_gemv_dec", "achieved": round(achieved, 1),
@@ -601,7 +680,7 @@ def run_ours(args):
         line["rows"] = rows
     if info.rank == 0:
         print(json.dumps(line), flush=True)
-    del g_step, g_gemv
+    del g_step
     dist.finalize()
     return 0
 

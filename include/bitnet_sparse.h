@@ -120,6 +120,30 @@ bitnet_status bitnet_pack_nm(const float *W, bitnet_packed_w *out, float eps,
                              bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_pack_nm_update - the per-step pack of a matrix that was packed before.
+ *
+ * "Sparse-BitNet" (gist.science), section 2 "Training Strategie": the mask
+ * and codes are recomputed every step from masters that move by one optimizer
+ * step.  Results are bit-identical to bitnet_pack_nm (2:4 only).  On entry
+ * out->gamma must hold the gamma of this matrix's previous pack (as written
+ * by bitnet_pack_nm / _update), or 0 when there is none.  With that hint the
+ * call reads W ONCE: it sums |W| exactly and writes every layout with the
+ * hint's threshold, listing the kept weights within a relative 2^-10 of that
+ * threshold; if the new threshold falls inside that band only the listed
+ * groups are rewritten, otherwise (or without a hint, or when the list is
+ * full) a second full pass runs.  The choice is made on the device.
+ *
+ *   W, out, eps, mask_bits  as in bitnet_pack_nm (n = 2, m = 4).
+ *   ws   >= bitnet_pack_update_workspace_size(n_out, k) bytes: the pack
+ *        scratch plus the list of near-threshold groups.
+ * Errors: as bitnet_pack_nm.
+ * ------------------------------------------------------------------------ */
+size_t bitnet_pack_update_workspace_size(int64_t n_out, int64_t k);
+bitnet_status bitnet_pack_nm_update(const float *W, bitnet_packed_w *out, float eps,
+                                    uint8_t *mask_bits, void *ws, size_t ws_bytes,
+                                    bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * bitnet_quant_act - per-token absmax int8 activation quantisation.
  *
  * "BitNet b1.58: Ternary Weights for 1.58-bit LLMs", section "The mechanism"

@@ -6,11 +6,11 @@ seeded synthetic input generators.
 """
 from ._abi import (  # noqa: F401
     BITNET_BF16, BITNET_F32, BitnetError, BitnetPackedW, PackedWeights, Workspace,
-    bitnet_dgrad, bitnet_pack_nm, bitnet_quant_act, bitnet_quant_linear, bitnet_read_device_status, bitnet_sparse_linear, load,
+    bitnet_dgrad, bitnet_pack_nm, bitnet_pack_nm_update, bitnet_quant_act, bitnet_quant_linear, bitnet_read_device_status, bitnet_sparse_linear, load,
 )
 
 __all__ = [
     "PackedWeights", "Workspace", "BitnetError", "BitnetPackedW", "load",
-    "bitnet_pack_nm", "bitnet_quant_act", "bitnet_quant_linear", "bitnet_sparse_linear", "bitnet_dgrad", "bitnet_read_device_status",
+    "bitnet_pack_nm", "bitnet_pack_nm_update", "bitnet_quant_act", "bitnet_quant_linear", "bitnet_sparse_linear", "bitnet_dgrad", "bitnet_read_device_status",
     "BITNET_F32", "BITNET_BF16",
 ]

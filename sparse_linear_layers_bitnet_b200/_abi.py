@@ -26,6 +26,7 @@ BITNET_BF16 = 1
 EXPORTED = [
     "bitnet_mma_meta_bytes", "bitnet_dec_bytes",
     "bitnet_pack_workspace_size", "bitnet_pack_nm", "bitnet_pack_nm_noalloc",
+    "bitnet_pack_update_workspace_size", "bitnet_pack_nm_update",
     "bitnet_quant_act",
     "bitnet_linear_workspace_size", "bitnet_sparse_linear",
     "bitnet_quant_linear_workspace_size", "bitnet_quant_linear",
@@ -73,6 +74,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_pack_workspace_size": (SZ, [I64, I64]),
         "bitnet_pack_nm": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P, SZ, P]),
         "bitnet_pack_nm_noalloc": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P]),
+        "bitnet_pack_update_workspace_size": (SZ, [I64, I64]),
+        "bitnet_pack_nm_update": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P, SZ, P]),
         "bitnet_quant_act": (I32, [P, I32, I64, I64, F, P, P, P]),
         "bitnet_linear_workspace_size": (SZ, []),
         "bitnet_sparse_linear": (I32, [P, P, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, SZ, P]),
@@ -176,6 +179,19 @@ def bitnet_pack_nm(W, out: PackedWeights, eps: float = 1e-5, mask_bits=None, ws:
     st = out.struct()
     check(lib.bitnet_pack_nm(_ptr(W), ctypes.byref(st), ctypes.c_float(eps), _ptr(mask_bits), ws.ptr,
                              ws.nbytes, _stream(stream)), "bitnet_pack_nm")
+    return out
+
+
+def bitnet_pack_nm_update(W, out: PackedWeights, eps: float = 1e-5, mask_bits=None, ws: Workspace | None = None,
+                          stream=None):
+    """Per-step pack reusing out.gamma (the previous gamma of this matrix) as a hint."""
+    lib = load()
+    assert W.dtype == _torch().float32 and W.is_contiguous()
+    if ws is None:
+        ws = Workspace(lib.bitnet_pack_update_workspace_size(out.n_out, out.k), W.device)
+    st = out.struct()
+    check(lib.bitnet_pack_nm_update(_ptr(W), ctypes.byref(st), ctypes.c_float(eps), _ptr(mask_bits), ws.ptr,
+                                    ws.nbytes, _stream(stream)), "bitnet_pack_nm_update")
     return out
 
 

@@ -81,6 +81,8 @@ bitnet_status bitnet_pack_nm(const float *W, bitnet_packed_w *out, float eps, ui
     if (k % 8 != 0) return fail(BITNET_ERR_INVALID_ARG, "pack: k must be a multiple of 8");
     if (!(eps >= 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "pack: eps must be >= 0");
     if (!aligned(W, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "pack: W and ws must be 16-byte aligned");
+    if (static_cast<double>(n_out) * static_cast<double>(k) / 4.0 > 4294967295.0)
+        return fail(BITNET_ERR_UNSUPPORTED, "pack: more than 2^32 groups of 4 in one matrix");
     const bool packed = out->group_bytes || out->mma_vals || out->mma_meta || out->dec_codes;
     if (packed && !(n == 2 && m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "pack: packed layouts exist for 2:4 only");
     if ((out->mma_vals == nullptr) != (out->mma_meta == nullptr))
@@ -96,6 +98,38 @@ bitnet_status bitnet_pack_nm(const float *W, bitnet_packed_w *out, float eps, ui
     return cuda_status(bitnet::launch_pack(W, n_out, k, n, m, eps, out->gamma, out->group_bytes, out->mma_vals,
                                            out->mma_meta, out->dec_codes, mask_bits, ws, s),
                        "pack");
+}
+
+size_t bitnet_pack_update_workspace_size(int64_t n_out, int64_t k) {
+    if (n_out <= 0 || k <= 0) return bitnet::kPackWsBytes;
+    // list room for 1/256 of the groups (Gaussian masters put ~0.06% of the
+    // weights within 2^-10 of the threshold), at least 16384 entries
+    const size_t groups = static_cast<size_t>(n_out) * static_cast<size_t>(k) / 4;
+    size_t cap = groups / 256;
+    if (cap < 16384) cap = 16384;
+    return bitnet::kPackWsBytes + cap * 4;
+}
+
+bitnet_status bitnet_pack_nm_update(const float *W, bitnet_packed_w *out, float eps, uint8_t *mask_bits, void *ws,
+                                    size_t ws_bytes, bitnet_stream_t stream) {
+    if (!W || !out || !out->gamma) return fail(BITNET_ERR_INVALID_ARG, "pack_update: W, out and out->gamma are required");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "pack_update: workspace is required");
+    const int64_t n_out = out->n_out, k = out->k;
+    if (n_out <= 0 || k <= 0 || k % 8) return fail(BITNET_ERR_INVALID_ARG, "pack_update: bad sizes (k %% 8 == 0)");
+    if (!(out->n == 2 && out->m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "pack_update: 2:4 only");
+    if (ws_bytes < bitnet::kPackWsBytes + 4) return fail(BITNET_ERR_WORKSPACE, "pack_update: workspace needs >= %zu bytes", bitnet::kPackWsBytes + 4);
+    if (!(eps >= 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "pack_update: eps must be >= 0");
+    if (!aligned(W, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "pack_update: W and ws must be 16-byte aligned");
+    if ((out->mma_vals == nullptr) != (out->mma_meta == nullptr))
+        return fail(BITNET_ERR_INVALID_ARG, "pack_update: mma_vals and mma_meta go together");
+    if (out->dec_codes && (!out->group_bytes || n_out % 16 || k % 64))
+        return fail(BITNET_ERR_INVALID_ARG, "pack_update: dec_codes need group_bytes, n_out %% 16 == 0, k %% 64 == 0");
+    if (static_cast<double>(n_out) * static_cast<double>(k) / 4.0 > 4294967295.0)
+        return fail(BITNET_ERR_UNSUPPORTED, "pack_update: more than 2^32 groups");
+    return cuda_status(bitnet::launch_pack_update(W, n_out, k, eps, out->gamma, out->group_bytes, out->mma_vals,
+                                                  out->mma_meta, out->dec_codes, mask_bits, ws, ws_bytes,
+                                                  reinterpret_cast<cudaStream_t>(stream)),
+                       "pack_update");
 }
 
 bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, int64_t K, float eps, int8_t *Xq,
@@ -177,7 +211,8 @@ bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps
     if (!aligned(X, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: X and ws must be 16-byte aligned");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool xb = x_dtype == BITNET_BF16, yb = y_dtype == BITNET_BF16;
-    if (T <= 8 && W->dec_codes && n_out % 16 == 0 && k % 64 == 0) {
+    if (T <= 8 && W->dec_codes && n_out % 16 == 0 && k % 64 == 0 &&
+        static_cast<size_t>(T) * static_cast<size_t>(k + 16) <= bitnet::kFusedMaxSmem) {
         if (!aligned(W->dec_codes, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: dec_codes alignment");
         return cuda_status(bitnet::launch_gemv_fused(X, xb, eps, W->gamma, W->dec_codes, T, n_out, k, Y, yb, acc_out,
                                                      xq_out, absmax_out, s),

@@ -329,6 +329,8 @@ cudaError_t launch_gemm_sp(const int8_t *Xq, const float *amax, const float *gam
     p.out_bf16 = y_bf16 ? 1 : 0;
     p.acc_out = acc;
     p.status = status;
+    if (T > 128)   // CTA-pair persistent kernel (gemm2.cu)
+        return launch_gemm_sp_pair(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
     const int bn = T <= 32 ? 32 : (T <= 128 ? 128 : 256);
     CUtensorMap ma, mb;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, vals, static_cast<uint64_t>(k / 2),
@@ -377,6 +379,9 @@ cudaError_t launch_dgrad(const void *dY, const float *gamma, const uint8_t *gb, 
     k_expand_wt<<<eg, 256, 0, s>>>(gb, n_out, k, wt);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    if (T > 128)   // CTA-pair persistent kernel (gemm2.cu)
+        return launch_gemm_bf16_pair(dY, wt, gamma, T, n_out, k, dX, dx_bf16,
+                                     reinterpret_cast<uint32_t *>(w8 + kStatusOffset), s);
     GemmParams p{};
     p.M = T;
     p.N = k;

@@ -1,0 +1,469 @@
+// Persistent CTA-pair tensor-core GEMM (tcgen05 .cta_group::2, sm_100a).
+//
+// Same products as gemm.cu: the 2:4-sparse int8 x ternary forward
+// ("BitNet b1.58: Ternary Weights for 1.58-bit LLMs", section "The mechanism";
+// "Sparse-BitNet" (gist.science), section 2) and the dense bf16 STE input
+// gradient ("Sparse-BitNet", section 2 "Training Strategie").  Results are
+// identical to gemm.cu (integer accumulation is exact; the fp32 epilogue does
+// the same operations in the same order).
+//
+// A cluster of two CTAs on two SMs computes one 256 x BN output tile with one
+// MMA instruction stream: each CTA holds 128 rows of A and BN/2 rows of B in
+// its own shared memory, and the pair's TMEM holds the 256 x BN accumulator
+// (128 lanes per CTA).  Per SM this halves the B bytes per MMA compared with a
+// 128 x BN single-CTA tile.  The CTA pair is persistent: it walks tiles
+// pair_id, pair_id + pairs, ...; two TMEM accumulator buffers let the
+// epilogue of one tile overlap the main loop of the next.
+//   warp 0     TMA producer in both CTAs (2-SM TMA: completion counted on the
+//              leader CTA's barrier), STAGES-deep ring;
+//   warp 1     TMEM allocation in both CTAs; the leader's lane 0 copies the
+//              2:4 metadata into TMEM and issues the MMAs; commits release the
+//              ring stage and publish an accumulator in both CTAs;
+//   warps 2-5  epilogue in both CTAs: TMEM -> registers -> scaled stores, then
+//              release of the accumulator buffer to the leader.
+// Every wait is bounded (2 s) and reports through the device status word.
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace bitnet {
+
+namespace pair {
+
+__device__ __forceinline__ uint32_t cta_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// arrive on the barrier at the same shared-memory offset in CTA `rank`
+__device__ __forceinline__ void arrive_remote(uint64_t *bar, uint32_t rank) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_u32(bar)),
+        "r"(rank)
+        : "memory");
+}
+
+// 2-SM TMA load: data lands in this CTA's shared memory; the transaction bytes
+// are counted on the leader CTA's barrier (same offset, peer bit cleared).
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint64_t *bar, void *dst, int32_t c0,
+                                                 int32_t c1) {
+    const uint32_t leader_bar = smem_u32(bar) & 0xFEFFFFFFu;
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(leader_bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc2(uint32_t *dst, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish2() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void mma_sp_i8_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t e,
+                                               uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.sp.cta_group::2.kind::i8 [%0], %1, %2, [%5], %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(e)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_cp_pair_128x128b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// arrive once on the barrier at this offset in both CTAs when the issued
+// tcgen05 operations are complete
+__device__ __forceinline__ void commit_both(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+
+}  // namespace pair
+
+template <bool SPARSE, int BN, int STAGES>
+struct PairCfg {
+    static constexpr int kHalfN = BN / 2;                  // B rows per CTA
+    static constexpr int kARowBytes = SPARSE ? 64 : 128;
+    static constexpr int kBRowBytes = 128;
+    static constexpr int kKStep = SPARSE ? 128 : 64;
+    static constexpr int kABytes = 128 * kARowBytes;
+    static constexpr int kBBytes = kHalfN * kBRowBytes;
+    static constexpr int kEBytes = SPARSE ? 2048 : 0;
+    static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;   // per CTA
+    static constexpr int kMmaPerStage = SPARSE ? 2 : 4;
+    static constexpr int kAAdvance = 32;
+    static constexpr int kBAdvance = SPARSE ? 64 : 32;
+    static constexpr int kAccStride = 256;                // TMEM columns between the two accumulators
+    static constexpr int kECol = 2 * kAccStride - 16;     // metadata columns (8 used)
+    static constexpr int kTmemCols = 512;
+    static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + 2048;
+    // M = 256 (two CTAs), N = BN
+    static constexpr uint32_t kIdesc = (SPARSE ? (1u << 2) : 0u) | ((SPARSE ? 2u : 1u) << 4) | (1u << 7) |
+                                       (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                                       (static_cast<uint32_t>(256 >> 4) << 24);
+    static_assert(!SPARSE || (BN % 32 == 0 && BN <= 224), "sparse pair tiles: N multiple of 32, two buffers + metadata");
+    static_assert(SPARSE || (BN % 32 == 0 && BN <= 256), "dense pair tiles: N multiple of 32");
+    static_assert(kBBytes % 1024 == 0, "B tile must keep the 128-byte swizzle atoms aligned");
+};
+
+struct PairParams {
+    int64_t M, N, K;
+    int64_t meta_rows;           // sparse: rows of one metadata k-block
+    const float *gamma;
+    const float *amax;           // sparse: per-token scale
+    void *out;
+    int out_bf16;
+    int32_t *acc_out;
+    uint32_t *status;
+};
+
+template <bool SPARSE, int BN, int STAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+    k_umma_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmE, PairParams p) {
+    using C = PairCfg<SPARSE, BN, STAGES>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sA = smem;
+    uint8_t *sB = sA + STAGES * C::kABytes;
+    uint8_t *sE = sB + STAGES * C::kBBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sE + STAGES * C::kEBytes);
+    uint64_t *empty = full + STAGES;
+    uint64_t *acc_full = empty + STAGES;       // [2]
+    uint64_t *acc_empty = acc_full + 2;        // [2], leader: one arrival per CTA
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+    float *s_scale = reinterpret_cast<float *>(s_tmem + 4);   // BN floats
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = pair::cta_rank();
+    const bool leader = rank == 0;
+    const int64_t pair_id = blockIdx.x >> 1, pairs = gridDim.x >> 1;
+    const int64_t m_tiles = (p.M + 255) / 256, n_tiles = (p.N + BN - 1) / BN;
+    const int64_t tiles = m_tiles * n_tiles;
+    const int ktiles = static_cast<int>((p.K + C::kKStep - 1) / C::kKStep);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 2);
+        }
+        *s_abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        pair::tmem_alloc2(s_tmem, C::kTmemCols);
+        pair::tmem_relinquish2();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmA);
+        prefetch_tensormap(&tmB);
+        if (SPARSE) prefetch_tensormap(&tmE);
+    }
+    tc_fence_before();
+    pair::cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int it = 0;
+            for (int64_t t = pair_id; t < tiles && !*s_abort; t += pairs) {
+                const int64_t mt = t / n_tiles, nt = t - mt * n_tiles;
+                const int32_t a_row = static_cast<int32_t>(mt * 256 + 128 * rank);
+                const int32_t b_row = static_cast<int32_t>(nt * BN + C::kHalfN * rank);
+                // metadata rows past the padded end (a ragged last pair) read a valid block:
+                // their A rows are zero-filled, so any valid index pattern gives zero
+                int64_t e_row = mt * 256 + 128 * rank;
+                if (e_row > p.meta_rows - 128) e_row = p.meta_rows - 128;
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (it >= STAGES && !mbar_wait_bounded(&empty[s], ((it / STAGES) - 1) & 1, s_abort, p.status))
+                        break;
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
+                    if (SPARSE) {
+                        pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * (C::kKStep / 2), a_row);
+                        pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
+                        pair::tma_load_2d_pair(&tmE, &full[s], sE + s * C::kEBytes, 0,
+                                               static_cast<int32_t>(kt * p.meta_rows + e_row));
+                    } else {
+                        pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * C::kKStep, a_row);
+                        pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer (leader CTA)
+        if (leader && lane == 0) {
+            int it = 0, local = 0;
+            for (int64_t t = pair_id; t < tiles && !*s_abort; t += pairs, ++local) {
+                const int b = local & 1;
+                // both CTAs' epilogues must have drained this accumulator buffer
+                if (local >= 2 && !mbar_wait_bounded(&acc_empty[b], ((local >> 1) - 1) & 1, s_abort, p.status)) break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + b * C::kAccStride;
+                for (int kt = 0; kt < ktiles; ++kt, ++it) {
+                    const int s = it % STAGES;
+                    if (!mbar_wait_bounded(&full[s], (it / STAGES) & 1, s_abort, p.status)) break;
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA + s * C::kABytes);
+                    const uint32_t b_base = smem_u32(sB + s * C::kBBytes);
+                    if (SPARSE) {
+                        const uint32_t e_col = tmem + C::kECol + 4u * (it & 1);
+                        pair::tmem_cp_pair_128x128b(
+                            e_col, make_smem_desc(smem_u32(sE + s * C::kEBytes), 16, 128, kSwizzleNone));
+#pragma unroll
+                        for (int j = 0; j < C::kMmaPerStage; ++j) {
+                            const uint64_t ad = make_smem_desc(a_base + j * C::kAAdvance, 16, 512, kSwizzle64B);
+                            const uint64_t bd = make_smem_desc(b_base + j * C::kBAdvance, 16, 1024, kSwizzle128B);
+                            pair::mma_sp_i8_pair(d_tmem, ad, bd, C::kIdesc, e_col + 2u * j, (kt | j) != 0);
+                        }
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < C::kMmaPerStage; ++j) {
+                            const uint64_t ad = make_smem_desc(a_base + j * C::kAAdvance, 16, 1024, kSwizzle128B);
+                            const uint64_t bd = make_smem_desc(b_base + j * C::kBAdvance, 16, 1024, kSwizzle128B);
+                            pair::mma_bf16_pair(d_tmem, ad, bd, C::kIdesc, (kt | j) != 0);
+                        }
+                    }
+                    pair::commit_both(&empty[s]);
+                }
+                pair::commit_both(&acc_full[b]);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue (warps 2..5, both CTAs)
+        const int quarter = warp & 3;
+        const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
+        int local = 0;
+        for (int64_t t = pair_id; t < tiles; t += pairs, ++local) {
+            const int b = local & 1;
+            const int64_t mt = t / n_tiles, nt = t - mt * n_tiles;
+            const int64_t m0 = mt * 256 + 128 * rank;   // this CTA's accumulator rows
+            const int64_t n0 = nt * BN;
+            if (SPARSE) {
+                const float g = *p.gamma;
+                asm volatile("bar.sync 1, 128;" ::: "memory");   // previous tile's scales are no longer read
+                for (int j = threadIdx.x - 64; j < BN; j += 128) {
+                    const int64_t tok = n0 + j;
+                    s_scale[j] = (tok < p.N) ? __fdiv_rn(__fmul_rn(g, p.amax[tok]), 127.0f) : 0.0f;
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+            }
+            const bool ok = mbar_wait_bounded(&acc_full[b], (local >> 1) & 1, s_abort, p.status);
+            tc_fence_after();
+            const int64_t m = m0 + 32 * quarter + lane;
+            const uint32_t taddr = tmem + lane_base + b * C::kAccStride;
+            if (ok) {
+#pragma unroll 1
+                for (int c = 0; c < BN / 16; ++c) {
+                    uint32_t r[16];
+                    tmem_ld_32x32b_x16(taddr + 16 * c, r);
+                    tmem_ld_wait();
+                    if (m >= p.M) continue;
+                    if (SPARSE) {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int64_t tok = n0 + 16 * c + j;
+                            if (tok < p.N) {
+                                const int acc = static_cast<int>(r[j]);
+                                const float y = __fmul_rn(__int2float_rn(acc), s_scale[16 * c + j]);
+                                if (p.out_bf16)
+                                    static_cast<__nv_bfloat16 *>(p.out)[tok * p.M + m] = __float2bfloat16_rn(y);
+                                else
+                                    static_cast<float *>(p.out)[tok * p.M + m] = y;
+                                if (p.acc_out) p.acc_out[tok * p.M + m] = acc;
+                            }
+                        }
+                    } else {
+                        const float g = *p.gamma;
+                        const int64_t nb = n0 + 16 * c;
+                        if (nb + 16 <= p.N) {
+                            if (p.out_bf16) {
+                                uint32_t h[8];
+#pragma unroll
+                                for (int j = 0; j < 8; ++j) {
+                                    const __nv_bfloat162 v = __floats2bfloat162_rn(
+                                        __fmul_rn(__uint_as_float(r[2 * j]), g), __fmul_rn(__uint_as_float(r[2 * j + 1]), g));
+                                    h[j] = *reinterpret_cast<const uint32_t *>(&v);
+                                }
+                                uint4 *dst = reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(p.out) + m * p.N + nb);
+                                dst[0] = make_uint4(h[0], h[1], h[2], h[3]);
+                                dst[1] = make_uint4(h[4], h[5], h[6], h[7]);
+                            } else {
+                                float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + m * p.N + nb);
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    dst[j] = make_float4(__fmul_rn(__uint_as_float(r[4 * j]), g),
+                                                         __fmul_rn(__uint_as_float(r[4 * j + 1]), g),
+                                                         __fmul_rn(__uint_as_float(r[4 * j + 2]), g),
+                                                         __fmul_rn(__uint_as_float(r[4 * j + 3]), g));
+                            }
+                        } else {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int64_t n = nb + j;
+                                if (n < p.N) {
+                                    const float y = __fmul_rn(__uint_as_float(r[j]), g);
+                                    if (p.out_bf16)
+                                        static_cast<__nv_bfloat16 *>(p.out)[m * p.N + n] = __float2bfloat16_rn(y);
+                                    else
+                                        static_cast<float *>(p.out)[m * p.N + n] = y;
+                                }
+                            }
+                        }
+                    }
+                }
+            }
+            // this CTA is done with the buffer: one arrival on the leader's barrier
+            tc_fence_before();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (threadIdx.x == 64) pair::arrive_remote(&acc_empty[b], 0);
+            if (!ok) break;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    pair::cluster_sync();   // no CTA leaves while its peer may still signal it
+    if (warp == 1) {
+        tc_fence_after();
+        pair::tmem_dealloc2(tmem, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- host side
+
+typedef CUresult (*PFN_encodeTiled2)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                     const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                     CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static PFN_encodeTiled2 encode_fn() {
+    static PFN_encodeTiled2 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_encodeTiled2>(ptr);
+    });
+    return fn;
+}
+
+static bool map2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                  uint64_t pitch_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
+    PFN_encodeTiled2 enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {pitch_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <bool SPARSE, int BN, int STAGES>
+static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &e, const PairParams &p,
+                            cudaStream_t s) {
+    using C = PairCfg<SPARSE, BN, STAGES>;
+    auto kern = k_umma_pair<SPARSE, BN, STAGES>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        if (err != cudaSuccess) return err;
+        attr_set = true;
+    }
+    const int64_t tiles = ((p.M + 255) / 256) * ((p.N + BN - 1) / BN);
+    int64_t pairs = num_sms() / 2;
+    if (pairs > tiles) pairs = tiles;
+    if (pairs < 1) pairs = 1;
+    kern<<<dim3(static_cast<unsigned>(2 * pairs)), 192, C::kSmemBytes, s>>>(a, b, e, p);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gemm_sp_pair(const int8_t *Xq, const float *amax, const float *gamma, const int8_t *vals,
+                                const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16,
+                                int32_t *acc, uint32_t *status, cudaStream_t s) {
+    constexpr int BN = 224;
+    PairParams p{};
+    p.M = n_out;
+    p.N = T;
+    p.K = k;
+    p.meta_rows = (n_out + 127) / 128 * 128;
+    p.gamma = gamma;
+    p.amax = amax;
+    p.out = Y;
+    p.out_bf16 = y_bf16 ? 1 : 0;
+    p.acc_out = acc;
+    p.status = status;
+    CUtensorMap ma, mb, me;
+    if (!map2d(&ma, CU_TENSOR_MAP_DATA_TYPE_UINT8, vals, static_cast<uint64_t>(k / 2), static_cast<uint64_t>(n_out),
+               static_cast<uint64_t>(k / 2), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    if (!map2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, static_cast<uint64_t>(k), static_cast<uint64_t>(T),
+               static_cast<uint64_t>(k), 128, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const uint64_t meta_total_rows = static_cast<uint64_t>((k + 127) / 128) * static_cast<uint64_t>(p.meta_rows);
+    if (!map2d(&me, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, 16, meta_total_rows, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    return run_pair<true, BN, 8>(ma, mb, me, p, s);
+}
+
+cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *wt, const float *gamma, int64_t T,
+                                  int64_t n_out, int64_t k, void *dX, bool dx_bf16, uint32_t *status, cudaStream_t s) {
+    constexpr int BN = 256;
+    PairParams p{};
+    p.M = T;
+    p.N = k;
+    p.K = n_out;
+    p.gamma = gamma;
+    p.out = dX;
+    p.out_bf16 = dx_bf16 ? 1 : 0;
+    p.status = status;
+    CUtensorMap ma, mb;
+    if (!map2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, static_cast<uint64_t>(n_out), static_cast<uint64_t>(T),
+               static_cast<uint64_t>(n_out) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!map2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wt, static_cast<uint64_t>(n_out), static_cast<uint64_t>(k),
+               static_cast<uint64_t>(n_out) * 2, 64, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    return run_pair<false, BN, 6>(ma, mb, ma, p, s);
+}
+
+}  // namespace bitnet

@@ -23,6 +23,7 @@
 namespace bitnet {
 
 constexpr int kDecWarps = 4;
+constexpr int kDecRegTiles = 16;   // k-tiles (8 bytes each) prefetched per lane per round
 
 // int8 code of one activation: clamp(rint(fp32(x * s)), -127, 127)
 __device__ __forceinline__ int8_t quant_code(float x, float s) {
@@ -64,35 +65,35 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_gemv_dec(const uint2 *__rest
     const bool tok = gid < T;
     const int8_t *xrow = Xq + static_cast<int64_t>(tok ? gid : 0) * K + 4 * tq;
 
+    // every weight record of this warp's first round is in flight before any use;
+    // they do not depend on the previous kernel, so they are issued before the wait
+    uint2 w[kDecRegTiles];
+#pragma unroll
+    for (int i = 0; i < kDecRegTiles; ++i)
+        if (kt0 + i < kt1) w[i] = __ldg(src + (kt0 + i) * 32);
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     int d[4] = {0, 0, 0, 0};
-    int64_t kt = kt0;
-    // two tiles per iteration: both 8-byte records are issued before use
-    for (; kt + 1 < kt1; kt += 2) {
-        const uint2 w0 = __ldg(src + kt * 32);
-        const uint2 w1 = __ldg(src + (kt + 1) * 32);
-        uint32_t b0[4], b1[4];
+    for (int64_t base = kt0; base < kt1; base += kDecRegTiles) {
+        if (base != kt0) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            b0[j] = tok ? __ldg(reinterpret_cast<const uint32_t *>(xrow + kt * 64 + 16 * j)) : 0u;
-            b1[j] = tok ? __ldg(reinterpret_cast<const uint32_t *>(xrow + (kt + 1) * 64 + 16 * j)) : 0u;
+            for (int i = 0; i < kDecRegTiles; ++i)
+                if (base + i < kt1) w[i] = __ldg(src + (base + i) * 32);
         }
-        uint32_t a0[4], a1[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-            a0[r] = expand_codes(w0.x, r);
-            a1[r] = expand_codes(w1.x, r);
+        for (int i = 0; i < kDecRegTiles; ++i) {
+            const int64_t kt = base + i;
+            if (kt < kt1) {
+                uint32_t a[4], b[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    b[j] = tok ? __ldg(reinterpret_cast<const uint32_t *>(xrow + kt * 64 + 16 * j)) : 0u;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) a[r] = expand_codes(w[i].x, r);
+                mma_sp_m16n8k64(d, a, b, w[i].y);
+            }
         }
-        mma_sp_m16n8k64(d, a0, b0, w0.y);
-        mma_sp_m16n8k64(d, a1, b1, w1.y);
-    }
-    if (kt < kt1) {
-        const uint2 w0 = __ldg(src + kt * 32);
-        uint32_t b0[4], a0[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) b0[j] = tok ? __ldg(reinterpret_cast<const uint32_t *>(xrow + kt * 64 + 16 * j)) : 0u;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) a0[r] = expand_codes(w0.x, r);
-        mma_sp_m16n8k64(d, a0, b0, w0.y);
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) s_part[warp][lane][q] = d[q];
@@ -100,10 +101,10 @@ __global__ void __launch_bounds__(kDecWarps * 32) k_gemv_dec(const uint2 *__rest
     if (warp != 0) return;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-        int s = 0;
+        int sum = 0;
 #pragma unroll
-        for (int w = 0; w < kDecWarps; ++w) s += s_part[w][lane][q];
-        d[q] = s;
+        for (int w2 = 0; w2 < kDecWarps; ++w2) sum += s_part[w2][lane][q];
+        d[q] = sum;
     }
     const float g = *gamma;
 #pragma unroll
@@ -180,7 +181,7 @@ __global__ void __launch_bounds__(256) k_gemv_gb(const uint8_t *__restrict__ gb,
 // Launched with programmatic stream serialisation, consecutive projections
 // overlap: the next kernel streams its weights while this one finishes.
 constexpr int kFusedWarps = 8;
-constexpr int kFusedRegTiles = 8;   // k-tiles prefetched per lane per round
+constexpr int kFusedRegTiles = 16;  // k-tiles prefetched per lane per round
 
 template <bool BF16>
 __device__ __forceinline__ float load_x(const void *X, int64_t idx) {
@@ -218,11 +219,14 @@ __device__ __forceinline__ uint32_t quant4(const void *X, int64_t idx, float s) 
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(kFusedWarps * 32) k_gemv_fused(const uint2 *__restrict__ dec, const void *__restrict__ X,
+__global__ void __launch_bounds__(kFusedWarps * 32, 2) k_gemv_fused(const uint2 *__restrict__ dec, const void *__restrict__ X,
                                                                  float eps, const float *__restrict__ gamma, int T,
                                                                  int64_t n_out, int64_t K, void *__restrict__ Y,
                                                                  int y_bf16, int32_t *__restrict__ acc_out,
                                                                  int8_t *__restrict__ xq_out, float *__restrict__ amax_out) {
+    // dynamic shared memory: the int8 codes of the T activation rows, row pitch
+    // K + 16 bytes so that the 8 token rows of a B fragment fall in different banks
+    extern __shared__ __align__(16) int8_t s_xq[];
     __shared__ int s_part[kFusedWarps][32][4];
     __shared__ float s_red[kFusedWarps][8];
     __shared__ float s_amax[8];
@@ -230,6 +234,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32) k_gemv_fused(const uint2 *__
     const int gid = lane >> 2, tq = lane & 3;
     const int64_t rt = blockIdx.x;
     const int64_t ktiles = K / 64;
+    const int64_t pitch = K + 16;
     const int64_t per_warp = (ktiles + kFusedWarps - 1) / kFusedWarps;
     const int64_t kt0 = warp * per_warp;
     const int64_t kt1 = (kt0 + per_warp < ktiles) ? kt0 + per_warp : ktiles;
@@ -272,11 +277,17 @@ __global__ void __launch_bounds__(kFusedWarps * 32) k_gemv_fused(const uint2 *__
         s_amax[threadIdx.x] = v > eps ? v : eps;
     }
     __syncthreads();
-    const bool tok = gid < T;
-    const float s_tok = tok ? __fdiv_rn(127.0f, s_amax[gid]) : 0.0f;
-    const int64_t xbase = static_cast<int64_t>(tok ? gid : 0) * K + 4 * tq;
+    // 3. quantise the rows once into shared memory (four codes per thread step, L1/L2 hits)
+    for (int t = 0; t < T; ++t) {
+        const float st = __fdiv_rn(127.0f, s_amax[t]);
+        for (int64_t i = 4 * threadIdx.x; i < K; i += 4 * blockDim.x)
+            *reinterpret_cast<uint32_t *>(s_xq + t * pitch + i) = quant4<BF16>(X, t * K + i, st);
+    }
+    __syncthreads();
 
-    // 3. sparse MMAs over this warp's k-range
+    // 4. sparse MMAs over this warp's k-range; B fragments from shared memory
+    const bool tok = gid < T;
+    const int8_t *xs = s_xq + (tok ? gid : 0) * pitch + 4 * tq;
     int d[4] = {0, 0, 0, 0};
     for (int64_t base = kt0; base < kt1; base += kFusedRegTiles) {
         if (base != kt0) {
@@ -290,7 +301,8 @@ __global__ void __launch_bounds__(kFusedWarps * 32) k_gemv_fused(const uint2 *__
             if (kt < kt1) {
                 uint32_t a[4], b[4];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) b[j] = tok ? quant4<BF16>(X, xbase + kt * 64 + 16 * j, s_tok) : 0u;
+                for (int j = 0; j < 4; ++j)
+                    b[j] = tok ? *reinterpret_cast<const uint32_t *>(xs + kt * 64 + 16 * j) : 0u;
 #pragma unroll
                 for (int r = 0; r < 4; ++r) a[r] = expand_codes(w[i].x, r);
                 mma_sp_m16n8k64(d, a, b, w[i].y);
@@ -302,8 +314,8 @@ __global__ void __launch_bounds__(kFusedWarps * 32) k_gemv_fused(const uint2 *__
     __syncthreads();
     if (blockIdx.x == 0 && (xq_out || amax_out)) {   // optional copy of the int8 activations
         for (int64_t i = threadIdx.x; i < static_cast<int64_t>(T) * K; i += blockDim.x) {
-            const int t = static_cast<int>(i / K);
-            if (xq_out) xq_out[i] = quant_code(load_x<BF16>(X, i), __fdiv_rn(127.0f, s_amax[t]));
+            const int64_t t = i / K;
+            if (xq_out) xq_out[i] = s_xq[t * pitch + (i - t * K)];
         }
         if (amax_out && threadIdx.x < T) amax_out[threadIdx.x] = s_amax[threadIdx.x];
     }
@@ -338,7 +350,7 @@ cudaError_t launch_gemv_fused(const void *X, bool x_bf16, float eps, const float
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_out / 16));
     cfg.blockDim = dim3(kFusedWarps * 32);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = static_cast<size_t>(T) * static_cast<size_t>(k + 16);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -348,6 +360,15 @@ cudaError_t launch_gemv_fused(const void *X, bool x_bf16, float eps, const float
     const uint2 *d2 = reinterpret_cast<const uint2 *>(dec);
     const int Ti = static_cast<int>(T);
     const int yb = y_bf16 ? 1 : 0;
+    static bool attr_done[2] = {false, false};
+    if (!attr_done[x_bf16 ? 1 : 0]) {
+        cudaError_t e = x_bf16 ? cudaFuncSetAttribute(k_gemv_fused<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(kFusedMaxSmem))
+                               : cudaFuncSetAttribute(k_gemv_fused<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(kFusedMaxSmem));
+        if (e != cudaSuccess) return e;
+        attr_done[x_bf16 ? 1 : 0] = true;
+    }
     if (x_bf16)
         return cudaLaunchKernelEx(&cfg, k_gemv_fused<true>, d2, X, eps, gamma, Ti, n_out, k, Y, yb, acc, xq_out,
                                   amax_out);
@@ -357,10 +378,17 @@ cudaError_t launch_gemv_fused(const void *X, bool x_bf16, float eps, const float
 cudaError_t launch_gemv_dec(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *dec,
                             int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                             cudaStream_t s) {
-    const unsigned grid = static_cast<unsigned>(n_out / 16);
-    k_gemv_dec<<<grid, kDecWarps * 32, 0, s>>>(reinterpret_cast<const uint2 *>(dec), Xq, amax, gamma,
-                                               static_cast<int>(T), n_out, k, Y, y_bf16 ? 1 : 0, acc);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_out / 16));
+    cfg.blockDim = dim3(kDecWarps * 32);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_gemv_dec, reinterpret_cast<const uint2 *>(dec), Xq, amax, gamma,
+                              static_cast<int>(T), n_out, k, Y, y_bf16 ? 1 : 0, acc);
 }
 
 cudaError_t launch_gemv_gb(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *gb,

@@ -3,6 +3,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 namespace bitnet {
@@ -11,8 +12,12 @@ namespace bitnet {
 // always the first 4 bytes.
 constexpr size_t kStatusOffset = 0;
 // pack: threshold bits, 128-bit window sum, 256 exponent bins
+constexpr size_t kPackWsCounterOffset = 4;
 constexpr size_t kPackWsThrOffset = 8;
+constexpr size_t kPackWsModeOffset = 12;
 constexpr size_t kPackWsWinOffset = 16;
+constexpr size_t kPackWsListCountOffset = 32;
+constexpr size_t kPackWsBandOffset = 40;
 constexpr size_t kPackWsBinsOffset = 256;
 constexpr size_t kPackWsBytes = 256 + 256 * 8;
 // linear: status word only
@@ -29,12 +34,19 @@ cudaError_t launch_pack(const float *W, int64_t n_out, int64_t k, int n, int m, 
                         uint8_t *gb, int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws,
                         cudaStream_t s);
 
+cudaError_t launch_pack_update(const float *W, int64_t n_out, int64_t k, float eps, float *gamma, uint8_t *gb,
+                               int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws, size_t ws_bytes,
+                               cudaStream_t s);
+
 cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xq, float *amax,
                              cudaStream_t s);
 
 cudaError_t launch_gemv_dec(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *dec,
                             int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                             cudaStream_t s);
+
+// Largest shared-memory staging of the fused decode kernel: T * (k + 16) bytes.
+constexpr size_t kFusedMaxSmem = 160 * 1024;
 
 cudaError_t launch_gemv_fused(const void *X, bool x_bf16, float eps, const float *gamma, const uint8_t *dec,
                               int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
@@ -47,6 +59,13 @@ cudaError_t launch_gemv_gb(const int8_t *Xq, const float *amax, const float *gam
 cudaError_t launch_gemm_sp(const int8_t *Xq, const float *amax, const float *gamma, const int8_t *vals,
                            const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16,
                            int32_t *acc, uint32_t *status, cudaStream_t s);
+
+cudaError_t launch_gemm_sp_pair(const int8_t *Xq, const float *amax, const float *gamma, const int8_t *vals,
+                                const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16,
+                                int32_t *acc, uint32_t *status, cudaStream_t s);
+
+cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *wt, const float *gamma, int64_t T,
+                                  int64_t n_out, int64_t k, void *dX, bool dx_bf16, uint32_t *status, cudaStream_t s);
 
 cudaError_t launch_dgrad(const void *dY, const float *gamma, const uint8_t *gb, int64_t T, int64_t n_out,
                          int64_t k, void *dX, bool dx_bf16, void *ws, cudaStream_t s);

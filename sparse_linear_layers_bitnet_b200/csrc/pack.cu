@@ -48,9 +48,91 @@ __device__ __forceinline__ void accumulate_abs(uint32_t bits, uint64_t &lo, uint
     }
 }
 
-__global__ void __launch_bounds__(256) k_abs_sum(const float4 *__restrict__ W, int64_t n4,
+// ---------------------------------------------------------------- finaliser
+
+// value += v * 2^shift on a little-endian array of 32-bit limbs (shared memory).
+__device__ void limbs_add(uint32_t *limb, int nlimb, uint64_t v, int shift) {
+    int q = shift >> 5, r = shift & 31;
+    // v * 2^r spans at most three limbs
+    const uint64_t lo = v << r;
+    const uint64_t hi = r ? (v >> (64 - r)) : 0ull;
+    uint64_t add[3] = {lo & 0xffffffffull, lo >> 32, hi};
+    uint64_t carry = 0;
+    for (int j = q; j < nlimb; ++j) {
+        const uint64_t a = (j - q < 3) ? add[j - q] : 0ull;
+        if (j - q >= 3 && carry == 0) break;
+        const uint64_t s2 = static_cast<uint64_t>(limb[j]) + a + carry;
+        limb[j] = static_cast<uint32_t>(s2);
+        carry = s2 >> 32;
+    }
+}
+
+constexpr int kLimbs = 12;   // 384 bits
+
+// Turns the exact integer sum (window + bins, in units of 2^-149) into gamma
+// and the code threshold.  Called by one thread; bins and limbs in shared memory.
+__device__ void finalize_gamma(const unsigned long long *s_bins, const int *s_nz, int n_nz, uint64_t wlo,
+                               uint64_t whi, int64_t n, float eps, uint32_t *limb, float *gamma, uint32_t *thr_out) {
+    for (int j = 0; j < kLimbs; ++j) limb[j] = 0;
+    // a magnitude with biased exponent e and significand m is m * 2^(max(e,1)-1)
+    // units; window entries were pre-shifted by (e - 96), so they carry 2^95
+    for (int i = 0; i < n_nz; ++i) {
+        const int e = s_nz[i];
+        limbs_add(limb, kLimbs, s_bins[e], (e == 0 ? 1 : e) - 1);
+    }
+    limbs_add(limb, kLimbs, wlo, 95);
+    limbs_add(limb, kLimbs, whi, 95 + 64);
+    // nearest fp64: the top 64 bits with everything below folded into a sticky
+    // bit 0, then the correctly rounded u64 -> f64 conversion
+    int L = -1;
+    for (int j = kLimbs - 1; j >= 0; --j)
+        if (limb[j]) {
+            L = j;
+            break;
+        }
+    double S = 0.0;
+    if (L >= 0) {
+        if (L <= 1) {
+            const uint64_t v = (static_cast<uint64_t>(L == 1 ? limb[1] : 0u) << 32) | limb[0];
+            S = __ull2double_rn(v) * 0x1p-149;   // power-of-two scaling, exact in the normal range
+        } else {
+            const unsigned __int128 top3 = (static_cast<unsigned __int128>(limb[L]) << 64) |
+                                           (static_cast<unsigned __int128>(limb[L - 1]) << 32) | limb[L - 2];
+            const int shift = 32 - __clz(limb[L]);          // keeps the top 64 bits of the 96
+            uint64_t w64 = static_cast<uint64_t>(top3 >> shift);
+            bool sticky = (top3 & ((static_cast<unsigned __int128>(1) << shift) - 1)) != 0;
+            for (int j = 0; j < L - 2 && !sticky; ++j) sticky = limb[j] != 0u;
+            if (sticky) w64 |= 1ull;   // bit 0 lies below the 53-bit rounding position
+            const int ex = 32 * (L - 2) + shift - 149;       // weight of bit 0 of w64
+            S = __ull2double_rn(w64) * __longlong_as_double(static_cast<long long>(1023 + ex) << 52);
+        }
+    }
+    const double mean = __ddiv_rn(S, static_cast<double>(n));
+    float g = __double2float_rn(mean);
+    g = __fadd_rn(g, eps);
+    *gamma = g;
+    // smallest t >= 0 with fp32(t / g) > 0.5
+    uint32_t t = __float_as_uint(__fmul_rn(g, 0.5f));
+    int it = 0;
+    if (__fdiv_rn(__uint_as_float(t), g) > 0.5f) {
+        while (t > 0u && __fdiv_rn(__uint_as_float(t - 1u), g) > 0.5f && it < 64) {
+            --t;
+            ++it;
+        }
+    } else {
+        while (!(__fdiv_rn(__uint_as_float(t), g) > 0.5f) && it < 64) {
+            ++t;
+            ++it;
+        }
+    }
+    *thr_out = t;
+}
+
+__global__ void __launch_bounds__(256, 4) k_abs_sum(const float4 *__restrict__ W, int64_t n4,
                                                  unsigned long long *__restrict__ win,
-                                                 unsigned long long *__restrict__ bins) {
+                                                 unsigned long long *__restrict__ bins,
+                                                 unsigned *__restrict__ counter, int64_t n_total, float eps,
+                                                 float *__restrict__ gamma, uint32_t *__restrict__ thr) {
     __shared__ unsigned long long s_bins[256];
     __shared__ unsigned long long s_lo[8], s_hi[8];
     __shared__ int s_rare;
@@ -113,102 +195,69 @@ __global__ void __launch_bounds__(256) k_abs_sum(const float4 *__restrict__ W, i
         for (int e = threadIdx.x; e < 256; e += blockDim.x)
             if (s_bins[e]) atomicAdd(&bins[e], s_bins[e]);
     }
-}
-
-// ---------------------------------------------------------------- finaliser
-
-// value += v * 2^shift on a little-endian array of 32-bit limbs.
-__device__ void limbs_add(uint32_t *limb, int nlimb, uint64_t v, int shift) {
-    int q = shift >> 5, r = shift & 31;
-    // v * 2^r spans at most three limbs
-    const uint64_t lo = v << r;
-    const uint64_t hi = r ? (v >> (64 - r)) : 0ull;
-    uint64_t add[3] = {lo & 0xffffffffull, lo >> 32, hi};
-    uint64_t carry = 0;
-    for (int j = q; j < nlimb; ++j) {
-        const uint64_t a = (j - q < 3) ? add[j - q] : 0ull;
-        if (j - q >= 3 && carry == 0) break;
-        const uint64_t s = static_cast<uint64_t>(limb[j]) + a + carry;
-        limb[j] = static_cast<uint32_t>(s);
-        carry = s >> 32;
+    // the last block to finish turns the sums into gamma and the threshold
+    __shared__ unsigned s_ticket;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_ticket = atomicAdd(counter, 1u);
+    __syncthreads();
+    if (s_ticket != gridDim.x - 1) return;
+    __threadfence();
+    __shared__ int s_nz[256];
+    __shared__ int s_nnz;
+    __shared__ uint32_t s_limb[kLimbs];
+    if (threadIdx.x == 0) s_nnz = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+        const unsigned long long b = atomicAdd(&bins[e], 0ull);   // coherent read of the final sums
+        s_bins[e] = b;
+        if (b) s_nz[atomicAdd(&s_nnz, 1)] = e;
     }
-}
-
-__global__ void k_finalize_gamma(const unsigned long long *__restrict__ win,
-                                 const unsigned long long *__restrict__ bins, int64_t n, float eps,
-                                 float *__restrict__ gamma, uint32_t *__restrict__ thr_out) {
-    if (threadIdx.x != 0 || blockIdx.x != 0) return;
-    constexpr int NL = 12;   // 384 bits
-    uint32_t limb[NL];
-    for (int j = 0; j < NL; ++j) limb[j] = 0;
-    // value is in units of 2^-149: a magnitude with biased exponent e and
-    // significand m contributes m * 2^(max(e,1)-1); window entries were
-    // pre-shifted by (e - 96), so they carry an extra 2^95.
-    for (int e = 0; e < 256; ++e) {
-        const uint64_t b = bins[e];
-        if (b) limbs_add(limb, NL, b, (e == 0 ? 1 : e) - 1);
-    }
-    limbs_add(limb, NL, win[0], 95);
-    limbs_add(limb, NL, win[1], 95 + 64);
-
-    // nearest fp64: take the top 64 bits, fold everything below into a sticky
-    // bit 0, and let the correctly rounded u64 -> f64 conversion round.
-    int top = -1;
-    for (int j = NL - 1; j >= 0; --j)
-        if (limb[j]) {
-            top = 32 * j + 31 - __clz(limb[j]);
-            break;
-        }
-    double S = 0.0;
-    if (top >= 0) {
-        const int low = top - 63;   // bit index of bit 0 of the 64-bit window
-        uint64_t w64 = 0;
-        bool sticky = false;
-        for (int b = 0; b < 64; ++b) {
-            const int p = low + b;
-            if (p >= 0 && ((limb[p >> 5] >> (p & 31)) & 1u)) w64 |= (1ull << b);
-        }
-        for (int p = 0; p < low; ++p)
-            if ((limb[p >> 5] >> (p & 31)) & 1u) {
-                sticky = true;
-                break;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // ascending exponent order is not needed (integer sums commute), but keep it deterministic
+        for (int i = 1; i < s_nnz; ++i)
+            for (int j = i; j > 0 && s_nz[j - 1] > s_nz[j]; --j) {
+                const int tmp = s_nz[j];
+                s_nz[j] = s_nz[j - 1];
+                s_nz[j - 1] = tmp;
             }
-        if (sticky) w64 |= 1ull;   // bit 0 lies below the 53-bit rounding position
-        const double w = __ull2double_rn(w64);
-        // scale by 2^(low - 149); |low - 149| keeps the factor a normal double
-        const int ex = low - 149;
-        const double scale = __longlong_as_double(static_cast<long long>(1023 + ex) << 52);
-        S = w * scale;
+        const uint64_t wlo = atomicAdd(&win[0], 0ull), whi = atomicAdd(&win[1], 0ull);
+        finalize_gamma(s_bins, s_nz, s_nnz, wlo, whi, n_total, eps, s_limb, gamma, thr);
     }
-    const double mean = __ddiv_rn(S, static_cast<double>(n));
-    float g = __double2float_rn(mean);
-    g = __fadd_rn(g, eps);
-    *gamma = g;
-
-    // smallest t >= 0 with fp32(t / g) > 0.5
-    uint32_t t = __float_as_uint(__fmul_rn(g, 0.5f));
-    auto pred = [g](uint32_t x) { return __fdiv_rn(__uint_as_float(x), g) > 0.5f; };
-    int it = 0;
-    if (pred(t)) {
-        while (t > 0u && pred(t - 1u) && it < 64) {
-            --t;
-            ++it;
-        }
-    } else {
-        while (!pred(t) && it < 64) {
-            ++t;
-            ++it;
-        }
-    }
-    *thr_out = t;
 }
 
 // ---------------------------------------------------------------- pass 2 (2:4)
+
+// Division of 32-bit indices by an invariant divisor with one multiply-high
+// (Granlund and Montgomery, "Division by Invariant Integers using
+// Multiplication", PLDI 1994, section 4: m = floor(2^32 (2^l - d) / d) + 1,
+// q = (t + ((n - t) >> 1)) >> (l - 1) with t = umulhi(m, n), l = ceil(log2 d)).
+struct FastDiv32 {
+    uint32_t d, m, s1, s2;
+};
+
+static FastDiv32 make_fastdiv(uint32_t d) {
+    FastDiv32 f;
+    f.d = d;
+    int l = 0;
+    while ((1ull << l) < d) ++l;   // l = ceil(log2 d)
+    f.m = static_cast<uint32_t>(((1ull << 32) * ((1ull << l) - d)) / d + 1);
+    f.s1 = l > 0 ? 1u : 0u;
+    f.s2 = l > 0 ? static_cast<uint32_t>(l - 1) : 0u;
+    return f;
+}
+
+__device__ __forceinline__ uint32_t fastdiv(uint32_t n, const FastDiv32 &f) {
+    const uint32_t t = __umulhi(f.m, n);
+    return (t + ((n - t) >> f.s1)) >> f.s2;
+}
 
 struct Pack24Args {
     const float4 *W;
     int64_t n_groups;    // n_out * k / 4
     int64_t gpr;         // groups per row = k / 4
+    FastDiv32 gpr_div;   // division by gpr (group indices < 2^32)
     int64_t n_out;
     int64_t k;
     int64_t meta_rows;   // rows of one metadata k-block = ceil(n_out/128)*128
@@ -219,59 +268,656 @@ struct Pack24Args {
     uint8_t *mask;       // [n_out*k/8] or null
 };
 
+// Bit q set when position q is among the two largest magnitudes of the group
+// (ties to the lower position).  Position p is ranked behind q < p when
+// mag[q] >= mag[p], and behind q > p when mag[q] > mag[p]; p is kept when at
+// most one position is ranked ahead of it.  Six comparisons.
+__device__ __forceinline__ uint32_t top2_of_4(const uint32_t (&mag)[4]) {
+    const uint32_t g01 = mag[0] >= mag[1], g02 = mag[0] >= mag[2], g03 = mag[0] >= mag[3];
+    const uint32_t g12 = mag[1] >= mag[2], g13 = mag[1] >= mag[3], g23 = mag[2] >= mag[3];
+    const uint32_t ahead0 = (1u - g01) + (1u - g02) + (1u - g03);
+    const uint32_t ahead1 = g01 + (1u - g12) + (1u - g13);
+    const uint32_t ahead2 = g02 + g12 + (1u - g23);
+    const uint32_t ahead3 = g03 + g13 + g23;
+    return (ahead0 < 2u ? 1u : 0u) | (ahead1 < 2u ? 2u : 0u) | (ahead2 < 2u ? 4u : 0u) | (ahead3 < 2u ? 8u : 0u);
+}
+
+// Ranks one group, writes every requested layout with threshold thr, and
+// returns whether one of its kept magnitudes lies in [band_lo, band_hi].
+__device__ __forceinline__ uint32_t pack_group(const Pack24Args &p, uint32_t thr, int lane, int64_t i, bool valid,
+                                               const float4 v, uint32_t band_lo, uint32_t band_hi) {
+    uint32_t bits[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z), __float_as_uint(v.w)};
+    uint32_t mag[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) mag[q] = bits[q] & 0x7fffffffu;   // |w| as ordered integers
+    const uint32_t keep = top2_of_4(mag);
+    const uint32_t i0 = __ffs(keep) - 1;
+    const uint32_t i1 = 31 - __clz(keep);
+    // register selects instead of a dynamically indexed array (no local memory)
+    const uint32_t b0 = i0 == 0 ? bits[0] : (i0 == 1 ? bits[1] : (i0 == 2 ? bits[2] : bits[3]));
+    const uint32_t b1 = i1 == 0 ? bits[0] : (i1 == 1 ? bits[1] : (i1 == 2 ? bits[2] : bits[3]));
+    const uint32_t nz0 = (b0 & 0x7fffffffu) >= thr, nz1 = (b1 & 0x7fffffffu) >= thr;
+    const uint32_t c0 = nz0 ? ((b0 >> 31) ? 3u : 1u) : 0u;
+    const uint32_t c1 = nz1 ? ((b1 >> 31) ? 3u : 1u) : 0u;
+    const uint32_t nib = i0 | (i1 << 2);
+    if (valid && p.gb) p.gb[i] = static_cast<uint8_t>(nib | (c0 << 4) | (c1 << 6));
+    if (valid && p.vals) {
+        const uint32_t v0 = nz0 ? ((b0 >> 31) ? 0xffu : 0x01u) : 0u;
+        const uint32_t v1 = nz1 ? ((b1 >> 31) ? 0xffu : 0x01u) : 0u;
+        p.vals[i] = static_cast<uint16_t>(v0 | (v1 << 8));
+    }
+    // neighbouring groups share a byte in the metadata and the mask
+    const uint32_t nib_hi = __shfl_xor_sync(0xffffffffu, nib, 1);
+    const uint32_t keep_hi = __shfl_xor_sync(0xffffffffu, keep, 1);
+    if (valid && (lane & 1) == 0) {
+        const uint32_t row32 = fastdiv(static_cast<uint32_t>(i), p.gpr_div);
+        const int64_t row = row32, g = i - row * p.gpr;
+        if (p.meta) {
+            const int64_t kb = g >> 5;
+            const int64_t off = ((kb * p.meta_rows + row) << 4) + ((g & 31) >> 1);
+            p.meta[off] = static_cast<uint8_t>(nib | (nib_hi << 4));
+        }
+        if (p.mask) p.mask[(row * p.k >> 3) + (g >> 1)] = static_cast<uint8_t>(keep | (keep_hi << 4));
+    }
+    const uint32_t m0 = b0 & 0x7fffffffu, m1 = b1 & 0x7fffffffu;
+    return ((m0 >= band_lo && m0 <= band_hi) || (m1 >= band_lo && m1 <= band_hi)) ? 1u : 0u;
+}
+
+// Rewrites the threshold-dependent bytes of one group (group byte and values).
+__device__ __forceinline__ void patch_group(const Pack24Args &p, uint32_t thr, int64_t i, const float4 v) {
+    uint32_t bits[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z), __float_as_uint(v.w)};
+    uint32_t mag[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) mag[q] = bits[q] & 0x7fffffffu;
+    const uint32_t keep = top2_of_4(mag);
+    const uint32_t i0 = __ffs(keep) - 1, i1 = 31 - __clz(keep);
+    const uint32_t b0 = i0 == 0 ? bits[0] : (i0 == 1 ? bits[1] : (i0 == 2 ? bits[2] : bits[3]));
+    const uint32_t b1 = i1 == 0 ? bits[0] : (i1 == 1 ? bits[1] : (i1 == 2 ? bits[2] : bits[3]));
+    const uint32_t nz0 = (b0 & 0x7fffffffu) >= thr, nz1 = (b1 & 0x7fffffffu) >= thr;
+    const uint32_t c0 = nz0 ? ((b0 >> 31) ? 3u : 1u) : 0u;
+    const uint32_t c1 = nz1 ? ((b1 >> 31) ? 3u : 1u) : 0u;
+    if (p.gb) p.gb[i] = static_cast<uint8_t>(i0 | (i1 << 2) | (c0 << 4) | (c1 << 6));
+    if (p.vals) {
+        const uint32_t v0 = nz0 ? ((b0 >> 31) ? 0xffu : 0x01u) : 0u;
+        const uint32_t v1 = nz1 ? ((b1 >> 31) ? 0xffu : 0x01u) : 0u;
+        p.vals[i] = static_cast<uint16_t>(v0 | (v1 << 8));
+    }
+}
+
+constexpr int kPackUnroll = 4;
+
 __global__ void __launch_bounds__(256) k_pack24(Pack24Args p) {
     const uint32_t thr = *p.thr;
     const int lane = threadIdx.x & 31;
-    const int64_t warp_stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    // warp-aligned iteration so that every lane takes part in the shuffles
-    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31));
+    const int64_t warp_stride = static_cast<int64_t>(gridDim.x) * blockDim.x * kPackUnroll;
+    // each warp takes 32 * kPackUnroll consecutive groups per round; all loads of
+    // the round are issued before any group is processed.  The iteration is
+    // warp-uniform so that every lane takes part in the shuffles.
+    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31)) * kPackUnroll;
          base < p.n_groups; base += warp_stride) {
-        const int64_t i = base + lane;
-        const bool valid = i < p.n_groups;
-        uint32_t bits[4] = {0u, 0u, 0u, 0u};
-        if (valid) {
-            const float4 v = __ldg(p.W + i);
-            bits[0] = __float_as_uint(v.x);
-            bits[1] = __float_as_uint(v.y);
-            bits[2] = __float_as_uint(v.z);
-            bits[3] = __float_as_uint(v.w);
-        }
-        uint32_t mag[4];
+        float4 v[kPackUnroll];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) mag[q] = bits[q] & 0x7fffffffu;   // |w| as ordered integers
-        uint32_t keep = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            int before = 0;   // positions ranked ahead of q: larger, or equal and lower
-#pragma unroll
-            for (int r = 0; r < 4; ++r) before += (mag[r] > mag[q]) || (r < q && mag[r] == mag[q]);
-            keep |= (before < 2 ? 1u : 0u) << q;
+        for (int u = 0; u < kPackUnroll; ++u) {
+            const int64_t i = base + 32 * u + lane;
+            v[u] = (i < p.n_groups) ? __ldg(p.W + i) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        const uint32_t i0 = __ffs(keep) - 1;
-        const uint32_t i1 = 31 - __clz(keep);
-        const uint32_t b0 = bits[i0], b1 = bits[i1];
-        const uint32_t nz0 = (b0 & 0x7fffffffu) >= thr, nz1 = (b1 & 0x7fffffffu) >= thr;
-        const uint32_t c0 = nz0 ? ((b0 >> 31) ? 3u : 1u) : 0u;
-        const uint32_t c1 = nz1 ? ((b1 >> 31) ? 3u : 1u) : 0u;
-        const uint32_t nib = i0 | (i1 << 2);
-        if (valid && p.gb) p.gb[i] = static_cast<uint8_t>(nib | (c0 << 4) | (c1 << 6));
-        if (valid && p.vals) {
-            const uint32_t v0 = nz0 ? ((b0 >> 31) ? 0xffu : 0x01u) : 0u;
-            const uint32_t v1 = nz1 ? ((b1 >> 31) ? 0xffu : 0x01u) : 0u;
-            p.vals[i] = static_cast<uint16_t>(v0 | (v1 << 8));
+#pragma unroll
+        for (int u = 0; u < kPackUnroll; ++u) {
+            const int64_t i = base + 32 * u + lane;
+            pack_group(p, thr, lane, i, i < p.n_groups, v[u], 0u, 0u);
         }
-        // neighbouring groups share a byte in the metadata and the mask
-        const uint32_t nib_hi = __shfl_xor_sync(0xffffffffu, nib, 1);
-        const uint32_t keep_hi = __shfl_xor_sync(0xffffffffu, keep, 1);
-        if (valid && (lane & 1) == 0) {
-            const int64_t row = i / p.gpr, g = i - row * p.gpr;
-            if (p.meta) {
-                const int64_t kb = g >> 5;
-                const int64_t off = ((kb * p.meta_rows + row) << 4) + ((g & 31) >> 1);
-                p.meta[off] = static_cast<uint8_t>(nib | (nib_hi << 4));
+    }
+}
+
+// ---------------------------------------------------------------- single-read update
+
+// Smallest t >= 0 with fp32(t / g) > 0.5 (the code threshold of gamma g).
+__device__ uint32_t code_threshold(float g) {
+    uint32_t t = __float_as_uint(__fmul_rn(g, 0.5f));
+    int it = 0;
+    if (__fdiv_rn(__uint_as_float(t), g) > 0.5f) {
+        while (t > 0u && __fdiv_rn(__uint_as_float(t - 1u), g) > 0.5f && it < 64) {
+            --t;
+            ++it;
+        }
+    } else {
+        while (!(__fdiv_rn(__uint_as_float(t), g) > 0.5f) && it < 64) {
+            ++t;
+            ++it;
+        }
+    }
+    return t;
+}
+
+struct UpdateArgs {
+    Pack24Args p;              // layouts (p.thr unused here)
+    const float *gamma_prev;   // previous gamma of this matrix (the hint), read before it is overwritten
+    float *gamma;              // out (same buffer as gamma_prev)
+    unsigned long long *win, *bins;
+    unsigned *counter;
+    uint32_t *thr;             // new threshold (out)
+    uint32_t *mode;            // 1: patch the listed groups, 2: full second pass
+    uint32_t *band;            // [t_lo, t_hi] of the hint, written by block 0
+    uint32_t *list;            // group indices whose kept weights lie in the band
+    unsigned *list_count;
+    uint32_t list_cap;
+    int64_t n_total;
+    float eps;
+};
+
+// Pass 1 of the update: exact sum of |W| for the new gamma and, when a valid
+// hint exists, every layout computed with the hint's threshold; kept weights
+// whose magnitude lies within a relative 2^-10 of that threshold are listed.
+// The last block forms the new gamma and threshold and chooses: if the new
+// threshold lies inside the band (and the list did not overflow), only the
+// listed groups can change and are patched; otherwise a full second pass runs.
+__global__ void __launch_bounds__(256, 4) k_pack_update(UpdateArgs u) {
+    __shared__ unsigned long long s_bins[256];
+    __shared__ unsigned long long s_lo[8], s_hi[8];
+    __shared__ int s_rare;
+    __shared__ uint32_t s_t, s_tlo, s_thi;
+    __shared__ int s_hint;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0ull;
+    if (threadIdx.x == 0) {
+        s_rare = 0;
+        const float gp = *u.gamma_prev;
+        s_hint = (gp > 0.0f && gp < 3.0e38f) ? 1 : 0;   // finite and positive
+        if (s_hint) {
+            s_t = code_threshold(gp);
+            const float tf = __uint_as_float(s_t);
+            s_tlo = __float_as_uint(__fmul_rd(tf, 1.0f - 0x1p-10f));
+            s_thi = __float_as_uint(__fmul_ru(tf, 1.0f + 0x1p-10f));
+            if (blockIdx.x == 0) {
+                u.band[0] = s_tlo;
+                u.band[1] = s_thi;
             }
-            if (p.mask) p.mask[(row * p.k >> 3) + (g >> 1)] = static_cast<uint8_t>(keep | (keep_hi << 4));
         }
+    }
+    __syncthreads();
+    const bool hint = s_hint != 0;
+    const uint32_t t_old = s_t, t_lo = s_tlo, t_hi = s_thi;
+    const Pack24Args &p = u.p;
+    const int lane = threadIdx.x & 31;
+    uint64_t lo = 0, hi = 0;
+    const int64_t warp_stride = static_cast<int64_t>(gridDim.x) * blockDim.x * kPackUnroll;
+    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31)) * kPackUnroll;
+         base < p.n_groups; base += warp_stride) {
+        float4 v[kPackUnroll];
+#pragma unroll
+        for (int q = 0; q < kPackUnroll; ++q) {
+            const int64_t i = base + 32 * q + lane;
+            v[q] = (i < p.n_groups) ? __ldg(p.W + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < kPackUnroll; ++q) {
+            const int64_t i = base + 32 * q + lane;
+            accumulate_abs(__float_as_uint(v[q].x), lo, hi, s_bins, &s_rare);
+            accumulate_abs(__float_as_uint(v[q].y), lo, hi, s_bins, &s_rare);
+            accumulate_abs(__float_as_uint(v[q].z), lo, hi, s_bins, &s_rare);
+            accumulate_abs(__float_as_uint(v[q].w), lo, hi, s_bins, &s_rare);
+            if (hint) {
+                const uint32_t in_band = pack_group(p, t_old, lane, i, i < p.n_groups, v[q], t_lo, t_hi);
+                if (in_band && i < p.n_groups) {
+                    const unsigned slot = atomicAdd(u.list_count, 1u);
+                    if (slot < u.list_cap) u.list[slot] = static_cast<uint32_t>(i);
+                }
+            }
+        }
+    }
+    // exact-sum reduction, as in k_abs_sum
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+        const uint64_t h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+        const uint64_t sum = lo + l2;
+        hi = hi + h2 + ((sum < lo) ? 1ull : 0ull);
+        lo = sum;
+    }
+    const int warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        s_lo[warp] = lo;
+        s_hi[warp] = hi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint64_t L = 0, H = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            const uint64_t sum = L + s_lo[w];
+            H = H + s_hi[w] + ((sum < L) ? 1ull : 0ull);
+            L = sum;
+        }
+        if (L | H) {
+            const unsigned long long old = atomicAdd(&u.win[0], static_cast<unsigned long long>(L));
+            const uint64_t carry = (static_cast<uint64_t>(old) + L < static_cast<uint64_t>(old)) ? 1ull : 0ull;
+            atomicAdd(&u.win[1], static_cast<unsigned long long>(H + carry));
+        }
+    }
+    if (s_rare) {
+        for (int e = threadIdx.x; e < 256; e += blockDim.x)
+            if (s_bins[e]) atomicAdd(&u.bins[e], s_bins[e]);
+    }
+    __shared__ unsigned s_ticket;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_ticket = atomicAdd(u.counter, 1u);
+    __syncthreads();
+    if (s_ticket != gridDim.x - 1) return;
+    __threadfence();
+    __shared__ int s_nz[256];
+    __shared__ int s_nnz;
+    __shared__ uint32_t s_limb[kLimbs];
+    if (threadIdx.x == 0) s_nnz = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+        const unsigned long long b = atomicAdd(&u.bins[e], 0ull);
+        s_bins[e] = b;
+        if (b) s_nz[atomicAdd(&s_nnz, 1)] = e;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int i = 1; i < s_nnz; ++i)
+            for (int j = i; j > 0 && s_nz[j - 1] > s_nz[j]; --j) {
+                const int tmp = s_nz[j];
+                s_nz[j] = s_nz[j - 1];
+                s_nz[j - 1] = tmp;
+            }
+        const uint64_t wlo = atomicAdd(&u.win[0], 0ull), whi = atomicAdd(&u.win[1], 0ull);
+        finalize_gamma(s_bins, s_nz, s_nnz, wlo, whi, u.n_total, u.eps, s_limb, u.gamma, u.thr);
+        const uint32_t t_new = *u.thr;
+        const unsigned listed = atomicAdd(u.list_count, 0u);
+        const bool patch = hint && t_new >= t_lo && t_new <= t_hi && listed <= u.list_cap;
+        *u.mode = patch ? 1u : 2u;
+    }
+}
+
+// Pass 2 of the update: either the full pass (mode 2) or a patch of the listed
+// groups with the new threshold (mode 1; the mask and metadata do not depend on
+// the threshold, so only the group bytes and the values are rewritten).
+__global__ void __launch_bounds__(256) k_pack_finish(UpdateArgs u) {
+    const uint32_t mode = *u.mode;
+    const uint32_t thr = *u.thr;
+    const Pack24Args &p = u.p;
+    if (mode == 2u) {
+        const int lane = threadIdx.x & 31;
+        const int64_t warp_stride = static_cast<int64_t>(gridDim.x) * blockDim.x * kPackUnroll;
+        for (int64_t base = (static_cast<int64_t>(blockIdx.x) * blockDim.x + (threadIdx.x & ~31)) * kPackUnroll;
+             base < p.n_groups; base += warp_stride) {
+            float4 v[kPackUnroll];
+#pragma unroll
+            for (int q = 0; q < kPackUnroll; ++q) {
+                const int64_t i = base + 32 * q + lane;
+                v[q] = (i < p.n_groups) ? __ldg(p.W + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int q = 0; q < kPackUnroll; ++q) {
+                const int64_t i = base + 32 * q + lane;
+                pack_group(p, thr, lane, i, i < p.n_groups, v[q], 0u, 0u);
+            }
+        }
+        return;
+    }
+    const unsigned listed = *u.list_count;
+    for (unsigned j = blockIdx.x * blockDim.x + threadIdx.x; j < listed; j += gridDim.x * blockDim.x) {
+        const int64_t i = u.list[j];
+        const float4 v = __ldg(p.W + i);
+        patch_group(p, thr, i, v);
+    }
+}
+
+// ---------------------------------------------------------------- lane-quad kernels (k % 16 == 0)
+//
+// Leaner inner loop for the HBM-bound pass: each lane takes 4 consecutive
+// groups of one row (16 weights), so its group bytes, values, metadata nibbles
+// and mask bits leave as one 4-, 8-, 2- and 2-byte store, with no shuffles and
+// one row division per 4 groups.  The exact sum of |W| takes an fp64 fast
+// path: magnitudes in [2^-20, 2) are integer multiples of 2^-43, and up to
+// 2^10 / 2^-43 = 2^53 units (fewer than 512 of them) add exactly in fp64; the
+// per-lane fp64 sum is moved into the 128-bit integer accumulator (units of
+// 2^-54) once per round.  Zeros need no work; every other magnitude takes the
+// exact path of accumulate_abs.
+
+__device__ __forceinline__ bool fast_mag(uint32_t a) {
+    return a == 0u || (a - 0x35800000u) < (0x40000000u - 0x35800000u);   // 0 or [2^-20, 2)
+}
+
+__device__ __forceinline__ void sum_float4(const float4 v, double &d, uint64_t &lo, uint64_t &hi,
+                                           unsigned long long *s_bins, int *s_rare) {
+    const uint32_t a0 = __float_as_uint(v.x) & 0x7fffffffu, a1 = __float_as_uint(v.y) & 0x7fffffffu;
+    const uint32_t a2 = __float_as_uint(v.z) & 0x7fffffffu, a3 = __float_as_uint(v.w) & 0x7fffffffu;
+    if (fast_mag(a0) && fast_mag(a1) && fast_mag(a2) && fast_mag(a3)) {
+        d += static_cast<double>(__uint_as_float(a0));
+        d += static_cast<double>(__uint_as_float(a1));
+        d += static_cast<double>(__uint_as_float(a2));
+        d += static_cast<double>(__uint_as_float(a3));
+    } else {
+        accumulate_abs(a0, lo, hi, s_bins, s_rare);
+        accumulate_abs(a1, lo, hi, s_bins, s_rare);
+        accumulate_abs(a2, lo, hi, s_bins, s_rare);
+        accumulate_abs(a3, lo, hi, s_bins, s_rare);
+    }
+}
+
+// fp64 partial sum (a multiple of 2^-43 below 2^6) -> 128-bit accumulator
+__device__ __forceinline__ void flush_sum(double &d, uint64_t &lo, uint64_t &hi) {
+    const uint64_t q = __double2ull_rn(d * 0x1p43);   // exact: an integer below 2^49
+    add128(lo, hi, q << 11);
+    d = 0.0;
+}
+
+struct QuadOut {
+    uint32_t gb;      // 4 group bytes
+    uint32_t vlo, vhi;   // 8 int8 values
+    uint32_t meta;    // 4 nibbles in the low 16 bits
+    uint32_t mask;    // 4 keep nibbles in the low 16 bits
+    uint32_t band;    // bit j: group j has a kept magnitude in [band_lo, band_hi]
+};
+
+__device__ __forceinline__ void one_group(const float4 v, uint32_t thr, uint32_t band_lo, uint32_t band_hi,
+                                          uint32_t &gbyte, uint32_t &vals16, uint32_t &nib, uint32_t &keep,
+                                          uint32_t &in_band) {
+    const uint32_t b[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z), __float_as_uint(v.w)};
+    const uint32_t mag[4] = {b[0] & 0x7fffffffu, b[1] & 0x7fffffffu, b[2] & 0x7fffffffu, b[3] & 0x7fffffffu};
+    keep = top2_of_4(mag);
+    const uint32_t i0 = __ffs(keep) - 1, i1 = 31 - __clz(keep);
+    const uint32_t b0 = i0 == 0 ? b[0] : (i0 == 1 ? b[1] : b[2]);   // i0 <= 2
+    const uint32_t b1 = i1 == 3 ? b[3] : (i1 == 2 ? b[2] : b[1]);   // i1 >= 1
+    const uint32_t m0 = b0 & 0x7fffffffu, m1 = b1 & 0x7fffffffu;
+    const uint32_t nz0 = m0 >= thr, nz1 = m1 >= thr;
+    const uint32_t s0 = b0 >> 31, s1 = b1 >> 31;
+    const uint32_t c0 = nz0 ? (s0 ? 3u : 1u) : 0u, c1 = nz1 ? (s1 ? 3u : 1u) : 0u;
+    nib = i0 | (i1 << 2);
+    gbyte = nib | (c0 << 4) | (c1 << 6);
+    vals16 = (nz0 ? (s0 ? 0xffu : 0x01u) : 0u) | ((nz1 ? (s1 ? 0xffu : 0x01u) : 0u) << 8);
+    in_band = ((m0 >= band_lo && m0 <= band_hi) || (m1 >= band_lo && m1 <= band_hi)) ? 1u : 0u;
+}
+
+__device__ __forceinline__ QuadOut pack_quad(const float4 (&v)[4], uint32_t thr, uint32_t band_lo, uint32_t band_hi) {
+    QuadOut o;
+    o.gb = o.vlo = o.vhi = o.meta = o.mask = o.band = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        uint32_t gbyte, vals16, nib, keep, inb;
+        one_group(v[j], thr, band_lo, band_hi, gbyte, vals16, nib, keep, inb);
+        o.gb |= gbyte << (8 * j);
+        if (j < 2) o.vlo |= vals16 << (16 * j);
+        else o.vhi |= vals16 << (16 * (j - 2));
+        o.meta |= nib << (4 * j);
+        o.mask |= keep << (4 * j);
+        o.band |= inb << j;
+    }
+    return o;
+}
+
+// quad q (4 consecutive groups starting at group 4q) -> its layouts
+__device__ __forceinline__ void store_quad(const Pack24Args &p, uint32_t q, const QuadOut &o) {
+    const uint32_t i = 4u * q;
+    const uint32_t row = fastdiv(i, p.gpr_div);
+    const uint32_t g = i - row * static_cast<uint32_t>(p.gpr);
+    if (p.gb) *reinterpret_cast<uint32_t *>(p.gb + i) = o.gb;
+    if (p.vals) *reinterpret_cast<uint2 *>(p.vals + i) = make_uint2(o.vlo, o.vhi);
+    if (p.meta) {
+        const size_t off = ((static_cast<size_t>(g >> 5) * static_cast<size_t>(p.meta_rows) + row) << 4) + ((g & 31u) >> 1);
+        *reinterpret_cast<uint16_t *>(p.meta + off) = static_cast<uint16_t>(o.meta);
+    }
+    if (p.mask)
+        *reinterpret_cast<uint16_t *>(p.mask + ((static_cast<size_t>(row) * static_cast<size_t>(p.k)) >> 3) + (g >> 1)) =
+            static_cast<uint16_t>(o.mask);
+}
+
+constexpr int kQuadUnroll = 2;   // quads per lane per round (8 x 16-byte loads in flight)
+
+// pass 1 of bitnet_pack_nm: exact sum of |W| (fast path), last block finalises
+__global__ void __launch_bounds__(256, 4) k_abs_sum_fast(const float4 *__restrict__ W, int64_t n4,
+                                                         unsigned long long *__restrict__ win,
+                                                         unsigned long long *__restrict__ bins,
+                                                         unsigned *__restrict__ counter, int64_t n_total, float eps,
+                                                         float *__restrict__ gamma, uint32_t *__restrict__ thr) {
+    __shared__ unsigned long long s_bins[256];
+    __shared__ unsigned long long s_lo[8], s_hi[8];
+    __shared__ int s_rare;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0ull;
+    if (threadIdx.x == 0) s_rare = 0;
+    __syncthreads();
+    uint64_t lo = 0, hi = 0;
+    double d = 0.0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (; i + 7 * stride < n4; i += 8 * stride) {
+        float4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldg(W + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) sum_float4(v[u], d, lo, hi, s_bins, &s_rare);
+        flush_sum(d, lo, hi);
+    }
+    for (; i < n4; i += stride) sum_float4(__ldg(W + i), d, lo, hi, s_bins, &s_rare);
+    flush_sum(d, lo, hi);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+        const uint64_t h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+        const uint64_t sum = lo + l2;
+        hi = hi + h2 + ((sum < lo) ? 1ull : 0ull);
+        lo = sum;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        s_lo[warp] = lo;
+        s_hi[warp] = hi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint64_t L = 0, H = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            const uint64_t sum = L + s_lo[w];
+            H = H + s_hi[w] + ((sum < L) ? 1ull : 0ull);
+            L = sum;
+        }
+        if (L | H) {
+            const unsigned long long old = atomicAdd(&win[0], static_cast<unsigned long long>(L));
+            const uint64_t carry = (static_cast<uint64_t>(old) + L < static_cast<uint64_t>(old)) ? 1ull : 0ull;
+            atomicAdd(&win[1], static_cast<unsigned long long>(H + carry));
+        }
+    }
+    if (s_rare) {
+        for (int e = threadIdx.x; e < 256; e += blockDim.x)
+            if (s_bins[e]) atomicAdd(&bins[e], s_bins[e]);
+    }
+    __shared__ unsigned s_ticket;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_ticket = atomicAdd(counter, 1u);
+    __syncthreads();
+    if (s_ticket != gridDim.x - 1) return;
+    __threadfence();
+    __shared__ int s_nz[256];
+    __shared__ int s_nnz;
+    __shared__ uint32_t s_limb[kLimbs];
+    if (threadIdx.x == 0) s_nnz = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+        const unsigned long long b = atomicAdd(&bins[e], 0ull);
+        s_bins[e] = b;
+        if (b) s_nz[atomicAdd(&s_nnz, 1)] = e;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int a = 1; a < s_nnz; ++a)
+            for (int j = a; j > 0 && s_nz[j - 1] > s_nz[j]; --j) {
+                const int tmp = s_nz[j];
+                s_nz[j] = s_nz[j - 1];
+                s_nz[j - 1] = tmp;
+            }
+        const uint64_t wlo = atomicAdd(&win[0], 0ull), whi = atomicAdd(&win[1], 0ull);
+        finalize_gamma(s_bins, s_nz, s_nnz, wlo, whi, n_total, eps, s_limb, gamma, thr);
+    }
+}
+
+// pass 2 of bitnet_pack_nm (and the full pass of the update): lane quads
+__device__ __forceinline__ void quad_pass(const Pack24Args &p, uint32_t thr) {
+    const uint32_t n_quads = static_cast<uint32_t>(p.n_groups >> 2);
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t warps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t base = warp_global * 32u * kQuadUnroll; base < n_quads; base += warps * 32u * kQuadUnroll) {
+        float4 v[kQuadUnroll][4];
+#pragma unroll
+        for (int u = 0; u < kQuadUnroll; ++u) {
+            const uint32_t q = base + 32u * u + lane;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                v[u][j] = q < n_quads ? __ldg(p.W + 4u * q + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < kQuadUnroll; ++u) {
+            const uint32_t q = base + 32u * u + lane;
+            if (q < n_quads) store_quad(p, q, pack_quad(v[u], thr, 0u, 0u));
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) k_pack24_quad(Pack24Args p) { quad_pass(p, *p.thr); }
+
+// single-read update, lane quads: sum + layouts with the hint's threshold + band list
+__global__ void __launch_bounds__(256, 4) k_pack_update_quad(UpdateArgs u) {
+    __shared__ unsigned long long s_bins[256];
+    __shared__ unsigned long long s_lo[8], s_hi[8];
+    __shared__ int s_rare;
+    __shared__ uint32_t s_t, s_tlo, s_thi;
+    __shared__ int s_hint;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0ull;
+    if (threadIdx.x == 0) {
+        s_rare = 0;
+        const float gp = *u.gamma_prev;
+        s_hint = (gp > 0.0f && gp < 3.0e38f) ? 1 : 0;
+        s_t = s_tlo = s_thi = 0u;
+        if (s_hint) {
+            s_t = code_threshold(gp);
+            const float tf = __uint_as_float(s_t);
+            s_tlo = __float_as_uint(__fmul_rd(tf, 1.0f - 0x1p-10f));
+            s_thi = __float_as_uint(__fmul_ru(tf, 1.0f + 0x1p-10f));
+            if (blockIdx.x == 0) {
+                u.band[0] = s_tlo;
+                u.band[1] = s_thi;
+            }
+        }
+    }
+    __syncthreads();
+    const bool hint = s_hint != 0;
+    const uint32_t t_old = s_t, t_lo = s_tlo, t_hi = s_thi;
+    const Pack24Args &p = u.p;
+    const uint32_t n_quads = static_cast<uint32_t>(p.n_groups >> 2);
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t warps = (gridDim.x * blockDim.x) >> 5;
+    uint64_t lo = 0, hi = 0;
+    double d = 0.0;
+    for (uint32_t base = warp_global * 32u * kQuadUnroll; base < n_quads; base += warps * 32u * kQuadUnroll) {
+        float4 v[kQuadUnroll][4];
+#pragma unroll
+        for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
+            const uint32_t q = base + 32u * k2 + lane;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                v[k2][j] = q < n_quads ? __ldg(p.W + 4u * q + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
+            const uint32_t q = base + 32u * k2 + lane;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sum_float4(v[k2][j], d, lo, hi, s_bins, &s_rare);
+            if (hint && q < n_quads) {
+                const QuadOut o = pack_quad(v[k2], t_old, t_lo, t_hi);
+                store_quad(p, q, o);
+                if (o.band) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if ((o.band >> j) & 1u) {
+                            const unsigned slot = atomicAdd(u.list_count, 1u);
+                            if (slot < u.list_cap) u.list[slot] = 4u * q + j;
+                        }
+                }
+            }
+        }
+        flush_sum(d, lo, hi);
+    }
+    flush_sum(d, lo, hi);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+        const uint64_t h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+        const uint64_t sum = lo + l2;
+        hi = hi + h2 + ((sum < lo) ? 1ull : 0ull);
+        lo = sum;
+    }
+    const int warp = threadIdx.x >> 5;
+    if (lane == 0) {
+        s_lo[warp] = lo;
+        s_hi[warp] = hi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint64_t L = 0, H = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            const uint64_t sum = L + s_lo[w];
+            H = H + s_hi[w] + ((sum < L) ? 1ull : 0ull);
+            L = sum;
+        }
+        if (L | H) {
+            const unsigned long long old = atomicAdd(&u.win[0], static_cast<unsigned long long>(L));
+            const uint64_t carry = (static_cast<uint64_t>(old) + L < static_cast<uint64_t>(old)) ? 1ull : 0ull;
+            atomicAdd(&u.win[1], static_cast<unsigned long long>(H + carry));
+        }
+    }
+    if (s_rare) {
+        for (int e = threadIdx.x; e < 256; e += blockDim.x)
+            if (s_bins[e]) atomicAdd(&u.bins[e], s_bins[e]);
+    }
+    __shared__ unsigned s_ticket;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_ticket = atomicAdd(u.counter, 1u);
+    __syncthreads();
+    if (s_ticket != gridDim.x - 1) return;
+    __threadfence();
+    __shared__ int s_nz[256];
+    __shared__ int s_nnz;
+    __shared__ uint32_t s_limb[kLimbs];
+    if (threadIdx.x == 0) s_nnz = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+        const unsigned long long b = atomicAdd(&u.bins[e], 0ull);
+        s_bins[e] = b;
+        if (b) s_nz[atomicAdd(&s_nnz, 1)] = e;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int a = 1; a < s_nnz; ++a)
+            for (int j = a; j > 0 && s_nz[j - 1] > s_nz[j]; --j) {
+                const int tmp = s_nz[j];
+                s_nz[j] = s_nz[j - 1];
+                s_nz[j - 1] = tmp;
+            }
+        const uint64_t wlo = atomicAdd(&u.win[0], 0ull), whi = atomicAdd(&u.win[1], 0ull);
+        finalize_gamma(s_bins, s_nz, s_nnz, wlo, whi, u.n_total, u.eps, s_limb, u.gamma, u.thr);
+        const uint32_t t_new = *u.thr;
+        const unsigned listed = atomicAdd(u.list_count, 0u);
+        const bool patch = hint && t_new >= t_lo && t_new <= t_hi && listed <= u.list_cap;
+        *u.mode = patch ? 1u : 2u;
+    }
+}
+
+__global__ void __launch_bounds__(256) k_pack_finish_quad(UpdateArgs u) {
+    const uint32_t mode = *u.mode;
+    const uint32_t thr = *u.thr;
+    if (mode == 2u) {
+        quad_pass(u.p, thr);
+        return;
+    }
+    const unsigned listed = *u.list_count;
+    for (unsigned j = blockIdx.x * blockDim.x + threadIdx.x; j < listed; j += gridDim.x * blockDim.x) {
+        const int64_t i = u.list[j];
+        patch_group(u.p, thr, i, __ldg(u.p.W + i));
     }
 }
 
@@ -412,14 +1058,16 @@ cudaError_t launch_pack(const float *W, int64_t n_out, int64_t k, int n, int m, 
     cudaError_t err = cudaMemsetAsync(ws, 0, kPackWsBytes, s);
     if (err != cudaSuccess) return err;
     const int64_t n_el = n_out * k;
-    k_abs_sum<<<grid_for(n_el / 4, 256, 8), 256, 0, s>>>(reinterpret_cast<const float4 *>(W), n_el / 4, win, bins);
-    k_finalize_gamma<<<1, 32, 0, s>>>(win, bins, n_el, eps, gamma, thr);
+    unsigned *counter = reinterpret_cast<unsigned *>(w8 + kPackWsCounterOffset);
+    k_abs_sum_fast<<<grid_for(n_el / 4, 256, 4), 256, 0, s>>>(reinterpret_cast<const float4 *>(W), n_el / 4, win,
+                                                             bins, counter, n_el, eps, gamma, thr);
     const bool packed = gb || vals || meta || dec;
     if (packed) {
         Pack24Args a;
         a.W = reinterpret_cast<const float4 *>(W);
         a.n_groups = n_el / 4;
         a.gpr = k / 4;
+        a.gpr_div = make_fastdiv(static_cast<uint32_t>(k / 4));
         a.n_out = n_out;
         a.k = k;
         a.meta_rows = (n_out + 127) / 128 * 128;
@@ -428,7 +1076,10 @@ cudaError_t launch_pack(const float *W, int64_t n_out, int64_t k, int n, int m, 
         a.vals = reinterpret_cast<uint16_t *>(vals);
         a.meta = meta;
         a.mask = (n == 2 && m == 4) ? mask : nullptr;
-        k_pack24<<<grid_for(a.n_groups, 256, 8), 256, 0, s>>>(a);
+        if (k % 16 == 0)
+            k_pack24_quad<<<grid_for((a.n_groups / 4 + kQuadUnroll - 1) / kQuadUnroll, 256, 8), 256, 0, s>>>(a);
+        else
+            k_pack24<<<grid_for((a.n_groups + kPackUnroll - 1) / kPackUnroll, 256, 8), 256, 0, s>>>(a);
         if (meta && (a.meta_rows != n_out || (k % 128) != 0))
             k_meta_pad<<<grid_for(((k + 127) / 128) * (a.meta_rows - n_out) * 16 + n_out * 16, 256, 4), 256, 0, s>>>(
                 meta, n_out, k, a.meta_rows);
@@ -440,6 +1091,57 @@ cudaError_t launch_pack(const float *W, int64_t n_out, int64_t k, int n, int m, 
         const int64_t groups = n_el / m;
         k_mask_nm<<<grid_for(groups, 256, 8), 256, 0, s>>>(W, groups, n, m, mask);
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_pack_update(const float *W, int64_t n_out, int64_t k, float eps, float *gamma, uint8_t *gb,
+                               int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws, size_t ws_bytes,
+                               cudaStream_t s) {
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    cudaError_t err = cudaMemsetAsync(ws, 0, kPackWsBytes, s);
+    if (err != cudaSuccess) return err;
+    const int64_t n_el = n_out * k;
+    UpdateArgs u;
+    u.p.W = reinterpret_cast<const float4 *>(W);
+    u.p.n_groups = n_el / 4;
+    u.p.gpr = k / 4;
+    u.p.gpr_div = make_fastdiv(static_cast<uint32_t>(k / 4));
+    u.p.n_out = n_out;
+    u.p.k = k;
+    u.p.meta_rows = (n_out + 127) / 128 * 128;
+    u.p.thr = nullptr;
+    u.p.gb = gb;
+    u.p.vals = reinterpret_cast<uint16_t *>(vals);
+    u.p.meta = meta;
+    u.p.mask = mask;
+    u.gamma_prev = gamma;
+    u.gamma = gamma;
+    u.win = reinterpret_cast<unsigned long long *>(w8 + kPackWsWinOffset);
+    u.bins = reinterpret_cast<unsigned long long *>(w8 + kPackWsBinsOffset);
+    u.counter = reinterpret_cast<unsigned *>(w8 + kPackWsCounterOffset);
+    u.thr = reinterpret_cast<uint32_t *>(w8 + kPackWsThrOffset);
+    u.mode = reinterpret_cast<uint32_t *>(w8 + kPackWsModeOffset);
+    u.band = reinterpret_cast<uint32_t *>(w8 + kPackWsBandOffset);
+    u.list_count = reinterpret_cast<unsigned *>(w8 + kPackWsListCountOffset);
+    u.list = reinterpret_cast<uint32_t *>(w8 + kPackWsBytes);
+    u.list_cap = static_cast<uint32_t>((ws_bytes - kPackWsBytes) / 4);
+    u.n_total = n_el;
+    u.eps = eps;
+    if (k % 16 == 0) {
+        const unsigned grid = grid_for((u.p.n_groups / 4 + kQuadUnroll - 1) / kQuadUnroll, 256, 4);
+        k_pack_update_quad<<<grid, 256, 0, s>>>(u);
+        k_pack_finish_quad<<<grid, 256, 0, s>>>(u);
+    } else {
+        const unsigned grid = grid_for((u.p.n_groups + kPackUnroll - 1) / kPackUnroll, 256, 4);
+        k_pack_update<<<grid, 256, 0, s>>>(u);
+        k_pack_finish<<<grid, 256, 0, s>>>(u);
+    }
+    if (meta && (u.p.meta_rows != n_out || (k % 128) != 0))
+        k_meta_pad<<<grid_for(((k + 127) / 128) * (u.p.meta_rows - n_out) * 16 + n_out * 16, 256, 4), 256, 0, s>>>(
+            meta, n_out, k, u.p.meta_rows);
+    if (dec)
+        k_make_dec<<<grid_for(n_out / 16 * (k / 64) * 32, 256, 8), 256, 0, s>>>(gb, n_out, k,
+                                                                                reinterpret_cast<uint2 *>(dec));
     return cudaGetLastError();
 }
 

@@ -63,6 +63,9 @@ __global__ void __launch_bounds__(kQuantThreads) k_quant_act(const uint4 *__rest
     C reg[kQuantMaxChunks];
     float m = 0.0f;
     const bool fits = nchunk <= static_cast<int64_t>(kQuantMaxChunks) * kQuantThreads;
+    // X may be the output of the previous kernel of the stream
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #pragma unroll
     for (int u = 0; u < kQuantMaxChunks; ++u) {
         const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
@@ -120,13 +123,20 @@ __global__ void __launch_bounds__(kQuantThreads) k_quant_act(const uint4 *__rest
 cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xq, float *amax,
                              cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
-    if (bf16)
-        k_quant_act<true><<<static_cast<unsigned>(T), kQuantThreads, 0, s>>>(static_cast<const uint4 *>(X), K, eps,
-                                                                            Xq, amax);
-    else
-        k_quant_act<false><<<static_cast<unsigned>(T), kQuantThreads, 0, s>>>(static_cast<const uint4 *>(X), K,
-                                                                             eps, Xq, amax);
-    return cudaGetLastError();
+    // programmatic serialisation: the kernel that consumes Xq may start its own
+    // independent loads while this one runs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(T));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const uint4 *x = static_cast<const uint4 *>(X);
+    if (bf16) return cudaLaunchKernelEx(&cfg, k_quant_act<true>, x, K, eps, Xq, amax);
+    return cudaLaunchKernelEx(&cfg, k_quant_act<false>, x, K, eps, Xq, amax);
 }
 
 }  // namespace bitnet

@@ -386,3 +386,65 @@ def test_quant_linear_chain_in_graph(bn):
     for l in range(layers):
         x = oracle.forward(Ws[l], x, 1e-5, 1e-5)["y"]
         assert np.array_equal(xs[l + 1].cpu().numpy(), x), l
+
+
+# ------------------------------------------------------------------ per-step pack with the previous gamma as hint
+
+def _pack_outputs(pw, mask):
+    return [pw.gamma.cpu().numpy().copy(), pw.group_bytes.cpu().numpy().copy(), pw.mma_vals.cpu().numpy().copy(),
+            pw.mma_meta.cpu().numpy().copy(), mask.cpu().numpy().copy(),
+            pw.dec_codes.cpu().numpy().copy() if pw.dec_codes is not None else None]
+
+
+@pytest.mark.parametrize("n_out,k", [(256, 512), (200, 352), (3200, 3200)])
+def test_pack_update_matches_pack_over_steps(bn, n_out, k):
+    """Random-walk steps W += N(0, 1e-4) (patch mode), a large jump (full
+    second pass), and the first call without a hint: every step bit-identical
+    to bitnet_pack_nm and to the oracle."""
+    W = synth.master_weights(n_out, k, 0.02, seed=900)
+    Wd = dev_f32(W)
+    upd = bn.PackedWeights(n_out, k)          # gamma starts at 0: no hint on the first call
+    mask_u = torch.zeros(n_out * k // 8, dtype=torch.uint8, device="cuda")
+    ws = bn.Workspace(bn.load().bitnet_pack_update_workspace_size(n_out, k))
+    for step in range(6):
+        if step > 0:
+            scale = 1e-4 if step != 4 else 5e-3   # step 4 moves gamma far outside the band
+            W = synth.random_walk_step(W, scale, seed=step)
+            Wd.copy_(dev_f32(W))
+        bn.bitnet_pack_nm_update(Wd, upd, 1e-5, mask_bits=mask_u, ws=ws)
+        ref = bn.PackedWeights(n_out, k)
+        mask_r = torch.zeros_like(mask_u)
+        bn.bitnet_pack_nm(Wd, ref, 1e-5, mask_bits=mask_r)
+        torch.cuda.synchronize()
+        for a, b in zip(_pack_outputs(upd, mask_u), _pack_outputs(ref, mask_r)):
+            assert (a is None and b is None) or np.array_equal(a, b), step
+        g, keep, wq, gb = oracle.pack_weights(W, 1e-5)
+        assert upd.gamma.item() == float(g) and np.array_equal(upd.group_bytes.cpu().numpy(), gb)
+
+
+def test_pack_update_small_list_falls_back(bn):
+    """A list with room for one entry overflows; the device then runs the full
+    second pass and the result is still exact."""
+    n_out, k = 512, 512
+    W = synth.master_weights(n_out, k, 0.02, seed=901)
+    pw = bn.PackedWeights(n_out, k)
+    bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5)
+    W2 = synth.random_walk_step(W, 1e-4, seed=3)
+    tiny = bn.Workspace(bn.load().bitnet_pack_workspace_size(n_out, k) + 4)
+    bn.bitnet_pack_nm_update(dev_f32(W2), pw, 1e-5, ws=tiny)
+    torch.cuda.synchronize()
+    g, keep, wq, gb = oracle.pack_weights(W2, 1e-5)
+    assert pw.gamma.item() == float(g)
+    assert np.array_equal(pw.group_bytes.cpu().numpy(), gb)
+    dwq, dkeep, _, _ = decode_mma(pw.mma_vals.cpu().numpy(), pw.mma_meta.cpu().numpy(), n_out, k)
+    assert np.array_equal(dwq, wq)
+
+
+@pytest.mark.parametrize("n_out,k,T", [(200, 352, 300), (136, 256, 500), (128, 8640, 229), (2560, 2560, 448),
+                                       (256, 1024, 1000)])
+def test_gemm_pair_kernel_ragged(bn, n_out, k, T):
+    """T > 128 runs the persistent CTA-pair kernel: ragged last 256-row pair
+    (including a second CTA entirely past n_out), ragged 224-token tiles,
+    k % 128 != 0, several tiles per pair."""
+    ref, acc, Y = _linear_case(bn, n_out, k, T, seed=n_out * 7 + T)
+    _check_outputs(ref, acc, Y)
