@@ -345,29 +345,61 @@ cudaError_t launch_gemm_sp(const int8_t *Xq, const float *amax, const float *gam
 }
 
 // Wq^T in bf16: wt[k, n] = code of weight (n, k), from the canonical group bytes.
+// One CTA per 64 (n) x 64 (k) tile: 64 rows of 16 group bytes come in with one
+// 16-byte load each, and the transposed tile leaves in 16-byte stores (8 bf16),
+// so both the 0.25-byte reads and the 2-byte writes per weight are coalesced.
 __global__ void __launch_bounds__(256) k_expand_wt(const uint8_t *__restrict__ gb, int64_t n_out, int64_t k,
                                                    __nv_bfloat16 *__restrict__ wt) {
-    // 32 x 32 tiles through shared memory: read rows of group bytes, write
-    // columns of the transpose.
-    __shared__ __nv_bfloat16 tile[32][33];
-    const int64_t kb = static_cast<int64_t>(blockIdx.x) * 32, nb = static_cast<int64_t>(blockIdx.y) * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 8 rows per pass
-    for (int r = ty; r < 32; r += 8) {
-        const int64_t n = nb + r, kk = kb + tx;
-        float v = 0.0f;
-        if (n < n_out && kk < k) {
-            const uint32_t b = gb[n * (k / 4) + (kk >> 2)];
-            const uint32_t pos = static_cast<uint32_t>(kk & 3);
-            const uint32_t i0 = b & 3u, i1 = (b >> 2) & 3u;
-            const uint32_t c = (pos == i0) ? ((b >> 4) & 3u) : ((pos == i1) ? ((b >> 6) & 3u) : 0u);
-            v = c == 1u ? 1.0f : (c == 3u ? -1.0f : 0.0f);
+    __shared__ __align__(16) uint8_t s_gb[64][16];
+    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 64, k0 = static_cast<int64_t>(blockIdx.x) * 64;
+    const int64_t gpr = k / 4;
+    const int tid = threadIdx.x;
+    if (tid < 64) {
+        const int64_t n = n0 + tid;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (n < n_out) {
+            const uint8_t *src = gb + n * gpr + k0 / 4;
+            if (k0 + 64 <= k && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+                v = __ldg(reinterpret_cast<const uint4 *>(src));
+            } else {
+                uint8_t tmp[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) tmp[j] = (k0 + 4 * j < k) ? src[j] : static_cast<uint8_t>(0x04);
+                v = *reinterpret_cast<const uint4 *>(tmp);
+            }
         }
-        tile[r][tx] = __float2bfloat16_rn(v);
+        *reinterpret_cast<uint4 *>(s_gb[tid]) = v;
     }
     __syncthreads();
-    for (int r = ty; r < 32; r += 8) {
-        const int64_t kk = kb + r, n = nb + tx;
-        if (kk < k && n < n_out) wt[kk * n_out + n] = tile[tx][r];
+    // thread (r, c): output row k0 + r, columns n0 + 16c .. +15
+    const int r = tid >> 2, c = tid & 3;
+    const int64_t kk = k0 + r;
+    if (kk >= k) return;
+    const int grp = r >> 2, pos = r & 3;
+    uint32_t h[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        uint32_t pair = 0;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const uint32_t b = s_gb[16 * c + 2 * j + e][grp];
+            const uint32_t i0 = b & 3u, i1 = (b >> 2) & 3u;
+            const uint32_t code = (static_cast<uint32_t>(pos) == i0) ? ((b >> 4) & 3u)
+                                  : (static_cast<uint32_t>(pos) == i1) ? ((b >> 6) & 3u) : 0u;
+            // bf16 bits: +1 = 0x3f80, -1 = 0xbf80, 0 = 0
+            const uint32_t bits = code == 1u ? 0x3f80u : (code == 3u ? 0xbf80u : 0u);
+            pair |= bits << (16 * e);
+        }
+        h[j] = pair;
+    }
+    const int64_t nb = n0 + 16 * c;
+    __nv_bfloat16 *dst = wt + kk * n_out + nb;
+    if (nb + 16 <= n_out && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+        reinterpret_cast<uint4 *>(dst)[0] = make_uint4(h[0], h[1], h[2], h[3]);
+        reinterpret_cast<uint4 *>(dst)[1] = make_uint4(h[4], h[5], h[6], h[7]);
+    } else {
+        for (int j = 0; j < 16; ++j)
+            if (nb + j < n_out) reinterpret_cast<uint16_t *>(dst)[j] = static_cast<uint16_t>(h[j >> 1] >> (16 * (j & 1)));
     }
 }
 
@@ -375,7 +407,7 @@ cudaError_t launch_dgrad(const void *dY, const float *gamma, const uint8_t *gb, 
                          void *dX, bool dx_bf16, void *ws, cudaStream_t s) {
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     __nv_bfloat16 *wt = reinterpret_cast<__nv_bfloat16 *>(w8 + kDgradWsHeader);
-    dim3 eg(static_cast<unsigned>((k + 31) / 32), static_cast<unsigned>((n_out + 31) / 32));
+    dim3 eg(static_cast<unsigned>((k + 63) / 64), static_cast<unsigned>((n_out + 63) / 64));
     k_expand_wt<<<eg, 256, 0, s>>>(gb, n_out, k, wt);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

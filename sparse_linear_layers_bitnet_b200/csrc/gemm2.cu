@@ -63,6 +63,17 @@ __device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap *map, uint64_
         : "memory");
 }
 
+// TMA tiled store shared -> global (bulk group), and its bookkeeping
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void *src, int32_t c0, int32_t c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(map),
+                 "r"(smem_u32(src)), "r"(c0), "r"(c1)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ void tmem_alloc2(uint32_t *dst, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
                  : "memory");
@@ -125,7 +136,8 @@ struct PairCfg {
     static constexpr int kAccStride = 256;                // TMEM columns between the two accumulators
     static constexpr int kECol = 2 * kAccStride - 16;     // metadata columns (8 used)
     static constexpr int kTmemCols = 512;
-    static constexpr int kSmemBytes = STAGES * kStageBytes + 1024 + 2048;
+    static constexpr int kStageOutBytes = SPARSE ? 2 * 16 * 128 * 4 : 0;   // two [16 tokens][128 rows] fp32 chunks
+    static constexpr int kSmemBytes = STAGES * kStageBytes + kStageOutBytes + 1024 + 2048;
     // M = 256 (two CTAs), N = BN
     static constexpr uint32_t kIdesc = (SPARSE ? (1u << 2) : 0u) | ((SPARSE ? 2u : 1u) << 4) | (1u << 7) |
                                        (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
@@ -137,6 +149,7 @@ struct PairCfg {
 
 struct PairParams {
     int64_t M, N, K;
+    int tma_store;               // sparse: output chunks leave through TMA stores
     int64_t meta_rows;           // sparse: rows of one metadata k-block
     const float *gamma;
     const float *amax;           // sparse: per-token scale
@@ -149,14 +162,15 @@ struct PairParams {
 template <bool SPARSE, int BN, int STAGES>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     k_umma_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmE, PairParams p) {
+                const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY, PairParams p) {
     using C = PairCfg<SPARSE, BN, STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
     uint8_t *sB = sA + STAGES * C::kABytes;
     uint8_t *sE = sB + STAGES * C::kBBytes;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sE + STAGES * C::kEBytes);
+    uint8_t *sOut = sE + STAGES * C::kEBytes;   // output staging (sparse)
+    uint64_t *full = reinterpret_cast<uint64_t *>(sOut + C::kStageOutBytes);
     uint64_t *empty = full + STAGES;
     uint64_t *acc_full = empty + STAGES;       // [2]
     uint64_t *acc_empty = acc_full + 2;        // [2], leader: one arrival per CTA
@@ -219,7 +233,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                         pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * (C::kKStep / 2), a_row);
                         pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
                         pair::tma_load_2d_pair(&tmE, &full[s], sE + s * C::kEBytes, 0,
-                                               static_cast<int32_t>(kt * p.meta_rows + e_row));
+                                               static_cast<int32_t>((kt * p.meta_rows + e_row) / 8));
                     } else {
                         pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * C::kKStep, a_row);
                         pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
@@ -272,6 +286,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         const int quarter = warp & 3;
         const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
         int local = 0;
+        int chunk_count = 0;   // output chunks staged so far (TMA-store double buffer)
         for (int64_t t = pair_id; t < tiles; t += pairs, ++local) {
             const int b = local & 1;
             const int64_t mt = t / n_tiles, nt = t - mt * n_tiles;
@@ -296,6 +311,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     uint32_t r[16];
                     tmem_ld_32x32b_x16(taddr + 16 * c, r);
                     tmem_ld_wait();
+                    if (SPARSE && p.tma_store) {
+                        // stage [16 tokens][128 rows] and send it with one TMA store
+                        const int buf = chunk_count & 1;
+                        uint8_t *stg = sOut + buf * (16 * 128 * 4);
+                        if (chunk_count >= 2) {
+                            if (threadIdx.x == 64) pair::bulk_wait_read1();   // the store of 2 chunks ago has read this buffer
+                            asm volatile("bar.sync 1, 128;" ::: "memory");
+                        }
+                        const int row = 32 * quarter + lane;
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const float y = __fmul_rn(__int2float_rn(static_cast<int>(r[j])), s_scale[16 * c + j]);
+                            if (p.out_bf16)
+                                reinterpret_cast<__nv_bfloat16 *>(stg)[j * 128 + row] = __float2bfloat16_rn(y);
+                            else
+                                reinterpret_cast<float *>(stg)[j * 128 + row] = y;
+                        }
+                        pair::fence_async_shared();
+                        asm volatile("bar.sync 1, 128;" ::: "memory");
+                        if (threadIdx.x == 64 && m0 < p.M && n0 + 16 * c < p.N) {
+                            pair::tma_store_2d(&tmY, stg, static_cast<int32_t>(m0), static_cast<int32_t>(n0 + 16 * c));
+                            pair::bulk_commit();
+                        }
+                        ++chunk_count;
+                        if (p.acc_out && m < p.M) {
+#pragma unroll
+                            for (int j = 0; j < 16; ++j) {
+                                const int64_t tok = n0 + 16 * c + j;
+                                if (tok < p.N) p.acc_out[tok * p.M + m] = static_cast<int>(r[j]);
+                            }
+                        }
+                        continue;
+                    }
                     if (m >= p.M) continue;
                     if (SPARSE) {
 #pragma unroll
@@ -358,6 +406,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             if (!ok) break;
         }
     }
+    if (SPARSE && p.tma_store && threadIdx.x == 64) pair::bulk_wait_all();   // stores have left shared memory
     tc_fence_before();
     __syncthreads();
     pair::cluster_sync();   // no CTA leaves while its peer may still signal it
@@ -399,8 +448,8 @@ static bool map2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, ui
 }
 
 template <bool SPARSE, int BN, int STAGES>
-static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &e, const PairParams &p,
-                            cudaStream_t s) {
+static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &e, const CUtensorMap &y,
+                            const PairParams &p, cudaStream_t s) {
     using C = PairCfg<SPARSE, BN, STAGES>;
     auto kern = k_umma_pair<SPARSE, BN, STAGES>;
     static bool attr_set = false;
@@ -413,13 +462,15 @@ static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CU
     int64_t pairs = num_sms() / 2;
     if (pairs > tiles) pairs = tiles;
     if (pairs < 1) pairs = 1;
-    kern<<<dim3(static_cast<unsigned>(2 * pairs)), 192, C::kSmemBytes, s>>>(a, b, e, p);
+    kern<<<dim3(static_cast<unsigned>(2 * pairs)), 192, C::kSmemBytes, s>>>(a, b, e, y, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_sp_pair(const int8_t *Xq, const float *amax, const float *gamma, const int8_t *vals,
                                 const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16,
                                 int32_t *acc, uint32_t *status, cudaStream_t s) {
+    // N = 224: two accumulators (2 x 224 columns) and the metadata fit in TMEM.
+    // (Narrower tiles cut wave quantisation but cost more per tile; measured slower.)
     constexpr int BN = 224;
     PairParams p{};
     p.M = n_out;
@@ -437,12 +488,23 @@ cudaError_t launch_gemm_sp_pair(const int8_t *Xq, const float *amax, const float
                static_cast<uint64_t>(k / 2), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     if (!map2d(&mb, CU_TENSOR_MAP_DATA_TYPE_UINT8, Xq, static_cast<uint64_t>(k), static_cast<uint64_t>(T),
-               static_cast<uint64_t>(k), 128, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+               static_cast<uint64_t>(k), 128, static_cast<uint32_t>(BN / 2), CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
+    // metadata as rows of 128 bytes: one k-step of a 128-row tile is 16 such rows (2 KB, contiguous)
     const uint64_t meta_total_rows = static_cast<uint64_t>((k + 127) / 128) * static_cast<uint64_t>(p.meta_rows);
-    if (!map2d(&me, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, 16, meta_total_rows, 16, 16, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!map2d(&me, CU_TENSOR_MAP_DATA_TYPE_UINT8, meta, 128, meta_total_rows / 8, 128, 128, 16,
+               CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    return run_pair<true, BN, 8>(ma, mb, me, p, s);
+    // output through TMA stores when the row pitch allows it (16-byte multiple)
+    CUtensorMap my = ma;
+    const size_t esz = y_bf16 ? 2 : 4;
+    p.tma_store = (static_cast<size_t>(n_out) * esz) % 16 == 0;
+    if (p.tma_store &&
+        !map2d(&my, y_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y,
+               static_cast<uint64_t>(n_out), static_cast<uint64_t>(T), static_cast<uint64_t>(n_out) * esz, 128, 16,
+               CU_TENSOR_MAP_SWIZZLE_NONE))
+        return cudaErrorInvalidValue;
+    return run_pair<true, BN, 8>(ma, mb, me, my, p, s);
 }
 
 cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *wt, const float *gamma, int64_t T,
@@ -461,9 +523,9 @@ cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *wt, const
                static_cast<uint64_t>(n_out) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     if (!map2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wt, static_cast<uint64_t>(n_out), static_cast<uint64_t>(k),
-               static_cast<uint64_t>(n_out) * 2, 64, BN / 2, CU_TENSOR_MAP_SWIZZLE_128B))
+               static_cast<uint64_t>(n_out) * 2, 64, static_cast<uint32_t>(BN / 2), CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    return run_pair<false, BN, 6>(ma, mb, ma, p, s);
+    return run_pair<false, BN, 6>(ma, mb, ma, ma, p, s);
 }
 
 }  // namespace bitnet

@@ -22,8 +22,11 @@
 
 namespace bitnet {
 
-constexpr int kDecWarps = 4;
 constexpr int kDecRegTiles = 16;   // k-tiles (8 bytes each) prefetched per lane per round
+
+// Warps per CTA so that one prefetch round holds every k-tile of a warp
+// (K <= 4096: 4 warps; K <= 8192: 8 warps; beyond, several rounds).
+inline int gemv_warps(int64_t k) { return (k / 64 + 3) / 4 <= kDecRegTiles ? 4 : 8; }
 
 // int8 code of one activation: clamp(rint(fp32(x * s)), -127, 127)
 __device__ __forceinline__ int8_t quant_code(float x, float s) {
@@ -47,6 +50,7 @@ __device__ __forceinline__ void mma_sp_m16n8k64(int (&d)[4], const uint32_t (&a)
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]), "r"(b[2]), "r"(b[3]), "r"(e));
 }
 
+template <int kDecWarps>
 __global__ void __launch_bounds__(kDecWarps * 32) k_gemv_dec(const uint2 *__restrict__ dec,
                                                               const int8_t *__restrict__ Xq,
                                                               const float *__restrict__ amax,
@@ -378,17 +382,22 @@ cudaError_t launch_gemv_fused(const void *X, bool x_bf16, float eps, const float
 cudaError_t launch_gemv_dec(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *dec,
                             int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                             cudaStream_t s) {
+    const int warps = gemv_warps(k);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_out / 16));
-    cfg.blockDim = dim3(kDecWarps * 32);
+    cfg.blockDim = dim3(warps * 32);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, k_gemv_dec, reinterpret_cast<const uint2 *>(dec), Xq, amax, gamma,
-                              static_cast<int>(T), n_out, k, Y, y_bf16 ? 1 : 0, acc);
+    const uint2 *d2 = reinterpret_cast<const uint2 *>(dec);
+    if (warps == 4)
+        return cudaLaunchKernelEx(&cfg, k_gemv_dec<4>, d2, Xq, amax, gamma, static_cast<int>(T), n_out, k, Y,
+                                  y_bf16 ? 1 : 0, acc);
+    return cudaLaunchKernelEx(&cfg, k_gemv_dec<8>, d2, Xq, amax, gamma, static_cast<int>(T), n_out, k, Y,
+                              y_bf16 ? 1 : 0, acc);
 }
 
 cudaError_t launch_gemv_gb(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *gb,

@@ -448,3 +448,27 @@ def test_gemm_pair_kernel_ragged(bn, n_out, k, T):
     k % 128 != 0, several tiles per pair."""
     ref, acc, Y = _linear_case(bn, n_out, k, T, seed=n_out * 7 + T)
     _check_outputs(ref, acc, Y)
+
+
+@pytest.mark.parametrize("n_out,k,T", [(4096, 256, 896), (2048, 256, 1344), (256, 512, 160)])
+def test_gemm_pair_tile_widths(bn, n_out, k, T):
+    """Larger pair-kernel shapes: many 256 x 224 tiles per CTA pair, ragged
+    last token tile."""
+    ref, acc, Y = _linear_case(bn, n_out, k, T, seed=n_out + T, y_dtype="bf16")
+    _check_outputs(ref, acc, Y)
+
+
+@pytest.mark.parametrize("T,n_out,k", [(512, 256, 8192), (256, 512, 256)])
+def test_dgrad_pair_tile_widths(bn, T, n_out, k):
+    """dgrad through the pair kernel: wide output (k = 8192, many tiles per
+    pair) and a single tile."""
+    W = synth.master_weights(n_out, k, 0.02, seed=T + n_out)
+    g, keep, wq, gb = oracle.pack_weights(W, 1e-5)
+    pw = bn.PackedWeights(n_out, k, mma=False, dec=False)
+    bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5)
+    dYd, dY32 = bf16_dev(synth.activations(T, n_out, seed=T + 1))
+    dX = bn.bitnet_dgrad(dYd, pw, dx_dtype=torch.float32)
+    torch.cuda.synchronize()
+    ref, absref = oracle.dgrad(dY32, wq, g)
+    tol = 2 * n_out * 2.0 ** -24 * absref + 1e-30
+    assert np.all(np.abs(dX.cpu().numpy().astype(np.float64) - ref) <= tol)
