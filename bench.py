@@ -55,6 +55,9 @@ def parse_args():
     ap.add_argument("--preroll-s", type=float, default=1.0, help="untimed warm-up seconds before timing")
     ap.add_argument("--tokens", type=int, default=1, help="decode batch (1..8)")
     ap.add_argument("--layers", type=int, default=30)
+    ap.add_argument("--decode", choices=["chain", "fused", "unfused"], default="unfused",
+                    help="decode step: one persistent launch for all projections (chain), one fused "
+                         "quant+GEMV launch per projection (fused), or quant_act + GEMV per projection")
     ap.add_argument("--no-rows", action="store_true", help="skip the sub-measurements of the other rows")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--pack-layers", type=int, default=None, help="layers of the pack workload (default: all 26)")
@@ -205,8 +208,10 @@ def decode_bytes_fused(T, K, N):
 
 
 class Decode:
-    def __init__(self, torch, bn, synth, T, layers, seed_base=0, fused=True):
-        self.torch, self.bn, self.T, self.L, self.fused = torch, bn, T, layers, fused
+    def __init__(self, torch, bn, synth, T, layers, seed_base=0, mode="chain"):
+        self.torch, self.bn, self.T, self.L, self.mode = torch, bn, T, layers, mode
+        fused = mode in ("chain", "chain_independent", "fused")
+        self.fused = fused
         dev = torch.device("cuda", torch.cuda.current_device())
         self.mats = decode_shapes()
         self.packed = []
@@ -254,9 +259,21 @@ class Decode:
         self.step_bytes = (self.fused_bytes_per_layer if fused else q + g) * layers
         self.weight_bytes = sum(N * K // 4 for _, K, N in self.mats) * layers
         self.launches_per_step = (1 if fused else 2) * len(self.mats) * layers
+        self.chain = None
+        if mode in ("chain", "chain_independent"):
+            # chain: the decode pass, every projection waits for the previous one;
+            # chain_independent: the same projections without the waits (each has its own input)
+            wait = 1 if mode == "chain" else 0
+            ops = [dict(X=self.x_views[l][j], W=self.packed[l][j], Y=self.y_views[l][j], wait_prev=wait)
+                   for l in range(layers) for j in range(len(self.mats))]
+            self.chain = bn.DecodeChain(ops, torch.bfloat16, torch.bfloat16, 1e-5, dev)
+            self.launches_per_step = (len(ops) + 127) // 128
 
     def step(self):
         bn = self.bn
+        if self.chain is not None:
+            self.chain()
+            return
         for l in range(self.L):
             for j in range(len(self.mats)):
                 if self.fused:
@@ -567,7 +584,8 @@ def run_ours(args):
     assert 1 <= T <= 8, "decode batch must be 1..8"
     dev_index = torch.cuda.current_device()
 
-    dec = Decode(torch, bn, synth, T, args.layers, seed_base=info.rank * 7919, fused=False)
+    fused = args.decode in ("chain", "fused")
+    dec = Decode(torch, bn, synth, T, args.layers, seed_base=info.rank * 7919, mode=args.decode)
     g_step = dec.capture(dec.step)
 
     clocks = ClockSampler(dev_index).start()
@@ -590,20 +608,28 @@ def run_ours(args):
     ms_total = dist.max_over_ranks(ms_total, device=torch.device("cuda", dev_index))
     value = dec.step_bytes * args.steps * info.world / (ms_total / 1e3) / 1e9
 
-    # dominant kernel: the GEMV alone, replayed from a graph of the same 120
-    # launches on the same stream
-    g_gemv = dec.capture(dec.gemv_only)
-    for _ in range(3):
-        g_gemv.replay()
-    reps = max(args.steps, 10)
-    with Timer(torch) as tk:
-        for _ in range(reps):
+    if fused:
+        # every kernel launch of the step is the decode chain kernel: its average
+        # launch duration is the timed region over the launches in it
+        roof_kernel = "k_decode_chain"
+        gemv_ms_per_launch = ms_total / args.steps / dec.launches_per_step
+        gemv_bytes_per_launch = dec.step_bytes / dec.launches_per_step
+    else:
+        # dominant kernel: the GEMV alone, replayed from a graph of the same
+        # launches on the same stream
+        roof_kernel = "k_gemv_dec"
+        g_gemv = dec.capture(dec.gemv_only)
+        for _ in range(3):
             g_gemv.replay()
-    gemv_ms_per_launch = tk.ms() / reps / (len(dec.mats) * dec.L)
-    gemv_bytes_per_launch = dec.gemv_bytes_per_layer / len(dec.mats)
+        reps = max(args.steps, 10)
+        with Timer(torch) as tk:
+            for _ in range(reps):
+                g_gemv.replay()
+        gemv_ms_per_launch = tk.ms() / reps / (len(dec.mats) * dec.L)
+        gemv_bytes_per_launch = dec.gemv_bytes_per_layer / len(dec.mats)
+        del g_gemv
     achieved = gemv_bytes_per_launch / (gemv_ms_per_launch / 1e3) / 1e9
-    traffic = ncu_traffic("k_gemv_dec", ["gemv.cu"])
-    del g_gemv
+    traffic = ncu_traffic(roof_kernel, ["gemv.cu"])
 
     # end to end: activations from pinned host memory, outputs back to host
     x_host = torch.empty(dec.x_flat.shape, dtype=dec.x_flat.dtype, pin_memory=True)
@@ -627,8 +653,9 @@ def run_ours(args):
     rows = {}
     if not args.no_rows and info.world == 1:
         rows["decode_batches"] = {}
-        for t2, fused in ((1, True), (4, False), (4, True), (8, False), (8, True)):
-            d2 = Decode(torch, bn, synth, t2, args.layers, seed_base=31, fused=fused)
+        for t2, mode in ((1, "chain_independent"), (1, "unfused"), (1, "fused"), (4, "chain"), (4, "unfused"),
+                         (8, "chain"), (8, "unfused")):
+            d2 = Decode(torch, bn, synth, t2, args.layers, seed_base=31, mode=mode)
             g2 = d2.capture(d2.step)
             for _ in range(3):
                 g2.replay()
@@ -636,7 +663,7 @@ def run_ours(args):
                 for _ in range(10):
                     g2.replay()
             per = t.ms() / 10
-            rows["decode_batches"][f"T{t2}_{'fused' if fused else 'quant+gemv'}"] = {
+            rows["decode_batches"][f"T{t2}_{mode}"] = {
                 "gbs": round(d2.step_bytes / (per / 1e3) / 1e9, 1), "ms_per_step": round(per, 4),
                 "launches_per_step": d2.launches_per_step}
             del g2, d2
@@ -657,11 +684,16 @@ def run_ours(args):
         "config": {"workload": f"decode GEMV, 2B LLaMA-alike (hidden 2560, FFN 6912), {args.layers} layers, batch {T}",
                    "tokens": T, "layers": args.layers,
                    "projections": [f"{n} {K}->{N}" for n, K, N in dec.mats],
-                   "step": "per layer and projection: int8 act quant (bitnet_quant_act) + sparse ternary GEMV "
-                           "(bitnet_sparse_linear), programmatic dependent launch, CUDA graph",
+                   "step": {"chain": "all projections of all layers in one persistent launch "
+                                     "(bitnet_decode_chain: per projection, int8 act quant + sparse ternary GEMV; "
+                                     "each projection waits for the previous one), CUDA graph",
+                            "fused": "per layer and projection: one fused launch (bitnet_quant_linear), CUDA graph",
+                            "unfused": "per layer and projection: int8 act quant (bitnet_quant_act) + sparse "
+                                       "ternary GEMV (bitnet_sparse_linear), programmatic dependent launch, "
+                                       "CUDA graph"}[args.decode],
                    "l2": f"inputs larger than L2: {dec.weight_bytes / 1e6:.0f} MB of packed weights per step",
                    "parallelism": f"replicas x{info.world} (independent layers, no collective)"},
-        "roofline": {"bound": "hbm", "kernel": "k_gemv_dec", "achieved": round(achieved, 1),
+        "roofline": {"bound": "hbm", "kernel": roof_kernel, "achieved": round(achieved, 1),
                      "peak": peaks["hbm"], "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
                      "traffic": traffic, "peak_source": peaks["source"],
                      "alg_bytes_per_launch": gemv_bytes_per_launch,

@@ -191,10 +191,9 @@ bitnet_status bitnet_sparse_linear(const int8_t *Xq, const float *absmax,
  * Same result as bitnet_quant_act followed by bitnet_sparse_linear (bit for
  * bit): "BitNet b1.58 ...", section "The mechanism" (per-token symmetric
  * 8-bit activations; ternary product as signed sums).  For T <= 8 with the
- * decode layout it is ONE kernel: each CTA starts streaming its packed weights
- * before waiting on the previous kernel of the stream (programmatic dependent
- * launch), then forms the token scales from X and quantises in registers.
- * Otherwise it runs the quantisation into the workspace and the GEMM.
+ * decode layout it is the decode chain below with one projection (one
+ * kernel, quantisation fused); otherwise, and for shapes the chain does not
+ * take, it runs the quantisation into the workspace and the GEMV or GEMM.
  *
  *   X        [T, K] fp32 or bf16 (x_dtype), 16-byte aligned, K == W->k.
  *   eps      activation eps (> 0).
@@ -209,6 +208,56 @@ size_t bitnet_quant_linear_workspace_size(int64_t T, int64_t K);
 bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps,
                                   const bitnet_packed_w *W, int64_t T, void *Y, bitnet_dtype y_dtype,
                                   int32_t *acc_out, int8_t *xq_out, float *absmax_out,
+                                  void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_decode_chain - a sequence of decode projections in one launch.
+ *
+ * Each op computes exactly bitnet_quant_linear(op.X, ...) for its own packed
+ * weights ("BitNet b1.58 ...", section "The mechanism"; "Sparse-BitNet"
+ * (gist.science), section 2 "Kerncomponenten"), for the T <= 8 tokens of a
+ * decode step.  The ops run in order inside one persistent kernel (one CTA
+ * per SM): ops[i] with wait_prev = 1 reads its X only after every CTA has
+ * finished ops[0..i-1], so ops[i].X may be the Y of an earlier op (a chain of
+ * layers); wait_prev = 0 lets an op whose X is ready start before the
+ * previous op has finished (for example Q, K and V read the same X).  Packed
+ * weights are streamed into shared memory ahead of use and must not be
+ * written while the call runs.
+ *
+ *   ops      host array of n_ops descriptors (read during the call only):
+ *              X        [T, W->k] of x_dtype, 16-byte aligned (device);
+ *              W        host struct; needs dec_codes (16-byte aligned),
+ *                       n = 2, m = 4, n_out % 16 == 0, k % 64 == 0 and
+ *                       n_out / 16 <= 32 x (number of SMs);
+ *              Y        [T, W->n_out] of y_dtype (device);
+ *              acc_out  [T, n_out] int32 or NULL (raw accumulators);
+ *              xq_out   [T, k] int8 or NULL; absmax_out [T] fp32 or NULL;
+ *              wait_prev  0 or 1 (ignored for ops[0]).
+ *            Y of one op must not overlap X, Y or the weights of another op
+ *            that may run at the same time.
+ *   n_ops    >= 0; more than 128 ops are split into launches of 128.
+ *   T        1..8 tokens (0: nothing to do).
+ *   eps      activation eps (> 0).
+ *   ws       >= bitnet_decode_chain_workspace_size(n_ops) bytes: status word,
+ *            abort word and one completion counter per op (cleared by the call).
+ * Shared memory bounds T * (max k + 16): the call returns UNSUPPORTED when
+ * fewer than two 16 KB weight stages would fit.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA; a wait that runs out
+ * inside the kernel sets the TIMEOUT bit of the device status word.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    const void *X;
+    const bitnet_packed_w *W;
+    void *Y;
+    int32_t *acc_out;
+    int8_t *xq_out;
+    float *absmax_out;
+    int32_t wait_prev;
+} bitnet_chain_op;
+
+size_t bitnet_decode_chain_workspace_size(int32_t n_ops);
+bitnet_status bitnet_decode_chain(const bitnet_chain_op *ops, int32_t n_ops, int64_t T,
+                                  bitnet_dtype x_dtype, bitnet_dtype y_dtype, float eps,
                                   void *ws, size_t ws_bytes, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------

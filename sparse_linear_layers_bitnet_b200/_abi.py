@@ -30,6 +30,7 @@ EXPORTED = [
     "bitnet_quant_act",
     "bitnet_linear_workspace_size", "bitnet_sparse_linear",
     "bitnet_quant_linear_workspace_size", "bitnet_quant_linear",
+    "bitnet_decode_chain_workspace_size", "bitnet_decode_chain",
     "bitnet_dgrad_workspace_size", "bitnet_dgrad",
     "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
 ]
@@ -46,6 +47,18 @@ class BitnetPackedW(ctypes.Structure):
         ("mma_vals", ctypes.c_void_p),
         ("mma_meta", ctypes.c_void_p),
         ("dec_codes", ctypes.c_void_p),
+    ]
+
+
+class BitnetChainOp(ctypes.Structure):
+    _fields_ = [
+        ("X", ctypes.c_void_p),
+        ("W", ctypes.POINTER(BitnetPackedW)),
+        ("Y", ctypes.c_void_p),
+        ("acc_out", ctypes.c_void_p),
+        ("xq_out", ctypes.c_void_p),
+        ("absmax_out", ctypes.c_void_p),
+        ("wait_prev", ctypes.c_int32),
     ]
 
 
@@ -81,6 +94,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_sparse_linear": (I32, [P, P, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, SZ, P]),
         "bitnet_quant_linear_workspace_size": (SZ, [I64, I64]),
         "bitnet_quant_linear": (I32, [P, I32, F, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, P, P, SZ, P]),
+        "bitnet_decode_chain_workspace_size": (SZ, [I32]),
+        "bitnet_decode_chain": (I32, [ctypes.POINTER(BitnetChainOp), I32, I64, I32, I32, F, P, SZ, P]),
         "bitnet_dgrad_workspace_size": (SZ, [I64, I64]),
         "bitnet_dgrad": (I32, [P, I32, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, SZ, P]),
         "bitnet_read_device_status": (I32, [P, P]),
@@ -243,6 +258,53 @@ def bitnet_quant_linear(X, W: PackedWeights, eps: float = 1e-5, Y=None, y_dtype=
                                   _dtype_code(Y.dtype), _ptr(acc_out), _ptr(xq_out), _ptr(absmax_out), ws.ptr,
                                   ws.nbytes, _stream(stream)), "bitnet_quant_linear")
     return Y
+
+
+class DecodeChain:
+    """A fixed sequence of decode projections for bitnet_decode_chain.
+
+    ops: list of dicts with keys X, W (PackedWeights), Y and optionally
+    acc_out, xq_out, absmax_out, wait_prev (default 1).  The descriptor array
+    is built once and kept alive with the chain, so the same call can be
+    repeated (or captured in a CUDA graph) without rebuilding it.
+    """
+
+    def __init__(self, ops, x_dtype, y_dtype, eps: float = 1e-5, device="cuda"):
+        lib = load()
+        self.n = len(ops)
+        self.T = int(ops[0]["X"].shape[0]) if ops else 0
+        self.eps = float(eps)
+        self.x_code, self.y_code = _dtype_code(x_dtype), _dtype_code(y_dtype)
+        self._keep = []
+        arr = (BitnetChainOp * max(self.n, 1))()
+        for i, o in enumerate(ops):
+            st = o["W"].struct()
+            self._keep.append(st)
+            arr[i].X = o["X"].data_ptr()
+            arr[i].W = ctypes.pointer(st)
+            arr[i].Y = o["Y"].data_ptr()
+            arr[i].acc_out = o["acc_out"].data_ptr() if o.get("acc_out") is not None else None
+            arr[i].xq_out = o["xq_out"].data_ptr() if o.get("xq_out") is not None else None
+            arr[i].absmax_out = o["absmax_out"].data_ptr() if o.get("absmax_out") is not None else None
+            arr[i].wait_prev = int(o.get("wait_prev", 1))
+        self._arr = arr
+        self.ws = Workspace(lib.bitnet_decode_chain_workspace_size(self.n), device)
+
+    def __call__(self, stream=None):
+        lib = load()
+        check(lib.bitnet_decode_chain(self._arr, self.n, self.T, self.x_code, self.y_code, ctypes.c_float(self.eps),
+                                      self.ws.ptr, self.ws.nbytes, _stream(stream)), "bitnet_decode_chain")
+
+
+def bitnet_decode_chain(ops, eps: float = 1e-5, y_dtype=None, stream=None) -> DecodeChain:
+    """Runs ops (see DecodeChain) once and returns the chain for reuse."""
+    torch = _torch()
+    x_dtype = ops[0]["X"].dtype if ops else torch.bfloat16
+    if y_dtype is None:
+        y_dtype = ops[0]["Y"].dtype if ops else torch.bfloat16
+    ch = DecodeChain(ops, x_dtype, y_dtype, eps, ops[0]["X"].device if ops else "cuda")
+    ch(stream)
+    return ch
 
 
 def bitnet_dgrad(dY, W: PackedWeights, dX=None, dx_dtype=None, ws: Workspace | None = None, stream=None):

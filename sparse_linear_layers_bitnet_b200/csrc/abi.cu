@@ -4,6 +4,8 @@
 #include <cstdio>
 #include <cstring>
 
+#include <vector>
+
 #include "../../include/bitnet_sparse.h"
 #include "kernels.h"
 
@@ -211,12 +213,13 @@ bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps
     if (!aligned(X, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: X and ws must be 16-byte aligned");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool xb = x_dtype == BITNET_BF16, yb = y_dtype == BITNET_BF16;
-    if (T <= 8 && W->dec_codes && n_out % 16 == 0 && k % 64 == 0 &&
-        static_cast<size_t>(T) * static_cast<size_t>(k + 16) <= bitnet::kFusedMaxSmem) {
+    if (T <= 8 && W->dec_codes && n_out % 16 == 0 && k % 64 == 0 && n_out / 16 <= bitnet::kChainMaxTiles * bitnet::num_sms() &&
+        bitnet::chain_stages(T, k) >= 2 && ws_bytes >= bitnet_decode_chain_workspace_size(1)) {
         if (!aligned(W->dec_codes, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: dec_codes alignment");
-        return cuda_status(bitnet::launch_gemv_fused(X, xb, eps, W->gamma, W->dec_codes, T, n_out, k, Y, yb, acc_out,
-                                                     xq_out, absmax_out, s),
-                           "quant_linear (fused decode GEMV)");
+        bitnet::ChainOpDev op = {X, W->dec_codes, W->gamma, Y, acc_out, xq_out, absmax_out,
+                                 static_cast<int32_t>(n_out), static_cast<int32_t>(k), 0, 0};
+        return cuda_status(bitnet::launch_decode_chain(&op, 1, T, xb, yb, eps, k, ws, s),
+                           "quant_linear (decode chain of one projection)");
     }
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     int8_t *xq = reinterpret_cast<int8_t *>(w8 + bitnet::kLinearWsBytes);
@@ -234,6 +237,53 @@ bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps
         if (e != cudaSuccess) return cuda_status(e, "quant_linear copy");
     }
     return BITNET_OK;
+}
+
+size_t bitnet_decode_chain_workspace_size(int32_t n_ops) {
+    const size_t n = n_ops > 0 ? static_cast<size_t>(n_ops) : 0;
+    return bitnet::kChainCountersOffset + align256(4 * n);
+}
+
+bitnet_status bitnet_decode_chain(const bitnet_chain_op *ops, int32_t n_ops, int64_t T, bitnet_dtype x_dtype,
+                                  bitnet_dtype y_dtype, float eps, void *ws, size_t ws_bytes, bitnet_stream_t stream) {
+    if (n_ops < 0) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: n_ops < 0");
+    if (T < 0 || T > 8) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: T must be in 0..8");
+    if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: bad x dtype");
+    if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: bad y dtype");
+    if (!(eps > 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: eps must be > 0");
+    if (n_ops == 0 || T == 0) return BITNET_OK;
+    if (!ops) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: null ops");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "decode_chain: workspace is required");
+    if (ws_bytes < bitnet_decode_chain_workspace_size(n_ops))
+        return fail(BITNET_ERR_WORKSPACE, "decode_chain: workspace needs %zu bytes",
+                    bitnet_decode_chain_workspace_size(n_ops));
+    if (!aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: ws must be 16-byte aligned");
+    const int64_t max_tiles = static_cast<int64_t>(bitnet::kChainMaxTiles) * bitnet::num_sms();
+    std::vector<bitnet::ChainOpDev> dev(static_cast<size_t>(n_ops));
+    int64_t kmax = 0;
+    for (int32_t i = 0; i < n_ops; ++i) {
+        const bitnet_chain_op &o = ops[i];
+        const bitnet_packed_w *W = o.W;
+        if (!W || !W->gamma || !W->dec_codes) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: op %d: null W, gamma or dec_codes", i);
+        if (!(W->n == 2 && W->m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: op %d: 2:4 only", i);
+        if (W->n_out <= 0 || W->k <= 0 || W->n_out % 16 || W->k % 64)
+            return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: op %d: needs n_out %% 16 == 0 and k %% 64 == 0", i);
+        if (W->n_out / 16 > max_tiles || W->n_out > INT32_MAX || W->k > INT32_MAX)
+            return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: op %d: n_out above 512 rows per SM", i);
+        if (!o.X || !o.Y) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: op %d: null X or Y", i);
+        if (!aligned(o.X, 16) || !aligned(W->dec_codes, 16))
+            return fail(BITNET_ERR_INVALID_ARG, "decode_chain: op %d: X and dec_codes must be 16-byte aligned", i);
+        if (o.wait_prev != 0 && o.wait_prev != 1) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: op %d: wait_prev must be 0 or 1", i);
+        kmax = W->k > kmax ? W->k : kmax;
+        dev[static_cast<size_t>(i)] = {o.X, W->dec_codes, W->gamma, o.Y, o.acc_out, o.xq_out, o.absmax_out,
+                                       static_cast<int32_t>(W->n_out), static_cast<int32_t>(W->k), o.wait_prev, 0};
+    }
+    if (bitnet::chain_stages(T, kmax) < 2)
+        return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: T * (k + 16) leaves no room for two weight stages");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return cuda_status(bitnet::launch_decode_chain(dev.data(), n_ops, T, x_dtype == BITNET_BF16, y_dtype == BITNET_BF16,
+                                                   eps, kmax, ws, s),
+                       "decode_chain");
 }
 
 bitnet_status bitnet_dgrad(const void *dY, bitnet_dtype dy_dtype, const bitnet_packed_w *W, int64_t T, void *dX,

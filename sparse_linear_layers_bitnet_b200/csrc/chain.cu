@@ -1,0 +1,479 @@
+// Decode chain: a sequence of quantise + sparse ternary GEMV projections in
+// one persistent launch (sm_100a).
+//
+// What each projection computes is the BitLinear forward of "BitNet b1.58:
+// Ternary Weights for 1.58-bit LLMs", section "The mechanism" (per-token
+// absmax int8 activations, ternary weights, integer sums, one rescale) with
+// the 2:4 mask of "Sparse-BitNet" (gist.science), section 2
+// "Kerncomponenten"; the numbers are those of bitnet_quant_act followed by
+// bitnet_sparse_linear, bit for bit.
+//
+// Why one launch: at decode sizes (T <= 8) a projection moves 1 to 10 MB of
+// packed weights, under 2 us of HBM time, while each dependent kernel launch
+// adds about 3 us of completion and dependency latency.  Here every SM runs
+// one CTA for the whole chain:
+//  * a producer warp streams the CTA's share of every projection's packed
+//    weights (a contiguous byte range of the decode layout) into a ring of
+//    16 KB shared-memory stages with bulk asynchronous copies.  Weights do not
+//    depend on activations, so the stream runs ahead across projection
+//    boundaries, limited only by free stages;
+//  * eight consumer warps, per projection: wait until every CTA has finished
+//    the previous projection (a grid-wide counter, acquire loads, bounded
+//    wait), read the T activation rows from L2, form the per-token scales and
+//    int8 codes in shared memory, run one m16n8k64 sparse MMA per 64-k tile
+//    of each weight record in the ring, sum the partial tiles in shared
+//    memory, write Y, and count themselves done (release add).
+// Row tiles of a projection are split over the CTAs in balanced contiguous
+// ranges, rotated per projection so that the larger shares move around.
+//
+// All waits are bounded (2 s): a stage that never fills, a counter that never
+// reaches the grid size or an abort raised by another CTA ends the kernel
+// with the timeout bit in the status word; outstanding copies are waited for
+// (bounded) before the CTA exits.
+#include "../../include/bitnet_sparse.h"
+#include "common.cuh"
+#include "frag.cuh"
+#include "kernels.h"
+
+namespace bitnet {
+
+constexpr int kChainConsumerWarps = 8;
+constexpr int kChainConsumers = kChainConsumerWarps * 32;
+constexpr int kChainThreads = kChainConsumers + 32;
+constexpr uint32_t kStageBytes = 16384;            // 64 weight records of 256 bytes
+constexpr int kChainMaxStages = 16;
+constexpr int kChainRegChunks = 16;                // 16-byte activation chunks cached per consumer thread
+
+struct ChainParams {
+    ChainOpDev op[kChainMaxOps];
+    int32_t n_ops, T, x_bf16, y_bf16, ns;
+    float eps;
+    uint32_t *counters;   // [n_ops], zero at launch
+    uint32_t *abort;      // grid-wide abort word, zero at launch
+    uint32_t *status;
+};
+
+// Row tiles [t0, t1) of projection j for this CTA.  The CTA's share index v
+// is its block index rotated by 61 j; share v is [v R / G, (v + 1) R / G).
+// Share G - 1 is never empty when R >= 1.
+__device__ __forceinline__ int chain_tiles(int j, int rows16, int &t0, int &t1) {
+    const int G = static_cast<int>(gridDim.x);
+    int v = static_cast<int>(blockIdx.x) + (j * 61) % G;
+    if (v >= G) v -= G;
+    t0 = static_cast<int>((static_cast<int64_t>(v) * rows16) / G);
+    t1 = static_cast<int>((static_cast<int64_t>(v + 1) * rows16) / G);
+    return v;
+}
+
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kChainConsumers) : "memory"); }
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Spins (bounded) until *ctr >= target.  On a timeout or a grid abort it sets
+// the CTA's abort flag (and, on a timeout, the grid abort word and status).
+__device__ bool wait_counter(const uint32_t *ctr, uint32_t target, const ChainParams &p, volatile int *s_abort) {
+    if (ld_acquire(ctr) >= target) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        __nanosleep(32);
+        if (ld_acquire(ctr) >= target) return true;
+        if (*reinterpret_cast<volatile uint32_t *>(p.abort) != 0u) {
+            *s_abort = 1;
+            return false;
+        }
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *s_abort = 1;
+            atomicOr(p.status, kStatusTimeout);
+            atomicExch(p.abort, 1u);
+            return false;
+        }
+    }
+}
+
+// Wait that ignores the abort flag, up to a deadline (for draining copies in flight).
+__device__ bool mbar_wait_until(uint64_t *bar, uint32_t parity, uint64_t deadline_ns) {
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() > deadline_ns) return false;
+    }
+    return true;
+}
+
+// Barrier of the consumer warps (hardware barrier 2; plain consumer barriers
+// use 1) that also ORs a predicate over them, so that every consumer takes the
+// same branch after it.
+__device__ __forceinline__ bool consumer_sync_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 2, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(v ? 1u : 0u), "n"(kChainConsumers)
+        : "memory");
+    return r != 0;
+}
+
+template <bool BF16>
+struct ChainChunk {
+    static constexpr int kElems = BF16 ? 8 : 4;
+    uint4 raw;
+    __device__ __forceinline__ float get(int j) const {
+        const int i = BF16 ? (j >> 1) : j;
+        const uint32_t w = i == 0 ? raw.x : (i == 1 ? raw.y : (i == 2 ? raw.z : raw.w));
+        if (BF16) return __uint_as_float((j & 1) ? (w & 0xffff0000u) : (w << 16));
+        return __uint_as_float(w);
+    }
+    __device__ __forceinline__ float absmax() const {
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kElems; ++j) m = fmaxf(m, fabsf(get(j)));
+        return m;
+    }
+    __device__ __forceinline__ void store_codes(int8_t *dst, float s) const {
+        uint32_t w[2] = {0u, 0u};
+#pragma unroll
+        for (int j = 0; j < kElems; ++j)
+            w[j >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(quant_code(get(j), s))) << (8 * (j & 3));
+        if (BF16)
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+        else
+            *reinterpret_cast<uint32_t *>(dst) = w[0];
+    }
+};
+
+// Per-token absmax and int8 codes of one projection's activations into
+// shared memory (row pitch k + 16).  X is read through L2 only (ld.global.cg):
+// it may have been written by other SMs earlier in this kernel.
+template <bool BF16>
+__device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float eps, int8_t *s_xq,
+                               float (*s_red)[8], float *s_amax, int ctid) {
+    using C = ChainChunk<BF16>;
+    const uint32_t cpr = static_cast<uint32_t>(k / C::kElems);
+    const uint32_t nchunk = static_cast<uint32_t>(T) * cpr;
+    const int warp = ctid >> 5, lane = ctid & 31;
+    C reg[kChainRegChunks];
+    float m[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) m[t] = 0.0f;
+#pragma unroll
+    for (int u = 0; u < kChainRegChunks; ++u) {
+        const uint32_t c = static_cast<uint32_t>(ctid) + static_cast<uint32_t>(u) * kChainConsumers;
+        if (c < nchunk) {
+            reg[u].raw = __ldcg(X + c);
+            const uint32_t tc = c / cpr;
+            const float a = reg[u].absmax();
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                if (static_cast<uint32_t>(t) == tc) m[t] = fmaxf(m[t], a);
+        }
+    }
+#pragma unroll 4
+    for (uint32_t c = static_cast<uint32_t>(ctid) + kChainRegChunks * kChainConsumers; c < nchunk;
+         c += kChainConsumers) {
+        C ch;
+        ch.raw = __ldcg(X + c);
+        const uint32_t tc = c / cpr;
+        const float a = ch.absmax();
+#pragma unroll
+        for (int t = 0; t < 8; ++t)
+            if (static_cast<uint32_t>(t) == tc) m[t] = fmaxf(m[t], a);
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        if (t < T) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m[t] = fmaxf(m[t], __shfl_xor_sync(0xffffffffu, m[t], o));
+        }
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int t = 0; t < 8; ++t) s_red[warp][t] = m[t];
+    }
+    consumer_sync();
+    if (ctid < 8) {
+        float v = 0.0f;
+#pragma unroll
+        for (int q = 0; q < kChainConsumerWarps; ++q) v = fmaxf(v, s_red[q][ctid]);
+        s_amax[ctid] = v > eps ? v : eps;
+    }
+    consumer_sync();
+    const uint32_t pitch = static_cast<uint32_t>(k) + 16u;
+#pragma unroll
+    for (int u = 0; u < kChainRegChunks; ++u) {
+        const uint32_t c = static_cast<uint32_t>(ctid) + static_cast<uint32_t>(u) * kChainConsumers;
+        if (c < nchunk) {
+            const uint32_t tc = c / cpr;
+            reg[u].store_codes(s_xq + tc * pitch + (c - tc * cpr) * C::kElems, __fdiv_rn(127.0f, s_amax[tc]));
+        }
+    }
+#pragma unroll 4
+    for (uint32_t c = static_cast<uint32_t>(ctid) + kChainRegChunks * kChainConsumers; c < nchunk;
+         c += kChainConsumers) {
+        C ch;
+        ch.raw = __ldcg(X + c);
+        const uint32_t tc = c / cpr;
+        ch.store_codes(s_xq + tc * pitch + (c - tc * cpr) * C::kElems, __fdiv_rn(127.0f, s_amax[tc]));
+    }
+}
+
+template <bool XBF16>
+__global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_constant__ ChainParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) uint64_t s_full[kChainMaxStages], s_empty[kChainMaxStages];
+    __shared__ float s_red[kChainConsumerWarps][8];
+    __shared__ float s_amax[8], s_scale[8];
+    __shared__ int s_abort;
+    const int tid = threadIdx.x;
+    const int ns = p.ns;
+    const int T = p.T;
+    const uint32_t G = gridDim.x;
+    // dynamic shared memory: ring [ns][16 KB] | partial sums [kChainMaxTiles][32][4] int | int8 rows
+    uint8_t *ring = smem;
+    int *s_acc = reinterpret_cast<int *>(smem + static_cast<size_t>(ns) * kStageBytes);
+    int8_t *s_xq = reinterpret_cast<int8_t *>(s_acc + kChainMaxTiles * 128);
+
+    for (int i = tid; i < kChainMaxTiles * 128; i += kChainThreads) s_acc[i] = 0;
+    if (tid == 0) {
+        s_abort = 0;
+        for (int s = 0; s < ns; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], kChainConsumerWarps);
+        }
+        fence_mbar_init();
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+
+    if (tid >= kChainConsumers) {
+        // ------------------------------------------------------------ producer
+        if (tid != kChainConsumers) return;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int j = 0; j < p.n_ops && ok; ++j) {
+            const ChainOpDev &op = p.op[j];
+            int t0, t1;
+            chain_tiles(j, op.n_out >> 4, t0, t1);
+            const uint32_t tile_bytes = static_cast<uint32_t>(op.k >> 6) * 256u;
+            const uint32_t bytes = static_cast<uint32_t>(t1 - t0) * tile_bytes;
+            const uint8_t *src = op.dec + static_cast<size_t>(t0) * tile_bytes;
+            // Warm L2 with this CTA's slice of the projection's activation rows
+            // (128-byte lines b, b + G, ...).  Only a cache hint: L2 is the
+            // coherence point, so a line prefetched before an earlier projection
+            // writes it is updated by that write.
+            {
+                const size_t xbytes = static_cast<size_t>(p.T) * static_cast<size_t>(op.k) * (p.x_bf16 ? 2u : 4u);
+                for (size_t l = static_cast<size_t>(blockIdx.x) * 128; l < xbytes; l += static_cast<size_t>(gridDim.x) * 128)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t *>(op.X) + l));
+            }
+            for (uint32_t off = 0; off < bytes; off += kStageBytes, ++it) {
+                const uint32_t s = it % static_cast<uint32_t>(ns);
+                if (it >= static_cast<uint32_t>(ns) &&
+                    !mbar_wait_bounded(&s_empty[s], ((it / ns) - 1u) & 1u, &s_abort, p.status)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t n = (bytes - off) < kStageBytes ? (bytes - off) : kStageBytes;
+                mbar_arrive_expect_tx(&s_full[s], n);
+                bulk_load(ring + static_cast<size_t>(s) * kStageBytes, src + off, n, &s_full[s]);
+            }
+        }
+        // drain: every issued stage must have landed before the CTA may exit
+        // (earlier stages were consumed before their slot was reused)
+        const uint32_t first = it > static_cast<uint32_t>(ns) ? it - ns : 0u;
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        for (uint32_t q = first; q < it; ++q) mbar_wait_until(&s_full[q % ns], (q / ns) & 1u, deadline);
+        return;
+    }
+
+    // ---------------------------------------------------------------- consumers
+    // Every branch that can differ between consumer threads (an expired wait,
+    // an abort) is decided through consumer_sync_or or a warp vote, so that the
+    // consumer barriers never miss a thread.
+    const int ctid = tid;
+    const int warp = ctid >> 5, lane = ctid & 31;
+    const int gid = lane >> 2, tq = lane & 3;
+    const bool tok = gid < T;
+    uint32_t it = 0;
+    for (int j = 0; j < p.n_ops; ++j) {
+        const ChainOpDev &op = p.op[j];
+        int t0, t1;
+        const int share = chain_tiles(j, op.n_out >> 4, t0, t1);
+        const int ntile = t1 - t0;
+        const int ktiles = op.k >> 6;
+        const uint32_t bytes = static_cast<uint32_t>(ntile) * static_cast<uint32_t>(ktiles) * 256u;
+        // gamma belongs to the packed weights: read before the wait
+        const float gamma = ntile > 0 ? __ldg(op.gamma) : 0.0f;
+        // 1. every CTA has finished the previous projection
+        if (j > 0 && op.wait_prev) {
+            bool bad = false;
+            if (ctid == 0) bad = !wait_counter(&p.counters[j - 1], G, p, &s_abort);
+            if (consumer_sync_or(bad || s_abort != 0)) break;
+        }
+        if (ntile > 0) {
+            // 2. int8 activations of this projection
+            if (XBF16)
+                chain_quantise<true>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, s_xq, s_red, s_amax, ctid);
+            else
+                chain_quantise<false>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, s_xq, s_red, s_amax, ctid);
+            if (ctid < 8) s_scale[ctid] = __fdiv_rn(__fmul_rn(gamma, s_amax[ctid]), 127.0f);
+            consumer_sync();
+            // 3. weight records from the ring: warp w takes records w, w + 8, ...
+            const int8_t *xs = s_xq + (tok ? gid : 0) * (op.k + 16) + 4 * tq;
+            int cur = -1;
+            int d[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};   // alternate records: two independent MMA chains
+            int par = 0;
+            bool failed = false;
+            for (uint32_t off = 0; off < bytes; off += kStageBytes, ++it) {
+                const uint32_t s = it % static_cast<uint32_t>(ns);
+                const bool ok = mbar_wait_bounded(&s_full[s], (it / ns) & 1u, &s_abort, p.status);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    failed = true;
+                    break;
+                }
+                const int nrec = static_cast<int>(((bytes - off) < kStageBytes ? (bytes - off) : kStageBytes) >> 8);
+                const int r0 = static_cast<int>(off >> 8) + warp;
+                int tile = r0 / ktiles;
+                int kt = r0 - tile * ktiles;
+                const uint2 *rec = reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(s) * kStageBytes) + lane;
+                for (int i = warp; i < nrec; i += kChainConsumerWarps) {
+                    if (tile != cur) {
+                        if (cur >= 0) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) atomicAdd(&s_acc[(cur * 32 + lane) * 4 + q], d[q] + d2[q]);
+                        }
+                        cur = tile;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) d[q] = d2[q] = 0;
+                    }
+                    const uint2 w = rec[i * 32];
+                    uint32_t a[4], b[4];
+#pragma unroll
+                    for (int jj = 0; jj < 4; ++jj)
+                        b[jj] = tok ? *reinterpret_cast<const uint32_t *>(xs + kt * 64 + 16 * jj) : 0u;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) a[r] = expand_codes(w.x, r);
+                    if (par)
+                        mma_sp_m16n8k64(d2, a, b, w.y);
+                    else
+                        mma_sp_m16n8k64(d, a, b, w.y);
+                    par ^= 1;
+                    kt += kChainConsumerWarps;
+                    while (kt >= ktiles) {
+                        kt -= ktiles;
+                        ++tile;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[s]);
+            }
+            if (cur >= 0) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) atomicAdd(&s_acc[(cur * 32 + lane) * 4 + q], d[q] + d2[q]);
+            }
+            if (consumer_sync_or(failed || s_abort != 0)) break;
+            // 4. dequantise and store this CTA's rows; clear the partial sums
+            for (int e = ctid; e < ntile * 128; e += kChainConsumers) {
+                const int tl = e >> 7, ln = (e >> 2) & 31, q = e & 3;
+                const int t = 2 * (ln & 3) + (q & 1);
+                const int acc = s_acc[e];
+                s_acc[e] = 0;
+                if (t >= T) continue;
+                const int64_t n = static_cast<int64_t>(t0 + tl) * 16 + (ln >> 2) + 8 * (q >> 1);
+                const int64_t o = static_cast<int64_t>(t) * op.n_out + n;
+                const float y = __fmul_rn(__int2float_rn(acc), s_scale[t]);
+                if (p.y_bf16)
+                    static_cast<__nv_bfloat16 *>(op.Y)[o] = __float2bfloat16_rn(y);
+                else
+                    static_cast<float *>(op.Y)[o] = y;
+                if (op.acc_out) op.acc_out[o] = acc;
+            }
+            // optional copies of the int8 activations and scales (by the CTA holding share G - 1)
+            if (share == static_cast<int>(G) - 1) {
+                if (op.xq_out) {
+                    for (int i = ctid; i < T * op.k; i += kChainConsumers) {
+                        const int t = i / op.k;
+                        op.xq_out[i] = s_xq[t * (op.k + 16) + (i - t * op.k)];
+                    }
+                }
+                if (op.amax_out && ctid < T) op.amax_out[ctid] = s_amax[ctid];
+            }
+            consumer_sync();
+        }
+        // 5. count this CTA done with projection j, after projection j - 1 (chain order)
+        bool bad = false;
+        if (ctid == 0) {
+            if (j > 0 && !op.wait_prev) bad = !wait_counter(&p.counters[j - 1], G, p, &s_abort);
+            // release: the consumer barrier above ordered every consumer's Y stores before this add
+            if (!bad) asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(&p.counters[j]), "r"(1u) : "memory");
+        }
+        if (j > 0 && !op.wait_prev && consumer_sync_or(bad)) break;
+    }
+}
+
+size_t chain_smem_bytes(int ns, int64_t T, int64_t kmax) {
+    return static_cast<size_t>(ns) * kStageBytes + static_cast<size_t>(kChainMaxTiles) * 128 * 4 +
+           static_cast<size_t>(T) * static_cast<size_t>(kmax + 16);
+}
+
+int chain_stages(int64_t T, int64_t kmax) {
+    const size_t fixed = chain_smem_bytes(0, T, kmax);
+    if (fixed >= kChainMaxSmem) return 0;
+    size_t ns = (kChainMaxSmem - fixed) / kStageBytes;
+    if (ns > static_cast<size_t>(kChainMaxStages)) ns = kChainMaxStages;
+    return static_cast<int>(ns);
+}
+
+cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
+                                int64_t kmax, void *ws, cudaStream_t s) {
+    const int ns = chain_stages(T, kmax);
+    if (ns < 2) return cudaErrorInvalidValue;
+    static bool attr_done[2] = {false, false};
+    if (!attr_done[x_bf16 ? 1 : 0]) {
+        cudaError_t e = x_bf16 ? cudaFuncSetAttribute(k_decode_chain<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(kChainMaxSmem))
+                               : cudaFuncSetAttribute(k_decode_chain<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      static_cast<int>(kChainMaxSmem));
+        if (e != cudaSuccess) return e;
+        attr_done[x_bf16 ? 1 : 0] = true;
+    }
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    for (int base = 0; base < n_ops; base += kChainMaxOps) {
+        const int n = (n_ops - base) < kChainMaxOps ? (n_ops - base) : kChainMaxOps;
+        ChainParams p;
+        for (int i = 0; i < n; ++i) p.op[i] = ops[base + i];
+        // a later launch continues the chain: its first projection waits for the previous launch by stream order
+        p.op[0].wait_prev = 0;
+        p.n_ops = n;
+        p.T = static_cast<int32_t>(T);
+        p.x_bf16 = x_bf16 ? 1 : 0;
+        p.y_bf16 = y_bf16 ? 1 : 0;
+        p.ns = ns;
+        p.eps = eps;
+        p.status = reinterpret_cast<uint32_t *>(w8 + kStatusOffset);
+        p.abort = reinterpret_cast<uint32_t *>(w8 + kChainAbortOffset);
+        p.counters = reinterpret_cast<uint32_t *>(w8 + kChainCountersOffset);
+        cudaError_t e = cudaMemsetAsync(w8 + kChainAbortOffset, 0,
+                                        kChainCountersOffset - kChainAbortOffset + static_cast<size_t>(n) * 4, s);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(num_sms()));
+        cfg.blockDim = dim3(kChainThreads);
+        cfg.dynamicSmemBytes = chain_smem_bytes(ns, T, kmax);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = x_bf16 ? cudaLaunchKernelEx(&cfg, k_decode_chain<true>, p) : cudaLaunchKernelEx(&cfg, k_decode_chain<false>, p);
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace bitnet

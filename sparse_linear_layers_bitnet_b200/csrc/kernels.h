@@ -45,12 +45,26 @@ cudaError_t launch_gemv_dec(const int8_t *Xq, const float *amax, const float *ga
                             int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                             cudaStream_t s);
 
-// Largest shared-memory staging of the fused decode kernel: T * (k + 16) bytes.
-constexpr size_t kFusedMaxSmem = 160 * 1024;
-
-cudaError_t launch_gemv_fused(const void *X, bool x_bf16, float eps, const float *gamma, const uint8_t *dec,
-                              int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
-                              int8_t *xq_out, float *amax_out, cudaStream_t s);
+// Decode chain (chain.cu): one projection as the kernel sees it.
+struct ChainOpDev {
+    const void *X;
+    const uint8_t *dec;
+    const float *gamma;
+    void *Y;
+    int32_t *acc_out;
+    int8_t *xq_out;
+    float *amax_out;
+    int32_t n_out, k, wait_prev, pad;
+};
+constexpr int kChainMaxOps = 128;                  // projections per launch (kernel parameter space)
+constexpr int kChainMaxTiles = 32;                 // 16-row tiles per CTA per projection
+constexpr size_t kChainMaxSmem = 227 * 1024 - 1024;   // dynamic shared memory (static use < 1 KB)
+constexpr size_t kChainAbortOffset = 4;            // workspace: grid abort word
+constexpr size_t kChainCountersOffset = 256;       // workspace: one counter per projection
+size_t chain_smem_bytes(int ns, int64_t T, int64_t kmax);
+int chain_stages(int64_t T, int64_t kmax);
+cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
+                                int64_t kmax, void *ws, cudaStream_t s);
 
 cudaError_t launch_gemv_gb(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *gb,
                            int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,

@@ -126,6 +126,51 @@ def test_linear_rejects_bad_arguments(lib):
     assert f(None, _fake(), ctypes.byref(_pw()), 4, _fake(), 0, None, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
 
 
+def _chain(ops_specs):
+    arr = (_abi.BitnetChainOp * max(len(ops_specs), 1))()
+    keep = []
+    for i, (st, x, y, wait) in enumerate(ops_specs):
+        keep.append(st)
+        arr[i].X = x
+        arr[i].W = ctypes.pointer(st) if st is not None else None
+        arr[i].Y = y
+        arr[i].wait_prev = wait
+    return arr, keep
+
+
+def test_decode_chain_rejects_bad_arguments(lib):
+    f = lib.bitnet_decode_chain
+    ws = lib.bitnet_decode_chain_workspace_size(2)
+    assert ws >= 256 + 8
+    good = _pw(n_out=256, k=256, dec=True)
+    arr, keep = _chain([(good, 4096, 8192, 1), (good, 4096, 8192, 1)])
+    bf = _abi.BITNET_BF16
+    assert f(arr, -1, 1, bf, bf, 1e-5, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(arr, 2, 9, bf, bf, 1e-5, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG    # T > 8
+    assert f(arr, 2, 1, 7, bf, 1e-5, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG     # x dtype
+    assert f(arr, 2, 1, bf, bf, 0.0, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG    # eps
+    assert f(None, 2, 1, bf, bf, 1e-5, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(arr, 2, 1, bf, bf, 1e-5, None, ws, None) == _abi.BITNET_ERR_WORKSPACE
+    assert f(arr, 2, 1, bf, bf, 1e-5, _fake(), ws - 4, None) == _abi.BITNET_ERR_WORKSPACE
+    assert f(arr, 2, 1, bf, bf, 1e-5, _fake(4100), ws, None) == _abi.BITNET_ERR_INVALID_ARG   # ws alignment
+    # nothing to do: no ops or no tokens
+    assert f(arr, 0, 1, bf, bf, 1e-5, None, 0, None) == _abi.BITNET_OK
+    assert f(arr, 2, 0, bf, bf, 1e-5, None, 0, None) == _abi.BITNET_OK
+    bad_cases = [
+        ((None, 4096, 8192, 1), _abi.BITNET_ERR_INVALID_ARG),                        # null W
+        ((_pw(dec=False), 4096, 8192, 1), _abi.BITNET_ERR_INVALID_ARG),               # no decode layout
+        ((_pw(n_out=256, k=288, dec=True), 4096, 8192, 1), _abi.BITNET_ERR_UNSUPPORTED),   # k % 64
+        ((_pw(n_out=200, k=256, dec=True), 4096, 8192, 1), _abi.BITNET_ERR_UNSUPPORTED),   # n_out % 16
+        ((_pw(n=1, m=4, dec=True), 4096, 8192, 1), _abi.BITNET_ERR_UNSUPPORTED),      # 2:4 only
+        ((good, None, 8192, 1), _abi.BITNET_ERR_INVALID_ARG),                         # null X
+        ((good, 4100, 8192, 1), _abi.BITNET_ERR_INVALID_ARG),                         # X alignment
+        ((good, 4096, 8192, 2), _abi.BITNET_ERR_INVALID_ARG),                         # wait_prev
+    ]
+    for spec, want in bad_cases:
+        arr2, keep2 = _chain([(good, 4096, 8192, 1), spec])
+        assert f(arr2, 2, 1, bf, bf, 1e-5, _fake(), ws, None) == want, spec
+
+
 def test_dgrad_rejects_bad_arguments(lib):
     f = lib.bitnet_dgrad
     ws = lib.bitnet_dgrad_workspace_size(256, 256)

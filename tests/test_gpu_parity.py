@@ -340,6 +340,34 @@ def test_quant_linear_fused_decode(bn, T, x_dtype, n_out, k):
     _check_outputs(ref, acc.cpu().numpy(), Y)
 
 
+@pytest.mark.parametrize("T,x_dtype", [(1, "bf16"), (8, "bf16"), (5, "f32")])
+@pytest.mark.parametrize("n_out,k", [(6912, 2560), (6928, 192), (9616, 128), (640, 64), (4752, 6912)])
+def test_quant_linear_streamed_row_tiles(bn, T, x_dtype, n_out, k):
+    """bitnet_quant_linear at T <= 8 runs the decode chain with one projection:
+    row tiles per CTA from 1 to 5 with ragged shares (6928 and 9616 rows),
+    k = 64 (one record per row tile, fewer records than warps) and odd k-tile
+    counts (k = 192)."""
+    W = synth.master_weights(n_out, k, 0.02, seed=420 + T)
+    X = synth.activations(T, k, seed=421 + T, outlier_p=0.01)
+    if x_dtype == "bf16":
+        Xd, X32 = bf16_dev(X)
+    else:
+        Xd, X32 = dev_f32(X), X
+    ref = oracle.forward(W, X32, 1e-5, 1e-5)
+    pw = bn.PackedWeights(n_out, k, mma=False)
+    bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5)
+    acc = torch.full((T, n_out), -7, dtype=torch.int32, device="cuda")
+    xq = torch.zeros((T, k), dtype=torch.int8, device="cuda")
+    am = torch.zeros((T,), dtype=torch.float32, device="cuda")
+    ws = bn.Workspace(bn.load().bitnet_quant_linear_workspace_size(T, k))
+    Y = bn.bitnet_quant_linear(Xd, pw, 1e-5, y_dtype=torch.bfloat16, acc_out=acc, xq_out=xq, absmax_out=am, ws=ws)
+    torch.cuda.synchronize()
+    assert bn.bitnet_read_device_status(ws) == 0
+    assert np.array_equal(xq.cpu().numpy(), ref["xq"])
+    assert np.array_equal(am.cpu().numpy(), ref["a"])
+    _check_outputs(ref, acc.cpu().numpy(), Y)
+
+
 @pytest.mark.parametrize("T", [16, 100])
 def test_quant_linear_unfused_path(bn, T):
     n_out, k = 384, 1024
@@ -386,6 +414,104 @@ def test_quant_linear_chain_in_graph(bn):
     for l in range(layers):
         x = oracle.forward(Ws[l], x, 1e-5, 1e-5)["y"]
         assert np.array_equal(xs[l + 1].cpu().numpy(), x), l
+
+
+# ------------------------------------------------------------------ decode chain (one persistent launch)
+
+def _packed_dec(bn, n_out, k, seed):
+    W = synth.master_weights(n_out, k, 0.02, seed=seed)
+    pw = bn.PackedWeights(n_out, k, group_bytes=True, mma=False, dec=True)
+    bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5)
+    return W, pw
+
+
+@pytest.mark.parametrize("T", [1, 3, 8])
+def test_decode_chain_layers(bn, T):
+    """A chain of layers: each op reads the previous op's Y (wait_prev = 1).
+    Every op is checked against the oracle on the input the GPU actually had."""
+    dims = [512, 768, 512, 2560, 64, 6912, 2560]
+    Ws, pws = [], []
+    for i in range(len(dims) - 1):
+        W, pw = _packed_dec(bn, dims[i + 1], dims[i], seed=800 + i)
+        Ws.append(W)
+        pws.append(pw)
+    x0 = synth.activations(T, dims[0], seed=900 + T, outlier_p=0.01)
+    xs = [dev_f32(x0)] + [torch.empty((T, d), dtype=torch.float32, device="cuda") for d in dims[1:]]
+    accs = [torch.full((T, d), -7, dtype=torch.int32, device="cuda") for d in dims[1:]]
+    ops = [dict(X=xs[i], W=pws[i], Y=xs[i + 1], acc_out=accs[i], wait_prev=1) for i in range(len(pws))]
+    ch = bn.bitnet_decode_chain(ops, 1e-5)
+    torch.cuda.synchronize()
+    assert bn.bitnet_read_device_status(ch.ws) == 0
+    for i in range(len(pws)):
+        ref = oracle.forward(Ws[i], xs[i].cpu().numpy(), 1e-5, 1e-5)
+        _check_outputs(ref, accs[i].cpu().numpy(), xs[i + 1])
+    # the same chain again (counters are cleared by every call)
+    y_first = xs[-1].clone()
+    for x in xs[1:]:
+        x.zero_()
+    ch()
+    torch.cuda.synchronize()
+    assert torch.equal(xs[-1], y_first)
+
+
+@pytest.mark.parametrize("T", [1, 5])
+def test_decode_chain_independent_and_ragged(bn, T):
+    """Independent ops (wait_prev 0 and 1 mixed), bf16 in and out, row counts
+    from one tile (most CTAs idle) to several tiles per CTA, k = 64 (one k-tile
+    per row tile, fewer records than warps) and odd k-tile counts."""
+    shapes = [(16, 64), (9616, 128), (48, 192), (2560, 6912), (4752, 2560), (640, 64), (13824, 2560)]
+    ops, refs = [], []
+    for i, (n_out, k) in enumerate(shapes):
+        W, pw = _packed_dec(bn, n_out, k, seed=1000 + i)
+        Xd, X32 = bf16_dev(synth.activations(T, k, seed=1100 + i, outlier_p=0.01))
+        Y = torch.empty((T, n_out), dtype=torch.bfloat16, device="cuda")
+        acc = torch.full((T, n_out), -7, dtype=torch.int32, device="cuda")
+        xq = torch.zeros((T, k), dtype=torch.int8, device="cuda")
+        am = torch.zeros((T,), dtype=torch.float32, device="cuda")
+        ops.append(dict(X=Xd, W=pw, Y=Y, acc_out=acc, xq_out=xq, absmax_out=am, wait_prev=i % 2))
+        refs.append(oracle.forward(W, X32, 1e-5, 1e-5))
+    ch = bn.bitnet_decode_chain(ops, 1e-5)
+    torch.cuda.synchronize()
+    assert bn.bitnet_read_device_status(ch.ws) == 0
+    for o, ref in zip(ops, refs):
+        assert np.array_equal(o["xq_out"].cpu().numpy(), ref["xq"])
+        assert np.array_equal(o["absmax_out"].cpu().numpy(), ref["a"])
+        _check_outputs(ref, o["acc_out"].cpu().numpy(), o["Y"])
+
+
+def test_decode_chain_split_launches_and_graph(bn):
+    """More ops than one launch takes (130 > 128): the library splits the chain;
+    captured in a CUDA graph and replayed."""
+    T, h = 2, 256
+    n_ops = 130
+    Ws, pws = [], []
+    for i in range(n_ops):
+        # master std 0.13 keeps the layer gain near 1 (0.8 std * sqrt(0.35 h)), so
+        # the activations neither vanish nor blow up over 130 layers
+        W = synth.master_weights(h, h, 0.13, seed=1200 + i)
+        pw = bn.PackedWeights(h, h, group_bytes=True, mma=False, dec=True)
+        bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5)
+        Ws.append(W)
+        pws.append(pw)
+    x0 = synth.activations(T, h, seed=1300)
+    xs = [dev_f32(x0)] + [torch.empty((T, h), dtype=torch.float32, device="cuda") for _ in range(n_ops)]
+    ops = [dict(X=xs[i], W=pws[i], Y=xs[i + 1], wait_prev=1) for i in range(n_ops)]
+    ch = bn.DecodeChain(ops, torch.float32, torch.float32, 1e-5)
+    ch()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ch()
+    for x in xs[1:]:
+        x.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert bn.bitnet_read_device_status(ch.ws) == 0
+    x = x0
+    for i in range(n_ops):
+        x = oracle.forward(Ws[i], x, 1e-5, 1e-5)["y"]
+        assert np.array_equal(xs[i + 1].cpu().numpy(), x), i
+    del g
 
 
 # ------------------------------------------------------------------ per-step pack with the previous gamma as hint
