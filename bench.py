@@ -405,21 +405,35 @@ def measure_pack(torch, bn, synth, peaks, steps=3, flip_steps=100, layers=None):
     alg_bytes = n_w * (4 + 0.25 + 0.5 + 0.125)   # read fp32, write group bytes, int8 values, metadata
     for W, pw in zip(Ws, pws):
         bn.bitnet_pack_nm(W, pw, 1e-5, ws=ws)
+    batch = bn.PackBatch(list(zip(Ws, pws)), 1e-5, dev)
     torch.cuda.synchronize()
-    ms = []
+    ms, ms_single = [], []
     for s in range(steps):
         for i, W in enumerate(Ws):
             synth.torch_random_walk_(W, 1e-4, seed=s * 1000 + i)
         with Timer(torch) as t:
+            batch()
+        ms.append(t.ms())
+    # the same step with one bitnet_pack_nm_update call per matrix, for comparison
+    for s in range(steps):
+        for i, W in enumerate(Ws):
+            synth.torch_random_walk_(W, 1e-4, seed=(steps + s) * 1000 + i)
+        with Timer(torch) as t:
             for W, pw in zip(Ws, pws):
                 bn.bitnet_pack_nm_update(W, pw, 1e-5, ws=ws)
-        ms.append(t.ms())
+        ms_single.append(t.ms())
     step_ms = statistics.mean(ms)
     gbs = alg_bytes / step_ms / 1e6
+    n_mats = len(Ws)
     out = {"weights": n_w, "step_ms": round(step_ms, 3), "gbs": round(gbs, 1),
            "frac_of_hbm": round(gbs / peaks["hbm"], 4),
-           "alg_bytes_per_weight": 4.875, "launches_per_matrix": 3,
-           "entry": "bitnet_pack_nm_update (previous step's gamma as hint; bit-identical to bitnet_pack_nm)"}
+           "alg_bytes_per_weight": 4.875, "launches_per_step": 2 * ((n_mats + 63) // 64),
+           "entry": "bitnet_pack_nm_update_batch over all matrices (each previous gamma as hint; "
+                    "bit-identical to bitnet_pack_nm)",
+           "per_matrix_calls": {"step_ms": round(statistics.mean(ms_single), 3),
+                                "gbs": round(alg_bytes / statistics.mean(ms_single) / 1e6, 1),
+                                "entry": "bitnet_pack_nm_update, one call per matrix"}}
+    del batch
     if flip_steps <= 0:
         del Ws, pws
         torch.cuda.empty_cache()

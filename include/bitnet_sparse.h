@@ -144,6 +144,40 @@ bitnet_status bitnet_pack_nm_update(const float *W, bitnet_packed_w *out, float 
                                     bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_pack_nm_update_batch - bitnet_pack_nm_update of many matrices at once.
+ *
+ * "Sparse-BitNet" (gist.science), section 2 "Training Strategie": every step
+ * re-derives the mask and codes of every layer from its masters.  Each item
+ * gets exactly what bitnet_pack_nm_update(items[i].W, items[i].out, eps,
+ * items[i].mask_bits, ...) gives it, bit for bit, including the use of
+ * out->gamma as the previous gamma.  The whole list runs in two kernel
+ * launches per 64 matrices (plus one per matrix that asks for dec_codes)
+ * instead of three or four per matrix, so the fixed cost of a launch, a
+ * workspace clear and a gamma finalisation is paid once per list.
+ *
+ *   items    host array of n_items descriptors (read during the call only):
+ *              W          [n_out x k] fp32 masters, 16-byte aligned (device);
+ *              out        host struct as for bitnet_pack_nm_update (n = 2,
+ *                         m = 4, k % 16 == 0); out->gamma holds the hint;
+ *              mask_bits  [n_out * k / 8] or NULL.
+ *            The items' output buffers must not overlap one another.
+ *   n_items  >= 0.
+ *   eps      >= 0.
+ *   ws       >= bitnet_pack_update_batch_workspace_size(items, n_items) bytes,
+ *            16-byte aligned: one scratch header per item, then the band lists.
+ * Errors: as bitnet_pack_nm_update; UNSUPPORTED when k % 16 != 0.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    const float *W;
+    bitnet_packed_w *out;
+    uint8_t *mask_bits;
+} bitnet_pack_item;
+
+size_t bitnet_pack_update_batch_workspace_size(const bitnet_pack_item *items, int32_t n_items);
+bitnet_status bitnet_pack_nm_update_batch(const bitnet_pack_item *items, int32_t n_items, float eps,
+                                          void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * bitnet_quant_act - per-token absmax int8 activation quantisation.
  *
  * "BitNet b1.58: Ternary Weights for 1.58-bit LLMs", section "The mechanism"

@@ -5,13 +5,13 @@ include/bitnet_sparse.h); this package is its thin Python binding plus the
 seeded synthetic input generators.
 """
 from ._abi import (  # noqa: F401
-    BITNET_BF16, BITNET_F32, BitnetChainOp, BitnetError, BitnetPackedW, DecodeChain, PackedWeights, Workspace,
-    bitnet_decode_chain, bitnet_dgrad, bitnet_pack_nm, bitnet_pack_nm_update, bitnet_quant_act, bitnet_quant_linear, bitnet_read_device_status, bitnet_sparse_linear, load,
+    BITNET_BF16, BITNET_F32, BitnetChainOp, BitnetError, BitnetPackedW, BitnetPackItem, DecodeChain, PackBatch, PackedWeights, Workspace,
+    bitnet_decode_chain, bitnet_dgrad, bitnet_pack_nm_update_batch, bitnet_pack_nm, bitnet_pack_nm_update, bitnet_quant_act, bitnet_quant_linear, bitnet_read_device_status, bitnet_sparse_linear, load,
 )
 
 __all__ = [
     "PackedWeights", "Workspace", "BitnetError", "BitnetPackedW", "BitnetChainOp", "DecodeChain", "load",
-    "bitnet_decode_chain",
+    "bitnet_decode_chain", "bitnet_pack_nm_update_batch", "PackBatch", "BitnetPackItem",
     "bitnet_pack_nm", "bitnet_pack_nm_update", "bitnet_quant_act", "bitnet_quant_linear", "bitnet_sparse_linear", "bitnet_dgrad", "bitnet_read_device_status",
     "BITNET_F32", "BITNET_BF16",
 ]

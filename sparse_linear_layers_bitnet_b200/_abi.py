@@ -27,6 +27,7 @@ EXPORTED = [
     "bitnet_mma_meta_bytes", "bitnet_dec_bytes",
     "bitnet_pack_workspace_size", "bitnet_pack_nm", "bitnet_pack_nm_noalloc",
     "bitnet_pack_update_workspace_size", "bitnet_pack_nm_update",
+    "bitnet_pack_update_batch_workspace_size", "bitnet_pack_nm_update_batch",
     "bitnet_quant_act",
     "bitnet_linear_workspace_size", "bitnet_sparse_linear",
     "bitnet_quant_linear_workspace_size", "bitnet_quant_linear",
@@ -47,6 +48,14 @@ class BitnetPackedW(ctypes.Structure):
         ("mma_vals", ctypes.c_void_p),
         ("mma_meta", ctypes.c_void_p),
         ("dec_codes", ctypes.c_void_p),
+    ]
+
+
+class BitnetPackItem(ctypes.Structure):
+    _fields_ = [
+        ("W", ctypes.c_void_p),
+        ("out", ctypes.POINTER(BitnetPackedW)),
+        ("mask_bits", ctypes.c_void_p),
     ]
 
 
@@ -89,6 +98,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_pack_nm_noalloc": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P]),
         "bitnet_pack_update_workspace_size": (SZ, [I64, I64]),
         "bitnet_pack_nm_update": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P, SZ, P]),
+        "bitnet_pack_update_batch_workspace_size": (SZ, [ctypes.POINTER(BitnetPackItem), I32]),
+        "bitnet_pack_nm_update_batch": (I32, [ctypes.POINTER(BitnetPackItem), I32, F, P, SZ, P]),
         "bitnet_quant_act": (I32, [P, I32, I64, I64, F, P, P, P]),
         "bitnet_linear_workspace_size": (SZ, []),
         "bitnet_sparse_linear": (I32, [P, P, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, SZ, P]),
@@ -208,6 +219,45 @@ def bitnet_pack_nm_update(W, out: PackedWeights, eps: float = 1e-5, mask_bits=No
     check(lib.bitnet_pack_nm_update(_ptr(W), ctypes.byref(st), ctypes.c_float(eps), _ptr(mask_bits), ws.ptr,
                                     ws.nbytes, _stream(stream)), "bitnet_pack_nm_update")
     return out
+
+
+class PackBatch:
+    """A fixed list of (W, PackedWeights[, mask_bits]) for bitnet_pack_nm_update_batch.
+
+    The descriptor array and the workspace are built once, so the same batch
+    can be repacked every step (or captured in a CUDA graph) without
+    rebuilding them.
+    """
+
+    def __init__(self, items, eps: float = 1e-5, device="cuda"):
+        lib = load()
+        self.n = len(items)
+        self.eps = float(eps)
+        self._keep = []
+        arr = (BitnetPackItem * max(self.n, 1))()
+        for i, it in enumerate(items):
+            W, out = it[0], it[1]
+            mask = it[2] if len(it) > 2 else None
+            assert W.dtype == _torch().float32 and W.is_contiguous()
+            st = out.struct()
+            self._keep.append((st, W, out, mask))
+            arr[i].W = W.data_ptr()
+            arr[i].out = ctypes.pointer(st)
+            arr[i].mask_bits = mask.data_ptr() if mask is not None else None
+        self._arr = arr
+        self.ws = Workspace(lib.bitnet_pack_update_batch_workspace_size(arr, self.n), device)
+
+    def __call__(self, stream=None):
+        lib = load()
+        check(lib.bitnet_pack_nm_update_batch(self._arr, self.n, ctypes.c_float(self.eps), self.ws.ptr,
+                                              self.ws.nbytes, _stream(stream)), "bitnet_pack_nm_update_batch")
+
+
+def bitnet_pack_nm_update_batch(items, eps: float = 1e-5, stream=None) -> PackBatch:
+    """Per-step pack of many matrices (each out.gamma is its hint); returns the batch for reuse."""
+    b = PackBatch(items, eps, items[0][0].device if items else "cuda")
+    b(stream)
+    return b
 
 
 def bitnet_quant_act(X, eps: float = 1e-5, Xq=None, absmax=None, stream=None):

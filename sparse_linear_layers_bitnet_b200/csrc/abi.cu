@@ -1,5 +1,6 @@
 // C ABI of the sparse ternary BitLinear library: host-side argument checks,
 // shape dispatch and launches.  Declarations and semantics: bitnet_sparse.h.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -104,12 +105,7 @@ bitnet_status bitnet_pack_nm(const float *W, bitnet_packed_w *out, float eps, ui
 
 size_t bitnet_pack_update_workspace_size(int64_t n_out, int64_t k) {
     if (n_out <= 0 || k <= 0) return bitnet::kPackWsBytes;
-    // list room for 1/256 of the groups (Gaussian masters put ~0.06% of the
-    // weights within 2^-10 of the threshold), at least 16384 entries
-    const size_t groups = static_cast<size_t>(n_out) * static_cast<size_t>(k) / 4;
-    size_t cap = groups / 256;
-    if (cap < 16384) cap = 16384;
-    return bitnet::kPackWsBytes + cap * 4;
+    return bitnet::kPackWsBytes + bitnet::update_list_bytes(n_out, k);
 }
 
 bitnet_status bitnet_pack_nm_update(const float *W, bitnet_packed_w *out, float eps, uint8_t *mask_bits, void *ws,
@@ -132,6 +128,56 @@ bitnet_status bitnet_pack_nm_update(const float *W, bitnet_packed_w *out, float 
                                                   out->mma_meta, out->dec_codes, mask_bits, ws, ws_bytes,
                                                   reinterpret_cast<cudaStream_t>(stream)),
                        "pack_update");
+}
+
+size_t bitnet_pack_update_batch_workspace_size(const bitnet_pack_item *items, int32_t n_items) {
+    if (!items || n_items <= 0) return 256;
+    std::vector<int64_t> n_out(static_cast<size_t>(n_items)), k(static_cast<size_t>(n_items));
+    for (int32_t i = 0; i < n_items; ++i) {
+        const bitnet_packed_w *o = items[i].out;
+        n_out[static_cast<size_t>(i)] = (o && o->n_out > 0) ? o->n_out : 0;
+        k[static_cast<size_t>(i)] = (o && o->k > 0) ? o->k : 0;
+    }
+    return bitnet::pack_batch_ws_bytes(n_out.data(), k.data(), n_items);
+}
+
+bitnet_status bitnet_pack_nm_update_batch(const bitnet_pack_item *items, int32_t n_items, float eps, void *ws,
+                                          size_t ws_bytes, bitnet_stream_t stream) {
+    if (n_items < 0) return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: n_items < 0");
+    if (n_items == 0) return BITNET_OK;
+    if (!items) return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: null items");
+    if (!(eps >= 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: eps must be >= 0");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "pack_update_batch: workspace is required");
+    if (!aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: ws must be 16-byte aligned");
+    std::vector<bitnet::PackBatchItemHost> h(static_cast<size_t>(n_items));
+    for (int32_t i = 0; i < n_items; ++i) {
+        const bitnet_pack_item &it = items[i];
+        const bitnet_packed_w *out = it.out;
+        if (!it.W || !out || !out->gamma)
+            return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: item %d: W, out and out->gamma are required", i);
+        const int64_t n_out = out->n_out, k = out->k;
+        if (n_out <= 0 || k <= 0 || k % 8) return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: item %d: bad sizes", i);
+        if (!(out->n == 2 && out->m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "pack_update_batch: item %d: 2:4 only", i);
+        if (k % 16) return fail(BITNET_ERR_UNSUPPORTED, "pack_update_batch: item %d: k %% 16 != 0", i);
+        if (!aligned(it.W, 16)) return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: item %d: W must be 16-byte aligned", i);
+        if ((out->mma_vals == nullptr) != (out->mma_meta == nullptr))
+            return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: item %d: mma_vals and mma_meta go together", i);
+        if (out->dec_codes && (!out->group_bytes || n_out % 16 || k % 64))
+            return fail(BITNET_ERR_INVALID_ARG,
+                        "pack_update_batch: item %d: dec_codes need group_bytes, n_out %% 16 == 0, k %% 64 == 0", i);
+        if (static_cast<double>(n_out) * static_cast<double>(k) / 4.0 > 4294967295.0)
+            return fail(BITNET_ERR_UNSUPPORTED, "pack_update_batch: item %d: more than 2^32 groups", i);
+        h[static_cast<size_t>(i)] = {it.W, n_out, k, out->gamma, out->group_bytes, out->mma_vals, out->mma_meta,
+                                     out->dec_codes, it.mask_bits};
+    }
+    const size_t need = bitnet_pack_update_batch_workspace_size(items, n_items);
+    if (ws_bytes < need) return fail(BITNET_ERR_WORKSPACE, "pack_update_batch: workspace needs %zu bytes", need);
+    double total_chunks = 0.0;
+    for (const auto &x : h) total_chunks += std::ceil(static_cast<double>(x.n_out) * static_cast<double>(x.k) / 8192.0);
+    if (total_chunks > 4294967295.0) return fail(BITNET_ERR_UNSUPPORTED, "pack_update_batch: too many weights in one call");
+    return cuda_status(bitnet::launch_pack_update_batch(h.data(), n_items, eps, ws,
+                                                        reinterpret_cast<cudaStream_t>(stream)),
+                       "pack_update_batch");
 }
 
 bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, int64_t K, float eps, int8_t *Xq,

@@ -17,7 +17,7 @@
 //    16 KB shared-memory stages with bulk asynchronous copies.  Weights do not
 //    depend on activations, so the stream runs ahead across projection
 //    boundaries, limited only by free stages;
-//  * eight consumer warps, per projection: wait until every CTA has finished
+//  * sixteen consumer warps, per projection: wait until every CTA has finished
 //    the previous projection (a grid-wide counter, acquire loads, bounded
 //    wait), read the T activation rows from L2, form the per-token scales and
 //    int8 codes in shared memory, run one m16n8k64 sparse MMA per 64-k tile
@@ -37,12 +37,11 @@
 
 namespace bitnet {
 
-constexpr int kChainConsumerWarps = 8;
+constexpr int kChainConsumerWarps = 16;
 constexpr int kChainConsumers = kChainConsumerWarps * 32;
 constexpr int kChainThreads = kChainConsumers + 32;
 constexpr uint32_t kStageBytes = 16384;            // 64 weight records of 256 bytes
 constexpr int kChainMaxStages = 16;
-constexpr int kChainRegChunks = 16;                // 16-byte activation chunks cached per consumer thread
 
 struct ChainParams {
     ChainOpDev op[kChainMaxOps];
@@ -89,6 +88,31 @@ __device__ bool wait_counter(const uint32_t *ctr, uint32_t target, const ChainPa
             *s_abort = 1;
             atomicOr(p.status, kStatusTimeout);
             atomicExch(p.abort, 1u);
+            return false;
+        }
+    }
+}
+
+// Producer's wait for a free stage: the thread is suspended in the barrier
+// (try_wait with a suspend-time hint) until the phase completes, instead of
+// spinning and taking issue slots from the consumer warps.  Bounded like
+// mbar_wait_bounded.
+__device__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+            : "memory");
+        if (ok) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicOr(status, kStatusTimeout);
             return false;
         }
     }
@@ -146,42 +170,57 @@ struct ChainChunk {
     }
 };
 
-// Per-token absmax and int8 codes of one projection's activations into
-// shared memory (row pitch k + 16).  X is read through L2 only (ld.global.cg):
-// it may have been written by other SMs earlier in this kernel.
+// Per-token absmax, scales and int8 codes of one projection's activations
+// (same arithmetic as bitnet_quant_act) into shared memory, row pitch k + 16.
+// X is read through L2 only (ld.global.cg): it may have been written by other
+// SMs earlier in this kernel.  Each thread walks the flattened 16-byte chunks
+// c = ctid, ctid + 256, ... with its token index tracked incrementally (no
+// division), two loads in flight per step; the second pass re-reads the chunks
+// from L2.  s_inv[t] = 127 / a_t and s_scale[t] = (gamma a_t) / 127 are formed
+// once per token.
 template <bool BF16>
-__device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float eps, int8_t *s_xq,
-                               float (*s_red)[8], float *s_amax, int ctid) {
+__device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float eps, float gamma, int8_t *s_xq,
+                               float (*s_red)[8], float *s_amax, float *s_inv, float *s_scale, int ctid) {
     using C = ChainChunk<BF16>;
-    const uint32_t cpr = static_cast<uint32_t>(k / C::kElems);
-    const uint32_t nchunk = static_cast<uint32_t>(T) * cpr;
+    const int cpr = k / C::kElems;             // chunks per token row (>= 8)
+    const int nchunk = T * cpr;
     const int warp = ctid >> 5, lane = ctid & 31;
-    C reg[kChainRegChunks];
     float m[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) m[t] = 0.0f;
-#pragma unroll
-    for (int u = 0; u < kChainRegChunks; ++u) {
-        const uint32_t c = static_cast<uint32_t>(ctid) + static_cast<uint32_t>(u) * kChainConsumers;
-        if (c < nchunk) {
-            reg[u].raw = __ldcg(X + c);
-            const uint32_t tc = c / cpr;
-            const float a = reg[u].absmax();
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-                if (static_cast<uint32_t>(t) == tc) m[t] = fmaxf(m[t], a);
+    {
+        int c = ctid, t = 0, i = ctid;
+        while (i >= cpr) {
+            i -= cpr;
+            ++t;
         }
-    }
-#pragma unroll 4
-    for (uint32_t c = static_cast<uint32_t>(ctid) + kChainRegChunks * kChainConsumers; c < nchunk;
-         c += kChainConsumers) {
-        C ch;
-        ch.raw = __ldcg(X + c);
-        const uint32_t tc = c / cpr;
-        const float a = ch.absmax();
+        while (c < nchunk) {
+            C a, b;
+            const int c2 = c + kChainConsumers;
+            a.raw = __ldcg(X + c);
+            if (c2 < nchunk) b.raw = __ldcg(X + c2);
+            const float ma = a.absmax();
 #pragma unroll
-        for (int t = 0; t < 8; ++t)
-            if (static_cast<uint32_t>(t) == tc) m[t] = fmaxf(m[t], a);
+            for (int tt = 0; tt < 8; ++tt)
+                if (tt == t) m[tt] = fmaxf(m[tt], ma);
+            i += kChainConsumers;
+            while (i >= cpr) {
+                i -= cpr;
+                ++t;
+            }
+            if (c2 < nchunk) {
+                const float mb = b.absmax();
+#pragma unroll
+                for (int tt = 0; tt < 8; ++tt)
+                    if (tt == t) m[tt] = fmaxf(m[tt], mb);
+                i += kChainConsumers;
+                while (i >= cpr) {
+                    i -= cpr;
+                    ++t;
+                }
+            }
+            c = c2 + kChainConsumers;
+        }
     }
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
@@ -195,29 +234,44 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
         for (int t = 0; t < 8; ++t) s_red[warp][t] = m[t];
     }
     consumer_sync();
-    if (ctid < 8) {
+    if (ctid < T) {
         float v = 0.0f;
 #pragma unroll
         for (int q = 0; q < kChainConsumerWarps; ++q) v = fmaxf(v, s_red[q][ctid]);
-        s_amax[ctid] = v > eps ? v : eps;
+        v = v > eps ? v : eps;
+        s_amax[ctid] = v;
+        s_inv[ctid] = __fdiv_rn(127.0f, v);
+        s_scale[ctid] = __fdiv_rn(__fmul_rn(gamma, v), 127.0f);
     }
     consumer_sync();
-    const uint32_t pitch = static_cast<uint32_t>(k) + 16u;
-#pragma unroll
-    for (int u = 0; u < kChainRegChunks; ++u) {
-        const uint32_t c = static_cast<uint32_t>(ctid) + static_cast<uint32_t>(u) * kChainConsumers;
-        if (c < nchunk) {
-            const uint32_t tc = c / cpr;
-            reg[u].store_codes(s_xq + tc * pitch + (c - tc * cpr) * C::kElems, __fdiv_rn(127.0f, s_amax[tc]));
+    const int pitch = k + 16;
+    {
+        int c = ctid, t = 0, i = ctid;
+        while (i >= cpr) {
+            i -= cpr;
+            ++t;
         }
-    }
-#pragma unroll 4
-    for (uint32_t c = static_cast<uint32_t>(ctid) + kChainRegChunks * kChainConsumers; c < nchunk;
-         c += kChainConsumers) {
-        C ch;
-        ch.raw = __ldcg(X + c);
-        const uint32_t tc = c / cpr;
-        ch.store_codes(s_xq + tc * pitch + (c - tc * cpr) * C::kElems, __fdiv_rn(127.0f, s_amax[tc]));
+        while (c < nchunk) {
+            C a, b;
+            const int c2 = c + kChainConsumers;
+            a.raw = __ldcg(X + c);
+            if (c2 < nchunk) b.raw = __ldcg(X + c2);
+            a.store_codes(s_xq + t * pitch + i * C::kElems, s_inv[t]);
+            i += kChainConsumers;
+            while (i >= cpr) {
+                i -= cpr;
+                ++t;
+            }
+            if (c2 < nchunk) {
+                b.store_codes(s_xq + t * pitch + i * C::kElems, s_inv[t]);
+                i += kChainConsumers;
+                while (i >= cpr) {
+                    i -= cpr;
+                    ++t;
+                }
+            }
+            c = c2 + kChainConsumers;
+        }
     }
 }
 
@@ -226,7 +280,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kChainMaxStages], s_empty[kChainMaxStages];
     __shared__ float s_red[kChainConsumerWarps][8];
-    __shared__ float s_amax[8], s_scale[8];
+    __shared__ float s_amax[8], s_inv[8], s_scale[8];
     __shared__ int s_abort;
     const int tid = threadIdx.x;
     const int ns = p.ns;
@@ -273,7 +327,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             for (uint32_t off = 0; off < bytes; off += kStageBytes, ++it) {
                 const uint32_t s = it % static_cast<uint32_t>(ns);
                 if (it >= static_cast<uint32_t>(ns) &&
-                    !mbar_wait_bounded(&s_empty[s], ((it / ns) - 1u) & 1u, &s_abort, p.status)) {
+                    !mbar_wait_sleep(&s_empty[s], ((it / ns) - 1u) & 1u, &s_abort, p.status)) {
                     ok = false;
                     break;
                 }
@@ -317,12 +371,13 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         if (ntile > 0) {
             // 2. int8 activations of this projection
             if (XBF16)
-                chain_quantise<true>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, s_xq, s_red, s_amax, ctid);
+                chain_quantise<true>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, gamma, s_xq, s_red, s_amax,
+                                     s_inv, s_scale, ctid);
             else
-                chain_quantise<false>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, s_xq, s_red, s_amax, ctid);
-            if (ctid < 8) s_scale[ctid] = __fdiv_rn(__fmul_rn(gamma, s_amax[ctid]), 127.0f);
+                chain_quantise<false>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, gamma, s_xq, s_red, s_amax,
+                                      s_inv, s_scale, ctid);
             consumer_sync();
-            // 3. weight records from the ring: warp w takes records w, w + 8, ...
+            // 3. weight records from the ring: warp w takes records w, w + 16, ...
             const int8_t *xs = s_xq + (tok ? gid : 0) * (op.k + 16) + 4 * tq;
             int cur = -1;
             int d[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};   // alternate records: two independent MMA chains

@@ -38,6 +38,31 @@ cudaError_t launch_pack_update(const float *W, int64_t n_out, int64_t k, float e
                                int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws, size_t ws_bytes,
                                cudaStream_t s);
 
+// Band-list bytes of the per-step pack of one matrix: room for 1/256 of the
+// groups (Gaussian masters put ~0.06% of the weights within 2^-10 of the
+// threshold), at least 16384 entries.
+inline size_t update_list_bytes(int64_t n_out, int64_t k) {
+    const size_t groups = static_cast<size_t>(n_out) * static_cast<size_t>(k) / 4;
+    size_t cap = groups / 256;
+    if (cap < 16384) cap = 16384;
+    return cap * 4;
+}
+
+// Batched per-step pack: one matrix as the host describes it.
+struct PackBatchItemHost {
+    const float *W;
+    int64_t n_out, k;
+    float *gamma;
+    uint8_t *gb;
+    int8_t *vals;
+    uint8_t *meta;
+    uint8_t *dec;
+    uint8_t *mask;
+};
+constexpr int kPackBatchMax = 64;   // matrices per launch (kernel parameter space)
+size_t pack_batch_ws_bytes(const int64_t *n_out, const int64_t *k, int n_items);
+cudaError_t launch_pack_update_batch(const PackBatchItemHost *items, int n_items, float eps, void *ws, cudaStream_t s);
+
 cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xq, float *amax,
                              cudaStream_t s);
 

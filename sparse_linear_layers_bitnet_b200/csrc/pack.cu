@@ -1145,4 +1145,351 @@ cudaError_t launch_pack_update(const float *W, int64_t n_out, int64_t k, float e
     return cudaGetLastError();
 }
 
+
+// ---------------------------------------------------------------- batched per-step pack (lane quads)
+//
+// bitnet_pack_nm_update over a list of matrices in two launches instead of
+// three or four per matrix.  The matrices' quads are cut into chunks of
+// kBatchChunkQuads; the update kernel gives every CTA a contiguous range of
+// the global chunk list, so a CTA meets one or two matrices.  Per matrix it
+// does what k_pack_update_quad does (exact sum, layouts with the previous
+// gamma's threshold, band list), with a per-matrix chunk counter in place of
+// the block ticket: the CTA that completes a matrix's last chunk forms its
+// gamma, threshold and mode.  The finish kernel then patches every listed
+// group (mode 1), reruns the layouts of the matrices whose threshold left the
+// band (mode 2) and writes the metadata padding, each over one flattened
+// index space across the matrices.  Results are those of
+// bitnet_pack_nm_update on each matrix, bit for bit.
+
+struct BatchItem {
+    Pack24Args p;              // layouts (p.thr unused)
+    float *gamma;              // previous gamma in (the hint), new gamma out
+    uint8_t *hdr;              // this matrix's kPackWsBytes scratch header (zeroed before the launch)
+    uint32_t *list;            // band list
+    uint32_t list_cap;
+    uint32_t chunk0, nchunks;  // this matrix's range of the global chunk list
+    uint32_t pad_bytes;        // metadata padding bytes (0: none)
+    int64_t n_total;
+};
+
+struct BatchParams {
+    BatchItem it[kPackBatchMax];
+    int32_t n;
+    uint32_t total_chunks;
+    float eps;
+};
+
+constexpr uint32_t kBatchChunkQuads = 512;   // 256 threads x 2 quads
+
+__device__ __forceinline__ int batch_item_of(const BatchParams &bp, uint32_t c) {
+    int lo = 0, hi = bp.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (bp.it[mid].chunk0 <= c) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(256, 4) k_pack_update_batch(const __grid_constant__ BatchParams bp) {
+    __shared__ unsigned long long s_bins[256];
+    __shared__ unsigned long long s_lo[8], s_hi[8];
+    __shared__ int s_rare;
+    __shared__ uint32_t s_t, s_tlo, s_thi;
+    __shared__ int s_hint;
+    __shared__ unsigned s_ticket;
+    __shared__ int s_nz[256];
+    __shared__ int s_nnz;
+    __shared__ uint32_t s_limb[kLimbs];
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t G = gridDim.x;
+    const uint32_t c_begin = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x) * bp.total_chunks) / G);
+    const uint32_t c_end = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x + 1) * bp.total_chunks) / G);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0ull;
+    uint32_t c = c_begin;
+    while (c < c_end) {
+        const int item = batch_item_of(bp, c);
+        const BatchItem &I = bp.it[item];
+        const uint32_t seg_end = min(c_end, I.chunk0 + I.nchunks);
+        uint8_t *hdr = I.hdr;
+        if (threadIdx.x == 0) {
+            s_rare = 0;
+            const float gp = *I.gamma;
+            s_hint = (gp > 0.0f && gp < 3.0e38f) ? 1 : 0;
+            s_t = s_tlo = s_thi = 0u;
+            if (s_hint) {
+                s_t = code_threshold(gp);
+                const float tf = __uint_as_float(s_t);
+                s_tlo = __float_as_uint(__fmul_rd(tf, 1.0f - 0x1p-10f));
+                s_thi = __float_as_uint(__fmul_ru(tf, 1.0f + 0x1p-10f));
+                if (c == I.chunk0) {
+                    reinterpret_cast<uint32_t *>(hdr + kPackWsBandOffset)[0] = s_tlo;
+                    reinterpret_cast<uint32_t *>(hdr + kPackWsBandOffset)[1] = s_thi;
+                }
+            }
+        }
+        __syncthreads();
+        const bool hint = s_hint != 0;
+        const uint32_t t_old = s_t, t_lo = s_tlo, t_hi = s_thi;
+        const Pack24Args &p = I.p;
+        const uint32_t n_quads = static_cast<uint32_t>(p.n_groups >> 2);
+        unsigned *list_count = reinterpret_cast<unsigned *>(hdr + kPackWsListCountOffset);
+        uint64_t lo = 0, hi = 0;
+        double d = 0.0;
+        for (uint32_t ch = c; ch < seg_end; ++ch) {
+            const uint32_t qbase = (ch - I.chunk0) * kBatchChunkQuads + warp * (32u * kQuadUnroll);
+            float4 v[kQuadUnroll][4];
+#pragma unroll
+            for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
+                const uint32_t q = qbase + 32u * k2 + lane;
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    v[k2][j] = q < n_quads ? __ldg(p.W + 4u * q + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
+                const uint32_t q = qbase + 32u * k2 + lane;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) sum_float4(v[k2][j], d, lo, hi, s_bins, &s_rare);
+                if (hint && q < n_quads) {
+                    const QuadOut o = pack_quad(v[k2], t_old, t_lo, t_hi);
+                    store_quad(p, q, o);
+                    if (o.band) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            if ((o.band >> j) & 1u) {
+                                const unsigned slot = atomicAdd(list_count, 1u);
+                                if (slot < I.list_cap) I.list[slot] = 4u * q + j;
+                            }
+                    }
+                }
+            }
+            flush_sum(d, lo, hi);
+        }
+        // this segment's exact partial sum into the matrix's accumulators
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint64_t l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+            const uint64_t h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+            const uint64_t sum = lo + l2;
+            hi = hi + h2 + ((sum < lo) ? 1ull : 0ull);
+            lo = sum;
+        }
+        if (lane == 0) {
+            s_lo[warp] = lo;
+            s_hi[warp] = hi;
+        }
+        __syncthreads();
+        unsigned long long *win = reinterpret_cast<unsigned long long *>(hdr + kPackWsWinOffset);
+        unsigned long long *bins = reinterpret_cast<unsigned long long *>(hdr + kPackWsBinsOffset);
+        if (threadIdx.x == 0) {
+            uint64_t L = 0, H = 0;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+                const uint64_t sum = L + s_lo[w];
+                H = H + s_hi[w] + ((sum < L) ? 1ull : 0ull);
+                L = sum;
+            }
+            if (L | H) {
+                const unsigned long long old = atomicAdd(&win[0], static_cast<unsigned long long>(L));
+                const uint64_t carry = (static_cast<uint64_t>(old) + L < static_cast<uint64_t>(old)) ? 1ull : 0ull;
+                atomicAdd(&win[1], static_cast<unsigned long long>(H + carry));
+            }
+        }
+        if (s_rare) {
+            for (int e = threadIdx.x; e < 256; e += blockDim.x)
+                if (s_bins[e]) {
+                    atomicAdd(&bins[e], s_bins[e]);
+                    s_bins[e] = 0ull;
+                }
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const unsigned done = seg_end - c;
+            s_ticket = atomicAdd(reinterpret_cast<unsigned *>(hdr + kPackWsCounterOffset), done) + done;
+        }
+        __syncthreads();
+        if (s_ticket == I.nchunks) {
+            // every chunk of this matrix is summed: form gamma, threshold and mode
+            __threadfence();
+            if (threadIdx.x == 0) s_nnz = 0;
+            __syncthreads();
+            for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+                const unsigned long long b = atomicAdd(&bins[e], 0ull);
+                s_bins[e] = b;
+                if (b) s_nz[atomicAdd(&s_nnz, 1)] = e;
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                for (int a = 1; a < s_nnz; ++a)
+                    for (int j = a; j > 0 && s_nz[j - 1] > s_nz[j]; --j) {
+                        const int tmp = s_nz[j];
+                        s_nz[j] = s_nz[j - 1];
+                        s_nz[j - 1] = tmp;
+                    }
+                const uint64_t wlo = atomicAdd(&win[0], 0ull), whi = atomicAdd(&win[1], 0ull);
+                uint32_t *thr = reinterpret_cast<uint32_t *>(hdr + kPackWsThrOffset);
+                finalize_gamma(s_bins, s_nz, s_nnz, wlo, whi, I.n_total, bp.eps, s_limb, I.gamma, thr);
+                const uint32_t t_new = *thr;
+                const unsigned listed = atomicAdd(list_count, 0u);
+                const bool patch = hint && t_new >= t_lo && t_new <= t_hi && listed <= I.list_cap;
+                *reinterpret_cast<uint32_t *>(hdr + kPackWsModeOffset) = patch ? 1u : 2u;
+            }
+            __syncthreads();
+            for (int e = threadIdx.x; e < 256; e += blockDim.x) s_bins[e] = 0ull;
+        }
+        __syncthreads();
+        c = seg_end;
+    }
+}
+
+// index of the last entry of pref[0..n] that is <= x (pref ascending, pref[0] = 0)
+__device__ __forceinline__ int batch_bucket(const uint32_t *pref, int n, uint32_t x) {
+    int lo = 0, hi = n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (pref[mid] <= x) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+// Byte j of the metadata padding of one matrix (k % 16 == 0, so no half-valid
+// bytes): the rows >= n_out of every k-block, then the bytes past the last
+// valid group of the last k-block.  Same bytes as k_meta_pad.
+__device__ __forceinline__ void meta_pad_at(const Pack24Args &p, uint32_t j) {
+    const int64_t kblocks = (p.k + 127) / 128;
+    const int64_t tail_groups = (p.k / 4) - (kblocks - 1) * 32;
+    const int64_t pad_rows = p.meta_rows - p.n_out;
+    const int64_t n_a = kblocks * pad_rows * 16;
+    if (static_cast<int64_t>(j) < n_a) {
+        const int64_t kb = j / (pad_rows * 16), rem = j - kb * pad_rows * 16;
+        p.meta[(kb * p.meta_rows + p.n_out) * 16 + rem] = 0x44;
+    } else {
+        const int64_t tail_first_byte = (tail_groups + 1) / 2;
+        const int64_t jj = j - n_a, per = 16 - tail_first_byte;
+        const int64_t row = jj / per, byte = tail_first_byte + (jj - row * per);
+        p.meta[((kblocks - 1) * p.meta_rows + row) * 16 + byte] = 0x44;
+    }
+}
+
+uint32_t meta_pad_bytes(int64_t n_out, int64_t k) {
+    const int64_t meta_rows = (n_out + 127) / 128 * 128;
+    const int64_t kblocks = (k + 127) / 128;
+    const int64_t tail_groups = (k / 4) - (kblocks - 1) * 32;
+    const int64_t n_a = kblocks * (meta_rows - n_out) * 16;
+    const int64_t n_b = (tail_groups < 32) ? n_out * (16 - (tail_groups + 1) / 2) : 0;
+    return static_cast<uint32_t>(n_a + n_b);
+}
+
+__global__ void __launch_bounds__(256) k_pack_finish_batch(const __grid_constant__ BatchParams bp) {
+    __shared__ uint32_t s_thr[kPackBatchMax];
+    __shared__ uint32_t s_patch[kPackBatchMax + 1], s_quads[kPackBatchMax + 1], s_pad[kPackBatchMax + 1];
+    const int n = bp.n;
+    if (threadIdx.x < n) {
+        const BatchItem &I = bp.it[threadIdx.x];
+        const uint32_t mode = *reinterpret_cast<const uint32_t *>(I.hdr + kPackWsModeOffset);
+        const unsigned listed = *reinterpret_cast<const unsigned *>(I.hdr + kPackWsListCountOffset);
+        s_thr[threadIdx.x] = *reinterpret_cast<const uint32_t *>(I.hdr + kPackWsThrOffset);
+        s_patch[threadIdx.x + 1] = mode == 1u ? (listed < I.list_cap ? listed : I.list_cap) : 0u;
+        s_quads[threadIdx.x + 1] = mode == 2u ? static_cast<uint32_t>(I.p.n_groups >> 2) : 0u;
+        s_pad[threadIdx.x + 1] = I.pad_bytes;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s_patch[0] = s_quads[0] = s_pad[0] = 0u;
+        for (int i = 1; i <= n; ++i) {
+            s_patch[i] += s_patch[i - 1];
+            s_quads[i] += s_quads[i - 1];
+            s_pad[i] += s_pad[i - 1];
+        }
+    }
+    __syncthreads();
+    const uint32_t gtid = blockIdx.x * blockDim.x + threadIdx.x;
+    const uint32_t gstride = gridDim.x * blockDim.x;
+    // 1. listed groups of the matrices whose threshold stayed in the band
+    for (uint32_t x = gtid; x < s_patch[n]; x += gstride) {
+        const int item = batch_bucket(s_patch, n, x);
+        const BatchItem &I = bp.it[item];
+        const int64_t i = I.list[x - s_patch[item]];
+        patch_group(I.p, s_thr[item], i, __ldg(I.p.W + i));
+    }
+    // 2. every quad of the matrices whose threshold left the band (or had no hint)
+    for (uint32_t x = gtid; x < s_quads[n]; x += gstride) {
+        const int item = batch_bucket(s_quads, n, x);
+        const BatchItem &I = bp.it[item];
+        const uint32_t q = x - s_quads[item];
+        float4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = __ldg(I.p.W + 4u * q + j);
+        store_quad(I.p, q, pack_quad(v, s_thr[item], 0u, 0u));
+    }
+    // 3. metadata padding
+    for (uint32_t x = gtid; x < s_pad[n]; x += gstride) {
+        const int item = batch_bucket(s_pad, n, x);
+        meta_pad_at(bp.it[item].p, x - s_pad[item]);
+    }
+}
+
+size_t pack_batch_ws_bytes(const int64_t *n_out, const int64_t *k, int n_items) {
+    size_t b = static_cast<size_t>(n_items) * kPackWsBytes;
+    for (int i = 0; i < n_items; ++i) b += update_list_bytes(n_out[i], k[i]);
+    return b;
+}
+
+cudaError_t launch_pack_update_batch(const PackBatchItemHost *items, int n_items, float eps, void *ws, cudaStream_t s) {
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    // every header first, then the lists: one memset clears all headers
+    cudaError_t err = cudaMemsetAsync(ws, 0, static_cast<size_t>(n_items) * kPackWsBytes, s);
+    if (err != cudaSuccess) return err;
+    uint8_t *lists = w8 + static_cast<size_t>(n_items) * kPackWsBytes;
+    for (int base = 0; base < n_items; base += kPackBatchMax) {
+        const int n = (n_items - base) < kPackBatchMax ? (n_items - base) : kPackBatchMax;
+        BatchParams bp;
+        uint32_t chunks = 0;
+        for (int i = 0; i < n; ++i) {
+            const PackBatchItemHost &h = items[base + i];
+            BatchItem &I = bp.it[i];
+            const int64_t n_el = h.n_out * h.k;
+            I.p.W = reinterpret_cast<const float4 *>(h.W);
+            I.p.n_groups = n_el / 4;
+            I.p.gpr = h.k / 4;
+            I.p.gpr_div = make_fastdiv(static_cast<uint32_t>(h.k / 4));
+            I.p.n_out = h.n_out;
+            I.p.k = h.k;
+            I.p.meta_rows = (h.n_out + 127) / 128 * 128;
+            I.p.thr = nullptr;
+            I.p.gb = h.gb;
+            I.p.vals = reinterpret_cast<uint16_t *>(h.vals);
+            I.p.meta = h.meta;
+            I.p.mask = h.mask;
+            I.gamma = h.gamma;
+            I.hdr = w8 + static_cast<size_t>(base + i) * kPackWsBytes;
+            I.list = reinterpret_cast<uint32_t *>(lists);
+            const size_t lb = update_list_bytes(h.n_out, h.k);
+            I.list_cap = static_cast<uint32_t>(lb / 4);
+            lists += lb;
+            const uint32_t quads = static_cast<uint32_t>(I.p.n_groups / 4);
+            I.chunk0 = chunks;
+            I.nchunks = (quads + kBatchChunkQuads - 1) / kBatchChunkQuads;
+            chunks += I.nchunks;
+            I.pad_bytes = (h.meta && (I.p.meta_rows != h.n_out || (h.k % 128) != 0)) ? meta_pad_bytes(h.n_out, h.k) : 0u;
+            I.n_total = n_el;
+        }
+        bp.n = n;
+        bp.total_chunks = chunks;
+        bp.eps = eps;
+        const unsigned grid = static_cast<unsigned>(num_sms() * 4);
+        k_pack_update_batch<<<grid, 256, 0, s>>>(bp);
+        k_pack_finish_batch<<<grid, 256, 0, s>>>(bp);
+        for (int i = 0; i < n; ++i) {
+            const PackBatchItemHost &h = items[base + i];
+            if (h.dec)
+                k_make_dec<<<grid_for(h.n_out / 16 * (h.k / 64) * 32, 256, 8), 256, 0, s>>>(
+                    h.gb, h.n_out, h.k, reinterpret_cast<uint2 *>(h.dec));
+        }
+    }
+    return cudaGetLastError();
+}
+
 }  // namespace bitnet

@@ -171,6 +171,41 @@ def test_decode_chain_rejects_bad_arguments(lib):
         assert f(arr2, 2, 1, bf, bf, 1e-5, _fake(), ws, None) == want, spec
 
 
+def test_pack_update_batch_rejects_bad_arguments(lib):
+    f = lib.bitnet_pack_nm_update_batch
+    good = _pw(n_out=256, k=256, mma=True)
+    arr = (_abi.BitnetPackItem * 2)()
+    for i in range(2):
+        arr[i].W = 4096
+        arr[i].out = ctypes.pointer(good)
+    ws = lib.bitnet_pack_update_batch_workspace_size(arr, 2)
+    assert ws >= 2 * (256 + 2048) + 2 * 16384 * 4
+    assert f(arr, -1, 1e-5, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(arr, 0, 1e-5, None, 0, None) == _abi.BITNET_OK
+    assert f(None, 2, 1e-5, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(arr, 2, -1.0, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert f(arr, 2, 1e-5, None, ws, None) == _abi.BITNET_ERR_WORKSPACE
+    assert f(arr, 2, 1e-5, _fake(), ws - 4, None) == _abi.BITNET_ERR_WORKSPACE
+    assert f(arr, 2, 1e-5, _fake(4100), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+    cases = [
+        (_pw(n_out=256, k=264, mma=True), 4096, _abi.BITNET_ERR_UNSUPPORTED),    # k % 16
+        (_pw(n_out=256, k=256, n=1, m=4), 4096, _abi.BITNET_ERR_UNSUPPORTED),    # 2:4 only
+        (_pw(n_out=256, k=256, gamma=False), 4096, _abi.BITNET_ERR_INVALID_ARG),
+        (good, None, _abi.BITNET_ERR_INVALID_ARG),                              # null W
+        (good, 4100, _abi.BITNET_ERR_INVALID_ARG),                              # W alignment
+        (_pw(n_out=200, k=256, dec=True), 4096, _abi.BITNET_ERR_INVALID_ARG),    # dec needs n_out % 16
+    ]
+    for st, w, want in cases:
+        arr[1].W = w
+        arr[1].out = ctypes.pointer(st)
+        assert f(arr, 2, 1e-5, _fake(), ws, None) == want, (st.n_out, st.k, w)
+    half = _pw(n_out=256, k=256)
+    half.mma_vals = 16384                                                       # vals without meta
+    arr[1].W = 4096
+    arr[1].out = ctypes.pointer(half)
+    assert f(arr, 2, 1e-5, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG
+
+
 def test_dgrad_rejects_bad_arguments(lib):
     f = lib.bitnet_dgrad
     ws = lib.bitnet_dgrad_workspace_size(256, 256)

@@ -548,6 +548,59 @@ def test_pack_update_matches_pack_over_steps(bn, n_out, k):
         assert upd.gamma.item() == float(g) and np.array_equal(upd.group_bytes.cpu().numpy(), gb)
 
 
+def test_pack_update_batch_matches_single(bn):
+    """The batched per-step pack over mixed shapes (metadata padding for
+    n_out % 128 != 0 and k % 128 != 0, decode layout, mask bits, a one-chunk
+    matrix), over random-walk steps, a jump that leaves the band for one matrix
+    only, and the first call without hints: every matrix bit-identical to
+    bitnet_pack_nm, and the gamma and group bytes to the oracle."""
+    shapes = [(256, 512), (200, 352), (96, 64), (1000, 1360), (3200, 3200), (640, 2560)]
+    Ws = [synth.master_weights(n, k, 0.02, seed=950 + i) for i, (n, k) in enumerate(shapes)]
+    Wd = [dev_f32(W) for W in Ws]
+    outs, masks = [], []
+    for (n, k) in shapes:
+        dec = n % 16 == 0 and k % 64 == 0
+        outs.append(bn.PackedWeights(n, k, dec=dec))      # gamma 0: no hint on the first call
+        masks.append(torch.zeros(n * k // 8, dtype=torch.uint8, device="cuda"))
+    batch = bn.PackBatch([(Wd[i], outs[i], masks[i]) for i in range(len(shapes))], 1e-5)
+    for step in range(5):
+        if step > 0:
+            for i in range(len(shapes)):
+                scale = 5e-3 if (step == 3 and i == 4) else 1e-4   # step 3: matrix 4 jumps out of the band
+                Ws[i] = synth.random_walk_step(Ws[i], scale, seed=100 * step + i)
+                Wd[i].copy_(dev_f32(Ws[i]))
+        batch()
+        torch.cuda.synchronize()
+        assert bn.bitnet_read_device_status(batch.ws) == 0
+        for i, (n, k) in enumerate(shapes):
+            ref = bn.PackedWeights(n, k, dec=outs[i].dec_codes is not None)
+            mask_r = torch.zeros_like(masks[i])
+            bn.bitnet_pack_nm(Wd[i], ref, 1e-5, mask_bits=mask_r)
+            torch.cuda.synchronize()
+            for a, b in zip(_pack_outputs(outs[i], masks[i]), _pack_outputs(ref, mask_r)):
+                assert (a is None and b is None) or np.array_equal(a, b), (step, i)
+            if n * k <= 1 << 20:
+                g, keep, wq, gb = oracle.pack_weights(Ws[i], 1e-5)
+                assert outs[i].gamma.item() == float(g) and np.array_equal(outs[i].group_bytes.cpu().numpy(), gb)
+
+
+def test_pack_update_batch_many_launch_groups(bn):
+    """More matrices than one launch takes (70 > 64)."""
+    n_items = 70
+    Ws = [synth.master_weights(64, 128, 0.02, seed=2000 + i) for i in range(n_items)]
+    Wd = [dev_f32(W) for W in Ws]
+    outs = [bn.PackedWeights(64, 128) for _ in range(n_items)]
+    batch = bn.bitnet_pack_nm_update_batch([(Wd[i], outs[i]) for i in range(n_items)], 1e-5)
+    batch()
+    torch.cuda.synchronize()
+    for i in range(n_items):
+        g, keep, wq, gb = oracle.pack_weights(Ws[i], 1e-5)
+        assert outs[i].gamma.item() == float(g), i
+        assert np.array_equal(outs[i].group_bytes.cpu().numpy(), gb), i
+        dwq, dkeep, _, _ = decode_mma(outs[i].mma_vals.cpu().numpy(), outs[i].mma_meta.cpu().numpy(), 64, 128)
+        assert np.array_equal(dwq, wq), i
+
+
 def test_pack_update_small_list_falls_back(bn):
     """A list with room for one entry overflows; the device then runs the full
     second pass and the result is still exact."""
