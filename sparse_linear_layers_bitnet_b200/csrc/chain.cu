@@ -45,7 +45,7 @@ constexpr int kChainMaxStages = 16;
 
 struct ChainParams {
     ChainOpDev op[kChainMaxOps];
-    int32_t n_ops, T, x_bf16, y_bf16, ns;
+    int32_t n_ops, T, x_bf16, y_bf16, ns, kmax;
     float eps;
     uint32_t *counters;   // [n_ops], zero at launch
     uint32_t *abort;      // grid-wide abort word, zero at launch
@@ -118,6 +118,30 @@ __device__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, volatile int *ab
     }
 }
 
+// Consumer's wait for a filled stage: suspended in the barrier (short hint)
+// rather than spinning; bounded like mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_wait_full(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(2000u)
+            : "memory");
+        if (ok) return true;
+        if (*abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicOr(status, kStatusTimeout);
+            return false;
+        }
+    }
+}
+
 // Wait that ignores the abort flag, up to a deadline (for draining copies in flight).
 __device__ bool mbar_wait_until(uint64_t *bar, uint32_t parity, uint64_t deadline_ns) {
     while (!mbar_try_wait(bar, parity)) {
@@ -140,6 +164,22 @@ __device__ __forceinline__ bool consumer_sync_or(bool v) {
         : "r"(v ? 1u : 0u), "n"(kChainConsumers)
         : "memory");
     return r != 0;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&b)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+                 : "r"(addr)
+                 : "memory");
+}
+
+// adds a row tile's partial sums (four accumulators) into the shared sums and clears them
+__device__ __forceinline__ void chain_flush(int *s_acc, int tile, int lane, int (&acc)[4][4]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        atomicAdd(&s_acc[(tile * 32 + lane) * 4 + q], acc[0][q] + acc[1][q] + acc[2][q] + acc[3][q]);
+        acc[0][q] = acc[1][q] = acc[2][q] = acc[3][q] = 0;
+    }
 }
 
 template <bool BF16>
@@ -188,6 +228,8 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
     float m[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) m[t] = 0.0f;
+    C keep_a, keep_b;   // the first two chunks stay in registers for the second pass
+    keep_a.raw = keep_b.raw = make_uint4(0u, 0u, 0u, 0u);
     {
         int c = ctid, t = 0, i = ctid;
         while (i >= cpr) {
@@ -199,6 +241,10 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
             const int c2 = c + kChainConsumers;
             a.raw = __ldcg(X + c);
             if (c2 < nchunk) b.raw = __ldcg(X + c2);
+            if (c == ctid) {
+                keep_a = a;
+                keep_b = b;
+            }
             const float ma = a.absmax();
 #pragma unroll
             for (int tt = 0; tt < 8; ++tt)
@@ -254,8 +300,13 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
         while (c < nchunk) {
             C a, b;
             const int c2 = c + kChainConsumers;
-            a.raw = __ldcg(X + c);
-            if (c2 < nchunk) b.raw = __ldcg(X + c2);
+            if (c == ctid) {
+                a = keep_a;
+                b = keep_b;
+            } else {
+                a.raw = __ldcg(X + c);
+                if (c2 < nchunk) b.raw = __ldcg(X + c2);
+            }
             a.store_codes(s_xq + t * pitch + i * C::kElems, s_inv[t]);
             i += kChainConsumers;
             while (i >= cpr) {
@@ -290,8 +341,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     uint8_t *ring = smem;
     int *s_acc = reinterpret_cast<int *>(smem + static_cast<size_t>(ns) * kStageBytes);
     int8_t *s_xq = reinterpret_cast<int8_t *>(s_acc + kChainMaxTiles * 128);
+    int8_t *s_zero = s_xq + static_cast<size_t>(T) * static_cast<size_t>(p.kmax + 16);   // 64 zero bytes
 
     for (int i = tid; i < kChainMaxTiles * 128; i += kChainThreads) s_acc[i] = 0;
+    for (int i = tid; i < 64; i += kChainThreads) s_zero[i] = 0;
     if (tid == 0) {
         s_abort = 0;
         for (int s = 0; s < ns; ++s) {
@@ -350,8 +403,6 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     // consumer barriers never miss a thread.
     const int ctid = tid;
     const int warp = ctid >> 5, lane = ctid & 31;
-    const int gid = lane >> 2, tq = lane & 3;
-    const bool tok = gid < T;
     uint32_t it = 0;
     for (int j = 0; j < p.n_ops; ++j) {
         const ChainOpDev &op = p.op[j];
@@ -377,59 +428,76 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                 chain_quantise<false>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, gamma, s_xq, s_red, s_amax,
                                       s_inv, s_scale, ctid);
             consumer_sync();
-            // 3. weight records from the ring: warp w takes records w, w + 16, ...
-            const int8_t *xs = s_xq + (tok ? gid : 0) * (op.k + 16) + 4 * tq;
+            // 3. weight records from the ring: in each stage, warp w takes the
+            //    contiguous records [w n / 16, (w + 1) n / 16).  The B fragments
+            //    (8 token rows x 64 k of int8) come from shared memory with one
+            //    ldmatrix.x4 per record: lane l gives the address of row l % 8
+            //    of matrix l / 8 (a 16-byte segment; rows >= T read zeros).
+            const uint32_t lrow = lane & 7, lmat = lane >> 3;
+            const uint32_t b_base = lrow < static_cast<uint32_t>(T)
+                                        ? smem_u32(s_xq) + lrow * static_cast<uint32_t>(op.k + 16) + 16u * lmat
+                                        : smem_u32(s_zero) + 16u * lmat;
+            const uint32_t b_step = lrow < static_cast<uint32_t>(T) ? 64u : 0u;   // bytes per k-tile
             int cur = -1;
-            int d[4] = {0, 0, 0, 0}, d2[4] = {0, 0, 0, 0};   // alternate records: two independent MMA chains
-            int par = 0;
+            int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
             bool failed = false;
             for (uint32_t off = 0; off < bytes; off += kStageBytes, ++it) {
                 const uint32_t s = it % static_cast<uint32_t>(ns);
-                const bool ok = mbar_wait_bounded(&s_full[s], (it / ns) & 1u, &s_abort, p.status);
+                const bool ok = mbar_wait_full(&s_full[s], (it / ns) & 1u, &s_abort, p.status);
                 if (!__all_sync(0xffffffffu, ok)) {
                     failed = true;
                     break;
                 }
                 const int nrec = static_cast<int>(((bytes - off) < kStageBytes ? (bytes - off) : kStageBytes) >> 8);
-                const int r0 = static_cast<int>(off >> 8) + warp;
-                int tile = r0 / ktiles;
-                int kt = r0 - tile * ktiles;
-                const uint2 *rec = reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(s) * kStageBytes) + lane;
-                for (int i = warp; i < nrec; i += kChainConsumerWarps) {
-                    if (tile != cur) {
-                        if (cur >= 0) {
-#pragma unroll
-                            for (int q = 0; q < 4; ++q) atomicAdd(&s_acc[(cur * 32 + lane) * 4 + q], d[q] + d2[q]);
+                const int i0 = (warp * nrec) / kChainConsumerWarps, i1 = ((warp + 1) * nrec) / kChainConsumerWarps;
+                if (i0 < i1) {
+                    const int r0 = static_cast<int>(off >> 8) + i0;
+                    int tile = r0 / ktiles;
+                    int kt = r0 - tile * ktiles;
+                    const uint2 *rec = reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(s) * kStageBytes) + lane;
+                    int i = i0;
+                    while (i < i1) {
+                        if (tile != cur) {
+                            if (cur >= 0) chain_flush(s_acc, cur, lane, acc);
+                            cur = tile;
                         }
-                        cur = tile;
+                        if (i + 4 <= i1 && kt + 4 <= ktiles) {
+                            // four records of one row tile: all loads first, then the MMAs
+                            uint2 w[4];
+                            uint32_t bf[4][4];
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) d[q] = d2[q] = 0;
-                    }
-                    const uint2 w = rec[i * 32];
-                    uint32_t a[4], b[4];
+                            for (int u = 0; u < 4; ++u) w[u] = rec[(i + u) * 32];
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj)
-                        b[jj] = tok ? *reinterpret_cast<const uint32_t *>(xs + kt * 64 + 16 * jj) : 0u;
+                            for (int u = 0; u < 4; ++u) ldsm_x4(bf[u], b_base + static_cast<uint32_t>(kt + u) * b_step);
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) a[r] = expand_codes(w.x, r);
-                    if (par)
-                        mma_sp_m16n8k64(d2, a, b, w.y);
-                    else
-                        mma_sp_m16n8k64(d, a, b, w.y);
-                    par ^= 1;
-                    kt += kChainConsumerWarps;
-                    while (kt >= ktiles) {
-                        kt -= ktiles;
-                        ++tile;
+                            for (int u = 0; u < 4; ++u) {
+                                uint32_t a4[4];
+#pragma unroll
+                                for (int r = 0; r < 4; ++r) a4[r] = expand_codes(w[u].x, r);
+                                mma_sp_m16n8k64(acc[u], a4, bf[u], w[u].y);
+                            }
+                            i += 4;
+                            kt += 4;
+                        } else {
+                            const uint2 w = rec[i * 32];
+                            uint32_t bf[4], a4[4];
+                            ldsm_x4(bf, b_base + static_cast<uint32_t>(kt) * b_step);
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) a4[r] = expand_codes(w.x, r);
+                            mma_sp_m16n8k64(acc[0], a4, bf, w.y);
+                            i += 1;
+                            kt += 1;
+                        }
+                        if (kt == ktiles) {
+                            kt = 0;
+                            ++tile;
+                        }
                     }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[s]);
             }
-            if (cur >= 0) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) atomicAdd(&s_acc[(cur * 32 + lane) * 4 + q], d[q] + d2[q]);
-            }
+            if (cur >= 0) chain_flush(s_acc, cur, lane, acc);
             if (consumer_sync_or(failed || s_abort != 0)) break;
             // 4. dequantise and store this CTA's rows; clear the partial sums
             for (int e = ctid; e < ntile * 128; e += kChainConsumers) {
@@ -472,7 +540,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
 
 size_t chain_smem_bytes(int ns, int64_t T, int64_t kmax) {
     return static_cast<size_t>(ns) * kStageBytes + static_cast<size_t>(kChainMaxTiles) * 128 * 4 +
-           static_cast<size_t>(T) * static_cast<size_t>(kmax + 16);
+           static_cast<size_t>(T) * static_cast<size_t>(kmax + 16) + 64;
 }
 
 int chain_stages(int64_t T, int64_t kmax) {
@@ -508,6 +576,7 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         p.x_bf16 = x_bf16 ? 1 : 0;
         p.y_bf16 = y_bf16 ? 1 : 0;
         p.ns = ns;
+        p.kmax = static_cast<int32_t>(kmax);
         p.eps = eps;
         p.status = reinterpret_cast<uint32_t *>(w8 + kStatusOffset);
         p.abort = reinterpret_cast<uint32_t *>(w8 + kChainAbortOffset);

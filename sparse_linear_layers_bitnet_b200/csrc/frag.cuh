@@ -15,9 +15,10 @@ __device__ __forceinline__ int8_t quant_code(float x, float s) {
 }
 
 __device__ __forceinline__ uint32_t expand_codes(uint32_t codes, int r) {
-    // bytes of t hold 2-bit codes {0: 0, 1: +1, 3: -1}; int8 = (t & 1) | (t & 2) * 0x7f
+    // bytes of t hold 2-bit codes {0: 0, 1: +1, 3: -1}; int8 = t + (t & 2) * 0x7e
+    // (3 -> 3 + 252 = 0xff, 1 -> 1, 0 -> 0; no byte carries into the next)
     const uint32_t t = (codes >> (2 * r)) & 0x03030303u;
-    return (t & 0x01010101u) + (t & 0x02020202u) * 0x7fu;
+    return (t & 0x02020202u) * 0x7eu + t;
 }
 
 __device__ __forceinline__ void mma_sp_m16n8k64(int (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[4],
