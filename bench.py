@@ -55,7 +55,7 @@ def parse_args():
     ap.add_argument("--preroll-s", type=float, default=1.0, help="untimed warm-up seconds before timing")
     ap.add_argument("--tokens", type=int, default=1, help="decode batch (1..8)")
     ap.add_argument("--layers", type=int, default=30)
-    ap.add_argument("--decode", choices=["chain", "fused", "unfused"], default="unfused",
+    ap.add_argument("--decode", choices=["chain", "fused", "unfused"], default="chain",
                     help="decode step: one persistent launch for all projections (chain), one fused "
                          "quant+GEMV launch per projection (fused), or quant_act + GEMV per projection")
     ap.add_argument("--no-rows", action="store_true", help="skip the sub-measurements of the other rows")

@@ -234,6 +234,12 @@ bitnet_status bitnet_sparse_linear(const int8_t *Xq, const float *absmax, const 
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
+static bool chain_fits(int64_t T, int64_t kmax) {
+    int ns = 0;
+    uint32_t stage = 0;
+    return bitnet::chain_ring(T, kmax, &ns, &stage);
+}
+
 size_t bitnet_quant_linear_workspace_size(int64_t T, int64_t K) {
     if (T <= 0 || K <= 0) return bitnet::kLinearWsBytes;
     return bitnet::kLinearWsBytes + align256(static_cast<size_t>(T) * static_cast<size_t>(K)) +
@@ -260,7 +266,7 @@ bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool xb = x_dtype == BITNET_BF16, yb = y_dtype == BITNET_BF16;
     if (T <= 8 && W->dec_codes && n_out % 16 == 0 && k % 64 == 0 && n_out / 16 <= bitnet::kChainMaxTiles * bitnet::num_sms() &&
-        bitnet::chain_stages(T, k) >= 2 && ws_bytes >= bitnet_decode_chain_workspace_size(1)) {
+        chain_fits(T, k) && ws_bytes >= bitnet_decode_chain_workspace_size(1)) {
         if (!aligned(W->dec_codes, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: dec_codes alignment");
         bitnet::ChainOpDev op = {X, W->dec_codes, W->gamma, Y, acc_out, xq_out, absmax_out,
                                  static_cast<int32_t>(n_out), static_cast<int32_t>(k), 0, 0};
@@ -324,7 +330,7 @@ bitnet_status bitnet_decode_chain(const bitnet_chain_op *ops, int32_t n_ops, int
         dev[static_cast<size_t>(i)] = {o.X, W->dec_codes, W->gamma, o.Y, o.acc_out, o.xq_out, o.absmax_out,
                                        static_cast<int32_t>(W->n_out), static_cast<int32_t>(W->k), o.wait_prev, 0};
     }
-    if (bitnet::chain_stages(T, kmax) < 2)
+    if (!chain_fits(T, kmax))
         return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: T * (k + 16) leaves no room for two weight stages");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return cuda_status(bitnet::launch_decode_chain(dev.data(), n_ops, T, x_dtype == BITNET_BF16, y_dtype == BITNET_BF16,

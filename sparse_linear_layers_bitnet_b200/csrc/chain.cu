@@ -14,7 +14,7 @@
 // one CTA for the whole chain:
 //  * a producer warp streams the CTA's share of every projection's packed
 //    weights (a contiguous byte range of the decode layout) into a ring of
-//    16 KB shared-memory stages with bulk asynchronous copies.  Weights do not
+//    64, 32 or 16 KB shared-memory stages with bulk asynchronous copies.  Weights do not
 //    depend on activations, so the stream runs ahead across projection
 //    boundaries, limited only by free stages;
 //  * sixteen consumer warps, per projection: wait until every CTA has finished
@@ -40,12 +40,12 @@ namespace bitnet {
 constexpr int kChainConsumerWarps = 16;
 constexpr int kChainConsumers = kChainConsumerWarps * 32;
 constexpr int kChainThreads = kChainConsumers + 32;
-constexpr uint32_t kStageBytes = 16384;            // 64 weight records of 256 bytes
 constexpr int kChainMaxStages = 16;
 
 struct ChainParams {
     ChainOpDev op[kChainMaxOps];
     int32_t n_ops, T, x_bf16, y_bf16, ns, kmax;
+    uint32_t stage_bytes;   // ring stage size: 16, 32 or 64 KB (a multiple of 256)
     float eps;
     uint32_t *counters;   // [n_ops], zero at launch
     uint32_t *abort;      // grid-wide abort word, zero at launch
@@ -55,13 +55,15 @@ struct ChainParams {
 // Row tiles [t0, t1) of projection j for this CTA.  The CTA's share index v
 // is its block index rotated by 61 j; share v is [v R / G, (v + 1) R / G).
 // Share G - 1 is never empty when R >= 1.
+// 32-bit arithmetic: v R < 2^31 since R <= 32 G (checked on the host) and G is
+// the number of SMs.
 __device__ __forceinline__ int chain_tiles(int j, int rows16, int &t0, int &t1) {
-    const int G = static_cast<int>(gridDim.x);
-    int v = static_cast<int>(blockIdx.x) + (j * 61) % G;
+    const uint32_t G = gridDim.x;
+    uint32_t v = blockIdx.x + (static_cast<uint32_t>(j) * 61u) % G;
     if (v >= G) v -= G;
-    t0 = static_cast<int>((static_cast<int64_t>(v) * rows16) / G);
-    t1 = static_cast<int>((static_cast<int64_t>(v + 1) * rows16) / G);
-    return v;
+    t0 = static_cast<int>((v * static_cast<uint32_t>(rows16)) / G);
+    t1 = static_cast<int>(((v + 1u) * static_cast<uint32_t>(rows16)) / G);
+    return static_cast<int>(v);
 }
 
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kChainConsumers) : "memory"); }
@@ -339,7 +341,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     const uint32_t G = gridDim.x;
     // dynamic shared memory: ring [ns][16 KB] | partial sums [kChainMaxTiles][32][4] int | int8 rows
     uint8_t *ring = smem;
-    int *s_acc = reinterpret_cast<int *>(smem + static_cast<size_t>(ns) * kStageBytes);
+    const uint32_t stage_bytes = p.stage_bytes;
+    int *s_acc = reinterpret_cast<int *>(smem + static_cast<size_t>(ns) * stage_bytes);
     int8_t *s_xq = reinterpret_cast<int8_t *>(s_acc + kChainMaxTiles * 128);
     int8_t *s_zero = s_xq + static_cast<size_t>(T) * static_cast<size_t>(p.kmax + 16);   // 64 zero bytes
 
@@ -377,16 +380,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                 for (size_t l = static_cast<size_t>(blockIdx.x) * 128; l < xbytes; l += static_cast<size_t>(gridDim.x) * 128)
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t *>(op.X) + l));
             }
-            for (uint32_t off = 0; off < bytes; off += kStageBytes, ++it) {
+            for (uint32_t off = 0; off < bytes; off += stage_bytes, ++it) {
                 const uint32_t s = it % static_cast<uint32_t>(ns);
                 if (it >= static_cast<uint32_t>(ns) &&
                     !mbar_wait_sleep(&s_empty[s], ((it / ns) - 1u) & 1u, &s_abort, p.status)) {
                     ok = false;
                     break;
                 }
-                const uint32_t n = (bytes - off) < kStageBytes ? (bytes - off) : kStageBytes;
+                const uint32_t n = (bytes - off) < stage_bytes ? (bytes - off) : stage_bytes;
                 mbar_arrive_expect_tx(&s_full[s], n);
-                bulk_load(ring + static_cast<size_t>(s) * kStageBytes, src + off, n, &s_full[s]);
+                bulk_load(ring + static_cast<size_t>(s) * stage_bytes, src + off, n, &s_full[s]);
             }
         }
         // drain: every issued stage must have landed before the CTA may exit
@@ -441,20 +444,20 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             int cur = -1;
             int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
             bool failed = false;
-            for (uint32_t off = 0; off < bytes; off += kStageBytes, ++it) {
+            for (uint32_t off = 0; off < bytes; off += stage_bytes, ++it) {
                 const uint32_t s = it % static_cast<uint32_t>(ns);
                 const bool ok = mbar_wait_full(&s_full[s], (it / ns) & 1u, &s_abort, p.status);
                 if (!__all_sync(0xffffffffu, ok)) {
                     failed = true;
                     break;
                 }
-                const int nrec = static_cast<int>(((bytes - off) < kStageBytes ? (bytes - off) : kStageBytes) >> 8);
+                const int nrec = static_cast<int>(((bytes - off) < stage_bytes ? (bytes - off) : stage_bytes) >> 8);
                 const int i0 = (warp * nrec) / kChainConsumerWarps, i1 = ((warp + 1) * nrec) / kChainConsumerWarps;
                 if (i0 < i1) {
                     const int r0 = static_cast<int>(off >> 8) + i0;
-                    int tile = r0 / ktiles;
+                    int tile = static_cast<int>(static_cast<uint32_t>(r0) / static_cast<uint32_t>(ktiles));
                     int kt = r0 - tile * ktiles;
-                    const uint2 *rec = reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(s) * kStageBytes) + lane;
+                    const uint2 *rec = reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(s) * stage_bytes) + lane;
                     int i = i0;
                     while (i < i1) {
                         if (tile != cur) {
@@ -538,23 +541,37 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     }
 }
 
-size_t chain_smem_bytes(int ns, int64_t T, int64_t kmax) {
-    return static_cast<size_t>(ns) * kStageBytes + static_cast<size_t>(kChainMaxTiles) * 128 * 4 +
+size_t chain_smem_bytes(int ns, uint32_t stage_bytes, int64_t T, int64_t kmax) {
+    return static_cast<size_t>(ns) * stage_bytes + static_cast<size_t>(kChainMaxTiles) * 128 * 4 +
            static_cast<size_t>(T) * static_cast<size_t>(kmax + 16) + 64;
 }
 
-int chain_stages(int64_t T, int64_t kmax) {
-    const size_t fixed = chain_smem_bytes(0, T, kmax);
-    if (fixed >= kChainMaxSmem) return 0;
-    size_t ns = (kChainMaxSmem - fixed) / kStageBytes;
-    if (ns > static_cast<size_t>(kChainMaxStages)) ns = kChainMaxStages;
-    return static_cast<int>(ns);
+// Ring geometry: the largest stage (64, 32 or 16 KB) that leaves three stages
+// (64 KB) or two (smaller) next to the activation rows.  Larger stages mean
+// fewer barrier waits and longer record runs per warp.  False when not even
+// two 16 KB stages fit.
+bool chain_ring(int64_t T, int64_t kmax, int *ns_out, uint32_t *stage_out) {
+    const size_t fixed = chain_smem_bytes(0, 0, T, kmax);
+    if (fixed >= kChainMaxSmem) return false;
+    const uint32_t sizes[3] = {65536u, 32768u, 16384u};
+    const int need[3] = {3, 2, 2};
+    for (int i = 0; i < 3; ++i) {
+        size_t ns = (kChainMaxSmem - fixed) / sizes[i];
+        if (ns > static_cast<size_t>(kChainMaxStages)) ns = kChainMaxStages;
+        if (static_cast<int>(ns) >= need[i]) {
+            *ns_out = static_cast<int>(ns);
+            *stage_out = sizes[i];
+            return true;
+        }
+    }
+    return false;
 }
 
 cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
                                 int64_t kmax, void *ws, cudaStream_t s) {
-    const int ns = chain_stages(T, kmax);
-    if (ns < 2) return cudaErrorInvalidValue;
+    int ns = 0;
+    uint32_t stage_bytes = 0;
+    if (!chain_ring(T, kmax, &ns, &stage_bytes)) return cudaErrorInvalidValue;
     static bool attr_done[2] = {false, false};
     if (!attr_done[x_bf16 ? 1 : 0]) {
         cudaError_t e = x_bf16 ? cudaFuncSetAttribute(k_decode_chain<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -576,6 +593,7 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         p.x_bf16 = x_bf16 ? 1 : 0;
         p.y_bf16 = y_bf16 ? 1 : 0;
         p.ns = ns;
+        p.stage_bytes = stage_bytes;
         p.kmax = static_cast<int32_t>(kmax);
         p.eps = eps;
         p.status = reinterpret_cast<uint32_t *>(w8 + kStatusOffset);
@@ -587,7 +605,7 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(num_sms()));
         cfg.blockDim = dim3(kChainThreads);
-        cfg.dynamicSmemBytes = chain_smem_bytes(ns, T, kmax);
+        cfg.dynamicSmemBytes = chain_smem_bytes(ns, stage_bytes, T, kmax);
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;

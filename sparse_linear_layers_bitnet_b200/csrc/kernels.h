@@ -86,8 +86,8 @@ constexpr int kChainMaxTiles = 32;                 // 16-row tiles per CTA per p
 constexpr size_t kChainMaxSmem = 227 * 1024 - 1024;   // dynamic shared memory (static use < 1 KB)
 constexpr size_t kChainAbortOffset = 4;            // workspace: grid abort word
 constexpr size_t kChainCountersOffset = 256;       // workspace: one counter per projection
-size_t chain_smem_bytes(int ns, int64_t T, int64_t kmax);
-int chain_stages(int64_t T, int64_t kmax);
+size_t chain_smem_bytes(int ns, uint32_t stage_bytes, int64_t T, int64_t kmax);
+bool chain_ring(int64_t T, int64_t kmax, int *ns, uint32_t *stage_bytes);
 cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
                                 int64_t kmax, void *ws, cudaStream_t s);
 
