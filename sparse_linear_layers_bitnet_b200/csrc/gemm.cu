@@ -345,61 +345,87 @@ cudaError_t launch_gemm_sp(const int8_t *Xq, const float *amax, const float *gam
 }
 
 // Wq^T in bf16: wt[k, n] = code of weight (n, k), from the canonical group bytes.
-// One CTA per 64 (n) x 64 (k) tile: 64 rows of 16 group bytes come in with one
-// 16-byte load each, and the transposed tile leaves in 16-byte stores (8 bf16),
-// so both the 0.25-byte reads and the 2-byte writes per weight are coalesced.
+// Persistent CTAs walk 64 (n) x 64 (k) tiles.  Per tile, 64 threads bring the
+// 64 rows of 16 group bytes in with one 16-byte load each (issued one tile
+// ahead, so the load overlaps the previous tile's work) into a padded shared
+// tile.  Thread (g, c) then decodes the four group bytes of rows n = 4c..4c+3
+// at group g once into 2-bit codes per position and writes the four output
+// rows k = 4g..4g+3 of those four columns as 8-byte stores; sixteen threads
+// cover one 128-byte output row segment.
+constexpr int kExpandRowWords = 17;   // 68-byte shared rows: the 16 column groups fall in different banks
+
+__device__ __forceinline__ uint4 expand_load(const uint8_t *__restrict__ gb, int64_t n_out, int64_t k, int64_t n,
+                                            int64_t k0) {
+    uint4 v = make_uint4(0x04040404u, 0x04040404u, 0x04040404u, 0x04040404u);   // idx (0,1), codes 0
+    if (n < n_out) {
+        const uint8_t *src = gb + n * (k / 4) + k0 / 4;
+        if (k0 + 64 <= k && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+            v = __ldg(reinterpret_cast<const uint4 *>(src));
+        } else {
+            uint8_t tmp[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) tmp[j] = (k0 + 4 * j < k) ? src[j] : static_cast<uint8_t>(0x04);
+            v = *reinterpret_cast<const uint4 *>(tmp);
+        }
+    }
+    return v;
+}
+
+// 2-bit codes of the four positions of a group byte: code of position p at bits 2p..2p+1
+__device__ __forceinline__ uint32_t group_codes4(uint32_t b) {
+    const uint32_t i0 = b & 3u, i1 = (b >> 2) & 3u;
+    return (((b >> 4) & 3u) << (2 * i0)) | ((b >> 6) << (2 * i1));
+}
+
+// bf16 bits of a 2-bit code {0: 0, 1: +1 = 0x3f80, 3: -1 = 0xbf80}
+__device__ __forceinline__ uint32_t code_bf16(uint32_t code) { return (code & 1u) * 0x3f80u | ((code & 2u) << 14); }
+
 __global__ void __launch_bounds__(256) k_expand_wt(const uint8_t *__restrict__ gb, int64_t n_out, int64_t k,
                                                    __nv_bfloat16 *__restrict__ wt) {
-    __shared__ __align__(16) uint8_t s_gb[64][16];
-    const int64_t n0 = static_cast<int64_t>(blockIdx.y) * 64, k0 = static_cast<int64_t>(blockIdx.x) * 64;
-    const int64_t gpr = k / 4;
+    __shared__ __align__(16) uint32_t s_gb[64 * kExpandRowWords];
     const int tid = threadIdx.x;
-    if (tid < 64) {
-        const int64_t n = n0 + tid;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (n < n_out) {
-            const uint8_t *src = gb + n * gpr + k0 / 4;
-            if (k0 + 64 <= k && (reinterpret_cast<uintptr_t>(src) & 15) == 0) {
-                v = __ldg(reinterpret_cast<const uint4 *>(src));
-            } else {
-                uint8_t tmp[16];
+    const int64_t ktiles = (k + 63) / 64, ntiles = (n_out + 63) / 64;
+    const int64_t tiles = ktiles * ntiles;
+    int64_t tile = blockIdx.x;
+    uint4 v;
+    if (tid < 64 && tile < tiles) v = expand_load(gb, n_out, k, (tile / ktiles) * 64 + tid, (tile % ktiles) * 64);
+    const int g = tid >> 4, c = tid & 15;
+    for (; tile < tiles; tile += gridDim.x) {
+        const int64_t n0 = (tile / ktiles) * 64, k0 = (tile % ktiles) * 64;
+        __syncthreads();   // the previous tile's reads of s_gb are done
+        if (tid < 64) {
+            uint32_t *row = s_gb + tid * kExpandRowWords;
+            row[0] = v.x;
+            row[1] = v.y;
+            row[2] = v.z;
+            row[3] = v.w;
+        }
+        __syncthreads();
+        const int64_t next = tile + gridDim.x;
+        if (tid < 64 && next < tiles) v = expand_load(gb, n_out, k, (next / ktiles) * 64 + tid, (next % ktiles) * 64);
+        // four group bytes: rows 4c + i, group g
+        uint32_t cd[4];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) tmp[j] = (k0 + 4 * j < k) ? src[j] : static_cast<uint8_t>(0x04);
-                v = *reinterpret_cast<const uint4 *>(tmp);
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t word = s_gb[(4 * c + i) * kExpandRowWords + (g >> 2)];
+            cd[i] = group_codes4((word >> (8 * (g & 3))) & 0xffu);
+        }
+        const int64_t nb = n0 + 4 * c;
+#pragma unroll
+        for (int pos = 0; pos < 4; ++pos) {
+            const int64_t kk = k0 + 4 * g + pos;
+            if (kk >= k) break;
+            uint32_t h[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) h[i] = code_bf16((cd[i] >> (2 * pos)) & 3u);
+            __nv_bfloat16 *dst = wt + kk * n_out + nb;
+            if (nb + 4 <= n_out) {
+                *reinterpret_cast<uint2 *>(dst) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+            } else {
+                for (int i = 0; i < 4; ++i)
+                    if (nb + i < n_out) reinterpret_cast<uint16_t *>(dst)[i] = static_cast<uint16_t>(h[i]);
             }
         }
-        *reinterpret_cast<uint4 *>(s_gb[tid]) = v;
-    }
-    __syncthreads();
-    // thread (r, c): output row k0 + r, columns n0 + 16c .. +15
-    const int r = tid >> 2, c = tid & 3;
-    const int64_t kk = k0 + r;
-    if (kk >= k) return;
-    const int grp = r >> 2, pos = r & 3;
-    uint32_t h[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        uint32_t pair = 0;
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const uint32_t b = s_gb[16 * c + 2 * j + e][grp];
-            const uint32_t i0 = b & 3u, i1 = (b >> 2) & 3u;
-            const uint32_t code = (static_cast<uint32_t>(pos) == i0) ? ((b >> 4) & 3u)
-                                  : (static_cast<uint32_t>(pos) == i1) ? ((b >> 6) & 3u) : 0u;
-            // bf16 bits: +1 = 0x3f80, -1 = 0xbf80, 0 = 0
-            const uint32_t bits = code == 1u ? 0x3f80u : (code == 3u ? 0xbf80u : 0u);
-            pair |= bits << (16 * e);
-        }
-        h[j] = pair;
-    }
-    const int64_t nb = n0 + 16 * c;
-    __nv_bfloat16 *dst = wt + kk * n_out + nb;
-    if (nb + 16 <= n_out && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
-        reinterpret_cast<uint4 *>(dst)[0] = make_uint4(h[0], h[1], h[2], h[3]);
-        reinterpret_cast<uint4 *>(dst)[1] = make_uint4(h[4], h[5], h[6], h[7]);
-    } else {
-        for (int j = 0; j < 16; ++j)
-            if (nb + j < n_out) reinterpret_cast<uint16_t *>(dst)[j] = static_cast<uint16_t>(h[j >> 1] >> (16 * (j & 1)));
     }
 }
 
@@ -407,8 +433,9 @@ cudaError_t launch_dgrad(const void *dY, const float *gamma, const uint8_t *gb, 
                          void *dX, bool dx_bf16, void *ws, cudaStream_t s) {
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     __nv_bfloat16 *wt = reinterpret_cast<__nv_bfloat16 *>(w8 + kDgradWsHeader);
-    dim3 eg(static_cast<unsigned>((k + 63) / 64), static_cast<unsigned>((n_out + 63) / 64));
-    k_expand_wt<<<eg, 256, 0, s>>>(gb, n_out, k, wt);
+    const int64_t tiles = ((k + 63) / 64) * ((n_out + 63) / 64);
+    const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+    k_expand_wt<<<static_cast<unsigned>(tiles < cap ? tiles : cap), 256, 0, s>>>(gb, n_out, k, wt);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (T > 128)   // CTA-pair persistent kernel (gemm2.cu)
