@@ -612,38 +612,52 @@ struct QuadOut {
     uint32_t band;    // bit j: group j has a kept magnitude in [band_lo, band_hi]
 };
 
-__device__ __forceinline__ void one_group(const float4 v, uint32_t thr, uint32_t band_lo, uint32_t band_hi,
-                                          uint32_t &gbyte, uint32_t &vals16, uint32_t &nib, uint32_t &keep,
-                                          uint32_t &in_band) {
-    const uint32_t b[4] = {__float_as_uint(v.x), __float_as_uint(v.y), __float_as_uint(v.z), __float_as_uint(v.w)};
-    const uint32_t mag[4] = {b[0] & 0x7fffffffu, b[1] & 0x7fffffffu, b[2] & 0x7fffffffu, b[3] & 0x7fffffffu};
-    keep = top2_of_4(mag);
-    const uint32_t i0 = __ffs(keep) - 1, i1 = 31 - __clz(keep);
-    const uint32_t b0 = i0 == 0 ? b[0] : (i0 == 1 ? b[1] : b[2]);   // i0 <= 2
-    const uint32_t b1 = i1 == 3 ? b[3] : (i1 == 2 ? b[2] : b[1]);   // i1 >= 1
-    const uint32_t m0 = b0 & 0x7fffffffu, m1 = b1 & 0x7fffffffu;
-    const uint32_t nz0 = m0 >= thr, nz1 = m1 >= thr;
-    const uint32_t s0 = b0 >> 31, s1 = b1 >> 31;
-    const uint32_t c0 = nz0 ? (s0 ? 3u : 1u) : 0u, c1 = nz1 ? (s1 ? 3u : 1u) : 0u;
-    nib = i0 | (i1 << 2);
+// One group of four: the two kept positions by a tournament (pair winners,
+// then the final; the runner-up is the final's loser or the champion's pair
+// partner; every comparison is >= so that ties go to the lower position, the
+// same selection as top2_of_4), then codes against thr, group byte, values,
+// metadata nibble and whether a kept magnitude lies in [band_lo, band_lo + band_span].
+__device__ __forceinline__ void one_group(const float4 v, uint32_t thr, uint32_t band_lo, uint32_t band_span,
+                                          uint32_t &gbyte, uint32_t &vals16, uint32_t &nib, uint32_t &in_band) {
+    const uint32_t b0 = __float_as_uint(v.x), b1 = __float_as_uint(v.y), b2 = __float_as_uint(v.z),
+                   b3 = __float_as_uint(v.w);
+    const uint32_t m0 = b0 & 0x7fffffffu, m1 = b1 & 0x7fffffffu, m2 = b2 & 0x7fffffffu, m3 = b3 & 0x7fffffffu;
+    const bool pa = m0 >= m1, pb = m2 >= m3;                       // pair winners: 0 / 2 on ties
+    const uint32_t wAm = pa ? m0 : m1, lAm = pa ? m1 : m0, wBm = pb ? m2 : m3, lBm = pb ? m3 : m2;
+    const bool fa = wAm >= wBm;                                    // champion from the pair (0, 1)
+    const bool k01 = fa && lAm >= wBm;                             // kept {0, 1}
+    const bool k23 = !fa && !(wAm >= lBm);                         // kept {2, 3}
+    const uint32_t wA = pa ? b0 : b1, wB = pb ? b2 : b3;           // otherwise kept: the two pair winners
+    const uint32_t x0 = k01 ? b0 : (k23 ? b2 : wA), x1 = k01 ? b1 : (k23 ? b3 : wB);
+    nib = k01 ? 0x4u : (k23 ? 0xeu : ((pa ? 0u : 1u) | ((pb ? 2u : 3u) << 2)));
+    const uint32_t y0 = x0 & 0x7fffffffu, y1 = x1 & 0x7fffffffu;
+    const uint32_t c0 = y0 >= thr ? ((x0 >> 30) & 2u) | 1u : 0u;   // {0, 1: +1, 3: -1}
+    const uint32_t c1 = y1 >= thr ? ((x1 >> 30) & 2u) | 1u : 0u;
     gbyte = nib | (c0 << 4) | (c1 << 6);
-    vals16 = (nz0 ? (s0 ? 0xffu : 0x01u) : 0u) | ((nz1 ? (s1 ? 0xffu : 0x01u) : 0u) << 8);
-    in_band = ((m0 >= band_lo && m0 <= band_hi) || (m1 >= band_lo && m1 <= band_hi)) ? 1u : 0u;
+    vals16 = ((c0 & 2u) * 0x7eu + c0) | (((c1 & 2u) * 0x7eu + c1) << 8);   // int8 +1 / -1 / 0
+    in_band = (y0 - band_lo <= band_span || y1 - band_lo <= band_span) ? 1u : 0u;
 }
 
+// band: [band_lo, band_hi]; band_hi < band_lo (no hint) lists nothing
 __device__ __forceinline__ QuadOut pack_quad(const float4 (&v)[4], uint32_t thr, uint32_t band_lo, uint32_t band_hi) {
     QuadOut o;
     o.gb = o.vlo = o.vhi = o.meta = o.mask = o.band = 0u;
+    const uint32_t span = band_hi - band_lo;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        uint32_t gbyte, vals16, nib, keep, inb;
-        one_group(v[j], thr, band_lo, band_hi, gbyte, vals16, nib, keep, inb);
+        uint32_t gbyte, vals16, nib, inb;
+        one_group(v[j], thr, band_lo, span, gbyte, vals16, nib, inb);
         o.gb |= gbyte << (8 * j);
         if (j < 2) o.vlo |= vals16 << (16 * j);
         else o.vhi |= vals16 << (16 * (j - 2));
         o.meta |= nib << (4 * j);
-        o.mask |= keep << (4 * j);
         o.band |= inb << j;
+    }
+    // keep bits of the four groups from their metadata nibbles
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const uint32_t nb = (o.meta >> (4 * j)) & 0xfu;
+        o.mask |= ((1u << (nb & 3u)) | (1u << (nb >> 2))) << (4 * j);
     }
     return o;
 }
