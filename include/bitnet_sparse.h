@@ -178,6 +178,50 @@ bitnet_status bitnet_pack_nm_update_batch(const bitnet_pack_item *items, int32_t
                                           void *ws, size_t ws_bytes, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_pack_6of8_windows - 6:8 masked ternary weights as 2:4 windows.
+ *
+ * "Sparse-BitNet" (gist.science), section 4 "Resultaten": the method trains
+ * at 6:8 (top-6 |W| of every 8 consecutive weights of a row).  "Is 2:4
+ * Sparsity Still Worth It? ..." (thelatestinai.com), its SlideSparse entry:
+ * a 6:8 block is rewritten without loss as three overlapping 4-wide windows
+ * (at positions 0, 2 and 4 of the block), each 2:4-compliant, so the 2:4
+ * tensor cores can run it.  Kept positions go, in increasing order, to the
+ * leftmost window that covers them and has a free slot (this always places
+ * all six).  gamma is the absmean of the dense W as for 2:4; ties in the mask
+ * go to the lower position.
+ *
+ *   W          [n_out x k] fp32 masters, 16-byte aligned, k % 64 == 0.
+ *   k          columns of W (the 6:8 width).
+ *   out        window-layout packed weights: out->n_out rows, out->k == k/2*3,
+ *              n = 2, m = 4.  group_bytes required; mma_vals + mma_meta and
+ *              dec_codes (n_out % 16 == 0 and k % 128 == 0) optional; they are
+ *              exactly the layouts bitnet_pack_nm writes for a 2:4 matrix of
+ *              width k/2*3.
+ *   mask_bits  [n_out * k / 8] or NULL: the 6:8 keep bits over the original k.
+ *   ws         >= bitnet_pack_workspace_size(n_out, k) bytes.
+ * bitnet_sparse_linear(Xl, absmax, out, ...) with Xl from
+ * bitnet_quant_act_lift_6of8 then computes the 6:8 product exactly.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_pack_6of8_windows(const float *W, int64_t k, float eps, bitnet_packed_w *out,
+                                       uint8_t *mask_bits, void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_quant_act_lift_6of8 - per-token int8 quantisation with the
+ * activation layout of bitnet_pack_6of8_windows.
+ *
+ * Same scale and codes as bitnet_quant_act ("BitNet b1.58 ...", section "The
+ * mechanism"); every block of 8 codes q[8b .. 8b+7] is written as the 12
+ * codes of its three windows: q[8b .. 8b+3], q[8b+2 .. 8b+5], q[8b+4 .. 8b+7].
+ *
+ *   X       [T, K] fp32 or bf16, 16-byte aligned, K % 8 == 0.
+ *   Xl      [T, K/2*3] int8 out, 16-byte aligned.   absmax [T] fp32 out.
+ * Errors: INVALID_ARG, CUDA.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_quant_act_lift_6of8(const void *X, bitnet_dtype x_dtype, int64_t T, int64_t K, float eps,
+                                         int8_t *Xl, float *absmax, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * bitnet_quant_act - per-token absmax int8 activation quantisation.
  *
  * "BitNet b1.58: Ternary Weights for 1.58-bit LLMs", section "The mechanism"

@@ -219,3 +219,15 @@ def forward(W: np.ndarray, X: np.ndarray, eps_w: float = 1e-5, eps_a: float = 1e
     acc = gemm_i32(Xq, wq)
     Y = dequant(acc, a, g)
     return dict(gamma=g, keep=keep, wq=wq, gb=gb, xq=Xq, a=a, acc=acc, y=Y)
+
+
+def forward_nm(W: np.ndarray, X: np.ndarray, n: int, m: int, eps_w: float = 1e-5, eps_a: float = 1e-5):
+    """Sparse-BitLinear forward with an n:m mask (e.g. 6:8): the plain dense
+    definition, with the same gamma, ternary and activation steps as forward()."""
+    g = gamma(W, eps_w)
+    keep = mask_nm(W, n, m)
+    wq = apply_mask(ternary(W, g), keep)
+    Xq, a = quant_act(X, eps_a)
+    acc = gemm_i32(Xq, wq)
+    Y = dequant(acc, a, g)
+    return dict(gamma=g, keep=keep, wq=wq, xq=Xq, a=a, acc=acc, y=Y)

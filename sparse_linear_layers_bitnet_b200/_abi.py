@@ -28,6 +28,7 @@ EXPORTED = [
     "bitnet_pack_workspace_size", "bitnet_pack_nm", "bitnet_pack_nm_noalloc",
     "bitnet_pack_update_workspace_size", "bitnet_pack_nm_update",
     "bitnet_pack_update_batch_workspace_size", "bitnet_pack_nm_update_batch",
+    "bitnet_pack_6of8_windows", "bitnet_quant_act_lift_6of8",
     "bitnet_quant_act",
     "bitnet_linear_workspace_size", "bitnet_sparse_linear",
     "bitnet_quant_linear_workspace_size", "bitnet_quant_linear",
@@ -100,6 +101,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_pack_nm_update": (I32, [P, ctypes.POINTER(BitnetPackedW), F, P, P, SZ, P]),
         "bitnet_pack_update_batch_workspace_size": (SZ, [ctypes.POINTER(BitnetPackItem), I32]),
         "bitnet_pack_nm_update_batch": (I32, [ctypes.POINTER(BitnetPackItem), I32, F, P, SZ, P]),
+        "bitnet_pack_6of8_windows": (I32, [P, I64, F, ctypes.POINTER(BitnetPackedW), P, P, SZ, P]),
+        "bitnet_quant_act_lift_6of8": (I32, [P, I32, I64, I64, F, P, P, P]),
         "bitnet_quant_act": (I32, [P, I32, I64, I64, F, P, P, P]),
         "bitnet_linear_workspace_size": (SZ, []),
         "bitnet_sparse_linear": (I32, [P, P, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, SZ, P]),
@@ -258,6 +261,36 @@ def bitnet_pack_nm_update_batch(items, eps: float = 1e-5, stream=None) -> PackBa
     b = PackBatch(items, eps, items[0][0].device if items else "cuda")
     b(stream)
     return b
+
+
+def packed_6of8(n_out: int, k: int, device="cuda", mma=True, dec=False) -> "PackedWeights":
+    """Buffers of the 2:4 window layout of a [n_out, k] 6:8 matrix (width k/2*3)."""
+    return PackedWeights(n_out, k // 2 * 3, device, group_bytes=True, mma=mma, dec=dec)
+
+
+def bitnet_pack_6of8_windows(W, out: "PackedWeights", eps: float = 1e-5, mask_bits=None, ws=None, stream=None):
+    lib = load()
+    assert W.dtype == _torch().float32 and W.is_contiguous()
+    if ws is None:
+        ws = Workspace(lib.bitnet_pack_workspace_size(W.shape[0], W.shape[1]), W.device)
+    st = out.struct()
+    check(lib.bitnet_pack_6of8_windows(_ptr(W), W.shape[1], ctypes.c_float(eps), ctypes.byref(st), _ptr(mask_bits),
+                                       ws.ptr, ws.nbytes, _stream(stream)), "bitnet_pack_6of8_windows")
+    return out
+
+
+def bitnet_quant_act_lift_6of8(X, eps: float = 1e-5, Xl=None, absmax=None, stream=None):
+    torch = _torch()
+    lib = load()
+    assert X.is_contiguous() and X.dim() == 2
+    T, K = X.shape
+    if Xl is None:
+        Xl = torch.empty((T, K // 2 * 3), dtype=torch.int8, device=X.device)
+    if absmax is None:
+        absmax = torch.empty((T,), dtype=torch.float32, device=X.device)
+    check(lib.bitnet_quant_act_lift_6of8(_ptr(X), _dtype_code(X.dtype), T, K, ctypes.c_float(eps), _ptr(Xl),
+                                         _ptr(absmax), _stream(stream)), "bitnet_quant_act_lift_6of8")
+    return Xl, absmax
 
 
 def bitnet_quant_act(X, eps: float = 1e-5, Xq=None, absmax=None, stream=None):

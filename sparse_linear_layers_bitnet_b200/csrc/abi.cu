@@ -180,6 +180,46 @@ bitnet_status bitnet_pack_nm_update_batch(const bitnet_pack_item *items, int32_t
                        "pack_update_batch");
 }
 
+bitnet_status bitnet_pack_6of8_windows(const float *W, int64_t k, float eps, bitnet_packed_w *out, uint8_t *mask_bits,
+                                       void *ws, size_t ws_bytes, bitnet_stream_t stream) {
+    if (!W || !out || !out->gamma || !out->group_bytes)
+        return fail(BITNET_ERR_INVALID_ARG, "pack_6of8: W, out, out->gamma and out->group_bytes are required");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "pack_6of8: workspace is required");
+    const int64_t n_out = out->n_out;
+    if (n_out <= 0 || k <= 0) return fail(BITNET_ERR_INVALID_ARG, "pack_6of8: bad sizes");
+    if (k % 64) return fail(BITNET_ERR_UNSUPPORTED, "pack_6of8: k %% 64 != 0");
+    if (out->k != k / 2 * 3 || !(out->n == 2 && out->m == 4))
+        return fail(BITNET_ERR_INVALID_ARG, "pack_6of8: out must describe the 2:4 window layout (k = k/2*3, n = 2, m = 4)");
+    if (ws_bytes < bitnet::kPackWsBytes) return fail(BITNET_ERR_WORKSPACE, "pack_6of8: workspace needs >= %zu bytes", bitnet::kPackWsBytes);
+    if (!(eps >= 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "pack_6of8: eps must be >= 0");
+    if (!aligned(W, 16) || !aligned(ws, 16) || !aligned(out->group_bytes, 4))
+        return fail(BITNET_ERR_INVALID_ARG, "pack_6of8: W and ws 16-byte, group_bytes 4-byte aligned");
+    if ((out->mma_vals == nullptr) != (out->mma_meta == nullptr))
+        return fail(BITNET_ERR_INVALID_ARG, "pack_6of8: mma_vals and mma_meta go together");
+    if (out->dec_codes && (n_out % 16 || k % 128))
+        return fail(BITNET_ERR_INVALID_ARG, "pack_6of8: dec_codes need n_out %% 16 == 0 and k %% 128 == 0");
+    if (static_cast<double>(n_out) * static_cast<double>(k) / 8.0 * 3.0 > 4294967295.0)
+        return fail(BITNET_ERR_UNSUPPORTED, "pack_6of8: more than 2^32 window groups");
+    return cuda_status(bitnet::launch_pack68(W, n_out, k, eps, out->gamma, out->group_bytes, out->mma_vals,
+                                             out->mma_meta, out->dec_codes, mask_bits, ws,
+                                             reinterpret_cast<cudaStream_t>(stream)),
+                       "pack_6of8");
+}
+
+bitnet_status bitnet_quant_act_lift_6of8(const void *X, bitnet_dtype x_dtype, int64_t T, int64_t K, float eps,
+                                         int8_t *Xl, float *absmax, bitnet_stream_t stream) {
+    if (T < 0 || K <= 0 || K % 8) return fail(BITNET_ERR_INVALID_ARG, "quant_lift: need T >= 0, K > 0, K %% 8 == 0");
+    if (T == 0) return BITNET_OK;
+    if (!X || !Xl || !absmax) return fail(BITNET_ERR_INVALID_ARG, "quant_lift: null pointer");
+    if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return fail(BITNET_ERR_INVALID_ARG, "quant_lift: bad dtype");
+    if (!aligned(X, 16) || !aligned(Xl, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_lift: X and Xl must be 16-byte aligned");
+    if (!(eps > 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "quant_lift: eps must be > 0");
+    if (T > 2147483647LL) return fail(BITNET_ERR_UNSUPPORTED, "quant_lift: T too large");
+    return cuda_status(bitnet::launch_quant_lift68(X, x_dtype == BITNET_BF16, T, K, eps, Xl, absmax,
+                                                   reinterpret_cast<cudaStream_t>(stream)),
+                       "quant_lift");
+}
+
 bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, int64_t K, float eps, int8_t *Xq,
                                float *absmax, bitnet_stream_t stream) {
     if (T < 0 || K <= 0 || K % 8) return fail(BITNET_ERR_INVALID_ARG, "quant_act: need T >= 0, K > 0, K %% 8 == 0");

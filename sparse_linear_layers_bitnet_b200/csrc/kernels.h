@@ -66,6 +66,12 @@ cudaError_t launch_pack_update_batch(const PackBatchItemHost *items, int n_items
 cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xq, float *amax,
                              cudaStream_t s);
 
+// 6:8 weights through three 2:4 windows per block of 8 (pack.cu, quant.cu)
+cudaError_t launch_pack68(const float *W, int64_t n_out, int64_t k, float eps, float *gamma, uint8_t *gbw,
+                          int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws, cudaStream_t s);
+cudaError_t launch_quant_lift68(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xl, float *amax,
+                                cudaStream_t s);
+
 cudaError_t launch_gemv_dec(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *dec,
                             int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                             cudaStream_t s);

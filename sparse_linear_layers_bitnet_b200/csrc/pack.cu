@@ -1506,4 +1506,134 @@ cudaError_t launch_pack_update_batch(const PackBatchItemHost *items, int n_items
     return cudaGetLastError();
 }
 
+
+// ---------------------------------------------------------------- 6:8 through 2:4 windows
+//
+// "Sparse-BitNet" (gist.science), section 4 "Resultaten": the method trains
+// at 6:8.  "Is 2:4 Sparsity Still Worth It? ..." (thelatestinai.com), its
+// SlideSparse entry: a (2N-2):2N block is rewritten, without loss, as N-1
+// overlapping 2:4-compliant windows, and the activations are rearranged to
+// match during per-token quantisation.  For 6:8 (N = 4) the three windows of
+// every block of 8 start at positions 0, 2 and 4 and are 4 wide.  The pages
+// do not give the assignment of kept positions to windows; here each kept
+// position goes, in increasing order, to the leftmost window that covers it
+// and has a free slot.  A position's windows form a contiguous range, so this
+// greedy assignment fills all six slots for every choice of six kept
+// positions.  The result is a canonical 2:4 matrix over k' = 3k/2 whose
+// product with the lifted activations equals the 6:8 product exactly.
+
+// one thread per block of 8 weights -> three group bytes of the window layout
+__global__ void __launch_bounds__(256) k_pack68(const float4 *__restrict__ W, int64_t n_blocks,
+                                               const uint32_t *__restrict__ thr_p, uint8_t *__restrict__ gbw) {
+    const uint32_t thr = *thr_p;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < n_blocks; b += stride) {
+        const float4 v0 = __ldg(W + 2 * b), v1 = __ldg(W + 2 * b + 1);
+        const uint32_t bits[8] = {__float_as_uint(v0.x), __float_as_uint(v0.y), __float_as_uint(v0.z),
+                                  __float_as_uint(v0.w), __float_as_uint(v1.x), __float_as_uint(v1.y),
+                                  __float_as_uint(v1.z), __float_as_uint(v1.w)};
+        uint32_t mag[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mag[i] = bits[i] & 0x7fffffffu;
+        // position i is kept when fewer than six positions rank ahead of it
+        // (larger magnitude, or equal magnitude at a lower position)
+        uint32_t keep = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            uint32_t ahead = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j != i) ahead += (j < i) ? (mag[j] >= mag[i] ? 1u : 0u) : (mag[j] > mag[i] ? 1u : 0u);
+            keep |= (ahead < 6u ? 1u : 0u) << i;
+        }
+        // greedy leftmost windows: positions 0,1 -> window 0; 2,3 -> 0 or 1; 4,5 -> 1 or 2; 6,7 -> 2
+        uint32_t g[3] = {0u, 0u, 0u}, f[3] = {0u, 0u, 0u};
+#pragma unroll
+        for (int pos = 0; pos < 8; ++pos) {
+            if (!((keep >> pos) & 1u)) continue;
+            const uint32_t c = mag[pos] >= thr ? (((bits[pos] >> 30) & 2u) | 1u) : 0u;
+            int w;
+            if (pos < 2) w = 0;
+            else if (pos < 4) w = f[0] < 2u ? 0 : 1;
+            else if (pos < 6) w = f[1] < 2u ? 1 : 2;
+            else w = 2;
+            const uint32_t rel = static_cast<uint32_t>(pos - 2 * w);
+#pragma unroll
+            for (int ww = 0; ww < 3; ++ww)
+                if (ww == w) {
+                    g[ww] |= f[ww] == 0u ? (rel | (c << 4)) : ((rel << 2) | (c << 6));
+                    ++f[ww];
+                }
+        }
+        uint8_t *dst = gbw + 3 * b;
+        dst[0] = static_cast<uint8_t>(g[0]);
+        dst[1] = static_cast<uint8_t>(g[1]);
+        dst[2] = static_cast<uint8_t>(g[2]);
+    }
+}
+
+// tensor-core values and metadata of a canonical 2:4 matrix from its group
+// bytes (four groups per thread; k % 16 == 0)
+__global__ void __launch_bounds__(256) k_gb_to_mma(const uint8_t *__restrict__ gb, Pack24Args p) {
+    const uint32_t n_quads = static_cast<uint32_t>(p.n_groups >> 2);
+    const uint32_t stride = gridDim.x * blockDim.x;
+    for (uint32_t q = blockIdx.x * blockDim.x + threadIdx.x; q < n_quads; q += stride) {
+        const uint32_t w = __ldg(reinterpret_cast<const uint32_t *>(gb) + q);
+        QuadOut o;
+        o.gb = w;
+        o.vlo = o.vhi = o.meta = o.mask = o.band = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t b = (w >> (8 * j)) & 0xffu;
+            const uint32_t c0 = (b >> 4) & 3u, c1 = b >> 6;
+            const uint32_t v = ((c0 & 2u) * 0x7eu + c0) | (((c1 & 2u) * 0x7eu + c1) << 8);
+            if (j < 2) o.vlo |= v << (16 * j);
+            else o.vhi |= v << (16 * (j - 2));
+            o.meta |= (b & 0xfu) << (4 * j);
+        }
+        store_quad(p, q, o);
+    }
+}
+
+cudaError_t launch_pack68(const float *W, int64_t n_out, int64_t k, float eps, float *gamma, uint8_t *gbw,
+                          int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws, cudaStream_t s) {
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    uint32_t *thr = reinterpret_cast<uint32_t *>(w8 + kPackWsThrOffset);
+    unsigned long long *win = reinterpret_cast<unsigned long long *>(w8 + kPackWsWinOffset);
+    unsigned long long *bins = reinterpret_cast<unsigned long long *>(w8 + kPackWsBinsOffset);
+    cudaError_t err = cudaMemsetAsync(ws, 0, kPackWsBytes, s);
+    if (err != cudaSuccess) return err;
+    const int64_t n_el = n_out * k;
+    unsigned *counter = reinterpret_cast<unsigned *>(w8 + kPackWsCounterOffset);
+    // gamma over the dense matrix, as for 2:4
+    k_abs_sum_fast<<<grid_for(n_el / 4, 256, 4), 256, 0, s>>>(reinterpret_cast<const float4 *>(W), n_el / 4, win,
+                                                             bins, counter, n_el, eps, gamma, thr);
+    k_pack68<<<grid_for(n_el / 8, 256, 8), 256, 0, s>>>(reinterpret_cast<const float4 *>(W), n_el / 8, thr, gbw);
+    const int64_t kw = k / 2 * 3;   // window layout width
+    if (vals || meta) {
+        Pack24Args a;
+        a.W = nullptr;
+        a.n_groups = n_out * kw / 4;
+        a.gpr = kw / 4;
+        a.gpr_div = make_fastdiv(static_cast<uint32_t>(kw / 4));
+        a.n_out = n_out;
+        a.k = kw;
+        a.meta_rows = (n_out + 127) / 128 * 128;
+        a.thr = nullptr;
+        a.gb = nullptr;
+        a.vals = reinterpret_cast<uint16_t *>(vals);
+        a.meta = meta;
+        a.mask = nullptr;
+        k_gb_to_mma<<<grid_for(a.n_groups / 4, 256, 8), 256, 0, s>>>(gbw, a);
+        if (meta && (a.meta_rows != n_out || (kw % 128) != 0))
+            k_meta_pad<<<grid_for(((kw + 127) / 128) * (a.meta_rows - n_out) * 16 + n_out * 16, 256, 4), 256, 0, s>>>(
+                meta, n_out, kw, a.meta_rows);
+    }
+    if (dec)
+        k_make_dec<<<grid_for(n_out / 16 * (kw / 64) * 32, 256, 8), 256, 0, s>>>(gbw, n_out, kw,
+                                                                                 reinterpret_cast<uint2 *>(dec));
+    if (mask) k_mask_nm<<<grid_for(n_el / 8, 256, 8), 256, 0, s>>>(W, n_el / 8, 6, 8, mask);
+    return cudaGetLastError();
+}
+
 }  // namespace bitnet

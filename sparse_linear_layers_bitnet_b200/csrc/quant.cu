@@ -139,4 +139,85 @@ cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, flo
     return cudaLaunchKernelEx(&cfg, k_quant_act<false>, x, K, eps, Xq, amax);
 }
 
+
+// ---------------------------------------------------------------- activation lifting for 6:8 windows
+//
+// "Is 2:4 Sparsity Still Worth It? ..." (thelatestinai.com), its SlideSparse
+// entry: the activation rearrangement that matches the window decomposition
+// of the weights is done inside per-token quantisation.  For 6:8 each block of
+// 8 activations x[8b .. 8b+7] becomes 12 codes, the three overlapping windows
+// x[8b + 2w .. 8b + 2w + 3] (w = 0, 1, 2).  The scale is the token's absmax
+// over its original row, so every code equals bitnet_quant_act's.
+template <bool BF16>
+__global__ void __launch_bounds__(kQuantThreads) k_quant_lift68(const uint8_t *__restrict__ X, int64_t K, float eps,
+                                                                int8_t *__restrict__ Xl, float *__restrict__ amax) {
+    __shared__ float s_red[32];
+    const int64_t t = blockIdx.x;
+    const int64_t esize = BF16 ? 2 : 4;
+    const uint8_t *row = X + t * K * esize;
+    const int64_t blocks = K / 8;
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    float m = 0.0f;
+    for (int64_t b = threadIdx.x; b < blocks; b += kQuantThreads) {
+        float v[8];
+        if (BF16) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(row) + b);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = __uint_as_float((j & 1) ? (w[j >> 1] & 0xffff0000u) : (w[j >> 1] << 16));
+        } else {
+            const float4 a = __ldg(reinterpret_cast<const float4 *>(row) + 2 * b);
+            const float4 c = __ldg(reinterpret_cast<const float4 *>(row) + 2 * b + 1);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+    }
+    m = block_max(m, s_red);
+    const float a = m > eps ? m : eps;
+    const float sc = __fdiv_rn(127.0f, a);
+    if (threadIdx.x == 0) amax[t] = a;
+    int8_t *out = Xl + t * (K / 2 * 3);
+    for (int64_t b = threadIdx.x; b < blocks; b += kQuantThreads) {
+        uint32_t q[8];
+        if (BF16) {
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(row) + b);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                q[j] = static_cast<uint8_t>(quant_one(
+                    __uint_as_float((j & 1) ? (w[j >> 1] & 0xffff0000u) : (w[j >> 1] << 16)), sc));
+        } else {
+            const float4 a4 = __ldg(reinterpret_cast<const float4 *>(row) + 2 * b);
+            const float4 c4 = __ldg(reinterpret_cast<const float4 *>(row) + 2 * b + 1);
+            const float v[8] = {a4.x, a4.y, a4.z, a4.w, c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int j = 0; j < 8; ++j) q[j] = static_cast<uint8_t>(quant_one(v[j], sc));
+        }
+        // windows 0, 1, 2: codes 0-3, 2-5, 4-7
+        uint32_t *dst = reinterpret_cast<uint32_t *>(out + 12 * b);
+        dst[0] = q[0] | (q[1] << 8) | (q[2] << 16) | (q[3] << 24);
+        dst[1] = q[2] | (q[3] << 8) | (q[4] << 16) | (q[5] << 24);
+        dst[2] = q[4] | (q[5] << 8) | (q[6] << 16) | (q[7] << 24);
+    }
+}
+
+cudaError_t launch_quant_lift68(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xl, float *amax,
+                                cudaStream_t s) {
+    if (T <= 0) return cudaSuccess;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(T));
+    cfg.blockDim = dim3(kQuantThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const uint8_t *x = static_cast<const uint8_t *>(X);
+    if (bf16) return cudaLaunchKernelEx(&cfg, k_quant_lift68<true>, x, K, eps, Xl, amax);
+    return cudaLaunchKernelEx(&cfg, k_quant_lift68<false>, x, K, eps, Xl, amax);
+}
+
 }  // namespace bitnet

@@ -416,6 +416,91 @@ def test_quant_linear_chain_in_graph(bn):
         assert np.array_equal(xs[l + 1].cpu().numpy(), x), l
 
 
+# ------------------------------------------------------------------ 6:8 through 2:4 windows
+
+def windows_to_dense(gbw, n_out, k):
+    """Window-layout group bytes [n_out, 3k/8] -> dense int8 [n_out, k] and keep.
+    Window w of block b covers positions 8b + 2w .. 8b + 2w + 3; every kept
+    position must appear in exactly one window slot."""
+    gbw = gbw.reshape(n_out, k // 8, 3).astype(np.int64)
+    wq = np.zeros((n_out, k), np.int8)
+    seen = np.zeros((n_out, k), np.int32)
+    code_val = np.array([0, 1, 0, -1], np.int8)
+    rows = np.arange(n_out)[:, None]
+    for w in range(3):
+        b = gbw[:, :, w]
+        i0, i1, c0, c1 = b & 3, (b >> 2) & 3, (b >> 4) & 3, b >> 6
+        assert (i0 < i1).all()
+        base = 8 * np.arange(k // 8)[None, :] + 2 * w
+        for idx, c in ((i0, c0), (i1, c1)):
+            pos = base + idx
+            wq[rows, pos] = code_val[c]
+            np.add.at(seen, (np.broadcast_to(rows, pos.shape), pos), 1)
+    return wq, seen
+
+
+@pytest.mark.parametrize("n_out,k", [(256, 512), (200, 384), (128, 1024), (48, 64)])
+def test_pack_6of8_windows(bn, n_out, k):
+    """gamma, the 6:8 keep bits and the window layouts against the oracle's
+    dense 6:8 masked ternary matrix; every kept position sits in exactly one
+    window slot; the tensor-core layout and the decode layout decode to the
+    same window matrix."""
+    W = synth.master_weights(n_out, k, 0.02, seed=3000 + n_out + k)
+    W[0, :8] = 0.01                                            # an all-tie block
+    W[1, 8:16] = [0.3, -0.3, 0.3, -0.3, 0.0, -0.0, 0.3, 0.3]   # ties and signed zeros
+    ref = oracle.forward_nm(W, synth.activations(1, k, seed=1), 6, 8)
+    dec = n_out % 16 == 0 and k % 128 == 0
+    pw = bn.packed_6of8(n_out, k, dec=dec)
+    mask = torch.zeros(n_out * k // 8, dtype=torch.uint8, device="cuda")
+    bn.bitnet_pack_6of8_windows(dev_f32(W), pw, 1e-5, mask_bits=mask)
+    torch.cuda.synchronize()
+    assert pw.gamma.item() == float(ref["gamma"])
+    assert np.array_equal(mask_bits_to_keep(mask.cpu().numpy(), n_out, k), ref["keep"])
+    gbw = pw.group_bytes.cpu().numpy()
+    wq, seen = windows_to_dense(gbw, n_out, k)
+    assert np.array_equal(seen, ref["keep"].astype(np.int32))
+    assert np.array_equal(wq, ref["wq"])
+    kw = k // 2 * 3
+    mwq, mkeep, _, _ = decode_mma(pw.mma_vals.cpu().numpy(), pw.mma_meta.cpu().numpy(), n_out, kw)
+    g2 = gbw.reshape(n_out, kw // 4).astype(np.int64)
+    cval = np.array([0, 1, 0, -1], np.int8)
+    dense_w = np.zeros((n_out, kw), np.int8)
+    r = np.arange(n_out)[:, None]
+    gi = 4 * np.arange(kw // 4)[None, :]
+    dense_w[r, gi + (g2 & 3)] = cval[(g2 >> 4) & 3]
+    dense_w[r, gi + ((g2 >> 2) & 3)] = cval[g2 >> 6]
+    assert np.array_equal(mwq, dense_w)
+    if dec:
+        assert np.array_equal(decode_dec(pw.dec_codes.cpu().numpy(), n_out, kw), g2.astype(np.uint32))
+
+
+@pytest.mark.parametrize("T,x_dtype", [(1, "bf16"), (5, "f32"), (8, "bf16"), (64, "bf16"), (300, "bf16")])
+@pytest.mark.parametrize("n_out,k", [(256, 1024), (2560, 2560)])
+def test_6of8_forward(bn, T, x_dtype, n_out, k):
+    """Lifted activations + the 2:4 GEMV (T <= 8) or tensor-core GEMM (T > 8)
+    on the window layout reproduce the oracle's dense 6:8 product: int32
+    accumulators bit-exact, outputs to 1e-5 / exact bf16."""
+    W = synth.master_weights(n_out, k, 0.02, seed=3100 + T)
+    X = synth.activations(T, k, seed=3101 + T, outlier_p=0.01)
+    if x_dtype == "bf16":
+        Xd, X32 = bf16_dev(X)
+    else:
+        Xd, X32 = dev_f32(X), X
+    ref = oracle.forward_nm(W, X32, 6, 8)
+    pw = bn.packed_6of8(n_out, k, dec=True)
+    bn.bitnet_pack_6of8_windows(dev_f32(W), pw, 1e-5)
+    Xl, am = bn.bitnet_quant_act_lift_6of8(Xd, 1e-5)
+    acc = torch.full((T, n_out), -7, dtype=torch.int32, device="cuda")
+    Y = bn.bitnet_sparse_linear(Xl, am, pw, y_dtype=torch.float32, acc_out=acc)
+    torch.cuda.synchronize()
+    xq = ref["xq"]
+    # block b, window w, position j -> code of column 8b + 2w + j
+    lifted = np.stack([xq.reshape(T, -1, 8)[:, :, 2 * w:2 * w + 4] for w in range(3)], axis=2).reshape(T, -1)
+    assert np.array_equal(Xl.cpu().numpy(), lifted)
+    assert np.array_equal(am.cpu().numpy(), ref["a"])
+    _check_outputs(ref, acc.cpu().numpy(), Y)
+
+
 # ------------------------------------------------------------------ decode chain (one persistent launch)
 
 def _packed_dec(bn, n_out, k, seed):

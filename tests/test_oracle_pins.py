@@ -271,6 +271,29 @@ def test_forward_matches_dense_masked_brute_force():
     assert np.all(np.abs(out["y"] - yfp) <= bound)
 
 
+def test_forward_6of8_matches_python_brute_force():
+    """The 6:8 forward of the oracle against pure-Python loops: top-6 of every
+    8 by (|w| desc, position asc), codes clip(rint(w / gamma)), integer sums."""
+    W = synth.master_weights(6, 32, 0.02, 31)
+    W[0, :8] = 0.01                      # an all-tie block: positions 0..5 kept
+    X = synth.activations(3, 32, 32)
+    out = oracle.forward_nm(W, X, 6, 8)
+    g = float(out["gamma"])
+    keep = _brute_mask(W, 6, 8)
+    assert np.array_equal(out["keep"], keep)
+    assert keep[0, :8].tolist() == [1, 1, 1, 1, 1, 1, 0, 0]
+    xq = out["xq"].astype(np.int64)
+    for r in range(W.shape[0]):
+        for t in range(X.shape[0]):
+            acc = 0
+            for c in range(W.shape[1]):
+                if keep[r, c]:
+                    q = int(np.clip(np.rint(np.float32(W[r, c]) / np.float32(g)), -1, 1))
+                    acc += q * int(xq[t, c])
+            assert acc == int(out["acc"][t, r])
+    assert (keep.reshape(6, -1, 8).sum(2) == 6).all()
+
+
 def test_dgrad_matches_numpy_fp64():
     r = np.random.default_rng(8)
     dY = r.normal(size=(6, 40)).astype(np.float32)
