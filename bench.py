@@ -62,7 +62,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--pack-layers", type=int, default=None, help="layers of the pack workload (default: all 26)")
     ap.add_argument("--flip-steps", type=int, default=100, help="random-walk steps of the mask flip-rate study")
-    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks"], default=None,
+    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks", "six_eight"], default=None,
                     help="run one sub-measurement alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -464,6 +464,80 @@ def measure_pack(torch, bn, synth, peaks, steps=3, flip_steps=100, layers=None):
     return out
 
 
+def measure_6of8(torch, bn, synth, reps=10):
+    """6:8 weights on the 2:4 tensor cores (window decomposition + activation
+    lifting) on the 7B prefill shapes, against cuBLASLt dense int8 on the same
+    T x K x N and against the 2:4 layer; plus the per-step 6:8 pack."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    out = {}
+    t68 = t24 = tdn = tq = 0.0
+    ops_all = 0.0
+    for name, T, K, N in synth.PREFILL_7B_GEMMS:
+        W = synth.torch_master_weights(N, K, 0.02, seed=21, device=dev)
+        pw = bn.packed_6of8(N, K, dev, mma=True, dec=False)
+        ws = bn.Workspace(bn.load().bitnet_pack_workspace_size(N, K), dev)
+        bn.bitnet_pack_6of8_windows(W, pw, 1e-5, ws=ws)
+        pk = []
+        for _ in range(3):
+            with Timer(torch) as t:
+                bn.bitnet_pack_6of8_windows(W, pw, 1e-5, ws=ws)
+            pk.append(t.ms())
+        p24 = bn.PackedWeights(N, K, dev, group_bytes=False, mma=True, dec=False)
+        bn.bitnet_pack_nm(W, p24, 1e-5)
+        del W
+        X = synth.torch_activations(T, K, seed=22, outlier_p=0.01, dtype=torch.bfloat16, device=dev)
+        Xl, a = bn.bitnet_quant_act_lift_6of8(X, 1e-5)
+        Xq, a2 = bn.bitnet_quant_act(X, 1e-5)
+        Y = torch.empty((T, N), dtype=torch.bfloat16, device=dev)
+        lws = bn.Workspace(256, dev)
+        Xi = torch.randint(-127, 128, (T, K), dtype=torch.int8, device=dev)
+        Bi = torch.randint(-1, 2, (K, N), dtype=torch.int8, device=dev)
+        for _ in range(3):
+            bn.bitnet_sparse_linear(Xl, a, pw, Y=Y, ws=lws)
+            bn.bitnet_sparse_linear(Xq, a2, p24, Y=Y, ws=lws)
+            torch._int_mm(Xi, Bi)
+        m68, m24, mdn, mq = [], [], [], []
+        for _ in range(reps):
+            flush_l2(torch, flush)
+            with Timer(torch) as t:
+                bn.bitnet_quant_act_lift_6of8(X, 1e-5, Xl=Xl, absmax=a)
+            mq.append(t.ms())
+            flush_l2(torch, flush)
+            with Timer(torch) as t:
+                bn.bitnet_sparse_linear(Xl, a, pw, Y=Y, ws=lws)
+            m68.append(t.ms())
+            flush_l2(torch, flush)
+            with Timer(torch) as t:
+                bn.bitnet_sparse_linear(Xq, a2, p24, Y=Y, ws=lws)
+            m24.append(t.ms())
+            flush_l2(torch, flush)
+            with Timer(torch) as t:
+                torch._int_mm(Xi, Bi)
+            mdn.append(t.ms())
+        ops = 2.0 * T * K * N
+        a68, a24, adn, aq = (statistics.mean(v) for v in (m68, m24, mdn, mq))
+        out[name] = {"T": T, "K": K, "N": N, "gemm_6of8_ms": round(a68, 4), "lift_quant_ms": round(aq, 4),
+                     "gemm_2of4_ms": round(a24, 4), "cublas_dense_int8_ms": round(adn, 4),
+                     "tops_6of8": round(ops / a68 / 1e9, 1), "speedup_vs_dense_int8": round(adn / a68, 3),
+                     "pack_6of8_ms": round(statistics.mean(pk), 4),
+                     "pack_6of8_gbs": round(N * K * (4 + 3 / 8 + 3 / 4 + 3 / 16) / statistics.mean(pk) / 1e6, 1)}
+        t68 += a68
+        t24 += a24
+        tdn += adn
+        tq += aq
+        ops_all += ops
+        del pw, p24, X, Xl, Xq, Y, Xi, Bi, ws
+    out["combined"] = {"tops_6of8": round(ops_all / t68 / 1e9, 1), "speedup_vs_dense_int8": round(tdn / t68, 3),
+                       "ratio_6of8_to_2of4_time": round(t68 / t24, 3),
+                       "note": "6:8 runs as a 2:4 GEMM over K' = 1.5 K: its ceiling is (2:4 speed-up over dense) / 1.5; "
+                               "tops_6of8 counts the 2 T K N dense-equivalent ops of the 6:8 layer",
+                       "l2": "flushed (256 MB write) before every timed launch"}
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
 def measure_dgrad(torch, bn, synth, peaks, reps=5):
     dev = torch.device("cuda", torch.cuda.current_device())
     T = 2048
@@ -590,7 +664,8 @@ def run_only(args):
     bn.load()
     peaks = load_peaks()
     fn = {"prefill": measure_prefill, "pack": measure_pack, "dgrad": measure_dgrad,
-          "peaks": lambda torch, bn, synth, peaks: measure_library_peaks(torch)}[args.only]
+          "peaks": lambda torch, bn, synth, peaks: measure_library_peaks(torch),
+          "six_eight": lambda torch, bn, synth, peaks: measure_6of8(torch, bn, synth)}[args.only]
     kw = {"steps": args.steps, "flip_steps": args.flip_steps, "layers": args.pack_layers} if args.only == "pack" else {}
     print(json.dumps({args.only: fn(torch, bn, synth, peaks, **kw)}), flush=True)
     return 0
@@ -703,6 +778,7 @@ def run_ours(args):
         pc["frac_of_2x_measured_int8_dense"] = round(pc["tops"] / (2 * lp), 4)
         pc["frac_of_measured_int8_dense"] = round(pc["tops"] / lp, 4)
         rows["dgrad"] = measure_dgrad(torch, bn, synth, peaks)
+        rows["six_eight"] = measure_6of8(torch, bn, synth)
         rows["pack"] = measure_pack(torch, bn, synth, peaks, flip_steps=args.flip_steps)
 
     line = {
