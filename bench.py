@@ -422,6 +422,20 @@ def measure_pack(torch, bn, synth, peaks, steps=3, flip_steps=100, layers=None):
             for W, pw in zip(Ws, pws):
                 bn.bitnet_pack_nm_update(W, pw, 1e-5, ws=ws)
         ms_single.append(t.ms())
+    # bf16 masters (the method keeps BF16 masters): same matrices rounded to bf16, 2 B/weight read
+    Wb = [W.to(torch.bfloat16) for W in Ws]
+    # the same output buffers: the gamma of the last fp32 step serves as the first hint
+    batch_b = bn.PackBatch(list(zip(Wb, pws)), 1e-5, dev)
+    batch_b()
+    ms_b = []
+    for s in range(steps):
+        for i, W in enumerate(Wb):
+            W.copy_((W.float() + torch.randn(W.shape, device=dev, generator=torch.Generator(device=dev).manual_seed(
+                (2 * steps + s) * 1000 + i)) * 1e-4).to(torch.bfloat16))
+        with Timer(torch) as t:
+            batch_b()
+        ms_b.append(t.ms())
+    del batch_b, Wb
     step_ms = statistics.mean(ms)
     gbs = alg_bytes / step_ms / 1e6
     n_mats = len(Ws)
@@ -430,6 +444,9 @@ def measure_pack(torch, bn, synth, peaks, steps=3, flip_steps=100, layers=None):
            "alg_bytes_per_weight": 4.875, "launches_per_step": 2 * ((n_mats + 63) // 64),
            "entry": "bitnet_pack_nm_update_batch over all matrices (each previous gamma as hint; "
                     "bit-identical to bitnet_pack_nm)",
+           "bf16_masters": {"step_ms": round(statistics.mean(ms_b), 3),
+                            "gbs": round(n_w * (2 + 0.875) / statistics.mean(ms_b) / 1e6, 1),
+                            "alg_bytes_per_weight": 2.875},
            "per_matrix_calls": {"step_ms": round(statistics.mean(ms_single), 3),
                                 "gbs": round(alg_bytes / statistics.mean(ms_single) / 1e6, 1),
                                 "entry": "bitnet_pack_nm_update, one call per matrix"}}

@@ -156,7 +156,12 @@ bitnet_status bitnet_pack_nm_update(const float *W, bitnet_packed_w *out, float 
  * workspace clear and a gamma finalisation is paid once per list.
  *
  *   items    host array of n_items descriptors (read during the call only):
- *              W          [n_out x k] fp32 masters, 16-byte aligned (device);
+ *              W          [n_out x k] masters of w_dtype, 16-byte aligned
+ *                         (device).  BITNET_BF16 masters ("Sparse-BitNet"
+ *                         (gist.science), section 2 "Kerncomponenten": the
+ *                         master weights are kept in BF16) are widened exactly
+ *                         to fp32, so the result is that of their fp32 values;
+ *              w_dtype    BITNET_F32 or BITNET_BF16;
  *              out        host struct as for bitnet_pack_nm_update (n = 2,
  *                         m = 4, k % 16 == 0); out->gamma holds the hint;
  *              mask_bits  [n_out * k / 8] or NULL.
@@ -168,9 +173,10 @@ bitnet_status bitnet_pack_nm_update(const float *W, bitnet_packed_w *out, float 
  * Errors: as bitnet_pack_nm_update; UNSUPPORTED when k % 16 != 0.
  * ------------------------------------------------------------------------ */
 typedef struct {
-    const float *W;
+    const void *W;
     bitnet_packed_w *out;
     uint8_t *mask_bits;
+    int32_t w_dtype;   /* bitnet_dtype of W */
 } bitnet_pack_item;
 
 size_t bitnet_pack_update_batch_workspace_size(const bitnet_pack_item *items, int32_t n_items);

@@ -57,6 +57,7 @@ class BitnetPackItem(ctypes.Structure):
         ("W", ctypes.c_void_p),
         ("out", ctypes.POINTER(BitnetPackedW)),
         ("mask_bits", ctypes.c_void_p),
+        ("w_dtype", ctypes.c_int32),
     ]
 
 
@@ -225,7 +226,8 @@ def bitnet_pack_nm_update(W, out: PackedWeights, eps: float = 1e-5, mask_bits=No
 
 
 class PackBatch:
-    """A fixed list of (W, PackedWeights[, mask_bits]) for bitnet_pack_nm_update_batch.
+    """A fixed list of (W, PackedWeights[, mask_bits]) for bitnet_pack_nm_update_batch
+    (W: fp32 or bf16 masters).
 
     The descriptor array and the workspace are built once, so the same batch
     can be repacked every step (or captured in a CUDA graph) without
@@ -241,10 +243,11 @@ class PackBatch:
         for i, it in enumerate(items):
             W, out = it[0], it[1]
             mask = it[2] if len(it) > 2 else None
-            assert W.dtype == _torch().float32 and W.is_contiguous()
+            assert W.dtype in (_torch().float32, _torch().bfloat16) and W.is_contiguous()
             st = out.struct()
             self._keep.append((st, W, out, mask))
             arr[i].W = W.data_ptr()
+            arr[i].w_dtype = _dtype_code(W.dtype)
             arr[i].out = ctypes.pointer(st)
             arr[i].mask_bits = mask.data_ptr() if mask is not None else None
         self._arr = arr

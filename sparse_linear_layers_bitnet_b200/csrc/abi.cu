@@ -159,6 +159,8 @@ bitnet_status bitnet_pack_nm_update_batch(const bitnet_pack_item *items, int32_t
         if (n_out <= 0 || k <= 0 || k % 8) return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: item %d: bad sizes", i);
         if (!(out->n == 2 && out->m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "pack_update_batch: item %d: 2:4 only", i);
         if (k % 16) return fail(BITNET_ERR_UNSUPPORTED, "pack_update_batch: item %d: k %% 16 != 0", i);
+        if (it.w_dtype != BITNET_F32 && it.w_dtype != BITNET_BF16)
+            return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: item %d: bad w_dtype", i);
         if (!aligned(it.W, 16)) return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: item %d: W must be 16-byte aligned", i);
         if ((out->mma_vals == nullptr) != (out->mma_meta == nullptr))
             return fail(BITNET_ERR_INVALID_ARG, "pack_update_batch: item %d: mma_vals and mma_meta go together", i);
@@ -168,7 +170,7 @@ bitnet_status bitnet_pack_nm_update_batch(const bitnet_pack_item *items, int32_t
         if (static_cast<double>(n_out) * static_cast<double>(k) / 4.0 > 4294967295.0)
             return fail(BITNET_ERR_UNSUPPORTED, "pack_update_batch: item %d: more than 2^32 groups", i);
         h[static_cast<size_t>(i)] = {it.W, n_out, k, out->gamma, out->group_bytes, out->mma_vals, out->mma_meta,
-                                     out->dec_codes, it.mask_bits};
+                                     out->dec_codes, it.mask_bits, it.w_dtype == BITNET_BF16};
     }
     const size_t need = bitnet_pack_update_batch_workspace_size(items, n_items);
     if (ws_bytes < need) return fail(BITNET_ERR_WORKSPACE, "pack_update_batch: workspace needs %zu bytes", need);

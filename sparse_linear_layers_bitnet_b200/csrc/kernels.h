@@ -50,7 +50,7 @@ inline size_t update_list_bytes(int64_t n_out, int64_t k) {
 
 // Batched per-step pack: one matrix as the host describes it.
 struct PackBatchItemHost {
-    const float *W;
+    const void *W;   // fp32 or bf16 masters (w_bf16)
     int64_t n_out, k;
     float *gamma;
     uint8_t *gb;
@@ -58,6 +58,7 @@ struct PackBatchItemHost {
     uint8_t *meta;
     uint8_t *dec;
     uint8_t *mask;
+    bool w_bf16;
 };
 constexpr int kPackBatchMax = 64;   // matrices per launch (kernel parameter space)
 size_t pack_batch_ws_bytes(const int64_t *n_out, const int64_t *k, int n_items);

@@ -1183,6 +1183,7 @@ struct BatchItem {
     uint32_t list_cap;
     uint32_t chunk0, nchunks;  // this matrix's range of the global chunk list
     uint32_t pad_bytes;        // metadata padding bytes (0: none)
+    uint32_t w_bf16;           // 1: the masters (p.W) are bf16, widened exactly to fp32 on load
     int64_t n_total;
 };
 
@@ -1195,6 +1196,32 @@ struct BatchParams {
 
 constexpr uint32_t kBatchChunkQuads = 512;   // 256 threads x 2 quads
 
+// four bf16 masters (8 bytes) widened exactly to fp32
+__device__ __forceinline__ float4 bf16x4_to_float4(uint2 u) {
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                       __uint_as_float(u.y & 0xffff0000u));
+}
+
+// the four groups (16 masters) of quad q, fp32 or bf16 storage
+__device__ __forceinline__ void load_quad(const Pack24Args &p, bool bf16, uint32_t q, float4 (&v)[4]) {
+    if (bf16) {
+        const uint4 *Wb = reinterpret_cast<const uint4 *>(p.W);
+        const uint4 a = __ldg(Wb + 2u * q), b = __ldg(Wb + 2u * q + 1u);
+        v[0] = bf16x4_to_float4(make_uint2(a.x, a.y));
+        v[1] = bf16x4_to_float4(make_uint2(a.z, a.w));
+        v[2] = bf16x4_to_float4(make_uint2(b.x, b.y));
+        v[3] = bf16x4_to_float4(make_uint2(b.z, b.w));
+    } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = __ldg(p.W + 4u * q + j);
+    }
+}
+
+__device__ __forceinline__ float4 load_group(const Pack24Args &p, bool bf16, int64_t i) {
+    if (bf16) return bf16x4_to_float4(__ldg(reinterpret_cast<const uint2 *>(p.W) + i));
+    return __ldg(p.W + i);
+}
+
 __device__ __forceinline__ int batch_item_of(const BatchParams &bp, uint32_t c) {
     int lo = 0, hi = bp.n - 1;
     while (lo < hi) {
@@ -1203,6 +1230,52 @@ __device__ __forceinline__ int batch_item_of(const BatchParams &bp, uint32_t c) 
         else hi = mid - 1;
     }
     return lo;
+}
+
+// One CTA's run of chunks [c, seg_end) of one matrix: exact partial sum of
+// |W| (into lo, hi) and, with a hint, every layout with the hint's threshold
+// plus the band list.  BF16: the masters are bf16.
+template <bool BF16>
+__device__ __forceinline__ void batch_segment(const BatchItem &I, uint32_t c, uint32_t seg_end, bool hint,
+                                              uint32_t t_old, uint32_t t_lo, uint32_t t_hi, unsigned *list_count,
+                                              uint64_t &lo, uint64_t &hi, unsigned long long *s_bins, int *s_rare) {
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const Pack24Args &p = I.p;
+    const uint32_t n_quads = static_cast<uint32_t>(p.n_groups >> 2);
+    double d = 0.0;
+    for (uint32_t ch = c; ch < seg_end; ++ch) {
+        const uint32_t qbase = (ch - I.chunk0) * kBatchChunkQuads + warp * (32u * kQuadUnroll);
+        float4 v[kQuadUnroll][4];
+#pragma unroll
+        for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
+            const uint32_t q = qbase + 32u * k2 + lane;
+            if (q < n_quads) {
+                load_quad(p, BF16, q, v[k2]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) v[k2][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
+            const uint32_t q = qbase + 32u * k2 + lane;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sum_float4(v[k2][j], d, lo, hi, s_bins, s_rare);
+            if (hint && q < n_quads) {
+                const QuadOut o = pack_quad(v[k2], t_old, t_lo, t_hi);
+                store_quad(p, q, o);
+                if (o.band) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if ((o.band >> j) & 1u) {
+                            const unsigned slot = atomicAdd(list_count, 1u);
+                            if (slot < I.list_cap) I.list[slot] = 4u * q + j;
+                        }
+                }
+            }
+        }
+        flush_sum(d, lo, hi);
+    }
 }
 
 __global__ void __launch_bounds__(256, 4) k_pack_update_batch(const __grid_constant__ BatchParams bp) {
@@ -1245,41 +1318,13 @@ __global__ void __launch_bounds__(256, 4) k_pack_update_batch(const __grid_const
         __syncthreads();
         const bool hint = s_hint != 0;
         const uint32_t t_old = s_t, t_lo = s_tlo, t_hi = s_thi;
-        const Pack24Args &p = I.p;
-        const uint32_t n_quads = static_cast<uint32_t>(p.n_groups >> 2);
+        const bool wbf16 = I.w_bf16 != 0u;
         unsigned *list_count = reinterpret_cast<unsigned *>(hdr + kPackWsListCountOffset);
         uint64_t lo = 0, hi = 0;
-        double d = 0.0;
-        for (uint32_t ch = c; ch < seg_end; ++ch) {
-            const uint32_t qbase = (ch - I.chunk0) * kBatchChunkQuads + warp * (32u * kQuadUnroll);
-            float4 v[kQuadUnroll][4];
-#pragma unroll
-            for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
-                const uint32_t q = qbase + 32u * k2 + lane;
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    v[k2][j] = q < n_quads ? __ldg(p.W + 4u * q + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-#pragma unroll
-            for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
-                const uint32_t q = qbase + 32u * k2 + lane;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) sum_float4(v[k2][j], d, lo, hi, s_bins, &s_rare);
-                if (hint && q < n_quads) {
-                    const QuadOut o = pack_quad(v[k2], t_old, t_lo, t_hi);
-                    store_quad(p, q, o);
-                    if (o.band) {
-#pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            if ((o.band >> j) & 1u) {
-                                const unsigned slot = atomicAdd(list_count, 1u);
-                                if (slot < I.list_cap) I.list[slot] = 4u * q + j;
-                            }
-                    }
-                }
-            }
-            flush_sum(d, lo, hi);
-        }
+        if (wbf16)
+            batch_segment<true>(I, c, seg_end, hint, t_old, t_lo, t_hi, list_count, lo, hi, s_bins, &s_rare);
+        else
+            batch_segment<false>(I, c, seg_end, hint, t_old, t_lo, t_hi, list_count, lo, hi, s_bins, &s_rare);
         // this segment's exact partial sum into the matrix's accumulators
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -1426,7 +1471,7 @@ __global__ void __launch_bounds__(256) k_pack_finish_batch(const __grid_constant
         const int item = batch_bucket(s_patch, n, x);
         const BatchItem &I = bp.it[item];
         const int64_t i = I.list[x - s_patch[item]];
-        patch_group(I.p, s_thr[item], i, __ldg(I.p.W + i));
+        patch_group(I.p, s_thr[item], i, load_group(I.p, I.w_bf16 != 0u, i));
     }
     // 2. every quad of the matrices whose threshold left the band (or had no hint)
     for (uint32_t x = gtid; x < s_quads[n]; x += gstride) {
@@ -1434,8 +1479,7 @@ __global__ void __launch_bounds__(256) k_pack_finish_batch(const __grid_constant
         const BatchItem &I = bp.it[item];
         const uint32_t q = x - s_quads[item];
         float4 v[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = __ldg(I.p.W + 4u * q + j);
+        load_quad(I.p, I.w_bf16 != 0u, q, v);
         store_quad(I.p, q, pack_quad(v, s_thr[item], 0u, 0u));
     }
     // 3. metadata padding
@@ -1466,6 +1510,7 @@ cudaError_t launch_pack_update_batch(const PackBatchItemHost *items, int n_items
             BatchItem &I = bp.it[i];
             const int64_t n_el = h.n_out * h.k;
             I.p.W = reinterpret_cast<const float4 *>(h.W);
+            I.w_bf16 = h.w_bf16 ? 1u : 0u;
             I.p.n_groups = n_el / 4;
             I.p.gpr = h.k / 4;
             I.p.gpr_div = make_fastdiv(static_cast<uint32_t>(h.k / 4));

@@ -199,6 +199,11 @@ def test_pack_update_batch_rejects_bad_arguments(lib):
         arr[1].W = w
         arr[1].out = ctypes.pointer(st)
         assert f(arr, 2, 1e-5, _fake(), ws, None) == want, (st.n_out, st.k, w)
+    arr[1].W = 4096
+    arr[1].out = ctypes.pointer(good)
+    arr[1].w_dtype = 5
+    assert f(arr, 2, 1e-5, _fake(), ws, None) == _abi.BITNET_ERR_INVALID_ARG       # bad master dtype
+    arr[1].w_dtype = _abi.BITNET_BF16
     half = _pw(n_out=256, k=256)
     half.mma_vals = 16384                                                       # vals without meta
     arr[1].W = 4096

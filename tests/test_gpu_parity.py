@@ -669,6 +669,47 @@ def test_pack_update_batch_matches_single(bn):
                 assert outs[i].gamma.item() == float(g) and np.array_equal(outs[i].group_bytes.cpu().numpy(), gb)
 
 
+def test_pack_update_batch_bf16_masters(bn):
+    """bf16 masters, mixed with fp32 ones in one batch: every matrix bit-identical
+    to bitnet_pack_nm of its values widened to fp32, and to the oracle, over
+    random-walk steps (rounded back to bf16 after every step)."""
+    shapes = [(256, 512), (200, 352), (640, 2560), (3200, 3200)]
+    bf = [True, False, True, True]
+    Ws32 = [synth.master_weights(n, k, 0.02, seed=970 + i) for i, (n, k) in enumerate(shapes)]
+    Wd, Wnp = [], []
+    for i, W in enumerate(Ws32):
+        if bf[i]:
+            d, w32 = bf16_dev(W)
+        else:
+            d, w32 = dev_f32(W), W
+        Wd.append(d)
+        Wnp.append(w32)
+    outs = [bn.PackedWeights(n, k, dec=(n % 16 == 0 and k % 64 == 0)) for (n, k) in shapes]
+    batch = bn.PackBatch([(Wd[i], outs[i]) for i in range(len(shapes))], 1e-5)
+    for step in range(4):
+        if step > 0:
+            for i in range(len(shapes)):
+                Wn = synth.random_walk_step(Wnp[i], 1e-4, seed=200 * step + i)
+                if bf[i]:
+                    d, Wn = bf16_dev(Wn)
+                    Wd[i].copy_(d)
+                else:
+                    Wd[i].copy_(dev_f32(Wn))
+                Wnp[i] = Wn
+        batch()
+        torch.cuda.synchronize()
+        for i, (n, k) in enumerate(shapes):
+            ref = bn.PackedWeights(n, k, dec=outs[i].dec_codes is not None)
+            bn.bitnet_pack_nm(dev_f32(Wnp[i]), ref, 1e-5)
+            torch.cuda.synchronize()
+            mask_dummy = torch.zeros(1, dtype=torch.uint8, device="cuda")
+            for a, b in zip(_pack_outputs(outs[i], mask_dummy), _pack_outputs(ref, mask_dummy)):
+                assert (a is None and b is None) or np.array_equal(a, b), (step, i)
+            if n * k <= 1 << 20:
+                g, keep, wq, gb = oracle.pack_weights(Wnp[i], 1e-5)
+                assert outs[i].gamma.item() == float(g) and np.array_equal(outs[i].group_bytes.cpu().numpy(), gb)
+
+
 def test_pack_update_batch_many_launch_groups(bn):
     """More matrices than one launch takes (70 > 64)."""
     n_items = 70
