@@ -348,10 +348,11 @@ cudaError_t launch_gemm_sp(const int8_t *Xq, const float *amax, const float *gam
 // Persistent CTAs walk 64 (n) x 64 (k) tiles.  Per tile, 64 threads bring the
 // 64 rows of 16 group bytes in with one 16-byte load each (issued one tile
 // ahead, so the load overlaps the previous tile's work) into a padded shared
-// tile.  Thread (g, c) then decodes the four group bytes of rows n = 4c..4c+3
-// at group g once into 2-bit codes per position and writes the four output
-// rows k = 4g..4g+3 of those four columns as 8-byte stores; sixteen threads
-// cover one 128-byte output row segment.
+// tile.  A 256-entry shared table holds, for every group byte, the bf16 values
+// of its four positions (8 bytes).  Thread (g, c) looks up the four group
+// bytes of rows n = 4c..4c+3 at group g and assembles the output rows
+// k = 4g..4g+3 of those four columns with byte permutes, as 8-byte stores;
+// sixteen threads cover one 128-byte output row segment.
 constexpr int kExpandRowWords = 17;   // 68-byte shared rows: the 16 column groups fall in different banks
 
 __device__ __forceinline__ uint4 expand_load(const uint8_t *__restrict__ gb, int64_t n_out, int64_t k, int64_t n,
@@ -371,19 +372,23 @@ __device__ __forceinline__ uint4 expand_load(const uint8_t *__restrict__ gb, int
     return v;
 }
 
-// 2-bit codes of the four positions of a group byte: code of position p at bits 2p..2p+1
-__device__ __forceinline__ uint32_t group_codes4(uint32_t b) {
-    const uint32_t i0 = b & 3u, i1 = (b >> 2) & 3u;
-    return (((b >> 4) & 3u) << (2 * i0)) | ((b >> 6) << (2 * i1));
-}
-
 // bf16 bits of a 2-bit code {0: 0, 1: +1 = 0x3f80, 3: -1 = 0xbf80}
 __device__ __forceinline__ uint32_t code_bf16(uint32_t code) { return (code & 1u) * 0x3f80u | ((code & 2u) << 14); }
+
+// the bf16 values of positions 0..3 of a group byte, position p in bits 16p..16p+15
+__device__ __forceinline__ uint2 group_bf16x4(uint32_t b) {
+    const uint32_t i0 = b & 3u, i1 = (b >> 2) & 3u;
+    const uint32_t c4 = (((b >> 4) & 3u) << (2 * i0)) | ((b >> 6) << (2 * i1));
+    return make_uint2(code_bf16(c4 & 3u) | (code_bf16((c4 >> 2) & 3u) << 16),
+                      code_bf16((c4 >> 4) & 3u) | (code_bf16(c4 >> 6) << 16));
+}
 
 __global__ void __launch_bounds__(256) k_expand_wt(const uint8_t *__restrict__ gb, int64_t n_out, int64_t k,
                                                    __nv_bfloat16 *__restrict__ wt) {
     __shared__ __align__(16) uint32_t s_gb[64 * kExpandRowWords];
+    __shared__ uint2 s_lut[256];
     const int tid = threadIdx.x;
+    s_lut[tid] = group_bf16x4(static_cast<uint32_t>(tid));
     const int64_t ktiles = (k + 63) / 64, ntiles = (n_out + 63) / 64;
     const int64_t tiles = ktiles * ntiles;
     int64_t tile = blockIdx.x;
@@ -392,7 +397,7 @@ __global__ void __launch_bounds__(256) k_expand_wt(const uint8_t *__restrict__ g
     const int g = tid >> 4, c = tid & 15;
     for (; tile < tiles; tile += gridDim.x) {
         const int64_t n0 = (tile / ktiles) * 64, k0 = (tile % ktiles) * 64;
-        __syncthreads();   // the previous tile's reads of s_gb are done
+        __syncthreads();   // the table is ready; the previous tile's reads of s_gb are done
         if (tid < 64) {
             uint32_t *row = s_gb + tid * kExpandRowWords;
             row[0] = v.x;
@@ -403,25 +408,28 @@ __global__ void __launch_bounds__(256) k_expand_wt(const uint8_t *__restrict__ g
         __syncthreads();
         const int64_t next = tile + gridDim.x;
         if (tid < 64 && next < tiles) v = expand_load(gb, n_out, k, (next / ktiles) * 64 + tid, (next % ktiles) * 64);
-        // four group bytes: rows 4c + i, group g
-        uint32_t cd[4];
+        // values of the four group bytes: rows 4c + i, group g
+        uint2 L[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t word = s_gb[(4 * c + i) * kExpandRowWords + (g >> 2)];
-            cd[i] = group_codes4((word >> (8 * (g & 3))) & 0xffu);
+            L[i] = s_lut[(word >> (8 * (g & 3))) & 0xffu];
         }
         const int64_t nb = n0 + 4 * c;
 #pragma unroll
         for (int pos = 0; pos < 4; ++pos) {
             const int64_t kk = k0 + 4 * g + pos;
             if (kk >= k) break;
-            uint32_t h[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) h[i] = code_bf16((cd[i] >> (2 * pos)) & 3u);
+            // position pos of columns nb..nb+3: bytes 2q, 2q+1 of the half holding it
+            constexpr uint32_t kSel[2] = {0x5410u, 0x7632u};
+            const uint32_t sel = kSel[pos & 1];
+            const uint32_t h01 = __byte_perm(pos < 2 ? L[0].x : L[0].y, pos < 2 ? L[1].x : L[1].y, sel);
+            const uint32_t h23 = __byte_perm(pos < 2 ? L[2].x : L[2].y, pos < 2 ? L[3].x : L[3].y, sel);
             __nv_bfloat16 *dst = wt + kk * n_out + nb;
             if (nb + 4 <= n_out) {
-                *reinterpret_cast<uint2 *>(dst) = make_uint2(h[0] | (h[1] << 16), h[2] | (h[3] << 16));
+                *reinterpret_cast<uint2 *>(dst) = make_uint2(h01, h23);
             } else {
+                const uint32_t h[4] = {h01 & 0xffffu, h01 >> 16, h23 & 0xffffu, h23 >> 16};
                 for (int i = 0; i < 4; ++i)
                     if (nb + i < n_out) reinterpret_cast<uint16_t *>(dst)[i] = static_cast<uint16_t>(h[i]);
             }
