@@ -244,6 +244,52 @@ bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, i
                                float eps, int8_t *Xq, float *absmax, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_rmsnorm_quant - RMSNorm fused into the per-token quantisation.
+ *
+ * "BitNet b1.58 ...", section "What this paper explains": the blocks around
+ * BitLinear are LLaMA-alike (RMSNorm, SwiGLU); section "The mechanism": the
+ * BitLinear input is quantised per token to [-127, 127].  Per token t:
+ *   S    = sum_k X[t,k]^2, exact, rounded once to fp64;
+ *   ms   = fp32(S / K);   r = fp32(1 / fp32(sqrt(fp32(ms + eps_norm))));
+ *   x_k  = fp32(X[t,k] * r), then fp32(x_k * w[k]) when w is given;
+ *   a[t] = max(max_k |x_k|, eps_act);  s = fp32(127 / a[t]);
+ *   Xq[t,k] = clamp(rint_half_even(fp32(x_k * s)), -127, 127).
+ * Every step is one IEEE fp32/fp64 operation in this order: the codes are the
+ * same bit for bit on any conforming implementation.
+ *
+ *   X        [T, K] bf16, 16-byte aligned, K % 8 == 0, K <= 65536.
+ *   w        [K] fp32 norm weight or NULL (no weight).
+ *   eps_norm > 0 (added to the mean square);  eps_act > 0 (absmax floor).
+ *   Xq       [T, K] int8 out, 16-byte aligned.  absmax [T] fp32 out (= a[t]).
+ *   rinv     [T] fp32 out (= r) or NULL.
+ * Errors: INVALID_ARG, UNSUPPORTED (T >= 2^31), CUDA.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_rmsnorm_quant(const void *X, const float *w, int64_t T, int64_t K, float eps_norm,
+                                   float eps_act, int8_t *Xq, float *absmax, float *rinv, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_swiglu_quant - SwiGLU gate fused into the per-token quantisation.
+ *
+ * Same pages and sections as bitnet_rmsnorm_quant.  Per token t and column f:
+ *   silu(g) = fp32(g / fp32(1 + exp32(-g)));   h = fp32(silu(g) * u);
+ * exp32(x): x clamped to [-87, 88]; n = rint(fp32(x * log2 e));
+ * r = fp32(fp32(x - fp32(n * C1)) - fp32(n * C2)) with ln 2 = C1 + C2
+ * (C1 = 0x3f317200, C2 = 0x35bfbe8e as fp32 bit patterns, log2 e =
+ * 0x3fb8aa3b); p = Horner form of the degree-6 Taylor polynomial of e^r with
+ * coefficients 1/720, 1/120, 1/24, 1/6 (0x3ab60b61, 0x3c088889, 0x3d2aaaab,
+ * 0x3e2aaaab), 1/2, 1, 1, one rounded multiply and one rounded add a step;
+ * exp32 = fp32(p * 2^n).  Then the codes of h exactly as bitnet_quant_act.
+ *
+ *   G, U     bf16, row t at G + t*ld and U + t*ld, F columns each (the gate
+ *            and up halves of one [T, 2F] buffer: U = G + F, ld = 2F).
+ *   F        % 8 == 0, F <= 51200;  ld >= F.   eps_act > 0.
+ *   Xq       [T, F] int8 out, 16-byte aligned.  absmax [T] fp32 out.
+ * Errors: INVALID_ARG, UNSUPPORTED (T >= 2^31), CUDA.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_swiglu_quant(const void *G, const void *U, int64_t ld, int64_t T, int64_t F, float eps_act,
+                                  int8_t *Xq, float *absmax, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * bitnet_sparse_linear - Y = dequant(Xq . Wq^T).
  *
  * "BitNet b1.58 ...", section "The mechanism": with ternary weights each

@@ -231,3 +231,66 @@ def forward_nm(W: np.ndarray, X: np.ndarray, n: int, m: int, eps_w: float = 1e-5
     acc = gemm_i32(Xq, wq)
     Y = dequant(acc, a, g)
     return dict(gamma=g, keep=keep, wq=wq, xq=Xq, a=a, acc=acc, y=Y)
+
+
+# ------------------------------------------------------------------ block epilogues fused into quantisation
+#
+# "BitNet b1.58: Ternary Weights for 1.58-bit LLMs", "What this paper explains"
+# item 3: the stack is LLaMA-alike (RMSNorm, SwiGLU, no biases).  The pages fix
+# no precision for these steps; the readings used here (and by the kernels):
+#   RMSNorm:  S_t = exact sum of x^2 over the row, rounded once to fp64;
+#             ms_t = fp32(S_t / K) (fp64 division, then fp32);
+#             r_t = fp32(1 / fp32(sqrt(fp32(ms_t + eps))));  x_n = fp32(x * r_t)
+#             [then fp32(x_n * w_k) when a weight is given]; then the usual
+#             per-token absmax int8 quantisation of x_n.
+#   SwiGLU:   h = fp32(silu(g) * u), silu(g) = fp32(g / fp32(1 + exp32(-g))),
+#             exp32 below; then the usual quantisation of h.
+
+def rmsnorm(X: np.ndarray, eps: float = 1e-6, w: np.ndarray | None = None, return_r: bool = False):
+    """RMSNorm of each row (the reading above); X holds fp32 values (bf16 widened).
+    With return_r, also the per-row fp32 factor r = 1 / sqrt(ms + eps)."""
+    import math
+    X = np.ascontiguousarray(X, dtype=np.float32)
+    T, K = X.shape
+    out = np.empty_like(X)
+    rs = np.empty((T,), np.float32)
+    for t in range(T):
+        sq = X[t].astype(np.float64) ** 2          # exact: squares of fp32 values fit fp64
+        S = math.fsum(sq.tolist())                 # exact sum, rounded once
+        ms = np.float32(S / K)
+        tt = np.float32(ms + np.float32(eps))
+        r = np.float32(np.float32(1.0) / np.sqrt(tt))
+        xn = (X[t] * r).astype(np.float32)
+        if w is not None:
+            xn = (xn * np.asarray(w, np.float32)).astype(np.float32)
+        out[t] = xn
+        rs[t] = r
+    return (out, rs) if return_r else out
+
+
+def exp32(x: np.ndarray) -> np.ndarray:
+    """exp in fp32 by Cody-Waite range reduction (x = n ln2 + r, ln2 split in two
+    parts) and the degree-6 Taylor polynomial of e^r on |r| <= ln2 / 2, each
+    step one IEEE fp32 operation (no fused multiply-add); x clamped to [-87, 88]."""
+    x = np.clip(np.asarray(x, np.float32), np.float32(-87.0), np.float32(88.0)).astype(np.float32)
+
+    def f(bits):   # constants as exact fp32 bit patterns
+        return np.uint32(bits).view(np.float32)
+    log2e, ln2_hi, ln2_lo = f(0x3fb8aa3b), f(0x3f317200), f(0x35bfbe8e)   # ln2_hi has 16 significant bits
+    n = np.rint((x * log2e).astype(np.float32)).astype(np.float32)
+    r = (x - (n * ln2_hi).astype(np.float32)).astype(np.float32)
+    r = (r - (n * ln2_lo).astype(np.float32)).astype(np.float32)
+    p = f(0x3ab60b61)                                                    # 1/720
+    for c in (f(0x3c088889), f(0x3d2aaaab), f(0x3e2aaaab), np.float32(0.5), np.float32(1.0), np.float32(1.0)):
+        p = ((p * r).astype(np.float32) + c).astype(np.float32)          # 1/120, 1/24, 1/6, 1/2, 1, 1
+    scale = ((n.astype(np.int32) + 127) << 23).astype(np.int32).view(np.float32)
+    return (p * scale).astype(np.float32)
+
+
+def swiglu(G: np.ndarray, U: np.ndarray) -> np.ndarray:
+    """h = silu(g) * u with the reading above (fp32)."""
+    G = np.ascontiguousarray(G, dtype=np.float32)
+    U = np.ascontiguousarray(U, dtype=np.float32)
+    e = exp32(-G)
+    silu = (G / (np.float32(1.0) + e).astype(np.float32)).astype(np.float32)
+    return (silu * U).astype(np.float32)

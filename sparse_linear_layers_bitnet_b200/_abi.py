@@ -29,7 +29,7 @@ EXPORTED = [
     "bitnet_pack_update_workspace_size", "bitnet_pack_nm_update",
     "bitnet_pack_update_batch_workspace_size", "bitnet_pack_nm_update_batch",
     "bitnet_pack_6of8_windows", "bitnet_quant_act_lift_6of8",
-    "bitnet_quant_act",
+    "bitnet_quant_act", "bitnet_rmsnorm_quant", "bitnet_swiglu_quant",
     "bitnet_linear_workspace_size", "bitnet_sparse_linear",
     "bitnet_quant_linear_workspace_size", "bitnet_quant_linear",
     "bitnet_decode_chain_workspace_size", "bitnet_decode_chain",
@@ -105,6 +105,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_pack_6of8_windows": (I32, [P, I64, F, ctypes.POINTER(BitnetPackedW), P, P, SZ, P]),
         "bitnet_quant_act_lift_6of8": (I32, [P, I32, I64, I64, F, P, P, P]),
         "bitnet_quant_act": (I32, [P, I32, I64, I64, F, P, P, P]),
+        "bitnet_rmsnorm_quant": (I32, [P, P, I64, I64, F, F, P, P, P, P]),
+        "bitnet_swiglu_quant": (I32, [P, P, I64, I64, I64, F, P, P, P]),
         "bitnet_linear_workspace_size": (SZ, []),
         "bitnet_sparse_linear": (I32, [P, P, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, P, SZ, P]),
         "bitnet_quant_linear_workspace_size": (SZ, [I64, I64]),
@@ -307,6 +309,43 @@ def bitnet_quant_act(X, eps: float = 1e-5, Xq=None, absmax=None, stream=None):
         absmax = torch.empty((T,), dtype=torch.float32, device=X.device)
     check(lib.bitnet_quant_act(_ptr(X), _dtype_code(X.dtype), T, K, ctypes.c_float(eps), _ptr(Xq), _ptr(absmax),
                                _stream(stream)), "bitnet_quant_act")
+    return Xq, absmax
+
+
+def bitnet_rmsnorm_quant(X, w=None, eps_norm: float = 1e-6, eps_act: float = 1e-5, Xq=None, absmax=None,
+                         rinv=None, stream=None):
+    """RMSNorm of each bf16 row of X (optional fp32 weight w), quantised per token to int8."""
+    torch = _torch()
+    lib = load()
+    assert X.is_contiguous() and X.dim() == 2 and X.dtype == torch.bfloat16
+    assert w is None or (w.is_contiguous() and w.dtype == torch.float32 and w.numel() == X.shape[1])
+    T, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((T, K), dtype=torch.int8, device=X.device)
+    if absmax is None:
+        absmax = torch.empty((T,), dtype=torch.float32, device=X.device)
+    check(lib.bitnet_rmsnorm_quant(_ptr(X), _ptr(w), T, K, ctypes.c_float(eps_norm), ctypes.c_float(eps_act),
+                                   _ptr(Xq), _ptr(absmax), _ptr(rinv), _stream(stream)), "bitnet_rmsnorm_quant")
+    return Xq, absmax
+
+
+def bitnet_swiglu_quant(GU, F: int | None = None, eps_act: float = 1e-5, Xq=None, absmax=None, stream=None):
+    """silu(gate) * up of a bf16 [T, 2F] buffer (gate = columns [0, F), up = [F, 2F)), quantised per token."""
+    torch = _torch()
+    lib = load()
+    assert GU.dim() == 2 and GU.dtype == torch.bfloat16 and GU.stride(1) == 1
+    T = GU.shape[0]
+    if F is None:
+        F = GU.shape[1] // 2
+    assert GU.shape[1] >= 2 * F
+    if Xq is None:
+        Xq = torch.empty((T, F), dtype=torch.int8, device=GU.device)
+    if absmax is None:
+        absmax = torch.empty((T,), dtype=torch.float32, device=GU.device)
+    G = GU.data_ptr()
+    U = G + 2 * F
+    check(lib.bitnet_swiglu_quant(ctypes.c_void_p(G), ctypes.c_void_p(U), GU.stride(0), T, F, ctypes.c_float(eps_act),
+                                  _ptr(Xq), _ptr(absmax), _stream(stream)), "bitnet_swiglu_quant")
     return Xq, absmax
 
 

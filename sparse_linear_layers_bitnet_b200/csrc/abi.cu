@@ -236,6 +236,34 @@ bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, i
                        "quant_act");
 }
 
+bitnet_status bitnet_rmsnorm_quant(const void *X, const float *w, int64_t T, int64_t K, float eps_norm,
+                                   float eps_act, int8_t *Xq, float *absmax, float *rinv, bitnet_stream_t stream) {
+    if (T < 0 || K <= 0 || K % 8 || K > 65536) return fail(BITNET_ERR_INVALID_ARG, "rmsnorm_quant: need T >= 0, 0 < K <= 65536, K %% 8 == 0");
+    if (!(eps_norm > 0.0f) || !(eps_act > 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "rmsnorm_quant: eps must be > 0");
+    if (T == 0) return BITNET_OK;
+    if (!X || !Xq || !absmax) return fail(BITNET_ERR_INVALID_ARG, "rmsnorm_quant: null pointer");
+    if (!aligned(X, 16) || !aligned(Xq, 16)) return fail(BITNET_ERR_INVALID_ARG, "rmsnorm_quant: X and Xq must be 16-byte aligned");
+    if (w && !aligned(w, 4)) return fail(BITNET_ERR_INVALID_ARG, "rmsnorm_quant: w must be 4-byte aligned");
+    if (T > 2147483647LL) return fail(BITNET_ERR_UNSUPPORTED, "rmsnorm_quant: T too large");
+    return cuda_status(bitnet::launch_rmsnorm_quant(X, w, T, K, eps_norm, eps_act, Xq, absmax, rinv,
+                                                    reinterpret_cast<cudaStream_t>(stream)),
+                       "rmsnorm_quant");
+}
+
+bitnet_status bitnet_swiglu_quant(const void *G, const void *U, int64_t ld, int64_t T, int64_t F, float eps_act,
+                                  int8_t *Xq, float *absmax, bitnet_stream_t stream) {
+    if (T < 0 || F <= 0 || F % 8 || ld < F) return fail(BITNET_ERR_INVALID_ARG, "swiglu_quant: need T >= 0, F > 0, F %% 8 == 0, ld >= F");
+    if (bitnet::swiglu_smem_bytes(F) > bitnet::kSwigluMaxSmem) return fail(BITNET_ERR_INVALID_ARG, "swiglu_quant: F too large");
+    if (!(eps_act > 0.0f)) return fail(BITNET_ERR_INVALID_ARG, "swiglu_quant: eps must be > 0");
+    if (T == 0) return BITNET_OK;
+    if (!G || !U || !Xq || !absmax) return fail(BITNET_ERR_INVALID_ARG, "swiglu_quant: null pointer");
+    if (!aligned(G, 2) || !aligned(U, 2) || !aligned(Xq, 16)) return fail(BITNET_ERR_INVALID_ARG, "swiglu_quant: alignment");
+    if (T > 2147483647LL) return fail(BITNET_ERR_UNSUPPORTED, "swiglu_quant: T too large");
+    return cuda_status(bitnet::launch_swiglu_quant(G, U, ld, T, F, eps_act, Xq, absmax,
+                                                   reinterpret_cast<cudaStream_t>(stream)),
+                       "swiglu_quant");
+}
+
 bitnet_status bitnet_sparse_linear(const int8_t *Xq, const float *absmax, const bitnet_packed_w *W, int64_t T,
                                    void *Y, bitnet_dtype y_dtype, int32_t *acc_out, void *ws, size_t ws_bytes,
                                    bitnet_stream_t stream) {

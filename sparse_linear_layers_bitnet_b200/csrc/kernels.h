@@ -73,6 +73,14 @@ cudaError_t launch_pack68(const float *W, int64_t n_out, int64_t k, float eps, f
 cudaError_t launch_quant_lift68(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xl, float *amax,
                                 cudaStream_t s);
 
+// Block epilogues fused into quantisation (block_quant.cu)
+constexpr size_t kSwigluMaxSmem = 200 * 1024;   // h of one token row in fp32
+size_t swiglu_smem_bytes(int64_t F);
+cudaError_t launch_rmsnorm_quant(const void *X, const float *w, int64_t T, int64_t K, float eps_n, float eps_a,
+                                 int8_t *Xq, float *amax, float *rinv, cudaStream_t s);
+cudaError_t launch_swiglu_quant(const void *G, const void *U, int64_t ld, int64_t T, int64_t F, float eps_a,
+                                int8_t *Xq, float *amax, cudaStream_t s);
+
 cudaError_t launch_gemv_dec(const int8_t *Xq, const float *amax, const float *gamma, const uint8_t *dec,
                             int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                             cudaStream_t s);

@@ -109,6 +109,30 @@ def test_quant_rejects_bad_arguments(lib):
     assert f(_fake(), 0, -1, 256, 1e-5, _fake(), _fake(), None) == _abi.BITNET_ERR_INVALID_ARG
 
 
+def test_block_quant_rejects_bad_arguments(lib):
+    f = lib.bitnet_rmsnorm_quant
+    ok = _abi.BITNET_OK
+    bad = _abi.BITNET_ERR_INVALID_ARG
+    assert f(None, None, 4, 256, 1e-6, 1e-5, _fake(), _fake(), None, None) == bad          # null X
+    assert f(_fake(), None, 4, 252, 1e-6, 1e-5, _fake(), _fake(), None, None) == bad       # K % 8
+    assert f(_fake(), None, 4, 65544, 1e-6, 1e-5, _fake(), _fake(), None, None) == bad     # K too large
+    assert f(_fake(), None, 4, 256, 0.0, 1e-5, _fake(), _fake(), None, None) == bad        # eps_norm
+    assert f(_fake(), None, 4, 256, 1e-6, -1.0, _fake(), _fake(), None, None) == bad       # eps_act
+    assert f(_fake(4104), None, 4, 256, 1e-6, 1e-5, _fake(), _fake(), None, None) == bad   # X alignment
+    assert f(_fake(), _fake(4098), 4, 256, 1e-6, 1e-5, _fake(), _fake(), None, None) == bad   # w alignment
+    assert f(_fake(), None, -1, 256, 1e-6, 1e-5, _fake(), _fake(), None, None) == bad
+    assert f(None, None, 0, 256, 1e-6, 1e-5, None, None, None, None) == ok                 # empty batch
+    g = lib.bitnet_swiglu_quant
+    assert g(None, _fake(), 512, 4, 256, 1e-5, _fake(), _fake(), None) == bad               # null G
+    assert g(_fake(), _fake(), 512, 4, 252, 1e-5, _fake(), _fake(), None) == bad            # F % 8
+    assert g(_fake(), _fake(), 100, 4, 256, 1e-5, _fake(), _fake(), None) == bad            # ld < F
+    assert g(_fake(), _fake(), 1 << 17, 4, 51208, 1e-5, _fake(), _fake(), None) == bad      # F beyond shared memory
+    assert g(_fake(), _fake(), 512, 4, 256, 0.0, _fake(), _fake(), None) == bad             # eps
+    assert g(_fake(4097), _fake(), 512, 4, 256, 1e-5, _fake(), _fake(), None) == bad        # G alignment
+    assert g(_fake(), _fake(), 512, 4, 256, 1e-5, _fake(4104), _fake(), None) == bad        # Xq alignment
+    assert g(None, None, 512, 0, 256, 1e-5, None, None, None) == ok                         # empty batch
+
+
 def test_linear_rejects_bad_arguments(lib):
     f = lib.bitnet_sparse_linear
     ws = lib.bitnet_linear_workspace_size()

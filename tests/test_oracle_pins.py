@@ -310,3 +310,59 @@ def test_quant_act_ties_golden():
     Xq, a = oracle.quant_act(X)
     assert Xq.ravel().tolist() == [int(v) for v in G["xq"]]
     assert a.tolist() == [float(v) for v in G["a"]]
+
+
+# ------------------------------------------------------------------ block epilogues (RMSNorm, SwiGLU)
+
+def test_exp32_within_5_ulp_of_exp_and_exact_at_zero():
+    x = np.linspace(-87.0, 88.0, 350001).astype(np.float32)
+    e = oracle.exp32(x).astype(np.float64)
+    ref = np.exp(x.astype(np.float64))
+    assert np.all(np.abs(e - ref) <= 5 * 2.0 ** -24 * ref)
+    assert oracle.exp32(np.zeros(3, np.float32)).tolist() == [1.0, 1.0, 1.0]
+    # at the reduction boundaries (x near n ln 2 for every n) the same bound holds
+    xs = (np.arange(-125, 127, dtype=np.float64) * math.log(2.0)).astype(np.float32)
+    xs = xs[(xs >= -87.0) & (xs <= 88.0)]
+    e2 = oracle.exp32(xs).astype(np.float64)
+    ref2 = np.exp(xs.astype(np.float64))
+    assert np.all(np.abs(e2 - ref2) <= 5 * 2.0 ** -24 * ref2)
+
+
+def test_swiglu_matches_fp64_and_limits():
+    r = np.random.default_rng(41)
+    G = (r.normal(size=(3, 2000)) * 6).astype(np.float32)
+    U = r.normal(size=(3, 2000)).astype(np.float32)
+    h = oracle.swiglu(G, U).astype(np.float64)
+    g64, u64 = G.astype(np.float64), U.astype(np.float64)
+    ref = g64 / (1.0 + np.exp(-g64)) * u64
+    assert np.all(np.abs(h - ref) <= 1e-6 * np.abs(ref) + 1e-30)
+    z = oracle.swiglu(np.zeros((1, 4), np.float32), np.ones((1, 4), np.float32))
+    assert z.tolist() == [[0.0, 0.0, 0.0, 0.0]]                      # silu(0) = 0
+    big = oracle.swiglu(np.full((1, 2), 60.0, np.float32), np.ones((1, 2), np.float32))
+    assert big.tolist() == [[60.0, 60.0]]                            # silu(g) = g for large g in fp32
+
+
+def test_rmsnorm_closed_forms_and_fp64():
+    import fractions
+    # constant row c: mean of squares is c^2 exactly
+    for c in (0.5, 3.0, 1.0 / 1024):
+        X = np.full((1, 3200), c, np.float32)
+        xn = oracle.rmsnorm(X, 1e-6)
+        ms = np.float32(c * c)
+        r = np.float32(np.float32(1.0) / np.sqrt(np.float32(ms + np.float32(1e-6))))
+        assert np.all(xn == np.float32(np.float32(c) * r))
+    # the exact sum: fsum of the squares equals the rational sum rounded once
+    r = np.random.default_rng(42)
+    X = (r.normal(size=(1, 257)) * 2.0 ** r.integers(-20, 10, size=(1, 257))).astype(np.float32)
+    exact = sum(fractions.Fraction(float(v)) ** 2 for v in X[0])
+    S = math.fsum((X[0].astype(np.float64) ** 2).tolist())
+    assert S == float(exact)
+    # against fp64 arithmetic on random rows
+    X = r.normal(size=(4, 3200)).astype(np.float32)
+    xn = oracle.rmsnorm(X, 1e-6).astype(np.float64)
+    ref = X / np.sqrt((X.astype(np.float64) ** 2).mean(1, keepdims=True) + 1e-6)
+    assert np.all(np.abs(xn - ref) <= 4 * 2.0 ** -24 * np.abs(ref))
+    # a weight scales the normalised row element by element
+    w = r.normal(size=3200).astype(np.float32)
+    xw = oracle.rmsnorm(X, 1e-6, w)
+    assert np.array_equal(xw, (oracle.rmsnorm(X, 1e-6) * w).astype(np.float32))
