@@ -62,7 +62,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--pack-layers", type=int, default=None, help="layers of the pack workload (default: all 26)")
     ap.add_argument("--flip-steps", type=int, default=100, help="random-walk steps of the mask flip-rate study")
-    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks", "six_eight"], default=None,
+    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks", "six_eight", "block"], default=None,
                     help="run one sub-measurement alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -603,6 +603,166 @@ def measure_dgrad(torch, bn, synth, peaks, reps=5):
     return out
 
 
+def _graph(torch, fn):
+    fn()   # first call outside capture (function attributes, lazy init)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def _time_graph(torch, g, flush, reps):
+    ts = []
+    for _ in range(reps):
+        flush_l2(torch, flush)
+        with Timer(torch) as t:
+            g.replay()
+        ts.append(t.ms())
+    return statistics.median(ts)
+
+
+def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
+    """One LLaMA-alike block at 3B shapes (hidden 3200, FFN 8640, 32 heads) over
+    T tokens, every BitLinear on the sparse ternary path: per-step pack of the
+    block's four matrices from fp32 masters; forward RMSNorm+quant -> QKV ->
+    causal attention -> quant -> O -> residual -> RMSNorm+quant -> gate|up ->
+    SwiGLU+quant -> down -> residual; STE dgrad of the four matrices.
+    Attention (torch SDPA) and the residual adds are library calls, timed and
+    listed apart.  Each stage is one CUDA graph timed alone after an L2 flush;
+    the whole step is one graph.  Context: the same block with dense bf16
+    weights through cuBLAS (torch.matmul) and torch elementwise ops."""
+    F = torch.nn.functional
+    dev = torch.device("cuda", torch.cuda.current_device())
+    h, f, H = synth.LLAMA_3B["hidden"], synth.LLAMA_3B["ffn"], synth.LLAMA_3B["heads"]
+    dh = h // H
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    mats = [("qkv", 3 * h, h), ("o", h, h), ("gate_up", 2 * f, h), ("down", h, f)]
+    lib = bn.load()
+    masters, pw = {}, {}
+    for i, (name, N, K) in enumerate(mats):
+        masters[name] = synth.torch_master_weights(N, K, 0.02, seed=300 + i, device=dev)
+        pw[name] = bn.PackedWeights(N, K, dev, group_bytes=True, mma=True, dec=False)
+        bn.bitnet_pack_nm(masters[name], pw[name], 1e-5)   # first pack sets each gamma hint
+    batch = bn.PackBatch([(masters[n], pw[n]) for n, _, _ in mats], 1e-5, dev)
+    ws_lin = bn.Workspace(lib.bitnet_linear_workspace_size(), dev)
+    ws_dg = bn.Workspace(max(lib.bitnet_dgrad_workspace_size(N, K) for _, N, K in mats), dev)
+    norm_w = (1.0 + 0.05 * torch.randn(h, device=dev)).float()
+    x = synth.torch_activations(T, h, seed=310, dtype=torch.bfloat16, device=dev)
+    bf = torch.bfloat16
+    buf = {
+        "xq1": torch.empty((T, h), dtype=torch.int8, device=dev), "a1": torch.empty(T, device=dev),
+        "qkv": torch.empty((T, 3 * h), dtype=bf, device=dev), "att": torch.empty((T, h), dtype=bf, device=dev),
+        "xq2": torch.empty((T, h), dtype=torch.int8, device=dev), "a2": torch.empty(T, device=dev),
+        "o": torch.empty((T, h), dtype=bf, device=dev), "x1": torch.empty((T, h), dtype=bf, device=dev),
+        "xq3": torch.empty((T, h), dtype=torch.int8, device=dev), "a3": torch.empty(T, device=dev),
+        "gu": torch.empty((T, 2 * f), dtype=bf, device=dev),
+        "xq4": torch.empty((T, f), dtype=torch.int8, device=dev), "a4": torch.empty(T, device=dev),
+        "d": torch.empty((T, h), dtype=bf, device=dev), "x2": torch.empty((T, h), dtype=bf, device=dev),
+    }
+    dY = {n: synth.torch_activations(T, N, seed=320 + i, dtype=bf, device=dev) for i, (n, N, K) in enumerate(mats)}
+    dX = {n: torch.empty((T, K), dtype=bf, device=dev) for n, N, K in mats}
+    b = buf
+
+    def s_pack():
+        batch()
+
+    def s_norm1():
+        bn.bitnet_rmsnorm_quant(x, norm_w, 1e-6, 1e-5, Xq=b["xq1"], absmax=b["a1"])
+
+    def s_qkv():
+        bn.bitnet_sparse_linear(b["xq1"], b["a1"], pw["qkv"], Y=b["qkv"], ws=ws_lin)
+
+    def s_attn():
+        q, k, v = b["qkv"].view(1, T, 3, H, dh).permute(2, 0, 3, 1, 4).unbind(0)
+        o = F.scaled_dot_product_attention(q, k, v, is_causal=True)
+        b["att"].copy_(o.transpose(1, 2).reshape(T, h))
+
+    def s_o():
+        bn.bitnet_quant_act(b["att"], 1e-5, Xq=b["xq2"], absmax=b["a2"])
+        bn.bitnet_sparse_linear(b["xq2"], b["a2"], pw["o"], Y=b["o"], ws=ws_lin)
+
+    def s_res1():
+        torch.add(x, b["o"], out=b["x1"])
+
+    def s_norm2():
+        bn.bitnet_rmsnorm_quant(b["x1"], norm_w, 1e-6, 1e-5, Xq=b["xq3"], absmax=b["a3"])
+
+    def s_gate_up():
+        bn.bitnet_sparse_linear(b["xq3"], b["a3"], pw["gate_up"], Y=b["gu"], ws=ws_lin)
+
+    def s_swiglu():
+        bn.bitnet_swiglu_quant(b["gu"], f, 1e-5, Xq=b["xq4"], absmax=b["a4"])
+
+    def s_down():
+        bn.bitnet_sparse_linear(b["xq4"], b["a4"], pw["down"], Y=b["d"], ws=ws_lin)
+
+    def s_res2():
+        torch.add(b["x1"], b["d"], out=b["x2"])
+
+    def s_dgrad():
+        for n, _, _ in mats:
+            bn.bitnet_dgrad(dY[n], pw[n], dX=dX[n], ws=ws_dg)
+
+    stages = [("pack", s_pack, "ours"), ("rmsnorm_quant_1", s_norm1, "ours"), ("qkv", s_qkv, "ours"),
+              ("attention", s_attn, "library"), ("quant_o", s_o, "ours"), ("residual_1", s_res1, "library"),
+              ("rmsnorm_quant_2", s_norm2, "ours"), ("gate_up", s_gate_up, "ours"),
+              ("swiglu_quant", s_swiglu, "ours"), ("down", s_down, "ours"), ("residual_2", s_res2, "library"),
+              ("dgrad_4", s_dgrad, "ours")]
+    out = {"T": T, "hidden": h, "ffn": f, "heads": H, "stages_ms": {}}
+    for name, fn, who in stages:
+        g = _graph(torch, fn)
+        out["stages_ms"][name] = {"ms": round(_time_graph(torch, g, flush, reps), 4), "impl": who}
+        del g
+
+    def step():
+        for _, fn, _ in stages:
+            fn()
+
+    g = _graph(torch, step)
+    step_ms = _time_graph(torch, g, flush, reps)
+    del g
+    st = out["stages_ms"]
+    ours_ms = sum(v["ms"] for v in st.values() if v["impl"] == "ours")
+    fwd_ops = 2.0 * T * sum(N * K for _, N, K in mats)
+    gemm_ms = sum(st[n]["ms"] for n in ("qkv", "gate_up", "down"))
+    out.update({
+        "step_ms": round(step_ms, 4),
+        "ours_ms": round(ours_ms, 4),
+        "library_ms": round(sum(v["ms"] for v in st.values() if v["impl"] == "library"), 4),
+        "forward_gemm_ops": fwd_ops,
+        "dgrad_tflops": round(fwd_ops / st["dgrad_4"]["ms"] / 1e9, 1),
+        "qkv_gate_up_down_tops": round(2.0 * T * sum(N * K for n, N, K in mats if n != "o") / gemm_ms / 1e9, 1),
+    })
+
+    # context: the same block with dense bf16 weights (cuBLAS through torch.matmul) and torch ops
+    Wd = {n: masters[n].to(bf) for n, _, _ in mats}
+    del masters, batch
+    tb = {"x1": torch.empty((T, h), dtype=bf, device=dev)}
+
+    def rms(v):
+        vf = v.float()
+        return (vf * torch.rsqrt(vf.pow(2).mean(-1, keepdim=True) + 1e-6) * norm_w).to(bf)
+
+    def t_step():
+        qkv = torch.matmul(rms(x), Wd["qkv"].t())
+        q, k, v = qkv.view(1, T, 3, H, dh).permute(2, 0, 3, 1, 4).unbind(0)
+        att = F.scaled_dot_product_attention(q, k, v, is_causal=True).transpose(1, 2).reshape(T, h)
+        x1 = x + torch.matmul(att, Wd["o"].t())
+        gu = torch.matmul(rms(x1), Wd["gate_up"].t())
+        hh = F.silu(gu[:, :f]) * gu[:, f:]
+        tb["x1"] = x1 + torch.matmul(hh, Wd["down"].t())
+        for n, _, _ in mats:
+            torch.matmul(dY[n], Wd[n])
+
+    g = _graph(torch, t_step)
+    out["torch_bf16_dense_step_ms"] = round(_time_graph(torch, g, flush, reps), 4)
+    del g, Wd
+    out["note"] = ("step = per-step pack + forward + STE dgrad of one block; the bf16 context runs the same "
+                   "block without the pack, on dense bf16 weights already in memory")
+    torch.cuda.empty_cache()
+    return out
 # ------------------------------------------------------------------ CPU oracle baseline
 
 def oracle_decode_sample(T, target_s):
@@ -682,7 +842,8 @@ def run_only(args):
     peaks = load_peaks()
     fn = {"prefill": measure_prefill, "pack": measure_pack, "dgrad": measure_dgrad,
           "peaks": lambda torch, bn, synth, peaks: measure_library_peaks(torch),
-          "six_eight": lambda torch, bn, synth, peaks: measure_6of8(torch, bn, synth)}[args.only]
+          "six_eight": lambda torch, bn, synth, peaks: measure_6of8(torch, bn, synth),
+          "block": measure_block}[args.only]
     kw = {"steps": args.steps, "flip_steps": args.flip_steps, "layers": args.pack_layers} if args.only == "pack" else {}
     print(json.dumps({args.only: fn(torch, bn, synth, peaks, **kw)}), flush=True)
     return 0
@@ -796,6 +957,7 @@ def run_ours(args):
         pc["frac_of_measured_int8_dense"] = round(pc["tops"] / lp, 4)
         rows["dgrad"] = measure_dgrad(torch, bn, synth, peaks)
         rows["six_eight"] = measure_6of8(torch, bn, synth)
+        rows["block"] = measure_block(torch, bn, synth, peaks)
         rows["pack"] = measure_pack(torch, bn, synth, peaks, flip_steps=args.flip_steps)
 
     line = {

@@ -45,11 +45,19 @@ def _rare_rows(X, rng):
         X[4, ::3] = 2e3
         X[4, 1::3] = 1e-25
         X[4, 2::7] = 0.0
+    sign = np.where(rng.random(K) < 0.5, -1.0, 1.0)
+    if T > 5:
+        X[5] = rng.uniform(512.0, 1020.0, K) * sign            # top of the window: largest exact chunk sums
+    if T > 6:
+        X[6] = rng.uniform(1.0, 2.0, K) * 2.0 ** -29 * sign    # bottom of the window: smallest chunk sums
     return X
 
 
+# K covers every register-cache width (chunks per thread 1, 2, 3, 4, 6, 8) and the
+# re-reading kernel beyond them (K = 65536)
 @pytest.mark.parametrize("T,K,weighted", [(1, 2560, False), (7, 3200, True), (64, 8192, False), (3, 8, True),
-                                          (9, 1000, False), (5, 65536, True), (130, 2048, True)])
+                                          (9, 1000, False), (5, 65536, True), (130, 2048, True), (6, 6144, True),
+                                          (5, 12288, False), (6, 16384, True), (4, 16392, True)])
 def test_rmsnorm_quant_parity(bn, T, K, weighted):
     rng = np.random.default_rng(T * 7 + K)
     X = synth.activations(T, K, seed=T + K, outlier_p=0.01)
@@ -63,6 +71,26 @@ def test_rmsnorm_quant_parity(bn, T, K, weighted):
     Xq, a = bn.bitnet_rmsnorm_quant(Xd, wd, 1e-6, 1e-5, rinv=rinv)
     torch.cuda.synchronize()
     assert np.array_equal(rinv.cpu().numpy().view(np.uint32), r_ref.view(np.uint32))
+    assert np.array_equal(a.cpu().numpy(), a_ref)
+    assert np.array_equal(Xq.cpu().numpy(), xq_ref)
+
+
+def test_rmsnorm_quant_unaligned_weight(bn):
+    """A weight vector without 16-byte alignment takes the kernel that reads it
+    one float at a time; same results."""
+    T, K = 6, 3200
+    rng = np.random.default_rng(11)
+    X = _rare_rows(synth.activations(T, K, seed=12, outlier_p=0.01), rng)
+    Xd, X32 = bf16_dev(X)
+    w = (1.0 + 0.1 * rng.standard_normal(K)).astype(np.float32)
+    wbuf = torch.zeros(K + 1, dtype=torch.float32, device="cuda")
+    wbuf[1:] = torch.from_numpy(w).cuda()
+    xn, r_ref = oracle.rmsnorm(X32, 1e-6, w, return_r=True)
+    xq_ref, a_ref = oracle.quant_act(xn, 1e-5)
+    rinv = torch.empty((T,), dtype=torch.float32, device="cuda")
+    Xq, a = bn.bitnet_rmsnorm_quant(Xd, wbuf[1:], 1e-6, 1e-5, rinv=rinv)
+    torch.cuda.synchronize()
+    assert np.array_equal(rinv.cpu().numpy(), r_ref)
     assert np.array_equal(a.cpu().numpy(), a_ref)
     assert np.array_equal(Xq.cpu().numpy(), xq_ref)
 
@@ -125,7 +153,10 @@ def _gate_values(T, F, rng):
     return G, U
 
 
-@pytest.mark.parametrize("T,F", [(1, 6912), (7, 8640), (33, 8192), (2, 8), (3, 1000), (300, 2048), (1, 51200)])
+# F covers every register-cache width (chunks per thread 1, 2, 3, 4, 6, 8) and the
+# kernel that keeps h in shared memory only (F beyond 16384)
+@pytest.mark.parametrize("T,F", [(1, 6912), (7, 8640), (33, 8192), (2, 8), (3, 1000), (300, 2048), (1, 51200),
+                                 (4, 3072), (5, 5120), (3, 16384), (2, 16392)])
 def test_swiglu_quant_parity(bn, T, F):
     rng = np.random.default_rng(T * 13 + F)
     G, U = _gate_values(T, F, rng)
@@ -139,9 +170,11 @@ def test_swiglu_quant_parity(bn, T, F):
     assert np.array_equal(Xq.cpu().numpy(), xq_ref)
 
 
-def test_swiglu_quant_strided_rows(bn):
-    """Gate and up halves inside a wider row (row stride > 2F)."""
-    T, F, extra = 5, 1024, 64
+@pytest.mark.parametrize("extra", [64, 3])
+def test_swiglu_quant_strided_rows(bn, extra):
+    """Gate and up halves inside a wider row (row stride > 2F; a stride that is
+    not a multiple of 8 takes the kernel with 2-byte loads)."""
+    T, F = 5, 1024
     rng = np.random.default_rng(5)
     G, U = _gate_values(T, F, rng)
     pad = rng.standard_normal((T, extra)).astype(np.float32)
