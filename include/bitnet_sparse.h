@@ -176,7 +176,10 @@ typedef struct {
     const void *W;
     bitnet_packed_w *out;
     uint8_t *mask_bits;
-    int32_t w_dtype;   /* bitnet_dtype of W */
+    int32_t w_dtype;       /* bitnet_dtype of W */
+    int32_t gamma_known;   /* nonzero: out->gamma already is the exact gamma of W
+                              (as bitnet_adamw_step writes it); the pack then
+                              reads W once, forms no sum and keeps out->gamma */
 } bitnet_pack_item;
 
 size_t bitnet_pack_update_batch_workspace_size(const bitnet_pack_item *items, int32_t n_items);
@@ -242,6 +245,56 @@ bitnet_status bitnet_quant_act_lift_6of8(const void *X, bitnet_dtype x_dtype, in
  * ------------------------------------------------------------------------ */
 bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, int64_t K,
                                float eps, int8_t *Xq, float *absmax, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_wgrad - weight gradient dW = dY^T . X (dense, every master).
+ *
+ * "Sparse-BitNet" (gist.science), section 2 "Training Strategie": the
+ * gradient passes straight through the quantiser and the 2:4 mask to all
+ * master weights, masked ones included; with both quantisers taken as the
+ * identity in the backward pass, dW[n, k] = sum_t dY[t, n] X[t, k], where X
+ * is the layer input (bf16) and dY the output gradient (bf16).
+ *   dY         [T, n_out] bf16, 16-byte aligned.   X  [T, k] bf16, 16-byte aligned.
+ *   n_out, k   positive multiples of 8; T >= 0.
+ *   dW         [n_out, k] fp32 out, 16-byte aligned; accumulate != 0 adds
+ *              the product to dW (gradient accumulation), else overwrites it
+ *              (T = 0: zeros).
+ *   ws         >= bitnet_wgrad_workspace_size() bytes (device status word).
+ * Products of bf16 values are exact in fp32; the sum is an fp32 tensor-core
+ * accumulation (order unspecified).
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+size_t bitnet_wgrad_workspace_size(void);
+bitnet_status bitnet_wgrad(const void *dY, const void *X, int64_t T, int64_t n_out, int64_t k, float *dW,
+                           int32_t accumulate, void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * bitnet_adamw_step - AdamW update of fp32 masters that also emits the exact
+ * absmean gamma of the updated matrix for the next pack.
+ *
+ * The pages keep latent fp32 masters and re-pack them every step ("BitNet
+ * b1.58 ...", section "What this paper explains"; "Sparse-BitNet"
+ * (gist.science), section 2 "Training Strategie"); they name no optimiser.
+ * Per element, each step one IEEE fp32 operation in this order:
+ *   m = b1 m + (1 - b1) g;   v = b2 v + (1 - b2) (g g);
+ *   u = (m / c1) / (sqrt(v / c2) + eps);   w = w - lr (u + wd w)
+ * with c1 = bias_correction1 = 1 - b1^t and c2 = 1 - b2^t supplied by the
+ * caller.  Then gamma_out = fp32(fp32(exact sum |w| / n) + eps_gamma), as
+ * bitnet_pack_nm forms it, so a pack item with gamma_known reads W once.
+ *   W, m, v    [n] fp32 in/out;  dW [n] fp32;  all 16-byte aligned; n % 4 == 0.
+ *   gamma_out  device fp32 scalar (normally the packed matrix's out->gamma).
+ *   ws         >= bitnet_adamw_workspace_size() bytes, 16-byte aligned.
+ * Errors: INVALID_ARG, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    float lr, beta1, beta2, eps, weight_decay;
+    float bias_correction1, bias_correction2;   /* 1 - beta1^t, 1 - beta2^t */
+} bitnet_adamw_hparams;
+
+size_t bitnet_adamw_workspace_size(void);
+bitnet_status bitnet_adamw_step(float *W, const float *dW, float *m, float *v, int64_t n,
+                                const bitnet_adamw_hparams *h, float eps_gamma, float *gamma_out, void *ws,
+                                size_t ws_bytes, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * bitnet_rmsnorm_quant - RMSNorm fused into the per-token quantisation.

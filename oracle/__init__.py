@@ -294,3 +294,33 @@ def swiglu(G: np.ndarray, U: np.ndarray) -> np.ndarray:
     e = exp32(-G)
     silu = (G / (np.float32(1.0) + e).astype(np.float32)).astype(np.float32)
     return (silu * U).astype(np.float32)
+
+
+def wgrad(dY: np.ndarray, X: np.ndarray) -> np.ndarray:
+    """dW[n, k] = sum_t dY[t, n] X[t, k] in fp64 ("Sparse-BitNet", section 2
+    "Training Strategie": gradients reach every master straight through the
+    quantisers and the mask; both quantisers act as the identity backward).
+    dY and X hold fp32 values (bf16 widened); products and sum in fp64."""
+    return np.asarray(dY, np.float64).T @ np.asarray(X, np.float64)
+
+
+def adamw(W, G, M, V, lr, b1, b2, eps, wd, c1, c2):
+    """One AdamW step in fp32, each operation rounded once, in this order:
+    m = b1 m + (1 - b1) g;  v = b2 v + (1 - b2) (g g);
+    u = (m / c1) / (sqrt(v / c2) + eps);  w = w - lr (u + wd w).
+    c1, c2 are the bias corrections 1 - b1^t, 1 - b2^t (inputs).  Returns
+    (W, M, V) as new fp32 arrays."""
+    f = np.float32
+    W, G, M, V = (np.asarray(a, f) for a in (W, G, M, V))
+    lr, b1, b2, eps, wd, c1, c2 = (f(x) for x in (lr, b1, b2, eps, wd, c1, c2))
+    omb1, omb2 = f(f(1.0) - b1), f(f(1.0) - b2)
+    M = (b1 * M).astype(f) + (omb1 * G).astype(f)
+    M = M.astype(f)
+    GG = (G * G).astype(f)
+    V = ((b2 * V).astype(f) + (omb2 * GG).astype(f)).astype(f)
+    mh = (M / c1).astype(f)
+    vh = (V / c2).astype(f)
+    den = (np.sqrt(vh).astype(f) + eps).astype(f)
+    u = (mh / den).astype(f)
+    W = (W - (lr * (u + (wd * W).astype(f)).astype(f)).astype(f)).astype(f)
+    return W, M, V

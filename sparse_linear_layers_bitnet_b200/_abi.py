@@ -34,6 +34,7 @@ EXPORTED = [
     "bitnet_quant_linear_workspace_size", "bitnet_quant_linear",
     "bitnet_decode_chain_workspace_size", "bitnet_decode_chain",
     "bitnet_dgrad_workspace_size", "bitnet_dgrad",
+    "bitnet_wgrad_workspace_size", "bitnet_wgrad", "bitnet_adamw_workspace_size", "bitnet_adamw_step",
     "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
 ]
 
@@ -58,7 +59,13 @@ class BitnetPackItem(ctypes.Structure):
         ("out", ctypes.POINTER(BitnetPackedW)),
         ("mask_bits", ctypes.c_void_p),
         ("w_dtype", ctypes.c_int32),
+        ("gamma_known", ctypes.c_int32),
     ]
+
+
+class BitnetAdamWHparams(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_float) for name in
+                ("lr", "beta1", "beta2", "eps", "weight_decay", "bias_correction1", "bias_correction2")]
 
 
 class BitnetChainOp(ctypes.Structure):
@@ -115,6 +122,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_decode_chain": (I32, [ctypes.POINTER(BitnetChainOp), I32, I64, I32, I32, F, P, SZ, P]),
         "bitnet_dgrad_workspace_size": (SZ, [I64, I64]),
         "bitnet_dgrad": (I32, [P, I32, ctypes.POINTER(BitnetPackedW), I64, P, I32, P, SZ, P]),
+        "bitnet_wgrad_workspace_size": (SZ, []),
+        "bitnet_wgrad": (I32, [P, P, I64, I64, I64, P, I32, P, SZ, P]),
+        "bitnet_adamw_workspace_size": (SZ, []),
+        "bitnet_adamw_step": (I32, [P, P, P, P, I64, ctypes.POINTER(BitnetAdamWHparams), F, P, P, SZ, P]),
         "bitnet_read_device_status": (I32, [P, P]),
         "bitnet_status_string": (ctypes.c_char_p, [I32]),
         "bitnet_last_error": (ctypes.c_char_p, []),
@@ -229,14 +240,15 @@ def bitnet_pack_nm_update(W, out: PackedWeights, eps: float = 1e-5, mask_bits=No
 
 class PackBatch:
     """A fixed list of (W, PackedWeights[, mask_bits]) for bitnet_pack_nm_update_batch
-    (W: fp32 or bf16 masters).
+    (W: fp32 or bf16 masters).  gamma_known: every out.gamma already is the exact
+    gamma of its W (as bitnet_adamw_step leaves it): one read of W, no sum.
 
     The descriptor array and the workspace are built once, so the same batch
     can be repacked every step (or captured in a CUDA graph) without
     rebuilding them.
     """
 
-    def __init__(self, items, eps: float = 1e-5, device="cuda"):
+    def __init__(self, items, eps: float = 1e-5, device="cuda", gamma_known: bool = False):
         lib = load()
         self.n = len(items)
         self.eps = float(eps)
@@ -252,6 +264,7 @@ class PackBatch:
             arr[i].w_dtype = _dtype_code(W.dtype)
             arr[i].out = ctypes.pointer(st)
             arr[i].mask_bits = mask.data_ptr() if mask is not None else None
+            arr[i].gamma_known = 1 if gamma_known else 0
         self._arr = arr
         self.ws = Workspace(lib.bitnet_pack_update_batch_workspace_size(arr, self.n), device)
 
@@ -266,6 +279,52 @@ def bitnet_pack_nm_update_batch(items, eps: float = 1e-5, stream=None) -> PackBa
     b = PackBatch(items, eps, items[0][0].device if items else "cuda")
     b(stream)
     return b
+
+
+def bitnet_wgrad(dY, X, dW=None, accumulate: bool = False, ws: "Workspace | None" = None, stream=None):
+    """dW[n, k] (+)= sum_t dY[t, n] X[t, k] (bf16 in, fp32 out)."""
+    torch = _torch()
+    lib = load()
+    assert dY.dtype == torch.bfloat16 and X.dtype == torch.bfloat16 and dY.is_contiguous() and X.is_contiguous()
+    T, n_out = dY.shape
+    assert X.shape[0] == T
+    k = X.shape[1]
+    if dW is None:
+        dW = torch.empty((n_out, k), dtype=torch.float32, device=dY.device)
+    if ws is None:
+        ws = Workspace(lib.bitnet_wgrad_workspace_size(), dY.device)
+    check(lib.bitnet_wgrad(_ptr(dY), _ptr(X), T, n_out, k, _ptr(dW), 1 if accumulate else 0, ws.ptr, ws.nbytes,
+                           _stream(stream)), "bitnet_wgrad")
+    return dW
+
+
+def bitnet_adamw_step(W, dW, m, v, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.95, eps: float = 1e-8,
+                      weight_decay: float = 0.0, gamma_out=None, eps_gamma: float = 1e-5,
+                      ws: "Workspace | None" = None, stream=None):
+    """AdamW on fp32 masters in place; writes the exact absmean gamma of the new W to gamma_out."""
+    torch = _torch()
+    lib = load()
+    for t in (W, dW, m, v):
+        assert t.dtype == torch.float32 and t.is_contiguous()
+    if gamma_out is None:
+        gamma_out = torch.empty(1, dtype=torch.float32, device=W.device)
+    if ws is None:
+        ws = Workspace(lib.bitnet_adamw_workspace_size(), W.device)
+    h = BitnetAdamWHparams(lr, beta1, beta2, eps, weight_decay, adam_bias_correction(beta1, step),
+                           adam_bias_correction(beta2, step))
+    check(lib.bitnet_adamw_step(_ptr(W), _ptr(dW), _ptr(m), _ptr(v), W.numel(), ctypes.byref(h),
+                                ctypes.c_float(eps_gamma), _ptr(gamma_out), ws.ptr, ws.nbytes, _stream(stream)),
+          "bitnet_adamw_step")
+    return gamma_out
+
+
+def adam_bias_correction(beta: float, step: int) -> float:
+    """fp32(1 - beta^step), with beta^step formed by repeated fp64 multiplication."""
+    import numpy as np
+    p = 1.0
+    for _ in range(step):
+        p *= float(np.float32(beta))
+    return float(np.float32(1.0 - p))
 
 
 def packed_6of8(n_out: int, k: int, device="cuda", mma=True, dec=False) -> "PackedWeights":

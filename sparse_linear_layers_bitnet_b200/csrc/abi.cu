@@ -170,7 +170,7 @@ bitnet_status bitnet_pack_nm_update_batch(const bitnet_pack_item *items, int32_t
         if (static_cast<double>(n_out) * static_cast<double>(k) / 4.0 > 4294967295.0)
             return fail(BITNET_ERR_UNSUPPORTED, "pack_update_batch: item %d: more than 2^32 groups", i);
         h[static_cast<size_t>(i)] = {it.W, n_out, k, out->gamma, out->group_bytes, out->mma_vals, out->mma_meta,
-                                     out->dec_codes, it.mask_bits, it.w_dtype == BITNET_BF16};
+                                     out->dec_codes, it.mask_bits, it.w_dtype == BITNET_BF16, it.gamma_known != 0};
     }
     const size_t need = bitnet_pack_update_batch_workspace_size(items, n_items);
     if (ws_bytes < need) return fail(BITNET_ERR_WORKSPACE, "pack_update_batch: workspace needs %zu bytes", need);
@@ -234,6 +234,51 @@ bitnet_status bitnet_quant_act(const void *X, bitnet_dtype x_dtype, int64_t T, i
     return cuda_status(bitnet::launch_quant_act(X, x_dtype == BITNET_BF16, T, K, eps, Xq, absmax,
                                                 reinterpret_cast<cudaStream_t>(stream)),
                        "quant_act");
+}
+
+size_t bitnet_wgrad_workspace_size(void) { return bitnet::kDgradWsHeader; }
+
+bitnet_status bitnet_wgrad(const void *dY, const void *X, int64_t T, int64_t n_out, int64_t k, float *dW,
+                           int32_t accumulate, void *ws, size_t ws_bytes, bitnet_stream_t stream) {
+    if (T < 0 || n_out <= 0 || k <= 0 || n_out % 8 || k % 8)
+        return fail(BITNET_ERR_INVALID_ARG, "wgrad: need T >= 0, n_out and k positive multiples of 8");
+    if (!dW) return fail(BITNET_ERR_INVALID_ARG, "wgrad: null dW");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "wgrad: workspace is required");
+    if (ws_bytes < bitnet_wgrad_workspace_size()) return fail(BITNET_ERR_WORKSPACE, "wgrad: workspace needs %zu bytes", bitnet_wgrad_workspace_size());
+    if (!aligned(dW, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "wgrad: dW and ws must be 16-byte aligned");
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (T == 0) {   // an empty sum: dW = 0, or unchanged when accumulating
+        if (accumulate) return BITNET_OK;
+        return cuda_status(cudaMemsetAsync(dW, 0, static_cast<size_t>(n_out) * static_cast<size_t>(k) * 4, s), "wgrad");
+    }
+    if (!dY || !X) return fail(BITNET_ERR_INVALID_ARG, "wgrad: null dY or X");
+    if (!aligned(dY, 16) || !aligned(X, 16)) return fail(BITNET_ERR_INVALID_ARG, "wgrad: dY and X must be 16-byte aligned");
+    if (T > 2147483647LL) return fail(BITNET_ERR_UNSUPPORTED, "wgrad: T too large");
+    return cuda_status(bitnet::launch_gemm_wgrad_pair(dY, X, T, n_out, k, dW, accumulate != 0,
+                                                      reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + bitnet::kStatusOffset), s),
+                       "wgrad");
+}
+
+size_t bitnet_adamw_workspace_size(void) { return bitnet::kPackWsBytes; }
+
+bitnet_status bitnet_adamw_step(float *W, const float *dW, float *m, float *v, int64_t n,
+                                const bitnet_adamw_hparams *h, float eps_gamma, float *gamma_out, void *ws,
+                                size_t ws_bytes, bitnet_stream_t stream) {
+    if (!h) return fail(BITNET_ERR_INVALID_ARG, "adamw: null hyper-parameters");
+    if (n <= 0 || n % 4) return fail(BITNET_ERR_INVALID_ARG, "adamw: n must be a positive multiple of 4");
+    if (!W || !dW || !m || !v || !gamma_out) return fail(BITNET_ERR_INVALID_ARG, "adamw: null pointer");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "adamw: workspace is required");
+    if (ws_bytes < bitnet_adamw_workspace_size()) return fail(BITNET_ERR_WORKSPACE, "adamw: workspace needs %zu bytes", bitnet_adamw_workspace_size());
+    if (!aligned(W, 16) || !aligned(dW, 16) || !aligned(m, 16) || !aligned(v, 16) || !aligned(ws, 16))
+        return fail(BITNET_ERR_INVALID_ARG, "adamw: W, dW, m, v and ws must be 16-byte aligned");
+    if (!(h->lr >= 0.0f) || !(h->beta1 >= 0.0f && h->beta1 < 1.0f) || !(h->beta2 >= 0.0f && h->beta2 < 1.0f) ||
+        !(h->eps > 0.0f) || !(h->weight_decay >= 0.0f) || !(h->bias_correction1 > 0.0f) ||
+        !(h->bias_correction2 > 0.0f) || !(eps_gamma >= 0.0f))
+        return fail(BITNET_ERR_INVALID_ARG, "adamw: hyper-parameters out of range");
+    return cuda_status(bitnet::launch_adamw_gamma(W, dW, m, v, n, h->lr, h->beta1, h->beta2, h->eps, h->weight_decay,
+                                                  h->bias_correction1, h->bias_correction2, eps_gamma, gamma_out, ws,
+                                                  reinterpret_cast<cudaStream_t>(stream)),
+                       "adamw");
 }
 
 bitnet_status bitnet_rmsnorm_quant(const void *X, const float *w, int64_t T, int64_t K, float eps_norm,

@@ -362,7 +362,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     if (tid >= kChainConsumers) {
         // ------------------------------------------------------------ producer
         if (tid != kChainConsumers) return;
-        uint32_t it = 0;
+        uint32_t it = 0, ps = 0, pph = 0;   // stages issued; slot it % ns; parity of fill round it / ns
         bool ok = true;
         for (int j = 0; j < p.n_ops && ok; ++j) {
             const ChainOpDev &op = p.op[j];
@@ -381,15 +381,18 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t *>(op.X) + l));
             }
             for (uint32_t off = 0; off < bytes; off += stage_bytes, ++it) {
-                const uint32_t s = it % static_cast<uint32_t>(ns);
-                if (it >= static_cast<uint32_t>(ns) &&
-                    !mbar_wait_sleep(&s_empty[s], ((it / ns) - 1u) & 1u, &s_abort, p.status)) {
+                // reuse of slot ps in round r >= 1 waits for the consumers' release of round r - 1
+                if (it >= static_cast<uint32_t>(ns) && !mbar_wait_sleep(&s_empty[ps], pph ^ 1u, &s_abort, p.status)) {
                     ok = false;
                     break;
                 }
                 const uint32_t n = (bytes - off) < stage_bytes ? (bytes - off) : stage_bytes;
-                mbar_arrive_expect_tx(&s_full[s], n);
-                bulk_load(ring + static_cast<size_t>(s) * stage_bytes, src + off, n, &s_full[s]);
+                mbar_arrive_expect_tx(&s_full[ps], n);
+                bulk_load(ring + static_cast<size_t>(ps) * stage_bytes, src + off, n, &s_full[ps]);
+                if (++ps == static_cast<uint32_t>(ns)) {
+                    ps = 0;
+                    pph ^= 1u;
+                }
             }
         }
         // drain: every issued stage must have landed before the CTA may exit
@@ -406,7 +409,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     // consumer barriers never miss a thread.
     const int ctid = tid;
     const int warp = ctid >> 5, lane = ctid & 31;
-    uint32_t it = 0;
+    uint32_t cs = 0, cph = 0;   // ring slot of the next stage and the parity of its fill round
     for (int j = 0; j < p.n_ops; ++j) {
         const ChainOpDev &op = p.op[j];
         int t0, t1;
@@ -444,9 +447,14 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             int cur = -1;
             int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
             bool failed = false;
-            for (uint32_t off = 0; off < bytes; off += stage_bytes, ++it) {
-                const uint32_t s = it % static_cast<uint32_t>(ns);
-                const bool ok = mbar_wait_full(&s_full[s], (it / ns) & 1u, &s_abort, p.status);
+            const float inv_kt = 1.0f / static_cast<float>(ktiles);
+            for (uint32_t off = 0; off < bytes; off += stage_bytes) {
+                const uint32_t s = cs;
+                const bool ok = mbar_wait_full(&s_full[s], cph, &s_abort, p.status);
+                if (++cs == static_cast<uint32_t>(ns)) {
+                    cs = 0;
+                    cph ^= 1u;
+                }
                 if (!__all_sync(0xffffffffu, ok)) {
                     failed = true;
                     break;
@@ -455,8 +463,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                 const int i0 = (warp * nrec) / kChainConsumerWarps, i1 = ((warp + 1) * nrec) / kChainConsumerWarps;
                 if (i0 < i1) {
                     const int r0 = static_cast<int>(off >> 8) + i0;
-                    int tile = static_cast<int>(static_cast<uint32_t>(r0) / static_cast<uint32_t>(ktiles));
+                    // r0 / ktiles through the reciprocal (r0 < 2^24: off by at most one, corrected)
+                    int tile = __float2int_rz(static_cast<float>(r0) * inv_kt);
                     int kt = r0 - tile * ktiles;
+                    if (kt < 0) {
+                        --tile;
+                        kt += ktiles;
+                    } else if (kt >= ktiles) {
+                        ++tile;
+                        kt -= ktiles;
+                    }
                     const uint2 *rec = reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(s) * stage_bytes) + lane;
                     int i = i0;
                     while (i < i1) {

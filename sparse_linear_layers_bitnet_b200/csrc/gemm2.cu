@@ -120,7 +120,11 @@ __device__ __forceinline__ void commit_both(uint64_t *bar) {
 
 }  // namespace pair
 
-template <bool SPARSE, int BN, int STAGES>
+// MN: dense operands stored with the M (A) and N (B) dimension contiguous
+// ("MN-major"): tiles arrive as 64-element-wide boxes of 64 k-rows, 128-byte
+// swizzled; the descriptors step 8 KB between 64-wide boxes (leading byte
+// offset) and 1 KB between groups of 8 k-rows (stride byte offset).
+template <bool SPARSE, int BN, int STAGES, bool MN = false>
 struct PairCfg {
     static constexpr int kHalfN = BN / 2;                  // B rows per CTA
     static constexpr int kARowBytes = SPARSE ? 64 : 128;
@@ -140,11 +144,14 @@ struct PairCfg {
     static constexpr int kSmemBytes = STAGES * kStageBytes + kStageOutBytes + 1024 + 2048;
     // M = 256 (two CTAs), N = BN
     static constexpr uint32_t kIdesc = (SPARSE ? (1u << 2) : 0u) | ((SPARSE ? 2u : 1u) << 4) | (1u << 7) |
-                                       (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-                                       (static_cast<uint32_t>(256 >> 4) << 24);
+                                       (1u << 10) | (MN ? (1u << 15) | (1u << 16) : 0u) |
+                                       (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
+    static constexpr int kMnBox = 64 * 64 * 2;             // one 64 (MN) x 64 (k) bf16 box
+    static constexpr int kMnAdvance = 2 * 1024;            // 16 k-rows per MMA
     static_assert(!SPARSE || (BN % 32 == 0 && BN <= 224), "sparse pair tiles: N multiple of 32, two buffers + metadata");
     static_assert(SPARSE || (BN % 32 == 0 && BN <= 256), "dense pair tiles: N multiple of 32");
     static_assert(kBBytes % 1024 == 0, "B tile must keep the 128-byte swizzle atoms aligned");
+    static_assert(!MN || (!SPARSE && kHalfN % 64 == 0), "MN-major tiles: dense, whole 64-wide boxes");
 };
 
 struct PairParams {
@@ -157,13 +164,14 @@ struct PairParams {
     int out_bf16;
     int32_t *acc_out;
     uint32_t *status;
+    int accumulate;              // dense fp32 output: out += result (else out = result)
 };
 
-template <bool SPARSE, int BN, int STAGES>
+template <bool SPARSE, int BN, int STAGES, bool MN = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     k_umma_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY, PairParams p) {
-    using C = PairCfg<SPARSE, BN, STAGES>;
+    using C = PairCfg<SPARSE, BN, STAGES, MN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
@@ -234,6 +242,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                         pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
                         pair::tma_load_2d_pair(&tmE, &full[s], sE + s * C::kEBytes, 0,
                                                static_cast<int32_t>((kt * p.meta_rows + e_row) / 8));
+                    } else if (MN) {
+                        // boxes of 64 MN-elements x 64 k-rows: two for A's 128 rows, kHalfN / 64 for B
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes + h * C::kMnBox, a_row + 64 * h,
+                                                   kt * C::kKStep);
+#pragma unroll
+                        for (int h = 0; h < C::kHalfN / 64; ++h)
+                            pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes + h * C::kMnBox, b_row + 64 * h,
+                                                   kt * C::kKStep);
                     } else {
                         pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * C::kKStep, a_row);
                         pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
@@ -266,6 +284,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                             const uint64_t ad = make_smem_desc(a_base + j * C::kAAdvance, 16, 512, kSwizzle64B);
                             const uint64_t bd = make_smem_desc(b_base + j * C::kBAdvance, 16, 1024, kSwizzle128B);
                             pair::mma_sp_i8_pair(d_tmem, ad, bd, C::kIdesc, e_col + 2u * j, (kt | j) != 0);
+                        }
+                    } else if (MN) {
+#pragma unroll
+                        for (int j = 0; j < C::kMmaPerStage; ++j) {
+                            const uint64_t ad = make_smem_desc(a_base + j * C::kMnAdvance, C::kMnBox, 1024, kSwizzle128B);
+                            const uint64_t bd = make_smem_desc(b_base + j * C::kMnAdvance, C::kMnBox, 1024, kSwizzle128B);
+                            pair::mma_bf16_pair(d_tmem, ad, bd, C::kIdesc, (kt | j) != 0);
                         }
                     } else {
 #pragma unroll
@@ -360,7 +385,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                             }
                         }
                     } else {
-                        const float g = *p.gamma;
+                        const float g = p.gamma ? *p.gamma : 1.0f;
                         const int64_t nb = n0 + 16 * c;
                         if (nb + 16 <= p.N) {
                             if (p.out_bf16) {
@@ -377,11 +402,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                             } else {
                                 float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.out) + m * p.N + nb);
 #pragma unroll
-                                for (int j = 0; j < 4; ++j)
-                                    dst[j] = make_float4(__fmul_rn(__uint_as_float(r[4 * j]), g),
-                                                         __fmul_rn(__uint_as_float(r[4 * j + 1]), g),
-                                                         __fmul_rn(__uint_as_float(r[4 * j + 2]), g),
-                                                         __fmul_rn(__uint_as_float(r[4 * j + 3]), g));
+                                for (int j = 0; j < 4; ++j) {
+                                    float4 y = make_float4(__fmul_rn(__uint_as_float(r[4 * j]), g),
+                                                           __fmul_rn(__uint_as_float(r[4 * j + 1]), g),
+                                                           __fmul_rn(__uint_as_float(r[4 * j + 2]), g),
+                                                           __fmul_rn(__uint_as_float(r[4 * j + 3]), g));
+                                    if (p.accumulate) {
+                                        const float4 o = dst[j];
+                                        y = make_float4(__fadd_rn(o.x, y.x), __fadd_rn(o.y, y.y), __fadd_rn(o.z, y.z),
+                                                        __fadd_rn(o.w, y.w));
+                                    }
+                                    dst[j] = y;
+                                }
                             }
                         } else {
 #pragma unroll
@@ -391,6 +423,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                                     const float y = __fmul_rn(__uint_as_float(r[j]), g);
                                     if (p.out_bf16)
                                         static_cast<__nv_bfloat16 *>(p.out)[m * p.N + n] = __float2bfloat16_rn(y);
+                                    else if (p.accumulate)
+                                        static_cast<float *>(p.out)[m * p.N + n] =
+                                            __fadd_rn(static_cast<float *>(p.out)[m * p.N + n], y);
                                     else
                                         static_cast<float *>(p.out)[m * p.N + n] = y;
                                 }
@@ -447,11 +482,11 @@ static bool map2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, ui
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool SPARSE, int BN, int STAGES>
+template <bool SPARSE, int BN, int STAGES, bool MN = false>
 static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &e, const CUtensorMap &y,
                             const PairParams &p, cudaStream_t s) {
-    using C = PairCfg<SPARSE, BN, STAGES>;
-    auto kern = k_umma_pair<SPARSE, BN, STAGES>;
+    using C = PairCfg<SPARSE, BN, STAGES, MN>;
+    auto kern = k_umma_pair<SPARSE, BN, STAGES, MN>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -526,6 +561,30 @@ cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *wt, const
                static_cast<uint64_t>(n_out) * 2, 64, static_cast<uint32_t>(BN / 2), CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     return run_pair<false, BN, 6>(ma, mb, ma, ma, p, s);
+}
+
+// Weight gradient dW[n, k] (+)= sum_t dY[t, n] X[t, k]: A = dY and B = X both
+// with the contraction index t as the outer (row) index, i.e. MN-major tiles.
+cudaError_t launch_gemm_wgrad_pair(const void *dY, const void *X, int64_t T, int64_t n_out, int64_t k, float *dW,
+                                   bool accumulate, uint32_t *status, cudaStream_t s) {
+    constexpr int BN = 256;
+    PairParams p{};
+    p.M = n_out;
+    p.N = k;
+    p.K = T;
+    p.gamma = nullptr;   // scale 1
+    p.out = dW;
+    p.out_bf16 = 0;
+    p.accumulate = accumulate ? 1 : 0;
+    p.status = status;
+    CUtensorMap ma, mb;
+    if (!map2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, static_cast<uint64_t>(n_out), static_cast<uint64_t>(T),
+               static_cast<uint64_t>(n_out) * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    if (!map2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(k), static_cast<uint64_t>(T),
+               static_cast<uint64_t>(k) * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    return run_pair<false, BN, 6, true>(ma, mb, ma, ma, p, s);
 }
 
 }  // namespace bitnet

@@ -59,6 +59,7 @@ struct PackBatchItemHost {
     uint8_t *dec;
     uint8_t *mask;
     bool w_bf16;
+    bool gamma_known;   // *gamma is already the exact gamma of W (from the optimiser step)
 };
 constexpr int kPackBatchMax = 64;   // matrices per launch (kernel parameter space)
 size_t pack_batch_ws_bytes(const int64_t *n_out, const int64_t *k, int n_items);
@@ -72,6 +73,15 @@ cudaError_t launch_pack68(const float *W, int64_t n_out, int64_t k, float eps, f
                           int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws, cudaStream_t s);
 cudaError_t launch_quant_lift68(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xl, float *amax,
                                 cudaStream_t s);
+
+// AdamW step of fp32 masters that also emits the exact absmean gamma of the result (pack.cu)
+cudaError_t launch_adamw_gamma(float *W, const float *G, float *M, float *V, int64_t n, float lr, float b1, float b2,
+                               float eps, float wd, float c1, float c2, float eps_gamma, float *gamma, void *ws,
+                               cudaStream_t s);
+
+// Weight gradient (gemm2.cu)
+cudaError_t launch_gemm_wgrad_pair(const void *dY, const void *X, int64_t T, int64_t n_out, int64_t k, float *dW,
+                                   bool accumulate, uint32_t *status, cudaStream_t s);
 
 // Block epilogues fused into quantisation (block_quant.cu)
 constexpr size_t kSwigluMaxSmem = 200 * 1024;   // h of one token row in fp32

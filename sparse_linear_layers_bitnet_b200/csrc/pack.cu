@@ -767,6 +767,147 @@ __global__ void __launch_bounds__(256, 4) k_abs_sum_fast(const float4 *__restric
     }
 }
 
+// ---------------------------------------------------------------- optimiser step emitting the next gamma
+//
+// "Sparse-BitNet" (gist.science), section 2 "Training Strategie": the
+// gradient passes straight through the quantiser and the mask to every fp32
+// master, so the optimiser updates all of them each step; the next step's pack
+// needs the absmean of the updated masters ("BitNet b1.58 ...", section "The
+// mechanism").  The update kernel therefore also sums |W_new| exactly (the
+// same accumulators as k_abs_sum_fast) and its last block forms gamma and the
+// code threshold: the following pack reads W once and needs no sum.
+//
+// AdamW, every step one IEEE fp32 operation in this order (no fused
+// multiply-add): m = b1 m + (1 - b1) g; v = b2 v + (1 - b2) (g g);
+// u = (m / c1) / (sqrt(v / c2) + eps); w = w - lr (u + wd w), with the bias
+// corrections c1 = 1 - b1^t and c2 = 1 - b2^t given by the caller.
+struct AdamWArgs {
+    float4 *W;
+    const float4 *G;
+    float4 *M, *V;
+    int64_t n4;
+    float lr, b1, b2, eps, wd, c1, c2;
+    unsigned long long *win, *bins;
+    unsigned *counter;
+    int64_t n_total;
+    float eps_gamma;
+    float *gamma;
+    uint32_t *thr;
+};
+
+__device__ __forceinline__ float adamw1(float w, float g, float &m, float &v, const AdamWArgs &a, float omb1,
+                                        float omb2) {
+    m = __fadd_rn(__fmul_rn(a.b1, m), __fmul_rn(omb1, g));
+    v = __fadd_rn(__fmul_rn(a.b2, v), __fmul_rn(omb2, __fmul_rn(g, g)));
+    const float u = __fdiv_rn(__fdiv_rn(m, a.c1), __fadd_rn(__fsqrt_rn(__fdiv_rn(v, a.c2)), a.eps));
+    return __fsub_rn(w, __fmul_rn(a.lr, __fadd_rn(u, __fmul_rn(a.wd, w))));
+}
+
+__global__ void __launch_bounds__(256, 4) k_adamw_gamma(const __grid_constant__ AdamWArgs a) {
+    __shared__ unsigned long long s_bins[256];
+    __shared__ unsigned long long s_lo[8], s_hi[8];
+    __shared__ int s_rare;
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0ull;
+    if (threadIdx.x == 0) s_rare = 0;
+    __syncthreads();
+    const float omb1 = __fsub_rn(1.0f, a.b1), omb2 = __fsub_rn(1.0f, a.b2);
+    uint64_t lo = 0, hi = 0;
+    double d = 0.0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    constexpr int kU = 4;   // float4 groups per thread per round (16 loads in flight)
+    for (; i < a.n4; i += kU * stride) {
+        float4 w[kU], g[kU], m[kU], v[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t j = i + u * stride;
+            if (j < a.n4) {
+                w[u] = a.W[j];
+                g[u] = __ldg(a.G + j);
+                m[u] = a.M[j];
+                v[u] = a.V[j];
+            } else {
+                w[u] = g[u] = m[u] = v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t j = i + u * stride;
+            if (j < a.n4) {
+                float4 wn;
+                wn.x = adamw1(w[u].x, g[u].x, m[u].x, v[u].x, a, omb1, omb2);
+                wn.y = adamw1(w[u].y, g[u].y, m[u].y, v[u].y, a, omb1, omb2);
+                wn.z = adamw1(w[u].z, g[u].z, m[u].z, v[u].z, a, omb1, omb2);
+                wn.w = adamw1(w[u].w, g[u].w, m[u].w, v[u].w, a, omb1, omb2);
+                a.W[j] = wn;
+                a.M[j] = m[u];
+                a.V[j] = v[u];
+                sum_float4(wn, d, lo, hi, s_bins, &s_rare);
+            }
+        }
+        flush_sum(d, lo, hi);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const uint64_t l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+        const uint64_t h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+        const uint64_t sum = lo + l2;
+        hi = hi + h2 + ((sum < lo) ? 1ull : 0ull);
+        lo = sum;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        s_lo[warp] = lo;
+        s_hi[warp] = hi;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint64_t L = 0, H = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+            const uint64_t sum = L + s_lo[w];
+            H = H + s_hi[w] + ((sum < L) ? 1ull : 0ull);
+            L = sum;
+        }
+        if (L | H) {
+            const unsigned long long old = atomicAdd(&a.win[0], static_cast<unsigned long long>(L));
+            const uint64_t carry = (static_cast<uint64_t>(old) + L < static_cast<uint64_t>(old)) ? 1ull : 0ull;
+            atomicAdd(&a.win[1], static_cast<unsigned long long>(H + carry));
+        }
+    }
+    if (s_rare) {
+        for (int e = threadIdx.x; e < 256; e += blockDim.x)
+            if (s_bins[e]) atomicAdd(&a.bins[e], s_bins[e]);
+    }
+    __shared__ unsigned s_ticket;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_ticket = atomicAdd(a.counter, 1u);
+    __syncthreads();
+    if (s_ticket != gridDim.x - 1) return;
+    __threadfence();
+    __shared__ int s_nz[256];
+    __shared__ int s_nnz;
+    __shared__ uint32_t s_limb[kLimbs];
+    if (threadIdx.x == 0) s_nnz = 0;
+    __syncthreads();
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+        const unsigned long long b = atomicAdd(&a.bins[e], 0ull);
+        s_bins[e] = b;
+        if (b) s_nz[atomicAdd(&s_nnz, 1)] = e;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int q = 1; q < s_nnz; ++q)
+            for (int j = q; j > 0 && s_nz[j - 1] > s_nz[j]; --j) {
+                const int tmp = s_nz[j];
+                s_nz[j] = s_nz[j - 1];
+                s_nz[j - 1] = tmp;
+            }
+        const uint64_t wlo = atomicAdd(&a.win[0], 0ull), whi = atomicAdd(&a.win[1], 0ull);
+        finalize_gamma(s_bins, s_nz, s_nnz, wlo, whi, a.n_total, a.eps_gamma, s_limb, a.gamma, a.thr);
+    }
+}
+
 // pass 2 of bitnet_pack_nm (and the full pass of the update): lane quads
 __device__ __forceinline__ void quad_pass(const Pack24Args &p, uint32_t thr) {
     const uint32_t n_quads = static_cast<uint32_t>(p.n_groups >> 2);
@@ -1108,6 +1249,36 @@ cudaError_t launch_pack(const float *W, int64_t n_out, int64_t k, int n, int m, 
     return cudaGetLastError();
 }
 
+cudaError_t launch_adamw_gamma(float *W, const float *G, float *M, float *V, int64_t n, float lr, float b1, float b2,
+                               float eps, float wd, float c1, float c2, float eps_gamma, float *gamma, void *ws,
+                               cudaStream_t s) {
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    cudaError_t err = cudaMemsetAsync(ws, 0, kPackWsBytes, s);
+    if (err != cudaSuccess) return err;
+    AdamWArgs a;
+    a.W = reinterpret_cast<float4 *>(W);
+    a.G = reinterpret_cast<const float4 *>(G);
+    a.M = reinterpret_cast<float4 *>(M);
+    a.V = reinterpret_cast<float4 *>(V);
+    a.n4 = n / 4;
+    a.lr = lr;
+    a.b1 = b1;
+    a.b2 = b2;
+    a.eps = eps;
+    a.wd = wd;
+    a.c1 = c1;
+    a.c2 = c2;
+    a.win = reinterpret_cast<unsigned long long *>(w8 + kPackWsWinOffset);
+    a.bins = reinterpret_cast<unsigned long long *>(w8 + kPackWsBinsOffset);
+    a.counter = reinterpret_cast<unsigned *>(w8 + kPackWsCounterOffset);
+    a.n_total = n;
+    a.eps_gamma = eps_gamma;
+    a.gamma = gamma;
+    a.thr = reinterpret_cast<uint32_t *>(w8 + kPackWsThrOffset);
+    k_adamw_gamma<<<grid_for((a.n4 + 3) / 4, 256, 4), 256, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pack_update(const float *W, int64_t n_out, int64_t k, float eps, float *gamma, uint8_t *gb,
                                int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws, size_t ws_bytes,
                                cudaStream_t s) {
@@ -1184,6 +1355,7 @@ struct BatchItem {
     uint32_t chunk0, nchunks;  // this matrix's range of the global chunk list
     uint32_t pad_bytes;        // metadata padding bytes (0: none)
     uint32_t w_bf16;           // 1: the masters (p.W) are bf16, widened exactly to fp32 on load
+    uint32_t gamma_known;      // 1: *gamma already is the exact gamma of W (no sum, no band, gamma kept)
     int64_t n_total;
 };
 
@@ -1235,7 +1407,7 @@ __device__ __forceinline__ int batch_item_of(const BatchParams &bp, uint32_t c) 
 // One CTA's run of chunks [c, seg_end) of one matrix: exact partial sum of
 // |W| (into lo, hi) and, with a hint, every layout with the hint's threshold
 // plus the band list.  BF16: the masters are bf16.
-template <bool BF16>
+template <bool BF16, bool KNOWN>
 __device__ __forceinline__ void batch_segment(const BatchItem &I, uint32_t c, uint32_t seg_end, bool hint,
                                               uint32_t t_old, uint32_t t_lo, uint32_t t_hi, unsigned *list_count,
                                               uint64_t &lo, uint64_t &hi, unsigned long long *s_bins, int *s_rare) {
@@ -1259,8 +1431,10 @@ __device__ __forceinline__ void batch_segment(const BatchItem &I, uint32_t c, ui
 #pragma unroll
         for (int k2 = 0; k2 < kQuadUnroll; ++k2) {
             const uint32_t q = qbase + 32u * k2 + lane;
+            if (!KNOWN) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) sum_float4(v[k2][j], d, lo, hi, s_bins, s_rare);
+                for (int j = 0; j < 4; ++j) sum_float4(v[k2][j], d, lo, hi, s_bins, s_rare);
+            }
             if (hint && q < n_quads) {
                 const QuadOut o = pack_quad(v[k2], t_old, t_lo, t_hi);
                 store_quad(p, q, o);
@@ -1321,10 +1495,19 @@ __global__ void __launch_bounds__(256, 4) k_pack_update_batch(const __grid_const
         const bool wbf16 = I.w_bf16 != 0u;
         unsigned *list_count = reinterpret_cast<unsigned *>(hdr + kPackWsListCountOffset);
         uint64_t lo = 0, hi = 0;
-        if (wbf16)
-            batch_segment<true>(I, c, seg_end, hint, t_old, t_lo, t_hi, list_count, lo, hi, s_bins, &s_rare);
-        else
-            batch_segment<false>(I, c, seg_end, hint, t_old, t_lo, t_hi, list_count, lo, hi, s_bins, &s_rare);
+        const bool known = hint && I.gamma_known != 0u;
+        if (known) {   // codes against the exact threshold: nothing to sum, no band to list
+            if (wbf16)
+                batch_segment<true, true>(I, c, seg_end, true, t_old, 0xffffffffu, 0xffffffffu, list_count, lo, hi,
+                                          s_bins, &s_rare);
+            else
+                batch_segment<false, true>(I, c, seg_end, true, t_old, 0xffffffffu, 0xffffffffu, list_count, lo, hi,
+                                           s_bins, &s_rare);
+        } else if (wbf16) {
+            batch_segment<true, false>(I, c, seg_end, hint, t_old, t_lo, t_hi, list_count, lo, hi, s_bins, &s_rare);
+        } else {
+            batch_segment<false, false>(I, c, seg_end, hint, t_old, t_lo, t_hi, list_count, lo, hi, s_bins, &s_rare);
+        }
         // this segment's exact partial sum into the matrix's accumulators
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -1368,7 +1551,7 @@ __global__ void __launch_bounds__(256, 4) k_pack_update_batch(const __grid_const
             s_ticket = atomicAdd(reinterpret_cast<unsigned *>(hdr + kPackWsCounterOffset), done) + done;
         }
         __syncthreads();
-        if (s_ticket == I.nchunks) {
+        if (s_ticket == I.nchunks && !known) {
             // every chunk of this matrix is summed: form gamma, threshold and mode
             __threadfence();
             if (threadIdx.x == 0) s_nnz = 0;
@@ -1511,6 +1694,7 @@ cudaError_t launch_pack_update_batch(const PackBatchItemHost *items, int n_items
             const int64_t n_el = h.n_out * h.k;
             I.p.W = reinterpret_cast<const float4 *>(h.W);
             I.w_bf16 = h.w_bf16 ? 1u : 0u;
+            I.gamma_known = h.gamma_known ? 1u : 0u;
             I.p.n_groups = n_el / 4;
             I.p.gpr = h.k / 4;
             I.p.gpr_div = make_fastdiv(static_cast<uint32_t>(h.k / 4));

@@ -366,3 +366,56 @@ def test_rmsnorm_closed_forms_and_fp64():
     w = r.normal(size=3200).astype(np.float32)
     xw = oracle.rmsnorm(X, 1e-6, w)
     assert np.array_equal(xw, (oracle.rmsnorm(X, 1e-6) * w).astype(np.float32))
+
+
+def test_wgrad_brute_force_and_one_hot():
+    r = np.random.default_rng(7)
+    T, N, K = 5, 3, 4
+    dY = r.normal(size=(T, N)).astype(np.float32)
+    X = r.normal(size=(T, K)).astype(np.float32)
+    dW = oracle.wgrad(dY, X)
+    for n in range(N):                      # brute force, one product at a time
+        for k in range(K):
+            s = math.fsum(float(dY[t, n]) * float(X[t, k]) for t in range(T))
+            assert abs(dW[n, k] - s) <= 1e-12 * max(1.0, abs(s))
+    # a one-hot output gradient picks one input row into one gradient row
+    e = np.zeros((T, N), np.float32)
+    e[2, 1] = 1.0
+    dW1 = oracle.wgrad(e, X)
+    assert np.array_equal(dW1[1], X[2].astype(np.float64)) and not dW1[[0, 2]].any()
+
+
+def test_adamw_closed_forms():
+    f = np.float32
+    r = np.random.default_rng(3)
+    W = r.normal(size=4096).astype(f)
+    G = (r.normal(size=4096) * 2.0 ** r.integers(-10, 4, size=4096)).astype(f)
+    z = np.zeros_like(W)
+    b1, b2 = 0.9, 0.95
+    # first step from zero moments: m / c1 = g and v / c2 = g^2 up to rounding, so the
+    # update is sign(g) (|g| >> eps): w' = w - lr sign(g)
+    W1, M1, V1 = oracle.adamw(W, G, z, z, 1e-3, b1, b2, 1e-12, 0.0, f(1 - b1), f(1 - b2))
+    assert np.all(np.abs((W1.astype(np.float64) - W) + 1e-3 * np.sign(G)) <= 1e-3 * 1e-5 + 4 * 2.0 ** -24 * np.abs(W))
+    # (1 - b1) is formed in fp32 from fp32(b1): a relative 2.4e-7 from 0.1, plus one rounding
+    assert np.allclose(M1, (1 - b1) * G.astype(np.float64), rtol=4e-7, atol=0)
+    assert np.allclose(V1, (1 - b2) * G.astype(np.float64) ** 2, rtol=8e-7, atol=0)
+    # no gradient and no moments: pure decoupled decay w' = w (1 - lr wd)
+    W2, M2, V2 = oracle.adamw(W, z, z, z, 1e-2, b1, b2, 1e-8, 0.1, f(0.5), f(0.5))
+    assert not M2.any() and not V2.any()
+    assert np.allclose(W2, W.astype(np.float64) * (1 - 1e-3), rtol=3e-7, atol=0)
+    # a constant gradient for t steps: the bias-corrected first moment is that gradient
+    g = f(0.25)
+    Wt, Mt, Vt = W[:8].copy(), np.zeros(8, f), np.zeros(8, f)
+    p1 = p2 = 1.0
+    for t in range(1, 6):
+        p1 *= b1
+        p2 *= b2
+        c1, c2 = f(1 - p1), f(1 - p2)
+        Wn, Mt, Vt = oracle.adamw(Wt, np.full(8, g, f), Mt, Vt, 1e-3, b1, b2, 1e-12, 0.0, c1, c2)
+        assert np.allclose(Mt / c1, g, rtol=1e-6) and np.allclose(np.sqrt(Vt / c2), g, rtol=1e-6)
+        assert np.allclose(Wt - Wn, 1e-3, rtol=1e-4)       # |update| = lr when m_hat = sqrt(v_hat)
+        Wt = Wn
+    # the update does not depend on the gradient's scale (eps negligible)
+    Wa, _, _ = oracle.adamw(W, G, z, z, 1e-3, b1, b2, 1e-30, 0.0, f(1 - b1), f(1 - b2))
+    Wb, _, _ = oracle.adamw(W, (G * f(8.0)).astype(f), z, z, 1e-3, b1, b2, 1e-30, 0.0, f(1 - b1), f(1 - b2))
+    assert np.allclose(Wa, Wb, rtol=0, atol=4 * 2.0 ** -24 * 4)
