@@ -624,15 +624,19 @@ def _time_graph(torch, g, flush, reps):
 
 
 def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
-    """One LLaMA-alike block at 3B shapes (hidden 3200, FFN 8640, 32 heads) over
-    T tokens, every BitLinear on the sparse ternary path: per-step pack of the
-    block's four matrices from fp32 masters; forward RMSNorm+quant -> QKV ->
+    """One training step of a LLaMA-alike block at 3B shapes (hidden 3200, FFN
+    8640, 32 heads) over T tokens, every BitLinear on the sparse ternary path:
+    pack of the block's four matrices from fp32 masters (gamma known from the
+    previous optimiser step: one read of W); forward RMSNorm+quant -> QKV ->
     causal attention -> quant -> O -> residual -> RMSNorm+quant -> gate|up ->
-    SwiGLU+quant -> down -> residual; STE dgrad of the four matrices.
-    Attention (torch SDPA) and the residual adds are library calls, timed and
-    listed apart.  Each stage is one CUDA graph timed alone after an L2 flush;
-    the whole step is one graph.  Context: the same block with dense bf16
-    weights through cuBLAS (torch.matmul) and torch elementwise ops."""
+    SwiGLU+quant -> down -> residual; backward: STE dgrad and the dense weight
+    gradient of the four matrices; AdamW on the masters, which also forms the
+    next gamma.  dY and the weight-gradient inputs are synthetic bf16 tensors of
+    the layer shapes.  Attention (torch SDPA) and the residual adds are library
+    calls, timed and listed apart.  Each stage is one CUDA graph timed alone
+    after an L2 flush; the whole step is one graph.  Context: the same step
+    with dense bf16 weights through cuBLAS (torch.matmul), torch elementwise ops
+    and torch's fused AdamW, without any pack."""
     F = torch.nn.functional
     dev = torch.device("cuda", torch.cuda.current_device())
     h, f, H = synth.LLAMA_3B["hidden"], synth.LLAMA_3B["ffn"], synth.LLAMA_3B["heads"]
@@ -645,7 +649,11 @@ def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
         masters[name] = synth.torch_master_weights(N, K, 0.02, seed=300 + i, device=dev)
         pw[name] = bn.PackedWeights(N, K, dev, group_bytes=True, mma=True, dec=False)
         bn.bitnet_pack_nm(masters[name], pw[name], 1e-5)   # first pack sets each gamma hint
-    batch = bn.PackBatch([(masters[n], pw[n]) for n, _, _ in mats], 1e-5, dev)
+    moments = {n: (torch.zeros_like(masters[n]), torch.zeros_like(masters[n])) for n, _, _ in mats}
+    ws_opt = bn.Workspace(lib.bitnet_adamw_workspace_size(), dev)
+    ws_wg = bn.Workspace(lib.bitnet_wgrad_workspace_size(), dev)
+    # the optimiser leaves the exact gamma of the updated masters in pw.gamma: the pack reads W once
+    batch = bn.PackBatch([(masters[n], pw[n]) for n, _, _ in mats], 1e-5, dev, gamma_known=True)
     ws_lin = bn.Workspace(lib.bitnet_linear_workspace_size(), dev)
     ws_dg = bn.Workspace(max(lib.bitnet_dgrad_workspace_size(N, K) for _, N, K in mats), dev)
     norm_w = (1.0 + 0.05 * torch.randn(h, device=dev)).float()
@@ -663,6 +671,9 @@ def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
     }
     dY = {n: synth.torch_activations(T, N, seed=320 + i, dtype=bf, device=dev) for i, (n, N, K) in enumerate(mats)}
     dX = {n: torch.empty((T, K), dtype=bf, device=dev) for n, N, K in mats}
+    Xin = {n: synth.torch_activations(T, K, seed=330 + i, dtype=bf, device=dev) for i, (n, N, K) in enumerate(mats)}
+    dWs = {n: torch.empty((N, K), dtype=torch.float32, device=dev) for n, N, K in mats}
+    step_no = [1]
     b = buf
 
     def s_pack():
@@ -705,11 +716,23 @@ def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
         for n, _, _ in mats:
             bn.bitnet_dgrad(dY[n], pw[n], dX=dX[n], ws=ws_dg)
 
+    def s_wgrad():
+        for n, _, _ in mats:
+            bn.bitnet_wgrad(dY[n], Xin[n], dW=dWs[n], ws=ws_wg)
+
+    def s_adamw():
+        for n, _, _ in mats:
+            bn.bitnet_adamw_step(masters[n], dWs[n], moments[n][0], moments[n][1], step_no[0], lr=1e-4,
+                                 weight_decay=0.1, gamma_out=pw[n].gamma, ws=ws_opt)
+
+    s_wgrad()
+    s_adamw()   # the first optimiser step sets every gamma the pack then takes as known
+
     stages = [("pack", s_pack, "ours"), ("rmsnorm_quant_1", s_norm1, "ours"), ("qkv", s_qkv, "ours"),
               ("attention", s_attn, "library"), ("quant_o", s_o, "ours"), ("residual_1", s_res1, "library"),
               ("rmsnorm_quant_2", s_norm2, "ours"), ("gate_up", s_gate_up, "ours"),
               ("swiglu_quant", s_swiglu, "ours"), ("down", s_down, "ours"), ("residual_2", s_res2, "library"),
-              ("dgrad_4", s_dgrad, "ours")]
+              ("dgrad_4", s_dgrad, "ours"), ("wgrad_4", s_wgrad, "ours"), ("adamw_4", s_adamw, "ours")]
     out = {"T": T, "hidden": h, "ffn": f, "heads": H, "stages_ms": {}}
     for name, fn, who in stages:
         g = _graph(torch, fn)
@@ -727,19 +750,29 @@ def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
     ours_ms = sum(v["ms"] for v in st.values() if v["impl"] == "ours")
     fwd_ops = 2.0 * T * sum(N * K for _, N, K in mats)
     gemm_ms = sum(st[n]["ms"] for n in ("qkv", "gate_up", "down"))
+    n_w = sum(N * K for _, N, K in mats)
     out.update({
         "step_ms": round(step_ms, 4),
         "ours_ms": round(ours_ms, 4),
         "library_ms": round(sum(v["ms"] for v in st.values() if v["impl"] == "library"), 4),
         "forward_gemm_ops": fwd_ops,
         "dgrad_tflops": round(fwd_ops / st["dgrad_4"]["ms"] / 1e9, 1),
+        "wgrad_tflops": round(fwd_ops / st["wgrad_4"]["ms"] / 1e9, 1),
+        "adamw_gbs": round(n_w * 28 / st["adamw_4"]["ms"] / 1e6, 1),   # W, g, m, v read; W, m, v written
+        "pack_gbs": round(n_w * 4.875 / st["pack"]["ms"] / 1e6, 1),
         "qkv_gate_up_down_tops": round(2.0 * T * sum(N * K for n, N, K in mats if n != "o") / gemm_ms / 1e9, 1),
     })
 
-    # context: the same block with dense bf16 weights (cuBLAS through torch.matmul) and torch ops
+    # context: the same step with dense bf16 weights (cuBLAS through torch.matmul), torch ops and
+    # torch's fused AdamW on fp32 masters
     Wd = {n: masters[n].to(bf) for n, _, _ in mats}
-    del masters, batch
+    del batch
     tb = {"x1": torch.empty((T, h), dtype=bf, device=dev)}
+    params = [masters[n] for n, _, _ in mats]
+    for pm, (n, _, _) in zip(params, mats):
+        pm.grad = dWs[n]
+    opt = torch.optim.AdamW(params, lr=1e-4, weight_decay=0.1, fused=True, capturable=True)
+    opt.step()   # state allocated outside the graph
 
     def rms(v):
         vf = v.float()
@@ -755,12 +788,15 @@ def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
         tb["x1"] = x1 + torch.matmul(hh, Wd["down"].t())
         for n, _, _ in mats:
             torch.matmul(dY[n], Wd[n])
+            torch.matmul(dY[n].t(), Xin[n])
+        opt.step()
 
     g = _graph(torch, t_step)
     out["torch_bf16_dense_step_ms"] = round(_time_graph(torch, g, flush, reps), 4)
-    del g, Wd
-    out["note"] = ("step = per-step pack + forward + STE dgrad of one block; the bf16 context runs the same "
-                   "block without the pack, on dense bf16 weights already in memory")
+    del g, Wd, opt, masters
+    out["note"] = ("step = pack (known gamma) + forward + STE dgrad + weight gradient + AdamW of one block; the "
+                   "bf16 context runs the same step without the pack, on dense bf16 weights already in memory, "
+                   "with torch's fused AdamW")
     torch.cuda.empty_cache()
     return out
 # ------------------------------------------------------------------ CPU oracle baseline

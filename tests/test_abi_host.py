@@ -133,6 +133,33 @@ def test_block_quant_rejects_bad_arguments(lib):
     assert g(None, None, 512, 0, 256, 1e-5, None, None, None) == ok                         # empty batch
 
 
+def test_train_step_entries_reject_bad_arguments(lib):
+    bad = _abi.BITNET_ERR_INVALID_ARG
+    ws = _fake()
+    f = lib.bitnet_wgrad
+    assert f(_fake(), _fake(), 64, 250, 256, _fake(), 0, ws, 1 << 20, None) == bad        # n_out % 8
+    assert f(_fake(), _fake(), 64, 256, 252, _fake(), 0, ws, 1 << 20, None) == bad        # k % 8
+    assert f(_fake(), _fake(), -1, 256, 256, _fake(), 0, ws, 1 << 20, None) == bad        # T < 0
+    assert f(_fake(), _fake(), 64, 256, 256, None, 0, ws, 1 << 20, None) == bad           # null dW
+    assert f(None, _fake(), 64, 256, 256, _fake(), 0, ws, 1 << 20, None) == bad           # null dY
+    assert f(_fake(4104), _fake(), 64, 256, 256, _fake(), 0, ws, 1 << 20, None) == bad    # dY alignment
+    assert f(_fake(), _fake(), 64, 256, 256, _fake(), 0, None, 0, None) == _abi.BITNET_ERR_WORKSPACE
+    assert f(None, None, 0, 256, 256, _fake(), 1, ws, 1 << 20, None) == _abi.BITNET_OK    # empty, accumulate
+    g = lib.bitnet_adamw_step
+    h = _abi.BitnetAdamWHparams(1e-3, 0.9, 0.95, 1e-8, 0.1, 0.1, 0.05)
+    ok_args = (_fake(), _fake(), _fake(), _fake(), 1024, ctypes.byref(h), 1e-5, _fake(), ws, 1 << 20, None)
+    assert g(_fake(), _fake(), _fake(), _fake(), 1022, ctypes.byref(h), 1e-5, _fake(), ws, 1 << 20, None) == bad
+    assert g(None, *ok_args[1:]) == bad
+    assert g(*ok_args[:7], None, *ok_args[8:]) == bad                                       # null gamma_out
+    assert g(_fake(4104), *ok_args[1:]) == bad                                              # W alignment
+    assert g(*ok_args[:8], None, 0, None) == _abi.BITNET_ERR_WORKSPACE
+    for field, value in (("beta1", 1.0), ("beta2", -0.1), ("eps", 0.0), ("bias_correction1", 0.0), ("lr", -1.0)):
+        hb = _abi.BitnetAdamWHparams(1e-3, 0.9, 0.95, 1e-8, 0.1, 0.1, 0.05)
+        setattr(hb, field, value)
+        assert g(*ok_args[:5], ctypes.byref(hb), *ok_args[6:]) == bad, field
+    assert g(*ok_args[:5], None, *ok_args[6:]) == bad                                      # null hyper-parameters
+
+
 def test_linear_rejects_bad_arguments(lib):
     f = lib.bitnet_sparse_linear
     ws = lib.bitnet_linear_workspace_size()
