@@ -803,7 +803,7 @@ __device__ __forceinline__ float adamw1(float w, float g, float &m, float &v, co
     return __fsub_rn(w, __fmul_rn(a.lr, __fadd_rn(u, __fmul_rn(a.wd, w))));
 }
 
-__global__ void __launch_bounds__(256, 4) k_adamw_gamma(const __grid_constant__ AdamWArgs a) {
+__global__ void __launch_bounds__(256, 6) k_adamw_gamma(const __grid_constant__ AdamWArgs a) {
     __shared__ unsigned long long s_bins[256];
     __shared__ unsigned long long s_lo[8], s_hi[8];
     __shared__ int s_rare;
@@ -815,7 +815,8 @@ __global__ void __launch_bounds__(256, 4) k_adamw_gamma(const __grid_constant__ 
     double d = 0.0;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    constexpr int kU = 4;   // float4 groups per thread per round (16 loads in flight)
+    constexpr int kU = 1;   // one float4 group per thread per round, latency hidden by 48 warps per SM (3B block:
+                            // 0.65 ms; four groups per thread at 32 warps: 0.77 ms; 64 warps spill registers)
     for (; i < a.n4; i += kU * stride) {
         float4 w[kU], g[kU], m[kU], v[kU];
 #pragma unroll
@@ -1275,7 +1276,7 @@ cudaError_t launch_adamw_gamma(float *W, const float *G, float *M, float *V, int
     a.eps_gamma = eps_gamma;
     a.gamma = gamma;
     a.thr = reinterpret_cast<uint32_t *>(w8 + kPackWsThrOffset);
-    k_adamw_gamma<<<grid_for((a.n4 + 3) / 4, 256, 4), 256, 0, s>>>(a);
+    k_adamw_gamma<<<grid_for(a.n4, 256, 6), 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
