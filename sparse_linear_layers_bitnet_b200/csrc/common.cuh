@@ -201,4 +201,16 @@ __device__ __forceinline__ uint32_t elect_one() {
     return pred;
 }
 
+// bf16 bits of a 2-bit ternary code {0: 0, 1: +1 = 0x3f80, 3: -1 = 0xbf80}
+__device__ __forceinline__ uint32_t code_bf16(uint32_t code) { return (code & 1u) * 0x3f80u | ((code & 2u) << 14); }
+
+// the bf16 values of positions 0..3 of a canonical group byte
+// (idx0 | idx1 << 2 | c0 << 4 | c1 << 6), position p in bits 16p..16p+15
+__device__ __forceinline__ uint2 group_bf16x4(uint32_t b) {
+    const uint32_t i0 = b & 3u, i1 = (b >> 2) & 3u;
+    const uint32_t c4 = (((b >> 4) & 3u) << (2 * i0)) | ((b >> 6) << (2 * i1));
+    return make_uint2(code_bf16(c4 & 3u) | (code_bf16((c4 >> 2) & 3u) << 16),
+                      code_bf16((c4 >> 4) & 3u) | (code_bf16(c4 >> 6) << 16));
+}
+
 }  // namespace bitnet

@@ -292,8 +292,12 @@ def test_linear_empty_batch(bn):
 
 # ------------------------------------------------------------------ STE input gradient
 
+# T > 128 forms the ternary tiles in shared memory from the group bytes: ragged
+# n_out (contraction tail), k not a multiple of 64 (column tail, unaligned
+# group-byte rows) and ragged T included
 @pytest.mark.parametrize("T,n_out,k,dx", [(128, 256, 256, "f32"), (200, 264, 384, "f32"), (300, 512, 1000, "bf16"),
-                                          (512, 3200, 640, "f32")])
+                                          (512, 3200, 640, "f32"), (129, 72, 136, "f32"), (700, 1000, 2600, "bf16"),
+                                          (2048, 9600, 3200, "bf16")])
 def test_dgrad_parity(bn, T, n_out, k, dx):
     W = synth.master_weights(n_out, k, 0.02, seed=T + k)
     g, keep, wq, gb = oracle.pack_weights(W, 1e-5)
