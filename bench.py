@@ -597,7 +597,7 @@ def measure_dgrad(torch, bn, synth, peaks, reps=5):
     tf = tot_f / tot_ms / 1e9
     out["combined"] = {"tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / peaks["bf16"], 4),
                        "cublas_same_shapes_tflops": round(tot_f / tot_ms_c / 1e9, 1),
-                       "note": "includes the bf16 expansion of Wq^T from group bytes; cuBLAS is given the dense "
+                       "note": "includes the bf16 expansion of Wq from group bytes; cuBLAS is given the dense "
                                "bf16 operand ready in memory"}
     torch.cuda.empty_cache()
     return out

@@ -12,8 +12,9 @@
 //
 // STE gradient ("Sparse-BitNet", section 2 "Training Strategie"):
 //     dX[t, k] = gamma * sum_n dY[t, n] Wq[n, k]      (bf16 in, fp32 in TMEM)
-// with A = dY (M = tokens), B = Wq^T expanded to bf16 (N = input features),
-// K = output features.
+// with A = dY (M = tokens), B = Wq expanded to bf16 (N = input features),
+// K = output features: here (T <= 128) as Wq^T, K-major; the CTA-pair kernel
+// (gemm2.cu, T > 128) reads untransposed bf16 rows of Wq as an MN-major operand.
 //
 // One CTA computes a 128 x BN output tile:
 //   warp 0      TMA producer: A and B tiles (and the 2 KB metadata block) per
@@ -426,18 +427,55 @@ __global__ void __launch_bounds__(256) k_expand_wt(const uint8_t *__restrict__ g
     }
 }
 
+// Wq as bf16 rows [n_out][k]: group byte i holds the weights 4i .. 4i + 3 of the
+// row-major matrix, so the expansion is a linear map.  Lane-consecutive
+// 16-byte output chunks (two group bytes each): loads and stores coalesced.
+__global__ void __launch_bounds__(256) k_expand_w(const uint8_t *__restrict__ gb, int64_t nbytes,
+                                                  __nv_bfloat16 *__restrict__ w) {
+    __shared__ uint2 s_lut[256];
+    s_lut[threadIdx.x] = group_bf16x4(threadIdx.x);
+    __syncthreads();
+    const int64_t nchunk = nbytes / 2;   // nbytes is even (k % 8 == 0)
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const uint16_t *src = reinterpret_cast<const uint16_t *>(gb);
+    uint4 *dst = reinterpret_cast<uint4 *>(w);
+    int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (; j + 3 * stride < nchunk; j += 4 * stride) {
+        uint32_t b[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) b[u] = __ldg(src + j + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const uint2 lo = s_lut[b[u] & 0xffu], hi = s_lut[b[u] >> 8];
+            dst[j + u * stride] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        }
+    }
+    for (; j < nchunk; j += stride) {
+        const uint32_t b = __ldg(src + j);
+        const uint2 lo = s_lut[b & 0xffu], hi = s_lut[b >> 8];
+        dst[j] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+    }
+}
+
 cudaError_t launch_dgrad(const void *dY, const float *gamma, const uint8_t *gb, int64_t T, int64_t n_out, int64_t k,
                          void *dX, bool dx_bf16, void *ws, cudaStream_t s) {
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     __nv_bfloat16 *wt = reinterpret_cast<__nv_bfloat16 *>(w8 + kDgradWsHeader);
+    if (T > 128) {   // CTA-pair persistent kernel (gemm2.cu) on Wq's untransposed bf16 rows
+        const int64_t nchunk = n_out * k / 8;
+        const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+        const int64_t blocks = (nchunk + 1023) / 1024;
+        k_expand_w<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(gb, n_out * k / 4, wt);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        return launch_gemm_bf16_pair(dY, wt, gamma, T, n_out, k, dX, dx_bf16,
+                                     reinterpret_cast<uint32_t *>(w8 + kStatusOffset), s);
+    }
     const int64_t tiles = ((k + 63) / 64) * ((n_out + 63) / 64);
     const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
     k_expand_wt<<<static_cast<unsigned>(tiles < cap ? tiles : cap), 256, 0, s>>>(gb, n_out, k, wt);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    if (T > 128)   // CTA-pair persistent kernel (gemm2.cu)
-        return launch_gemm_bf16_pair(dY, wt, gamma, T, n_out, k, dX, dx_bf16,
-                                     reinterpret_cast<uint32_t *>(w8 + kStatusOffset), s);
     GemmParams p{};
     p.M = T;
     p.N = k;

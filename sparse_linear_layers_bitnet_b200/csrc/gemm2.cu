@@ -120,11 +120,12 @@ __device__ __forceinline__ void commit_both(uint64_t *bar) {
 
 }  // namespace pair
 
-// MN: dense operands stored with the M (A) and N (B) dimension contiguous
-// ("MN-major"): tiles arrive as 64-element-wide boxes of 64 k-rows, 128-byte
-// swizzled; the descriptors step 8 KB between 64-wide boxes (leading byte
-// offset) and 1 KB between groups of 8 k-rows (stride byte offset).
-template <bool SPARSE, int BN, int STAGES, bool MN = false>
+// MN (dense only), a mask: 1 = A, 2 = B stored with its M (A) or N (B)
+// dimension contiguous ("MN-major"): its tiles arrive as 64-element-wide boxes
+// of 64 k-rows, 128-byte swizzled; the descriptors step 8 KB between 64-wide
+// boxes (leading byte offset) and 1 KB between groups of 8 k-rows (stride byte
+// offset).  The other operand stays K-major.
+template <bool SPARSE, int BN, int STAGES, int MN = 0>
 struct PairCfg {
     static constexpr int kHalfN = BN / 2;                  // B rows per CTA
     static constexpr int kARowBytes = SPARSE ? 64 : 128;
@@ -144,14 +145,14 @@ struct PairCfg {
     static constexpr int kSmemBytes = STAGES * kStageBytes + kStageOutBytes + 1024 + 2048;
     // M = 256 (two CTAs), N = BN
     static constexpr uint32_t kIdesc = (SPARSE ? (1u << 2) : 0u) | ((SPARSE ? 2u : 1u) << 4) | (1u << 7) |
-                                       (1u << 10) | (MN ? (1u << 15) | (1u << 16) : 0u) |
+                                       (1u << 10) | ((MN & 1) ? (1u << 15) : 0u) | ((MN & 2) ? (1u << 16) : 0u) |
                                        (static_cast<uint32_t>(BN >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
     static constexpr int kMnBox = 64 * 64 * 2;             // one 64 (MN) x 64 (k) bf16 box
     static constexpr int kMnAdvance = 2 * 1024;            // 16 k-rows per MMA
     static_assert(!SPARSE || (BN % 32 == 0 && BN <= 224), "sparse pair tiles: N multiple of 32, two buffers + metadata");
     static_assert(SPARSE || (BN % 32 == 0 && BN <= 256), "dense pair tiles: N multiple of 32");
     static_assert(kBBytes % 1024 == 0, "B tile must keep the 128-byte swizzle atoms aligned");
-    static_assert(!MN || (!SPARSE && kHalfN % 64 == 0), "MN-major tiles: dense, whole 64-wide boxes");
+    static_assert(!MN || (!SPARSE && (!(MN & 2) || kHalfN % 64 == 0)), "MN-major tiles: dense, whole 64-wide boxes");
 };
 
 struct PairParams {
@@ -167,7 +168,7 @@ struct PairParams {
     int accumulate;              // dense fp32 output: out += result (else out = result)
 };
 
-template <bool SPARSE, int BN, int STAGES, bool MN = false>
+template <bool SPARSE, int BN, int STAGES, int MN = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     k_umma_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY, PairParams p) {
@@ -243,15 +244,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                         pair::tma_load_2d_pair(&tmE, &full[s], sE + s * C::kEBytes, 0,
                                                static_cast<int32_t>((kt * p.meta_rows + e_row) / 8));
                     } else if (MN) {
-                        // boxes of 64 MN-elements x 64 k-rows: two for A's 128 rows, kHalfN / 64 for B
+                        // MN-major: boxes of 64 MN-elements x 64 k-rows (two for A's 128 rows, kHalfN / 64
+                        // for B); K-major: one box of 64 k x all rows
+                        if (MN & 1) {
 #pragma unroll
-                        for (int h = 0; h < 2; ++h)
-                            pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes + h * C::kMnBox, a_row + 64 * h,
-                                                   kt * C::kKStep);
+                            for (int h = 0; h < 2; ++h)
+                                pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes + h * C::kMnBox,
+                                                       a_row + 64 * h, kt * C::kKStep);
+                        } else {
+                            pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * C::kKStep, a_row);
+                        }
+                        if (MN & 2) {
 #pragma unroll
-                        for (int h = 0; h < C::kHalfN / 64; ++h)
-                            pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes + h * C::kMnBox, b_row + 64 * h,
-                                                   kt * C::kKStep);
+                            for (int h = 0; h < C::kHalfN / 64; ++h)
+                                pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes + h * C::kMnBox,
+                                                       b_row + 64 * h, kt * C::kKStep);
+                        } else {
+                            pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
+                        }
                     } else {
                         pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * C::kKStep, a_row);
                         pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
@@ -288,8 +298,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     } else if (MN) {
 #pragma unroll
                         for (int j = 0; j < C::kMmaPerStage; ++j) {
-                            const uint64_t ad = make_smem_desc(a_base + j * C::kMnAdvance, C::kMnBox, 1024, kSwizzle128B);
-                            const uint64_t bd = make_smem_desc(b_base + j * C::kMnAdvance, C::kMnBox, 1024, kSwizzle128B);
+                            const uint64_t ad = (MN & 1) ? make_smem_desc(a_base + j * C::kMnAdvance, C::kMnBox, 1024, kSwizzle128B)
+                                                         : make_smem_desc(a_base + j * C::kAAdvance, 16, 1024, kSwizzle128B);
+                            const uint64_t bd = (MN & 2) ? make_smem_desc(b_base + j * C::kMnAdvance, C::kMnBox, 1024, kSwizzle128B)
+                                                         : make_smem_desc(b_base + j * C::kBAdvance, 16, 1024, kSwizzle128B);
                             pair::mma_bf16_pair(d_tmem, ad, bd, C::kIdesc, (kt | j) != 0);
                         }
                     } else {
@@ -482,7 +494,7 @@ static bool map2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, ui
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool SPARSE, int BN, int STAGES, bool MN = false>
+template <bool SPARSE, int BN, int STAGES, int MN = 0>
 static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &e, const CUtensorMap &y,
                             const PairParams &p, cudaStream_t s) {
     using C = PairCfg<SPARSE, BN, STAGES, MN>;
@@ -542,7 +554,9 @@ cudaError_t launch_gemm_sp_pair(const int8_t *Xq, const float *amax, const float
     return run_pair<true, BN, 8>(ma, mb, me, my, p, s);
 }
 
-cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *wt, const float *gamma, int64_t T,
+// dX = gamma dY . Wq with Wq as bf16 rows [n_out][k] (expanded from the group
+// bytes without a transpose): B (N = k, K = n_out) is MN-major.
+cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *w, const float *gamma, int64_t T,
                                   int64_t n_out, int64_t k, void *dX, bool dx_bf16, uint32_t *status, cudaStream_t s) {
     constexpr int BN = 256;
     PairParams p{};
@@ -557,10 +571,10 @@ cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *wt, const
     if (!map2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dY, static_cast<uint64_t>(n_out), static_cast<uint64_t>(T),
                static_cast<uint64_t>(n_out) * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    if (!map2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wt, static_cast<uint64_t>(n_out), static_cast<uint64_t>(k),
-               static_cast<uint64_t>(n_out) * 2, 64, static_cast<uint32_t>(BN / 2), CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!map2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w, static_cast<uint64_t>(k), static_cast<uint64_t>(n_out),
+               static_cast<uint64_t>(k) * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    return run_pair<false, BN, 6>(ma, mb, ma, ma, p, s);
+    return run_pair<false, BN, 6, 2>(ma, mb, ma, ma, p, s);
 }
 
 // Weight gradient dW[n, k] (+)= sum_t dY[t, n] X[t, k]: A = dY and B = X both
@@ -584,7 +598,7 @@ cudaError_t launch_gemm_wgrad_pair(const void *dY, const void *X, int64_t T, int
     if (!map2d(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(k), static_cast<uint64_t>(T),
                static_cast<uint64_t>(k) * 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    return run_pair<false, BN, 6, true>(ma, mb, ma, ma, p, s);
+    return run_pair<false, BN, 6, 3>(ma, mb, ma, ma, p, s);
 }
 
 }  // namespace bitnet

@@ -128,7 +128,7 @@ cudaError_t launch_gemm_sp_pair(const int8_t *Xq, const float *amax, const float
                                 const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16,
                                 int32_t *acc, uint32_t *status, cudaStream_t s);
 
-cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *wt, const float *gamma, int64_t T,
+cudaError_t launch_gemm_bf16_pair(const void *dY, const __nv_bfloat16 *w, const float *gamma, int64_t T,
                                   int64_t n_out, int64_t k, void *dX, bool dx_bf16, uint32_t *status, cudaStream_t s);
 
 cudaError_t launch_dgrad(const void *dY, const float *gamma, const uint8_t *gb, int64_t T, int64_t n_out,
