@@ -493,6 +493,23 @@ bitnet_status bitnet_pack_nm_noalloc(const float *W, bitnet_packed_w *out, float
                                      uint8_t *mask_bits, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_wait_selftest - exercises the error path of the bounded waits.
+ *
+ * Every wait of the kernels (mbarrier phases of the GEMM and pack pipelines,
+ * the decode chain's grid counters) gives up after a time limit, sets the
+ * timeout bit of the workspace status word and lets the kernel end, so the
+ * CUDA context stays usable.  This call runs one wait of each kind on an
+ * event that never happens, with the limit limit_us (1 .. 2e6 microseconds),
+ * on the given stream; afterwards bitnet_read_device_status(ws) returns
+ * BITNET_ERR_TIMEOUT.  It faults nothing and hangs nothing: it is the health
+ * check of the timeout path.
+ *   ws   >= bitnet_decode_chain_workspace_size(1) bytes, 16-byte aligned
+ *        (cleared by the call).
+ * Errors: INVALID_ARG, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_wait_selftest(void *ws, size_t ws_bytes, int32_t limit_us, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Status helpers.
  * bitnet_read_device_status synchronises `stream`, reads the status word that
  * the kernels of the last call on `ws` left (BITNET_OK or BITNET_ERR_TIMEOUT

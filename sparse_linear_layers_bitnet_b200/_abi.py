@@ -35,7 +35,7 @@ EXPORTED = [
     "bitnet_decode_chain_workspace_size", "bitnet_decode_chain",
     "bitnet_dgrad_workspace_size", "bitnet_dgrad",
     "bitnet_wgrad_workspace_size", "bitnet_wgrad", "bitnet_adamw_workspace_size", "bitnet_adamw_step",
-    "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
+    "bitnet_wait_selftest", "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
 ]
 
 
@@ -126,6 +126,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_wgrad": (I32, [P, P, I64, I64, I64, P, I32, P, SZ, P]),
         "bitnet_adamw_workspace_size": (SZ, []),
         "bitnet_adamw_step": (I32, [P, P, P, P, I64, ctypes.POINTER(BitnetAdamWHparams), F, P, P, SZ, P]),
+        "bitnet_wait_selftest": (I32, [P, SZ, I32, P]),
         "bitnet_read_device_status": (I32, [P, P]),
         "bitnet_status_string": (ctypes.c_char_p, [I32]),
         "bitnet_last_error": (ctypes.c_char_p, []),
@@ -505,6 +506,15 @@ def bitnet_dgrad(dY, W: PackedWeights, dX=None, dx_dtype=None, ws: Workspace | N
     check(lib.bitnet_dgrad(_ptr(dY), _dtype_code(dY.dtype), ctypes.byref(st), T, _ptr(dX), _dtype_code(dX.dtype),
                            ws.ptr, ws.nbytes, _stream(stream)), "bitnet_dgrad")
     return dX
+
+
+def bitnet_wait_selftest(limit_us: int = 50000, device="cuda", stream=None) -> int:
+    """Runs both kinds of bounded wait on events that never happen (limit limit_us)
+    and returns the device status code that follows (BITNET_ERR_TIMEOUT expected)."""
+    lib = load()
+    ws = Workspace(lib.bitnet_decode_chain_workspace_size(1), device)
+    check(lib.bitnet_wait_selftest(ws.ptr, ws.nbytes, int(limit_us), _stream(stream)), "bitnet_wait_selftest")
+    return lib.bitnet_read_device_status(ws.ptr, _stream(stream))
 
 
 def bitnet_read_device_status(ws: Workspace, stream=None) -> int:

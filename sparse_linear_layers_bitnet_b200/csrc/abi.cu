@@ -473,6 +473,17 @@ bitnet_status bitnet_dgrad(const void *dY, bitnet_dtype dy_dtype, const bitnet_p
                        "dgrad");
 }
 
+bitnet_status bitnet_wait_selftest(void *ws, size_t ws_bytes, int32_t limit_us, bitnet_stream_t stream) {
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "wait_selftest: workspace is required");
+    if (ws_bytes < bitnet_decode_chain_workspace_size(1))
+        return fail(BITNET_ERR_WORKSPACE, "wait_selftest: workspace needs %zu bytes", bitnet_decode_chain_workspace_size(1));
+    if (!aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "wait_selftest: ws must be 16-byte aligned");
+    if (limit_us <= 0 || limit_us > 2000000) return fail(BITNET_ERR_INVALID_ARG, "wait_selftest: limit_us must be in [1, 2e6]");
+    return cuda_status(bitnet::launch_wait_selftest(ws, static_cast<uint64_t>(limit_us) * 1000ull,
+                                                    reinterpret_cast<cudaStream_t>(stream)),
+                       "wait_selftest");
+}
+
 bitnet_status bitnet_read_device_status(void *ws, bitnet_stream_t stream) {
     if (!ws) return fail(BITNET_ERR_INVALID_ARG, "read_device_status: null workspace");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

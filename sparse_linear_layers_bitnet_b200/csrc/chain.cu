@@ -74,9 +74,11 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
     return v;
 }
 
-// Spins (bounded) until *ctr >= target.  On a timeout or a grid abort it sets
-// the CTA's abort flag (and, on a timeout, the grid abort word and status).
-__device__ bool wait_counter(const uint32_t *ctr, uint32_t target, const ChainParams &p, volatile int *s_abort) {
+// Spins (bounded by limit_ns) until *ctr >= target.  On a timeout or a grid
+// abort it sets the CTA's abort flag (and, on a timeout, the grid abort word
+// and status).
+__device__ bool wait_counter(const uint32_t *ctr, uint32_t target, const ChainParams &p, volatile int *s_abort,
+                             uint64_t limit_ns = kWaitLimitNs) {
     if (ld_acquire(ctr) >= target) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
@@ -86,7 +88,7 @@ __device__ bool wait_counter(const uint32_t *ctr, uint32_t target, const ChainPa
             *s_abort = 1;
             return false;
         }
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if (globaltimer_ns() - t0 > limit_ns) {
             *s_abort = 1;
             atomicOr(p.status, kStatusTimeout);
             atomicExch(p.abort, 1u);
@@ -635,6 +637,44 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+// ---------------------------------------------------------------- health check of the bounded waits
+//
+// Runs the two kinds of bounded wait the kernels use on events that never
+// happen, with a short limit: warp 0 waits on an mbarrier nobody arrives at
+// (mbar_wait_bounded, the wait of the GEMM and pack pipelines), warp 1 on a
+// grid counter nobody increments (wait_counter, the decode chain's wait).
+// Both give up after limit_ns, set the timeout bit of the status word and
+// return; the kernel ends normally and the context stays usable.
+__global__ void k_wait_selftest(uint32_t *status, uint32_t *abort_word, const uint32_t *counter, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int s_abort_mbar, s_abort_ctr;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        s_abort_mbar = 0;
+        s_abort_ctr = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &s_abort_mbar, status, limit_ns);
+    if (threadIdx.x == 32) {
+        ChainParams p;
+        p.status = status;
+        p.abort = abort_word;
+        p.counters = nullptr;
+        wait_counter(counter, 1u, p, &s_abort_ctr, limit_ns);
+    }
+}
+
+cudaError_t launch_wait_selftest(void *ws, uint64_t limit_ns, cudaStream_t s) {
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    cudaError_t e = cudaMemsetAsync(ws, 0, kChainCountersOffset + 4, s);
+    if (e != cudaSuccess) return e;
+    k_wait_selftest<<<1, 64, 0, s>>>(reinterpret_cast<uint32_t *>(w8 + kStatusOffset),
+                                     reinterpret_cast<uint32_t *>(w8 + kChainAbortOffset),
+                                     reinterpret_cast<const uint32_t *>(w8 + kChainCountersOffset), limit_ns);
+    return cudaGetLastError();
 }
 
 }  // namespace bitnet

@@ -58,18 +58,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// kWaitLimitNs, or as soon as *abort becomes non-zero; on giving up it sets
-// *abort and ORs kStatusTimeout into the device status word.  Returns true
-// when the phase completed.
+// limit_ns (kWaitLimitNs unless a caller asks for less), or as soon as *abort
+// becomes non-zero; on giving up it sets *abort and ORs kStatusTimeout into
+// the device status word.  Returns true when the phase completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                                  uint32_t *status) {
+                                                  uint32_t *status, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0u) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 *abort = 1;
                 if (status) atomicOr(status, kStatusTimeout);
                 return false;

@@ -79,6 +79,9 @@ cudaError_t launch_adamw_gamma(float *W, const float *G, float *M, float *V, int
                                float eps, float wd, float c1, float c2, float eps_gamma, float *gamma, void *ws,
                                cudaStream_t s);
 
+// Health check of the bounded waits (chain.cu): both kinds of wait run out on events that never happen
+cudaError_t launch_wait_selftest(void *ws, uint64_t limit_ns, cudaStream_t s);
+
 // Weight gradient (gemm2.cu)
 cudaError_t launch_gemm_wgrad_pair(const void *dY, const void *X, int64_t T, int64_t n_out, int64_t k, float *dW,
                                    bool accumulate, uint32_t *status, cudaStream_t s);

@@ -160,6 +160,15 @@ def test_train_step_entries_reject_bad_arguments(lib):
     assert g(*ok_args[:5], None, *ok_args[6:]) == bad                                      # null hyper-parameters
 
 
+def test_wait_selftest_rejects_bad_arguments(lib):
+    n = lib.bitnet_decode_chain_workspace_size(1)
+    assert lib.bitnet_wait_selftest(None, n, 1000, None) == _abi.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_wait_selftest(_fake(), n - 1, 1000, None) == _abi.BITNET_ERR_WORKSPACE
+    assert lib.bitnet_wait_selftest(_fake(4104), n, 1000, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_wait_selftest(_fake(), n, 0, None) == _abi.BITNET_ERR_INVALID_ARG
+    assert lib.bitnet_wait_selftest(_fake(), n, 2000001, None) == _abi.BITNET_ERR_INVALID_ARG
+
+
 def test_linear_rejects_bad_arguments(lib):
     f = lib.bitnet_sparse_linear
     ws = lib.bitnet_linear_workspace_size()

@@ -314,6 +314,28 @@ def test_dgrad_parity(bn, T, n_out, k, dx):
     assert np.all(np.abs(got - ref) <= tol)
 
 
+def test_bounded_waits_time_out_cleanly(bn):
+    """Both kinds of bounded wait (mbarrier phase, grid counter) run out on
+    events that never happen: the status word reports the timeout, the kernel
+    ends, and the context keeps working (a pack and a quantisation afterwards
+    are exact, and their own status is clear)."""
+    import time
+    t0 = time.time()
+    assert bn.bitnet_wait_selftest(limit_us=50000) == 5          # BITNET_ERR_TIMEOUT
+    assert time.time() - t0 < 30.0
+    W = synth.master_weights(256, 256, 0.02, seed=3)
+    pw = bn.PackedWeights(256, 256)
+    ws = bn.Workspace(bn.load().bitnet_pack_workspace_size(256, 256))
+    bn.bitnet_pack_nm(dev_f32(W), pw, 1e-5, ws=ws)
+    X = synth.activations(4, 256, seed=4)
+    Xq, a = bn.bitnet_quant_act(dev_f32(X), 1e-5)
+    torch.cuda.synchronize()
+    g, keep, wq, gb = oracle.pack_weights(W, 1e-5)
+    assert pw.gamma.item() == float(g) and np.array_equal(pw.group_bytes.cpu().numpy(), gb)
+    assert np.array_equal(Xq.cpu().numpy(), oracle.quant_act(X, 1e-5)[0])
+    assert bn.bitnet_read_device_status(ws) == 0
+
+
 def test_device_status_clear_after_runs(bn):
     ws = bn.Workspace(256)
     ref, acc, Y = _linear_case(bn, 256, 256, 64, seed=5)
