@@ -182,6 +182,20 @@ class Timer:
         return self.e0.elapsed_time(self.e1)
 
 
+class Nvtx:
+    """NVTX range around a phase of the run, for timeline profilers (host-side marks only)."""
+
+    def __init__(self, torch, name):
+        self.torch, self.name = torch, name
+
+    def __enter__(self):
+        self.torch.cuda.nvtx.range_push(self.name)
+        return self
+
+    def __exit__(self, *a):
+        self.torch.cuda.nvtx.range_pop()
+
+
 def flush_l2(torch, buf):
     buf.add_(1)   # write 256 MB: evicts the 126 MB L2
 
@@ -915,7 +929,7 @@ def run_ours(args):
         g_step.replay()
     dist.barrier()
     torch.cuda.synchronize()
-    with Timer(torch) as tm:
+    with Nvtx(torch, "decode timed steps"), Timer(torch) as tm:
         for _ in range(args.steps):
             g_step.replay()
     torch.cuda.synchronize()
@@ -958,7 +972,7 @@ def run_ours(args):
         y_host.copy_(dec.y_flat, non_blocking=True)
     torch.cuda.synchronize()
     dist.barrier()
-    with Timer(torch) as te:
+    with Nvtx(torch, "decode e2e steps"), Timer(torch) as te:
         for _ in range(args.steps):
             dec.x_flat.copy_(x_host, non_blocking=True)
             g_step.replay()
@@ -985,16 +999,22 @@ def run_ours(args):
                 "launches_per_step": d2.launches_per_step}
             del g2, d2
             torch.cuda.empty_cache()
-        rows["library_peaks"] = measure_library_peaks(torch)
-        rows["prefill_gemm"] = measure_prefill(torch, bn, synth, peaks)
+        with Nvtx(torch, "row library_peaks"):
+            rows["library_peaks"] = measure_library_peaks(torch)
+        with Nvtx(torch, "row prefill_gemm"):
+            rows["prefill_gemm"] = measure_prefill(torch, bn, synth, peaks)
         lp = rows["library_peaks"]["int8_dense_tops"]
         pc = rows["prefill_gemm"]["combined"]
         pc["frac_of_2x_measured_int8_dense"] = round(pc["tops"] / (2 * lp), 4)
         pc["frac_of_measured_int8_dense"] = round(pc["tops"] / lp, 4)
-        rows["dgrad"] = measure_dgrad(torch, bn, synth, peaks)
-        rows["six_eight"] = measure_6of8(torch, bn, synth)
-        rows["block"] = measure_block(torch, bn, synth, peaks)
-        rows["pack"] = measure_pack(torch, bn, synth, peaks, flip_steps=args.flip_steps)
+        with Nvtx(torch, "row dgrad"):
+            rows["dgrad"] = measure_dgrad(torch, bn, synth, peaks)
+        with Nvtx(torch, "row six_eight"):
+            rows["six_eight"] = measure_6of8(torch, bn, synth)
+        with Nvtx(torch, "row block"):
+            rows["block"] = measure_block(torch, bn, synth, peaks)
+        with Nvtx(torch, "row pack"):
+            rows["pack"] = measure_pack(torch, bn, synth, peaks, flip_steps=args.flip_steps)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": info.world, "steps": args.steps,
