@@ -871,8 +871,11 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "i8", "data": "synthetic",
-        "config": {"workload": f"decode GEMV, 2B LLaMA-alike shapes, batch {T}", "tokens": T,
-                   "sample": "one layer per step (QKV, O, gate|up, down)"},
+        "config": {"workload": f"decode GEMV, 2B LLaMA-alike (hidden 2560, FFN 6912), {args.layers} layers, batch {T}",
+                   "tokens": T, "layers": args.layers,
+                   "step": "the CPU oracle (per projection: int8 act quant, int32 product, dequant) on the host "
+                           "cores; each timed step is a bounded sample of one layer (QKV, O, gate|up, down), "
+                           "GB/s counted on that layer's algorithmic bytes"},
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": f"one 2B layer per step, {args.steps} steps, T={T}"},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
