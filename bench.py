@@ -62,7 +62,7 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--pack-layers", type=int, default=None, help="layers of the pack workload (default: all 26)")
     ap.add_argument("--flip-steps", type=int, default=100, help="random-walk steps of the mask flip-rate study")
-    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks", "six_eight", "block"], default=None,
+    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks", "six_eight", "block", "optimizer"], default=None,
                     help="run one sub-measurement alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -617,6 +617,48 @@ def measure_dgrad(torch, bn, synth, peaks, reps=5):
     return out
 
 
+def measure_optimizer(torch, bn, synth, peaks, steps=3):
+    """The AdamW step with the next gamma over every linear weight of the 3B
+    model (26 layers x 7 matrices, 3.22 G fp32 masters): one batched call per
+    step against one call per matrix.  28 algorithmic bytes per weight."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    layers = synth.LLAMA_3B["layers"]
+    mats = synth.LAYER_3B_MATRICES
+    Ws, Gs, Ms, Vs = [], [], [], []
+    for l in range(layers):
+        for j, (name, N, K) in enumerate(mats):
+            Ws.append(synth.torch_master_weights(N, K, 0.02, seed=60000 + 10 * l + j, device=dev).reshape(-1))
+            Gs.append(synth.torch_master_weights(N, K, 1e-3, seed=70000 + 10 * l + j, device=dev).reshape(-1))
+            Ms.append(torch.zeros_like(Ws[-1]))
+            Vs.append(torch.zeros_like(Ws[-1]))
+    gam = torch.zeros(len(Ws), device=dev)
+    n_w = sum(w.numel() for w in Ws)
+    batch = bn.AdamWBatch([(Ws[i], Gs[i], Ms[i], Vs[i], gam[i:i + 1]) for i in range(len(Ws))], dev)
+    ws1 = bn.Workspace(bn.load().bitnet_adamw_workspace_size(), dev)
+    batch(1, lr=1e-4, weight_decay=0.1)
+    ms_b, ms_s = [], []
+    for st in range(2, 2 + steps):
+        with Timer(torch) as t:
+            batch(st, lr=1e-4, weight_decay=0.1)
+        ms_b.append(t.ms())
+    for st in range(2 + steps, 2 + 2 * steps):
+        with Timer(torch) as t:
+            for i in range(len(Ws)):
+                bn.bitnet_adamw_step(Ws[i], Gs[i], Ms[i], Vs[i], st, lr=1e-4, weight_decay=0.1,
+                                     gamma_out=gam[i:i + 1], ws=ws1)
+        ms_s.append(t.ms())
+    mb, msg = statistics.mean(ms_b), statistics.mean(ms_s)
+    out = {"weights": n_w, "matrices": len(Ws), "alg_bytes_per_weight": 28,
+           "batched": {"step_ms": round(mb, 3), "gbs": round(n_w * 28 / mb / 1e6, 1),
+                       "frac_of_hbm": round(n_w * 28 / mb / 1e6 / peaks["hbm"], 4),
+                       "entry": "bitnet_adamw_step_batch over all matrices"},
+           "per_matrix_calls": {"step_ms": round(msg, 3), "gbs": round(n_w * 28 / msg / 1e6, 1),
+                                "entry": "bitnet_adamw_step, one call per matrix"}}
+    del batch, Ws, Gs, Ms, Vs
+    torch.cuda.empty_cache()
+    return out
+
+
 def _graph(torch, fn):
     fn()   # first call outside capture (function attributes, lazy init)
     torch.cuda.synchronize()
@@ -664,7 +706,6 @@ def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
         pw[name] = bn.PackedWeights(N, K, dev, group_bytes=True, mma=True, dec=False)
         bn.bitnet_pack_nm(masters[name], pw[name], 1e-5)   # first pack sets each gamma hint
     moments = {n: (torch.zeros_like(masters[n]), torch.zeros_like(masters[n])) for n, _, _ in mats}
-    ws_opt = bn.Workspace(lib.bitnet_adamw_workspace_size(), dev)
     ws_wg = bn.Workspace(lib.bitnet_wgrad_workspace_size(), dev)
     # the optimiser leaves the exact gamma of the updated masters in pw.gamma: the pack reads W once
     batch = bn.PackBatch([(masters[n], pw[n]) for n, _, _ in mats], 1e-5, dev, gamma_known=True)
@@ -734,10 +775,11 @@ def measure_block(torch, bn, synth, peaks, reps=10, T=2048):
         for n, _, _ in mats:
             bn.bitnet_wgrad(dY[n], Xin[n], dW=dWs[n], ws=ws_wg)
 
-    def s_adamw():
-        for n, _, _ in mats:
-            bn.bitnet_adamw_step(masters[n], dWs[n], moments[n][0], moments[n][1], step_no[0], lr=1e-4,
-                                 weight_decay=0.1, gamma_out=pw[n].gamma, ws=ws_opt)
+    opt_batch = bn.AdamWBatch([(masters[n], dWs[n], moments[n][0], moments[n][1], pw[n].gamma) for n, _, _ in mats],
+                              dev)
+
+    def s_adamw():   # one launch for the block's four matrices
+        opt_batch(step_no[0], lr=1e-4, weight_decay=0.1)
 
     s_wgrad()
     s_adamw()   # the first optimiser step sets every gamma the pack then takes as known
@@ -896,7 +938,7 @@ def run_only(args):
     fn = {"prefill": measure_prefill, "pack": measure_pack, "dgrad": measure_dgrad,
           "peaks": lambda torch, bn, synth, peaks: measure_library_peaks(torch),
           "six_eight": lambda torch, bn, synth, peaks: measure_6of8(torch, bn, synth),
-          "block": measure_block}[args.only]
+          "block": measure_block, "optimizer": measure_optimizer}[args.only]
     kw = {"steps": args.steps, "flip_steps": args.flip_steps, "layers": args.pack_layers} if args.only == "pack" else {}
     print(json.dumps({args.only: fn(torch, bn, synth, peaks, **kw)}), flush=True)
     return 0
@@ -1018,6 +1060,8 @@ def run_ours(args):
             rows["block"] = measure_block(torch, bn, synth, peaks)
         with Nvtx(torch, "row pack"):
             rows["pack"] = measure_pack(torch, bn, synth, peaks, flip_steps=args.flip_steps)
+        with Nvtx(torch, "row optimizer"):
+            rows["optimizer"] = measure_optimizer(torch, bn, synth, peaks)
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": info.world, "steps": args.steps,

@@ -297,6 +297,31 @@ bitnet_status bitnet_adamw_step(float *W, const float *dW, float *m, float *v, i
                                 size_t ws_bytes, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_adamw_step_batch - bitnet_adamw_step over a list of matrices in one
+ * launch (per 64 matrices): the same update and the same gamma_out, bit for
+ * bit, as one call per matrix.
+ *   items   host array of n_items descriptors (read during the call only):
+ *             W, dW, m, v  [n] fp32 device arrays, 16-byte aligned, n % 4 == 0;
+ *             gamma_out    device fp32 scalar of that matrix.
+ *           The items' arrays must not overlap one another.
+ *   h, eps_gamma   as bitnet_adamw_step (one set for the whole list).
+ *   ws      >= bitnet_adamw_batch_workspace_size(n_items) bytes, 16-byte aligned.
+ * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    float *W;
+    const float *dW;
+    float *m;
+    float *v;
+    int64_t n;
+    float *gamma_out;
+} bitnet_adamw_item;
+
+size_t bitnet_adamw_batch_workspace_size(int32_t n_items);
+bitnet_status bitnet_adamw_step_batch(const bitnet_adamw_item *items, int32_t n_items, const bitnet_adamw_hparams *h,
+                                      float eps_gamma, void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * bitnet_rmsnorm_quant - RMSNorm fused into the per-token quantisation.
  *
  * "BitNet b1.58 ...", section "What this paper explains": the blocks around

@@ -35,6 +35,7 @@ EXPORTED = [
     "bitnet_decode_chain_workspace_size", "bitnet_decode_chain",
     "bitnet_dgrad_workspace_size", "bitnet_dgrad",
     "bitnet_wgrad_workspace_size", "bitnet_wgrad", "bitnet_adamw_workspace_size", "bitnet_adamw_step",
+    "bitnet_adamw_batch_workspace_size", "bitnet_adamw_step_batch",
     "bitnet_wait_selftest", "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
 ]
 
@@ -61,6 +62,11 @@ class BitnetPackItem(ctypes.Structure):
         ("w_dtype", ctypes.c_int32),
         ("gamma_known", ctypes.c_int32),
     ]
+
+
+class BitnetAdamWItem(ctypes.Structure):
+    _fields_ = [("W", ctypes.c_void_p), ("dW", ctypes.c_void_p), ("m", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("n", ctypes.c_int64), ("gamma_out", ctypes.c_void_p)]
 
 
 class BitnetAdamWHparams(ctypes.Structure):
@@ -126,6 +132,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_wgrad": (I32, [P, P, I64, I64, I64, P, I32, P, SZ, P]),
         "bitnet_adamw_workspace_size": (SZ, []),
         "bitnet_adamw_step": (I32, [P, P, P, P, I64, ctypes.POINTER(BitnetAdamWHparams), F, P, P, SZ, P]),
+        "bitnet_adamw_batch_workspace_size": (SZ, [I32]),
+        "bitnet_adamw_step_batch": (I32, [ctypes.POINTER(BitnetAdamWItem), I32, ctypes.POINTER(BitnetAdamWHparams), F,
+                                          P, SZ, P]),
         "bitnet_wait_selftest": (I32, [P, SZ, I32, P]),
         "bitnet_read_device_status": (I32, [P, P]),
         "bitnet_status_string": (ctypes.c_char_p, [I32]),
@@ -317,6 +326,34 @@ def bitnet_adamw_step(W, dW, m, v, step: int, lr: float, beta1: float = 0.9, bet
                                 ctypes.c_float(eps_gamma), _ptr(gamma_out), ws.ptr, ws.nbytes, _stream(stream)),
           "bitnet_adamw_step")
     return gamma_out
+
+
+class AdamWBatch:
+    """A fixed list of (W, dW, m, v, gamma_out) for bitnet_adamw_step_batch; the
+    descriptors and the workspace are built once, each call runs one step."""
+
+    def __init__(self, items, device="cuda"):
+        torch = _torch()
+        lib = load()
+        self.n = len(items)
+        arr = (BitnetAdamWItem * max(self.n, 1))()
+        self._keep = []
+        for i, (W, G, M, V, gamma) in enumerate(items):
+            for t in (W, G, M, V, gamma):
+                assert t.dtype == torch.float32 and t.is_contiguous()
+            self._keep.append((W, G, M, V, gamma))
+            arr[i] = BitnetAdamWItem(W.data_ptr(), G.data_ptr(), M.data_ptr(), V.data_ptr(), W.numel(),
+                                     gamma.data_ptr())
+        self._arr = arr
+        self.ws = Workspace(max(lib.bitnet_adamw_batch_workspace_size(self.n), 16), device)
+
+    def __call__(self, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.95, eps: float = 1e-8,
+                 weight_decay: float = 0.0, eps_gamma: float = 1e-5, stream=None):
+        lib = load()
+        h = BitnetAdamWHparams(lr, beta1, beta2, eps, weight_decay, adam_bias_correction(beta1, step),
+                               adam_bias_correction(beta2, step))
+        check(lib.bitnet_adamw_step_batch(self._arr, self.n, ctypes.byref(h), ctypes.c_float(eps_gamma), self.ws.ptr,
+                                          self.ws.nbytes, _stream(stream)), "bitnet_adamw_step_batch")
 
 
 def adam_bias_correction(beta: float, step: int) -> float:

@@ -281,6 +281,42 @@ bitnet_status bitnet_adamw_step(float *W, const float *dW, float *m, float *v, i
                        "adamw");
 }
 
+size_t bitnet_adamw_batch_workspace_size(int32_t n_items) {
+    return n_items > 0 ? static_cast<size_t>(n_items) * bitnet::kPackWsBytes : 0;
+}
+
+bitnet_status bitnet_adamw_step_batch(const bitnet_adamw_item *items, int32_t n_items, const bitnet_adamw_hparams *h,
+                                      float eps_gamma, void *ws, size_t ws_bytes, bitnet_stream_t stream) {
+    if (n_items < 0) return fail(BITNET_ERR_INVALID_ARG, "adamw_batch: n_items < 0");
+    if (n_items == 0) return BITNET_OK;
+    if (!items || !h) return fail(BITNET_ERR_INVALID_ARG, "adamw_batch: null items or hyper-parameters");
+    if (!(h->lr >= 0.0f) || !(h->beta1 >= 0.0f && h->beta1 < 1.0f) || !(h->beta2 >= 0.0f && h->beta2 < 1.0f) ||
+        !(h->eps > 0.0f) || !(h->weight_decay >= 0.0f) || !(h->bias_correction1 > 0.0f) ||
+        !(h->bias_correction2 > 0.0f) || !(eps_gamma >= 0.0f))
+        return fail(BITNET_ERR_INVALID_ARG, "adamw_batch: hyper-parameters out of range");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "adamw_batch: workspace is required");
+    if (ws_bytes < bitnet_adamw_batch_workspace_size(n_items))
+        return fail(BITNET_ERR_WORKSPACE, "adamw_batch: workspace needs %zu bytes", bitnet_adamw_batch_workspace_size(n_items));
+    if (!aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "adamw_batch: ws must be 16-byte aligned");
+    std::vector<bitnet::AdamWItemHost> hv(static_cast<size_t>(n_items));
+    double total_chunks = 0.0;
+    for (int32_t i = 0; i < n_items; ++i) {
+        const bitnet_adamw_item &it = items[i];
+        if (it.n <= 0 || it.n % 4) return fail(BITNET_ERR_INVALID_ARG, "adamw_batch: item %d: n must be a positive multiple of 4", i);
+        if (!it.W || !it.dW || !it.m || !it.v || !it.gamma_out)
+            return fail(BITNET_ERR_INVALID_ARG, "adamw_batch: item %d: null pointer", i);
+        if (!aligned(it.W, 16) || !aligned(it.dW, 16) || !aligned(it.m, 16) || !aligned(it.v, 16))
+            return fail(BITNET_ERR_INVALID_ARG, "adamw_batch: item %d: W, dW, m, v must be 16-byte aligned", i);
+        total_chunks += std::ceil(static_cast<double>(it.n) / 8192.0);
+        hv[static_cast<size_t>(i)] = {it.W, it.dW, it.m, it.v, it.n, it.gamma_out};
+    }
+    if (total_chunks > 4294967295.0) return fail(BITNET_ERR_UNSUPPORTED, "adamw_batch: too many weights in one call");
+    return cuda_status(bitnet::launch_adamw_gamma_batch(hv.data(), n_items, h->lr, h->beta1, h->beta2, h->eps,
+                                                        h->weight_decay, h->bias_correction1, h->bias_correction2,
+                                                        eps_gamma, ws, reinterpret_cast<cudaStream_t>(stream)),
+                       "adamw_batch");
+}
+
 bitnet_status bitnet_rmsnorm_quant(const void *X, const float *w, int64_t T, int64_t K, float eps_norm,
                                    float eps_act, int8_t *Xq, float *absmax, float *rinv, bitnet_stream_t stream) {
     if (T < 0 || K <= 0 || K % 8 || K > 65536) return fail(BITNET_ERR_INVALID_ARG, "rmsnorm_quant: need T >= 0, 0 < K <= 65536, K %% 8 == 0");

@@ -82,6 +82,18 @@ cudaError_t launch_adamw_gamma(float *W, const float *G, float *M, float *V, int
 // Health check of the bounded waits (chain.cu): both kinds of wait run out on events that never happen
 cudaError_t launch_wait_selftest(void *ws, uint64_t limit_ns, cudaStream_t s);
 
+// The AdamW step with gamma over a list of matrices (pack.cu)
+struct AdamWItemHost {
+    float *W;
+    const float *G;
+    float *M, *V;
+    int64_t n;
+    float *gamma;
+};
+constexpr int kAdamWBatchMax = 64;   // matrices per launch (kernel parameter space)
+cudaError_t launch_adamw_gamma_batch(const AdamWItemHost *items, int n_items, float lr, float b1, float b2, float eps,
+                                     float wd, float c1, float c2, float eps_gamma, void *ws, cudaStream_t s);
+
 // Weight gradient (gemm2.cu)
 cudaError_t launch_gemm_wgrad_pair(const void *dY, const void *X, int64_t T, int64_t n_out, int64_t k, float *dW,
                                    bool accumulate, uint32_t *status, cudaStream_t s);

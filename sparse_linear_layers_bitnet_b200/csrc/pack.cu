@@ -1280,6 +1280,201 @@ cudaError_t launch_adamw_gamma(float *W, const float *G, float *M, float *V, int
     return cudaGetLastError();
 }
 
+// The same AdamW step over a list of matrices in one launch: every matrix is cut
+// into chunks of kAdamWChunk float4 groups and every CTA takes a contiguous
+// range of the global chunk list (so it meets one or two matrices); per matrix
+// the exact partial sums go to its own workspace header, and the CTA that
+// completes its last chunk forms its gamma.
+constexpr uint32_t kAdamWChunk = 2048;   // float4 groups per chunk (8192 weights)
+
+struct AdamWBatchItem {
+    float4 *W;
+    const float4 *G;
+    float4 *M, *V;
+    int64_t n4;
+    float *gamma;
+    uint8_t *hdr;             // kPackWsBytes scratch header (zeroed before the launch)
+    uint32_t chunk0, nchunks;
+};
+
+struct AdamWBatchParams {
+    AdamWBatchItem it[kAdamWBatchMax];
+    int32_t n;
+    uint32_t total_chunks;
+    float lr, b1, b2, eps, wd, c1, c2, eps_gamma;
+};
+
+__device__ __forceinline__ int adamw_item_of(const AdamWBatchParams &bp, uint32_t c) {
+    int lo = 0, hi = bp.n - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (bp.it[mid].chunk0 <= c) lo = mid;
+        else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void __launch_bounds__(256, 6) k_adamw_gamma_batch(const __grid_constant__ AdamWBatchParams bp) {
+    __shared__ unsigned long long s_bins[256];
+    __shared__ unsigned long long s_lo[8], s_hi[8];
+    __shared__ int s_rare;
+    __shared__ unsigned s_ticket;
+    __shared__ int s_nz[256];
+    __shared__ int s_nnz;
+    __shared__ uint32_t s_limb[kLimbs];
+    const uint32_t lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t G = gridDim.x;
+    const uint32_t c_begin = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x) * bp.total_chunks) / G);
+    const uint32_t c_end = static_cast<uint32_t>((static_cast<uint64_t>(blockIdx.x + 1) * bp.total_chunks) / G);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) s_bins[i] = 0ull;
+    if (threadIdx.x == 0) s_rare = 0;
+    __syncthreads();
+    AdamWArgs a;   // the scalar hyper-parameters in the form adamw1 takes them
+    a.lr = bp.lr;
+    a.b1 = bp.b1;
+    a.b2 = bp.b2;
+    a.eps = bp.eps;
+    a.wd = bp.wd;
+    a.c1 = bp.c1;
+    a.c2 = bp.c2;
+    const float omb1 = __fsub_rn(1.0f, bp.b1), omb2 = __fsub_rn(1.0f, bp.b2);
+    uint32_t c = c_begin;
+    while (c < c_end) {
+        const int item = adamw_item_of(bp, c);
+        const AdamWBatchItem &I = bp.it[item];
+        const uint32_t seg_end = min(c_end, I.chunk0 + I.nchunks);
+        uint64_t lo = 0, hi = 0;
+        double d = 0.0;
+        for (uint32_t ch = c; ch < seg_end; ++ch) {
+            const int64_t base = static_cast<int64_t>(ch - I.chunk0) * kAdamWChunk;
+            const int64_t end = min(base + static_cast<int64_t>(kAdamWChunk), I.n4);
+            for (int64_t j = base + threadIdx.x; j < end; j += blockDim.x) {
+                const float4 w = I.W[j], g = __ldg(I.G + j);
+                float4 m = I.M[j], v = I.V[j];
+                float4 wn;
+                wn.x = adamw1(w.x, g.x, m.x, v.x, a, omb1, omb2);
+                wn.y = adamw1(w.y, g.y, m.y, v.y, a, omb1, omb2);
+                wn.z = adamw1(w.z, g.z, m.z, v.z, a, omb1, omb2);
+                wn.w = adamw1(w.w, g.w, m.w, v.w, a, omb1, omb2);
+                I.W[j] = wn;
+                I.M[j] = m;
+                I.V[j] = v;
+                sum_float4(wn, d, lo, hi, s_bins, &s_rare);
+            }
+            flush_sum(d, lo, hi);   // at most 8 groups (32 magnitudes) per thread per chunk
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const uint64_t l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+            const uint64_t h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+            const uint64_t sum = lo + l2;
+            hi = hi + h2 + ((sum < lo) ? 1ull : 0ull);
+            lo = sum;
+        }
+        if (lane == 0) {
+            s_lo[warp] = lo;
+            s_hi[warp] = hi;
+        }
+        __syncthreads();
+        unsigned long long *win = reinterpret_cast<unsigned long long *>(I.hdr + kPackWsWinOffset);
+        unsigned long long *bins = reinterpret_cast<unsigned long long *>(I.hdr + kPackWsBinsOffset);
+        if (threadIdx.x == 0) {
+            uint64_t L = 0, H = 0;
+            for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+                const uint64_t sum = L + s_lo[w];
+                H = H + s_hi[w] + ((sum < L) ? 1ull : 0ull);
+                L = sum;
+            }
+            if (L | H) {
+                const unsigned long long old = atomicAdd(&win[0], static_cast<unsigned long long>(L));
+                const uint64_t carry = (static_cast<uint64_t>(old) + L < static_cast<uint64_t>(old)) ? 1ull : 0ull;
+                atomicAdd(&win[1], static_cast<unsigned long long>(H + carry));
+            }
+        }
+        if (s_rare) {
+            for (int e = threadIdx.x; e < 256; e += blockDim.x)
+                if (s_bins[e]) {
+                    atomicAdd(&bins[e], s_bins[e]);
+                    s_bins[e] = 0ull;
+                }
+        }
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            s_rare = 0;
+            const unsigned done = seg_end - c;
+            s_ticket = atomicAdd(reinterpret_cast<unsigned *>(I.hdr + kPackWsCounterOffset), done) + done;
+        }
+        __syncthreads();
+        if (s_ticket == I.nchunks) {   // every chunk of this matrix is summed: its gamma
+            __threadfence();
+            if (threadIdx.x == 0) s_nnz = 0;
+            __syncthreads();
+            for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+                const unsigned long long b = atomicAdd(&bins[e], 0ull);
+                s_bins[e] = b;
+                if (b) s_nz[atomicAdd(&s_nnz, 1)] = e;
+            }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                for (int q = 1; q < s_nnz; ++q)
+                    for (int j = q; j > 0 && s_nz[j - 1] > s_nz[j]; --j) {
+                        const int tmp = s_nz[j];
+                        s_nz[j] = s_nz[j - 1];
+                        s_nz[j - 1] = tmp;
+                    }
+                const uint64_t wlo = atomicAdd(&win[0], 0ull), whi = atomicAdd(&win[1], 0ull);
+                finalize_gamma(s_bins, s_nz, s_nnz, wlo, whi, I.n4 * 4, bp.eps_gamma, s_limb, I.gamma,
+                               reinterpret_cast<uint32_t *>(I.hdr + kPackWsThrOffset));
+            }
+            __syncthreads();
+            for (int e = threadIdx.x; e < 256; e += blockDim.x) s_bins[e] = 0ull;
+            __syncthreads();
+        }
+        c = seg_end;
+    }
+}
+
+cudaError_t launch_adamw_gamma_batch(const AdamWItemHost *items, int n_items, float lr, float b1, float b2, float eps,
+                                     float wd, float c1, float c2, float eps_gamma, void *ws, cudaStream_t s) {
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    cudaError_t err = cudaMemsetAsync(ws, 0, static_cast<size_t>(n_items) * kPackWsBytes, s);
+    if (err != cudaSuccess) return err;
+    for (int base = 0; base < n_items; base += kAdamWBatchMax) {
+        const int n = (n_items - base) < kAdamWBatchMax ? (n_items - base) : kAdamWBatchMax;
+        AdamWBatchParams bp;
+        uint32_t chunks = 0;
+        for (int i = 0; i < n; ++i) {
+            const AdamWItemHost &h = items[base + i];
+            AdamWBatchItem &I = bp.it[i];
+            I.W = reinterpret_cast<float4 *>(h.W);
+            I.G = reinterpret_cast<const float4 *>(h.G);
+            I.M = reinterpret_cast<float4 *>(h.M);
+            I.V = reinterpret_cast<float4 *>(h.V);
+            I.n4 = h.n / 4;
+            I.gamma = h.gamma;
+            I.hdr = w8 + static_cast<size_t>(base + i) * kPackWsBytes;
+            I.chunk0 = chunks;
+            I.nchunks = static_cast<uint32_t>((I.n4 + kAdamWChunk - 1) / kAdamWChunk);
+            chunks += I.nchunks;
+        }
+        bp.n = n;
+        bp.total_chunks = chunks;
+        bp.lr = lr;
+        bp.b1 = b1;
+        bp.b2 = b2;
+        bp.eps = eps;
+        bp.wd = wd;
+        bp.c1 = c1;
+        bp.c2 = c2;
+        bp.eps_gamma = eps_gamma;
+        const uint32_t want = static_cast<uint32_t>(num_sms() * 6);
+        const unsigned grid = chunks < want ? chunks : want;
+        k_adamw_gamma_batch<<<grid, 256, 0, s>>>(bp);
+    }
+    return cudaGetLastError();
+}
+
 cudaError_t launch_pack_update(const float *W, int64_t n_out, int64_t k, float eps, float *gamma, uint8_t *gb,
                                int8_t *vals, uint8_t *meta, uint8_t *dec, uint8_t *mask, void *ws, size_t ws_bytes,
                                cudaStream_t s) {

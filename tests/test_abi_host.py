@@ -160,6 +160,28 @@ def test_train_step_entries_reject_bad_arguments(lib):
     assert g(*ok_args[:5], None, *ok_args[6:]) == bad                                      # null hyper-parameters
 
 
+def test_adamw_batch_rejects_bad_arguments(lib):
+    bad = _abi.BITNET_ERR_INVALID_ARG
+    h = _abi.BitnetAdamWHparams(1e-3, 0.9, 0.95, 1e-8, 0.1, 0.1, 0.05)
+    items = (_abi.BitnetAdamWItem * 2)()
+    for it in items:
+        it.W, it.dW, it.m, it.v, it.n, it.gamma_out = 4096, 4096, 4096, 4096, 1024, 4096
+    ws, n = _fake(), lib.bitnet_adamw_batch_workspace_size(2)
+    assert n == 2 * lib.bitnet_adamw_workspace_size()
+    assert lib.bitnet_adamw_step_batch(items, 0, ctypes.byref(h), 1e-5, None, 0, None) == _abi.BITNET_OK
+    assert lib.bitnet_adamw_step_batch(items, -1, ctypes.byref(h), 1e-5, ws, n, None) == bad
+    assert lib.bitnet_adamw_step_batch(items, 2, None, 1e-5, ws, n, None) == bad
+    assert lib.bitnet_adamw_step_batch(items, 2, ctypes.byref(h), 1e-5, ws, n - 1, None) == _abi.BITNET_ERR_WORKSPACE
+    items[1].n = 1022
+    assert lib.bitnet_adamw_step_batch(items, 2, ctypes.byref(h), 1e-5, ws, n, None) == bad      # n % 4
+    items[1].n = 1024
+    items[1].v = 4100
+    assert lib.bitnet_adamw_step_batch(items, 2, ctypes.byref(h), 1e-5, ws, n, None) == bad      # alignment
+    items[1].v = 4096
+    items[0].gamma_out = None
+    assert lib.bitnet_adamw_step_batch(items, 2, ctypes.byref(h), 1e-5, ws, n, None) == bad      # null gamma
+
+
 def test_wait_selftest_rejects_bad_arguments(lib):
     n = lib.bitnet_decode_chain_workspace_size(1)
     assert lib.bitnet_wait_selftest(None, n, 1000, None) == _abi.BITNET_ERR_WORKSPACE

@@ -132,3 +132,38 @@ def test_pack_with_known_gamma(bn):
             if n * k <= 1 << 20:
                 g, keep, wq, gb = oracle.pack_weights(Ws[i].cpu().numpy(), 1e-5)
                 assert outs[i].gamma.item() == float(g) and np.array_equal(outs[i].group_bytes.cpu().numpy(), gb)
+
+
+def test_adamw_batch_matches_single_calls(bn):
+    """The one-launch AdamW over a list of matrices (mixed sizes: one chunk,
+    many chunks, rare magnitudes) leaves W, m, v and every gamma bit-identical
+    to one bitnet_adamw_step per matrix, over three steps; gamma also equals
+    the oracle's."""
+    shapes = [(256, 512, False), (96, 64, True), (3200, 3200, False), (200, 352, True), (640, 2560, False)]
+    r = np.random.default_rng(21)
+    Wb, Ws = [], []
+    for i, (n, k, rare) in enumerate(shapes):
+        W = _masters(n, k, 700 + i, rare).reshape(-1)
+        Wb.append(torch.from_numpy(W.copy()).cuda())
+        Ws.append(torch.from_numpy(W.copy()).cuda())
+    Mb = [torch.zeros_like(w) for w in Wb]
+    Vb = [torch.zeros_like(w) for w in Wb]
+    Ms = [torch.zeros_like(w) for w in Ws]
+    Vs = [torch.zeros_like(w) for w in Ws]
+    gb = torch.zeros(len(shapes), device="cuda")
+    gs = torch.zeros(len(shapes), device="cuda")
+    Gs = [torch.empty_like(w) for w in Wb]
+    batch = bn.AdamWBatch([(Wb[i], Gs[i], Mb[i], Vb[i], gb[i:i + 1]) for i in range(len(shapes))])
+    for step in range(1, 4):
+        for G in Gs:
+            G.copy_(torch.from_numpy((r.normal(size=G.numel()) * 1e-3).astype(np.float32)))
+        batch(step, lr=1e-3, weight_decay=0.1)
+        for i in range(len(shapes)):
+            bn.bitnet_adamw_step(Ws[i], Gs[i], Ms[i], Vs[i], step, lr=1e-3, weight_decay=0.1, gamma_out=gs[i:i + 1])
+        torch.cuda.synchronize()
+        for i in range(len(shapes)):
+            assert torch.equal(Wb[i], Ws[i]) and torch.equal(Mb[i], Ms[i]) and torch.equal(Vb[i], Vs[i]), (step, i)
+        assert torch.equal(gb, gs), step
+        for i, (n, k, _) in enumerate(shapes):
+            if n * k <= 1 << 20:
+                assert gb[i].item() == float(oracle.gamma(Wb[i].cpu().numpy().reshape(n, k), 1e-5)), (step, i)
