@@ -52,23 +52,30 @@ __device__ __forceinline__ int8_t quant_one(float x, float s) {
     return static_cast<int8_t>(q);
 }
 
-template <bool BF16>
-__global__ void __launch_bounds__(kQuantThreads) k_quant_act(const uint4 *__restrict__ X, int64_t K, float eps,
+// TPC tokens per CTA, kQuantThreads / TPC threads (a whole number of warps) per
+// token: short rows pack several tokens into one CTA, so each thread keeps up
+// to kQuantMaxChunks loads in flight instead of one or two.
+template <bool BF16, int TPC>
+__global__ void __launch_bounds__(kQuantThreads) k_quant_act(const uint4 *__restrict__ X, int64_t T, int64_t K, float eps,
                                                              int8_t *__restrict__ Xq, float *__restrict__ amax) {
     using C = Chunk<BF16>;
+    constexpr int kTpt = kQuantThreads / TPC;   // threads per token
+    constexpr int kWpt = kTpt / 32;             // warps per token
     __shared__ float s_red[32];
-    const int64_t t = blockIdx.x;
-    const int64_t nchunk = K / C::kElems;
-    const uint4 *row = X + t * nchunk;
+    const int grp = threadIdx.x / kTpt, gt = threadIdx.x % kTpt;
+    const int64_t t = static_cast<int64_t>(blockIdx.x) * TPC + grp;
+    const bool valid = t < T;
+    const int64_t nchunk = valid ? K / C::kElems : 0;
+    const uint4 *row = X + t * (K / C::kElems);
     C reg[kQuantMaxChunks];
     float m = 0.0f;
-    const bool fits = nchunk <= static_cast<int64_t>(kQuantMaxChunks) * kQuantThreads;
+    const bool fits = nchunk <= static_cast<int64_t>(kQuantMaxChunks) * kTpt;
     // X may be the output of the previous kernel of the stream
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 #pragma unroll
     for (int u = 0; u < kQuantMaxChunks; ++u) {
-        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        const int64_t c = gt + static_cast<int64_t>(u) * kTpt;
         if (c < nchunk) {
             reg[u].raw = __ldg(row + c);
 #pragma unroll
@@ -76,22 +83,32 @@ __global__ void __launch_bounds__(kQuantThreads) k_quant_act(const uint4 *__rest
         }
     }
     if (!fits) {   // rows longer than the register cache: a second read later
-        for (int64_t c = threadIdx.x + static_cast<int64_t>(kQuantMaxChunks) * kQuantThreads; c < nchunk;
-             c += kQuantThreads) {
+        for (int64_t c = gt + static_cast<int64_t>(kQuantMaxChunks) * kTpt; c < nchunk; c += kTpt) {
             C ch;
             ch.raw = __ldg(row + c);
 #pragma unroll
             for (int j = 0; j < C::kElems; ++j) m = fmaxf(m, fabsf(ch.get(j)));
         }
     }
-    m = block_max(m, s_red);
+    if (TPC == 1) {
+        m = block_max(m, s_red);
+    } else {   // the token's own warps
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+        __syncthreads();
+        m = s_red[grp * kWpt];
+#pragma unroll
+        for (int w = 1; w < kWpt; ++w) m = fmaxf(m, s_red[grp * kWpt + w]);
+    }
+    if (!valid) return;
     const float a = m > eps ? m : eps;
     const float s = __fdiv_rn(127.0f, a);
-    if (threadIdx.x == 0) amax[t] = a;
+    if (gt == 0) amax[t] = a;
     int8_t *out = Xq + t * K;
 #pragma unroll
     for (int u = 0; u < kQuantMaxChunks; ++u) {
-        const int64_t c = threadIdx.x + static_cast<int64_t>(u) * kQuantThreads;
+        const int64_t c = gt + static_cast<int64_t>(u) * kTpt;
         if (c < nchunk) {
             uint32_t w[2] = {0u, 0u};
 #pragma unroll
@@ -104,8 +121,7 @@ __global__ void __launch_bounds__(kQuantThreads) k_quant_act(const uint4 *__rest
         }
     }
     if (!fits) {
-        for (int64_t c = threadIdx.x + static_cast<int64_t>(kQuantMaxChunks) * kQuantThreads; c < nchunk;
-             c += kQuantThreads) {
+        for (int64_t c = gt + static_cast<int64_t>(kQuantMaxChunks) * kTpt; c < nchunk; c += kTpt) {
             C ch;
             ch.raw = __ldg(row + c);
             uint32_t w[2] = {0u, 0u};
@@ -120,13 +136,28 @@ __global__ void __launch_bounds__(kQuantThreads) k_quant_act(const uint4 *__rest
     }
 }
 
+template <bool BF16, int TPC>
+static cudaError_t quant_launch(cudaLaunchConfig_t &cfg, const uint4 *x, int64_t T, int64_t K, float eps, int8_t *Xq,
+                                float *amax) {
+    return cudaLaunchKernelEx(&cfg, k_quant_act<BF16, TPC>, x, T, K, eps, Xq, amax);
+}
+
 cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, float eps, int8_t *Xq, float *amax,
                              cudaStream_t s) {
     if (T <= 0) return cudaSuccess;
+    // tokens per CTA: the most whose rows still fit the register cache (and at least one chunk per thread)
+    const int64_t nchunk = K / (bf16 ? 8 : 4);
+    int tpc = 1;
+    for (int c = 8; c > 1; c >>= 1)
+        if (nchunk <= static_cast<int64_t>(kQuantMaxChunks) * (kQuantThreads / c) && nchunk >= kQuantThreads / c &&
+            T >= 2 * c) {
+            tpc = c;
+            break;
+        }
     // programmatic serialisation: the kernel that consumes Xq may start its own
     // independent loads while this one runs
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(T));
+    cfg.gridDim = dim3(static_cast<unsigned>((T + tpc - 1) / tpc));
     cfg.blockDim = dim3(kQuantThreads);
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -135,8 +166,12 @@ cudaError_t launch_quant_act(const void *X, bool bf16, int64_t T, int64_t K, flo
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     const uint4 *x = static_cast<const uint4 *>(X);
-    if (bf16) return cudaLaunchKernelEx(&cfg, k_quant_act<true>, x, K, eps, Xq, amax);
-    return cudaLaunchKernelEx(&cfg, k_quant_act<false>, x, K, eps, Xq, amax);
+    switch (tpc) {
+        case 8: return bf16 ? quant_launch<true, 8>(cfg, x, T, K, eps, Xq, amax) : quant_launch<false, 8>(cfg, x, T, K, eps, Xq, amax);
+        case 4: return bf16 ? quant_launch<true, 4>(cfg, x, T, K, eps, Xq, amax) : quant_launch<false, 4>(cfg, x, T, K, eps, Xq, amax);
+        case 2: return bf16 ? quant_launch<true, 2>(cfg, x, T, K, eps, Xq, amax) : quant_launch<false, 2>(cfg, x, T, K, eps, Xq, amax);
+        default: return bf16 ? quant_launch<true, 1>(cfg, x, T, K, eps, Xq, amax) : quant_launch<false, 1>(cfg, x, T, K, eps, Xq, amax);
+    }
 }
 
 
