@@ -2,10 +2,14 @@
 //
 // Same products as gemm.cu: the 2:4-sparse int8 x ternary forward
 // ("BitNet b1.58: Ternary Weights for 1.58-bit LLMs", section "The mechanism";
-// "Sparse-BitNet" (gist.science), section 2) and the dense bf16 STE input
-// gradient ("Sparse-BitNet", section 2 "Training Strategie").  Results are
-// identical to gemm.cu (integer accumulation is exact; the fp32 epilogue does
-// the same operations in the same order).
+// "Sparse-BitNet" (gist.science), section 2), the dense bf16 STE input
+// gradient and the dense weight gradient dW = dY^T X ("Sparse-BitNet",
+// section 2 "Training Strategie").  The forward results are identical to
+// gemm.cu (integer accumulation is exact; the fp32 epilogue does the same
+// operations in the same order).  Dense operands are K-major or MN-major
+// (template mask MN): the input gradient reads Wq as bf16 rows (B MN-major),
+// the weight gradient reads dY and X with the token index as the contraction
+// (both MN-major), so no operand is ever transposed in memory.
 //
 // A cluster of two CTAs on two SMs computes one 256 x BN output tile with one
 // MMA instruction stream: each CTA holds 128 rows of A and BN/2 rows of B in
