@@ -307,16 +307,6 @@ __device__ __forceinline__ void window_add_f64(double s, uint64_t &lo, uint64_t 
     add128_sq(lo, hi, vl, vh);
 }
 
-__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
-__device__ __forceinline__ uint32_t vmin_u16x2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
 
 // |x| of a normal bf16 (15 bits: exponent E and 7 mantissa bits, at bit 13 of
 // a word) as an fp64: the high word with the exponent rebiased by 1023 - 127
@@ -379,18 +369,6 @@ __device__ __forceinline__ void chunk_f32(const uint4 &u, float *f) {
     f[4] = bf16_lo(u.z); f[5] = bf16_hi(u.z); f[6] = bf16_lo(u.w); f[7] = bf16_hi(u.w);
 }
 
-// Eight codes at once.  With |v| <= a and s = fp32(127 / a), |v s| <= 127 (1 + 2^-24)
-// rounds to at most 127 in magnitude, so the clamp never acts; after adding
-// 1.5 2^23 the low byte of the sum's bits is the code in two's complement.
-__device__ __forceinline__ uint2 codes8_fast(const float *v, float s) {
-    uint32_t b[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) b[e] = __float_as_uint(__fadd_rn(__fmul_rn(v[e], s), 12582912.0f));
-    uint2 q;
-    q.x = __byte_perm(__byte_perm(b[0], b[1], 0x0040u), __byte_perm(b[2], b[3], 0x0040u), 0x5410u);
-    q.y = __byte_perm(__byte_perm(b[4], b[5], 0x0040u), __byte_perm(b[6], b[7], 0x0040u), 0x5410u);
-    return q;
-}
 
 __device__ __forceinline__ uint2 codes8(const float *v, float s) {
     uint2 q;

@@ -213,4 +213,41 @@ __device__ __forceinline__ uint2 group_bf16x4(uint32_t b) {
                       code_bf16((c4 >> 4) & 3u) | (code_bf16(c4 >> 6) << 16));
 }
 
+// ---------------------------------------------------------------- int8 activation codes
+//
+// The per-token code is clamp(rint(fp32(x s)), -127, 127) with s = fp32(127 / a)
+// and a >= max |x| of the token.  Then |x s| <= 127 (1 + 2^-24), which rounds
+// to at most 127 in magnitude, so the clamp never acts; adding 1.5 2^23 to the
+// product rounds it to an integer (ties to even, exactly as rint, since
+// |x s| < 2^22) and the low byte of the sum's bits is the code in two's
+// complement.  No float-to-int conversion instruction is needed.
+
+// Four codes packed little-endian into one word.
+__device__ __forceinline__ uint32_t codes4_fast(float v0, float v1, float v2, float v3, float s) {
+    const uint32_t b0 = __float_as_uint(__fadd_rn(__fmul_rn(v0, s), 12582912.0f));
+    const uint32_t b1 = __float_as_uint(__fadd_rn(__fmul_rn(v1, s), 12582912.0f));
+    const uint32_t b2 = __float_as_uint(__fadd_rn(__fmul_rn(v2, s), 12582912.0f));
+    const uint32_t b3 = __float_as_uint(__fadd_rn(__fmul_rn(v3, s), 12582912.0f));
+    return __byte_perm(__byte_perm(b0, b1, 0x0040u), __byte_perm(b2, b3, 0x0040u), 0x5410u);
+}
+
+// Eight codes (v[0..7]) in two words.
+__device__ __forceinline__ uint2 codes8_fast(const float *v, float s) {
+    return make_uint2(codes4_fast(v[0], v[1], v[2], v[3], s), codes4_fast(v[4], v[5], v[6], v[7], s));
+}
+
+// Per-lane unsigned 16-bit max / min of two packed pairs.  On bf16 bit
+// patterns with the sign bit cleared the order of the patterns is the order of
+// the magnitudes, so max.u16x2 is a two-wide |x| max.
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t vmin_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 }  // namespace bitnet

@@ -195,6 +195,30 @@ def test_quant_act_parity(bn, T, K, dtype):
     assert np.array_equal(a.cpu().numpy(), a_ref)
 
 
+# Hundreds to thousands of token groups (more CTAs than fit on the GPU at
+# once), ragged last groups (T not a multiple of the tokens per CTA), every
+# group size (8, 4, 2, 1 tokens per CTA), rows past the register cache, and
+# per-row scales spread over six decades so that a token quantised with another
+# token's scale fails.
+@pytest.mark.parametrize("T,K,dtype", [(4099, 4096, "bf16"), (2501, 3200, "bf16"), (701, 11008, "bf16"),
+                                      (3003, 1024, "f32"), (1201, 4096, "f32"), (333, 40000, "bf16"),
+                                      (4096, 11008, "bf16")])
+def test_quant_act_many_groups_per_cta(bn, T, K, dtype):
+    X = synth.activations(T, K, seed=3 * T + K, outlier_p=0.01)
+    X *= (10.0 ** synth.rng(T).uniform(-3.0, 3.0, size=(T, 1))).astype(np.float32)
+    X[0, :] = 0.0
+    X[T - 1, :] = 0.0   # eps clamp in the ragged last group
+    if dtype == "bf16":
+        Xd, X32 = bf16_dev(X)
+    else:
+        Xd, X32 = dev_f32(X), X
+    xq_ref, a_ref = oracle.quant_act(X32, 1e-5)
+    Xq, a = bn.bitnet_quant_act(Xd, 1e-5)
+    torch.cuda.synchronize()
+    assert np.array_equal(a.cpu().numpy(), a_ref)
+    assert np.array_equal(Xq.cpu().numpy(), xq_ref)
+
+
 # ------------------------------------------------------------------ sparse linear
 
 def _linear_case(bn, n_out, k, T, seed, dec=True, y_dtype="f32"):
