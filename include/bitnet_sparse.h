@@ -448,7 +448,7 @@ bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps
  *   eps      activation eps (> 0).
  *   ws       >= bitnet_decode_chain_workspace_size(n_ops) bytes: status word,
  *            abort word and one completion counter per op (cleared by the call).
- * Shared memory bounds T * (max k + 16): the call returns UNSUPPORTED when
+ * Shared memory bounds T * (max k + 128): the call returns UNSUPPORTED when
  * fewer than two 16 KB weight stages would fit.
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA; a wait that runs out
  * inside the kernel sets the TIMEOUT bit of the device status word.

@@ -482,7 +482,7 @@ bitnet_status bitnet_decode_chain(const bitnet_chain_op *ops, int32_t n_ops, int
                                        static_cast<int32_t>(W->n_out), static_cast<int32_t>(W->k), o.wait_prev, 0};
     }
     if (!chain_fits(T, kmax))
-        return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: T * (k + 16) leaves no room for two weight stages");
+        return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: T * (k + 128) leaves no room for two weight stages");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return cuda_status(bitnet::launch_decode_chain(dev.data(), n_ops, T, x_dtype == BITNET_BF16, y_dtype == BITNET_BF16,
                                                    eps, kmax, ws, s),

@@ -170,13 +170,6 @@ __device__ __forceinline__ bool consumer_sync_or(bool v) {
     return r != 0;
 }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&b)[4], uint32_t addr) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
-                 : "r"(addr)
-                 : "memory");
-}
-
 // adds a row tile's partial sums (four accumulators) into the shared sums and clears them
 __device__ __forceinline__ void chain_flush(int *s_acc, int tile, int lane, int (&acc)[4][4]) {
 #pragma unroll
@@ -202,20 +195,37 @@ struct ChainChunk {
         for (int j = 0; j < kElems; ++j) m = fmaxf(m, fabsf(get(j)));
         return m;
     }
-    __device__ __forceinline__ void store_codes(int8_t *dst, float s) const {
-        uint32_t w[2] = {0u, 0u};
+    // Codes of the chunk's elements e0 .. e0 + kElems - 1 of a token row whose
+    // shared copy starts at row.  Within each 64-element k-tile the sixteen
+    // 4-byte words are stored transposed (word 4 j + q at 4 q + j), so that the
+    // 16 bytes lane q of a token takes as its m16n8k64 B fragment (k = 4 q + 16 j
+    // + 0..3, j = 0..3) are contiguous.
+    __device__ __forceinline__ void store_codes(int8_t *row, int e0, float s) const {
+        int8_t *tile = row + (e0 & ~63);
+        const int u0 = (e0 & 63) >> 2;   // first word within the tile
+        if constexpr (BF16) {
+            float v[8];
 #pragma unroll
-        for (int j = 0; j < kElems; ++j)
-            w[j >> 2] |= static_cast<uint32_t>(static_cast<uint8_t>(quant_code(get(j), s))) << (8 * (j & 3));
-        if (BF16)
-            *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
-        else
-            *reinterpret_cast<uint32_t *>(dst) = w[0];
+            for (int j = 0; j < 8; ++j) v[j] = get(j);
+            const uint2 q = codes8_fast(v, s);
+            const int u1 = u0 + 1;
+            *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u0 & 3) + (u0 >> 2))) = q.x;
+            *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u1 & 3) + (u1 >> 2))) = q.y;
+        } else {
+            *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u0 & 3) + (u0 >> 2))) =
+                codes4_fast(get(0), get(1), get(2), get(3), s);
+        }
     }
 };
 
+// Row pitch of the shared int8 activations: k + 64 or k + 128, whichever is
+// 64 mod 128 bytes, so that the two token rows one quarter-warp reads in a
+// 16-byte-per-lane load fall in disjoint banks.
+__device__ __host__ __forceinline__ int64_t chain_pitch(int64_t k) { return k + 64 + (k & 64); }
+
 // Per-token absmax, scales and int8 codes of one projection's activations
-// (same arithmetic as bitnet_quant_act) into shared memory, row pitch k + 16.
+// (same arithmetic as bitnet_quant_act) into shared memory, row pitch
+// chain_pitch(k), each 64-k tile in fragment order (see store_codes).
 // X is read through L2 only (ld.global.cg): it may have been written by other
 // SMs earlier in this kernel.  Thread ctid takes the flattened 16-byte chunks
 // c = ctid + 512 u.  The first kChainKeep of them are loaded together (all in
@@ -308,14 +318,14 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
         s_scale[ctid] = __fdiv_rn(__fmul_rn(gamma, v), 127.0f);
     }
     consumer_sync();
-    const int pitch = k + 16;
+    const int pitch = chain_pitch(k);
 #pragma unroll
     for (int u = 0; u < kChainKeep; ++u) {
         const int c = ctid + u * kChainConsumers;
         if (c < nchunk) {
             int t, i;
             chain_chunk_pos<BF16>(c, cpr, inv_cpr, t, i);
-            keep[u].store_codes(s_xq + t * pitch + i * C::kElems, s_inv[t]);
+            keep[u].store_codes(s_xq + t * pitch, i * C::kElems, s_inv[t]);
         }
     }
     for (int c0 = ctid + kChainKeep * kChainConsumers; c0 < nchunk; c0 += kChainKeep * kChainConsumers) {
@@ -331,7 +341,7 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
             if (c < nchunk) {
                 int t, i;
                 chain_chunk_pos<BF16>(c, cpr, inv_cpr, t, i);
-                v[u].store_codes(s_xq + t * pitch + i * C::kElems, s_inv[t]);
+                v[u].store_codes(s_xq + t * pitch, i * C::kElems, s_inv[t]);
             }
         }
     }
@@ -353,10 +363,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     const uint32_t stage_bytes = p.stage_bytes;
     int *s_acc = reinterpret_cast<int *>(smem + static_cast<size_t>(ns) * stage_bytes);
     int8_t *s_xq = reinterpret_cast<int8_t *>(s_acc + kChainMaxTiles * 128);
-    int8_t *s_zero = s_xq + static_cast<size_t>(T) * static_cast<size_t>(p.kmax + 16);   // 64 zero bytes
 
     for (int i = tid; i < kChainMaxTiles * 128; i += kChainThreads) s_acc[i] = 0;
-    for (int i = tid; i < 64; i += kChainThreads) s_zero[i] = 0;
     if (tid == 0) {
         s_abort = 0;
         for (int s = 0; s < ns; ++s) {
@@ -440,15 +448,15 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                                   s_scale, ctid);
             consumer_sync();
             // 3. weight records from the ring: in each stage, warp w takes the
-            //    contiguous records [w n / 16, (w + 1) n / 16).  The B fragments
-            //    (8 token rows x 64 k of int8) come from shared memory with one
-            //    ldmatrix.x4 per record: lane l gives the address of row l % 8
-            //    of matrix l / 8 (a 16-byte segment; rows >= T read zeros).
-            const uint32_t lrow = lane & 7, lmat = lane >> 3;
-            const uint32_t b_base = lrow < static_cast<uint32_t>(T)
-                                        ? smem_u32(s_xq) + lrow * static_cast<uint32_t>(op.k + 16) + 16u * lmat
-                                        : smem_u32(s_zero) + 16u * lmat;
-            const uint32_t b_step = lrow < static_cast<uint32_t>(T) ? 64u : 0u;   // bytes per k-tile
+            //    contiguous records [w n / 16, (w + 1) n / 16).  Lane l holds the
+            //    B fragment of token l / 4 (zero for tokens >= T): the 16 bytes
+            //    lane l % 4 needs of each 64-k tile sit contiguously in the
+            //    shared row (fragment order), one 16-byte load per record.
+            const int bn = lane >> 2;
+            const bool has_b = bn < T;
+            const uint4 *b_src =
+                reinterpret_cast<const uint4 *>(s_xq + static_cast<int64_t>(has_b ? bn : 0) * chain_pitch(op.k)) +
+                (lane & 3);
             int cur = -1;
             int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
             bool failed = false;
@@ -492,7 +500,13 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
 #pragma unroll
                             for (int u = 0; u < 4; ++u) w[u] = rec[(i + u) * 32];
 #pragma unroll
-                            for (int u = 0; u < 4; ++u) ldsm_x4(bf[u], b_base + static_cast<uint32_t>(kt + u) * b_step);
+                            for (int u = 0; u < 4; ++u) {
+                                const uint4 v = has_b ? b_src[(kt + u) * 4] : make_uint4(0u, 0u, 0u, 0u);
+                                bf[u][0] = v.x;
+                                bf[u][1] = v.y;
+                                bf[u][2] = v.z;
+                                bf[u][3] = v.w;
+                            }
 #pragma unroll
                             for (int u = 0; u < 4; ++u) {
                                 uint32_t a4[4];
@@ -505,7 +519,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                         } else {
                             const uint2 w = rec[i * 32];
                             uint32_t bf[4], a4[4];
-                            ldsm_x4(bf, b_base + static_cast<uint32_t>(kt) * b_step);
+                            const uint4 v = has_b ? b_src[kt * 4] : make_uint4(0u, 0u, 0u, 0u);
+                            bf[0] = v.x;
+                            bf[1] = v.y;
+                            bf[2] = v.z;
+                            bf[3] = v.w;
 #pragma unroll
                             for (int r = 0; r < 4; ++r) a4[r] = expand_codes(w.x, r);
                             mma_sp_m16n8k64(acc[0], a4, bf, w.y);
@@ -544,7 +562,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                 if (op.xq_out) {
                     for (int i = ctid; i < T * op.k; i += kChainConsumers) {
                         const int t = i / op.k;
-                        op.xq_out[i] = s_xq[t * (op.k + 16) + (i - t * op.k)];
+                        const int e = i - t * op.k, u = (e & 63) >> 2;   // undo the fragment order
+                        op.xq_out[i] = s_xq[t * chain_pitch(op.k) + (e & ~63) + 4 * (4 * (u & 3) + (u >> 2)) + (e & 3)];
                     }
                 }
                 if (op.amax_out && ctid < T) op.amax_out[ctid] = s_amax[ctid];
@@ -564,7 +583,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
 
 size_t chain_smem_bytes(int ns, uint32_t stage_bytes, int64_t T, int64_t kmax) {
     return static_cast<size_t>(ns) * stage_bytes + static_cast<size_t>(kChainMaxTiles) * 128 * 4 +
-           static_cast<size_t>(T) * static_cast<size_t>(kmax + 16) + 64;
+           static_cast<size_t>(T) * static_cast<size_t>(kmax + 128);
 }
 
 // Ring geometry: the largest stage (64, 32 or 16 KB) that leaves three stages
