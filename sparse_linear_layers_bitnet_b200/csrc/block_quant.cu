@@ -505,6 +505,38 @@ __device__ __forceinline__ float swiglu1(float g, float u) {
     return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, exp32(-g))), u);
 }
 
+// exp32 of two values at once with the paired fp32 add and multiply of
+// sm_100, which round each component exactly as the scalar __fadd_rn and
+// __fmul_rn do: the same operations in the same order, so the results equal
+// exp32's bit for bit.  A subtraction a - b is the addition a + fp32(n (-c))
+// with the constant negated, which rounds to the same value.
+__device__ __forceinline__ float2 exp32x2(float2 x) {
+    x.x = fminf(fmaxf(x.x, -87.0f), 88.0f);
+    x.y = fminf(fmaxf(x.y, -87.0f), 88.0f);
+    const float l2e = __uint_as_float(0x3fb8aa3bu), hi = __uint_as_float(0xbf317200u), lo = __uint_as_float(0xb5bfbe8eu);
+    const float2 big = __fadd2_rn(__fmul2_rn(x, make_float2(l2e, l2e)), make_float2(12582912.0f, 12582912.0f));
+    const float2 n = __fadd2_rn(big, make_float2(-12582912.0f, -12582912.0f));
+    const int n0 = __float_as_int(big.x) - 0x4b400000, n1 = __float_as_int(big.y) - 0x4b400000;
+    float2 r = __fadd2_rn(x, __fmul2_rn(n, make_float2(hi, hi)));
+    r = __fadd2_rn(r, __fmul2_rn(n, make_float2(lo, lo)));
+    const float c5 = __uint_as_float(0x3ab60b61u), c4 = __uint_as_float(0x3c088889u), c3 = __uint_as_float(0x3d2aaaabu),
+                c2 = __uint_as_float(0x3e2aaaabu);
+    float2 p = make_float2(c5, c5);
+    p = __fadd2_rn(__fmul2_rn(p, r), make_float2(c4, c4));
+    p = __fadd2_rn(__fmul2_rn(p, r), make_float2(c3, c3));
+    p = __fadd2_rn(__fmul2_rn(p, r), make_float2(c2, c2));
+    p = __fadd2_rn(__fmul2_rn(p, r), make_float2(0.5f, 0.5f));
+    p = __fadd2_rn(__fmul2_rn(p, r), make_float2(1.0f, 1.0f));
+    p = __fadd2_rn(__fmul2_rn(p, r), make_float2(1.0f, 1.0f));
+    return __fmul2_rn(p, make_float2(__int_as_float((n0 + 127) << 23), __int_as_float((n1 + 127) << 23)));
+}
+
+// swiglu1 of two (g, u) pairs; the divisions stay scalar IEEE divisions
+__device__ __forceinline__ float2 swiglu2(float2 g, float2 u) {
+    const float2 d = __fadd2_rn(make_float2(1.0f, 1.0f), exp32x2(make_float2(-g.x, -g.y)));
+    return __fmul2_rn(make_float2(__fdiv_rn(g.x, d.x), __fdiv_rn(g.y, d.y)), u);
+}
+
 // h goes to shared memory (F fp32) between the absmax and the codes; the raw
 // gate and up chunks stay in registers only until h is formed.
 template <int CPT>
@@ -534,9 +566,11 @@ __global__ void __launch_bounds__(256) k_swiglu_quant_rc(const uint4 *__restrict
             chunk_f32(gv[j], g);
             chunk_f32(uv[j], u);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                h[e] = swiglu1(g[e], u[e]);
-                m = fmaxf(m, fabsf(h[e]));
+            for (int e = 0; e < 8; e += 2) {
+                const float2 hp = swiglu2(make_float2(g[e], g[e + 1]), make_float2(u[e], u[e + 1]));
+                h[e] = hp.x;
+                h[e + 1] = hp.y;
+                m = fmaxf(m, fmaxf(fabsf(hp.x), fabsf(hp.y)));
             }
             s_h4[2 * c] = make_float4(h[0], h[1], h[2], h[3]);
             s_h4[2 * c + 1] = make_float4(h[4], h[5], h[6], h[7]);
