@@ -805,10 +805,12 @@ def test_gemm_pair_kernel_ragged(bn, n_out, k, T):
     _check_outputs(ref, acc, Y)
 
 
-@pytest.mark.parametrize("n_out,k,T", [(4096, 256, 896), (2048, 256, 1344), (256, 512, 160)])
+@pytest.mark.parametrize("n_out,k,T", [(4096, 256, 896), (2048, 256, 1344), (256, 512, 160), (3200, 320, 2048),
+                                       (1040, 448, 700)])
 def test_gemm_pair_tile_widths(bn, n_out, k, T):
-    """Larger pair-kernel shapes: many 256 x 224 tiles per CTA pair, ragged
-    last token tile."""
+    """Larger pair-kernel shapes: many tiles per CTA pair and a ragged last
+    token tile, at both token-tile widths (224 for T = 896, 1344; 192 for
+    T = 160, 700, 2048, where it leaves fewer padded columns)."""
     ref, acc, Y = _linear_case(bn, n_out, k, T, seed=n_out + T, y_dtype="bf16")
     _check_outputs(ref, acc, Y)
 
