@@ -17,7 +17,8 @@ def test_decode_step_bytes():
     """A fused projection moves its bf16 activations in, its packed weights at
     2 bits per weight, gamma and its bf16 outputs.  For the 2B shapes
     (hidden 2560, FFN 6912) at T = 1 a layer is 69.47 M weights = 17.37 MB of
-    codes plus 72.7 KB of activations: 17,441,808 bytes, 523,254,240 for the
+    codes plus 74.8 KB of bf16 activations in and out and the gammas:
+    17,441,808 bytes, 523,254,240 for the
     30-layer step the benchmark times."""
     mats = synth.DECODE_2B_MATRICES
     assert sum(N * K for _, K, N in mats) == 69_468_160
