@@ -502,12 +502,15 @@ bitnet_status bitnet_dgrad(const void *dY, bitnet_dtype dy_dtype, const bitnet_p
  * GPU that loads the library until the process exits.  Everything else is as
  * in bitnet_pack_nm, with bit-identical results.
  *
- *   Limit: n_out * k <= 2^40 weights (the exactness bound of the fixed
- *          scratch's 64-bit exponent bins); larger matrices are rejected with
- *          BITNET_ERR_UNSUPPORTED.
+ *   Limit: n_out * k <= 2^34 weights (2^32 groups of 4, the bound of the
+ *          pack's group indexing); larger matrices are rejected with
+ *          BITNET_ERR_UNSUPPORTED before any pointer is touched.
  *   First call on a device looks up the array's device address with
  *          cudaGetSymbolAddress (once per device, with that device current);
- *          make that first call before any stream capture.
+ *          make that first call before any stream capture.  The address is
+ *          kept with the identity of the device's context: after a
+ *          cudaDeviceReset the next call looks it up again (make that call
+ *          outside stream capture too).
  *   Sharing: every call reuses the same array and clears it first; calls whose
  *          kernels overlap on the GPU (other streams, other host threads on the
  *          same device) race on it - serialise them on one stream.

@@ -68,8 +68,6 @@ def _load():
     lib.oracle_gemm_i32.argtypes = [P, P, I64, I64, I64, P]
     lib.oracle_dequant.restype = None
     lib.oracle_dequant.argtypes = [P, P, F, I64, I64, P]
-    lib.oracle_dequant_f64.restype = None
-    lib.oracle_dequant_f64.argtypes = [P, P, F, I64, I64, P]
     lib.oracle_dgrad.restype = None
     lib.oracle_dgrad.argtypes = [P, P, F, I64, I64, I64, P, P]
     lib.oracle_set_threads.restype = None
@@ -178,15 +176,6 @@ def dequant(acc: np.ndarray, a: np.ndarray, g: float) -> np.ndarray:
     T, N = acc.shape
     Y = np.empty((T, N), np.float32)
     _load().oracle_dequant(_p(acc), _p(a), np.float32(g), T, N, _p(Y))
-    return Y
-
-
-def dequant_f64(acc: np.ndarray, a: np.ndarray, g: float) -> np.ndarray:
-    acc = np.ascontiguousarray(acc, dtype=np.int32)
-    a = np.ascontiguousarray(a, dtype=np.float32)
-    T, N = acc.shape
-    Y = np.empty((T, N), np.float64)
-    _load().oracle_dequant_f64(_p(acc), _p(a), np.float32(g), T, N, _p(Y))
     return Y
 
 

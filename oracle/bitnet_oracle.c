@@ -266,13 +266,6 @@ void oracle_dequant(const int32_t *acc, const float *a, float gamma, int64_t T, 
     }
 }
 
-/* Same output in fp64 arithmetic from the same integers, for reporting. */
-void oracle_dequant_f64(const int32_t *acc, const float *a, float gamma, int64_t T, int64_t N, double *Y) {
-    for (int64_t t = 0; t < T; ++t)
-        for (int64_t n = 0; n < N; ++n)
-            Y[t * N + n] = (double)acc[t * N + n] * ((double)gamma * (double)a[t] / 127.0);
-}
-
 /* ------------------------------------------------------------------------ */
 /* Input gradient under the straight-through estimator.  [P4] "Training      */
 /* Strategie" (dual STE): the quantiser and the mask pass the gradient       */

@@ -661,12 +661,9 @@ size_t swiglu_smem_bytes(int64_t F) { return static_cast<size_t>(F) * 4; }
 template <int CPT>
 static cudaError_t swi_rc(cudaLaunchConfig_t &cfg, const void *G, const void *U, int64_t ld, int64_t F, float eps_a,
                           int8_t *Xq, float *amax) {
-    static bool attr_done = false;   // per instantiation
-    if (!attr_done) {
-        cudaError_t e = cudaFuncSetAttribute(k_swiglu_quant_rc<CPT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(kSwigluMaxSmem));
+    {
+        cudaError_t e = smem_attr(reinterpret_cast<const void *>(k_swiglu_quant_rc<CPT>), static_cast<int>(kSwigluMaxSmem));
         if (e != cudaSuccess) return e;
-        attr_done = true;
     }
     return cudaLaunchKernelEx(&cfg, k_swiglu_quant_rc<CPT>, static_cast<const uint4 *>(G), static_cast<const uint4 *>(U),
                               ld / 8, static_cast<int>(F), eps_a, Xq, amax);
@@ -680,12 +677,9 @@ cudaError_t launch_swiglu_quant(const void *G, const void *U, int64_t ld, int64_
     const bool vec = !(reinterpret_cast<uintptr_t>(G) & 15u) && !(reinterpret_cast<uintptr_t>(U) & 15u) && ld % 8 == 0;
     const int cpt = vec ? pick_cpt(F / 8, kSwiCpt, 6, 256, &threads) : 0;
     if (cpt == 0) {   // rows beyond the register cache, or rows without 16-byte alignment
-        static bool attr_done = false;
-        if (!attr_done) {
-            cudaError_t e = cudaFuncSetAttribute(k_swiglu_quant, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(kSwigluMaxSmem));
+        {
+            cudaError_t e = smem_attr(reinterpret_cast<const void *>(k_swiglu_quant), static_cast<int>(kSwigluMaxSmem));
             if (e != cudaSuccess) return e;
-            attr_done = true;
         }
         cudaLaunchConfig_t cfg = bq_config(T, kBqThreads, swiglu_smem_bytes(F), s, attr);
         return cudaLaunchKernelEx(&cfg, k_swiglu_quant, static_cast<const uint16_t *>(G),

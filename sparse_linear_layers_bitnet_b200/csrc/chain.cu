@@ -627,12 +627,9 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
     const bool one = T == 1;
     auto kern = x_bf16 ? (one ? k_decode_chain<true, 1> : k_decode_chain<true, 8>)
                        : (one ? k_decode_chain<false, 1> : k_decode_chain<false, 8>);
-    static bool attr_done[2][2] = {{false, false}, {false, false}};
-    if (!attr_done[x_bf16 ? 1 : 0][one ? 1 : 0]) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(kChainMaxSmem));
+    {
+        cudaError_t e = smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(kChainMaxSmem));
         if (e != cudaSuccess) return e;
-        attr_done[x_bf16 ? 1 : 0][one ? 1 : 0] = true;
     }
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     for (int base = 0; base < n_ops; base += kChainMaxOps) {

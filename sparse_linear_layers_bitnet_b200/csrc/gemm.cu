@@ -304,11 +304,9 @@ template <bool SPARSE, int BN, int STAGES>
 static cudaError_t run_gemm(const CUtensorMap &a, const CUtensorMap &b, const GemmParams &p, cudaStream_t s) {
     using C = GemmCfg<SPARSE, BN, STAGES>;
     auto kern = k_umma_gemm<SPARSE, BN, STAGES>;
-    static bool attr_set = false;   // per instantiation
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    {
+        cudaError_t e = smem_attr(reinterpret_cast<const void *>(kern), C::kSmemBytes);
         if (e != cudaSuccess) return e;
-        attr_set = true;
     }
     dim3 grid(static_cast<unsigned>((p.M + C::kBM - 1) / C::kBM), static_cast<unsigned>((p.N + BN - 1) / BN));
     kern<<<grid, 192, C::kSmemBytes, s>>>(a, b, p);

@@ -503,11 +503,9 @@ static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CU
                             const PairParams &p, cudaStream_t s) {
     using C = PairCfg<SPARSE, BN, STAGES, MN>;
     auto kern = k_umma_pair<SPARSE, BN, STAGES, MN>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    {
+        cudaError_t err = smem_attr(reinterpret_cast<const void *>(kern), C::kSmemBytes);
         if (err != cudaSuccess) return err;
-        attr_set = true;
     }
     const int64_t tiles = ((p.M + 255) / 256) * ((p.N + BN - 1) / BN);
     int64_t pairs = num_sms() / 2;

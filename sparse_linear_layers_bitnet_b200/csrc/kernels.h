@@ -26,6 +26,8 @@ constexpr size_t kLinearWsBytes = 256;
 constexpr size_t kDgradWsHeader = 256;
 
 int num_sms();
+// Raises func's dynamic shared-memory limit on the current device (once per device and function).
+cudaError_t smem_attr(const void *func, int bytes);
 
 // Sets the message bitnet_last_error() returns on this thread.
 void set_last_error(const char *msg);

@@ -23,6 +23,10 @@
 // Pass 2 (k_pack24) reads each group of 4 weights once (one float4 per
 // thread, coalesced), ranks the magnitudes (ties to the lower position) and
 // writes every requested layout.
+#include <atomic>
+#include <mutex>
+#include <vector>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -1187,15 +1191,54 @@ __global__ void __launch_bounds__(256) k_make_dec(const uint8_t *__restrict__ gb
 
 // ---------------------------------------------------------------- host side
 
+// SM count of the current device, looked up once per device (a process may
+// drive several GPUs; each keeps its own entry).
 int num_sms() {
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (sms <= 0) sms = 148;
+    constexpr int kMaxDev = 64;
+    static std::atomic<int> sms[kMaxDev];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= kMaxDev) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        return n > 0 ? n : 148;
     }
-    return sms;
+    int n = sms[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+        sms[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+// Raises a kernel's dynamic shared-memory limit to bytes on the current
+// device.  The attribute belongs to the function in one device's context, so
+// the record of what was set is kept per (device, function); a second device
+// in the same process gets its own call.
+cudaError_t smem_attr(const void *func, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    struct Entry {
+        int dev;
+        const void *func;
+        int bytes;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> done;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry &d : done)
+        if (d.dev == dev && d.func == func && d.bytes >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    for (Entry &d : done)
+        if (d.dev == dev && d.func == func) {
+            d.bytes = bytes;
+            return cudaSuccess;
+        }
+    done.push_back(Entry{dev, func, bytes});
+    return cudaSuccess;
 }
 
 static unsigned grid_for(int64_t work, int threads, int per_sm) {

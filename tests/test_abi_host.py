@@ -99,6 +99,13 @@ def test_pack_rejects_bad_arguments(lib):
     assert b"required" in lib.bitnet_last_error() or b"derived" in lib.bitnet_last_error()
 
 
+def test_pack_noalloc_rejects_oversized_matrix_on_host(lib):
+    # between the 2^34-weight limit and 2^40: refused before any device call
+    bad = _pw(n_out=1 << 18, k=1 << 17)
+    assert lib.bitnet_pack_nm_noalloc(_fake(), ctypes.byref(bad), 1e-5, None, None) == _abi.BITNET_ERR_UNSUPPORTED
+    assert b"2^34" in lib.bitnet_last_error()
+
+
 def test_quant_rejects_bad_arguments(lib):
     f = lib.bitnet_quant_act
     assert f(None, 0, 4, 256, 1e-5, _fake(), _fake(), None) == _abi.BITNET_ERR_INVALID_ARG

@@ -191,6 +191,24 @@ def test_pack_round_trip_and_invariants():
 
 # ---------------------------------------------------------------- golden forward
 
+def test_apply_mask_zeroes_exactly_the_dropped_entries():
+    # hand example: codes of every sign, a kept zero code and dropped non-zero codes
+    wt = np.array([[1, -1, 0, 1, -1, -1, 1, 0]], np.int8)
+    keep = np.array([[1, 0, 1, 0, 0, 1, 1, 0]], np.uint8)
+    assert oracle.apply_mask(wt, keep).tolist() == [[1, 0, 0, 0, 0, -1, 1, 0]]
+
+
+def test_bf16_widening_known_bit_patterns():
+    # bf16 is the top half of the fp32 pattern: values fixed by the IEEE format
+    u = np.array([0x3F80, 0xC000, 0x0000, 0x8000, 0x0001, 0x7F7F, 0x3EAB], np.uint16)
+    got = oracle.bf16_to_f32(u)
+    assert got[0] == 1.0 and got[1] == -2.0 and got[2] == 0.0
+    assert got[3] == 0.0 and np.signbit(got[3])
+    assert got[4] == np.float32(2.0 ** -133)                           # smallest bf16 subnormal
+    assert got[5] == np.float32((2 - 2.0 ** -7) * 2.0 ** 127)          # largest finite bf16
+    assert got[6] == np.float32((1 + 0x2B / 128) * 2.0 ** -2)          # 0.333984375
+
+
 def test_worked_example():
     G = load_golden("worked_2x8.txt")
     f = lambda k: np.array([float(v) for v in G[k]], np.float32)

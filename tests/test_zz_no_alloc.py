@@ -68,9 +68,11 @@ def test_noalloc_pack_matches_workspace_pack_twice(cuda_device):
 def test_noalloc_rejects_oversized_matrix(cuda_device):
     import sparse_linear_layers_bitnet_b200 as bn
     lib = bn.load()
-    st = bn.BitnetPackedW()
-    st.n_out, st.k, st.n, st.m = 1 << 21, 1 << 20, 2, 4
-    st.gamma = 4096
-    rc = lib.bitnet_pack_nm_noalloc(ctypes.c_void_p(4096), ctypes.byref(st), ctypes.c_float(1e-5), None, None)
-    assert rc == bn._abi.BITNET_ERR_UNSUPPORTED
-    assert b"2^40" in lib.bitnet_last_error()
+    # 2^35 weights (just above the 2^34 limit) and 2^41: both refused before any pointer is used
+    for n_out, k in ((1 << 18, 1 << 17), (1 << 21, 1 << 20)):
+        st = bn.BitnetPackedW()
+        st.n_out, st.k, st.n, st.m = n_out, k, 2, 4
+        st.gamma = 4096
+        rc = lib.bitnet_pack_nm_noalloc(ctypes.c_void_p(4096), ctypes.byref(st), ctypes.c_float(1e-5), None, None)
+        assert rc == bn._abi.BITNET_ERR_UNSUPPORTED
+        assert b"2^34" in lib.bitnet_last_error()
