@@ -31,6 +31,7 @@ import hashlib
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -62,7 +63,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--pack-layers", type=int, default=None, help="layers of the pack workload (default: all 26)")
     ap.add_argument("--flip-steps", type=int, default=100, help="random-walk steps of the mask flip-rate study")
-    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks", "six_eight", "block", "optimizer"], default=None,
+    ap.add_argument("--only", choices=["prefill", "pack", "dgrad", "peaks", "six_eight", "block", "optimizer",
+                                       "decode_rows", "oracle"], default=None,
                     help="run one sub-measurement alone and print it (for profiling)")
     return ap.parse_args()
 
@@ -410,6 +412,41 @@ def measure_library_peaks(torch, n=8192, reps=10):
     out["how"] = f"{n}^3, best of {reps}, CUDA events; int8: torch._int_mm (cuBLASLt), bf16: torch.matmul"
     del a, b
     torch.cuda.empty_cache()
+    return out
+
+
+def measure_mma_ceilings(torch, bn, secs=1.0, iters=20000):
+    """Ceiling of each tensor-core instruction form the GEMMs issue, on this GPU:
+    bitnet_tensor_peak (MMAs back to back on operands resident in shared memory,
+    no loads, no epilogue), launches timed with CUDA events for about `secs`,
+    SM clocks sampled meanwhile.  Dense-equivalent rates (2 M N K per MMA)."""
+    dev_index = torch.cuda.current_device()
+    dev = torch.device("cuda", dev_index)
+    ws = bn.Workspace(bn.load().bitnet_linear_workspace_size(), dev)
+    out = {}
+    forms = ((0, "sparse_i8_mma_loop_tops", "tcgen05.mma.sp.cta_group::2.kind::i8 M256 N224 K64"),
+             (1, "dense_i8_mma_loop_tops", "tcgen05.mma.cta_group::2.kind::i8 M256 N256 K32"),
+             (2, "bf16_mma_loop_tflops", "tcgen05.mma.cta_group::2.kind::f16 (bf16) M256 N256 K16"))
+    for kind, name, form in forms:
+        for _ in range(3):
+            bn.bitnet_tensor_peak(kind, iters, ws)
+        torch.cuda.synchronize()
+        ck = ClockSampler(dev_index).start()
+        ts, ops = [], 0.0
+        t_end = time.time() + secs
+        while time.time() < t_end:
+            with Timer(torch) as t:
+                ops = bn.bitnet_tensor_peak(kind, iters, ws)
+            ts.append(t.ms())
+        c = ck.stop()
+        status = bn.bitnet_read_device_status(ws)
+        med = ops / (statistics.median(ts) / 1e3) / 1e12
+        out[name] = round(ops / (min(ts) / 1e3) / 1e12, 1)
+        out[name + "_median"] = round(med, 1)
+        out[name + "_per_sm_mhz"] = round(med / c["sm_mhz"], 4) if c.get("sm_mhz") else None
+        out[name + "_clocks"] = c
+        out[name + "_form"] = f"{form}; {iters} MMAs per CTA pair per launch, {len(ts)} launches, status {status}"
+    del ws
     return out
 
 
@@ -915,6 +952,100 @@ def oracle_decode_sample(T, target_s):
     return bytes_layer, reps, t_total, oracle.max_threads(), prepared
 
 
+def _cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def measure_oracle(target_s=1.5):
+    """The CPU oracle, as it stands, on bounded samples of every configuration,
+    single-threaded and on all host cores (OpenMP): the reported CPU baseline.
+    Units follow the GPU rows: ms per forward (config 1), GB/s of algorithmic
+    bytes (configs 2 and 4), dense-equivalent TOPS (config 3), ms per block step
+    extrapolated from a token sample (config 5)."""
+    import numpy as np
+
+    import oracle
+    from sparse_linear_layers_bitnet_b200 import synth
+
+    def timed(fn):
+        reps, t = 0, 0.0
+        while t < target_s or reps == 0:
+            t0 = time.perf_counter()
+            fn()
+            t += time.perf_counter() - t0
+            reps += 1
+        return t / reps
+
+    cores = oracle.max_threads()
+    out = {"nproc": os.cpu_count(), "cpu_model": _cpu_model(), "omp_threads_all": cores}
+    # inputs (built once, outside the timed regions)
+    W1, X1 = synth.master_weights(256, 256, 0.02, seed=0), synth.activations(16, 256, seed=0)
+    dec = []
+    for j, (name, K, N) in enumerate(decode_shapes()):
+        g, keep, wq, gb = oracle.pack_weights(synth.master_weights(N, K, 0.02, seed=j), 1e-5)
+        dec.append((g, wq, synth.bf16_bits_to_f32(synth.to_bf16_bits(synth.activations(1, K, seed=100 + j)))))
+    dec_bytes = sum(decode_bytes_fused(1, K, N) for _, K, N in decode_shapes())
+    Ts = 8   # prefill token sample
+    pre = []
+    for name, T, K, N in synth.PREFILL_7B_GEMMS:
+        g, keep, wq, gb = oracle.pack_weights(synth.master_weights(N, K, 0.02, seed=11), 1e-5)
+        pre.append((g, wq, synth.activations(Ts, K, seed=12, outlier_p=0.01), K, N))
+    Wp = synth.master_weights(3200, 3200, 0.02, seed=21)
+    Tb = 4   # block token sample
+    blk = []
+    for name, K, N in (("qkv", 3200, 9600), ("o", 3200, 3200), ("gate_up", 3200, 17280), ("down", 8640, 3200)):
+        g, keep, wq, gb = oracle.pack_weights(synth.master_weights(N, K, 0.02, seed=31), 1e-5)
+        blk.append((g, wq, synth.activations(Tb, K, seed=32), synth.activations(Tb, N, seed=33), K, N))
+
+    def c1():
+        oracle.forward(W1, X1)
+
+    def c2():
+        for g, wq, X in dec:
+            xq, a = oracle.quant_act(X, 1e-5)
+            oracle.dequant(oracle.gemm_i32(xq, wq), a, g)
+
+    def c3():
+        for g, wq, X, K, N in pre:
+            xq, a = oracle.quant_act(X, 1e-5)
+            oracle.dequant(oracle.gemm_i32(xq, wq), a, g)
+
+    def c4():
+        oracle.pack_weights(Wp, 1e-5)
+
+    def c5():
+        for g, wq, X, dY, K, N in blk:
+            xq, a = oracle.quant_act(X, 1e-5)
+            oracle.dequant(oracle.gemm_i32(xq, wq), a, g)
+            oracle.dgrad(dY, wq, g)
+
+    pre_ops = sum(2.0 * Ts * K * N for _, _, _, K, N in pre)
+    for threads in (1, cores):
+        oracle.set_threads(threads)
+        key = f"threads_{threads}"
+        out[key] = {
+            "config1_tiny_ms_per_forward": round(timed(c1) * 1e3, 4),
+            "config2_decode_gbs": round(dec_bytes / timed(c2) / 1e9, 4),
+            "config3_prefill_tops": round(pre_ops / timed(c3) / 1e12, 5),
+            "config4_pack_gbs": round(Wp.size * 4.875 / timed(c4) / 1e9, 4),
+            "config5_block_ms_per_step": round(timed(c5) * 2048 / Tb * 1e3, 1),
+        }
+    oracle.set_threads(cores)
+    out["samples"] = ("config 1: one tiny forward (16 x 256 x 256); config 2: one 2B layer (4 projections) at "
+                      "T = 1, bf16-valued activations; config 3: both 7B prefill GEMMs (quant, int32 product, "
+                      f"dequant) on {Ts} of the 4096 tokens; config 4: pack of one 3200 x 3200 fp32 matrix "
+                      f"(4.875 B per weight); config 5: forward and STE dgrad of the 3B block's four "
+                      f"projections on {Tb} of 2048 tokens, scaled to 2048")
+    return out
+
+
 def run_reference(args):
     """--impl reference: the CPU oracle on the host cores (rank 0 only)."""
     from sparse_linear_layers_bitnet_b200 import dist
@@ -939,7 +1070,7 @@ def run_reference(args):
         one_step()
     dt = time.perf_counter() - t0
     value = bytes_layer * args.steps / dt / 1e9
-    threads = 1 if T == 1 else min(T, cores)
+    threads = cores
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
@@ -967,12 +1098,35 @@ def run_only(args):
     bn.load()
     peaks = load_peaks()
     fn = {"prefill": measure_prefill, "pack": measure_pack, "dgrad": measure_dgrad,
-          "peaks": lambda torch, bn, synth, peaks: measure_library_peaks(torch),
+          "peaks": lambda torch, bn, synth, peaks: {**measure_library_peaks(torch), **measure_mma_ceilings(torch, bn)},
+          "decode_rows": lambda torch, bn, synth, peaks: measure_decode_rows(torch, bn, synth, args.layers),
+          "oracle": lambda torch, bn, synth, peaks: measure_oracle(),
           "six_eight": lambda torch, bn, synth, peaks: measure_6of8(torch, bn, synth),
           "block": measure_block, "optimizer": measure_optimizer}[args.only]
     kw = {"steps": args.steps, "flip_steps": args.flip_steps, "layers": args.pack_layers} if args.only == "pack" else {}
     print(json.dumps({args.only: fn(torch, bn, synth, peaks, **kw)}), flush=True)
     return 0
+
+
+def measure_decode_rows(torch, bn, synth, layers):
+    """The decode step in its other forms: independent and dependent chains at
+    T = 1, 4, 8, and the fused and unfused per-projection launches."""
+    out = {}
+    for t2, mode in ((1, "chain_independent"), (1, "chain"), (1, "unfused"), (1, "fused"), (4, "chain_independent"),
+                     (4, "chain"), (4, "unfused"), (8, "chain_independent"), (8, "chain"), (8, "unfused")):
+        d2 = Decode(torch, bn, synth, t2, layers, seed_base=31, mode=mode)
+        g2 = d2.capture(d2.step)
+        for _ in range(3):
+            g2.replay()
+        with Timer(torch) as t:
+            for _ in range(10):
+                g2.replay()
+        per = t.ms() / 10
+        out[f"T{t2}_{mode}"] = {"gbs": round(d2.step_bytes / (per / 1e3) / 1e9, 1), "ms_per_step": round(per, 4),
+                                "launches_per_step": d2.launches_per_step}
+        del g2, d2
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args):
@@ -1059,30 +1213,18 @@ def run_ours(args):
 
     rows = {}
     if not args.no_rows and info.world == 1:
-        rows["decode_batches"] = {}
-        for t2, mode in ((1, "chain_independent"), (1, "unfused"), (1, "fused"), (4, "chain"), (4, "unfused"),
-                         (8, "chain"), (8, "unfused")):
-            d2 = Decode(torch, bn, synth, t2, args.layers, seed_base=31, mode=mode)
-            g2 = d2.capture(d2.step)
-            for _ in range(3):
-                g2.replay()
-            with Timer(torch) as t:
-                for _ in range(10):
-                    g2.replay()
-            per = t.ms() / 10
-            rows["decode_batches"][f"T{t2}_{mode}"] = {
-                "gbs": round(d2.step_bytes / (per / 1e3) / 1e9, 1), "ms_per_step": round(per, 4),
-                "launches_per_step": d2.launches_per_step}
-            del g2, d2
-            torch.cuda.empty_cache()
+        rows["decode_batches"] = measure_decode_rows(torch, bn, synth, args.layers)
         with Nvtx(torch, "row library_peaks"):
             rows["library_peaks"] = measure_library_peaks(torch)
+            rows["library_peaks"].update(measure_mma_ceilings(torch, bn))
         with Nvtx(torch, "row prefill_gemm"):
             rows["prefill_gemm"] = measure_prefill(torch, bn, synth, peaks)
         lp = rows["library_peaks"]["int8_dense_tops"]
         pc = rows["prefill_gemm"]["combined"]
         pc["frac_of_2x_measured_int8_dense"] = round(pc["tops"] / (2 * lp), 4)
         pc["frac_of_measured_int8_dense"] = round(pc["tops"] / lp, 4)
+        sp = rows["library_peaks"]["sparse_i8_mma_loop_tops_median"]
+        pc["frac_of_measured_sparse_i8_mma_loop"] = round(pc["tops"] / sp, 4)
         with Nvtx(torch, "row dgrad"):
             rows["dgrad"] = measure_dgrad(torch, bn, synth, peaks)
         with Nvtx(torch, "row six_eight"):
@@ -1093,6 +1235,7 @@ def run_ours(args):
             rows["pack"] = measure_pack(torch, bn, synth, peaks, flip_steps=args.flip_steps)
         with Nvtx(torch, "row optimizer"):
             rows["optimizer"] = measure_optimizer(torch, bn, synth, peaks)
+        rows["oracle"] = measure_oracle()
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": info.world, "steps": args.steps,
@@ -1121,10 +1264,18 @@ def run_ours(args):
         "clocks": ck,
     }
     if info.rank == 0 and info.world == 1:
-        b, reps, secs, cores, _ = oracle_decode_sample(T, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": round(b * reps / secs / 1e9, 4), "unit": "GB/s",
-                                "cores": 1 if T == 1 else min(T, cores), "kind": "oracle",
-                                "sample": f"{reps} passes over one 2B layer (4 projections), T={T}, {secs:.1f} s"}
+        import oracle
+        cores = oracle.max_threads()
+        oracle.set_threads(1)
+        b1, reps1, secs1, _, _ = oracle_decode_sample(T, args.cpu_seconds / 2)
+        oracle.set_threads(cores)
+        b, reps, secs, _, _ = oracle_decode_sample(T, args.cpu_seconds / 2)
+        line["cpu_baseline"] = {"value": round(b * reps / secs / 1e9, 4), "unit": "GB/s", "cores": cores,
+                                "kind": "oracle", "value_1_thread": round(b1 * reps1 / secs1 / 1e9, 4),
+                                "cpu_model": _cpu_model(), "nproc": os.cpu_count(),
+                                "sample": f"{reps} passes over one 2B layer (4 projections), T={T}, {secs:.1f} s on "
+                                          f"{cores} threads (OpenMP over outputs); {reps1} passes, {secs1:.1f} s "
+                                          f"on 1 thread"}
     if rows:
         line["rows"] = rows
     if info.rank == 0:

@@ -538,6 +538,30 @@ bitnet_status bitnet_pack_nm_noalloc(const float *W, bitnet_packed_w *out, float
 bitnet_status bitnet_wait_selftest(void *ws, size_t ws_bytes, int32_t limit_us, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * bitnet_tensor_peak - throughput ceiling of a tensor-core instruction form.
+ *
+ * No counterpart in the paper: it measures the denominator of the GEMMs'
+ * roofline on the GPU that runs them.  "Is 2:4 Sparsity Still Worth It?"
+ * (SlideSparse entry) bounds the gain of 2:4 by twice the dense rate, which a
+ * given device need not deliver for a given instruction; this call measures
+ * what it delivers.  One CTA pair per two SMs issues MMAs back to back on
+ * operands resident in shared memory (no loads, no epilogue):
+ *   kind 0  tcgen05.mma.sp.cta_group::2.kind::i8, M 256, N 224, K 64 (the
+ *           2:4-sparse int8 instruction of the prefill GEMM);
+ *   kind 1  tcgen05.mma.cta_group::2.kind::i8, M 256, N 256, K 32 (dense int8);
+ *   kind 2  tcgen05.mma.cta_group::2.kind::f16 (bf16), M 256, N 256, K 16.
+ *   iters   MMAs per CTA pair (rounded up to a whole stage), >= 1.
+ *   ops     host pointer; receives the dense-equivalent operations of the
+ *           launch, 2 M N K per MMA summed over the pairs (time the launch on
+ *           the stream with events; ops / seconds is the ceiling).
+ *   ws      >= bitnet_linear_workspace_size() bytes, 16-byte aligned: status
+ *           word of the bounded wait for the tensor pipe to drain.
+ * Errors: INVALID_ARG, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------ */
+bitnet_status bitnet_tensor_peak(int32_t kind, int64_t iters, double *ops, void *ws, size_t ws_bytes,
+                                 bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Status helpers.
  * bitnet_read_device_status synchronises `stream`, reads the status word that
  * the kernels of the last call on `ws` left (BITNET_OK or BITNET_ERR_TIMEOUT

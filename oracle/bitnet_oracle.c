@@ -246,7 +246,8 @@ void oracle_quant_act(const float *X, int64_t T, int64_t K, float eps, int8_t *X
 
 int oracle_gemm_i32(const int8_t *Xq, const int8_t *Wq, int64_t T, int64_t N, int64_t K, int32_t *acc) {
     int bad = 0;
-    #pragma omp parallel for schedule(static) reduction(|:bad)
+    /* every (t, n) is its own sum in k order: the threads share the outputs */
+    #pragma omp parallel for collapse(2) schedule(static) reduction(|:bad)
     for (int64_t t = 0; t < T; ++t)
         for (int64_t n = 0; n < N; ++n) {
             int64_t s = 0;

@@ -7,13 +7,13 @@ seeded synthetic input generators.
 from ._abi import (  # noqa: F401
     BITNET_BF16, BITNET_F32, BitnetChainOp, BitnetError, BitnetPackedW, BitnetPackItem, DecodeChain, PackBatch, PackedWeights, Workspace,
     bitnet_decode_chain, bitnet_dgrad, bitnet_pack_nm_update_batch, bitnet_pack_6of8_windows,
-    bitnet_quant_act_lift_6of8, packed_6of8, bitnet_pack_nm, bitnet_pack_nm_update, bitnet_quant_act, bitnet_rmsnorm_quant, bitnet_swiglu_quant, bitnet_wgrad, bitnet_adamw_step, AdamWBatch, adam_bias_correction, bitnet_quant_linear, bitnet_read_device_status, bitnet_wait_selftest, bitnet_sparse_linear, load,
+    bitnet_quant_act_lift_6of8, packed_6of8, bitnet_pack_nm, bitnet_pack_nm_update, bitnet_quant_act, bitnet_rmsnorm_quant, bitnet_swiglu_quant, bitnet_wgrad, bitnet_adamw_step, AdamWBatch, adam_bias_correction, bitnet_quant_linear, bitnet_read_device_status, bitnet_wait_selftest, bitnet_tensor_peak, bitnet_sparse_linear, load,
 )
 
 __all__ = [
     "PackedWeights", "Workspace", "BitnetError", "BitnetPackedW", "BitnetChainOp", "DecodeChain", "load",
     "bitnet_decode_chain", "bitnet_pack_nm_update_batch", "PackBatch", "BitnetPackItem",
     "bitnet_pack_6of8_windows", "bitnet_quant_act_lift_6of8", "packed_6of8",
-    "bitnet_pack_nm", "bitnet_pack_nm_update", "bitnet_quant_act", "bitnet_rmsnorm_quant", "bitnet_swiglu_quant", "bitnet_wgrad", "bitnet_adamw_step", "AdamWBatch", "adam_bias_correction", "bitnet_quant_linear", "bitnet_sparse_linear", "bitnet_dgrad", "bitnet_read_device_status", "bitnet_wait_selftest",
+    "bitnet_pack_nm", "bitnet_pack_nm_update", "bitnet_quant_act", "bitnet_rmsnorm_quant", "bitnet_swiglu_quant", "bitnet_wgrad", "bitnet_adamw_step", "AdamWBatch", "adam_bias_correction", "bitnet_quant_linear", "bitnet_sparse_linear", "bitnet_dgrad", "bitnet_read_device_status", "bitnet_wait_selftest", "bitnet_tensor_peak",
     "BITNET_F32", "BITNET_BF16",
 ]

@@ -36,7 +36,7 @@ EXPORTED = [
     "bitnet_dgrad_workspace_size", "bitnet_dgrad",
     "bitnet_wgrad_workspace_size", "bitnet_wgrad", "bitnet_adamw_workspace_size", "bitnet_adamw_step",
     "bitnet_adamw_batch_workspace_size", "bitnet_adamw_step_batch",
-    "bitnet_wait_selftest", "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
+    "bitnet_wait_selftest", "bitnet_tensor_peak", "bitnet_read_device_status", "bitnet_status_string", "bitnet_last_error", "bitnet_abi_version",
 ]
 
 
@@ -136,6 +136,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         "bitnet_adamw_step_batch": (I32, [ctypes.POINTER(BitnetAdamWItem), I32, ctypes.POINTER(BitnetAdamWHparams), F,
                                           P, SZ, P]),
         "bitnet_wait_selftest": (I32, [P, SZ, I32, P]),
+        "bitnet_tensor_peak": (I32, [I32, I64, P, P, SZ, P]),
         "bitnet_read_device_status": (I32, [P, P]),
         "bitnet_status_string": (ctypes.c_char_p, [I32]),
         "bitnet_last_error": (ctypes.c_char_p, []),
@@ -552,6 +553,15 @@ def bitnet_wait_selftest(limit_us: int = 50000, device="cuda", stream=None) -> i
     ws = Workspace(lib.bitnet_decode_chain_workspace_size(1), device)
     check(lib.bitnet_wait_selftest(ws.ptr, ws.nbytes, int(limit_us), _stream(stream)), "bitnet_wait_selftest")
     return lib.bitnet_read_device_status(ws.ptr, _stream(stream))
+
+
+def bitnet_tensor_peak(kind: int, iters: int, ws: Workspace, stream=None) -> float:
+    """Launches the tensor-core ceiling loop (kind 0 sparse int8, 1 dense int8,
+    2 bf16) and returns the dense-equivalent operations of the launch."""
+    ops = ctypes.c_double(0.0)
+    check(load().bitnet_tensor_peak(int(kind), int(iters), ctypes.byref(ops), ws.ptr, ws.nbytes, _stream(stream)),
+          "bitnet_tensor_peak")
+    return ops.value
 
 
 def bitnet_read_device_status(ws: Workspace, stream=None) -> int:

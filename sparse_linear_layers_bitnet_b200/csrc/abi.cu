@@ -385,10 +385,14 @@ bitnet_status bitnet_sparse_linear(const int8_t *Xq, const float *absmax, const 
 
 static size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
-static bool chain_fits(int64_t T, int64_t kmax) {
-    int ns = 0;
-    uint32_t stage = 0;
-    return bitnet::chain_ring(T, kmax, &ns, &stage);
+// The decode chain's shared memory holds the activations of one projection
+// (T rows of k), the weight ring and the partial sums of the CTA's row tiles.
+static bool chain_fits(int64_t T, int64_t kmax, bool x_bf16, int64_t n_out_max) {
+    const int64_t G = bitnet::num_sms();
+    const int64_t tiles = (n_out_max / 16 + G - 1) / G;
+    if (tiles > bitnet::kChainMaxTiles) return false;
+    bitnet::ChainLayout L;
+    return bitnet::chain_layout(T, kmax, x_bf16, static_cast<int>(tiles < 1 ? 1 : tiles), &L);
 }
 
 size_t bitnet_quant_linear_workspace_size(int64_t T, int64_t K) {
@@ -416,8 +420,9 @@ bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps
     if (!aligned(X, 16) || !aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: X and ws must be 16-byte aligned");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool xb = x_dtype == BITNET_BF16, yb = y_dtype == BITNET_BF16;
-    if (T <= 8 && W->dec_codes && n_out % 16 == 0 && k % 64 == 0 && n_out / 16 <= bitnet::kChainMaxTiles * bitnet::num_sms() &&
-        chain_fits(T, k) && ws_bytes >= bitnet_decode_chain_workspace_size(1)) {
+    if (T <= 8 && W->dec_codes && n_out % 16 == 0 && k % 64 == 0 && k <= bitnet::kChainMaxK &&
+        n_out / 16 <= bitnet::kChainMaxTiles * bitnet::num_sms() && chain_fits(T, k, xb, n_out) &&
+        ws_bytes >= bitnet_decode_chain_workspace_size(1)) {
         if (!aligned(W->dec_codes, 16)) return fail(BITNET_ERR_INVALID_ARG, "quant_linear: dec_codes alignment");
         bitnet::ChainOpDev op = {X, W->dec_codes, W->gamma, Y, acc_out, xq_out, absmax_out,
                                  static_cast<int32_t>(n_out), static_cast<int32_t>(k), 0, 0};
@@ -463,7 +468,7 @@ bitnet_status bitnet_decode_chain(const bitnet_chain_op *ops, int32_t n_ops, int
     if (!aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: ws must be 16-byte aligned");
     const int64_t max_tiles = static_cast<int64_t>(bitnet::kChainMaxTiles) * bitnet::num_sms();
     std::vector<bitnet::ChainOpDev> dev(static_cast<size_t>(n_ops));
-    int64_t kmax = 0;
+    int64_t kmax = 0, nmax = 0;
     for (int32_t i = 0; i < n_ops; ++i) {
         const bitnet_chain_op &o = ops[i];
         const bitnet_packed_w *W = o.W;
@@ -471,18 +476,21 @@ bitnet_status bitnet_decode_chain(const bitnet_chain_op *ops, int32_t n_ops, int
         if (!(W->n == 2 && W->m == 4)) return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: op %d: 2:4 only", i);
         if (W->n_out <= 0 || W->k <= 0 || W->n_out % 16 || W->k % 64)
             return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: op %d: needs n_out %% 16 == 0 and k %% 64 == 0", i);
-        if (W->n_out / 16 > max_tiles || W->n_out > INT32_MAX || W->k > INT32_MAX)
-            return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: op %d: n_out above 512 rows per SM", i);
+        if (W->n_out / 16 > max_tiles || W->n_out > INT32_MAX || W->k > bitnet::kChainMaxK)
+            return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: op %d: n_out above 512 rows per SM or k above %d", i,
+                        bitnet::kChainMaxK);
         if (!o.X || !o.Y) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: op %d: null X or Y", i);
         if (!aligned(o.X, 16) || !aligned(W->dec_codes, 16))
             return fail(BITNET_ERR_INVALID_ARG, "decode_chain: op %d: X and dec_codes must be 16-byte aligned", i);
         if (o.wait_prev != 0 && o.wait_prev != 1) return fail(BITNET_ERR_INVALID_ARG, "decode_chain: op %d: wait_prev must be 0 or 1", i);
         kmax = W->k > kmax ? W->k : kmax;
+        nmax = W->n_out > nmax ? W->n_out : nmax;
         dev[static_cast<size_t>(i)] = {o.X, W->dec_codes, W->gamma, o.Y, o.acc_out, o.xq_out, o.absmax_out,
                                        static_cast<int32_t>(W->n_out), static_cast<int32_t>(W->k), o.wait_prev, 0};
     }
-    if (!chain_fits(T, kmax))
-        return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: T * (k + 128) leaves no room for two weight stages");
+    if (!chain_fits(T, kmax, x_dtype == BITNET_BF16, nmax))
+        return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: one activation row of the largest k, the int8 activations "
+                                            "and two weight stages do not fit in shared memory");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return cuda_status(bitnet::launch_decode_chain(dev.data(), n_ops, T, x_dtype == BITNET_BF16, y_dtype == BITNET_BF16,
                                                    eps, kmax, ws, s),
@@ -518,6 +526,19 @@ bitnet_status bitnet_wait_selftest(void *ws, size_t ws_bytes, int32_t limit_us, 
     return cuda_status(bitnet::launch_wait_selftest(ws, static_cast<uint64_t>(limit_us) * 1000ull,
                                                     reinterpret_cast<cudaStream_t>(stream)),
                        "wait_selftest");
+}
+
+bitnet_status bitnet_tensor_peak(int32_t kind, int64_t iters, double *ops, void *ws, size_t ws_bytes,
+                                 bitnet_stream_t stream) {
+    if (kind < 0 || kind > 2) return fail(BITNET_ERR_INVALID_ARG, "tensor_peak: kind must be 0, 1 or 2");
+    if (iters < 1 || iters > (int64_t(1) << 40)) return fail(BITNET_ERR_INVALID_ARG, "tensor_peak: iters must be in [1, 2^40]");
+    if (!ops) return fail(BITNET_ERR_INVALID_ARG, "tensor_peak: ops is required");
+    if (!ws) return fail(BITNET_ERR_WORKSPACE, "tensor_peak: workspace is required");
+    if (ws_bytes < bitnet::kLinearWsBytes) return fail(BITNET_ERR_WORKSPACE, "tensor_peak: workspace needs %zu bytes", bitnet::kLinearWsBytes);
+    if (!aligned(ws, 16)) return fail(BITNET_ERR_INVALID_ARG, "tensor_peak: ws must be 16-byte aligned");
+    uint32_t *status = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + bitnet::kStatusOffset);
+    return cuda_status(bitnet::launch_tensor_peak(kind, iters, status, ops, reinterpret_cast<cudaStream_t>(stream)),
+                       "tensor_peak");
 }
 
 bitnet_status bitnet_read_device_status(void *ws, bitnet_stream_t stream) {

@@ -10,31 +10,48 @@
 //
 // Why one launch: at decode sizes (T <= 8) a projection moves 1 to 10 MB of
 // packed weights, under 2 us of HBM time, while each dependent kernel launch
-// adds about 3 us of completion and dependency latency.  Here every SM runs
-// one CTA for the whole chain:
-//  * a producer warp streams the CTA's share of every projection's packed
-//    weights (a contiguous byte range of the decode layout) into a ring of
-//    64, 32 or 16 KB shared-memory stages with bulk asynchronous copies.  Weights do not
-//    depend on activations, so the stream runs ahead across projection
-//    boundaries, limited only by free stages;
-//  * sixteen consumer warps, per projection: wait until every CTA has finished
-//    the previous projection (a grid-wide counter, acquire loads, bounded
-//    wait), read the T activation rows from L2, form the per-token scales and
-//    int8 codes in shared memory, run one m16n8k64 sparse MMA per 64-k tile
-//    of each weight record in the ring, sum the partial tiles in shared
-//    memory, write Y, and count themselves done (release add).
-// Row tiles of a projection are split over the CTAs in balanced contiguous
-// ranges, rotated per projection so that the larger shares move around.
+// adds about 3 us of completion and dependency latency.  Every SM runs one CTA
+// for the whole chain, split into roles that hand work to each other through
+// mbarriers, so that no role waits for a CTA-wide barrier and the weight
+// stream never pauses at a projection boundary:
+//  * weight producer (one thread): streams the CTA's share of every
+//    projection's packed weights (a contiguous byte range of the decode
+//    layout), the shares of consecutive projections back to back, into a
+//    ring of 32 KB (or 16 KB) shared-memory stages with bulk asynchronous
+//    copies, so that every stage is full and the bytes in flight do not
+//    depend on how small a share is.  Weights do not depend on activations,
+//    so it runs ahead across projections, limited only by free stages;
+//  * activation loader (one thread): copies each projection's T bf16/fp32
+//    activation rows, one row per bulk copy, into four staging slots (one per
+//    quantiser warp); the weight producer has already warmed L2 with them.
+//    A projection marked wait_prev is loaded only once every CTA has counted
+//    itself done with the previous projection (grid-wide counter, acquire);
+//  * quantisers (four warps, one token row of one projection per warp at a
+//    time): per-token absmax, scale and int8 codes from the staging slot into
+//    one of up to four int8 buffers, in the fragment order the MMA warps read,
+//    so that the quantisers run ahead of the MMA warps;
+//  * MMA warps (sixteen): for every projection piece of every ring stage, a
+//    contiguous run of its 16x64 weight records each; one m16n8k64 sparse
+//    MMA per record, partial sums of row tiles added into one of two shared
+//    partial-sum buffers;
+//  * epilogue (one warp): dequantises the CTA's outputs of a projection,
+//    writes Y, clears the buffer and counts the CTA done (release add).
+// So while the MMA warps run projection j, the quantisers prepare j + 1 and
+// the epilogue finishes j - 1.  Row tiles of a projection are split over the
+// CTAs in balanced contiguous ranges, rotated per projection so that the
+// larger shares move around.
+//
+// The 2-bit codes are expanded to int8 values 64 c (bits 6-7 of each byte),
+// which takes two instructions per register; the int32 sums are 64 times the
+// ternary ones, exactly, and the epilogue shifts them back.
 //
 // Two instantiations per activation type: any T <= 8, and T = 1 with the token
-// count folded to a constant (no per-token selects or chunk-to-token division
-// in the quantisation): 10% fewer instructions, and a 30-layer decode step at
-// T = 1 takes 0.492 ms against 0.521 ms with the general kernel.
+// count folded to a constant.
 //
 // All waits are bounded (2 s): a stage that never fills, a counter that never
-// reaches the grid size or an abort raised by another CTA ends the kernel
-// with the timeout bit in the status word; outstanding copies are waited for
-// (bounded) before the CTA exits.
+// reaches the grid size or an abort raised by another CTA ends every role of
+// the kernel with the timeout bit in the status word; outstanding copies are
+// waited for (bounded) before the copy threads exit.
 #include "../../include/bitnet_sparse.h"
 #include "common.cuh"
 #include "frag.cuh"
@@ -42,16 +59,31 @@
 
 namespace bitnet {
 
-constexpr int kChainConsumerWarps = 16;
-constexpr int kChainConsumers = kChainConsumerWarps * 32;
-constexpr int kChainThreads = kChainConsumers + 32;
+constexpr int kChainMmaWarps = 16;
+constexpr int kChainQuantWarps = 4;
+constexpr int kChainQuantThreads = kChainQuantWarps * 32;
+constexpr int kWarpQuant0 = kChainMmaWarps;                 // first quantiser warp
+constexpr int kWarpEpi = kWarpQuant0 + kChainQuantWarps;    // epilogue warp
+constexpr int kWarpXLoad = kWarpEpi + 1;                    // activation loader
+constexpr int kWarpWLoad = kWarpXLoad + 1;                  // weight producer
+constexpr int kChainThreads = (kWarpWLoad + 1) * 32;
 constexpr int kChainMaxStages = 16;
+constexpr int kChainMaxNb = 4;                              // int8 activation buffers (1 .. 4)
+constexpr int kChainScaleSlots = kChainMaxNb + 2;           // see the epilogue
+constexpr uint32_t kChainStageMax = 32768;   // weight ring stages of 32 KB, or 16 KB when a smaller ring must do
 
 struct ChainParams {
     ChainOpDev op[kChainMaxOps];
-    int32_t n_ops, T, x_bf16, y_bf16, ns, kmax;
-    uint32_t stage_bytes;   // ring stage size: 16, 32 or 64 KB (a multiple of 256)
+    int32_t n_ops, T, x_bf16, y_bf16;
+    int32_t ns;                // weight ring stages
+    uint32_t stage_bytes;      // 32 or 16 KB
+    int32_t nb;                // int8 activation buffers (1 .. kChainMaxNb)
+    uint32_t xq_bytes;         // one int8 buffer: T rows of pitch chain_pitch(kmax)
+    uint32_t xs_bytes;         // one staging slot: one activation row of kmax elements
+    int32_t tiles_max;         // most row tiles a CTA takes of one projection
+    uint32_t acc_bytes;        // one partial-sum buffer: T x tiles_max x 16 int32
     float eps;
+    int32_t release;      // some projection of this launch waits for its predecessor: count CTAs done
     uint32_t *counters;   // [n_ops], zero at launch
     uint32_t *abort;      // grid-wide abort word, zero at launch
     uint32_t *status;
@@ -71,8 +103,6 @@ __device__ __forceinline__ int chain_tiles(int j, int rows16, int &t0, int &t1) 
     return static_cast<int>(v);
 }
 
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kChainConsumers) : "memory"); }
-
 __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
@@ -81,75 +111,79 @@ __device__ __forceinline__ uint32_t ld_acquire(const uint32_t *p) {
 
 // Spins (bounded by limit_ns) until *ctr >= target.  On a timeout or a grid
 // abort it sets the CTA's abort flag (and, on a timeout, the grid abort word
-// and status).
+// and status).  The clock and the abort words are read every 16th poll only:
+// reading %globaltimer takes issue slots of a pipe the other warps need.
 __device__ bool wait_counter(const uint32_t *ctr, uint32_t target, const ChainParams &p, volatile int *s_abort,
                              uint64_t limit_ns = kWaitLimitNs) {
     if (ld_acquire(ctr) >= target) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (;;) {
+    uint64_t t0 = 0;
+    for (uint32_t i = 1;; ++i) {
         __nanosleep(32);
         if (ld_acquire(ctr) >= target) return true;
-        if (*reinterpret_cast<volatile uint32_t *>(p.abort) != 0u) {
-            *s_abort = 1;
-            return false;
-        }
-        if (globaltimer_ns() - t0 > limit_ns) {
-            *s_abort = 1;
-            atomicOr(p.status, kStatusTimeout);
-            atomicExch(p.abort, 1u);
-            return false;
-        }
-    }
-}
-
-// Producer's wait for a free stage: the thread is suspended in the barrier
-// (try_wait with a suspend-time hint) until the phase completes, instead of
-// spinning and taking issue slots from the consumer warps.  Bounded like
-// mbar_wait_bounded.
-__device__ bool mbar_wait_sleep(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
-    const uint64_t t0 = globaltimer_ns();
-    for (;;) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
-            : "memory");
-        if (ok) return true;
-        if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort = 1;
-            atomicOr(status, kStatusTimeout);
-            return false;
+        if ((i & 15u) == 0u) {
+            if (*reinterpret_cast<volatile uint32_t *>(p.abort) != 0u || *s_abort) {
+                *s_abort = 1;
+                return false;
+            }
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > limit_ns) {
+                *s_abort = 1;
+                atomicOr(p.status, kStatusTimeout);
+                atomicExch(p.abort, 1u);
+                return false;
+            }
         }
     }
 }
 
-// Consumer's wait for a filled stage: suspended in the barrier (short hint)
-// rather than spinning; bounded like mbar_wait_bounded.
-__device__ __forceinline__ bool mbar_wait_full(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
+// Wait for a phase.  try_wait may suspend the thread for a while, but it
+// can also return at once, so the loop keeps the cost of a failed round low:
+// the abort flag (a shared load) every 64th round, the clock (%globaltimer,
+// which takes issue slots of a pipe other warps need) every 1024th.  Gives up
+// when the CTA's abort flag is raised or after kWaitLimitNs (then it raises
+// the flag and the status bit).
+__device__ __forceinline__ bool mbar_wait_cta(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
     if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (;;) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(smem_u32(bar)), "r"(parity), "r"(2000u)
-            : "memory");
-        if (ok) return true;
-        if (*abort) return false;
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            *abort = 1;
-            atomicOr(status, kStatusTimeout);
-            return false;
+    uint64_t t0 = 0;
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((i & 63u) == 0u) {
+            if (*abort) return false;
+            if ((i & 1023u) == 0u) {
+                const uint64_t now = globaltimer_ns();
+                if (t0 == 0) {
+                    t0 = now;
+                } else if (now - t0 > kWaitLimitNs) {
+                    *abort = 1;
+                    atomicOr(status, kStatusTimeout);
+                    return false;
+                }
+            }
         }
     }
 }
+
+// Barrier of the MMA warps (hardware barrier 2) that also ORs a predicate
+// over them: one warp waits for a ring stage, the others block here without
+// issuing instructions, and all of them learn whether the wait succeeded.
+__device__ __forceinline__ bool mma_sync_or(bool v) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 2, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(v ? 1u : 0u), "n"(kChainMmaWarps * 32)
+        : "memory");
+    return r != 0;
+}
+
+#ifndef CHAIN_NB_MAX
+#define CHAIN_NB_MAX 4
+#endif
 
 // Wait that ignores the abort flag, up to a deadline (for draining copies in flight).
 __device__ bool mbar_wait_until(uint64_t *bar, uint32_t parity, uint64_t deadline_ns) {
@@ -159,202 +193,84 @@ __device__ bool mbar_wait_until(uint64_t *bar, uint32_t parity, uint64_t deadlin
     return true;
 }
 
-// Barrier of the consumer warps (hardware barrier 2; plain consumer barriers
-// use 1) that also ORs a predicate over them, so that every consumer takes the
-// same branch after it.
-__device__ __forceinline__ bool consumer_sync_or(bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 2, %2, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(v ? 1u : 0u), "n"(kChainConsumers)
-        : "memory");
-    return r != 0;
+// Adds bytes to the transaction count of the barrier's current phase (no arrival).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
-// adds a row tile's partial sums (four accumulators) into the shared sums and clears them
-__device__ __forceinline__ void chain_flush(int *s_acc, int tile, int lane, int (&acc)[4][4]) {
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        atomicAdd(&s_acc[(tile * 32 + lane) * 4 + q], acc[0][q] + acc[1][q] + acc[2][q] + acc[3][q]);
-        acc[0][q] = acc[1][q] = acc[2][q] = acc[3][q] = 0;
-    }
-}
-
-template <bool BF16>
-struct ChainChunk {
-    static constexpr int kElems = BF16 ? 8 : 4;
-    uint4 raw;
-    __device__ __forceinline__ float get(int j) const {
-        const int i = BF16 ? (j >> 1) : j;
-        const uint32_t w = i == 0 ? raw.x : (i == 1 ? raw.y : (i == 2 ? raw.z : raw.w));
-        if (BF16) return __uint_as_float((j & 1) ? (w & 0xffff0000u) : (w << 16));
-        return __uint_as_float(w);
-    }
-    __device__ __forceinline__ float absmax() const {
-        float m = 0.0f;
-#pragma unroll
-        for (int j = 0; j < kElems; ++j) m = fmaxf(m, fabsf(get(j)));
-        return m;
-    }
-    // Codes of the chunk's elements e0 .. e0 + kElems - 1 of a token row whose
-    // shared copy starts at row.  Within each 64-element k-tile the sixteen
-    // 4-byte words are stored transposed (word 4 j + q at 4 q + j), so that the
-    // 16 bytes lane q of a token takes as its m16n8k64 B fragment (k = 4 q + 16 j
-    // + 0..3, j = 0..3) are contiguous.
-    __device__ __forceinline__ void store_codes(int8_t *row, int e0, float s) const {
-        int8_t *tile = row + (e0 & ~63);
-        const int u0 = (e0 & 63) >> 2;   // first word within the tile
-        if constexpr (BF16) {
-            float v[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) v[j] = get(j);
-            const uint2 q = codes8_fast(v, s);
-            const int u1 = u0 + 1;
-            *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u0 & 3) + (u0 >> 2))) = q.x;
-            *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u1 & 3) + (u1 >> 2))) = q.y;
-        } else {
-            *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u0 & 3) + (u0 >> 2))) =
-                codes4_fast(get(0), get(1), get(2), get(3), s);
-        }
-    }
-};
+// Barrier of the quantiser warps (hardware barrier 1), used once, after
+// they have loaded every projection's gamma into shared memory.
+__device__ __forceinline__ void quant_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kChainQuantThreads) : "memory"); }
 
 // Row pitch of the shared int8 activations: k + 64 or k + 128, whichever is
 // 64 mod 128 bytes, so that the two token rows one quarter-warp reads in a
 // 16-byte-per-lane load fall in disjoint banks.
 __device__ __host__ __forceinline__ int64_t chain_pitch(int64_t k) { return k + 64 + (k & 64); }
 
-// Per-token absmax, scales and int8 codes of one projection's activations
-// (same arithmetic as bitnet_quant_act) into shared memory, row pitch
-// chain_pitch(k), each 64-k tile in fragment order (see store_codes).
-// X is read through L2 only (ld.global.cg): it may have been written by other
-// SMs earlier in this kernel.  Thread ctid takes the flattened 16-byte chunks
-// c = ctid + 512 u.  The first kChainKeep of them are loaded together (all in
-// flight at once) and stay in registers for the second pass; any further ones
-// are loaded kChainKeep at a time in each pass.  Two is the measured best
-// (decode step at T = 1: 0.533 ms against 0.550 with three and 0.557 with four
-// cached chunks; T = 8: 1.03, 0.98 and 0.98 ms): a larger cache costs the
-// one- and two-chunk rows of T = 1 more than it saves at T = 8.  A chunk's token is
-// floor((c + 1/2) / cpr) through a float reciprocal: c / cpr <= 8 and c < 2^20,
-// so the rounding error is far below the 1 / (2 cpr) margin.
-// s_inv[t] = 127 / a_t and s_scale[t] = (gamma a_t) / 127 are formed once per
-// token.
-constexpr int kChainKeep = 2;
-
-template <int TM>
-__device__ __forceinline__ void chain_chunk_pos(int c, int cpr, float inv_cpr, int &t, int &i) {
-    if (TM == 1) {   // one token: every chunk is in row 0
-        t = 0;
-        i = c;
-        return;
+// |x| bits of a 16-byte chunk folded into one word whose unsigned order is the
+// order of the largest magnitude: for bf16 a u16x2 max of the magnitude bits
+// (sign cleared); for fp32 the u32 max of the magnitude bits.  Non-negative
+// floats order like their bit patterns.
+template <bool BF16>
+__device__ __forceinline__ uint32_t chunk_absbits(const uint4 v) {
+    if constexpr (BF16) {
+        const uint32_t m = 0x7fff7fffu;
+        return vmax_u16x2(vmax_u16x2(v.x & m, v.y & m), vmax_u16x2(v.z & m, v.w & m));
+    } else {
+        const uint32_t m = 0x7fffffffu;
+        return max(max(v.x & m, v.y & m), max(v.z & m, v.w & m));
     }
-    t = __float2int_rz((static_cast<float>(c) + 0.5f) * inv_cpr);
-    i = c - t * cpr;
+}
+// the fp32 bits of a folded magnitude word
+template <bool BF16>
+__device__ __forceinline__ uint32_t absbits_to_f32(uint32_t m) {
+    if constexpr (BF16) return max(m & 0xffffu, m >> 16) << 16;
+    return m;
 }
 
-// TM: the most tokens the instantiation handles (1, or 8 for any T <= 8).
-template <bool BF16, int TM>
-__device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float eps, float gamma, int8_t *s_xq,
-                               float (*s_red)[8], float *s_amax, float *s_inv, float *s_scale, int ctid) {
-    using C = ChainChunk<BF16>;
-    const int cpr = k / C::kElems;             // chunks per token row (>= 8)
-    const int nchunk = T * cpr;
-    const float inv_cpr = 1.0f / static_cast<float>(cpr);
-    const int warp = ctid >> 5, lane = ctid & 31;
-    float m[TM];
+// Codes of one 16-byte chunk (elements e0 .. e0 + 7 for bf16, e0 .. e0 + 3 for
+// fp32 of a token row whose shared int8 copy starts at row).  Within each
+// 64-element k-tile the sixteen 4-byte words are stored transposed (word
+// 4 j + q at 4 q + j), so that the 16 bytes lane q of a token takes as its
+// m16n8k64 B fragment (k = 4 q + 16 j + 0..3, j = 0..3) are contiguous.
+template <bool BF16>
+__device__ __forceinline__ uint2 chunk_store_codes(const uint4 v, int8_t *row, int e0, float s) {
+    int8_t *tile = row + (e0 & ~63);
+    const int u0 = (e0 & 63) >> 2;   // first word within the tile
+    if constexpr (BF16) {
+        float f[8];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int t = 0; t < TM; ++t) m[t] = 0.0f;
-    C keep[kChainKeep];
-#pragma unroll
-    for (int u = 0; u < kChainKeep; ++u) {
-        const int c = ctid + u * kChainConsumers;
-        keep[u].raw = c < nchunk ? __ldcg(X + c) : make_uint4(0u, 0u, 0u, 0u);
-    }
-#pragma unroll
-    for (int u = 0; u < kChainKeep; ++u) {
-        const int c = ctid + u * kChainConsumers;
-        if (c < nchunk) {
-            int t, i;
-            chain_chunk_pos<TM>(c, cpr, inv_cpr, t, i);
-            const float ma = keep[u].absmax();
-#pragma unroll
-            for (int tt = 0; tt < TM; ++tt)
-                if (tt == t) m[tt] = fmaxf(m[tt], ma);
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
         }
+        const uint2 q = codes8_fast(f, s);
+        const int u1 = u0 + 1;
+        *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u0 & 3) + (u0 >> 2))) = q.x;
+        *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u1 & 3) + (u1 >> 2))) = q.y;
+        return q;
+    } else {
+        const uint32_t q =
+            codes4_fast(__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w), s);
+        *reinterpret_cast<uint32_t *>(tile + 4 * (4 * (u0 & 3) + (u0 >> 2))) = q;
+        return make_uint2(q, 0u);
     }
-    // chunks beyond the register cache (long rows of several tokens): kChainKeep loads in flight per round
-    for (int c0 = ctid + kChainKeep * kChainConsumers; c0 < nchunk; c0 += kChainKeep * kChainConsumers) {
-        C v[kChainKeep];
+}
+
+// Adds a row tile's partial sums (four accumulators) into the shared sums,
+// layout [token][tile][row of 16], and clears them.  Lane l's value q belongs
+// to row l / 4 + 8 (q / 2) and token 2 (l % 4) + q % 2 of the m16n8 tile.
+template <int TM>
+__device__ __forceinline__ void chain_flush(int *acc_buf, int tiles_max, int tile, int lane, int T, int (&acc)[4][4]) {
 #pragma unroll
-        for (int u = 0; u < kChainKeep; ++u) {
-            const int c = c0 + u * kChainConsumers;
-            if (c < nchunk) v[u].raw = __ldcg(X + c);
-        }
-#pragma unroll
-        for (int u = 0; u < kChainKeep; ++u) {
-            const int c = c0 + u * kChainConsumers;
-            if (c < nchunk) {
-                int t, i;
-                chain_chunk_pos<TM>(c, cpr, inv_cpr, t, i);
-                const float ma = v[u].absmax();
-#pragma unroll
-                for (int tt = 0; tt < TM; ++tt)
-                    if (tt == t) m[tt] = fmaxf(m[tt], ma);
-            }
-        }
-    }
-#pragma unroll
-    for (int t = 0; t < TM; ++t) {
-        if (t < T) {
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) m[t] = fmaxf(m[t], __shfl_xor_sync(0xffffffffu, m[t], o));
-        }
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int t = 0; t < TM; ++t) s_red[warp][t] = m[t];
-    }
-    consumer_sync();
-    if (ctid < T) {
-        float v = 0.0f;
-#pragma unroll
-        for (int q = 0; q < kChainConsumerWarps; ++q) v = fmaxf(v, s_red[q][ctid]);
-        v = v > eps ? v : eps;
-        s_amax[ctid] = v;
-        s_inv[ctid] = __fdiv_rn(127.0f, v);
-        s_scale[ctid] = __fdiv_rn(__fmul_rn(gamma, v), 127.0f);
-    }
-    consumer_sync();
-    const int pitch = chain_pitch(k);
-#pragma unroll
-    for (int u = 0; u < kChainKeep; ++u) {
-        const int c = ctid + u * kChainConsumers;
-        if (c < nchunk) {
-            int t, i;
-            chain_chunk_pos<TM>(c, cpr, inv_cpr, t, i);
-            keep[u].store_codes(s_xq + t * pitch, i * C::kElems, s_inv[t]);
-        }
-    }
-    for (int c0 = ctid + kChainKeep * kChainConsumers; c0 < nchunk; c0 += kChainKeep * kChainConsumers) {
-        C v[kChainKeep];
-#pragma unroll
-        for (int u = 0; u < kChainKeep; ++u) {
-            const int c = c0 + u * kChainConsumers;
-            if (c < nchunk) v[u].raw = __ldcg(X + c);
-        }
-#pragma unroll
-        for (int u = 0; u < kChainKeep; ++u) {
-            const int c = c0 + u * kChainConsumers;
-            if (c < nchunk) {
-                int t, i;
-                chain_chunk_pos<TM>(c, cpr, inv_cpr, t, i);
-                v[u].store_codes(s_xq + t * pitch, i * C::kElems, s_inv[t]);
-            }
-        }
+    for (int q = 0; q < 4; ++q) {
+        const int t = 2 * (lane & 3) + (q & 1);
+        const int row = (lane >> 2) + 8 * (q >> 1);
+        const int v = acc[0][q] + acc[1][q] + acc[2][q] + acc[3][q];
+        const bool real = TM == 1 ? t == 0 : t < T;
+        if (real) atomicAdd(&acc_buf[(t * tiles_max + tile) * 16 + row], v);
+        acc[0][q] = acc[1][q] = acc[2][q] = acc[3][q] = 0;
     }
 }
 
@@ -362,36 +278,61 @@ template <bool XBF16, int TM>
 __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_constant__ ChainParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kChainMaxStages], s_empty[kChainMaxStages];
-    __shared__ float s_red[kChainConsumerWarps][8];
-    __shared__ float s_amax[8], s_inv[8], s_scale[8];
+    __shared__ __align__(8) uint64_t s_xs_full[kChainQuantWarps], s_xs_empty[kChainQuantWarps];
+    __shared__ __align__(8) uint64_t s_xq_full[kChainMaxNb], s_xq_empty[kChainMaxNb];
+    __shared__ __align__(8) uint64_t s_acc_full[2], s_acc_empty[2];
+    __shared__ float s_gamma[kChainMaxOps];
+    __shared__ float s_scale[kChainScaleSlots][8];
+    __shared__ float s_amax[kChainScaleSlots][8];
     __shared__ int s_abort;
     const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
     const int ns = p.ns;
     const int T = TM == 1 ? 1 : p.T;   // a one-token instantiation folds T away
     const uint32_t G = gridDim.x;
-    // dynamic shared memory: ring [ns][16 KB] | partial sums [kChainMaxTiles][32][4] int | int8 rows
+    // dynamic shared memory: weight ring | staging slots | int8 buffers | partial-sum buffers
     uint8_t *ring = smem;
     const uint32_t stage_bytes = p.stage_bytes;
-    int *s_acc = reinterpret_cast<int *>(smem + static_cast<size_t>(ns) * stage_bytes);
-    int8_t *s_xq = reinterpret_cast<int8_t *>(s_acc + kChainMaxTiles * 128);
+    uint8_t *xs = ring + static_cast<size_t>(ns) * stage_bytes;
+    int8_t *xqb = reinterpret_cast<int8_t *>(xs + static_cast<size_t>(kChainQuantWarps) * p.xs_bytes);
+    int *sacc = reinterpret_cast<int *>(xqb + static_cast<size_t>(p.nb) * p.xq_bytes);
+    const int acc_words = static_cast<int>(p.acc_bytes >> 2);
 
-    for (int i = tid; i < kChainMaxTiles * 128; i += kChainThreads) s_acc[i] = 0;
+    for (int i = tid; i < 2 * acc_words; i += kChainThreads) sacc[i] = 0;
     if (tid == 0) {
         s_abort = 0;
         for (int s = 0; s < ns; ++s) {
             mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], kChainConsumerWarps);
+            mbar_init(&s_empty[s], kChainMmaWarps);
+        }
+        for (int s = 0; s < kChainQuantWarps; ++s) {
+            mbar_init(&s_xs_full[s], 1);
+            mbar_init(&s_xs_empty[s], 1);
+        }
+        for (int s = 0; s < p.nb; ++s) {
+            mbar_init(&s_xq_full[s], static_cast<uint32_t>(T));                    // one arrival per row
+            mbar_init(&s_xq_empty[s], kChainMmaWarps);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_acc_full[s], kChainMmaWarps);
+            mbar_init(&s_acc_empty[s], 1);
         }
         fence_mbar_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
     __syncthreads();
 
-    if (tid >= kChainConsumers) {
-        // ------------------------------------------------------------ producer
-        if (tid != kChainConsumers) return;
-        uint32_t it = 0, ps = 0, pph = 0;   // stages issued; slot it % ns; parity of fill round it / ns
-        bool ok = true;
+    if (warp == kWarpWLoad) {
+        // ------------------------------------------------------------ weight producer
+        if (lane != 0) return;
+        // The CTA's shares of all projections go back to back into the ring:
+        // stage k holds stream bytes [k S, (k + 1) S), one bulk copy per piece of
+        // a projection in it; the stage's single arrival comes when it is full
+        // (or the stream ends), so its phase completes only once every piece of
+        // it has landed.
+        uint32_t it = 0, ps = 0, pph = 0;   // stages opened; slot it % ns; parity of fill round it / ns
+        uint32_t fill = 0;                  // bytes placed in the open stage
+        bool open = false, ok = true;
         for (int j = 0; j < p.n_ops && ok; ++j) {
             const ChainOpDev &op = p.op[j];
             int t0, t1;
@@ -400,30 +341,46 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             const uint32_t bytes = static_cast<uint32_t>(t1 - t0) * tile_bytes;
             const uint8_t *src = op.dec + static_cast<size_t>(t0) * tile_bytes;
             // Warm L2 with this CTA's slice of the projection's activation rows
-            // (128-byte lines b, b + G, ...).  Only a cache hint: L2 is the
-            // coherence point, so a line prefetched before an earlier projection
-            // writes it is updated by that write.
+            // (128-byte lines b, b + G, ...), so that the loader's copy, issued
+            // later, does not queue behind the weight stream in HBM.  Only a
+            // cache hint: L2 is the coherence point, so a line prefetched before
+            // an earlier projection writes it is updated by that write.
             {
-                const size_t xbytes = static_cast<size_t>(p.T) * static_cast<size_t>(op.k) * (p.x_bf16 ? 2u : 4u);
-                for (size_t l = static_cast<size_t>(blockIdx.x) * 128; l < xbytes; l += static_cast<size_t>(gridDim.x) * 128)
+                const size_t xbytes = static_cast<size_t>(T) * static_cast<size_t>(op.k) * (XBF16 ? 2u : 4u);
+                for (size_t l = static_cast<size_t>(blockIdx.x) * 128; l < xbytes; l += static_cast<size_t>(G) * 128)
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(static_cast<const uint8_t *>(op.X) + l));
             }
-            for (uint32_t off = 0; off < bytes; off += stage_bytes, ++it) {
-                // reuse of slot ps in round r >= 1 waits for the consumers' release of round r - 1
-                if (it >= static_cast<uint32_t>(ns) && !mbar_wait_sleep(&s_empty[ps], pph ^ 1u, &s_abort, p.status)) {
-                    ok = false;
-                    break;
+            for (uint32_t off = 0; off < bytes;) {
+                if (!open) {
+                    // reuse of slot ps in round r >= 1 waits for the MMA warps' release of round r - 1
+                    if (it >= static_cast<uint32_t>(ns) && !mbar_wait_cta(&s_empty[ps], pph ^ 1u, &s_abort, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    open = true;
+                    fill = 0;
                 }
-                const uint32_t n = (bytes - off) < stage_bytes ? (bytes - off) : stage_bytes;
-                mbar_arrive_expect_tx(&s_full[ps], n);
-                bulk_load(ring + static_cast<size_t>(ps) * stage_bytes, src + off, n, &s_full[ps]);
-                if (++ps == static_cast<uint32_t>(ns)) {
-                    ps = 0;
-                    pph ^= 1u;
+                const uint32_t n = (bytes - off) < (stage_bytes - fill) ? (bytes - off) : (stage_bytes - fill);
+                mbar_expect_tx(&s_full[ps], n);
+                bulk_load(ring + static_cast<size_t>(ps) * stage_bytes + fill, src + off, n, &s_full[ps]);
+                fill += n;
+                off += n;
+                if (fill == stage_bytes) {
+                    mbar_arrive(&s_full[ps]);
+                    open = false;
+                    ++it;
+                    if (++ps == static_cast<uint32_t>(ns)) {
+                        ps = 0;
+                        pph ^= 1u;
+                    }
                 }
             }
         }
-        // drain: every issued stage must have landed before the CTA may exit
+        if (open && ok) {   // the stream's last, partly filled stage
+            mbar_arrive(&s_full[ps]);
+            ++it;
+        }
+        // drain: every issued stage must have landed before the thread exits
         // (earlier stages were consumed before their slot was reused)
         const uint32_t first = it > static_cast<uint32_t>(ns) ? it - ns : 0u;
         const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
@@ -431,187 +388,376 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         return;
     }
 
-    // ---------------------------------------------------------------- consumers
-    // Every branch that can differ between consumer threads (an expired wait,
-    // an abort) is decided through consumer_sync_or or a warp vote, so that the
-    // consumer barriers never miss a thread.
-    const int ctid = tid;
-    const int warp = ctid >> 5, lane = ctid & 31;
-    uint32_t cs = 0, cph = 0;   // ring slot of the next stage and the parity of its fill round
-    for (int j = 0; j < p.n_ops; ++j) {
-        const ChainOpDev &op = p.op[j];
-        int t0, t1;
-        const int share = chain_tiles(j, op.n_out >> 4, t0, t1);
-        const int ntile = t1 - t0;
-        const int ktiles = op.k >> 6;
-        const uint32_t bytes = static_cast<uint32_t>(ntile) * static_cast<uint32_t>(ktiles) * 256u;
-        // gamma belongs to the packed weights: read before the wait
-        const float gamma = ntile > 0 ? __ldg(op.gamma) : 0.0f;
-        // 1. every CTA has finished the previous projection
-        if (j > 0 && op.wait_prev) {
-            bool bad = false;
-            if (ctid == 0) bad = !wait_counter(&p.counters[j - 1], G, p, &s_abort);
-            if (consumer_sync_or(bad || s_abort != 0)) break;
-        }
-        if (ntile > 0) {
-            // 2. int8 activations of this projection
-            chain_quantise<XBF16, TM>(static_cast<const uint4 *>(op.X), T, op.k, p.eps, gamma, s_xq, s_red, s_amax, s_inv,
-                                  s_scale, ctid);
-            consumer_sync();
-            // 3. weight records from the ring: in each stage, warp w takes the
-            //    contiguous records [w n / 16, (w + 1) n / 16).  Lane l holds the
-            //    B fragment of token l / 4 (zero for tokens >= T): the 16 bytes
-            //    lane l % 4 needs of each 64-k tile sit contiguously in the
-            //    shared row (fragment order), one 16-byte load per record.
-            const int bn = lane >> 2;
-            const bool has_b = bn < T;
-            const uint4 *b_src =
-                reinterpret_cast<const uint4 *>(s_xq + static_cast<int64_t>(has_b ? bn : 0) * chain_pitch(op.k)) +
-                (lane & 3);
-            int cur = -1;
-            int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
-            bool failed = false;
-            const float inv_kt = 1.0f / static_cast<float>(ktiles);
-            for (uint32_t off = 0; off < bytes; off += stage_bytes) {
-                const uint32_t s = cs;
-                const bool ok = mbar_wait_full(&s_full[s], cph, &s_abort, p.status);
-                if (++cs == static_cast<uint32_t>(ns)) {
-                    cs = 0;
-                    cph ^= 1u;
+    if (warp == kWarpXLoad) {
+        // ------------------------------------------------------------ activation loader
+        if (lane != 0) return;
+        // one bulk copy per activation row: row item (counting the rows of every
+        // projection with rows here) goes to staging slot item % 4, which belongs
+        // to quantiser warp item % 4
+        uint32_t item = 0;
+        bool ok = true;
+        for (int j = 0; j < p.n_ops && ok; ++j) {
+            const ChainOpDev &op = p.op[j];
+            int t0, t1;
+            chain_tiles(j, op.n_out >> 4, t0, t1);
+            if (t1 == t0) continue;   // no rows here: the activations are not needed
+            if (j > 0 && op.wait_prev) {
+                // every CTA has finished projection j - 1 (and, in chain order, all before it)
+                if (!wait_counter(&p.counters[j - 1], G, p, &s_abort)) {
+                    ok = false;
+                    break;
                 }
+                // the activations were written by other SMs' generic stores, made visible by the
+                // acquire above; order that before the bulk copy's async-proxy reads
+                asm volatile("fence.proxy.async.global;" ::: "memory");
+            }
+            const uint32_t row_bytes = static_cast<uint32_t>(op.k) * (XBF16 ? 2u : 4u);
+            for (int t = 0; t < T; ++t, ++item) {
+                const uint32_t slot = item % kChainQuantWarps, round = item / kChainQuantWarps;
+                if (round >= 1u && !mbar_wait_cta(&s_xs_empty[slot], (round - 1u) & 1u, &s_abort, p.status)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&s_xs_full[slot], row_bytes);
+                bulk_load(xs + static_cast<size_t>(slot) * p.xs_bytes,
+                          static_cast<const uint8_t *>(op.X) + static_cast<size_t>(t) * row_bytes, row_bytes,
+                          &s_xs_full[slot]);
+            }
+        }
+        const uint32_t first = item > kChainQuantWarps ? item - kChainQuantWarps : 0u;
+        const uint64_t deadline = globaltimer_ns() + kWaitLimitNs;
+        for (uint32_t q = first; q < item; ++q)
+            mbar_wait_until(&s_xs_full[q % kChainQuantWarps], (q / kChainQuantWarps) & 1u, deadline);
+        return;
+    }
+
+    if (warp >= kWarpQuant0 && warp < kWarpEpi) {
+        // ------------------------------------------------------------ quantisers
+        // Work item = one token row of one projection, in chain order; item i
+        // belongs to quantiser warp i % 4 and arrives in staging slot i % 4, so
+        // that several projections (T = 1) or several rows (T > 1) are
+        // quantised at once and no barrier joins the quantiser warps.  A row:
+        // absmax of the lane's 16-byte chunks (bit patterns), one warp
+        // reduction, the scale, then the codes into the int8 buffer in
+        // fragment order.
+        // Parity waits see only the last two phases of a barrier, so every
+        // warp must meet each barrier it waits on in consecutive rounds: its
+        // staging slot is its own; an int8 buffer is met by the warps owning a
+        // row of its projections, which for T >= 4 is every warp, and for
+        // T < 4 (the host then takes four buffers) depends only on the
+        // projection's index mod 4, the same for every use of the buffer.
+        const int qw = warp - kWarpQuant0;
+        const int qt = tid - kWarpQuant0 * 32;
+        for (int i = qt; i < p.n_ops; i += kChainQuantThreads) s_gamma[i] = __ldg(p.op[i].gamma);
+        quant_sync();   // gamma of every projection in shared memory (no load on the per-row path)
+        constexpr int kElems = XBF16 ? 8 : 4;
+        const uint32_t nbu = static_cast<uint32_t>(p.nb);
+        uint32_t uq = 0, item = 0;   // projections and rows passed so far
+        bool failed = false;
+        for (int j = 0; j < p.n_ops && !failed; ++j) {
+            const ChainOpDev &op = p.op[j];
+            int t0, t1;
+            const int share = chain_tiles(j, op.n_out >> 4, t0, t1);
+            if (t1 == t0) continue;
+            const int xb = static_cast<int>(uq % nbu);
+            const uint32_t xround = uq / nbu;
+            const int sc = static_cast<int>(uq % kChainScaleSlots);
+            const int k = op.k;
+            const int pitch = static_cast<int>(chain_pitch(k));
+            const int cpr = k / kElems;   // 16-byte chunks per row
+            const bool copy_out = share == static_cast<int>(G) - 1;
+            const bool xq_vec = op.xq_out && (reinterpret_cast<uintptr_t>(op.xq_out) & 7u) == 0u;
+            bool waited = false;
+            for (int t = 0; t < T; ++t, ++item) {
+                if (item % kChainQuantWarps != static_cast<uint32_t>(qw)) continue;
+                // the MMA warps are done with this buffer's previous projection
+                bool ok = waited || xround == 0u ||
+                          mbar_wait_cta(&s_xq_empty[xb], (xround - 1u) & 1u, &s_abort, p.status);
+                waited = true;
+                // this warp's own staging slot: its rows arrive there in consecutive rounds
+                ok = ok && mbar_wait_cta(&s_xs_full[qw], (item / kChainQuantWarps) & 1u, &s_abort, p.status);
                 if (!__all_sync(0xffffffffu, ok)) {
                     failed = true;
                     break;
                 }
-                const int nrec = static_cast<int>(((bytes - off) < stage_bytes ? (bytes - off) : stage_bytes) >> 8);
-                const int i0 = (warp * nrec) / kChainConsumerWarps, i1 = ((warp + 1) * nrec) / kChainConsumerWarps;
-                if (i0 < i1) {
-                    const int r0 = static_cast<int>(off >> 8) + i0;
-                    // r0 / ktiles through the reciprocal (r0 < 2^24: off by at most one, corrected)
-                    int tile = __float2int_rz(static_cast<float>(r0) * inv_kt);
-                    int kt = r0 - tile * ktiles;
-                    if (kt < 0) {
-                        --tile;
-                        kt += ktiles;
-                    } else if (kt >= ktiles) {
-                        ++tile;
-                        kt -= ktiles;
-                    }
-                    const uint2 *rec = reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(s) * stage_bytes) + lane;
-                    int i = i0;
-                    while (i < i1) {
-                        if (tile != cur) {
-                            if (cur >= 0) chain_flush(s_acc, cur, lane, acc);
-                            cur = tile;
-                        }
-                        if (i + 4 <= i1 && kt + 4 <= ktiles) {
-                            // four records of one row tile: all loads first, then the MMAs
-                            uint2 w[4];
-                            uint32_t bf[4][4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) w[u] = rec[(i + u) * 32];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const uint4 v = has_b ? b_src[(kt + u) * 4] : make_uint4(0u, 0u, 0u, 0u);
-                                bf[u][0] = v.x;
-                                bf[u][1] = v.y;
-                                bf[u][2] = v.z;
-                                bf[u][3] = v.w;
-                            }
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                uint32_t a4[4];
-#pragma unroll
-                                for (int r = 0; r < 4; ++r) a4[r] = expand_codes(w[u].x, r);
-                                mma_sp_m16n8k64(acc[u], a4, bf[u], w[u].y);
-                            }
-                            i += 4;
-                            kt += 4;
+                const uint4 *src = reinterpret_cast<const uint4 *>(xs + static_cast<size_t>(qw) * p.xs_bytes);
+                // pass 1: absmax of the row
+                uint32_t m = 0u;
+                for (int c = lane; c < cpr; c += 32) {
+                    const uint32_t a = chunk_absbits<XBF16>(src[c]);
+                    m = XBF16 ? vmax_u16x2(m, a) : max(m, a);
+                }
+                float a = __uint_as_float(__reduce_max_sync(0xffffffffu, absbits_to_f32<XBF16>(m)));
+                a = a > p.eps ? a : p.eps;
+                const float s_inv = __fdiv_rn(127.0f, a);
+                if (lane == 0) {
+                    s_scale[sc][t] = __fdiv_rn(__fmul_rn(s_gamma[j], a), 127.0f);
+                    s_amax[sc][t] = a;
+                    if (copy_out && op.amax_out) op.amax_out[t] = a;
+                }
+                // pass 2: codes (and, on one CTA, their copy in natural order)
+                int8_t *row = xqb + static_cast<size_t>(xb) * p.xq_bytes + static_cast<size_t>(t) * pitch;
+                for (int c = lane; c < cpr; c += 32) {
+                    const uint2 q = chunk_store_codes<XBF16>(src[c], row, c * kElems, s_inv);
+                    if (copy_out && op.xq_out) {
+                        int8_t *dst = op.xq_out + static_cast<size_t>(t) * k + static_cast<size_t>(c) * kElems;
+                        if (xq_vec && XBF16) {
+                            *reinterpret_cast<uint2 *>(dst) = q;
+                        } else if (xq_vec) {
+                            *reinterpret_cast<uint32_t *>(dst) = q.x;
                         } else {
-                            const uint2 w = rec[i * 32];
-                            uint32_t bf[4], a4[4];
-                            const uint4 v = has_b ? b_src[kt * 4] : make_uint4(0u, 0u, 0u, 0u);
-                            bf[0] = v.x;
-                            bf[1] = v.y;
-                            bf[2] = v.z;
-                            bf[3] = v.w;
 #pragma unroll
-                            for (int r = 0; r < 4; ++r) a4[r] = expand_codes(w.x, r);
-                            mma_sp_m16n8k64(acc[0], a4, bf, w.y);
-                            i += 1;
-                            kt += 1;
-                        }
-                        if (kt == ktiles) {
-                            kt = 0;
-                            ++tile;
+                            for (int e = 0; e < kElems; ++e)
+                                dst[e] = static_cast<int8_t>(((e < 4 ? q.x : q.y) >> (8 * (e & 3))) & 0xffu);
                         }
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[s]);
+                if (lane == 0) {
+                    mbar_arrive(&s_xq_full[xb]);   // T arrivals per projection
+                    mbar_arrive(&s_xs_empty[qw]);
+                }
             }
-            if (cur >= 0) chain_flush(s_acc, cur, lane, acc);
-            if (consumer_sync_or(failed || s_abort != 0)) break;
-            // 4. dequantise and store this CTA's rows; clear the partial sums
-            for (int e = ctid; e < ntile * 128; e += kChainConsumers) {
-                const int tl = e >> 7, ln = (e >> 2) & 31, q = e & 3;
-                const int t = 2 * (ln & 3) + (q & 1);
-                const int acc = s_acc[e];
-                s_acc[e] = 0;
-                if (t >= T) continue;
-                const int64_t n = static_cast<int64_t>(t0 + tl) * 16 + (ln >> 2) + 8 * (q >> 1);
-                const int64_t o = static_cast<int64_t>(t) * op.n_out + n;
-                const float y = __fmul_rn(__int2float_rn(acc), s_scale[t]);
-                if (p.y_bf16)
-                    static_cast<__nv_bfloat16 *>(op.Y)[o] = __float2bfloat16_rn(y);
-                else
-                    static_cast<float *>(op.Y)[o] = y;
-                if (op.acc_out) op.acc_out[o] = acc;
+            ++uq;
+        }
+        return;
+    }
+
+    if (warp == kWarpEpi) {
+        // ------------------------------------------------------------ epilogue
+        uint32_t ua = 0;   // projections finished (partial-sum buffer ua % 2, scale slot ua % kChainScaleSlots)
+        for (int j = 0; j < p.n_ops; ++j) {
+            const ChainOpDev &op = p.op[j];
+            int t0, t1;
+            chain_tiles(j, op.n_out >> 4, t0, t1);
+            const int ntile = t1 - t0;
+            if (ntile > 0) {
+                const int ab = static_cast<int>(ua & 1u);
+                const bool ok = mbar_wait_cta(&s_acc_full[ab], (ua >> 1) & 1u, &s_abort, p.status);
+                if (!__all_sync(0xffffffffu, ok)) break;
+                // Scale slot ua % (kChainMaxNb + 2) was written by the
+                // quantisers after the MMA warps released int8 buffer use
+                // ua - nb, which they do only after taking partial-sum buffer
+                // use ua - nb, i.e. after this warp finished projection use
+                // ua - nb - 2 >= ua - kChainMaxNb - 2.
+                const int sc = static_cast<int>(ua % kChainScaleSlots);
+                int *acc_buf = sacc + ab * acc_words;
+                const int per_t = ntile * 16;
+                for (int e = lane; e < T * per_t; e += 32) {
+                    const int t = TM == 1 ? 0 : e / per_t;
+                    const int rem = e - t * per_t;
+                    const int idx = (t * p.tiles_max + (rem >> 4)) * 16 + (rem & 15);
+                    const int v = acc_buf[idx] >> 6;   // the products were 64 times the ternary ones
+                    acc_buf[idx] = 0;
+                    const int64_t o = static_cast<int64_t>(t) * op.n_out + static_cast<int64_t>(t0) * 16 + rem;
+                    const float y = __fmul_rn(__int2float_rn(v), s_scale[sc][t]);
+                    if (p.y_bf16)
+                        static_cast<__nv_bfloat16 *>(op.Y)[o] = __float2bfloat16_rn(y);
+                    else
+                        static_cast<float *>(op.Y)[o] = y;
+                    if (op.acc_out) op.acc_out[o] = v;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_acc_empty[ab]);
+                ++ua;
             }
-            // optional copies of the int8 activations and scales (by the CTA holding share G - 1)
-            if (share == static_cast<int>(G) - 1) {
-                if (op.xq_out) {
-                    for (int i = ctid; i < T * op.k; i += kChainConsumers) {
-                        const int t = i / op.k;
-                        const int e = i - t * op.k, u = (e & 63) >> 2;   // undo the fragment order
-                        op.xq_out[i] = s_xq[t * chain_pitch(op.k) + (e & ~63) + 4 * (4 * (u & 3) + (u >> 2)) + (e & 3)];
+            // count this CTA done with projection j (and, by program order, with every
+            // earlier one): the warp barrier orders every lane's Y stores before the
+            // release.  A release waits until those stores have reached L2, about a
+            // microsecond, so it is issued only when a later projection of the launch
+            // waits for it (the end of the launch orders everything for what follows).
+            __syncwarp();
+            if (p.release && lane == 0)
+                asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(&p.counters[j]), "r"(1u) : "memory");
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------- MMA warps
+    // The ring carries this CTA's shares of all projections back to back; a
+    // stage may end one projection and begin the next.  Each warp meets every
+    // stage once (wait for it, its records of every projection in it, release
+    // it) and every projection once (take its buffers, records, flush, hand
+    // the partial sums to the epilogue).
+    uint32_t cs = 0, cph = 0;   // ring slot of the current stage and the parity of its fill round
+    uint32_t spos = 0;          // stream offset of the current stage
+    bool have = false;          // the current stage has been waited for and not yet released
+    uint32_t ppos = 0;          // stream offset of the next projection's records
+    uint32_t ua = 0;            // projections with rows here (partial-sum buffer ua % 2, int8 buffer ua % nb)
+    bool failed = false;
+    for (int j = 0; j < p.n_ops && !failed; ++j) {
+        const ChainOpDev &op = p.op[j];
+        int t0, t1;
+        chain_tiles(j, op.n_out >> 4, t0, t1);
+        const int ntile = t1 - t0;
+        if (ntile == 0) continue;
+        const int ktiles = op.k >> 6;
+        const uint32_t bytes = static_cast<uint32_t>(ntile) * static_cast<uint32_t>(ktiles) * 256u;
+        const int ab = static_cast<int>(ua & 1u);
+        const int xb = static_cast<int>(ua % static_cast<uint32_t>(p.nb));
+        // the epilogue is done with this partial-sum buffer's previous projection; the int8 activations are
+        // ready (warp 0 waits; the other MMA warps learn it from the barrier, which also orders the
+        // quantisers' shared-memory writes that warp 0 has acquired before their reads)
+        bool ok = true;
+        if (warp == 0) {
+            ok = ua < 2u || mbar_wait_cta(&s_acc_empty[ab], ((ua >> 1) - 1u) & 1u, &s_abort, p.status);
+            ok = ok && mbar_wait_cta(&s_xq_full[xb], (ua / static_cast<uint32_t>(p.nb)) & 1u, &s_abort, p.status);
+        }
+        if (mma_sync_or(!ok)) break;
+        int *acc_buf = sacc + ab * acc_words;
+        // Lane l holds the B fragment of token l / 4 (zero for tokens >= T):
+        // the 16 bytes lane l % 4 needs of each 64-k tile sit contiguously in
+        // the shared row (fragment order), one 16-byte load per record.
+        const int bn = lane >> 2;
+        const bool has_b = bn < T;
+        const uint4 *b_src = reinterpret_cast<const uint4 *>(xqb + static_cast<size_t>(xb) * p.xq_bytes +
+                                                             static_cast<int64_t>(has_b ? bn : 0) * chain_pitch(op.k)) +
+                             (lane & 3);
+        int cur = -1;
+        int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
+        const float inv_kt = 1.0f / static_cast<float>(ktiles);
+        const uint32_t end = ppos + bytes;
+        for (uint32_t pos = ppos; pos < end;) {
+            if (!have) {
+                // warp 0 waits for the stage's data; the bulk copies' writes it has
+                // observed are ordered before the barrier for the other warps
+                const bool okf = warp != 0 || mbar_wait_cta(&s_full[cs], cph, &s_abort, p.status);
+                if (mma_sync_or(!okf)) {
+                    failed = true;
+                    break;
+                }
+                have = true;
+            }
+            const uint32_t seg_end = end < spos + stage_bytes ? end : spos + stage_bytes;
+            // this segment's records: warp w takes the contiguous run [w n / 16, (w + 1) n / 16)
+            const int nrec = static_cast<int>((seg_end - pos) >> 8);
+            const int i0 = (warp * nrec) / kChainMmaWarps, i1 = ((warp + 1) * nrec) / kChainMmaWarps;
+            if (i0 < i1) {
+                const int r0 = static_cast<int>((pos - ppos) >> 8) + i0;   // record index within the CTA's share
+                // r0 / ktiles through the reciprocal (r0 < 2^24: off by at most one, corrected)
+                int tile = __float2int_rz(static_cast<float>(r0) * inv_kt);
+                int kt = r0 - tile * ktiles;
+                if (kt < 0) {
+                    --tile;
+                    kt += ktiles;
+                } else if (kt >= ktiles) {
+                    ++tile;
+                    kt -= ktiles;
+                }
+                const uint2 *rec =
+                    reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(cs) * stage_bytes + (pos - spos)) + lane;
+                int i = i0;
+                while (i < i1) {
+                    if (tile != cur) {
+                        if (cur >= 0) chain_flush<TM>(acc_buf, p.tiles_max, cur, lane, T, acc);
+                        cur = tile;
+                    }
+                    if (i + 4 <= i1 && kt + 4 <= ktiles) {
+                        // four records of one row tile: all loads first, then the MMAs
+                        uint2 w[4];
+                        uint32_t bf[4][4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) w[u] = rec[(i + u) * 32];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const uint4 v = has_b ? b_src[(kt + u) * 4] : make_uint4(0u, 0u, 0u, 0u);
+                            bf[u][0] = v.x;
+                            bf[u][1] = v.y;
+                            bf[u][2] = v.z;
+                            bf[u][3] = v.w;
+                        }
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            uint32_t a4[4];
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) a4[r] = expand_codes_x64(w[u].x, r);
+                            mma_sp_m16n8k64(acc[u], a4, bf[u], w[u].y);
+                        }
+                        i += 4;
+                        kt += 4;
+                    } else {
+                        const uint2 w = rec[i * 32];
+                        uint32_t bf[4], a4[4];
+                        const uint4 v = has_b ? b_src[kt * 4] : make_uint4(0u, 0u, 0u, 0u);
+                        bf[0] = v.x;
+                        bf[1] = v.y;
+                        bf[2] = v.z;
+                        bf[3] = v.w;
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) a4[r] = expand_codes_x64(w.x, r);
+                        mma_sp_m16n8k64(acc[0], a4, bf, w.y);
+                        i += 1;
+                        kt += 1;
+                    }
+                    if (kt == ktiles) {
+                        kt = 0;
+                        ++tile;
                     }
                 }
-                if (op.amax_out && ctid < T) op.amax_out[ctid] = s_amax[ctid];
             }
-            consumer_sync();
+            pos = seg_end;
+            if (pos == spos + stage_bytes) {   // the stage is used up: release it to the producer
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[cs]);
+                have = false;
+                spos += stage_bytes;
+                if (++cs == static_cast<uint32_t>(ns)) {
+                    cs = 0;
+                    cph ^= 1u;
+                }
+            }
         }
-        // 5. count this CTA done with projection j, after projection j - 1 (chain order)
-        bool bad = false;
-        if (ctid == 0) {
-            if (j > 0 && !op.wait_prev) bad = !wait_counter(&p.counters[j - 1], G, p, &s_abort);
-            // release: the consumer barrier above ordered every consumer's Y stores before this add
-            if (!bad) asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(&p.counters[j]), "r"(1u) : "memory");
+        if (failed) break;
+        if (cur >= 0) chain_flush<TM>(acc_buf, p.tiles_max, cur, lane, T, acc);
+        // the shared atomics of every lane are ordered before the release of the arrivals
+        __syncwarp();
+        if (lane == 0) {
+            mbar_arrive(&s_acc_full[ab]);
+            mbar_arrive(&s_xq_empty[xb]);
         }
-        if (j > 0 && !op.wait_prev && consumer_sync_or(bad)) break;
+        ++ua;
+        ppos = end;
+    }
+    if (have && !failed) {   // the stream's last, partly used stage
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[cs]);
     }
 }
 
-size_t chain_smem_bytes(int ns, uint32_t stage_bytes, int64_t T, int64_t kmax) {
-    return static_cast<size_t>(ns) * stage_bytes + static_cast<size_t>(kChainMaxTiles) * 128 * 4 +
-           static_cast<size_t>(T) * static_cast<size_t>(kmax + 128);
-}
+// ---------------------------------------------------------------- host side
 
-// Ring geometry: the largest stage (64, 32 or 16 KB) that leaves three stages
-// (64 KB) or two (smaller) next to the activation rows.  Larger stages mean
-// fewer barrier waits and longer record runs per warp.  False when not even
-// two 16 KB stages fit.
-bool chain_ring(int64_t T, int64_t kmax, int *ns_out, uint32_t *stage_out) {
-    const size_t fixed = chain_smem_bytes(0, 0, T, kmax);
-    if (fixed >= kChainMaxSmem) return false;
-    const uint32_t sizes[3] = {65536u, 32768u, 16384u};
-    const int need[3] = {3, 2, 2};
-    for (int i = 0; i < 3; ++i) {
-        size_t ns = (kChainMaxSmem - fixed) / sizes[i];
-        if (ns > static_cast<size_t>(kChainMaxStages)) ns = kChainMaxStages;
-        if (static_cast<int>(ns) >= need[i]) {
-            *ns_out = static_cast<int>(ns);
-            *stage_out = sizes[i];
+static size_t round128(size_t x) { return (x + 127) / 128 * 128; }
+
+// Shared-memory layout: four staging slots of one activation row each, the
+// most int8 buffers (up to four; exactly four for T < 4, see the quantisers)
+// and a weight ring of at least 128 KB in 32 KB stages; else 96 KB, then a
+// single int8 buffer (T >= 4) and 64 KB, then 16 KB stages, down to two of
+// them.  False when even that does not fit.
+bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayout *L) {
+    if (T < 1 || T > 8 || kmax < 64 || tiles_max < 1 || tiles_max > kChainMaxTiles) return false;
+    const size_t acc = round128(static_cast<size_t>(T) * static_cast<size_t>(tiles_max) * 16 * 4);
+    const size_t xq = round128(static_cast<size_t>(T) * static_cast<size_t>(chain_pitch(kmax)));
+    const size_t xs = static_cast<size_t>(kmax) * (x_bf16 ? 2 : 4);
+    const int nb_lo = T < 4 ? kChainMaxNb : 1;
+    const size_t min_ring[5] = {128 * 1024, 96 * 1024, 64 * 1024, 2 * 32768, 2 * 16384};
+    const uint32_t stage[5] = {32768, 32768, 32768, 32768, 16384};
+    const int min_nb[5] = {2, 2, 1, 1, 1};
+    for (int pass = 0; pass < 5; ++pass) {
+        for (int nb = CHAIN_NB_MAX; nb >= (min_nb[pass] > nb_lo ? min_nb[pass] : nb_lo); --nb) {
+            if (T < 4 && nb != kChainMaxNb) continue;
+            const size_t fixed = 2 * acc + static_cast<size_t>(nb) * xq + kChainQuantWarps * xs;
+            if (fixed >= kChainMaxSmem) continue;
+            size_t ns = (kChainMaxSmem - fixed) / stage[pass];
+            if (ns > static_cast<size_t>(kChainMaxStages)) ns = kChainMaxStages;
+            if (ns < 2 || ns * stage[pass] < min_ring[pass]) continue;
+            L->ns = static_cast<int>(ns);
+            L->stage_bytes = stage[pass];
+            L->nb = nb;
+            L->xq_bytes = static_cast<uint32_t>(xq);
+            L->xs_bytes = static_cast<uint32_t>(xs);
+            L->tiles_max = tiles_max;
+            L->acc_bytes = static_cast<uint32_t>(acc);
+            L->smem = ns * stage[pass] + fixed;
             return true;
         }
     }
@@ -620,9 +766,15 @@ bool chain_ring(int64_t T, int64_t kmax, int *ns_out, uint32_t *stage_out) {
 
 cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
                                 int64_t kmax, void *ws, cudaStream_t s) {
-    int ns = 0;
-    uint32_t stage_bytes = 0;
-    if (!chain_ring(T, kmax, &ns, &stage_bytes)) return cudaErrorInvalidValue;
+    const int G = num_sms();
+    int tiles_max = 1;
+    for (int i = 0; i < n_ops; ++i) {
+        const int rows16 = ops[i].n_out >> 4;
+        const int t = (rows16 + G - 1) / G;
+        tiles_max = t > tiles_max ? t : tiles_max;
+    }
+    ChainLayout L;
+    if (!chain_layout(T, kmax, x_bf16, tiles_max, &L)) return cudaErrorInvalidValue;
     // one-token chains take the instantiation with T folded to 1
     const bool one = T == 1;
     auto kern = x_bf16 ? (one ? k_decode_chain<true, 1> : k_decode_chain<true, 8>)
@@ -639,12 +791,18 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         // a later launch continues the chain: its first projection waits for the previous launch by stream order
         p.op[0].wait_prev = 0;
         p.n_ops = n;
+        p.release = 0;
+        for (int i = 1; i < n; ++i) p.release |= p.op[i].wait_prev != 0 ? 1 : 0;
         p.T = static_cast<int32_t>(T);
         p.x_bf16 = x_bf16 ? 1 : 0;
         p.y_bf16 = y_bf16 ? 1 : 0;
-        p.ns = ns;
-        p.stage_bytes = stage_bytes;
-        p.kmax = static_cast<int32_t>(kmax);
+        p.ns = L.ns;
+        p.stage_bytes = L.stage_bytes;
+        p.nb = L.nb;
+        p.xq_bytes = L.xq_bytes;
+        p.xs_bytes = L.xs_bytes;
+        p.tiles_max = L.tiles_max;
+        p.acc_bytes = L.acc_bytes;
         p.eps = eps;
         p.status = reinterpret_cast<uint32_t *>(w8 + kStatusOffset);
         p.abort = reinterpret_cast<uint32_t *>(w8 + kChainAbortOffset);
@@ -653,9 +811,9 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
                                         kChainCountersOffset - kChainAbortOffset + static_cast<size_t>(n) * 4, s);
         if (e != cudaSuccess) return e;
         cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(static_cast<unsigned>(num_sms()));
+        cfg.gridDim = dim3(static_cast<unsigned>(G));
         cfg.blockDim = dim3(kChainThreads);
-        cfg.dynamicSmemBytes = chain_smem_bytes(ns, stage_bytes, T, kmax);
+        cfg.dynamicSmemBytes = L.smem;
         cfg.stream = s;
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeCooperative;

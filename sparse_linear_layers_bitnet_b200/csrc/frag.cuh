@@ -21,6 +21,15 @@ __device__ __forceinline__ uint32_t expand_codes(uint32_t codes, int r) {
     return (t & 0x02020202u) * 0x7eu + t;
 }
 
+// Codes of register r as int8 values 64 c (c in {-1, 0, 1}): the two code bits
+// moved to bits 6-7 of each byte, the rest cleared (00 -> 0, 01 -> 64,
+// 11 -> -64).  Two instructions instead of four; a product accumulated from
+// these is 64 times the ternary one, exactly (int32 holds 64 * 127 * k / 2
+// for k < 2^18), and an arithmetic shift by 6 recovers it.
+__device__ __forceinline__ uint32_t expand_codes_x64(uint32_t codes, int r) {
+    return (codes << (6 - 2 * r)) & 0xC0C0C0C0u;
+}
+
 __device__ __forceinline__ void mma_sp_m16n8k64(int (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[4],
                                                 uint32_t e) {
     asm volatile(

@@ -81,6 +81,9 @@ cudaError_t launch_adamw_gamma(float *W, const float *G, float *M, float *V, int
                                float eps, float wd, float c1, float c2, float eps_gamma, float *gamma, void *ws,
                                cudaStream_t s);
 
+// Tensor-core instruction throughput ceiling (peak.cu); *ops = dense-equivalent operations of the launch
+cudaError_t launch_tensor_peak(int kind, int64_t iters, uint32_t *status, double *ops, cudaStream_t s);
+
 // Health check of the bounded waits (chain.cu): both kinds of wait run out on events that never happen
 cudaError_t launch_wait_selftest(void *ws, uint64_t limit_ns, cudaStream_t s);
 
@@ -125,11 +128,20 @@ struct ChainOpDev {
 };
 constexpr int kChainMaxOps = 128;                  // projections per launch (kernel parameter space)
 constexpr int kChainMaxTiles = 32;                 // 16-row tiles per CTA per projection
-constexpr size_t kChainMaxSmem = 227 * 1024 - 1024;   // dynamic shared memory (static use < 1 KB)
+constexpr int kChainMaxK = 1 << 17;                // 64 * 127 * k / 2 stays inside int32 (codes expanded x64)
+constexpr size_t kChainMaxSmem = 227 * 1024 - 2048;   // dynamic shared memory (static use < 2 KB)
 constexpr size_t kChainAbortOffset = 4;            // workspace: grid abort word
 constexpr size_t kChainCountersOffset = 256;       // workspace: one counter per projection
-size_t chain_smem_bytes(int ns, uint32_t stage_bytes, int64_t T, int64_t kmax);
-bool chain_ring(int64_t T, int64_t kmax, int *ns, uint32_t *stage_bytes);
+// Shared-memory layout of one chain launch (chain.cu).
+struct ChainLayout {
+    int ns;               // weight ring stages
+    uint32_t stage_bytes; // bytes of one stage
+    int nb;               // int8 activation buffers
+    int tiles_max;        // most row tiles one CTA takes of one projection
+    uint32_t xq_bytes, xs_bytes, acc_bytes;
+    size_t smem;          // dynamic shared memory of the launch
+};
+bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayout *L);
 cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
                                 int64_t kmax, void *ws, cudaStream_t s);
 
