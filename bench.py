@@ -426,7 +426,11 @@ def measure_mma_ceilings(torch, bn, secs=1.0, iters=20000):
     out = {}
     forms = ((0, "sparse_i8_mma_loop_tops", "tcgen05.mma.sp.cta_group::2.kind::i8 M256 N224 K64"),
              (1, "dense_i8_mma_loop_tops", "tcgen05.mma.cta_group::2.kind::i8 M256 N256 K32"),
-             (2, "bf16_mma_loop_tflops", "tcgen05.mma.cta_group::2.kind::f16 (bf16) M256 N256 K16"))
+             (2, "bf16_mma_loop_tflops", "tcgen05.mma.cta_group::2.kind::f16 (bf16) M256 N256 K16"),
+             (3, "sparse_i8_mma_loop_meta_copy_tops", "as the sparse loop, with each stage's metadata copied into "
+                                                     "TMEM (tcgen05.cp) right before its two MMAs, two slots"),
+             (4, "sparse_i8_mma_loop_meta_ahead_tops", "as the sparse loop, with each metadata copy issued four "
+                                                      "stages ahead of its MMAs, eight slots"))
     for kind, name, form in forms:
         for _ in range(3):
             bn.bitnet_tensor_peak(kind, iters, ws)

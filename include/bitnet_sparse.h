@@ -549,7 +549,10 @@ bitnet_status bitnet_wait_selftest(void *ws, size_t ws_bytes, int32_t limit_us, 
  *   kind 0  tcgen05.mma.sp.cta_group::2.kind::i8, M 256, N 224, K 64 (the
  *           2:4-sparse int8 instruction of the prefill GEMM);
  *   kind 1  tcgen05.mma.cta_group::2.kind::i8, M 256, N 256, K 32 (dense int8);
- *   kind 2  tcgen05.mma.cta_group::2.kind::f16 (bf16), M 256, N 256, K 16.
+ *   kind 2  tcgen05.mma.cta_group::2.kind::f16 (bf16), M 256, N 256, K 16;
+ *   kind 3  kind 0 with each stage's 2:4 metadata copied into TMEM
+ *           (tcgen05.cp) right before the stage's two MMAs, two slots;
+ *   kind 4  kind 3 with every copy issued four stages ahead, eight slots.
  *   iters   MMAs per CTA pair (rounded up to a whole stage), >= 1.
  *   ops     host pointer; receives the dense-equivalent operations of the
  *           launch, 2 M N K per MMA summed over the pairs (time the launch on

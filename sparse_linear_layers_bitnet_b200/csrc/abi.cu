@@ -488,9 +488,11 @@ bitnet_status bitnet_decode_chain(const bitnet_chain_op *ops, int32_t n_ops, int
         dev[static_cast<size_t>(i)] = {o.X, W->dec_codes, W->gamma, o.Y, o.acc_out, o.xq_out, o.absmax_out,
                                        static_cast<int32_t>(W->n_out), static_cast<int32_t>(W->k), o.wait_prev, 0};
     }
-    if (!chain_fits(T, kmax, x_dtype == BITNET_BF16, nmax))
-        return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: one activation row of the largest k, the int8 activations "
-                                            "and two weight stages do not fit in shared memory");
+    bool any_wait = false;
+    for (int32_t i = 1; i < n_ops; ++i) any_wait = any_wait || ops[i].wait_prev != 0;
+    if (any_wait ? !bitnet::chain_serial_fits(T, kmax) : !chain_fits(T, kmax, x_dtype == BITNET_BF16, nmax))
+        return fail(BITNET_ERR_UNSUPPORTED, "decode_chain: the activations of the largest k and two weight stages do "
+                                            "not fit in shared memory");
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return cuda_status(bitnet::launch_decode_chain(dev.data(), n_ops, T, x_dtype == BITNET_BF16, y_dtype == BITNET_BF16,
                                                    eps, kmax, ws, s),
@@ -530,7 +532,7 @@ bitnet_status bitnet_wait_selftest(void *ws, size_t ws_bytes, int32_t limit_us, 
 
 bitnet_status bitnet_tensor_peak(int32_t kind, int64_t iters, double *ops, void *ws, size_t ws_bytes,
                                  bitnet_stream_t stream) {
-    if (kind < 0 || kind > 2) return fail(BITNET_ERR_INVALID_ARG, "tensor_peak: kind must be 0, 1 or 2");
+    if (kind < 0 || kind > 4) return fail(BITNET_ERR_INVALID_ARG, "tensor_peak: kind must be 0 .. 4");
     if (iters < 1 || iters > (int64_t(1) << 40)) return fail(BITNET_ERR_INVALID_ARG, "tensor_peak: iters must be in [1, 2^40]");
     if (!ops) return fail(BITNET_ERR_INVALID_ARG, "tensor_peak: ops is required");
     if (!ws) return fail(BITNET_ERR_WORKSPACE, "tensor_peak: workspace is required");

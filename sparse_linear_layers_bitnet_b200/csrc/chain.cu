@@ -52,6 +52,8 @@
 // reaches the grid size or an abort raised by another CTA ends every role of
 // the kernel with the timeout bit in the status word; outstanding copies are
 // waited for (bounded) before the copy threads exit.
+#include <cstring>
+
 #include "../../include/bitnet_sparse.h"
 #include "common.cuh"
 #include "frag.cuh"
@@ -59,7 +61,10 @@
 
 namespace bitnet {
 
-constexpr int kChainMmaWarps = 16;
+#ifndef CHAIN_MMA_WARPS
+#define CHAIN_MMA_WARPS 16
+#endif
+constexpr int kChainMmaWarps = CHAIN_MMA_WARPS;
 constexpr int kChainQuantWarps = 4;
 constexpr int kChainQuantThreads = kChainQuantWarps * 32;
 constexpr int kWarpQuant0 = kChainMmaWarps;                 // first quantiser warp
@@ -77,7 +82,8 @@ struct ChainParams {
     int32_t n_ops, T, x_bf16, y_bf16;
     int32_t ns;                // weight ring stages
     uint32_t stage_bytes;      // 32 or 16 KB
-    int32_t nb;                // int8 activation buffers (1 .. kChainMaxNb)
+    int32_t nb;                // int8 activation buffers: 1, 2 or 4
+    int32_t nb_log2;
     uint32_t xq_bytes;         // one int8 buffer: T rows of pitch chain_pitch(kmax)
     uint32_t xs_bytes;         // one staging slot: one activation row of kmax elements
     int32_t tiles_max;         // most row tiles a CTA takes of one projection
@@ -282,6 +288,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     __shared__ __align__(8) uint64_t s_xq_full[kChainMaxNb], s_xq_empty[kChainMaxNb];
     __shared__ __align__(8) uint64_t s_acc_full[2], s_acc_empty[2];
     __shared__ float s_gamma[kChainMaxOps];
+    __shared__ int2 s_tiles[kChainMaxOps];    // this CTA's row tiles [x, y) of every projection
+    __shared__ int s_share[kChainMaxOps];     // and its share index
     __shared__ float s_scale[kChainScaleSlots][8];
     __shared__ float s_amax[kChainScaleSlots][8];
     __shared__ int s_abort;
@@ -299,6 +307,12 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     const int acc_words = static_cast<int>(p.acc_bytes >> 2);
 
     for (int i = tid; i < 2 * acc_words; i += kChainThreads) sacc[i] = 0;
+    // every projection's share of this CTA, once (each role reads the table instead of dividing)
+    for (int i = tid; i < p.n_ops; i += kChainThreads) {
+        int t0, t1;
+        s_share[i] = chain_tiles(i, p.op[i].n_out >> 4, t0, t1);
+        s_tiles[i] = make_int2(t0, t1);
+    }
     if (tid == 0) {
         s_abort = 0;
         for (int s = 0; s < ns; ++s) {
@@ -335,8 +349,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         bool open = false, ok = true;
         for (int j = 0; j < p.n_ops && ok; ++j) {
             const ChainOpDev &op = p.op[j];
-            int t0, t1;
-            chain_tiles(j, op.n_out >> 4, t0, t1);
+            const int t0 = s_tiles[j].x, t1 = s_tiles[j].y;
             const uint32_t tile_bytes = static_cast<uint32_t>(op.k >> 6) * 256u;
             const uint32_t bytes = static_cast<uint32_t>(t1 - t0) * tile_bytes;
             const uint8_t *src = op.dec + static_cast<size_t>(t0) * tile_bytes;
@@ -398,8 +411,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         bool ok = true;
         for (int j = 0; j < p.n_ops && ok; ++j) {
             const ChainOpDev &op = p.op[j];
-            int t0, t1;
-            chain_tiles(j, op.n_out >> 4, t0, t1);
+            const int t0 = s_tiles[j].x, t1 = s_tiles[j].y;
             if (t1 == t0) continue;   // no rows here: the activations are not needed
             if (j > 0 && op.wait_prev) {
                 // every CTA has finished projection j - 1 (and, in chain order, all before it)
@@ -456,11 +468,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         bool failed = false;
         for (int j = 0; j < p.n_ops && !failed; ++j) {
             const ChainOpDev &op = p.op[j];
-            int t0, t1;
-            const int share = chain_tiles(j, op.n_out >> 4, t0, t1);
+            const int t0 = s_tiles[j].x, t1 = s_tiles[j].y;
+            const int share = s_share[j];
             if (t1 == t0) continue;
-            const int xb = static_cast<int>(uq % nbu);
-            const uint32_t xround = uq / nbu;
+            const int xb = static_cast<int>(uq & (nbu - 1u));
+            const uint32_t xround = uq >> p.nb_log2;
             const int sc = static_cast<int>(uq % kChainScaleSlots);
             const int k = op.k;
             const int pitch = static_cast<int>(chain_pitch(k));
@@ -528,8 +540,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         uint32_t ua = 0;   // projections finished (partial-sum buffer ua % 2, scale slot ua % kChainScaleSlots)
         for (int j = 0; j < p.n_ops; ++j) {
             const ChainOpDev &op = p.op[j];
-            int t0, t1;
-            chain_tiles(j, op.n_out >> 4, t0, t1);
+            const int t0 = s_tiles[j].x, t1 = s_tiles[j].y;
             const int ntile = t1 - t0;
             if (ntile > 0) {
                 const int ab = static_cast<int>(ua & 1u);
@@ -587,21 +598,20 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     bool failed = false;
     for (int j = 0; j < p.n_ops && !failed; ++j) {
         const ChainOpDev &op = p.op[j];
-        int t0, t1;
-        chain_tiles(j, op.n_out >> 4, t0, t1);
+        const int t0 = s_tiles[j].x, t1 = s_tiles[j].y;
         const int ntile = t1 - t0;
         if (ntile == 0) continue;
         const int ktiles = op.k >> 6;
         const uint32_t bytes = static_cast<uint32_t>(ntile) * static_cast<uint32_t>(ktiles) * 256u;
         const int ab = static_cast<int>(ua & 1u);
-        const int xb = static_cast<int>(ua % static_cast<uint32_t>(p.nb));
+        const int xb = static_cast<int>(ua & static_cast<uint32_t>(p.nb - 1));
         // the epilogue is done with this partial-sum buffer's previous projection; the int8 activations are
         // ready (warp 0 waits; the other MMA warps learn it from the barrier, which also orders the
         // quantisers' shared-memory writes that warp 0 has acquired before their reads)
         bool ok = true;
         if (warp == 0) {
             ok = ua < 2u || mbar_wait_cta(&s_acc_empty[ab], ((ua >> 1) - 1u) & 1u, &s_abort, p.status);
-            ok = ok && mbar_wait_cta(&s_xq_full[xb], (ua / static_cast<uint32_t>(p.nb)) & 1u, &s_abort, p.status);
+            ok = ok && mbar_wait_cta(&s_xq_full[xb], (ua >> p.nb_log2) & 1u, &s_abort, p.status);
         }
         if (mma_sync_or(!ok)) break;
         int *acc_buf = sacc + ab * acc_words;
@@ -615,7 +625,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                              (lane & 3);
         int cur = -1;
         int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
-        const float inv_kt = 1.0f / static_cast<float>(ktiles);
+        const float inv_kt = __int_as_float(op.pad);   // 1 / ktiles, formed on the host
         const uint32_t end = ppos + bytes;
         for (uint32_t pos = ppos; pos < end;) {
             if (!have) {
@@ -743,7 +753,7 @@ bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayo
     const uint32_t stage[5] = {32768, 32768, 32768, 32768, 16384};
     const int min_nb[5] = {2, 2, 1, 1, 1};
     for (int pass = 0; pass < 5; ++pass) {
-        for (int nb = CHAIN_NB_MAX; nb >= (min_nb[pass] > nb_lo ? min_nb[pass] : nb_lo); --nb) {
+        for (int nb = CHAIN_NB_MAX; nb >= (min_nb[pass] > nb_lo ? min_nb[pass] : nb_lo); nb >>= 1) {
             if (T < 4 && nb != kChainMaxNb) continue;
             const size_t fixed = 2 * acc + static_cast<size_t>(nb) * xq + kChainQuantWarps * xs;
             if (fixed >= kChainMaxSmem) continue;
@@ -766,6 +776,11 @@ bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayo
 
 cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
                                 int64_t kmax, void *ws, cudaStream_t s) {
+    // A projection that waits for its predecessor makes the chain latency-bound:
+    // such chains take the kernel of chain_serial.cu, whose path from one
+    // projection to the next has no hand-over between warp roles.
+    for (int i = 1; i < n_ops; ++i)
+        if (ops[i].wait_prev) return launch_decode_chain_serial(ops, n_ops, T, x_bf16, y_bf16, eps, kmax, ws, s);
     const int G = num_sms();
     int tiles_max = 1;
     for (int i = 0; i < n_ops; ++i) {
@@ -787,7 +802,13 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
     for (int base = 0; base < n_ops; base += kChainMaxOps) {
         const int n = (n_ops - base) < kChainMaxOps ? (n_ops - base) : kChainMaxOps;
         ChainParams p;
-        for (int i = 0; i < n; ++i) p.op[i] = ops[base + i];
+        for (int i = 0; i < n; ++i) {
+            p.op[i] = ops[base + i];
+            // 1 / (k / 64) for the record-to-tile division on the device (r / ktiles via a float
+            // product, corrected there); formed here in IEEE fp32
+            const float inv_kt = 1.0f / static_cast<float>(p.op[i].k >> 6);
+            std::memcpy(&p.op[i].pad, &inv_kt, 4);
+        }
         // a later launch continues the chain: its first projection waits for the previous launch by stream order
         p.op[0].wait_prev = 0;
         p.n_ops = n;
@@ -799,6 +820,7 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         p.ns = L.ns;
         p.stage_bytes = L.stage_bytes;
         p.nb = L.nb;
+        p.nb_log2 = L.nb == 4 ? 2 : (L.nb == 2 ? 1 : 0);
         p.xq_bytes = L.xq_bytes;
         p.xs_bytes = L.xs_bytes;
         p.tiles_max = L.tiles_max;

@@ -129,7 +129,7 @@ struct ChainOpDev {
 constexpr int kChainMaxOps = 128;                  // projections per launch (kernel parameter space)
 constexpr int kChainMaxTiles = 32;                 // 16-row tiles per CTA per projection
 constexpr int kChainMaxK = 1 << 17;                // 64 * 127 * k / 2 stays inside int32 (codes expanded x64)
-constexpr size_t kChainMaxSmem = 227 * 1024 - 2048;   // dynamic shared memory (static use < 2 KB)
+constexpr size_t kChainMaxSmem = 227 * 1024 - 3072;   // dynamic shared memory (static use < 3 KB)
 constexpr size_t kChainAbortOffset = 4;            // workspace: grid abort word
 constexpr size_t kChainCountersOffset = 256;       // workspace: one counter per projection
 // Shared-memory layout of one chain launch (chain.cu).
@@ -142,6 +142,10 @@ struct ChainLayout {
     size_t smem;          // dynamic shared memory of the launch
 };
 bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayout *L);
+// The latency-oriented chain for projections that wait for their predecessor (chain_serial.cu).
+bool chain_serial_fits(int64_t T, int64_t kmax);
+cudaError_t launch_decode_chain_serial(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
+                                       int64_t kmax, void *ws, cudaStream_t s);
 cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
                                 int64_t kmax, void *ws, cudaStream_t s);
 

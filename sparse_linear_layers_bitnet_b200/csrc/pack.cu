@@ -577,18 +577,18 @@ __global__ void __launch_bounds__(256) k_pack_finish(UpdateArgs u) {
 // path: magnitudes in [2^-20, 2) are integer multiples of 2^-43, and up to
 // 2^10 / 2^-43 = 2^53 units (fewer than 512 of them) add exactly in fp64; the
 // per-lane fp64 sum is moved into the 128-bit integer accumulator (units of
-// 2^-54) once per round.  Zeros need no work; every other magnitude takes the
-// exact path of accumulate_abs.
-
-__device__ __forceinline__ bool fast_mag(uint32_t a) {
-    return a == 0u || (a - 0x35800000u) < (0x40000000u - 0x35800000u);   // 0 or [2^-20, 2)
-}
+// 2^-54) once per round.  A group with any other magnitude (a zero included)
+// takes the exact path of accumulate_abs.
 
 __device__ __forceinline__ void sum_float4(const float4 v, double &d, uint64_t &lo, uint64_t &hi,
                                            unsigned long long *s_bins, int *s_rare) {
     const uint32_t a0 = __float_as_uint(v.x) & 0x7fffffffu, a1 = __float_as_uint(v.y) & 0x7fffffffu;
     const uint32_t a2 = __float_as_uint(v.z) & 0x7fffffffu, a3 = __float_as_uint(v.w) & 0x7fffffffu;
-    if (fast_mag(a0) && fast_mag(a1) && fast_mag(a2) && fast_mag(a3)) {
+    // all four magnitudes in [2^-20, 2): the smallest and the largest bit pattern
+    // decide it (non-negative floats order like their bits); anything else,
+    // zeros included, takes the exact path below
+    const uint32_t mn = min(min(a0, a1), min(a2, a3)), mx = max(max(a0, a1), max(a2, a3));
+    if (mn >= 0x35800000u && mx < 0x40000000u) {
         d += static_cast<double>(__uint_as_float(a0));
         d += static_cast<double>(__uint_as_float(a1));
         d += static_cast<double>(__uint_as_float(a2));

@@ -81,11 +81,14 @@ __device__ __forceinline__ void commit_both(uint64_t *bar) {
 //   kind 0: 2:4-sparse int8, N = 224, K = 64 logical (32 stored bytes of A per row), two per 128-k stage
 //   kind 1: dense int8, N = 256, K = 32, four per 128-byte stage
 //   kind 2: dense bf16, N = 256, K = 16, four per 128-byte stage
+//   kind 3: kind 0 with the stage's metadata copied into TMEM (tcgen05.cp) right before its two MMAs,
+//           in a ring of two slots, as a GEMM stage does
+//   kind 4: kind 3 with each copy issued four stages ahead of its MMAs (ring of eight slots)
 struct PeakForm {
     int n, k, per_stage;
 };
 __host__ __device__ constexpr PeakForm peak_form(int kind) {
-    return kind == 0 ? PeakForm{224, 64, 2} : (kind == 1 ? PeakForm{256, 32, 4} : PeakForm{256, 16, 4});
+    return (kind == 0 || kind >= 3) ? PeakForm{224, 64, 2} : (kind == 1 ? PeakForm{256, 32, 4} : PeakForm{256, 16, 4});
 }
 
 constexpr int kPeakABytes = 128 * 128;   // 128 rows x 128 bytes (sparse: 64 used per row)
@@ -97,7 +100,8 @@ template <int KIND>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1) k_tensor_peak(int64_t iters, uint32_t *status) {
     constexpr PeakForm F = peak_form(KIND);
     // s32 (kinds 0, 1) or f32 (kind 2) accumulators; s8 / bf16 operands; M = 256, N = F.n
-    constexpr uint32_t kIdesc = (KIND == 0 ? (1u << 2) : 0u) | ((KIND == 2 ? 1u : 2u) << 4) | (1u << 7) | (1u << 10) |
+    constexpr bool kSparse = KIND == 0 || KIND >= 3;
+    constexpr uint32_t kIdesc = (kSparse ? (1u << 2) : 0u) | ((KIND == 2 ? 1u : 2u) << 4) | (1u << 7) | (1u << 10) |
                                 (static_cast<uint32_t>(F.n >> 3) << 17) | (static_cast<uint32_t>(256 >> 4) << 24);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -138,15 +142,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1) k_tensor_pea
     if (leader && warp == 0 && lane == 0) {
         const uint32_t a_base = smem_u32(sA), b_base = smem_u32(sB);
         const uint32_t e_col = tmem + 256;
-        if (KIND == 0) peak::tmem_cp2_128x128b(e_col, make_smem_desc(smem_u32(sE), 16, 128, kSwizzleNone));
-        for (int64_t it = 0; it < iters; it += F.per_stage) {
+        const uint64_t e_desc = make_smem_desc(smem_u32(sE), 16, 128, kSwizzleNone);
+        if (KIND == 0) peak::tmem_cp2_128x128b(e_col, e_desc);
+        if (KIND == 4)
+            for (int q = 0; q < 4; ++q) peak::tmem_cp2_128x128b(e_col + 4u * q, e_desc);
+        for (int64_t it = 0, st = 0; it < iters; it += F.per_stage, ++st) {
+            uint32_t e_stage = e_col;
+            if (KIND == 3) {   // this stage's metadata, then its MMAs
+                e_stage = e_col + 4u * static_cast<uint32_t>(st & 1);
+                peak::tmem_cp2_128x128b(e_stage, e_desc);
+            } else if (KIND == 4) {   // stage st + 4's metadata, then stage st's MMAs
+                e_stage = e_col + 4u * static_cast<uint32_t>(st & 7);
+                peak::tmem_cp2_128x128b(e_col + 4u * static_cast<uint32_t>((st + 4) & 7), e_desc);
+            }
 #pragma unroll
             for (int j = 0; j < F.per_stage; ++j) {
                 const uint32_t acc = (it | j) != 0;
-                if (KIND == 0) {
+                if (kSparse) {
                     const uint64_t ad = make_smem_desc(a_base + j * 32, 16, 512, kSwizzle64B);
                     const uint64_t bd = make_smem_desc(b_base + j * 64, 16, 1024, kSwizzle128B);
-                    peak::mma_sp_i8_2(tmem, ad, bd, kIdesc, e_col + 2u * j, acc);
+                    peak::mma_sp_i8_2(tmem, ad, bd, kIdesc, e_stage + 2u * j, acc);
                 } else if (KIND == 1) {
                     const uint64_t ad = make_smem_desc(a_base + j * 32, 16, 1024, kSwizzle128B);
                     const uint64_t bd = make_smem_desc(b_base + j * 32, 16, 1024, kSwizzle128B);
@@ -177,7 +192,9 @@ cudaError_t launch_tensor_peak(int kind, int64_t iters, uint32_t *status, double
     const PeakForm F = peak_form(kind);
     const int64_t per = (iters + F.per_stage - 1) / F.per_stage * F.per_stage;   // MMAs per pair
     *ops = 2.0 * 256.0 * F.n * F.k * static_cast<double>(per) * (ctas / 2);
-    auto kern = kind == 0 ? k_tensor_peak<0> : (kind == 1 ? k_tensor_peak<1> : k_tensor_peak<2>);
+    auto kern = kind == 0 ? k_tensor_peak<0>
+                          : (kind == 1 ? k_tensor_peak<1>
+                                       : (kind == 2 ? k_tensor_peak<2> : (kind == 3 ? k_tensor_peak<3> : k_tensor_peak<4>)));
     cudaError_t e = smem_attr(reinterpret_cast<const void *>(kern), kPeakSmem);
     if (e != cudaSuccess) return e;
     kern<<<dim3(static_cast<unsigned>(ctas)), 128, kPeakSmem, s>>>(per, status);
