@@ -56,9 +56,10 @@ def parse_args():
     ap.add_argument("--preroll-s", type=float, default=1.0, help="untimed warm-up seconds before timing")
     ap.add_argument("--tokens", type=int, default=1, help="decode batch (1..8)")
     ap.add_argument("--layers", type=int, default=30)
-    ap.add_argument("--decode", choices=["chain", "fused", "unfused"], default="chain",
-                    help="decode step: one persistent launch for all projections (chain), one fused "
-                         "quant+GEMV launch per projection (fused), or quant_act + GEMV per projection")
+    ap.add_argument("--decode", choices=["chain_independent", "chain", "fused", "unfused"], default="chain_independent",
+                    help="decode step: one persistent launch for all projections, independent of each other "
+                         "(chain_independent) or each waiting for the previous one (chain); one fused quant+GEMV "
+                         "launch per projection (fused); or quant_act + GEMV per projection (unfused)")
     ap.add_argument("--no-rows", action="store_true", help="skip the sub-measurements of the other rows")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle baseline")
     ap.add_argument("--pack-layers", type=int, default=None, help="layers of the pack workload (default: all 26)")
@@ -1149,7 +1150,7 @@ def run_ours(args):
     assert 1 <= T <= 8, "decode batch must be 1..8"
     dev_index = torch.cuda.current_device()
 
-    fused = args.decode in ("chain", "fused")
+    fused = args.decode in ("chain", "chain_independent", "fused")
     dec = Decode(torch, bn, synth, T, args.layers, seed_base=info.rank * 7919, mode=args.decode)
     g_step = dec.capture(dec.step)
 
@@ -1176,7 +1177,7 @@ def run_ours(args):
     if fused:
         # every kernel launch of the step is the decode chain kernel: its average
         # launch duration is the timed region over the launches in it
-        roof_kernel = "k_decode_chain"
+        roof_kernel = "k_decode_chain_serial" if args.decode == "chain" else "k_decode_chain"
         gemv_ms_per_launch = ms_total / args.steps / dec.launches_per_step
         gemv_bytes_per_launch = dec.step_bytes / dec.launches_per_step
     else:
@@ -1194,7 +1195,9 @@ def run_ours(args):
         gemv_bytes_per_launch = dec.gemv_bytes_per_layer / len(dec.mats)
         del g_gemv
     achieved = gemv_bytes_per_launch / (gemv_ms_per_launch / 1e3) / 1e9
-    traffic = ncu_traffic(roof_kernel, ["chain.cu", "frag.cuh"] if fused else ["gemv.cu", "frag.cuh"])
+    traffic = ncu_traffic(roof_kernel, {"k_decode_chain": ["chain.cu", "frag.cuh"],
+                                        "k_decode_chain_serial": ["chain_serial.cu", "frag.cuh"]}.get(
+                                            roof_kernel, ["gemv.cu", "frag.cuh"]))
 
     # end to end: activations from pinned host memory, outputs back to host
     x_host = torch.empty(dec.x_flat.shape, dtype=dec.x_flat.dtype, pin_memory=True)
@@ -1248,7 +1251,11 @@ def run_ours(args):
         "config": {"workload": f"decode GEMV, 2B LLaMA-alike (hidden 2560, FFN 6912), {args.layers} layers, batch {T}",
                    "tokens": T, "layers": args.layers,
                    "projections": [f"{n} {K}->{N}" for n, K, N in dec.mats],
-                   "step": {"chain": "all projections of all layers in one persistent launch "
+                   "step": {"chain_independent": "all projections of all layers in one persistent launch "
+                                                 "(bitnet_decode_chain, no projection waiting for another: per "
+                                                 "projection, int8 act quant + sparse ternary GEMV, each on its own "
+                                                 "synthetic activations), CUDA graph",
+                            "chain": "all projections of all layers in one persistent launch "
                                      "(bitnet_decode_chain: per projection, int8 act quant + sparse ternary GEMV; "
                                      "each projection waits for the previous one), CUDA graph",
                             "fused": "per layer and projection: one fused launch (bitnet_quant_linear), CUDA graph",

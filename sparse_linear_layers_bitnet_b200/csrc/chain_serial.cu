@@ -362,7 +362,7 @@ __device__ void chain_quantise(const uint4 *__restrict__ X, int T, int k, float 
 }
 
 template <bool XBF16, int TM>
-__global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_constant__ ChainParams p) {
+__global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain_serial(const __grid_constant__ ChainParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kChainMaxStages], s_empty[kChainMaxStages];
     __shared__ float s_red[kChainConsumerWarps][8];
@@ -628,8 +628,8 @@ cudaError_t launch_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf1
     if (!chain_ring(T, kmax, &ns, &stage_bytes)) return cudaErrorInvalidValue;
     // one-token chains take the instantiation with T folded to 1
     const bool one = T == 1;
-    auto kern = x_bf16 ? (one ? k_decode_chain<true, 1> : k_decode_chain<true, 8>)
-                       : (one ? k_decode_chain<false, 1> : k_decode_chain<false, 8>);
+    auto kern = x_bf16 ? (one ? k_decode_chain_serial<true, 1> : k_decode_chain_serial<true, 8>)
+                       : (one ? k_decode_chain_serial<false, 1> : k_decode_chain_serial<false, 8>);
     {
         cudaError_t e = smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(kSerialMaxSmem));
         if (e != cudaSuccess) return e;

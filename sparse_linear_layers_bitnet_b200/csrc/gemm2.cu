@@ -129,28 +129,21 @@ __device__ __forceinline__ void commit_both(uint64_t *bar) {
 // of 64 k-rows, 128-byte swizzled; the descriptors step 8 KB between 64-wide
 // boxes (leading byte offset) and 1 KB between groups of 8 k-rows (stride byte
 // offset).  The other operand stays K-major.
-// MSUB (sparse only): 256-row sub-tiles of A per pair tile.  With 2 the pair
-// computes a 512 x BN tile: both sub-tiles' MMAs read the same B stage, so each
-// B byte staged in shared memory feeds twice the MMAs, at the price of a single
-// accumulator set (2 x BN columns + metadata fill TMEM): the epilogue of one
-// tile is not overlapped with the next tile's main loop.
-template <bool SPARSE, int BN, int STAGES, int MN = 0, int MSUB = 1>
+template <bool SPARSE, int BN, int STAGES, int MN = 0>
 struct PairCfg {
     static constexpr int kHalfN = BN / 2;                  // B rows per CTA
     static constexpr int kARowBytes = SPARSE ? 64 : 128;
     static constexpr int kBRowBytes = 128;
     static constexpr int kKStep = SPARSE ? 128 : 64;
-    static constexpr int kASubBytes = 128 * kARowBytes;   // one sub-tile's 128 rows of A in this CTA
-    static constexpr int kABytes = MSUB * kASubBytes;
+    static constexpr int kABytes = 128 * kARowBytes;
     static constexpr int kBBytes = kHalfN * kBRowBytes;
-    static constexpr int kEBytes = SPARSE ? MSUB * 2048 : 0;
+    static constexpr int kEBytes = SPARSE ? 2048 : 0;
     static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;   // per CTA
     static constexpr int kMmaPerStage = SPARSE ? 2 : 4;
     static constexpr int kAAdvance = 32;
     static constexpr int kBAdvance = SPARSE ? 64 : 32;
-    static constexpr int kNumAcc = MSUB == 2 ? 1 : 2;     // accumulator sets (double-buffered with one sub-tile)
-    static constexpr int kAccStride = 256;                // TMEM columns between accumulators (sets or sub-tiles)
-    static constexpr int kECol = MSUB == 2 ? 2 * kAccStride - 32 : 2 * kAccStride - 16;   // metadata: 8 columns per sub-tile
+    static constexpr int kAccStride = 256;                // TMEM columns between the two accumulators
+    static constexpr int kECol = 2 * kAccStride - 16;     // metadata columns (8 used)
     static constexpr int kTmemCols = 512;
     static constexpr int kStageOutBytes = SPARSE ? 2 * 16 * 128 * 4 : 0;   // two [16 tokens][128 rows] fp32 chunks
     static constexpr int kSmemBytes = STAGES * kStageBytes + kStageOutBytes + 1024 + 2048;
@@ -164,7 +157,6 @@ struct PairCfg {
     static_assert(SPARSE || (BN % 32 == 0 && BN <= 256), "dense pair tiles: N multiple of 32");
     static_assert(kBBytes % 1024 == 0, "B tile must keep the 128-byte swizzle atoms aligned");
     static_assert(!MN || (!SPARSE && (!(MN & 2) || kHalfN % 64 == 0)), "MN-major tiles: dense, whole 64-wide boxes");
-    static_assert(MSUB == 1 || (SPARSE && BN <= 224 && !MN), "two sub-tiles: sparse, N <= 224");
 };
 
 struct PairParams {
@@ -180,12 +172,11 @@ struct PairParams {
     int accumulate;              // dense fp32 output: out += result (else out = result)
 };
 
-template <bool SPARSE, int BN, int STAGES, int MN = 0, int MSUB = 1>
+template <bool SPARSE, int BN, int STAGES, int MN = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     k_umma_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY, PairParams p) {
-    using C = PairCfg<SPARSE, BN, STAGES, MN, MSUB>;
-    constexpr int kTileM = 256 * MSUB;
+    using C = PairCfg<SPARSE, BN, STAGES, MN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = smem;
@@ -204,7 +195,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     const uint32_t rank = pair::cta_rank();
     const bool leader = rank == 0;
     const int64_t pair_id = blockIdx.x >> 1, pairs = gridDim.x >> 1;
-    const int64_t m_tiles = (p.M + kTileM - 1) / kTileM, n_tiles = (p.N + BN - 1) / BN;
+    const int64_t m_tiles = (p.M + 255) / 256, n_tiles = (p.N + BN - 1) / BN;
     const int64_t tiles = m_tiles * n_tiles;
     const int ktiles = static_cast<int>((p.K + C::kKStep - 1) / C::kKStep);
 
@@ -240,26 +231,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
             int it = 0;
             for (int64_t t = pair_id; t < tiles && !*s_abort; t += pairs) {
                 const int64_t mt = t / n_tiles, nt = t - mt * n_tiles;
-                const int32_t a_row = static_cast<int32_t>(mt * kTileM + 128 * rank);
+                const int32_t a_row = static_cast<int32_t>(mt * 256 + 128 * rank);
                 const int32_t b_row = static_cast<int32_t>(nt * BN + C::kHalfN * rank);
+                // metadata rows past the padded end (a ragged last pair) read a valid block:
+                // their A rows are zero-filled, so any valid index pattern gives zero
+                int64_t e_row = mt * 256 + 128 * rank;
+                if (e_row > p.meta_rows - 128) e_row = p.meta_rows - 128;
                 for (int kt = 0; kt < ktiles; ++kt, ++it) {
                     const int s = it % STAGES;
                     if (it >= STAGES && !mbar_wait_bounded(&empty[s], ((it / STAGES) - 1) & 1, s_abort, p.status))
                         break;
                     if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
                     if (SPARSE) {
-#pragma unroll
-                        for (int sub = 0; sub < MSUB; ++sub) {
-                            // metadata rows past the padded end (a ragged last tile) read a valid block:
-                            // their A rows are zero-filled, so any valid index pattern gives zero
-                            int64_t e_row = static_cast<int64_t>(a_row) + 256 * sub;
-                            if (e_row > p.meta_rows - 128) e_row = p.meta_rows - 128;
-                            pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes + sub * C::kASubBytes,
-                                                   kt * (C::kKStep / 2), a_row + 256 * sub);
-                            pair::tma_load_2d_pair(&tmE, &full[s], sE + s * C::kEBytes + sub * 2048, 0,
-                                                   static_cast<int32_t>((kt * p.meta_rows + e_row) / 8));
-                        }
+                        pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * (C::kKStep / 2), a_row);
                         pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
+                        pair::tma_load_2d_pair(&tmE, &full[s], sE + s * C::kEBytes, 0,
+                                               static_cast<int32_t>((kt * p.meta_rows + e_row) / 8));
                     } else if (MN) {
                         // MN-major: boxes of 64 MN-elements x 64 k-rows (two for A's 128 rows, kHalfN / 64
                         // for B); K-major: one box of 64 k x all rows
@@ -291,9 +278,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         if (leader && lane == 0) {
             int it = 0, local = 0;
             for (int64_t t = pair_id; t < tiles && !*s_abort; t += pairs, ++local) {
-                const int b = local % C::kNumAcc, u = local / C::kNumAcc;
-                // both CTAs' epilogues must have drained this accumulator set
-                if (u >= 1 && !mbar_wait_bounded(&acc_empty[b], (u - 1) & 1, s_abort, p.status)) break;
+                const int b = local & 1;
+                // both CTAs' epilogues must have drained this accumulator buffer
+                if (local >= 2 && !mbar_wait_bounded(&acc_empty[b], ((local >> 1) - 1) & 1, s_abort, p.status)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + b * C::kAccStride;
                 for (int kt = 0; kt < ktiles; ++kt, ++it) {
@@ -303,19 +290,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     const uint32_t a_base = smem_u32(sA + s * C::kABytes);
                     const uint32_t b_base = smem_u32(sB + s * C::kBBytes);
                     if (SPARSE) {
+                        const uint32_t e_col = tmem + C::kECol + 4u * (it & 1);
+                        pair::tmem_cp_pair_128x128b(
+                            e_col, make_smem_desc(smem_u32(sE + s * C::kEBytes), 16, 128, kSwizzleNone));
 #pragma unroll
-                        for (int sub = 0; sub < MSUB; ++sub) {
-                            const uint32_t e_col = tmem + C::kECol + 8u * sub + 4u * (it & 1);
-                            pair::tmem_cp_pair_128x128b(
-                                e_col, make_smem_desc(smem_u32(sE + s * C::kEBytes + sub * 2048), 16, 128, kSwizzleNone));
-                            const uint32_t d_sub = d_tmem + static_cast<uint32_t>(sub * C::kAccStride);
-#pragma unroll
-                            for (int j = 0; j < C::kMmaPerStage; ++j) {
-                                const uint64_t ad = make_smem_desc(a_base + sub * C::kASubBytes + j * C::kAAdvance, 16,
-                                                                   512, kSwizzle64B);
-                                const uint64_t bd = make_smem_desc(b_base + j * C::kBAdvance, 16, 1024, kSwizzle128B);
-                                pair::mma_sp_i8_pair(d_sub, ad, bd, C::kIdesc, e_col + 2u * j, (kt | j) != 0);
-                            }
+                        for (int j = 0; j < C::kMmaPerStage; ++j) {
+                            const uint64_t ad = make_smem_desc(a_base + j * C::kAAdvance, 16, 512, kSwizzle64B);
+                            const uint64_t bd = make_smem_desc(b_base + j * C::kBAdvance, 16, 1024, kSwizzle128B);
+                            pair::mma_sp_i8_pair(d_tmem, ad, bd, C::kIdesc, e_col + 2u * j, (kt | j) != 0);
                         }
                     } else if (MN) {
 #pragma unroll
@@ -347,8 +329,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
         int local = 0;
         int chunk_count = 0;   // output chunks staged so far (TMA-store double buffer)
         for (int64_t t = pair_id; t < tiles; t += pairs, ++local) {
-            const int b = local % C::kNumAcc, u = local / C::kNumAcc;
+            const int b = local & 1;
             const int64_t mt = t / n_tiles, nt = t - mt * n_tiles;
+            const int64_t m0 = mt * 256 + 128 * rank;   // this CTA's accumulator rows
             const int64_t n0 = nt * BN;
             if (SPARSE) {
                 const float g = *p.gamma;
@@ -359,12 +342,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                 }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
             }
-            const bool ok = mbar_wait_bounded(&acc_full[b], u & 1, s_abort, p.status);
+            const bool ok = mbar_wait_bounded(&acc_full[b], (local >> 1) & 1, s_abort, p.status);
             tc_fence_after();
-            for (int sub = 0; sub < MSUB; ++sub) {
-            const int64_t m0 = mt * kTileM + 256 * sub + 128 * rank;   // this CTA's accumulator rows
             const int64_t m = m0 + 32 * quarter + lane;
-            const uint32_t taddr = tmem + lane_base + (MSUB == 2 ? sub : b) * C::kAccStride;
+            const uint32_t taddr = tmem + lane_base + b * C::kAccStride;
             if (ok) {
 #pragma unroll 1
                 for (int c = 0; c < BN / 16; ++c) {
@@ -469,7 +450,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     }
                 }
             }
-            }   // sub-tiles
             // this CTA is done with the buffer: one arrival on the leader's barrier
             tc_fence_before();
             asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -518,16 +498,16 @@ static bool map2d(CUtensorMap *map, CUtensorMapDataType dt, const void *base, ui
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <bool SPARSE, int BN, int STAGES, int MN = 0, int MSUB = 1>
+template <bool SPARSE, int BN, int STAGES, int MN = 0>
 static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CUtensorMap &e, const CUtensorMap &y,
                             const PairParams &p, cudaStream_t s) {
-    using C = PairCfg<SPARSE, BN, STAGES, MN, MSUB>;
-    auto kern = k_umma_pair<SPARSE, BN, STAGES, MN, MSUB>;
+    using C = PairCfg<SPARSE, BN, STAGES, MN>;
+    auto kern = k_umma_pair<SPARSE, BN, STAGES, MN>;
     {
         cudaError_t err = smem_attr(reinterpret_cast<const void *>(kern), C::kSmemBytes);
         if (err != cudaSuccess) return err;
     }
-    const int64_t tiles = ((p.M + 256 * MSUB - 1) / (256 * MSUB)) * ((p.N + BN - 1) / BN);
+    const int64_t tiles = ((p.M + 255) / 256) * ((p.N + BN - 1) / BN);
     int64_t pairs = num_sms() / 2;
     if (pairs > tiles) pairs = tiles;
     if (pairs < 1) pairs = 1;
@@ -535,7 +515,7 @@ static cudaError_t run_pair(const CUtensorMap &a, const CUtensorMap &b, const CU
     return cudaGetLastError();
 }
 
-template <int BN, int MSUB>
+template <int BN>
 static cudaError_t sp_pair(const int8_t *Xq, const float *amax, const float *gamma, const int8_t *vals,
                            const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16, int32_t *acc,
                            uint32_t *status, cudaStream_t s) {
@@ -571,7 +551,6 @@ static cudaError_t sp_pair(const int8_t *Xq, const float *amax, const float *gam
                static_cast<uint64_t>(n_out), static_cast<uint64_t>(T), static_cast<uint64_t>(n_out) * esz, 128, 16,
                CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    if (MSUB == 2) return run_pair<true, BN, 6, 0, 2>(ma, mb, me, my, p, s);
     return run_pair<true, BN, 8>(ma, mb, me, my, p, s);
 }
 
@@ -582,19 +561,13 @@ static cudaError_t sp_pair(const int8_t *Xq, const float *amax, const float *gam
 // (a last tile 86% padding) but 10 x 192 + 128: the 3B block's QKV product
 // measured 63.6 us with 224 and 59.4 us with 192.  At T = 4096 the two cost
 // the same and 224 stays (the 7B down projection: 137 us either way).
-#ifndef SP_PAIR_MSUB
-#define SP_PAIR_MSUB 2
-#endif
 cudaError_t launch_gemm_sp_pair(const int8_t *Xq, const float *amax, const float *gamma, const int8_t *vals,
                                 const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16,
                                 int32_t *acc, uint32_t *status, cudaStream_t s) {
     auto cost = [&](int64_t bn) { return static_cast<double>((T + bn - 1) / bn) * static_cast<double>(bn + 32); };
-    const bool two = SP_PAIR_MSUB == 2 && n_out > 256;
     if (cost(192) < 0.98 * cost(224))
-        return two ? sp_pair<192, 2>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s)
-                   : sp_pair<192, 1>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
-    return two ? sp_pair<224, 2>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s)
-               : sp_pair<224, 1>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
+        return sp_pair<192>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
+    return sp_pair<224>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
 }
 
 // dX = gamma dY . Wq with Wq as bf16 rows [n_out][k] (expanded from the group

@@ -614,6 +614,82 @@ def test_decode_chain_independent_and_ragged(bn, T):
         _check_outputs(ref, o["acc_out"].cpu().numpy(), o["Y"])
 
 
+@pytest.mark.parametrize("T,x_dtype", [(1, "bf16"), (2, "f32"), (3, "bf16"), (5, "bf16"), (8, "f32")])
+def test_decode_chain_all_independent(bn, T, x_dtype):
+    """A chain with no waits at all runs the pipelined kernel: weight shares of
+    consecutive projections share ring stages, the quantiser warps run ahead in
+    up to four int8 buffers and the epilogue trails.  40 projections cycle every
+    buffer many times; shapes from one row tile (most CTAs idle) to several per
+    CTA, k = 64 and odd k-tile counts; every fourth op also copies out its int8
+    activations and scales."""
+    base = [(16, 64), (3840, 2560), (208, 192), (2560, 6912), (640, 64), (1040, 320), (6928, 192), (96, 2560)]
+    shapes = [base[i % len(base)] for i in range(40)]
+    packed = {}
+    ops, refs = [], []
+    for i, (n_out, k) in enumerate(shapes):
+        if (n_out, k) not in packed:
+            packed[(n_out, k)] = _packed_dec(bn, n_out, k, seed=1500 + len(packed))
+        W, pw = packed[(n_out, k)]
+        X = synth.activations(T, k, seed=1600 + i, outlier_p=0.01)
+        if x_dtype == "bf16":
+            Xd, X32 = bf16_dev(X)
+        else:
+            Xd, X32 = dev_f32(X), X
+        Y = torch.empty((T, n_out), dtype=torch.bfloat16 if i % 2 else torch.float32, device="cuda")
+        acc = torch.full((T, n_out), -7, dtype=torch.int32, device="cuda")
+        o = dict(X=Xd, W=pw, Y=Y, acc_out=acc, wait_prev=0)
+        if i % 4 == 0:
+            o["xq_out"] = torch.zeros((T, k), dtype=torch.int8, device="cuda")
+            o["absmax_out"] = torch.zeros((T,), dtype=torch.float32, device="cuda")
+        ops.append(o)
+        refs.append(oracle.forward(W, X32, 1e-5, 1e-5))
+    # one y dtype per chain: split into the float32 and the bf16 halves
+    for half in (0, 1):
+        sub = [(o, r) for i, (o, r) in enumerate(zip(ops, refs)) if i % 2 == half]
+        ch = bn.bitnet_decode_chain([o for o, _ in sub], 1e-5)
+        torch.cuda.synchronize()
+        assert bn.bitnet_read_device_status(ch.ws) == 0
+        for o, ref in sub:
+            if "xq_out" in o:
+                assert np.array_equal(o["xq_out"].cpu().numpy(), ref["xq"])
+                assert np.array_equal(o["absmax_out"].cpu().numpy(), ref["a"])
+            _check_outputs(ref, o["acc_out"].cpu().numpy(), o["Y"])
+        # again, outputs cleared: the chain is repeatable
+        for o, _ in sub:
+            o["acc_out"].fill_(-7)
+        ch()
+        torch.cuda.synchronize()
+        for o, ref in sub:
+            _check_outputs(ref, o["acc_out"].cpu().numpy(), o["Y"])
+
+
+def test_decode_chain_independent_split_launches(bn):
+    """130 independent projections: more than one launch takes, each launch the
+    pipelined kernel; captured in a CUDA graph and replayed."""
+    T, h = 1, 256
+    ops, refs = [], []
+    W, pw = _packed_dec(bn, h, h, seed=1700)
+    for i in range(130):
+        Xd, X32 = bf16_dev(synth.activations(T, h, seed=1800 + i))
+        ops.append(dict(X=Xd, W=pw, Y=torch.empty((T, h), dtype=torch.bfloat16, device="cuda"), wait_prev=0))
+        refs.append(oracle.forward(W, X32, 1e-5, 1e-5))
+    ch = bn.DecodeChain(ops, torch.bfloat16, torch.bfloat16, 1e-5)
+    ch()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        ch()
+    for o in ops:
+        o["Y"].zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert bn.bitnet_read_device_status(ch.ws) == 0
+    for o, ref in zip(ops, refs):
+        yb = o["Y"].view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(yb, synth.to_bf16_bits(ref["y"]))
+    del g
+
+
 def test_decode_chain_split_launches_and_graph(bn):
     """More ops than one launch takes (130 > 128): the library splits the chain;
     captured in a CUDA graph and replayed."""
