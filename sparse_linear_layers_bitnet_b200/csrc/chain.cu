@@ -30,14 +30,20 @@
 //    time): per-token absmax, scale and int8 codes from the staging slot into
 //    one of up to four int8 buffers, in the fragment order the MMA warps read,
 //    so that the quantisers run ahead of the MMA warps;
-//  * MMA warps (sixteen): for every projection piece of every ring stage, a
-//    contiguous run of its 16x64 weight records each; one m16n8k64 sparse
-//    MMA per record, partial sums of row tiles added into one of two shared
-//    partial-sum buffers;
+//  * MMA warps (sixteen, in one group or in four groups of four): group g
+//    takes every GR-th projection with rows on this CTA; for every piece of
+//    its projections in a ring stage, each warp of the group takes a
+//    contiguous run of the piece's 16x64 weight records; one m16n8k64 sparse
+//    MMA per record, partial sums of row tiles added into the projection's
+//    shared partial-sum buffer.  A projection's share is a few dozen to a few
+//    hundred records per CTA, so sixteen warps on one projection spend much
+//    of it on the projection's fixed latency (barrier, the first loads, the
+//    last MMA, the flush); four groups overlap that latency across four
+//    projections;
 //  * epilogue (one warp): dequantises the CTA's outputs of a projection,
 //    writes Y, clears the buffer and counts the CTA done (release add).
-// So while the MMA warps run projection j, the quantisers prepare j + 1 and
-// the epilogue finishes j - 1.  Row tiles of a projection are split over the
+// So while the MMA warps run projections j .. j + GR - 1, the quantisers
+// prepare the next ones and the epilogue finishes the earlier ones.  Row tiles of a projection are split over the
 // CTAs in balanced contiguous ranges, rotated per projection so that the
 // larger shares move around.
 //
@@ -45,8 +51,9 @@
 // which takes two instructions per register; the int32 sums are 64 times the
 // ternary ones, exactly, and the epilogue shifts them back.
 //
-// Two instantiations per activation type: any T <= 8, and T = 1 with the token
-// count folded to a constant.
+// Instantiations per activation type: T = 1 with the token count folded to a
+// constant and four MMA groups; any T <= 8 with four groups (four int8
+// buffers) or with one.
 //
 // All waits are bounded (2 s): a stage that never fills, a counter that never
 // reaches the grid size or an abort raised by another CTA ends every role of
@@ -74,7 +81,9 @@ constexpr int kWarpWLoad = kWarpXLoad + 1;                  // weight producer
 constexpr int kChainThreads = (kWarpWLoad + 1) * 32;
 constexpr int kChainMaxStages = 16;
 constexpr int kChainMaxNb = 4;                              // int8 activation buffers (1 .. 4)
-constexpr int kChainScaleSlots = kChainMaxNb + 2;           // see the epilogue
+constexpr int kChainMaxGroups = 4;                          // MMA warp groups (1 or 4)
+constexpr int kChainAccBufs = 4;                            // partial-sum buffers (max(2, groups) used)
+constexpr int kChainScaleSlots = kChainMaxNb + kChainAccBufs;   // see the epilogue
 constexpr uint32_t kChainStageMax = 32768;   // weight ring stages of 32 KB, or 16 KB when a smaller ring must do
 
 struct ChainParams {
@@ -171,18 +180,20 @@ __device__ __forceinline__ bool mbar_wait_cta(uint64_t *bar, uint32_t parity, vo
     }
 }
 
-// Barrier of the MMA warps (hardware barrier 2) that also ORs a predicate
-// over them: one warp waits for a ring stage, the others block here without
-// issuing instructions, and all of them learn whether the wait succeeded.
-__device__ __forceinline__ bool mma_sync_or(bool v) {
+// Barrier of one group of MMA warps (hardware barrier 2 + group) that also
+// ORs a predicate over them: one warp waits for a ring stage, the others
+// block here without issuing instructions, and all of them learn whether the
+// wait succeeded.
+template <int NWARPS>
+__device__ __forceinline__ bool mma_sync_or(int group, bool v) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, 2, %2, p;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(v ? 1u : 0u), "n"(kChainMmaWarps * 32)
+        : "r"(v ? 1u : 0u), "r"(2 + group), "n"(NWARPS * 32)
         : "memory");
     return r != 0;
 }
@@ -280,13 +291,16 @@ __device__ __forceinline__ void chain_flush(int *acc_buf, int tiles_max, int til
     }
 }
 
-template <bool XBF16, int TM>
+template <bool XBF16, int TM, int GR>
 __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_constant__ ChainParams p) {
+    static_assert(GR == 1 || GR == kChainMaxGroups, "one group, or one per int8 buffer");
+    constexpr int kWpg = kChainMmaWarps / GR;             // MMA warps per group
+    constexpr int kNacc = GR > 2 ? GR : 2;                // partial-sum buffers in use
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kChainMaxStages], s_empty[kChainMaxStages];
     __shared__ __align__(8) uint64_t s_xs_full[kChainQuantWarps], s_xs_empty[kChainQuantWarps];
     __shared__ __align__(8) uint64_t s_xq_full[kChainMaxNb], s_xq_empty[kChainMaxNb];
-    __shared__ __align__(8) uint64_t s_acc_full[2], s_acc_empty[2];
+    __shared__ __align__(8) uint64_t s_acc_full[kChainAccBufs], s_acc_empty[kChainAccBufs];
     __shared__ float s_gamma[kChainMaxOps];
     __shared__ int2 s_tiles[kChainMaxOps];    // this CTA's row tiles [x, y) of every projection
     __shared__ int s_share[kChainMaxOps];     // and its share index
@@ -306,7 +320,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     int *sacc = reinterpret_cast<int *>(xqb + static_cast<size_t>(p.nb) * p.xq_bytes);
     const int acc_words = static_cast<int>(p.acc_bytes >> 2);
 
-    for (int i = tid; i < 2 * acc_words; i += kChainThreads) sacc[i] = 0;
+    for (int i = tid; i < kNacc * acc_words; i += kChainThreads) sacc[i] = 0;
     // every projection's share of this CTA, once (each role reads the table instead of dividing)
     for (int i = tid; i < p.n_ops; i += kChainThreads) {
         int t0, t1;
@@ -325,10 +339,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         }
         for (int s = 0; s < p.nb; ++s) {
             mbar_init(&s_xq_full[s], static_cast<uint32_t>(T));                    // one arrival per row
-            mbar_init(&s_xq_empty[s], kChainMmaWarps);
+            mbar_init(&s_xq_empty[s], kWpg);   // the group that ran the projection
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&s_acc_full[s], kChainMmaWarps);
+        for (int s = 0; s < kNacc; ++s) {
+            mbar_init(&s_acc_full[s], kWpg);
             mbar_init(&s_acc_empty[s], 1);
         }
         fence_mbar_init();
@@ -537,20 +551,20 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
 
     if (warp == kWarpEpi) {
         // ------------------------------------------------------------ epilogue
-        uint32_t ua = 0;   // projections finished (partial-sum buffer ua % 2, scale slot ua % kChainScaleSlots)
+        uint32_t ua = 0;   // projections finished (partial-sum buffer ua % kNacc, scale slot ua % kChainScaleSlots)
         for (int j = 0; j < p.n_ops; ++j) {
             const ChainOpDev &op = p.op[j];
             const int t0 = s_tiles[j].x, t1 = s_tiles[j].y;
             const int ntile = t1 - t0;
             if (ntile > 0) {
-                const int ab = static_cast<int>(ua & 1u);
-                const bool ok = mbar_wait_cta(&s_acc_full[ab], (ua >> 1) & 1u, &s_abort, p.status);
+                const int ab = static_cast<int>(ua % kNacc);
+                const bool ok = mbar_wait_cta(&s_acc_full[ab], (ua / kNacc) & 1u, &s_abort, p.status);
                 if (!__all_sync(0xffffffffu, ok)) break;
-                // Scale slot ua % (kChainMaxNb + 2) was written by the
-                // quantisers after the MMA warps released int8 buffer use
+                // Scale slot ua % (kChainMaxNb + kChainAccBufs) was written by
+                // the quantisers after the MMA warps released int8 buffer use
                 // ua - nb, which they do only after taking partial-sum buffer
                 // use ua - nb, i.e. after this warp finished projection use
-                // ua - nb - 2 >= ua - kChainMaxNb - 2.
+                // ua - nb - kNacc >= ua - kChainMaxNb - kChainAccBufs.
                 const int sc = static_cast<int>(ua % kChainScaleSlots);
                 int *acc_buf = sacc + ab * acc_words;
                 const int per_t = ntile * 16;
@@ -586,16 +600,42 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
 
     // ---------------------------------------------------------------- MMA warps
     // The ring carries this CTA's shares of all projections back to back; a
-    // stage may end one projection and begin the next.  Each warp meets every
-    // stage once (wait for it, its records of every projection in it, release
-    // it) and every projection once (take its buffers, records, flush, hand
-    // the partial sums to the epilogue).
+    // stage may end one projection and begin the next.  Group g (warps
+    // g kWpg .. (g + 1) kWpg - 1) runs the projection uses g, g + GR, ...
+    // (uses count the projections with rows here).  Every warp meets every
+    // stage once, in stream order (wait for it, its group's records in it,
+    // release it), also the stages that hold only other groups' records: a
+    // warp may release a fill round of a slot only once that round has landed
+    // (else its arrival could count towards the slot's previous round), and
+    // the producer refills a slot only after all sixteen warps released it.
+    // Each group meets each of its projections once: take its buffers, run
+    // its records, flush, hand the partial sums to the epilogue.
+    const int grp = warp / kWpg, gw = warp % kWpg;
     uint32_t cs = 0, cph = 0;   // ring slot of the current stage and the parity of its fill round
     uint32_t spos = 0;          // stream offset of the current stage
     bool have = false;          // the current stage has been waited for and not yet released
     uint32_t ppos = 0;          // stream offset of the next projection's records
-    uint32_t ua = 0;            // projections with rows here (partial-sum buffer ua % 2, int8 buffer ua % nb)
+    uint32_t ua = 0;            // projections with rows here so far
     bool failed = false;
+    // The current stage has landed: the group's first warp waits, the others
+    // learn it from the group barrier, which also orders the bulk copies'
+    // writes that warp has observed before their reads.
+    auto take_stage = [&]() -> bool {
+        const bool okf = gw != 0 || mbar_wait_cta(&s_full[cs], cph, &s_abort, p.status);
+        if (mma_sync_or<kWpg>(grp, !okf)) return false;
+        have = true;
+        return true;
+    };
+    auto release_stage = [&]() {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[cs]);
+        have = false;
+        spos += stage_bytes;
+        if (++cs == static_cast<uint32_t>(ns)) {
+            cs = 0;
+            cph ^= 1u;
+        }
+    };
     for (int j = 0; j < p.n_ops && !failed; ++j) {
         const ChainOpDev &op = p.op[j];
         const int t0 = s_tiles[j].x, t1 = s_tiles[j].y;
@@ -603,17 +643,36 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         if (ntile == 0) continue;
         const int ktiles = op.k >> 6;
         const uint32_t bytes = static_cast<uint32_t>(ntile) * static_cast<uint32_t>(ktiles) * 256u;
-        const int ab = static_cast<int>(ua & 1u);
-        const int xb = static_cast<int>(ua & static_cast<uint32_t>(p.nb - 1));
-        // the epilogue is done with this partial-sum buffer's previous projection; the int8 activations are
-        // ready (warp 0 waits; the other MMA warps learn it from the barrier, which also orders the
-        // quantisers' shared-memory writes that warp 0 has acquired before their reads)
-        bool ok = true;
-        if (warp == 0) {
-            ok = ua < 2u || mbar_wait_cta(&s_acc_empty[ab], ((ua >> 1) - 1u) & 1u, &s_abort, p.status);
-            ok = ok && mbar_wait_cta(&s_xq_full[xb], (ua >> p.nb_log2) & 1u, &s_abort, p.status);
+        const uint32_t end = ppos + bytes;
+        const uint32_t use = ua++;
+        if (static_cast<int>(use % GR) != grp) {   // another group's projection
+            ppos = end;
+            continue;
         }
-        if (mma_sync_or(!ok)) break;
+        // release the stages that lie wholly before this projection's records
+        while (spos + stage_bytes <= ppos) {
+            if (!have && !take_stage()) {
+                failed = true;
+                break;
+            }
+            release_stage();
+        }
+        if (failed) break;
+        const int ab = static_cast<int>(use % kNacc);
+        const int xb = static_cast<int>(use & static_cast<uint32_t>(p.nb - 1));
+        // the epilogue is done with this partial-sum buffer's previous projection; the int8 activations are
+        // ready (the group's first warp waits; the others learn it from the group barrier, which also orders
+        // the quantisers' shared-memory writes that warp has acquired before their reads)
+        bool ok = true;
+        if (gw == 0) {
+            ok = use < static_cast<uint32_t>(kNacc) ||
+                 mbar_wait_cta(&s_acc_empty[ab], ((use / kNacc) - 1u) & 1u, &s_abort, p.status);
+            ok = ok && mbar_wait_cta(&s_xq_full[xb], (use >> p.nb_log2) & 1u, &s_abort, p.status);
+        }
+        if (mma_sync_or<kWpg>(grp, !ok)) {
+            failed = true;
+            break;
+        }
         int *acc_buf = sacc + ab * acc_words;
         // Lane l holds the B fragment of token l / 4 (zero for tokens >= T):
         // the 16 bytes lane l % 4 needs of each 64-k tile sit contiguously in
@@ -626,22 +685,15 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         int cur = -1;
         int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
         const float inv_kt = __int_as_float(op.pad);   // 1 / ktiles, formed on the host
-        const uint32_t end = ppos + bytes;
         for (uint32_t pos = ppos; pos < end;) {
-            if (!have) {
-                // warp 0 waits for the stage's data; the bulk copies' writes it has
-                // observed are ordered before the barrier for the other warps
-                const bool okf = warp != 0 || mbar_wait_cta(&s_full[cs], cph, &s_abort, p.status);
-                if (mma_sync_or(!okf)) {
-                    failed = true;
-                    break;
-                }
-                have = true;
+            if (!have && !take_stage()) {
+                failed = true;
+                break;
             }
             const uint32_t seg_end = end < spos + stage_bytes ? end : spos + stage_bytes;
-            // this segment's records: warp w takes the contiguous run [w n / 16, (w + 1) n / 16)
+            // this segment's records: warp w of the group takes the contiguous run [w n / kWpg, (w + 1) n / kWpg)
             const int nrec = static_cast<int>((seg_end - pos) >> 8);
-            const int i0 = (warp * nrec) / kChainMmaWarps, i1 = ((warp + 1) * nrec) / kChainMmaWarps;
+            const int i0 = (gw * nrec) / kWpg, i1 = ((gw + 1) * nrec) / kWpg;
             if (i0 < i1) {
                 const int r0 = static_cast<int>((pos - ppos) >> 8) + i0;   // record index within the CTA's share
                 // r0 / ktiles through the reciprocal (r0 < 2^24: off by at most one, corrected)
@@ -706,16 +758,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                 }
             }
             pos = seg_end;
-            if (pos == spos + stage_bytes) {   // the stage is used up: release it to the producer
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[cs]);
-                have = false;
-                spos += stage_bytes;
-                if (++cs == static_cast<uint32_t>(ns)) {
-                    cs = 0;
-                    cph ^= 1u;
-                }
-            }
+            if (pos == spos + stage_bytes) release_stage();   // the stage is used up
         }
         if (failed) break;
         if (cur >= 0) chain_flush<TM>(acc_buf, p.tiles_max, cur, lane, T, acc);
@@ -725,12 +768,13 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             mbar_arrive(&s_acc_full[ab]);
             mbar_arrive(&s_xq_empty[xb]);
         }
-        ++ua;
         ppos = end;
     }
-    if (have && !failed) {   // the stream's last, partly used stage
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[cs]);
+    // the rest of the stream (other groups' records): released in order, since the producer may still refill
+    // these slots
+    while (!failed && spos < ppos) {
+        if (!have && !take_stage()) break;
+        release_stage();
     }
 }
 
@@ -755,7 +799,7 @@ bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayo
     for (int pass = 0; pass < 5; ++pass) {
         for (int nb = CHAIN_NB_MAX; nb >= (min_nb[pass] > nb_lo ? min_nb[pass] : nb_lo); nb >>= 1) {
             if (T < 4 && nb != kChainMaxNb) continue;
-            const size_t fixed = 2 * acc + static_cast<size_t>(nb) * xq + kChainQuantWarps * xs;
+            const size_t fixed = kChainAccBufs * acc + static_cast<size_t>(nb) * xq + kChainQuantWarps * xs;
             if (fixed >= kChainMaxSmem) continue;
             size_t ns = (kChainMaxSmem - fixed) / stage[pass];
             if (ns > static_cast<size_t>(kChainMaxStages)) ns = kChainMaxStages;
@@ -790,10 +834,14 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
     }
     ChainLayout L;
     if (!chain_layout(T, kmax, x_bf16, tiles_max, &L)) return cudaErrorInvalidValue;
-    // one-token chains take the instantiation with T folded to 1
+    // one-token chains take the instantiation with T folded to 1; four MMA
+    // groups need one int8 buffer each (always the case for T < 4)
     const bool one = T == 1;
-    auto kern = x_bf16 ? (one ? k_decode_chain<true, 1> : k_decode_chain<true, 8>)
-                       : (one ? k_decode_chain<false, 1> : k_decode_chain<false, 8>);
+    const bool groups = L.nb == kChainMaxGroups;
+    auto kern = x_bf16 ? (one ? k_decode_chain<true, 1, 4>
+                              : (groups ? k_decode_chain<true, 8, 4> : k_decode_chain<true, 8, 1>))
+                       : (one ? k_decode_chain<false, 1, 4>
+                              : (groups ? k_decode_chain<false, 8, 4> : k_decode_chain<false, 8, 1>));
     {
         cudaError_t e = smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(kChainMaxSmem));
         if (e != cudaSuccess) return e;
