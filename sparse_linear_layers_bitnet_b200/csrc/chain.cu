@@ -28,8 +28,10 @@
 //    itself done with the previous projection (grid-wide counter, acquire);
 //  * quantisers (four warps, one token row of one projection per warp at a
 //    time): per-token absmax, scale and int8 codes from the staging slot into
-//    one of up to four int8 buffers, in the fragment order the MMA warps read,
-//    so that the quantisers run ahead of the MMA warps;
+//    one of up to eight int8 buffers, in the fragment order the MMA warps
+//    read, so that the quantisers run ahead of the MMA warps (with eight
+//    buffers and four groups, a group's next projection is quantised while it
+//    runs the current one);
 //  * MMA warps (sixteen, in one group or in four groups of four): group g
 //    takes every GR-th projection with rows on this CTA; for every piece of
 //    its projections in a ring stage, each warp of the group takes a
@@ -80,10 +82,11 @@ constexpr int kWarpXLoad = kWarpEpi + 1;                    // activation loader
 constexpr int kWarpWLoad = kWarpXLoad + 1;                  // weight producer
 constexpr int kChainThreads = (kWarpWLoad + 1) * 32;
 constexpr int kChainMaxStages = 16;
-constexpr int kChainMaxNb = 4;                              // int8 activation buffers (1 .. 4)
+constexpr int kChainMaxNb = 8;                              // int8 activation buffers (1, 2, 4 or 8)
 constexpr int kChainMaxGroups = 4;                          // MMA warp groups (1 or 4)
 constexpr int kChainAccBufs = 4;                            // partial-sum buffers (max(2, groups) used)
-constexpr int kChainScaleSlots = kChainMaxNb + kChainAccBufs;   // see the epilogue
+constexpr int kChainScaleSlots = 16;                        // >= kChainMaxNb + kChainAccBufs: see the epilogue
+static_assert(kChainScaleSlots >= kChainMaxNb + kChainAccBufs, "scale slots");
 constexpr uint32_t kChainStageMax = 32768;   // weight ring stages of 32 KB, or 16 KB when a smaller ring must do
 
 struct ChainParams {
@@ -91,7 +94,7 @@ struct ChainParams {
     int32_t n_ops, T, x_bf16, y_bf16;
     int32_t ns;                // weight ring stages
     uint32_t stage_bytes;      // 32 or 16 KB
-    int32_t nb;                // int8 activation buffers: 1, 2 or 4
+    int32_t nb;                // int8 activation buffers: 1, 2, 4 or 8
     int32_t nb_log2;
     uint32_t xq_bytes;         // one int8 buffer: T rows of pitch chain_pitch(kmax)
     uint32_t xs_bytes;         // one staging slot: one activation row of kmax elements
@@ -198,9 +201,6 @@ __device__ __forceinline__ bool mma_sync_or(int group, bool v) {
     return r != 0;
 }
 
-#ifndef CHAIN_NB_MAX
-#define CHAIN_NB_MAX 4
-#endif
 
 // Wait that ignores the abort flag, up to a deadline (for draining copies in flight).
 __device__ bool mbar_wait_until(uint64_t *bar, uint32_t parity, uint64_t deadline_ns) {
@@ -470,8 +470,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         // warp must meet each barrier it waits on in consecutive rounds: its
         // staging slot is its own; an int8 buffer is met by the warps owning a
         // row of its projections, which for T >= 4 is every warp, and for
-        // T < 4 (the host then takes four buffers) depends only on the
-        // projection's index mod 4, the same for every use of the buffer.
+        // T < 4 (the host then takes four or eight buffers) depends only on
+        // the projection's index mod 4, the same for every use of the buffer.
         const int qw = warp - kWarpQuant0;
         const int qt = tid - kWarpQuant0 * 32;
         for (int i = qt; i < p.n_ops; i += kChainQuantThreads) s_gamma[i] = __ldg(p.op[i].gamma);
@@ -782,23 +782,26 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
 
 static size_t round128(size_t x) { return (x + 127) / 128 * 128; }
 
-// Shared-memory layout: four staging slots of one activation row each, the
-// most int8 buffers (up to four; exactly four for T < 4, see the quantisers)
-// and a weight ring of at least 128 KB in 32 KB stages; else 96 KB, then a
-// single int8 buffer (T >= 4) and 64 KB, then 16 KB stages, down to two of
-// them.  False when even that does not fit.
+// Shared-memory layout: four staging slots of one activation row each,
+// four partial-sum buffers, int8 buffers and a weight ring, in this order of
+// preference: eight int8 buffers (two per MMA group) and a ring of at least
+// 96 KB in 32 KB stages; four or two buffers and 128 KB; four or two and
+// 96 KB; down to one buffer (T >= 4) and 64 KB; then 16 KB stages, down to
+// two of them.  For T < 4 the buffers are four or eight (see the
+// quantisers).  False when even that does not fit.
 bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayout *L) {
     if (T < 1 || T > 8 || kmax < 64 || tiles_max < 1 || tiles_max > kChainMaxTiles) return false;
     const size_t acc = round128(static_cast<size_t>(T) * static_cast<size_t>(tiles_max) * 16 * 4);
     const size_t xq = round128(static_cast<size_t>(T) * static_cast<size_t>(chain_pitch(kmax)));
     const size_t xs = static_cast<size_t>(kmax) * (x_bf16 ? 2 : 4);
-    const int nb_lo = T < 4 ? kChainMaxNb : 1;
-    const size_t min_ring[5] = {128 * 1024, 96 * 1024, 64 * 1024, 2 * 32768, 2 * 16384};
-    const uint32_t stage[5] = {32768, 32768, 32768, 32768, 16384};
-    const int min_nb[5] = {2, 2, 1, 1, 1};
-    for (int pass = 0; pass < 5; ++pass) {
-        for (int nb = CHAIN_NB_MAX; nb >= (min_nb[pass] > nb_lo ? min_nb[pass] : nb_lo); nb >>= 1) {
-            if (T < 4 && nb != kChainMaxNb) continue;
+    constexpr int kPasses = 6;
+    const size_t min_ring[kPasses] = {96 * 1024, 128 * 1024, 96 * 1024, 64 * 1024, 2 * 32768, 2 * 16384};
+    const uint32_t stage[kPasses] = {32768, 32768, 32768, 32768, 32768, 16384};
+    const int max_nb[kPasses] = {8, 4, 4, 4, 4, 4};
+    const int min_nb[kPasses] = {8, 2, 2, 1, 1, 1};
+    for (int pass = 0; pass < kPasses; ++pass) {
+        for (int nb = max_nb[pass]; nb >= min_nb[pass]; nb >>= 1) {
+            if (T < 4 && nb % 4 != 0) continue;
             const size_t fixed = kChainAccBufs * acc + static_cast<size_t>(nb) * xq + kChainQuantWarps * xs;
             if (fixed >= kChainMaxSmem) continue;
             size_t ns = (kChainMaxSmem - fixed) / stage[pass];
@@ -835,9 +838,10 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
     ChainLayout L;
     if (!chain_layout(T, kmax, x_bf16, tiles_max, &L)) return cudaErrorInvalidValue;
     // one-token chains take the instantiation with T folded to 1; four MMA
-    // groups need one int8 buffer each (always the case for T < 4)
+    // groups need a multiple of four int8 buffers, so that each buffer
+    // belongs to one group (always the case for T < 4)
     const bool one = T == 1;
-    const bool groups = L.nb == kChainMaxGroups;
+    const bool groups = L.nb % kChainMaxGroups == 0;
     auto kern = x_bf16 ? (one ? k_decode_chain<true, 1, 4>
                               : (groups ? k_decode_chain<true, 8, 4> : k_decode_chain<true, 8, 1>))
                        : (one ? k_decode_chain<false, 1, 4>
@@ -868,7 +872,7 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         p.ns = L.ns;
         p.stage_bytes = L.stage_bytes;
         p.nb = L.nb;
-        p.nb_log2 = L.nb == 4 ? 2 : (L.nb == 2 ? 1 : 0);
+        p.nb_log2 = L.nb == 8 ? 3 : (L.nb == 4 ? 2 : (L.nb == 2 ? 1 : 0));
         p.xq_bytes = L.xq_bytes;
         p.xs_bytes = L.xs_bytes;
         p.tiles_max = L.tiles_max;
