@@ -29,23 +29,20 @@
 //  * quantisers (four warps, one token row of one projection per warp at a
 //    time): per-token absmax, scale and int8 codes from the staging slot into
 //    one of up to eight int8 buffers, in the fragment order the MMA warps
-//    read, so that the quantisers run ahead of the MMA warps (with eight
-//    buffers and four groups, a group's next projection is quantised while it
-//    runs the current one);
-//  * MMA warps (sixteen, in one group or in four groups of four): group g
-//    takes every GR-th projection with rows on this CTA; for every piece of
-//    its projections in a ring stage, each warp of the group takes a
-//    contiguous run of the piece's 16x64 weight records; one m16n8k64 sparse
-//    MMA per record, partial sums of row tiles added into the projection's
-//    shared partial-sum buffer.  A projection's share is a few dozen to a few
-//    hundred records per CTA, so sixteen warps on one projection spend much
-//    of it on the projection's fixed latency (barrier, the first loads, the
-//    last MMA, the flush); four groups overlap that latency across four
-//    projections;
+//    read, so that the quantisers run ahead of the MMA warps;
+//  * MMA warps (sixteen): every ring stage is split over them in contiguous
+//    runs of 16x64 weight records, regardless of projection boundaries, so
+//    that the ring drains in stream order and every warp does the same work
+//    per stage; one m16n8k64 sparse MMA per record, partial sums of row tiles
+//    added into the projection's shared partial-sum buffer.  There is no
+//    barrier per projection: each warp passes every projection in order with
+//    its own waits and arrivals, so the fixed latency of a projection (the
+//    first loads, the last MMA, the flush) overlaps with other warps' work on
+//    the next one;
 //  * epilogue (one warp): dequantises the CTA's outputs of a projection,
 //    writes Y, clears the buffer and counts the CTA done (release add).
-// So while the MMA warps run projections j .. j + GR - 1, the quantisers
-// prepare the next ones and the epilogue finishes the earlier ones.  Row tiles of a projection are split over the
+// So while the MMA warps run projection j, the quantisers prepare the next
+// ones and the epilogue finishes the earlier ones.  Row tiles of a projection are split over the
 // CTAs in balanced contiguous ranges, rotated per projection so that the
 // larger shares move around.
 //
@@ -53,15 +50,15 @@
 // which takes two instructions per register; the int32 sums are 64 times the
 // ternary ones, exactly, and the epilogue shifts them back.
 //
-// Instantiations per activation type: T = 1 with the token count folded to a
-// constant and four MMA groups; any T <= 8 with four groups (four int8
-// buffers) or with one.
+// Two instantiations per activation type: any T <= 8, and T = 1 with the
+// token count folded to a constant.
 //
 // All waits are bounded (2 s): a stage that never fills, a counter that never
 // reaches the grid size or an abort raised by another CTA ends every role of
 // the kernel with the timeout bit in the status word; outstanding copies are
 // waited for (bounded) before the copy threads exit.
 #include <cstring>
+#include <vector>
 
 #include "../../include/bitnet_sparse.h"
 #include "common.cuh"
@@ -81,23 +78,23 @@ constexpr int kWarpEpi = kWarpQuant0 + kChainQuantWarps;    // epilogue warp
 constexpr int kWarpXLoad = kWarpEpi + 1;                    // activation loader
 constexpr int kWarpWLoad = kWarpXLoad + 1;                  // weight producer
 constexpr int kChainThreads = (kWarpWLoad + 1) * 32;
-constexpr int kChainMaxStages = 16;
+constexpr int kChainMaxStages = 16;                         // ring slots: one per MMA warp
+static_assert(kChainMmaWarps == kChainMaxStages, "each MMA warp owns one ring slot");
 constexpr int kChainMaxNb = 8;                              // int8 activation buffers (1, 2, 4 or 8)
-constexpr int kChainMaxGroups = 4;                          // MMA warp groups (1 or 4)
-constexpr int kChainAccBufs = 4;                            // partial-sum buffers (max(2, groups) used)
+constexpr int kChainAccBufs = 8;                            // partial-sum buffers
 constexpr int kChainScaleSlots = 16;                        // >= kChainMaxNb + kChainAccBufs: see the epilogue
 static_assert(kChainScaleSlots >= kChainMaxNb + kChainAccBufs, "scale slots");
-constexpr uint32_t kChainStageMax = 32768;   // weight ring stages of 32 KB, or 16 KB when a smaller ring must do
 
 struct ChainParams {
     ChainOpDev op[kChainMaxOps];
     int32_t n_ops, T, x_bf16, y_bf16;
     int32_t ns;                // weight ring stages
-    uint32_t stage_bytes;      // 32 or 16 KB
+    uint32_t stage_bytes;      // bytes of one ring stage: a multiple of 256, at most 32 KB
     int32_t nb;                // int8 activation buffers: 1, 2, 4 or 8
     int32_t nb_log2;
-    uint32_t xq_bytes;         // one int8 buffer: T rows of pitch chain_pitch(kmax)
-    uint32_t xs_bytes;         // one staging slot: one activation row of kmax elements
+    uint32_t xs_off[kChainQuantWarps];   // dynamic shared memory offsets of the staging slots (one row each),
+    uint32_t xq_off[kChainMaxNb];        // the int8 buffers (T rows each)
+    uint32_t acc_off;                    // and the partial-sum buffers
     int32_t tiles_max;         // most row tiles a CTA takes of one projection
     uint32_t acc_bytes;        // one partial-sum buffer: T x tiles_max x 16 int32
     float eps;
@@ -156,51 +153,31 @@ __device__ bool wait_counter(const uint32_t *ctr, uint32_t target, const ChainPa
     }
 }
 
-// Wait for a phase.  try_wait may suspend the thread for a while, but it
-// can also return at once, so the loop keeps the cost of a failed round low:
-// the abort flag (a shared load) every 64th round, the clock (%globaltimer,
-// which takes issue slots of a pipe other warps need) every 1024th.  Gives up
-// when the CTA's abort flag is raised or after kWaitLimitNs (then it raises
-// the flag and the status bit).
+// Wait for a phase.  The waiting warp is suspended in try_wait until the
+// phase completes (or about kSuspendNs pass), so that waiting roles take no
+// issue slots from the working ones; between suspensions it reads the
+// CTA's abort flag and, every 16th round, the clock.  Gives up when the
+// abort flag is raised or after kWaitLimitNs (then it raises the flag and
+// the status bit).
+constexpr uint32_t kSuspendNs = 20000;
 __device__ __forceinline__ bool mbar_wait_cta(uint64_t *bar, uint32_t parity, volatile int *abort, uint32_t *status) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = 0;
     for (uint32_t i = 1;; ++i) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63u) == 0u) {
-            if (*abort) return false;
-            if ((i & 1023u) == 0u) {
-                const uint64_t now = globaltimer_ns();
-                if (t0 == 0) {
-                    t0 = now;
-                } else if (now - t0 > kWaitLimitNs) {
-                    *abort = 1;
-                    atomicOr(status, kStatusTimeout);
-                    return false;
-                }
+        if (mbar_try_wait_suspend(bar, parity, kSuspendNs)) return true;
+        if (*abort) return false;
+        if ((i & 15u) == 0u) {
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicOr(status, kStatusTimeout);
+                return false;
             }
         }
     }
 }
-
-// Barrier of one group of MMA warps (hardware barrier 2 + group) that also
-// ORs a predicate over them: one warp waits for a ring stage, the others
-// block here without issuing instructions, and all of them learn whether the
-// wait succeeded.
-template <int NWARPS>
-__device__ __forceinline__ bool mma_sync_or(int group, bool v) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.or.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"(v ? 1u : 0u), "r"(2 + group), "n"(NWARPS * 32)
-        : "memory");
-    return r != 0;
-}
-
 
 // Wait that ignores the abort flag, up to a deadline (for draining copies in flight).
 __device__ bool mbar_wait_until(uint64_t *bar, uint32_t parity, uint64_t deadline_ns) {
@@ -291,11 +268,9 @@ __device__ __forceinline__ void chain_flush(int *acc_buf, int tiles_max, int til
     }
 }
 
-template <bool XBF16, int TM, int GR>
+template <bool XBF16, int TM>
 __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_constant__ ChainParams p) {
-    static_assert(GR == 1 || GR == kChainMaxGroups, "one group, or one per int8 buffer");
-    constexpr int kWpg = kChainMmaWarps / GR;             // MMA warps per group
-    constexpr int kNacc = GR > 2 ? GR : 2;                // partial-sum buffers in use
+    constexpr int kNacc = kChainAccBufs;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kChainMaxStages], s_empty[kChainMaxStages];
     __shared__ __align__(8) uint64_t s_xs_full[kChainQuantWarps], s_xs_empty[kChainQuantWarps];
@@ -304,6 +279,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     __shared__ float s_gamma[kChainMaxOps];
     __shared__ int2 s_tiles[kChainMaxOps];    // this CTA's row tiles [x, y) of every projection
     __shared__ int s_share[kChainMaxOps];     // and its share index
+    __shared__ uint32_t s_ustart[kChainMaxOps + 1];   // stream offset of each use (projection with rows here), and the end
+    __shared__ uint8_t s_uj[kChainMaxOps];            // the projection of each use
+    __shared__ int2 s_uk[kChainMaxOps];               // and its k and 1 / (k / 64) (fp32 bits)
+    __shared__ int s_nuses;
     __shared__ float s_scale[kChainScaleSlots][8];
     __shared__ float s_amax[kChainScaleSlots][8];
     __shared__ int s_abort;
@@ -312,12 +291,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     const int ns = p.ns;
     const int T = TM == 1 ? 1 : p.T;   // a one-token instantiation folds T away
     const uint32_t G = gridDim.x;
-    // dynamic shared memory: weight ring | staging slots | int8 buffers | partial-sum buffers
+    // dynamic shared memory: weight ring | staging slots | int8 buffers | partial-sum buffers, each slot and
+    // buffer sized by the host for the rows it receives
     uint8_t *ring = smem;
     const uint32_t stage_bytes = p.stage_bytes;
-    uint8_t *xs = ring + static_cast<size_t>(ns) * stage_bytes;
-    int8_t *xqb = reinterpret_cast<int8_t *>(xs + static_cast<size_t>(kChainQuantWarps) * p.xs_bytes);
-    int *sacc = reinterpret_cast<int *>(xqb + static_cast<size_t>(p.nb) * p.xq_bytes);
+    int *sacc = reinterpret_cast<int *>(smem + p.acc_off);
     const int acc_words = static_cast<int>(p.acc_bytes >> 2);
 
     for (int i = tid; i < kNacc * acc_words; i += kChainThreads) sacc[i] = 0;
@@ -331,7 +309,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         s_abort = 0;
         for (int s = 0; s < ns; ++s) {
             mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], kChainMmaWarps);
+            mbar_init(&s_empty[s], 1);   // the slot's MMA warp
         }
         for (int s = 0; s < kChainQuantWarps; ++s) {
             mbar_init(&s_xs_full[s], 1);
@@ -339,14 +317,54 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         }
         for (int s = 0; s < p.nb; ++s) {
             mbar_init(&s_xq_full[s], static_cast<uint32_t>(T));                    // one arrival per row
-            mbar_init(&s_xq_empty[s], kWpg);   // the group that ran the projection
+            mbar_init(&s_xq_empty[s], kChainMmaWarps);
         }
         for (int s = 0; s < kNacc; ++s) {
-            mbar_init(&s_acc_full[s], kWpg);
+            mbar_init(&s_acc_full[s], kChainMmaWarps);
             mbar_init(&s_acc_empty[s], 1);
         }
         fence_mbar_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // the uses and their offsets in this CTA's weight stream: lane l scans projections 4 l .. 4 l + 3
+        uint32_t cnt = 0, bytes = 0, b[4];
+        bool has[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int j = 4 * lane + e;
+            const int nt = j < p.n_ops ? s_tiles[j].y - s_tiles[j].x : 0;
+            has[e] = nt > 0;
+            b[e] = has[e] ? static_cast<uint32_t>(nt) * static_cast<uint32_t>(p.op[j].k >> 6) * 256u : 0u;
+            cnt += has[e] ? 1u : 0u;
+            bytes += b[e];
+        }
+        uint32_t c_ex = cnt, b_ex = bytes;   // inclusive scans, then made exclusive
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const uint32_t c = __shfl_up_sync(0xffffffffu, c_ex, d), bb = __shfl_up_sync(0xffffffffu, b_ex, d);
+            if (lane >= d) {
+                c_ex += c;
+                b_ex += bb;
+            }
+        }
+        c_ex -= cnt;
+        b_ex -= bytes;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            if (has[e]) {
+                s_uj[c_ex] = static_cast<uint8_t>(4 * lane + e);
+                s_uk[c_ex] = make_int2(p.op[4 * lane + e].k, p.op[4 * lane + e].pad);
+                s_ustart[c_ex] = b_ex;
+                ++c_ex;
+                b_ex += b[e];
+            }
+        }
+        if (lane == 31) {
+            s_nuses = static_cast<int>(c_ex);
+            s_ustart[c_ex] = b_ex;
+        }
     }
     __syncthreads();
 
@@ -445,7 +463,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                     break;
                 }
                 mbar_arrive_expect_tx(&s_xs_full[slot], row_bytes);
-                bulk_load(xs + static_cast<size_t>(slot) * p.xs_bytes,
+                bulk_load(smem + p.xs_off[slot],
                           static_cast<const uint8_t *>(op.X) + static_cast<size_t>(t) * row_bytes, row_bytes,
                           &s_xs_full[slot]);
             }
@@ -506,7 +524,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                     failed = true;
                     break;
                 }
-                const uint4 *src = reinterpret_cast<const uint4 *>(xs + static_cast<size_t>(qw) * p.xs_bytes);
+                const uint4 *src = reinterpret_cast<const uint4 *>(smem + p.xs_off[qw]);
                 // pass 1: absmax of the row
                 uint32_t m = 0u;
                 for (int c = lane; c < cpr; c += 32) {
@@ -522,7 +540,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                     if (copy_out && op.amax_out) op.amax_out[t] = a;
                 }
                 // pass 2: codes (and, on one CTA, their copy in natural order)
-                int8_t *row = xqb + static_cast<size_t>(xb) * p.xq_bytes + static_cast<size_t>(t) * pitch;
+                int8_t *row = reinterpret_cast<int8_t *>(smem + p.xq_off[xb]) + static_cast<size_t>(t) * pitch;
                 for (int c = lane; c < cpr; c += 32) {
                     const uint2 q = chunk_store_codes<XBF16>(src[c], row, c * kElems, s_inv);
                     if (copy_out && op.xq_out) {
@@ -599,168 +617,57 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     }
 
     // ---------------------------------------------------------------- MMA warps
-    // The ring carries this CTA's shares of all projections back to back; a
-    // stage may end one projection and begin the next.  Group g (warps
-    // g kWpg .. (g + 1) kWpg - 1) runs the projection uses g, g + GR, ...
-    // (uses count the projections with rows here).  Every warp meets every
-    // stage once, in stream order (wait for it, its group's records in it,
-    // release it), also the stages that hold only other groups' records: a
-    // warp may release a fill round of a slot only once that round has landed
-    // (else its arrival could count towards the slot's previous round), and
-    // the producer refills a slot only after all sixteen warps released it.
-    // Each group meets each of its projections once: take its buffers, run
-    // its records, flush, hand the partial sums to the epilogue.
-    const int grp = warp / kWpg, gw = warp % kWpg;
-    uint32_t cs = 0, cph = 0;   // ring slot of the current stage and the parity of its fill round
-    uint32_t spos = 0;          // stream offset of the current stage
-    bool have = false;          // the current stage has been waited for and not yet released
-    uint32_t ppos = 0;          // stream offset of the next projection's records
-    uint32_t ua = 0;            // projections with rows here so far
+    // The ring carries this CTA's shares of all projections back to back, in
+    // stages of S bytes; stage s sits in ring slot s % 16, and MMA warp w owns
+    // slot w: it runs every record of the stages w, w + 16, ... (whatever
+    // projections they belong to) and alone releases them.  A warp passes
+    // every use (a projection with rows here) in stream order: it opens it
+    // (the use's partial-sum buffer is free, its int8 activations are ready),
+    // runs its records of it, if any of its stages holds some, and closes it
+    // (flush, arrivals on the partial-sum and int8 buffers' barriers).  Every
+    // warp therefore meets every barrier in consecutive rounds: parity waits
+    // stay unambiguous, and no arrival can count towards a round it does not
+    // belong to.  A warp closes a use as soon as it knows it has no more
+    // records of it: when its stage reaches the use's end, or when its next
+    // stage starts at or after it.
+    const int n_uses = s_nuses;
+    const uint32_t total = s_ustart[n_uses];
+    int u = 0;                  // the next use to close
+    bool opened = false;        // use u has been opened
     bool failed = false;
-    // The current stage has landed: the group's first warp waits, the others
-    // learn it from the group barrier, which also orders the bulk copies'
-    // writes that warp has observed before their reads.
-    auto take_stage = [&]() -> bool {
-        const bool okf = gw != 0 || mbar_wait_cta(&s_full[cs], cph, &s_abort, p.status);
-        if (mma_sync_or<kWpg>(grp, !okf)) return false;
-        have = true;
+    // state of the open use
+    int ab = 0, xb = 0, ktiles = 1, cur = -1;
+    uint32_t ustart = 0, uend = 0;
+    float inv_kt = 1.0f;
+    int *acc_buf = sacc;
+    const uint4 *b_src = nullptr;
+    int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
+    // Lane l holds the B fragment of token l / 4 (zero for tokens >= T): the
+    // 16 bytes lane l % 4 needs of each 64-k tile sit contiguously in the
+    // shared row (fragment order), one 16-byte load per record.
+    const int bn = lane >> 2;
+    const bool has_b = bn < T;
+    auto open_use = [&]() -> bool {
+        const int2 uk = s_uk[u];   // k, and 1 / ktiles formed on the host
+        ab = u % kNacc;
+        xb = u & (p.nb - 1);
+        bool ok = u < kNacc || mbar_wait_cta(&s_acc_empty[ab], ((u / kNacc) - 1) & 1, &s_abort, p.status);
+        ok = ok && mbar_wait_cta(&s_xq_full[xb], (static_cast<uint32_t>(u) >> p.nb_log2) & 1u, &s_abort, p.status);
+        if (!__all_sync(0xffffffffu, ok)) return false;
+        acc_buf = sacc + ab * acc_words;
+        b_src = reinterpret_cast<const uint4 *>(smem + p.xq_off[xb] +
+                                                static_cast<int64_t>(has_b ? bn : 0) * chain_pitch(uk.x)) +
+                (lane & 3);
+        ktiles = uk.x >> 6;
+        inv_kt = __int_as_float(uk.y);
+        ustart = s_ustart[u];
+        uend = s_ustart[u + 1];
+        cur = -1;
+        opened = true;
         return true;
     };
-    auto release_stage = [&]() {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s_empty[cs]);
-        have = false;
-        spos += stage_bytes;
-        if (++cs == static_cast<uint32_t>(ns)) {
-            cs = 0;
-            cph ^= 1u;
-        }
-    };
-    for (int j = 0; j < p.n_ops && !failed; ++j) {
-        const ChainOpDev &op = p.op[j];
-        const int t0 = s_tiles[j].x, t1 = s_tiles[j].y;
-        const int ntile = t1 - t0;
-        if (ntile == 0) continue;
-        const int ktiles = op.k >> 6;
-        const uint32_t bytes = static_cast<uint32_t>(ntile) * static_cast<uint32_t>(ktiles) * 256u;
-        const uint32_t end = ppos + bytes;
-        const uint32_t use = ua++;
-        if (static_cast<int>(use % GR) != grp) {   // another group's projection
-            ppos = end;
-            continue;
-        }
-        // release the stages that lie wholly before this projection's records
-        while (spos + stage_bytes <= ppos) {
-            if (!have && !take_stage()) {
-                failed = true;
-                break;
-            }
-            release_stage();
-        }
-        if (failed) break;
-        const int ab = static_cast<int>(use % kNacc);
-        const int xb = static_cast<int>(use & static_cast<uint32_t>(p.nb - 1));
-        // the epilogue is done with this partial-sum buffer's previous projection; the int8 activations are
-        // ready (the group's first warp waits; the others learn it from the group barrier, which also orders
-        // the quantisers' shared-memory writes that warp has acquired before their reads)
-        bool ok = true;
-        if (gw == 0) {
-            ok = use < static_cast<uint32_t>(kNacc) ||
-                 mbar_wait_cta(&s_acc_empty[ab], ((use / kNacc) - 1u) & 1u, &s_abort, p.status);
-            ok = ok && mbar_wait_cta(&s_xq_full[xb], (use >> p.nb_log2) & 1u, &s_abort, p.status);
-        }
-        if (mma_sync_or<kWpg>(grp, !ok)) {
-            failed = true;
-            break;
-        }
-        int *acc_buf = sacc + ab * acc_words;
-        // Lane l holds the B fragment of token l / 4 (zero for tokens >= T):
-        // the 16 bytes lane l % 4 needs of each 64-k tile sit contiguously in
-        // the shared row (fragment order), one 16-byte load per record.
-        const int bn = lane >> 2;
-        const bool has_b = bn < T;
-        const uint4 *b_src = reinterpret_cast<const uint4 *>(xqb + static_cast<size_t>(xb) * p.xq_bytes +
-                                                             static_cast<int64_t>(has_b ? bn : 0) * chain_pitch(op.k)) +
-                             (lane & 3);
-        int cur = -1;
-        int acc[4][4] = {};   // partial sums of the current row tile, one accumulator per record slot
-        const float inv_kt = __int_as_float(op.pad);   // 1 / ktiles, formed on the host
-        for (uint32_t pos = ppos; pos < end;) {
-            if (!have && !take_stage()) {
-                failed = true;
-                break;
-            }
-            const uint32_t seg_end = end < spos + stage_bytes ? end : spos + stage_bytes;
-            // this segment's records: warp w of the group takes the contiguous run [w n / kWpg, (w + 1) n / kWpg)
-            const int nrec = static_cast<int>((seg_end - pos) >> 8);
-            const int i0 = (gw * nrec) / kWpg, i1 = ((gw + 1) * nrec) / kWpg;
-            if (i0 < i1) {
-                const int r0 = static_cast<int>((pos - ppos) >> 8) + i0;   // record index within the CTA's share
-                // r0 / ktiles through the reciprocal (r0 < 2^24: off by at most one, corrected)
-                int tile = __float2int_rz(static_cast<float>(r0) * inv_kt);
-                int kt = r0 - tile * ktiles;
-                if (kt < 0) {
-                    --tile;
-                    kt += ktiles;
-                } else if (kt >= ktiles) {
-                    ++tile;
-                    kt -= ktiles;
-                }
-                const uint2 *rec =
-                    reinterpret_cast<const uint2 *>(ring + static_cast<size_t>(cs) * stage_bytes + (pos - spos)) + lane;
-                int i = i0;
-                while (i < i1) {
-                    if (tile != cur) {
-                        if (cur >= 0) chain_flush<TM>(acc_buf, p.tiles_max, cur, lane, T, acc);
-                        cur = tile;
-                    }
-                    if (i + 4 <= i1 && kt + 4 <= ktiles) {
-                        // four records of one row tile: all loads first, then the MMAs
-                        uint2 w[4];
-                        uint32_t bf[4][4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) w[u] = rec[(i + u) * 32];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const uint4 v = has_b ? b_src[(kt + u) * 4] : make_uint4(0u, 0u, 0u, 0u);
-                            bf[u][0] = v.x;
-                            bf[u][1] = v.y;
-                            bf[u][2] = v.z;
-                            bf[u][3] = v.w;
-                        }
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            uint32_t a4[4];
-#pragma unroll
-                            for (int r = 0; r < 4; ++r) a4[r] = expand_codes_x64(w[u].x, r);
-                            mma_sp_m16n8k64(acc[u], a4, bf[u], w[u].y);
-                        }
-                        i += 4;
-                        kt += 4;
-                    } else {
-                        const uint2 w = rec[i * 32];
-                        uint32_t bf[4], a4[4];
-                        const uint4 v = has_b ? b_src[kt * 4] : make_uint4(0u, 0u, 0u, 0u);
-                        bf[0] = v.x;
-                        bf[1] = v.y;
-                        bf[2] = v.z;
-                        bf[3] = v.w;
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) a4[r] = expand_codes_x64(w.x, r);
-                        mma_sp_m16n8k64(acc[0], a4, bf, w.y);
-                        i += 1;
-                        kt += 1;
-                    }
-                    if (kt == ktiles) {
-                        kt = 0;
-                        ++tile;
-                    }
-                }
-            }
-            pos = seg_end;
-            if (pos == spos + stage_bytes) release_stage();   // the stage is used up
-        }
-        if (failed) break;
+    auto close_use = [&]() -> bool {
+        if (!opened && !open_use()) return false;
         if (cur >= 0) chain_flush<TM>(acc_buf, p.tiles_max, cur, lane, T, acc);
         // the shared atomics of every lane are ordered before the release of the arrivals
         __syncwarp();
@@ -768,57 +675,196 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             mbar_arrive(&s_acc_full[ab]);
             mbar_arrive(&s_xq_empty[xb]);
         }
-        ppos = end;
+        opened = false;
+        ++u;
+        return true;
+    };
+    const uint32_t ring_step = stage_bytes * static_cast<uint32_t>(kChainMmaWarps);
+    uint8_t *slot = ring + static_cast<size_t>(warp) * stage_bytes;
+    uint32_t round = 0;
+    for (uint32_t a = static_cast<uint32_t>(warp) * stage_bytes; a < total; a += ring_step, ++round) {
+        const uint32_t b = total - a < stage_bytes ? total : a + stage_bytes;
+        // the uses that end before this stage
+        while (u < n_uses && s_ustart[u + 1] <= a && !failed) failed = !close_use();
+        if (failed) break;
+        const bool okf = mbar_wait_cta(&s_full[warp], round & 1u, &s_abort, p.status);
+        if (!__all_sync(0xffffffffu, okf)) {
+            failed = true;
+            break;
+        }
+        for (uint32_t pos = a; pos < b && !failed;) {
+            if (!opened && !open_use()) {
+                failed = true;
+                break;
+            }
+            const uint32_t seg_end = b < uend ? b : uend;
+            // records [pos, seg_end) of the open use; r0 = the first one's index in the CTA's share
+            const int r0 = static_cast<int>((pos - ustart) >> 8);
+            const int cnt = static_cast<int>((seg_end - pos) >> 8);
+            // r0 / ktiles through the reciprocal (r0 < 2^24: off by at most one, corrected)
+            int tile = __float2int_rz(static_cast<float>(r0) * inv_kt);
+            int kt = r0 - tile * ktiles;
+            if (kt < 0) {
+                --tile;
+                kt += ktiles;
+            } else if (kt >= ktiles) {
+                ++tile;
+                kt -= ktiles;
+            }
+            const uint2 *rec = reinterpret_cast<const uint2 *>(slot + (pos - a)) + lane;
+            int i = 0;
+            while (i < cnt) {
+                if (tile != cur) {
+                    if (cur >= 0) chain_flush<TM>(acc_buf, p.tiles_max, cur, lane, T, acc);
+                    cur = tile;
+                }
+                if (i + 4 <= cnt && kt + 4 <= ktiles) {
+                    // four records of one row tile: all loads first, then the MMAs
+                    uint2 w[4];
+                    uint32_t bf[4][4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) w[e] = rec[(i + e) * 32];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const uint4 v = has_b ? b_src[(kt + e) * 4] : make_uint4(0u, 0u, 0u, 0u);
+                        bf[e][0] = v.x;
+                        bf[e][1] = v.y;
+                        bf[e][2] = v.z;
+                        bf[e][3] = v.w;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        uint32_t a4[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) a4[r] = expand_codes_x64(w[e].x, r);
+                        mma_sp_m16n8k64(acc[e], a4, bf[e], w[e].y);
+                    }
+                    i += 4;
+                    kt += 4;
+                } else {
+                    const uint2 w = rec[i * 32];
+                    uint32_t bf[4], a4[4];
+                    const uint4 v = has_b ? b_src[kt * 4] : make_uint4(0u, 0u, 0u, 0u);
+                    bf[0] = v.x;
+                    bf[1] = v.y;
+                    bf[2] = v.z;
+                    bf[3] = v.w;
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) a4[r] = expand_codes_x64(w.x, r);
+                    mma_sp_m16n8k64(acc[0], a4, bf, w.y);
+                    i += 1;
+                    kt += 1;
+                }
+                if (kt == ktiles) {
+                    kt = 0;
+                    ++tile;
+                }
+            }
+            pos = seg_end;
+            if (pos == uend && !close_use()) failed = true;
+        }
+        if (failed) break;
+        // release the stage to the producer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s_empty[warp]);
+        // the uses that end before this warp's next stage
+        const uint32_t na = a + ring_step < total ? a + ring_step : total;
+        while (u < n_uses && s_ustart[u + 1] <= na && !failed) failed = !close_use();
+        if (failed) break;
     }
-    // the rest of the stream (other groups' records): released in order, since the producer may still refill
-    // these slots
-    while (!failed && spos < ppos) {
-        if (!have && !take_stage()) break;
-        release_stage();
-    }
+    while (!failed && u < n_uses) failed = !close_use();
 }
 
 // ---------------------------------------------------------------- host side
 
 static size_t round128(size_t x) { return (x + 127) / 128 * 128; }
 
-// Shared-memory layout: four staging slots of one activation row each,
-// four partial-sum buffers, int8 buffers and a weight ring, in this order of
-// preference: eight int8 buffers (two per MMA group) and a ring of at least
-// 96 KB in 32 KB stages; four or two buffers and 128 KB; four or two and
-// 96 KB; down to one buffer (T >= 4) and 64 KB; then 16 KB stages, down to
-// two of them.  For T < 4 the buffers are four or eight (see the
-// quantisers).  False when even that does not fit.
-bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayout *L) {
-    if (T < 1 || T > 8 || kmax < 64 || tiles_max < 1 || tiles_max > kChainMaxTiles) return false;
+// Shared-memory layout: the weight ring (one slot per MMA warp), four
+// staging slots (slot s holds the activation rows i = s mod 4 of the chain,
+// xs_slot[s] bytes), int8 buffers (buffer b holds the uses u = b mod nb,
+// xq_use[u] bytes each) and eight partial-sum buffers.  The ring takes what
+// is left, in stages of a multiple of 256 bytes (one record) up to 32 KB, in
+// this order of preference: eight int8 buffers (the quantisers run further
+// ahead) with stages of at least 8 KB; four or two buffers with 8 KB; down to
+// one buffer (T >= 4) with 2 KB.  For T < 4 the buffers are four or eight
+// (see the quantisers).  Every size is a multiple of 128 bytes.  False when
+// even the last form does not fit.
+static bool chain_layout_sized(int64_t T, const size_t xs_slot[kChainQuantWarps], const size_t *xq_use, int n_uses,
+                               int tiles_max, ChainLayout *L) {
+    if (T < 1 || T > 8 || n_uses < 1 || tiles_max < 1 || tiles_max > kChainMaxTiles) return false;
     const size_t acc = round128(static_cast<size_t>(T) * static_cast<size_t>(tiles_max) * 16 * 4);
-    const size_t xq = round128(static_cast<size_t>(T) * static_cast<size_t>(chain_pitch(kmax)));
-    const size_t xs = static_cast<size_t>(kmax) * (x_bf16 ? 2 : 4);
-    constexpr int kPasses = 6;
-    const size_t min_ring[kPasses] = {96 * 1024, 128 * 1024, 96 * 1024, 64 * 1024, 2 * 32768, 2 * 16384};
-    const uint32_t stage[kPasses] = {32768, 32768, 32768, 32768, 32768, 16384};
-    const int max_nb[kPasses] = {8, 4, 4, 4, 4, 4};
-    const int min_nb[kPasses] = {8, 2, 2, 1, 1, 1};
+    size_t xs_total = 0;
+    for (int q = 0; q < kChainQuantWarps; ++q) xs_total += xs_slot[q];
+    constexpr int kPasses = 3;
+    const size_t min_stage[kPasses] = {8192, 8192, 2048};
+    const int max_nb[kPasses] = {8, 4, 4};
+    const int min_nb[kPasses] = {8, 2, 1};
     for (int pass = 0; pass < kPasses; ++pass) {
         for (int nb = max_nb[pass]; nb >= min_nb[pass]; nb >>= 1) {
             if (T < 4 && nb % 4 != 0) continue;
-            const size_t fixed = kChainAccBufs * acc + static_cast<size_t>(nb) * xq + kChainQuantWarps * xs;
+            size_t xq_size[kChainMaxNb] = {};
+            size_t xq_total = 0;
+            for (int u = 0; u < n_uses; ++u)
+                xq_size[u % nb] = xq_use[u] > xq_size[u % nb] ? xq_use[u] : xq_size[u % nb];
+            for (int b = 0; b < nb; ++b) xq_total += xq_size[b];
+            const size_t fixed = kChainAccBufs * acc + xq_total + xs_total;
             if (fixed >= kChainMaxSmem) continue;
-            size_t ns = (kChainMaxSmem - fixed) / stage[pass];
-            if (ns > static_cast<size_t>(kChainMaxStages)) ns = kChainMaxStages;
-            if (ns < 2 || ns * stage[pass] < min_ring[pass]) continue;
-            L->ns = static_cast<int>(ns);
-            L->stage_bytes = stage[pass];
+            size_t stage = (kChainMaxSmem - fixed) / kChainMaxStages / 256 * 256;
+            if (stage > 32768) stage = 32768;
+            if (stage < min_stage[pass]) continue;
+            L->ns = kChainMaxStages;
+            L->stage_bytes = static_cast<uint32_t>(stage);
             L->nb = nb;
-            L->xq_bytes = static_cast<uint32_t>(xq);
-            L->xs_bytes = static_cast<uint32_t>(xs);
+            size_t off = kChainMaxStages * stage;
+            for (int q = 0; q < kChainQuantWarps; ++q) {
+                L->xs_off[q] = static_cast<uint32_t>(off);
+                off += xs_slot[q];
+            }
+            for (int b = 0; b < kChainMaxNb; ++b) {
+                L->xq_off[b] = static_cast<uint32_t>(off);
+                if (b < nb) off += xq_size[b];
+            }
+            L->acc_off = static_cast<uint32_t>(off);
             L->tiles_max = tiles_max;
             L->acc_bytes = static_cast<uint32_t>(acc);
-            L->smem = ns * stage[pass] + fixed;
+            L->smem = off + kChainAccBufs * acc;
             return true;
         }
     }
     return false;
+}
+
+bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayout *L) {
+    if (kmax < 64) return false;
+    const size_t xs = round128(static_cast<size_t>(kmax) * (x_bf16 ? 2 : 4));
+    const size_t xs_slot[kChainQuantWarps] = {xs, xs, xs, xs};
+    size_t xq_use[kChainMaxNb];
+    for (int b = 0; b < kChainMaxNb; ++b)
+        xq_use[b] = round128(static_cast<size_t>(T) * static_cast<size_t>(chain_pitch(kmax)));
+    return chain_layout_sized(T, xs_slot, xq_use, kChainMaxNb, tiles_max, L);
+}
+
+// The layout of one launch over ops[0, n).  When every projection has at
+// least one row tile on every CTA (n_out / 16 >= G), the k-th
+// projection with rows on a CTA is projection k on every CTA, so each slot and
+// buffer can be sized for the rows it actually receives; otherwise every one
+// holds rows of kmax.
+static bool chain_layout_for(const ChainOpDev *ops, int n, int64_t T, bool x_bf16, int64_t kmax, int G, int tiles_max,
+                             ChainLayout *L) {
+    bool every_cta = true;
+    for (int i = 0; i < n; ++i) every_cta = every_cta && (ops[i].n_out >> 4) >= G;
+    if (!every_cta) return chain_layout(T, kmax, x_bf16, tiles_max, L);
+    size_t xs_slot[kChainQuantWarps] = {};
+    std::vector<size_t> xq_use(static_cast<size_t>(n));
+    for (int i = 0; i < n; ++i) {
+        const size_t row = round128(static_cast<size_t>(ops[i].k) * (x_bf16 ? 2 : 4));
+        for (int64_t t = 0; t < T; ++t) {
+            const int q = static_cast<int>((static_cast<int64_t>(i) * T + t) % kChainQuantWarps);
+            xs_slot[q] = row > xs_slot[q] ? row : xs_slot[q];
+        }
+        xq_use[static_cast<size_t>(i)] = round128(static_cast<size_t>(T) * static_cast<size_t>(chain_pitch(ops[i].k)));
+    }
+    return chain_layout_sized(T, xs_slot, xq_use.data(), n, tiles_max, L);
 }
 
 cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, bool x_bf16, bool y_bf16, float eps,
@@ -835,24 +881,19 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         const int t = (rows16 + G - 1) / G;
         tiles_max = t > tiles_max ? t : tiles_max;
     }
-    ChainLayout L;
-    if (!chain_layout(T, kmax, x_bf16, tiles_max, &L)) return cudaErrorInvalidValue;
-    // one-token chains take the instantiation with T folded to 1; four MMA
-    // groups need a multiple of four int8 buffers, so that each buffer
-    // belongs to one group (always the case for T < 4)
-    const bool one = T == 1;
-    const bool groups = L.nb % kChainMaxGroups == 0;
-    auto kern = x_bf16 ? (one ? k_decode_chain<true, 1, 4>
-                              : (groups ? k_decode_chain<true, 8, 4> : k_decode_chain<true, 8, 1>))
-                       : (one ? k_decode_chain<false, 1, 4>
-                              : (groups ? k_decode_chain<false, 8, 4> : k_decode_chain<false, 8, 1>));
-    {
-        cudaError_t e = smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(kChainMaxSmem));
-        if (e != cudaSuccess) return e;
-    }
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     for (int base = 0; base < n_ops; base += kChainMaxOps) {
         const int n = (n_ops - base) < kChainMaxOps ? (n_ops - base) : kChainMaxOps;
+        ChainLayout L;
+        if (!chain_layout_for(ops + base, n, T, x_bf16, kmax, G, tiles_max, &L)) return cudaErrorInvalidValue;
+        // one-token chains take the instantiation with T folded to 1
+        const bool one = T == 1;
+        auto kern = x_bf16 ? (one ? k_decode_chain<true, 1> : k_decode_chain<true, 8>)
+                           : (one ? k_decode_chain<false, 1> : k_decode_chain<false, 8>);
+        {
+            cudaError_t e = smem_attr(reinterpret_cast<const void *>(kern), static_cast<int>(kChainMaxSmem));
+            if (e != cudaSuccess) return e;
+        }
         ChainParams p;
         for (int i = 0; i < n; ++i) {
             p.op[i] = ops[base + i];
@@ -873,8 +914,9 @@ cudaError_t launch_decode_chain(const ChainOpDev *ops, int n_ops, int64_t T, boo
         p.stage_bytes = L.stage_bytes;
         p.nb = L.nb;
         p.nb_log2 = L.nb == 8 ? 3 : (L.nb == 4 ? 2 : (L.nb == 2 ? 1 : 0));
-        p.xq_bytes = L.xq_bytes;
-        p.xs_bytes = L.xs_bytes;
+        for (int q = 0; q < kChainQuantWarps; ++q) p.xs_off[q] = L.xs_off[q];
+        for (int b = 0; b < kChainMaxNb; ++b) p.xq_off[b] = L.xq_off[b];
+        p.acc_off = L.acc_off;
         p.tiles_max = L.tiles_max;
         p.acc_bytes = L.acc_bytes;
         p.eps = eps;

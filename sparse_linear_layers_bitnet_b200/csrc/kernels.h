@@ -129,7 +129,7 @@ struct ChainOpDev {
 constexpr int kChainMaxOps = 128;                  // projections per launch (kernel parameter space)
 constexpr int kChainMaxTiles = 32;                 // 16-row tiles per CTA per projection
 constexpr int kChainMaxK = 1 << 17;                // 64 * 127 * k / 2 stays inside int32 (codes expanded x64)
-constexpr size_t kChainMaxSmem = 227 * 1024 - 4096;   // dynamic shared memory (static use < 4 KB)
+constexpr size_t kChainMaxSmem = 227 * 1024 - 5120;   // dynamic shared memory (static use < 5 KB)
 constexpr size_t kChainAbortOffset = 4;            // workspace: grid abort word
 constexpr size_t kChainCountersOffset = 256;       // workspace: one counter per projection
 // Shared-memory layout of one chain launch (chain.cu).
@@ -138,9 +138,14 @@ struct ChainLayout {
     uint32_t stage_bytes; // bytes of one stage
     int nb;               // int8 activation buffers
     int tiles_max;        // most row tiles one CTA takes of one projection
-    uint32_t xq_bytes, xs_bytes, acc_bytes;
+    uint32_t xs_off[4];   // byte offsets in dynamic shared memory: activation staging slots,
+    uint32_t xq_off[8];   // int8 buffers
+    uint32_t acc_off;     // and the partial-sum buffers
+    uint32_t acc_bytes;   // one partial-sum buffer
     size_t smem;          // dynamic shared memory of the launch
 };
+// A layout in which every staging slot and int8 buffer holds rows of kmax
+// (the launch may size them tighter, for the rows they actually receive).
 bool chain_layout(int64_t T, int64_t kmax, bool x_bf16, int tiles_max, ChainLayout *L);
 // The latency-oriented chain for projections that wait for their predecessor (chain_serial.cu).
 bool chain_serial_fits(int64_t T, int64_t kmax);
