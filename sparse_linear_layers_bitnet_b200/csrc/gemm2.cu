@@ -134,11 +134,18 @@ struct PairCfg {
     static constexpr int kHalfN = BN / 2;                  // B rows per CTA
     static constexpr int kARowBytes = SPARSE ? 64 : 128;
     static constexpr int kBRowBytes = 128;
-    static constexpr int kKStep = SPARSE ? 128 : 64;
-    static constexpr int kABytes = 128 * kARowBytes;
-    static constexpr int kBBytes = kHalfN * kBRowBytes;
-    static constexpr int kEBytes = SPARSE ? 2048 : 0;
-    static constexpr int kStageBytes = kABytes + kBBytes + kEBytes;   // per CTA
+    static constexpr int kKStep = SPARSE ? 128 : 64;       // k of one k-step (one metadata block when sparse)
+    // k-steps per ring stage: a sparse k-step is only 2 x 64 of k, about 150 ns of
+    // MMA at the instruction's rate, so two share a stage and its barrier round trip
+    static constexpr int kSub = SPARSE ? 2 : 1;
+    static constexpr int kASub = 128 * kARowBytes;          // one k-step's A, B and metadata bytes
+    static constexpr int kBSub = kHalfN * kBRowBytes;
+    static constexpr int kESub = SPARSE ? 2048 : 0;
+    static constexpr int kABytes = kSub * kASub;
+    static constexpr int kBBytes = kSub * kBSub;
+    static constexpr int kEBytes = kSub * kESub;
+    static constexpr int kSubBytes = kASub + kBSub + kESub;
+    static constexpr int kStageBytes = kSub * kSubBytes;   // per CTA
     static constexpr int kMmaPerStage = SPARSE ? 2 : 4;
     static constexpr int kAAdvance = 32;
     static constexpr int kBAdvance = SPARSE ? 64 : 32;
@@ -155,7 +162,7 @@ struct PairCfg {
     static constexpr int kMnAdvance = 2 * 1024;            // 16 k-rows per MMA
     static_assert(!SPARSE || (BN % 32 == 0 && BN <= 224), "sparse pair tiles: N multiple of 32, two buffers + metadata");
     static_assert(SPARSE || (BN % 32 == 0 && BN <= 256), "dense pair tiles: N multiple of 32");
-    static_assert(kBBytes % 1024 == 0, "B tile must keep the 128-byte swizzle atoms aligned");
+    static_assert(kBSub % 1024 == 0, "B tile must keep the 128-byte swizzle atoms aligned");
     static_assert(!MN || (!SPARSE && (!(MN & 2) || kHalfN % 64 == 0)), "MN-major tiles: dense, whole 64-wide boxes");
 };
 
@@ -197,7 +204,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
     const int64_t pair_id = blockIdx.x >> 1, pairs = gridDim.x >> 1;
     const int64_t m_tiles = (p.M + 255) / 256, n_tiles = (p.N + BN - 1) / BN;
     const int64_t tiles = m_tiles * n_tiles;
-    const int ktiles = static_cast<int>((p.K + C::kKStep - 1) / C::kKStep);
+    const int ksteps = static_cast<int>((p.K + C::kKStep - 1) / C::kKStep);
+    // ring stages per tile.  When a tile has an odd number of sparse k-steps the
+    // last stage's second one lies past K: TMA fills its A and B boxes with
+    // zeros and its metadata load is clamped to the last valid block, so its
+    // MMAs add exactly zero and every stage has the same shape.
+    const int ktiles = (ksteps + C::kSub - 1) / C::kSub;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -243,10 +255,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                         break;
                     if (leader) mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
                     if (SPARSE) {
-                        pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes, kt * (C::kKStep / 2), a_row);
-                        pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes, kt * C::kKStep, b_row);
-                        pair::tma_load_2d_pair(&tmE, &full[s], sE + s * C::kEBytes, 0,
-                                               static_cast<int32_t>((kt * p.meta_rows + e_row) / 8));
+#pragma unroll
+                        for (int sub = 0; sub < C::kSub; ++sub) {
+                            const int kk = kt * C::kSub + sub;
+                            const int ke = kk < ksteps ? kk : ksteps - 1;   // a valid metadata block
+                            pair::tma_load_2d_pair(&tmA, &full[s], sA + s * C::kABytes + sub * C::kASub,
+                                                   kk * (C::kKStep / 2), a_row);
+                            pair::tma_load_2d_pair(&tmB, &full[s], sB + s * C::kBBytes + sub * C::kBSub, kk * C::kKStep,
+                                                   b_row);
+                            pair::tma_load_2d_pair(&tmE, &full[s], sE + s * C::kEBytes + sub * C::kESub, 0,
+                                                   static_cast<int32_t>((ke * p.meta_rows + e_row) / 8));
+                        }
                     } else if (MN) {
                         // MN-major: boxes of 64 MN-elements x 64 k-rows (two for A's 128 rows, kHalfN / 64
                         // for B); K-major: one box of 64 k x all rows
@@ -290,14 +309,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     const uint32_t a_base = smem_u32(sA + s * C::kABytes);
                     const uint32_t b_base = smem_u32(sB + s * C::kBBytes);
                     if (SPARSE) {
-                        const uint32_t e_col = tmem + C::kECol + 4u * (it & 1);
-                        pair::tmem_cp_pair_128x128b(
-                            e_col, make_smem_desc(smem_u32(sE + s * C::kEBytes), 16, 128, kSwizzleNone));
 #pragma unroll
-                        for (int j = 0; j < C::kMmaPerStage; ++j) {
-                            const uint64_t ad = make_smem_desc(a_base + j * C::kAAdvance, 16, 512, kSwizzle64B);
-                            const uint64_t bd = make_smem_desc(b_base + j * C::kBAdvance, 16, 1024, kSwizzle128B);
-                            pair::mma_sp_i8_pair(d_tmem, ad, bd, C::kIdesc, e_col + 2u * j, (kt | j) != 0);
+                        for (int sub = 0; sub < C::kSub; ++sub) {
+                            // metadata of consecutive k-steps alternate between two TMEM column groups
+                            const uint32_t e_col = tmem + C::kECol + 4u * ((it * C::kSub + sub) & 1);
+                            pair::tmem_cp_pair_128x128b(
+                                e_col, make_smem_desc(smem_u32(sE + s * C::kEBytes + sub * C::kESub), 16, 128,
+                                                      kSwizzleNone));
+#pragma unroll
+                            for (int j = 0; j < C::kMmaPerStage; ++j) {
+                                const uint64_t ad = make_smem_desc(a_base + sub * C::kASub + j * C::kAAdvance, 16, 512,
+                                                                   kSwizzle64B);
+                                const uint64_t bd = make_smem_desc(b_base + sub * C::kBSub + j * C::kBAdvance, 16, 1024,
+                                                                   kSwizzle128B);
+                                pair::mma_sp_i8_pair(d_tmem, ad, bd, C::kIdesc, e_col + 2u * j, (kt | j | sub) != 0);
+                            }
                         }
                     } else if (MN) {
 #pragma unroll
@@ -551,7 +577,7 @@ static cudaError_t sp_pair(const int8_t *Xq, const float *amax, const float *gam
                static_cast<uint64_t>(n_out), static_cast<uint64_t>(T), static_cast<uint64_t>(n_out) * esz, 128, 16,
                CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorInvalidValue;
-    return run_pair<true, BN, 8>(ma, mb, me, my, p, s);
+    return run_pair<true, BN, 4>(ma, mb, me, my, p, s);
 }
 
 // Tile width of the sparse pair GEMM over the T tokens: 224 (two 224-column
