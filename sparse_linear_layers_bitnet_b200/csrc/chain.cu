@@ -30,15 +30,14 @@
 //    time): per-token absmax, scale and int8 codes from the staging slot into
 //    one of up to eight int8 buffers, in the fragment order the MMA warps
 //    read, so that the quantisers run ahead of the MMA warps;
-//  * MMA warps (sixteen): every ring stage is split over them in contiguous
-//    runs of 16x64 weight records, regardless of projection boundaries, so
-//    that the ring drains in stream order and every warp does the same work
-//    per stage; one m16n8k64 sparse MMA per record, partial sums of row tiles
-//    added into the projection's shared partial-sum buffer.  There is no
-//    barrier per projection: each warp passes every projection in order with
-//    its own waits and arrivals, so the fixed latency of a projection (the
-//    first loads, the last MMA, the flush) overlaps with other warps' work on
-//    the next one;
+//  * MMA warps (twelve): each owns one ring slot and runs every record of the
+//    stages that land in it (every twelfth stage of the stream), whatever
+//    projections they hold: one m16n8k64 sparse MMA per 16x64 weight record,
+//    partial sums of row tiles added into the projection's shared partial-sum
+//    buffer.  There is no barrier per projection: each warp passes every
+//    projection in order with its own waits and arrivals, so the fixed
+//    latency of a projection (the first loads, the last MMA, the flush)
+//    overlaps with other warps' work on the next one;
 //  * epilogue (one warp): dequantises the CTA's outputs of a projection,
 //    writes Y, clears the buffer and counts the CTA done (release add).
 // So while the MMA warps run projection j, the quantisers prepare the next
@@ -68,7 +67,7 @@
 namespace bitnet {
 
 #ifndef CHAIN_MMA_WARPS
-#define CHAIN_MMA_WARPS 16
+#define CHAIN_MMA_WARPS 12
 #endif
 constexpr int kChainMmaWarps = CHAIN_MMA_WARPS;
 constexpr int kChainQuantWarps = 4;
@@ -78,8 +77,7 @@ constexpr int kWarpEpi = kWarpQuant0 + kChainQuantWarps;    // epilogue warp
 constexpr int kWarpXLoad = kWarpEpi + 1;                    // activation loader
 constexpr int kWarpWLoad = kWarpXLoad + 1;                  // weight producer
 constexpr int kChainThreads = (kWarpWLoad + 1) * 32;
-constexpr int kChainMaxStages = 16;                         // ring slots: one per MMA warp
-static_assert(kChainMmaWarps == kChainMaxStages, "each MMA warp owns one ring slot");
+constexpr int kChainMaxStages = kChainMmaWarps;             // ring slots: one per MMA warp
 constexpr int kChainMaxNb = 8;                              // int8 activation buffers (1, 2, 4 or 8)
 constexpr int kChainAccBufs = 8;                            // partial-sum buffers
 constexpr int kChainScaleSlots = 16;                        // >= kChainMaxNb + kChainAccBufs: see the epilogue
@@ -618,9 +616,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
 
     // ---------------------------------------------------------------- MMA warps
     // The ring carries this CTA's shares of all projections back to back, in
-    // stages of S bytes; stage s sits in ring slot s % 16, and MMA warp w owns
-    // slot w: it runs every record of the stages w, w + 16, ... (whatever
-    // projections they belong to) and alone releases them.  A warp passes
+    // stages of S bytes; with W MMA warps, stage s sits in ring slot s % W, and
+    // MMA warp w owns slot w: it runs every record of the stages w, w + W, ...
+    // (whatever projections they belong to) and alone releases them.  A warp passes
     // every use (a projection with rows here) in stream order: it opens it
     // (the use's partial-sum buffer is free, its int8 activations are ready),
     // runs its records of it, if any of its stages holds some, and closes it
