@@ -580,20 +580,20 @@ static cudaError_t sp_pair(const int8_t *Xq, const float *amax, const float *gam
     return run_pair<true, BN, 4>(ma, mb, me, my, p, s);
 }
 
-// Tile width of the sparse pair GEMM over the T tokens: 224 (two 224-column
-// accumulators and the metadata fill TMEM) unless 192-wide tiles waste clearly
-// fewer padded columns.  Cost model: ceil(T / BN) x (BN + 32), the padded
-// columns of one tile row plus a fixed cost per tile.  T = 2048 is 9 x 224 + 32
-// (a last tile 86% padding) but 10 x 192 + 128: the 3B block's QKV product
-// measured 63.6 us with 224 and 59.4 us with 192.  At T = 4096 the two cost
-// the same and 224 stays (the 7B down projection: 137 us either way).
+// Tile width of the sparse pair GEMM over the T tokens: 192 unless 224-wide
+// tiles waste clearly fewer padded columns.  Cost model: ceil(T / BN) x
+// (BN + 32), the padded columns of one tile row plus a fixed cost per tile.
+// With two k-steps per ring stage the 192-wide tiles measured faster even
+// where the model has them slightly dearer: at T = 4096 (7B up and down)
+// 3503 against 3355 TOPS; 160- and 128-wide tiles measured 3035 and 2683.
+// T = 2048 is 9 x 224 + 32 (a last tile 86% padding) but 10 x 192 + 128.
 cudaError_t launch_gemm_sp_pair(const int8_t *Xq, const float *amax, const float *gamma, const int8_t *vals,
                                 const uint8_t *meta, int64_t T, int64_t n_out, int64_t k, void *Y, bool y_bf16,
                                 int32_t *acc, uint32_t *status, cudaStream_t s) {
     auto cost = [&](int64_t bn) { return static_cast<double>((T + bn - 1) / bn) * static_cast<double>(bn + 32); };
-    if (cost(192) < 0.98 * cost(224))
-        return sp_pair<192>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
-    return sp_pair<224>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
+    if (cost(224) < 0.95 * cost(192))
+        return sp_pair<224>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
+    return sp_pair<192>(Xq, amax, gamma, vals, meta, T, n_out, k, Y, y_bf16, acc, status, s);
 }
 
 // dX = gamma dY . Wq with Wq as bf16 rows [n_out][k] (expanded from the group
