@@ -34,10 +34,11 @@
 //    stages that land in it (every twelfth stage of the stream), whatever
 //    projections they hold: one m16n8k64 sparse MMA per 16x64 weight record,
 //    partial sums of row tiles added into the projection's shared partial-sum
-//    buffer.  There is no barrier per projection: each warp passes every
-//    projection in order with its own waits and arrivals, so the fixed
-//    latency of a projection (the first loads, the last MMA, the flush)
-//    overlaps with other warps' work on the next one;
+//    buffer.  There is no barrier per projection: the hand-overs between the
+//    roles go through monotonic counters in shared memory (rows quantised,
+//    records run, projections finished by the epilogue), so a warp waits and
+//    signals only for the projections it has records of, and the fixed
+//    latency of a projection overlaps with other warps' work on the next one;
 //  * epilogue (one warp): dequantises the CTA's outputs of a projection,
 //    writes Y, clears the buffer and counts the CTA done (release add).
 // So while the MMA warps run projection j, the quantisers prepare the next
@@ -185,6 +186,38 @@ __device__ bool mbar_wait_until(uint64_t *bar, uint32_t parity, uint64_t deadlin
     return true;
 }
 
+// Monotonic shared-memory counters of the hand-overs between the roles (see
+// the MMA warps): an acquire load, a release add, and a bounded wait for a
+// count to reach a target.  A count only grows, so a wait can never mistake
+// an earlier round for its own.
+__device__ __forceinline__ uint32_t ld_acquire_cta(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+    return v;
+}
+__device__ __forceinline__ void red_release_cta(uint32_t *p, uint32_t v) {
+    asm volatile("red.release.cta.shared::cta.add.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ bool wait_count(const uint32_t *ctr, uint32_t target, volatile int *abort, uint32_t *status) {
+    if (ld_acquire_cta(ctr) >= target) return true;
+    uint64_t t0 = 0;
+    for (uint32_t i = 1;; ++i) {
+        __nanosleep(256);   // a waiting warp leaves the issue slots to the others (quantisers at T > 1)
+        if (ld_acquire_cta(ctr) >= target) return true;
+        if ((i & 15u) == 0u) {
+            if (*abort) return false;
+            const uint64_t now = globaltimer_ns();
+            if (t0 == 0) {
+                t0 = now;
+            } else if (now - t0 > kWaitLimitNs) {
+                *abort = 1;
+                atomicOr(status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
 // Adds bytes to the transaction count of the barrier's current phase (no arrival).
 __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
@@ -272,8 +305,10 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ __align__(8) uint64_t s_full[kChainMaxStages], s_empty[kChainMaxStages];
     __shared__ __align__(8) uint64_t s_xs_full[kChainQuantWarps], s_xs_empty[kChainQuantWarps];
-    __shared__ __align__(8) uint64_t s_xq_full[kChainMaxNb], s_xq_empty[kChainMaxNb];
-    __shared__ __align__(8) uint64_t s_acc_full[kChainAccBufs], s_acc_empty[kChainAccBufs];
+    // hand-over counters (monotonic): rows quantised into each int8 buffer, records run against each int8 and
+    // each partial-sum buffer, projections the epilogue has finished per partial-sum buffer
+    __shared__ uint32_t s_rows_q[kChainMaxNb], s_recs_x[kChainMaxNb];
+    __shared__ uint32_t s_recs_a[kChainAccBufs], s_freed[kChainAccBufs];
     __shared__ float s_gamma[kChainMaxOps];
     __shared__ int2 s_tiles[kChainMaxOps];    // this CTA's row tiles [x, y) of every projection
     __shared__ int s_share[kChainMaxOps];     // and its share index
@@ -281,6 +316,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     __shared__ uint8_t s_uj[kChainMaxOps];            // the projection of each use
     __shared__ int2 s_uk[kChainMaxOps];               // and its k and 1 / (k / 64) (fp32 bits)
     __shared__ int s_nuses;
+    __shared__ uint32_t s_cumx[kChainMaxOps];         // records of the earlier uses of the same int8 buffer
+    __shared__ uint32_t s_cuma[kChainMaxOps];         // and of the same partial-sum buffer
     __shared__ float s_scale[kChainScaleSlots][8];
     __shared__ float s_amax[kChainScaleSlots][8];
     __shared__ int s_abort;
@@ -313,14 +350,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             mbar_init(&s_xs_full[s], 1);
             mbar_init(&s_xs_empty[s], 1);
         }
-        for (int s = 0; s < p.nb; ++s) {
-            mbar_init(&s_xq_full[s], static_cast<uint32_t>(T));                    // one arrival per row
-            mbar_init(&s_xq_empty[s], kChainMmaWarps);
-        }
-        for (int s = 0; s < kNacc; ++s) {
-            mbar_init(&s_acc_full[s], kChainMmaWarps);
-            mbar_init(&s_acc_empty[s], 1);
-        }
+        for (int s = 0; s < kChainMaxNb; ++s) s_rows_q[s] = s_recs_x[s] = 0;
+        for (int s = 0; s < kChainAccBufs; ++s) s_recs_a[s] = s_freed[s] = 0;
         fence_mbar_init();
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -363,6 +394,16 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             s_nuses = static_cast<int>(c_ex);
             s_ustart[c_ex] = b_ex;
         }
+    }
+    __syncthreads();
+    // hand-over targets: per use, the records of the earlier uses that share its int8 buffer (u mod nb) and its
+    // partial-sum buffer (u mod kNacc)
+    for (int i = tid; i < s_nuses; i += kChainThreads) {
+        uint32_t cx = 0, ca = 0;
+        for (int v = i - p.nb; v >= 0; v -= p.nb) cx += (s_ustart[v + 1] - s_ustart[v]) >> 8;
+        for (int v = i - kNacc; v >= 0; v -= kNacc) ca += (s_ustart[v + 1] - s_ustart[v]) >> 8;
+        s_cumx[i] = cx;
+        s_cuma[i] = ca;
     }
     __syncthreads();
 
@@ -482,12 +523,11 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         // absmax of the lane's 16-byte chunks (bit patterns), one warp
         // reduction, the scale, then the codes into the int8 buffer in
         // fragment order.
-        // Parity waits see only the last two phases of a barrier, so every
-        // warp must meet each barrier it waits on in consecutive rounds: its
-        // staging slot is its own; an int8 buffer is met by the warps owning a
-        // row of its projections, which for T >= 4 is every warp, and for
-        // T < 4 (the host then takes four or eight buffers) depends only on
-        // the projection's index mod 4, the same for every use of the buffer.
+        // The staging slot is waited on by parity, which sees only the last
+        // two phases of a barrier: it is this warp's own and its rows arrive
+        // in consecutive rounds.  The int8 buffers are handed over through
+        // the monotonic counters (records run against a buffer, rows
+        // quantised into it).
         const int qw = warp - kWarpQuant0;
         const int qt = tid - kWarpQuant0 * 32;
         for (int i = qt; i < p.n_ops; i += kChainQuantThreads) s_gamma[i] = __ldg(p.op[i].gamma);
@@ -512,9 +552,8 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             bool waited = false;
             for (int t = 0; t < T; ++t, ++item) {
                 if (item % kChainQuantWarps != static_cast<uint32_t>(qw)) continue;
-                // the MMA warps are done with this buffer's previous projection
-                bool ok = waited || xround == 0u ||
-                          mbar_wait_cta(&s_xq_empty[xb], (xround - 1u) & 1u, &s_abort, p.status);
+                // every record of this buffer's earlier projections has been run
+                bool ok = waited || xround == 0u || wait_count(&s_recs_x[xb], s_cumx[uq], &s_abort, p.status);
                 waited = true;
                 // this warp's own staging slot: its rows arrive there in consecutive rounds
                 ok = ok && mbar_wait_cta(&s_xs_full[qw], (item / kChainQuantWarps) & 1u, &s_abort, p.status);
@@ -556,7 +595,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                 }
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&s_xq_full[xb]);   // T arrivals per projection
+                    red_release_cta(&s_rows_q[xb], 1u);   // T rows per projection
                     mbar_arrive(&s_xs_empty[qw]);
                 }
             }
@@ -574,7 +613,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             const int ntile = t1 - t0;
             if (ntile > 0) {
                 const int ab = static_cast<int>(ua % kNacc);
-                const bool ok = mbar_wait_cta(&s_acc_full[ab], (ua / kNacc) & 1u, &s_abort, p.status);
+                // every record of this projection (and of the buffer's earlier ones) has been run and flushed
+                const bool ok = wait_count(&s_recs_a[ab], s_cuma[ua] + static_cast<uint32_t>(ntile * (op.k >> 6)),
+                                           &s_abort, p.status);
                 if (!__all_sync(0xffffffffu, ok)) break;
                 // Scale slot ua % (kChainMaxNb + kChainAccBufs) was written by
                 // the quantisers after the MMA warps released int8 buffer use
@@ -599,7 +640,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                     if (op.acc_out) op.acc_out[o] = v;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&s_acc_empty[ab]);
+                if (lane == 0) red_release_cta(&s_freed[ab], 1u);   // the buffer is clear for its next projection
                 ++ua;
             }
             // count this CTA done with projection j (and, by program order, with every
@@ -618,20 +659,21 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
     // The ring carries this CTA's shares of all projections back to back, in
     // stages of S bytes; with W MMA warps, stage s sits in ring slot s % W, and
     // MMA warp w owns slot w: it runs every record of the stages w, w + W, ...
-    // (whatever projections they belong to) and alone releases them.  A warp passes
-    // every use (a projection with rows here) in stream order: it opens it
-    // (the use's partial-sum buffer is free, its int8 activations are ready),
-    // runs its records of it, if any of its stages holds some, and closes it
-    // (flush, arrivals on the partial-sum and int8 buffers' barriers).  Every
-    // warp therefore meets every barrier in consecutive rounds: parity waits
-    // stay unambiguous, and no arrival can count towards a round it does not
-    // belong to.  A warp closes a use as soon as it knows it has no more
-    // records of it: when its stage reaches the use's end, or when its next
-    // stage starts at or after it.
+    // (whatever projections they belong to) and alone releases them.  The
+    // hand-overs go through monotonic counters, so a warp deals only with the
+    // uses (projections with rows here) it has records of: it opens use u
+    // when it meets u's records (u's partial-sum buffer has been cleared by
+    // the epilogue for u's round, all T rows of u are quantised), runs them,
+    // and closes u as soon as it knows it has no more records of it (its stage
+    // reaches u's end, or its next stage starts at or after it): it flushes
+    // its partial sums and adds its record count to both buffers' counters.
+    // The epilogue takes u once every record of u has been counted; the
+    // quantisers refill u's int8 buffer once every record of it has been.
     const int n_uses = s_nuses;
     const uint32_t total = s_ustart[n_uses];
-    int u = 0;                  // the next use to close
-    bool opened = false;        // use u has been opened
+    int u = 0;                  // cursor: the use holding the current stream position (or an earlier one)
+    bool opened = false;        // use u is open
+    uint32_t mine = 0;          // records of the open use run by this warp
     bool failed = false;
     // state of the open use
     int ab = 0, xb = 0, ktiles = 1, cur = -1;
@@ -649,8 +691,9 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         const int2 uk = s_uk[u];   // k, and 1 / ktiles formed on the host
         ab = u % kNacc;
         xb = u & (p.nb - 1);
-        bool ok = u < kNacc || mbar_wait_cta(&s_acc_empty[ab], ((u / kNacc) - 1) & 1, &s_abort, p.status);
-        ok = ok && mbar_wait_cta(&s_xq_full[xb], (static_cast<uint32_t>(u) >> p.nb_log2) & 1u, &s_abort, p.status);
+        bool ok = wait_count(&s_freed[ab], static_cast<uint32_t>(u / kNacc), &s_abort, p.status);
+        ok = ok && wait_count(&s_rows_q[xb], static_cast<uint32_t>(T) * ((static_cast<uint32_t>(u) >> p.nb_log2) + 1u),
+                              &s_abort, p.status);
         if (!__all_sync(0xffffffffu, ok)) return false;
         acc_buf = sacc + ab * acc_words;
         b_src = reinterpret_cast<const uint4 *>(smem + p.xq_off[xb] +
@@ -661,30 +704,29 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
         ustart = s_ustart[u];
         uend = s_ustart[u + 1];
         cur = -1;
+        mine = 0;
         opened = true;
         return true;
     };
-    auto close_use = [&]() -> bool {
-        if (!opened && !open_use()) return false;
+    auto close_use = [&]() {
         if (cur >= 0) chain_flush<TM>(acc_buf, p.tiles_max, cur, lane, T, acc);
-        // the shared atomics of every lane are ordered before the release of the arrivals
+        // every lane's shared atomics (and shared loads of the int8 buffer) are
+        // ordered before the release of the counts
         __syncwarp();
         if (lane == 0) {
-            mbar_arrive(&s_acc_full[ab]);
-            mbar_arrive(&s_xq_empty[xb]);
+            red_release_cta(&s_recs_a[ab], mine);
+            red_release_cta(&s_recs_x[xb], mine);
         }
         opened = false;
         ++u;
-        return true;
     };
     const uint32_t ring_step = stage_bytes * static_cast<uint32_t>(kChainMmaWarps);
     uint8_t *slot = ring + static_cast<size_t>(warp) * stage_bytes;
     uint32_t round = 0;
     for (uint32_t a = static_cast<uint32_t>(warp) * stage_bytes; a < total; a += ring_step, ++round) {
         const uint32_t b = total - a < stage_bytes ? total : a + stage_bytes;
-        // the uses that end before this stage
-        while (u < n_uses && s_ustart[u + 1] <= a && !failed) failed = !close_use();
-        if (failed) break;
+        // the open use, if it ended before this stage (it was closed then), and other warps' uses
+        while (u < n_uses && s_ustart[u + 1] <= a) ++u;
         const bool okf = mbar_wait_cta(&s_full[warp], round & 1u, &s_abort, p.status);
         if (!__all_sync(0xffffffffu, okf)) {
             failed = true;
@@ -699,6 +741,7 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
             // records [pos, seg_end) of the open use; r0 = the first one's index in the CTA's share
             const int r0 = static_cast<int>((pos - ustart) >> 8);
             const int cnt = static_cast<int>((seg_end - pos) >> 8);
+            mine += static_cast<uint32_t>(cnt);
             // r0 / ktiles through the reciprocal (r0 < 2^24: off by at most one, corrected)
             int tile = __float2int_rz(static_cast<float>(r0) * inv_kt);
             int kt = r0 - tile * ktiles;
@@ -759,18 +802,17 @@ __global__ void __launch_bounds__(kChainThreads, 1) k_decode_chain(const __grid_
                 }
             }
             pos = seg_end;
-            if (pos == uend && !close_use()) failed = true;
+            if (pos == uend) close_use();
         }
         if (failed) break;
         // release the stage to the producer
         __syncwarp();
         if (lane == 0) mbar_arrive(&s_empty[warp]);
-        // the uses that end before this warp's next stage
+        // the open use, if it ends before this warp's next stage
         const uint32_t na = a + ring_step < total ? a + ring_step : total;
-        while (u < n_uses && s_ustart[u + 1] <= na && !failed) failed = !close_use();
-        if (failed) break;
+        if (opened && uend <= na) close_use();
     }
-    while (!failed && u < n_uses) failed = !close_use();
+    if (!failed && opened) close_use();
 }
 
 // ---------------------------------------------------------------- host side

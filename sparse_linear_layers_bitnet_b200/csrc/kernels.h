@@ -129,7 +129,7 @@ struct ChainOpDev {
 constexpr int kChainMaxOps = 128;                  // projections per launch (kernel parameter space)
 constexpr int kChainMaxTiles = 32;                 // 16-row tiles per CTA per projection
 constexpr int kChainMaxK = 1 << 17;                // 64 * 127 * k / 2 stays inside int32 (codes expanded x64)
-constexpr size_t kChainMaxSmem = 227 * 1024 - 5120;   // dynamic shared memory (static use < 5 KB)
+constexpr size_t kChainMaxSmem = 227 * 1024 - 6144;   // dynamic shared memory (static use < 6 KB)
 constexpr size_t kChainAbortOffset = 4;            // workspace: grid abort word
 constexpr size_t kChainCountersOffset = 256;       // workspace: one counter per projection
 // Shared-memory layout of one chain launch (chain.cu).
