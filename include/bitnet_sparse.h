@@ -448,8 +448,13 @@ bitnet_status bitnet_quant_linear(const void *X, bitnet_dtype x_dtype, float eps
  *   eps      activation eps (> 0).
  *   ws       >= bitnet_decode_chain_workspace_size(n_ops) bytes: status word,
  *            abort word and one completion counter per op (cleared by the call).
- * Shared memory bounds T * (max k + 128): the call returns UNSUPPORTED when
- * fewer than two 16 KB weight stages would fit.
+ * Kernels: a chain with no wait_prev runs on the pipelined kernel (warp roles
+ * joined by barriers and shared-memory counters); a chain with any wait_prev
+ * on the latency-oriented one.  Shared memory holds the activation rows (one
+ * staging row per quantiser warp, the int8 rows of several projections) and
+ * the weight ring: the call returns UNSUPPORTED when they do not fit beside
+ * weight stages of at least 2 KB per MMA warp (pipelined) or two 16 KB stages
+ * (with waits).
  * Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA; a wait that runs out
  * inside the kernel sets the TIMEOUT bit of the device status word.
  * ------------------------------------------------------------------------ */
