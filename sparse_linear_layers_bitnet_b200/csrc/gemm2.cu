@@ -111,6 +111,9 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t d, uint64_t a, uint64_t b
 __device__ __forceinline__ void tmem_cp_pair_128x128b(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::2.128x128b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
+__device__ __forceinline__ void tmem_cp_pair_128x256b(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
 
 // arrive once on the barrier at this offset in both CTAs when the issued
 // tcgen05 operations are complete
@@ -150,7 +153,7 @@ struct PairCfg {
     static constexpr int kAAdvance = 32;
     static constexpr int kBAdvance = SPARSE ? 64 : 32;
     static constexpr int kAccStride = 256;                // TMEM columns between the two accumulators
-    static constexpr int kECol = 2 * kAccStride - 16;     // metadata columns (8 used)
+    static constexpr int kECol = 2 * kAccStride - 16;     // metadata columns (two groups of 8)
     static constexpr int kTmemCols = 512;
     static constexpr int kStageOutBytes = SPARSE ? 2 * 16 * 128 * 4 : 0;   // two [16 tokens][128 rows] fp32 chunks
     static constexpr int kSmemBytes = STAGES * kStageBytes + kStageOutBytes + 1024 + 2048;
@@ -309,13 +312,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
                     const uint32_t a_base = smem_u32(sA + s * C::kABytes);
                     const uint32_t b_base = smem_u32(sB + s * C::kBBytes);
                     if (SPARSE) {
+                        // both k-steps' metadata in one copy of 128 lanes x 256 bits: k-step 0's block (the
+                        // first 16-byte core-matrix column) lands in columns 0..3, k-step 1's (C::kESub bytes on)
+                        // in 4..7; consecutive stages alternate between two groups of 8 columns
+                        static_assert(!SPARSE || C::kSub == 2, "one 256-bit metadata copy covers two k-steps");
+                        const uint32_t e_stage = tmem + C::kECol + 8u * (it & 1);
+                        pair::tmem_cp_pair_128x256b(
+                            e_stage, make_smem_desc(smem_u32(sE + s * C::kEBytes), C::kESub, 128, kSwizzleNone));
 #pragma unroll
                         for (int sub = 0; sub < C::kSub; ++sub) {
-                            // metadata of consecutive k-steps alternate between two TMEM column groups
-                            const uint32_t e_col = tmem + C::kECol + 4u * ((it * C::kSub + sub) & 1);
-                            pair::tmem_cp_pair_128x128b(
-                                e_col, make_smem_desc(smem_u32(sE + s * C::kEBytes + sub * C::kESub), 16, 128,
-                                                      kSwizzleNone));
+                            const uint32_t e_col = e_stage + 4u * sub;
 #pragma unroll
                             for (int j = 0; j < C::kMmaPerStage; ++j) {
                                 const uint64_t ad = make_smem_desc(a_base + sub * C::kASub + j * C::kAAdvance, 16, 512,
